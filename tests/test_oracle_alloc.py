@@ -1,0 +1,79 @@
+"""Pins of the oracle allocator against brute force (Everett's theorem) and its invariants."""
+import numpy as np
+import pytest
+
+from oracle.alloc import (build_options, allocate, brute_force_allocate, evaluate, lower_hull,
+                          BudgetError)
+from synth import make_random_tables
+
+PHI = [1.0, 0.12, 0.0075, 2.9e-5]
+
+
+def small_instance(n_cells, seed, n_rt=3, n_rd=3, T=64, d=32, Lg=2, H=2, sf=2):
+    n2, tT, td = make_random_tables(n_cells, n_rt, n_rd, seed)
+    return [build_options(n2[c], tT[c], td[c], PHI, T, d, Lg, H, sf) for c in range(n_cells)]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_everett_against_brute_force(seed):
+    opts = small_instance(3, seed)
+    lo = sum(min(o[0] for o in c) for c in opts)
+    hi = sum(max(o[0] for o in c) for c in opts)
+    for frac in np.linspace(0.0, 1.0, 9):
+        budget = int(lo + frac * (hi - lo))
+        ch, lam, total = allocate(opts, budget)
+        B, E = evaluate(opts, ch)
+        assert B == total <= budget
+        best = brute_force_allocate(opts, B)
+        assert E <= best[0] * (1 + 1e-12) + 1e-12
+
+
+def test_lambda_monotone_in_budget():
+    opts = small_instance(4, 11, n_rt=5, n_rd=4)
+    lo = sum(min(o[0] for o in c) for c in opts)
+    hi = sum(max(o[0] for o in c) for c in opts)
+    lams, Es = [], []
+    for frac in np.linspace(0.0, 1.0, 25):
+        ch, lam, total = allocate(opts, int(lo + frac * (hi - lo)))
+        lams.append(lam)
+        Es.append(evaluate(opts, ch)[1])
+    assert all(a >= b for a, b in zip(lams, lams[1:]))
+    assert all(a >= b for a, b in zip(Es, Es[1:]))
+
+
+def test_infeasible_budget():
+    opts = small_instance(2, 3)
+    lo = sum(min(o[0] for o in c) for c in opts)
+    with pytest.raises(BudgetError):
+        allocate(opts, lo - 1)
+    ch, lam, total = allocate(opts, lo)
+    assert total == lo
+
+
+def test_unbounded_budget_takes_min_error():
+    opts = small_instance(3, 5)
+    ch, lam, total = allocate(opts, 10 ** 15)
+    for c, o in zip(ch, opts):
+        best = min(x[1] for x in o)
+        assert next(x for x in o if tuple(x[2:5]) == tuple(c))[1] == best
+    assert lam == 0.0
+
+
+def test_hull_is_convex_and_decreasing():
+    opts = small_instance(1, 7, n_rt=8, n_rd=5)[0]
+    h = lower_hull(opts)
+    B = np.array([v[0] for v in h], float)
+    E = np.array([v[1] for v in h])
+    assert np.all(np.diff(B) > 0) and np.all(np.diff(E) < 0)
+    sl = -np.diff(E) / np.diff(B)
+    assert np.all(np.diff(sl) <= 1e-12 * sl[:-1])
+    # every option lies on or above the hull's piecewise-linear envelope
+    for o in opts:
+        if B[0] <= o[0] <= B[-1]:
+            assert o[1] >= np.interp(o[0], B, E) * (1 - 1e-12)
+
+
+def test_zero_rank_pairs_with_zero_rank():
+    opts = small_instance(1, 2)[0]
+    for B, E, rT, rd, b in opts:
+        assert (rT == 0) == (rd == 0)
