@@ -1,0 +1,230 @@
+/*
+ * jolt.h — C ABI of the JoLT KV-cache codec for NVIDIA B200 (sm_100a).
+ *
+ * JoLT compresses a transformer's prefill KV cache by a partial Tucker decomposition of each
+ * (layer group, K|V) cell along its token and feature modes, plus a randomly rotated, uniformly
+ * quantised residual; one Lagrange multiplier allocates ranks and residual bits across cells
+ * under a global byte budget; decode attention runs directly over the stored factors.
+ * Sources: "A JoLT for the KV cache: Near-Lossless KV Cache Compression via Joint Rank-bit
+ * Allocation" (arXiv:2607.12550v4 summary on paperlayer.ai), §3 Method, §3.1 FlashJoLT,
+ * §4.5 Fused decode kernel; "Technische Samenvatting: Een JOLT voor de KV Cache"
+ * (gist.science/nl), Methodologie 1-4; "JoLT: совместное распределение ранга и бит в KV-кэше"
+ * (sarnas.ru), sections on the KV-cache size and on building cos/sin inside the kernel.
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are CUDA device pointers of the current device; "host" are host
+ *     pointers. The caller owns every buffer; the library never allocates device memory and
+ *     keeps no state between calls except read-only device constants.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - Device-side errors (numeric range, bounded waits that gave up) are written to an error
+ *     word at the start of the workspace `ws`; calls that synchronise report them, the
+ *     asynchronous decode call leaves them for jolt_check().
+ *   - Invalid arguments return JOLT_ERR_INVALID_ARG before any launch.
+ *
+ * Tensor layouts (row-major, last index fastest):
+ *   K, V   [batch][n_layers][n_kv][T][d_h]           io dtype
+ *   q, out [batch][n_layers_call][n_q][d_h]           io dtype
+ *   cells are indexed c = (b * n_groups + g) * 2 + kv, kv = 0 for K and 1 for V; a cell holds
+ *   layers [g*L_g, (g+1)*L_g) of sequence b: the tensor X[L_g][n_kv][T][d_h].
+ *   Query head h' reads KV head floor(h' / (n_q / n_kv)).
+ *
+ * Stored cache, per cell, five segments each starting on a 256-byte boundary:
+ *   U_T   [T][r_T]                 factor dtype   token basis
+ *   U_d   [d_h][r_d]               factor dtype   feature basis
+ *   G     [L_g][n_kv][r_T][r_d]    factor dtype   core
+ *   codes [L_g][n_kv][T][d_h*b/8]  uint8          packed residual codes (absent when b == 0)
+ *   sz    [L_g][n_kv][T][2]        fp16           per-row (scale, zero)  (absent when b == 0)
+ * Code j of a row occupies bits [(j*b) mod 8, +b) of byte floor(j*b/8).
+ */
+#ifndef JOLT_H_
+#define JOLT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  JOLT_OK = 0,
+  JOLT_ERR_INVALID_ARG = -1,   /* bad shape, pointer, size or option */
+  JOLT_ERR_CUDA = -2,          /* a CUDA runtime/driver call failed */
+  JOLT_ERR_TIMEOUT = -3,       /* a bounded device-side wait gave up */
+  JOLT_ERR_BUDGET = -4,        /* byte budget below the cheapest allocation */
+  JOLT_ERR_NUMERIC = -5,       /* non-finite input or fp16 scale/zero out of range */
+  JOLT_ERR_WORKSPACE = -6,     /* workspace smaller than jolt_workspace_bytes() */
+  JOLT_ERR_STATE = -7          /* jolt_compress without a matching jolt_analyze */
+} jolt_status;
+
+typedef enum { JOLT_F32 = 0, JOLT_BF16 = 1 } jolt_dtype;
+
+typedef enum { JOLT_OP_COMPRESS = 0, JOLT_OP_DECODE = 1 } jolt_op;
+
+/* Problem description shared by all calls. */
+typedef struct {
+  int32_t batch;              /* sequences B >= 1 */
+  int32_t n_layers;           /* L >= 1 */
+  int32_t layers_per_group;   /* L_g, divides L: a cell groups L_g consecutive layers */
+  int32_t n_kv;               /* KV heads >= 1 */
+  int32_t n_q;                /* query heads, a multiple of n_kv */
+  int32_t T;                  /* cached tokens per sequence >= 1 */
+  int32_t d_h;                /* head dimension: 64 or 128 */
+  int32_t io_dtype;           /* jolt_dtype of K, V, q, out */
+  int32_t factor_dtype;       /* jolt_dtype of the stored U_T, U_d, G */
+  int32_t keys_pre_rope;      /* 1: keys were captured before RoPE; decode re-applies RoPE */
+  int32_t q_cap;              /* token-rank cap, multiple of 16, <= min(T, L_g*n_kv*d_h) */
+  int32_t sketch_cols;        /* l: sketch width of the randomized token SVD, q_cap <= l <=
+                                 min(T, L_g*n_kv*d_h), multiple of 16 */
+  int32_t power_iters;        /* q >= 0 power iterations of the range finder */
+  int32_t cells_per_pass;     /* cells processed together by jolt_analyze (>= 1) */
+  uint64_t rot_seed;          /* seed of the residual rotation's sign diagonal */
+  uint64_t sketch_seed;       /* seed of the Rademacher sketch matrix */
+  float attn_scale;           /* softmax scale, usually 1/sqrt(d_h) */
+  float rope_attention_scaling; /* multiplies cos and sin (1.0 for plain RoPE) */
+} jolt_shape;
+
+/* Per-cell rank/bit choice: r_T, r_d multiples of 16 (both 0 or both > 0), b in {0,2,4,8}. */
+typedef struct {
+  int32_t r_T;
+  int32_t r_d;
+  int32_t b;
+} jolt_cell_choice;
+
+/* Human-readable status. Never NULL. */
+const char* jolt_status_string(jolt_status s);
+
+/* Library version (major*10000 + minor*100 + patch). */
+int32_t jolt_version(void);
+
+/* Checks a shape; JOLT_OK or JOLT_ERR_INVALID_ARG. */
+jolt_status jolt_shape_check(const jolt_shape* shape);
+
+/* Dense KV-cache bytes 2 * L * n_kv * d_h * T * dtype_bytes ("JoLT: совместное распределение ранга
+ * и бит в KV-кэше", section on the KV-cache size formula). */
+uint64_t jolt_kv_bytes(int32_t n_layers, int32_t n_kv, int32_t d_h, int64_t T, int32_t dtype_bytes);
+
+/* Bytes one cell stores for a choice, without alignment padding (the allocator's byte model):
+ * s_f*(T*r_T + d_h*r_d + L_g*n_kv*r_T*r_d) + [b>0]*L_g*n_kv*T*(d_h*b/8 + 4).
+ * Returns 0 for an invalid choice. */
+uint64_t jolt_cell_bytes(const jolt_shape* shape, jolt_cell_choice choice);
+
+/* Layout of the stored cache for per-cell choices (host array, n_cells = 2*B*L/L_g entries).
+ * offsets (host, may be NULL): n_cells*5 byte offsets of U_T, U_d, G, codes, sz per cell.
+ * total_bytes (host): bytes of the whole cache buffer. */
+jolt_status jolt_cache_layout(const jolt_shape* shape, const jolt_cell_choice* choices,
+                              uint64_t* offsets, uint64_t* total_bytes);
+
+/* Error fraction phi(b) of the rotated b-bit quantiser for b = 0, 2, 4, 8 (phi(0) = 1), measured
+ * on n_rows Gaussian rows of dimension d_h drawn from `seed` (host computation). The allocator's
+ * surrogate multiplies the discarded mass by it ("A JoLT for the KV cache", §3). */
+jolt_status jolt_phi(int32_t d_h, int32_t n_rows, uint64_t seed, double phi_out[4]);
+
+/* Joint allocation with one Lagrange multiplier ("A JoLT for the KV cache", §3): for n_cells
+ * cells with spectra tails
+ *   norm2[c]                = ||X_c||^2,
+ *   tail_T[c*n_rt + k]      = discarded token-mode mass at r_T = 16k  (k < n_rt),
+ *   tail_d[c*n_rd + j]      = discarded feature-mode mass at r_d = 16j (j < n_rd),
+ * (all host, float64) choose per cell (r_T, r_d, b) minimising sum E subject to
+ * sum bytes <= budget, E = phi(b) * (r_T ? min(norm2, tail_T + tail_d) : norm2), bytes from
+ * jolt_cell_bytes. Hull segments are bought in order of falling price dE/dbytes while the budget
+ * holds; lambda_out (host, may be NULL) is the price of the first segment that did not fit.
+ * Host-only and deterministic. JOLT_ERR_BUDGET if the cheapest choices exceed the budget. */
+jolt_status jolt_allocate(const jolt_shape* shape, int32_t n_cells, const double* norm2,
+                          const double* tail_T, int32_t n_rt, const double* tail_d, int32_t n_rd,
+                          const double phi[4], uint64_t budget, jolt_cell_choice* choices_out,
+                          double* lambda_out, uint64_t* total_bytes_out);
+
+/* Workspace bytes for an operation (device memory the caller allocates and passes as `ws`).
+ * JOLT_OP_COMPRESS covers jolt_analyze followed by jolt_compress on the same ws;
+ * JOLT_OP_DECODE covers jolt_decode_attn with any n_layers_call <= n_layers. 0 on bad shape. */
+size_t jolt_workspace_bytes(const jolt_shape* shape, int32_t op);
+
+/* Spectra of every cell ("A JoLT for the KV cache", §3.1 FlashJoLT): a randomized token-mode SVD
+ * (Rademacher sketch, power iterations with CholeskyQR orthonormalisation, Rayleigh-Ritz) gives
+ * the top q_cap token directions; the energy it did not find, ||X||^2 minus the captured part,
+ * closes the token tail; the feature tail comes from the eigenvalues of the cell's feature Gram.
+ *   k, v        device, [B][L][n_kv][T][d_h] io dtype
+ *   norm2_out   host [n_cells];  tail_T_out host [n_cells][q_cap/16+1];
+ *   tail_d_out  host [n_cells][d_h/16+1]
+ *   ws          device, >= jolt_workspace_bytes(shape, JOLT_OP_COMPRESS); on return holds the
+ *               cells' token bases for jolt_compress.
+ * Synchronises `stream`. */
+jolt_status jolt_analyze(const jolt_shape* shape, const void* k, const void* v, double* norm2_out,
+                         double* tail_T_out, double* tail_d_out, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* Compress every cell with its choice ("A JoLT for the KV cache", §3): U_T = the first r_T token
+ * directions found by jolt_analyze, U_d = top-r_d eigenvectors of the feature Gram of U_T^T X,
+ * G = U_T^T X U_d, residual R = X - U_T G U_d^T against the stored (rounded) factors, rotated by
+ * (1/sqrt(d_h)) H D (Hadamard times seeded signs), quantised per row and packed.
+ *   k, v      device, as for jolt_analyze — the same tensors the preceding analyze saw
+ *   choices   host [n_cells]
+ *   cache     device, cache_bytes >= jolt_cache_layout total
+ *   ws        device, the workspace jolt_analyze filled (JOLT_ERR_STATE otherwise)
+ * Synchronises `stream`. */
+jolt_status jolt_compress(const jolt_shape* shape, const void* k, const void* v,
+                          const jolt_cell_choice* choices, void* cache, uint64_t cache_bytes,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Decode attention of one query token per (sequence, layer, query head) over all T stored
+ * tokens, evaluated on the stored factors without materialising dense K/V ("A JoLT for the KV
+ * cache", §4.5): scores U_T (G (U_d^T q)) + (R q) . deq(codes) and values
+ * U_d G^T (U_T^T p) + R^T (deq(codes)^T p); with keys_pre_rope, each key is rebuilt per token
+ * tile and rotated by RoPE at position pos_offset + t before the dot product, cos/sin computed in
+ * the kernel from inv_freq ("JoLT: совместное распределение ранга и бит в KV-кэше", section on
+ * building cos/sin in the kernel).
+ *   cache        device, filled by jolt_compress (or laid out by jolt_cache_layout)
+ *   layer_begin, n_layers_call: layers [layer_begin, layer_begin + n_layers_call)
+ *   q            device [B][n_layers_call][n_q][d_h] io dtype
+ *   out          device [B][n_layers_call][n_q][d_h] io dtype
+ *   lse          device [B][n_layers_call][n_q] fp32 log-sum-exp of the scaled scores, or NULL
+ *   inv_freq     device [d_h/2] fp32 (required when keys_pre_rope), may carry RoPE scaling
+ *   pos_offset   position of cached token 0
+ *   ws           device, >= jolt_workspace_bytes(shape, JOLT_OP_DECODE); calls sharing a ws
+ *                must not overlap in time
+ * Asynchronous on `stream`. */
+jolt_status jolt_decode_attn(const jolt_shape* shape, const jolt_cell_choice* choices,
+                             const void* cache, int32_t layer_begin, int32_t n_layers_call,
+                             const void* q, void* out, float* lse, const float* inv_freq,
+                             int32_t pos_offset, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream` and returns the device error word of `ws` (then clears it). */
+jolt_status jolt_check(void* ws, void* stream);
+
+/* Building blocks, exposed for bit-exact testing and for callers that quantise their own data. */
+
+/* Rotate rows by (1/sqrt(d)) H D (inverse = 0) or its transpose D H / sqrt(d) (inverse = 1),
+ * D the seeded sign diagonal. in/out device fp32 [n_rows][d], d in {64, 128}; may alias. */
+jolt_status jolt_rotate_rows(const float* in, float* out, int64_t n_rows, int32_t d,
+                             uint64_t seed, int32_t inverse, void* stream);
+
+/* Quantise fp32 rows per row (fp16 scale = (max-min)/(2^b-1), fp16 zero = min, codes rounded to
+ * nearest even and clipped) and pack them. rows device fp32 [n_rows][d]; codes device uint8
+ * [n_rows][d*b/8]; sz device fp16 [n_rows][2]; err device int32 (set to JOLT_ERR_NUMERIC when a
+ * scale or zero is out of fp16 range; never cleared by the kernel). b in {2,4,8}. */
+jolt_status jolt_quantize_pack(const float* rows, int64_t n_rows, int32_t d, int32_t b,
+                               uint8_t* codes, void* sz, int32_t* err, void* stream);
+
+/* Unpack and dequantise: out = fp32(code * scale + zero) (one rounding). */
+jolt_status jolt_unpack_dequant(const uint8_t* codes, const void* sz, int64_t n_rows, int32_t d,
+                                int32_t b, float* out, void* stream);
+
+/* Plain batched GEMM on the tcgen05 tensor cores (the kernel the compressor's contractions use):
+ *   C[z][m][n] (+)= sum_k A[z](m,k) * B[z](k,n),  bf16 operands, fp32 accumulation and output.
+ * A (device, bf16): element (m,k) at A[z*stride_a + m*lda + k] (a_mn_major = 0) or
+ *   A[z*stride_a + k*lda + m] (a_mn_major = 1).  B (device, bf16): element (k,n) at
+ *   B[z*stride_b + n*ldb + k] (b_mn_major = 0) or B[z*stride_b + k*ldb + n] (b_mn_major = 1).
+ * C (device, fp32): element (m,n) at C[z*stride_c + m*ldc + n]. Strides in elements; lda and ldb
+ * must be multiples of 8 and the base pointers 16-byte aligned. k_split > 1 splits K over CTAs
+ * and requires accumulate = 1 (atomic adds into C, which the caller zeroes first). */
+jolt_status jolt_gemm_bf16(const void* A, int32_t a_mn_major, const void* B, int32_t b_mn_major,
+                           float* C, int32_t M, int32_t N, int32_t K, int64_t lda, int64_t ldb,
+                           int64_t ldc, int32_t batch, int64_t stride_a, int64_t stride_b,
+                           int64_t stride_c, int32_t k_split, int32_t accumulate, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* JOLT_H_ */

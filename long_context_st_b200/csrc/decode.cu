@@ -1,0 +1,162 @@
+// jolt_decode_attn: argument checks, workspace carving, split choice and kernel dispatch.
+#include <algorithm>
+#include <vector>
+
+#include "common.cuh"
+#include "decode.cuh"
+
+namespace jolt {
+
+namespace {
+
+constexpr int kSMs = 148;
+
+int choose_splits(const jolt_shape& s, int Lc) {
+  const int64_t units = int64_t(s.batch) * Lc * s.n_kv;
+  int S = int((2 * kSMs + units - 1) / units);
+  S = std::max(1, std::min(S, std::min(64, (s.T + 63) / 64)));
+  return S;
+}
+
+struct DecodeWs {
+  size_t qrot, qsum, P, Bh, part, total;
+};
+
+DecodeWs decode_ws_layout(const jolt_shape& s, int Lc, int S) {
+  DecodeWs w{};
+  const size_t B = s.batch, nq = s.n_q, d = s.d_h, qc = std::max(s.q_cap, 16);
+  size_t off = sizeof(WsHeader);
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  w.qrot = take(B * Lc * nq * d * 4);
+  w.qsum = take(B * Lc * nq * 4);
+  w.P = take(s.keys_pre_rope ? 0 : B * Lc * nq * qc * 4);
+  w.Bh = take(s.keys_pre_rope ? B * Lc * s.n_kv * qc * d * 4 : 0);
+  w.part = take(B * Lc * nq * size_t(S) * (2 + qc + d) * 4);
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+size_t decode_workspace_bytes(const jolt_shape& s) {
+  size_t mx = 0;
+  for (int Lc = 1; Lc <= s.n_layers; ++Lc) mx = std::max(mx, decode_ws_layout(s, Lc, choose_splits(s, Lc)).total);
+  return mx;
+}
+
+}  // namespace jolt
+
+using namespace jolt;
+
+extern "C" jolt_status jolt_decode_attn(const jolt_shape* shape, const jolt_cell_choice* choices,
+                                        const void* cache, int32_t layer_begin, int32_t n_layers_call,
+                                        const void* q, void* out, float* lse, const float* inv_freq,
+                                        int32_t pos_offset, void* ws, size_t ws_bytes, void* stream) {
+  if (!shape_ok(shape) || !choices || !cache || !q || !out || !ws) return JOLT_ERR_INVALID_ARG;
+  const jolt_shape& s = *shape;
+  if (layer_begin < 0 || n_layers_call < 1 || layer_begin + n_layers_call > s.n_layers)
+    return JOLT_ERR_INVALID_ARG;
+  if (s.keys_pre_rope && !inv_freq) return JOLT_ERR_INVALID_ARG;
+  if (pos_offset < 0 || int64_t(pos_offset) + s.T > (int64_t(1) << 24)) return JOLT_ERR_INVALID_ARG;
+  const int nc = n_cells(s);
+  for (int c = 0; c < nc; ++c)
+    if (!choice_ok(s, choices[c])) return JOLT_ERR_INVALID_ARG;
+  const int Lc = n_layers_call;
+  const int S = choose_splits(s, Lc);
+  const DecodeWs wl = decode_ws_layout(s, Lc, S);
+  if (ws_bytes < wl.total) return JOLT_ERR_WORKSPACE;
+
+  // cell offsets of the whole cache (host arithmetic, same layout as jolt_cache_layout)
+  std::vector<uint64_t> cell_off(nc);
+  {
+    uint64_t off = 0;
+    for (int c = 0; c < nc; ++c) {
+      cell_off[c] = off;
+      off += cell_segments(s, choices[c]).size;
+    }
+  }
+  const int G = n_groups(s);
+  const int g_first = layer_begin / s.layers_per_group;
+  const int g_last = (layer_begin + Lc - 1) / s.layers_per_group;
+  const int Gc = g_last - g_first + 1;
+
+  DecodeParams p{};
+  p.cache = static_cast<const uint8_t*>(cache);
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.inv_freq = inv_freq;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  p.err = reinterpret_cast<int32_t*>(wsb);
+  p.ws_qrot = reinterpret_cast<float*>(wsb + wl.qrot);
+  p.ws_qsum = reinterpret_cast<float*>(wsb + wl.qsum);
+  p.ws_P = reinterpret_cast<float*>(wsb + wl.P);
+  p.ws_Bh = reinterpret_cast<float*>(wsb + wl.Bh);
+  p.ws_part = reinterpret_cast<float*>(wsb + wl.part);
+  p.rot_seed = s.rot_seed;
+  p.attn_scale = s.attn_scale;
+  p.rope_scaling = s.rope_attention_scaling;
+  p.Lg = s.layers_per_group;
+  p.n_kv = s.n_kv;
+  p.n_q = s.n_q;
+  p.gq = s.n_q / s.n_kv;
+  p.T = s.T;
+  p.d_h = s.d_h;
+  p.Lc = Lc;
+  p.layer_begin = layer_begin;
+  p.S = S;
+  p.q_cap = std::max(s.q_cap, 16);
+  p.pos_offset = pos_offset;
+  p.io_f32 = s.io_dtype == JOLT_F32;
+  p.fac_f32 = s.factor_dtype == JOLT_F32;
+  p.pre_rope = s.keys_pre_rope;
+  p.g_first = g_first;
+  p.Gc = Gc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // one launch set per batch range whose cells fit the parameter table
+  const int bchunk = std::max(1, kMaxCallCells / (2 * Gc));
+  for (int b0 = 0; b0 < s.batch; b0 += bchunk) {
+    const int nb = std::min(bchunk, s.batch - b0);
+    DecodeParams pc = p;
+    pc.B = nb;
+    for (int bi = 0; bi < nb; ++bi)
+      for (int gi = 0; gi < Gc; ++gi)
+        for (int kv = 0; kv < 2; ++kv) {
+          const int c = ((b0 + bi) * G + g_first + gi) * 2 + kv;
+          CellRef r;
+          r.offset = cell_off[c];
+          r.r_T = choices[c].r_T;
+          r.r_d = choices[c].r_d;
+          r.b = choices[c].b;
+          r.pad = 0;
+          pc.cells[(bi * Gc + gi) * 2 + kv] = r;
+        }
+    // shift the batch-major tensors to this batch range
+    const size_t row = size_t(Lc) * s.n_q;
+    const int iob = s.io_dtype == JOLT_F32 ? 4 : 2;
+    pc.q = static_cast<const uint8_t*>(q) + size_t(b0) * row * s.d_h * iob;
+    pc.out = static_cast<uint8_t*>(out) + size_t(b0) * row * s.d_h * iob;
+    pc.lse = lse ? lse + size_t(b0) * row : nullptr;
+    jolt_status st_ = launch_decode_simt(pc, st);
+    if (st_ != JOLT_OK) return st_;
+  }
+  return JOLT_OK;
+}
+
+extern "C" jolt_status jolt_check(void* ws, void* stream) {
+  if (!ws) return JOLT_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  JOLT_CUDA_TRY(cudaStreamSynchronize(st));
+  int32_t err = 0;
+  JOLT_CUDA_TRY(cudaMemcpy(&err, ws, sizeof(int32_t), cudaMemcpyDeviceToHost));
+  if (err) {
+    const int32_t zero = 0;
+    JOLT_CUDA_TRY(cudaMemcpy(ws, &zero, sizeof(int32_t), cudaMemcpyHostToDevice));
+  }
+  return static_cast<jolt_status>(err);
+}

@@ -1,0 +1,46 @@
+// Host interface of the tcgen05 GEMM: C[z] (+)= sum_t A_t[z] * B_t[z], bf16 operands in global
+// memory described by TMA tensor maps, fp32 accumulation in TMEM, fp32 output.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace jolt {
+
+enum Major { kMajorK = 0, kMajorMN = 1 };
+
+// One bf16 operand. Logical matrix A[mn][k] (or B[k][mn]); `major` says which index is
+// contiguous in memory. The contiguous ("inner") index may be folded: inner = fold_index * fold +
+// r (0 <= r < fold), where consecutive folds are `fold_stride` elements apart — this is how the
+// token unfolding X_(T)[t][(l,h,j)] of a [L_g*n_kv][T][d_h] cell is addressed without a copy.
+struct Operand {
+  const void* ptr = nullptr;  // bf16
+  int major = kMajorK;
+  int64_t inner = 0;          // extent of the contiguous index (fold length when folded)
+  int64_t outer = 0;          // extent of the other index
+  int64_t outer_stride = 0;   // elements between consecutive outer indices
+  int64_t fold = 0;           // 0: not folded
+  int64_t nfold = 1;          // number of folds
+  int64_t fold_stride = 0;    // elements between folds
+  int64_t batch = 1;
+  int64_t batch_stride = 0;   // elements between batch entries
+};
+
+struct GemmCall {
+  int M = 0, N = 0, K = 0;
+  int n_terms = 1;
+  Operand A[3], B[3];
+  float* C = nullptr;
+  int64_t ldc = 0;
+  int64_t c_batch_stride = 0;  // elements between C batch entries
+  int c_batch_div = 1;         // C entry of operand batch z is z / c_batch_div
+  int batch = 1;               // operand batch entries (grid z)
+  int k_split = 1;             // split-K factor; > 1 (or c_batch_div > 1) requires accumulate
+  bool accumulate = false;     // atomically add into C instead of storing
+  int32_t* err = nullptr;
+};
+
+// Launch; validates shapes and alignment (JOLT_ERR_INVALID_ARG) before any launch.
+jolt_status gemm_tc(const GemmCall& g, cudaStream_t st);
+
+}  // namespace jolt

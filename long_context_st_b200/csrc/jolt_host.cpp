@@ -1,0 +1,313 @@
+// Host-side part of the JoLT library: shape checks, byte model, stored-cache layout, the
+// quantiser error fraction phi(b), and the single-multiplier allocator.
+//
+// Compiled with -ffp-contract=off so that E + lambda*bytes style expressions round exactly as
+// written (no fused multiply-add).
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "jolt_internal.h"
+
+namespace jolt {
+
+bool shape_ok(const jolt_shape* s) {
+  if (!s) return false;
+  if (s->batch < 1 || s->n_layers < 1 || s->layers_per_group < 1 || s->n_kv < 1 || s->T < 1)
+    return false;
+  if (s->n_layers % s->layers_per_group) return false;
+  if (s->n_q < s->n_kv || s->n_q % s->n_kv) return false;
+  if (s->d_h != 64 && s->d_h != 128) return false;
+  if (s->io_dtype != JOLT_F32 && s->io_dtype != JOLT_BF16) return false;
+  if (s->factor_dtype != JOLT_F32 && s->factor_dtype != JOLT_BF16) return false;
+  const int64_t n = n_cols(*s);
+  const int64_t lim = std::min<int64_t>(n, s->T);
+  if (s->q_cap < 0 || s->q_cap % kRankStep || s->q_cap > lim) return false;
+  if (s->sketch_cols % kRankStep || s->sketch_cols < s->q_cap || s->sketch_cols > lim) return false;
+  if (s->q_cap > 0 && s->sketch_cols < 16) return false;
+  if (s->power_iters < 0 || s->power_iters > 8) return false;
+  if (s->cells_per_pass < 1) return false;
+  if (!(s->attn_scale > 0.f) || !std::isfinite(s->attn_scale)) return false;
+  if (!std::isfinite(s->rope_attention_scaling)) return false;
+  if (s->T > (1 << 24)) return false;
+  return true;
+}
+
+bool choice_ok(const jolt_shape& s, const jolt_cell_choice& c) {
+  if (c.r_T < 0 || c.r_d < 0 || c.r_T % kRankStep || c.r_d % kRankStep) return false;
+  if ((c.r_T == 0) != (c.r_d == 0)) return false;
+  if (c.r_T > s.q_cap || c.r_d > s.d_h) return false;
+  if (!(c.b == 0 || c.b == 2 || c.b == 4 || c.b == 8)) return false;
+  return true;
+}
+
+CellSegs cell_segments(const jolt_shape& s, const jolt_cell_choice& c) {
+  const SegOffsets o = seg_offsets(s.T, s.d_h, s.layers_per_group, s.n_kv, dtype_bytes(s.factor_dtype),
+                                   c.r_T, c.r_d, c.b);
+  const uint64_t rows = uint64_t(s.layers_per_group) * s.n_kv * s.T;
+  CellSegs g{o.ut, o.ud, o.g, o.codes, o.sz, 0};
+  g.size = align_up(o.sz + (c.b ? rows * 4 : 0), kSegAlign);
+  return g;
+}
+
+// ---- fp16 / Gaussian helpers for phi --------------------------------------------------------
+
+static inline uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Standard normal pairs by the Box-Muller transform on two counter-hashed uniforms in (0, 1).
+static inline void normal_pair(uint64_t seed, uint64_t i, double* a, double* b) {
+  const double u1 = (double((splitmix64((seed << 32) ^ (2 * i)) >> 11)) + 0.5) * 0x1.0p-53;
+  const double u2 = (double((splitmix64((seed << 32) ^ (2 * i + 1)) >> 11)) + 0.5) * 0x1.0p-53;
+  const double r = std::sqrt(-2.0 * std::log(u1));
+  *a = r * std::cos(6.283185307179586 * u2);
+  *b = r * std::sin(6.283185307179586 * u2);
+}
+
+static inline float to_f16_and_back(float x, bool* overflow) {
+  _Float16 h = (_Float16)x;  // round to nearest even
+  float y = (float)h;
+  if (!std::isfinite(y)) *overflow = true;
+  return y;
+}
+
+}  // namespace jolt
+
+using namespace jolt;
+
+extern "C" {
+
+const char* jolt_status_string(jolt_status s) {
+  switch (s) {
+    case JOLT_OK: return "ok";
+    case JOLT_ERR_INVALID_ARG: return "invalid argument";
+    case JOLT_ERR_CUDA: return "CUDA error";
+    case JOLT_ERR_TIMEOUT: return "device wait timed out";
+    case JOLT_ERR_BUDGET: return "byte budget infeasible";
+    case JOLT_ERR_NUMERIC: return "numeric range error";
+    case JOLT_ERR_WORKSPACE: return "workspace too small";
+    case JOLT_ERR_STATE: return "workspace not prepared by jolt_analyze";
+  }
+  return "unknown status";
+}
+
+int32_t jolt_version(void) { return 100; }
+
+jolt_status jolt_shape_check(const jolt_shape* s) {
+  return shape_ok(s) ? JOLT_OK : JOLT_ERR_INVALID_ARG;
+}
+
+uint64_t jolt_kv_bytes(int32_t n_layers, int32_t n_kv, int32_t d_h, int64_t T, int32_t dtype_bytes_) {
+  if (n_layers < 0 || n_kv < 0 || d_h < 0 || T < 0 || dtype_bytes_ < 0) return 0;
+  return 2ull * uint64_t(n_layers) * uint64_t(n_kv) * uint64_t(d_h) * uint64_t(T) *
+         uint64_t(dtype_bytes_);
+}
+
+uint64_t jolt_cell_bytes(const jolt_shape* s, jolt_cell_choice c) {
+  if (!shape_ok(s) || !choice_ok(*s, c)) return 0;
+  const uint64_t sf = dtype_bytes(s->factor_dtype);
+  const uint64_t T = s->T, d = s->d_h, Lg = s->layers_per_group, H = s->n_kv;
+  uint64_t bytes = sf * (T * c.r_T + d * c.r_d + Lg * H * uint64_t(c.r_T) * c.r_d);
+  if (c.b > 0) bytes += Lg * H * T * (d * c.b / 8 + 4);
+  return bytes;
+}
+
+jolt_status jolt_cache_layout(const jolt_shape* s, const jolt_cell_choice* choices,
+                              uint64_t* offsets, uint64_t* total_bytes) {
+  if (!shape_ok(s) || !choices || !total_bytes) return JOLT_ERR_INVALID_ARG;
+  const int nc = n_cells(*s);
+  uint64_t off = 0;
+  for (int c = 0; c < nc; ++c) {
+    if (!choice_ok(*s, choices[c])) return JOLT_ERR_INVALID_ARG;
+    CellSegs g = cell_segments(*s, choices[c]);
+    if (offsets) {
+      offsets[5 * c + 0] = off + g.ut;
+      offsets[5 * c + 1] = off + g.ud;
+      offsets[5 * c + 2] = off + g.g;
+      offsets[5 * c + 3] = off + g.codes;
+      offsets[5 * c + 4] = off + g.sz;
+    }
+    off += g.size;
+  }
+  *total_bytes = off;
+  return JOLT_OK;
+}
+
+jolt_status jolt_phi(int32_t d_h, int32_t n_rows, uint64_t seed, double phi_out[4]) {
+  if (!phi_out || d_h < 2 || d_h > 4096 || n_rows < 1) return JOLT_ERR_INVALID_ARG;
+  std::vector<float> row(d_h);
+  double tot = 0.0, err[3] = {0.0, 0.0, 0.0};
+  const int bits[3] = {2, 4, 8};
+  bool ovf = false;
+  for (int64_t r = 0; r < n_rows; ++r) {
+    for (int j = 0; j < d_h; j += 2) {
+      double a, b;
+      normal_pair(seed, uint64_t(r) * d_h + j, &a, &b);
+      row[j] = float(a);
+      if (j + 1 < d_h) row[j + 1] = float(b);
+    }
+    float mn = row[0], mx = row[0];
+    for (int j = 0; j < d_h; ++j) {
+      mn = std::min(mn, row[j]);
+      mx = std::max(mx, row[j]);
+      tot += double(row[j]) * double(row[j]);
+    }
+    for (int bi = 0; bi < 3; ++bi) {
+      const int b = bits[bi];
+      const float levels = float((1 << b) - 1);
+      const float rng = mx - mn;
+      const float step = rng / levels;
+      const float scale = to_f16_and_back(step, &ovf);
+      const float zero = to_f16_and_back(mn, &ovf);
+      for (int j = 0; j < d_h; ++j) {
+        float code = 0.f;
+        if (scale != 0.f) {
+          const float diff = row[j] - zero;
+          code = std::nearbyint(diff / scale);  // default rounding mode: nearest even
+          code = std::min(std::max(code, 0.f), levels);
+        }
+        const float deq = float(double(code) * double(scale) + double(zero));
+        const double e = double(row[j]) - double(deq);
+        err[bi] += e * e;
+      }
+    }
+  }
+  if (ovf) return JOLT_ERR_NUMERIC;
+  phi_out[0] = 1.0;
+  for (int bi = 0; bi < 3; ++bi) phi_out[bi + 1] = err[bi] / tot;
+  return JOLT_OK;
+}
+
+// ---- allocator ------------------------------------------------------------------------------
+
+namespace {
+struct Opt {
+  uint64_t B;
+  double E;
+  int rT, rd, b;
+};
+struct Seg {
+  double price;
+  int cell, idx;
+  uint64_t dB;
+};
+
+double cross3(const Opt& a, const Opt& b, const Opt& c) {
+  const double t1 = (double(b.B) - double(a.B)) * (c.E - a.E);
+  const double t2 = (b.E - a.E) * (double(c.B) - double(a.B));
+  return t1 - t2;
+}
+}  // namespace
+
+jolt_status jolt_allocate(const jolt_shape* s, int32_t nc, const double* norm2,
+                          const double* tail_T, int32_t nrt, const double* tail_d, int32_t nrd,
+                          const double phi[4], uint64_t budget, jolt_cell_choice* out,
+                          double* lambda_out, uint64_t* total_out) {
+  if (!shape_ok(s) || nc < 1 || !norm2 || !tail_T || !tail_d || !phi || !out) return JOLT_ERR_INVALID_ARG;
+  if (nrt < 1 || nrd < 1 || (nrt - 1) * kRankStep > s->q_cap || (nrd - 1) * kRankStep > s->d_h)
+    return JOLT_ERR_INVALID_ARG;
+  for (int i = 0; i < 4; ++i)
+    if (!(phi[i] >= 0.0) || !std::isfinite(phi[i])) return JOLT_ERR_INVALID_ARG;
+  const int bits[4] = {0, 2, 4, 8};
+  std::vector<std::vector<Opt>> hulls(nc);
+  for (int c = 0; c < nc; ++c) {
+    std::vector<Opt> opts;
+    opts.reserve(size_t(1 + (nrt - 1) * (nrd - 1)) * 4);
+    for (int k = 0; k < nrt; ++k) {
+      for (int j = 0; j < nrd; ++j) {
+        if ((k == 0) != (j == 0)) continue;
+        if (k == 0 && j != 0) continue;
+        double D;
+        if (k == 0) {
+          D = norm2[c];
+        } else {
+          const double sum = tail_T[size_t(c) * nrt + k] + tail_d[size_t(c) * nrd + j];
+          D = std::min(norm2[c], sum);
+        }
+        if (!std::isfinite(D)) return JOLT_ERR_NUMERIC;
+        for (int bi = 0; bi < 4; ++bi) {
+          jolt_cell_choice ch{k * kRankStep, j * kRankStep, bits[bi]};
+          Opt o;
+          o.B = jolt_cell_bytes(s, ch);
+          o.E = D * phi[bi];
+          o.rT = ch.r_T;
+          o.rd = ch.r_d;
+          o.b = ch.b;
+          opts.push_back(o);
+        }
+      }
+    }
+    std::sort(opts.begin(), opts.end(), [](const Opt& a, const Opt& b) {
+      if (a.B != b.B) return a.B < b.B;
+      if (a.E != b.E) return a.E < b.E;
+      if (a.rT != b.rT) return a.rT < b.rT;
+      if (a.rd != b.rd) return a.rd < b.rd;
+      return a.b < b.b;
+    });
+    std::vector<Opt> front;
+    for (const Opt& o : opts) {
+      if (!front.empty() && front.back().B == o.B) continue;
+      if (!front.empty() && !(o.E < front.back().E)) continue;
+      front.push_back(o);
+    }
+    std::vector<Opt>& h = hulls[c];
+    for (const Opt& o : front) {
+      while (h.size() >= 2 && cross3(h[h.size() - 2], h[h.size() - 1], o) <= 0.0) h.pop_back();
+      h.push_back(o);
+    }
+  }
+  uint64_t total = 0;
+  for (int c = 0; c < nc; ++c) total += hulls[c][0].B;
+  if (total > budget) return JOLT_ERR_BUDGET;
+  std::vector<Seg> segs;
+  for (int c = 0; c < nc; ++c) {
+    double prev = INFINITY;
+    const auto& h = hulls[c];
+    for (size_t i = 1; i < h.size(); ++i) {
+      const uint64_t dB = h[i].B - h[i - 1].B;
+      const double dE = h[i - 1].E - h[i].E;
+      double price = dE / double(dB);
+      price = std::min(price, prev);
+      prev = price;
+      segs.push_back(Seg{price, c, int(i), dB});
+    }
+  }
+  std::sort(segs.begin(), segs.end(), [](const Seg& a, const Seg& b) {
+    if (a.price != b.price) return a.price > b.price;
+    if (a.cell != b.cell) return a.cell < b.cell;
+    return a.idx < b.idx;
+  });
+  std::vector<int> pos(nc, 0);
+  double lam = 0.0;
+  for (const Seg& sg : segs) {
+    if (total + sg.dB <= budget) {
+      if (pos[sg.cell] != sg.idx - 1) return JOLT_ERR_NUMERIC;  // cannot happen on a valid hull
+      pos[sg.cell] = sg.idx;
+      total += sg.dB;
+    } else {
+      lam = sg.price;
+      break;
+    }
+  }
+  for (int c = 0; c < nc; ++c) {
+    const Opt& o = hulls[c][pos[c]];
+    out[c] = jolt_cell_choice{o.rT, o.rd, o.b};
+  }
+  if (lambda_out) *lambda_out = lam;
+  if (total_out) *total_out = total;
+  return JOLT_OK;
+}
+
+size_t jolt_workspace_bytes(const jolt_shape* s, int32_t op) {
+  if (!shape_ok(s)) return 0;
+  if (op == JOLT_OP_COMPRESS) return compress_workspace_bytes(*s);
+  if (op == JOLT_OP_DECODE) return decode_workspace_bytes(*s);
+  return 0;
+}
+
+}  // extern "C"

@@ -62,17 +62,19 @@ def st_hosvd(X: np.ndarray, r_T: int, r_d: int):
     L, H, T, d = X.shape
     XT = token_unfolding(X)
     U_T, sig2 = _token_svd(XT, r_T)
-    Y = np.einsum("tr,lhtj->lhrj", U_T, X)
-    S_Y = np.einsum("lhrj,lhrk->jk", Y, Y)
+    Y = np.matmul(U_T.T, X)                      # [L_g, n_kv, r_T, d_h]
+    Yf = Y.reshape(-1, d)
+    S_Y = Yf.T @ Yf
     U_d, lam_Y = _top_eigvecs(S_Y, r_d)
-    G = np.einsum("lhrj,jk->lhrk", Y, U_d)
+    G = np.matmul(Y, U_d)
     return U_T, U_d, G, sig2, lam_Y
 
 
 def reconstruct(U_T: np.ndarray, G: np.ndarray, U_d: np.ndarray) -> np.ndarray:
     """X~[l,h] = U_T G[l,h] U_d^T, float64 [L_g, n_kv, T, d_h]."""
-    return np.einsum("tr,lhrk,jk->lhtj", U_T.astype(np.float64), G.astype(np.float64),
-                     U_d.astype(np.float64))
+    U_T = np.asarray(U_T, dtype=np.float64)
+    return np.matmul(np.matmul(U_T, np.asarray(G, dtype=np.float64)),
+                     np.asarray(U_d, dtype=np.float64).T)
 
 
 def spectra_tails(X: np.ndarray, qcap: int, step: int = 16):
@@ -83,7 +85,8 @@ def spectra_tails(X: np.ndarray, qcap: int, step: int = 16):
     norm2 = float(np.sum(X * X))
     XT = token_unfolding(X)
     _, sig2 = _token_svd(XT, 0)
-    S_d = np.einsum("lhtj,lhtk->jk", X, X)
+    Xf = X.reshape(-1, d)
+    S_d = Xf.T @ Xf
     lam_d = np.linalg.eigvalsh(S_d)[::-1]
     csT = np.concatenate([[0.0], np.cumsum(sig2)])
     csd = np.concatenate([[0.0], np.cumsum(lam_d)])

@@ -1,0 +1,47 @@
+"""tcgen05 GEMM building block (jolt_gemm_bf16) vs a float64 product of the same bf16 inputs."""
+import pytest
+import torch
+
+from long_context_st_b200 import api
+
+pytestmark = pytest.mark.gpu
+
+
+def ref_mm(A, B, a_mn, b_mn):
+    A64 = A.double()
+    B64 = B.double()
+    Al = A64.transpose(-1, -2) if a_mn else A64       # [.., M, K]
+    Bl = B64 if b_mn else B64.transpose(-1, -2)       # [.., K, N]
+    return Al @ Bl
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("M,N,K", [(128, 128, 64), (1000, 1152, 1000), (304, 96, 4160),
+                                   (4096, 256, 128), (64, 384, 200)])
+def test_gemm_majors_and_ragged(cuda_ok, a_mn, b_mn, M, N, K):
+    g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K + a_mn * 2 + b_mn)
+    A = torch.randn((K, M) if a_mn else (M, K), generator=g, device="cuda").to(torch.bfloat16)
+    B = torch.randn((K, N) if b_mn else (N, K), generator=g, device="cuda").to(torch.bfloat16)
+    C = api.gemm_bf16(A, B, a_mn, b_mn)
+    torch.cuda.synchronize()
+    R = ref_mm(A, B, a_mn, b_mn)
+    err = (C.double() - R).abs().max().item() / R.abs().max().item()
+    assert err < tol(K), err
+
+
+def tol(K):
+    # fp32 accumulation of exact bf16 products: relative error grows like sqrt(K) * 2^-24
+    return 2e-7 * K ** 0.5 + 1e-6
+
+
+def test_gemm_split_k_and_batch(cuda_ok):
+    g = torch.Generator(device="cuda").manual_seed(1)
+    bt, M, N, K = 3, 384, 256, 8192
+    A = torch.randn(bt, K, M, generator=g, device="cuda").to(torch.bfloat16)
+    B = torch.randn(bt, K, N, generator=g, device="cuda").to(torch.bfloat16)
+    C = torch.zeros(bt, M, N, device="cuda")
+    api.gemm_bf16(A, B, True, True, C=C, k_split=8, accumulate=True)
+    torch.cuda.synchronize()
+    R = ref_mm(A, B, True, True)
+    err = (C.double() - R).abs().max().item() / R.abs().max().item()
+    assert err < tol(K), err

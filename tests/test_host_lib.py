@@ -1,0 +1,127 @@
+"""Host-side library checks (no GPU): exported symbols, byte model, layout, phi, allocator.
+
+The allocator must choose bit-identically to the oracle's when both get identical tables.
+"""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle.alloc import tables_to_options, allocate as oracle_allocate, BudgetError
+from oracle.bytes_model import cell_bytes as oracle_cell_bytes, raw_sequence_bytes
+from synth import get_workload, make_random_tables
+from long_context_st_b200 import api, _lib
+from long_context_st_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build()
+
+
+def header_symbols():
+    txt = open(os.path.join(ROOT, "include", "jolt.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(jolt_[a-z_0-9]+)\s*\(", txt)))
+
+
+def test_exports_every_declared_symbol():
+    L = _lib.lib()
+    syms = header_symbols()
+    assert len(syms) >= 14
+    for name in syms:
+        assert hasattr(L, name), name
+    declared = {n for n, _, _ in _lib.SIGNATURES}
+    assert set(syms) <= declared, set(syms) - declared
+
+
+def test_kv_bytes_formula():
+    assert api.kv_bytes(80, 8, 128, 1, 2) == 327680
+    assert api.kv_bytes(80, 64, 128, 1, 2) == 2621440
+    assert api.kv_bytes(80, 8, 128, 131072, 2) == 40 * 2 ** 30
+    assert api.kv_bytes(32, 8, 128, 2048, 2) == 268435456
+
+
+@pytest.mark.parametrize("name", ["toy", "llama8b_layer", "llama8b_32k", "llama70b_128k"])
+def test_cell_bytes_matches_oracle(name):
+    w = get_workload(name)
+    s = api.make_shape(w)
+    for ch in [(0, 0, 0), (0, 0, 2), (16, 16, 0), (32, 32, 4), (s.q_cap, w.d_h, 8), (64, 96, 2)]:
+        if ch[0] > s.q_cap or ch[1] > w.d_h:
+            continue
+        want = oracle_cell_bytes(w.T, w.d_h, w.layers_per_group, w.n_kv, w.factor_bytes, *ch)
+        assert api.cell_bytes(s, ch) == want
+
+
+def test_invalid_choices_and_shapes():
+    w = get_workload("toy")
+    s = api.make_shape(w)
+    assert api.cell_bytes(s, (16, 0, 0)) == 0      # r_T > 0 needs r_d > 0
+    assert api.cell_bytes(s, (8, 8, 0)) == 0       # not on the 16 grid
+    assert api.cell_bytes(s, (16, 16, 3)) == 0     # b not in {0,2,4,8}
+    with pytest.raises(api.JoltError):
+        api.make_shape(w, q_cap=48, sketch_cols=32)  # sketch narrower than the cap
+
+
+def test_cache_layout_alignment_and_sizes():
+    w = get_workload("llama8b_32k")
+    s = api.make_shape(w)
+    rng = np.random.default_rng(0)
+    nc = api.n_cells(s)
+    choices = []
+    for _ in range(nc):
+        rT = int(rng.integers(0, s.q_cap // 16 + 1)) * 16
+        rd = int(rng.integers(1, 9)) * 16 if rT else 0
+        choices.append((rT, rd, int(rng.choice([0, 2, 4, 8]))))
+    offs, total = api.cache_layout(s, choices)
+    assert np.all(offs % 256 == 0)
+    alg = sum(api.cell_bytes(s, c) for c in choices)
+    assert alg <= total <= alg + nc * 5 * 256
+    for c in range(nc - 1):
+        assert offs[c + 1, 0] >= offs[c, 4]
+
+
+def test_phi_agrees_with_oracle_statistically():
+    for d in (64, 128):
+        a = api.phi(d, 1 << 14, 3)
+        b = oracle.phi_table(d, 1 << 14, 1)
+        assert a[0] == 1.0
+        for x, y in zip(a[1:], b[1:]):
+            assert abs(x / y - 1) < 0.03
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_allocator_bit_exact_vs_oracle(seed):
+    w = get_workload(["llama8b_32k", "llama70b_128k", "toy", "llama8b_layer"][seed % 4])
+    s = api.make_shape(w)
+    nc = 2 * (w.n_layers // w.layers_per_group)
+    nrt, nrd = s.q_cap // 16 + 1, w.d_h // 16 + 1
+    n2, tT, td = make_random_tables(nc, nrt, nrd, 100 + seed)
+    phi = oracle.phi_table(w.d_h, 1 << 12, 1)
+    raw = raw_sequence_bytes(w)
+    opts = tables_to_options(n2, tT, td, phi, w)
+    for ratio in (2.0, 3.0, 5.0, 8.0):
+        budget = int(raw / ratio)
+        try:
+            want, lam_o, tot_o = oracle_allocate(opts, budget)
+        except BudgetError:
+            with pytest.raises(api.JoltError):
+                api.allocate(s, n2, tT, td, phi, budget)
+            continue
+        got, lam_g, tot_g = api.allocate(s, n2, tT, td, phi, budget)
+        assert [tuple(c) for c in got] == [tuple(c) for c in want]
+        assert lam_g == lam_o and tot_g == tot_o
+
+
+def test_allocator_zero_budget_stores_nothing():
+    # The empty choice (r_T = r_d = b = 0) costs no bytes, so every budget is feasible; at a
+    # zero budget every cell keeps nothing and its error is its whole mass.
+    w = get_workload("toy")
+    s = api.make_shape(w)
+    n2, tT, td = make_random_tables(2, s.q_cap // 16 + 1, w.d_h // 16 + 1, 1)
+    ch, lam, tot = api.allocate(s, n2, tT, td, [1.0, 0.1, 0.01, 0.0001], 0)
+    assert ch == [(0, 0, 0), (0, 0, 0)] and tot == 0 and lam > 0
