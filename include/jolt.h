@@ -223,6 +223,14 @@ jolt_status jolt_gemm_bf16(const void* A, int32_t a_mn_major, const void* B, int
                            int64_t ldc, int32_t batch, int64_t stride_a, int64_t stride_b,
                            int64_t stride_c, int32_t k_split, int32_t accumulate, void* stream);
 
+/* Symmetric eigendecomposition of `batch` fp32 matrices A [batch][n][n] (device) by block Jacobi
+ * (the solver the compressor uses for the Rayleigh-Ritz and feature-mode steps): eigenvalues
+ * descending into evals [batch][n], eigenvectors as the columns of evecs [batch][n][n] (device).
+ * ws (device) >= jolt_sym_eig_workspace(n, batch). Synchronises `stream`. */
+size_t jolt_sym_eig_workspace(int32_t n, int32_t batch);
+jolt_status jolt_sym_eig(const float* A, int32_t n, int32_t batch, float* evals, float* evecs,
+                         void* ws, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

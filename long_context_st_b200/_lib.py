@@ -65,6 +65,8 @@ SIGNATURES = [
     ("jolt_gemm_bf16", C.c_int, [_P, C.c_int32, _P, C.c_int32, _P, C.c_int32, C.c_int32, C.c_int32,
                                  C.c_int64, C.c_int64, C.c_int64, C.c_int32, C.c_int64, C.c_int64,
                                  C.c_int64, C.c_int32, C.c_int32, _P]),
+    ("jolt_sym_eig_workspace", C.c_size_t, [C.c_int32, C.c_int32]),
+    ("jolt_sym_eig", C.c_int, [_P, C.c_int32, C.c_int32, _P, _P, _P, C.c_size_t, _P]),
 ]
 
 _lib = None

@@ -189,7 +189,21 @@ def gemm_bf16(A, B, a_mn_major=False, b_mn_major=False, C=None, k_split=1, accum
     return C3 if batched else C3[0]
 
 
-__all__ = ["gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
+def sym_eig(A, stream=None):
+    """Eigen-decomposition of symmetric fp32 matrices [batch?, n, n] on the GPU (block Jacobi).
+    Returns (evals descending [batch?, n], evecs [batch?, n, n] with eigenvectors as columns)."""
+    batched = A.dim() == 3
+    A3 = (A if batched else A[None]).contiguous().float()
+    bt, n = A3.shape[0], A3.shape[1]
+    ev = torch.empty(bt, n, dtype=torch.float32, device=A.device)
+    V = torch.empty(bt, n, n, dtype=torch.float32, device=A.device)
+    ws = torch.empty(int(lib().jolt_sym_eig_workspace(n, bt)), dtype=torch.uint8, device=A.device)
+    check(lib().jolt_sym_eig(_ptr(A3), n, bt, _ptr(ev), _ptr(V), _ptr(ws), ws.numel(), _stream(stream)),
+          "jolt_sym_eig")
+    return (ev, V) if batched else (ev[0], V[0])
+
+
+__all__ = ["sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
            "allocate", "workspace_bytes", "new_workspace", "analyze", "compress", "decode_attn",
            "check_ws", "rotate_rows", "quantize_pack", "unpack_dequant", "JoltError",
            "JOLT_OP_COMPRESS", "JOLT_OP_DECODE"]

@@ -1,7 +1,856 @@
-// Placeholder, replaced by the compressor.
-#include "common.cuh"
+// jolt_analyze and jolt_compress: the compressor half of the codec.
+//
+// analyze, per pass of up to cells_per_pass cells of one kind (K or V), all batched:
+//   ||X||^2 (fp64), S_d = sum_lh X_lh^T X_lh (tcgen05), Y = X_(T) Omega (tcgen05, Rademacher Omega),
+//   q power iterations Y <- X_(T) orth(X_(T)^T orth(Y)), Q = orth(Y), B^T = X_(T)^T Q (hi/lo terms),
+//   W = B B^T, eig(W) (block Jacobi), U_T = Q V[:, :q_cap] (hi/lo terms) kept in the workspace.
+//   orth() is shifted CholeskyQR3: three passes of Gram (hi/lo terms) -> fp64 Cholesky of
+//   G + s*I -> Y R^{-1} (hi/lo terms), shifts 1e-4*max(diag), 1e-4*max(diag), 0.
+// compress, per cell: U_T (first r_T columns) stored; Y_lh = U_T^T X_lh (tcgen05);
+//   S_Y = sum Y_lh^T Y_lh; U_d = top-r_d eigenvectors (block Jacobi); G = Y U_d; X~ = U_T (G U_d^T)
+//   from the stored (rounded) factors (tcgen05, hi/lo terms); residual X - X~ rotated by the
+//   seeded randomized Hadamard, quantised per row and packed.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "gemm_tc.cuh"
+#include "linalg.cuh"
+#include "pack.cuh"
+
 namespace jolt {
-size_t compress_workspace_bytes(const jolt_shape& s) { (void)s; return 256; }
+
+namespace {
+
+constexpr uint64_t kAnalyzeMagic = 0x4A4F4C54414E4C5Aull;  // "JOLTANLZ"
+
+uint64_t shape_tag(const jolt_shape& s) {
+  uint64_t h = kAnalyzeMagic;
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(&s);
+  for (size_t i = 0; i < sizeof(jolt_shape) / 4; ++i) h = mix64(h ^ w[i]);
+  return h;
 }
-extern "C" jolt_status jolt_analyze(const jolt_shape*, const void*, const void*, double*, double*, double*, void*, size_t, void*) { return JOLT_ERR_INVALID_ARG; }
-extern "C" jolt_status jolt_compress(const jolt_shape*, const void*, const void*, const jolt_cell_choice*, void*, uint64_t, void*, size_t, void*) { return JOLT_ERR_INVALID_ARG; }
+
+struct Plan {
+  int C;          // cells per pass
+  int T, d, LgH, n, l, qcap;
+  int64_t cell_elems;
+  size_t off_ut, off_pass, off_cmp, total;
+  // pass scratch offsets (relative to off_pass)
+  size_t om, Y, Yh, Yl, Gm, Rh, Rl, Z, Zh, Zl, ev, evec, Vh, Vl, Sd, evd, evecd, nrm, chol, jac, xb;
+  size_t g64, ev64, evec64, sd64, evd64, evecd64;  // exact path (sketch width == n)
+  // compress scratch (relative to off_cmp)
+  size_t uh, ul, um, ylh, sy, evy, evecy, ud, blh, bh, bm, bl, xt, jac2;
+};
+
+Plan make_plan(const jolt_shape& s) {
+  Plan p{};
+  p.T = s.T;
+  p.d = s.d_h;
+  p.LgH = s.layers_per_group * s.n_kv;
+  p.n = p.LgH * p.d;
+  p.l = s.sketch_cols;
+  p.qcap = s.q_cap;
+  p.cell_elems = int64_t(p.LgH) * s.T * s.d_h;
+  const int per_kind = s.batch * n_groups(s);
+  p.C = std::max(1, std::min(s.cells_per_pass, per_kind));
+  const size_t C = p.C, T = p.T, l = std::max(p.l, 16), n = p.n, d = p.d, q = std::max(p.qcap, 16);
+  size_t off = sizeof(WsHeader);
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  p.off_ut = take(size_t(n_cells(s)) * T * q * 4);
+  const size_t pass0 = off;
+  auto rel = [&](size_t bytes) { return take(bytes) - pass0; };
+  p.off_pass = pass0;
+  const size_t rowsmax = std::max(T, n);
+  p.om = rel(l * n * 2);
+  p.Y = rel(C * rowsmax * l * 4);
+  p.Yh = rel(C * rowsmax * l * 2);
+  p.Yl = rel(C * rowsmax * l * 2);
+  p.Gm = rel(C * l * l * 4);
+  p.Rh = rel(C * l * l * 2);
+  p.Rl = rel(C * l * l * 2);
+  p.Z = rel(C * n * l * 4);
+  p.Zh = rel(C * n * l * 2);
+  p.Zl = rel(C * n * l * 2);
+  p.ev = rel(C * l * 4);
+  p.evec = rel(C * l * l * 4);
+  p.Vh = rel(C * l * l * 2);
+  p.Vl = rel(C * l * l * 2);
+  p.Sd = rel(C * d * d * 4);
+  p.evd = rel(C * d * 4);
+  p.evecd = rel(C * d * d * 4);
+  p.nrm = rel(C * 8);
+  p.chol = rel(chol_scratch_bytes(int(C), int(l)));
+  p.jac = rel(std::max(jacobi_scratch_bytes(int(C), int(l)), jacobi_scratch_bytes(int(C), int(d))));
+  p.xb = rel(s.io_dtype == JOLT_F32 ? 2 * C * size_t(p.cell_elems) * 2 : 0);  // hi/lo bf16 of f32 inputs
+  const bool exact = (p.l == p.n);
+  p.g64 = rel(exact ? C * n * n * 8 : 0);
+  p.ev64 = rel(exact ? C * n * 8 : 0);
+  p.evec64 = rel(exact ? C * n * n * 8 : 0);
+  p.sd64 = rel(C * d * d * 8);
+  p.evd64 = rel(C * d * 8);
+  p.evecd64 = rel(C * d * d * 8);
+  if (exact) p.jac = rel(std::max(jacobi_scratch_bytes(int(C), int(n)), jacobi_scratch_bytes(int(C), int(d))));
+  const size_t cmp0 = off;
+  auto relc = [&](size_t bytes) { return take(bytes) - cmp0; };
+  p.off_cmp = cmp0;
+  p.uh = relc(T * q * 2);
+  p.ul = relc(T * q * 2);
+  p.um = relc(T * q * 2);
+  p.ylh = relc(size_t(p.LgH) * q * d * 4);
+  p.sy = relc(d * d * 4);
+  p.evy = relc(d * 4);
+  p.evecy = relc(d * d * 4);
+  p.ud = relc(d * d * 4);
+  p.blh = relc(size_t(p.LgH) * q * d * 4);
+  p.bh = relc(size_t(p.LgH) * q * d * 2);
+  p.bm = relc(size_t(p.LgH) * q * d * 2);
+  p.bl = relc(size_t(p.LgH) * q * d * 2);
+  p.xt = relc(size_t(p.LgH) * T * d * 4);
+  p.jac2 = relc(jacobi_scratch_bytes(1, int(d)));
+  p.total = off;
+  return p;
+}
+
+// ---- small kernels ------------------------------------------------------------------------------
+
+__global__ void k_omega(__nv_bfloat16* om, int l, int n, uint64_t seed) {
+  const int64_t total = int64_t(l) * n;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    // om[j][i] = Omega[i][j]: the sketch matrix stored K-major (row j holds column j of Omega)
+    const int64_t j = e / n, i = e % n;
+    const uint64_t ctr = (seed << 32) + uint64_t(i) * uint64_t(l) + uint64_t(j);
+    om[e] = __float2bfloat16_rn((mix64(ctr) >> 63) ? -1.f : 1.f);
+  }
+}
+
+template <typename T>
+__global__ void k_norm2(const T* __restrict__ X, int64_t cell_elems, double* out) {
+  const int c = blockIdx.y;
+  const T* x = X + int64_t(c) * cell_elems;
+  double acc = 0.0;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < cell_elems; e += int64_t(gridDim.x) * blockDim.x) {
+    const double v = ld_as_float(x, e);
+    acc += v * v;
+  }
+  for (int m = 16; m; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if ((threadIdx.x & 31) == 0) atomicAdd(&out[c], acc);
+}
+
+__global__ void k_f32_to_bf16(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, int64_t n) {
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x)
+    y[e] = __float2bfloat16_rn(x[e]);
+}
+
+// Copy the first r columns of U [T][q] (fp32) to the stored cache (dtype) and to bf16 GEMM operands
+// [T][r]: hi, mid, lo with U ~ hi + mid + lo (mid may be null). With bf16 storage the stored
+// value is hi.
+__global__ void k_store_ut(const float* __restrict__ U, int T, int q, int r, int fac_f32, uint8_t* cache_ut,
+                           __nv_bfloat16* hi, __nv_bfloat16* mid, __nv_bfloat16* lo) {
+  const int64_t total = int64_t(T) * r;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t t = e / r, c = e % r;
+    const float v = U[t * q + c];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    if (fac_f32) reinterpret_cast<float*>(cache_ut)[e] = v;
+    else reinterpret_cast<__nv_bfloat16*>(cache_ut)[e] = h;
+    if (hi) hi[e] = h;
+    if (mid) {
+      mid[e] = m;
+      lo[e] = __float2bfloat16_rn(r1 - __bfloat162float(m));
+    } else if (lo) {
+      lo[e] = m;
+    }
+  }
+}
+
+// S = sum_b Y_b^T Y_b, Y [nb][r][d] fp32, S [d][d] fp32 (pre-zeroed), partial sums per CTA.
+__global__ void __launch_bounds__(256) k_gram_small(const float* __restrict__ Y, int nrows, int d, float* S) {
+  extern __shared__ float sy[];  // [32][d]
+  const int i0 = blockIdx.y * 32, j0 = blockIdx.z * 32;
+  const int ti = threadIdx.x / 32, tj = threadIdx.x % 32;  // 8 x 32 threads, 4 rows each
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int r0 = blockIdx.x * 32; r0 < nrows; r0 += gridDim.x * 32) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
+      const int rr = e / 64, cc = e % 64;
+      const int row = r0 + rr;
+      const int col = cc < 32 ? i0 + cc : j0 + cc - 32;
+      sy[rr * 64 + cc] = (row < nrows && col < d) ? Y[int64_t(row) * d + col] : 0.f;
+    }
+    __syncthreads();
+    for (int rr = 0; rr < 32; ++rr) {
+      const float bj = sy[rr * 64 + 32 + tj];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] += sy[rr * 64 + ti * 4 + u] * bj;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = i0 + ti * 4 + u, j = j0 + tj;
+    if (i < d && j < d) atomicAdd(&S[i * d + j], acc[u]);
+  }
+}
+
+// out[b][r][j] = sum_i Y[b][r][i] * M[i][j]  (Y [nb][r][d], M [d][ldm] first m columns)
+// optionally rounded to the factor dtype and written to the cache.
+__global__ void k_proj_small(const float* __restrict__ Y, int64_t nrows, int d, const float* __restrict__ M,
+                             int ldm, int m, int fac_f32, uint8_t* __restrict__ out) {
+  const int64_t total = nrows * m;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = e / m;
+    const int j = int(e % m);
+    float a = 0.f;
+    for (int i = 0; i < d; ++i) a += Y[r * d + i] * M[int64_t(i) * ldm + j];
+    if (fac_f32) reinterpret_cast<float*>(out)[e] = a;
+    else reinterpret_cast<__nv_bfloat16*>(out)[e] = __float2bfloat16_rn(a);
+  }
+}
+
+__device__ __forceinline__ float ld_fac_any(const uint8_t* p, int64_t i, int f32) {
+  return f32 ? reinterpret_cast<const float*>(p)[i] : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+// B[lh][r][i] = sum_j G[lh][r][j] * U_d[i][j] from the stored values (fp32 out).
+__global__ void k_recon_b(const uint8_t* __restrict__ G, const uint8_t* __restrict__ Ud, int64_t nrows, int rd,
+                          int d, int f32, float* __restrict__ B) {
+  const int64_t total = nrows * d;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = e / d;
+    const int i = int(e % d);
+    float a = 0.f;
+    for (int j = 0; j < rd; ++j) a += ld_fac_any(G, r * rd + j, f32) * ld_fac_any(Ud, int64_t(i) * rd + j, f32);
+    B[e] = a;
+  }
+}
+
+// Residual rows: x = X[row] - Xt[row] (Xt may be null), rotated, quantised and packed.
+template <int E, typename TX>
+__global__ void __launch_bounds__(256) k_residual(const TX* __restrict__ X, const float* __restrict__ Xt, int64_t rows,
+                                                  int b, uint64_t seed, uint8_t* __restrict__ codes,
+                                                  __half2* __restrict__ sz, int32_t* err) {
+  constexpr int D = 32 * E;
+  __shared__ uint8_t stage[8][D];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t warps = int64_t(gridDim.x) * 8;
+  const int nbytes = D * b / 8;
+  const float isd = rsqrtf(float(D));
+  for (int64_t r = int64_t(blockIdx.x) * 8 + w; r < rows; r += warps) {
+    float x[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const int64_t idx = r * D + lane * E + i;
+      x[i] = ld_as_float(X, idx) - (Xt ? Xt[idx] : 0.f);
+    }
+    warp_rotate<E>(x, seed, isd);
+    uint8_t c[E];
+    __half hs, hz;
+    bool ok = true;
+#pragma unroll
+    for (int i = 0; i < E; ++i) ok &= isfinite(x[i]);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!warp_quantize<E>(x, b, c, &hs, &hz)) ok = false;
+    if (!ok && lane == 0) report_error(err, JOLT_ERR_NUMERIC);
+    warp_pack_store<E>(c, b, stage[w], codes + r * nbytes);
+    if (lane == 0) sz[r] = __halves2half2(hs, hz);
+  }
+}
+
+// fp64 Gram of the token unfolding: G[a][b] += sum_t Xu[t][a] Xu[t][b], Xu(t, c) = X[c/d][t][c%d].
+// grid (n/64, n/64, C*ks); each CTA covers a 64x64 tile over its slice of t.
+template <typename TX>
+__global__ void __launch_bounds__(256) k_gram64(const TX* __restrict__ X, int64_t cell_elems, int T, int d, int n,
+                                                int ks, double* __restrict__ G) {
+  __shared__ double As[16][64], Bs[16][64];
+  const int a0 = blockIdx.x * 64, b0 = blockIdx.y * 64;
+  const int c = blockIdx.z / ks, kz = blockIdx.z % ks;
+  const TX* x = X + int64_t(c) * cell_elems;
+  const int chunk = (T + ks - 1) / ks;
+  const int t_beg = kz * chunk, t_end = min(T, t_beg + chunk);
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[4][4] = {};
+  const int la = a0 / d, ja = a0 % d, lb = b0 / d, jb = b0 % d;
+  for (int t0 = t_beg; t0 < t_end; t0 += 16) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < 16 * 64; e += blockDim.x) {
+      const int tt = e / 64, cc = e % 64, t = t0 + tt;
+      const bool ok = t < t_end;
+      As[tt][cc] = ok ? double(ld_as_float(x, (int64_t(la) * T + t) * d + ja + cc)) : 0.0;
+      Bs[tt][cc] = ok ? double(ld_as_float(x, (int64_t(lb) * T + t) * d + jb + cc)) : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int tt = 0; tt < 16; ++tt) {
+      double av[4], bv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) av[u] = As[tt][ty * 4 + u];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) bv[v] = Bs[tt][tx * 4 + v];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] += av[u] * bv[v];
+    }
+  }
+  double* g = G + int64_t(c) * n * n;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) atomicAdd(&g[int64_t(a0 + ty * 4 + u) * n + b0 + tx * 4 + v], acc[u][v]);
+}
+
+// U[t][r] = sum_c Xu[t][c] V[c][r] / sqrt(lambda_r)  (fp64 math, fp32 out), r < q; grid (q/64, ceil(T/64), C)
+template <typename TX>
+__global__ void __launch_bounds__(256) k_xv64(const TX* __restrict__ X, int64_t cell_elems, int T, int d, int n,
+                                              const double* __restrict__ Vv, const double* __restrict__ lam, int q,
+                                              float* __restrict__ U, int64_t u_cell_stride) {
+  __shared__ double As[64][17], Bs[16][64];
+  const int r0 = blockIdx.x * 64, t0 = blockIdx.y * 64, c = blockIdx.z;
+  const TX* x = X + int64_t(c) * cell_elems;
+  const double* vv = Vv + int64_t(c) * n * n;
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[4][4] = {};
+  for (int c0 = 0; c0 < n; c0 += 16) {
+    __syncthreads();
+    const int lh = c0 / d, j0 = c0 % d;
+    for (int e = threadIdx.x; e < 64 * 16; e += blockDim.x) {
+      const int tt = e / 16, cc = e % 16, t = t0 + tt;
+      As[tt][cc] = (t < T) ? double(ld_as_float(x, (int64_t(lh) * T + t) * d + j0 + cc)) : 0.0;
+      const int rr = e % 64, kk = e / 64;
+      Bs[kk][rr] = (r0 + rr < q) ? vv[int64_t(c0 + kk) * n + r0 + rr] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < 16; ++kk) {
+      double av[4], bv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) av[u] = As[ty * 4 + u][kk];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) bv[v] = Bs[kk][tx * 4 + v];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] += av[u] * bv[v];
+    }
+  }
+  float* out = U + int64_t(c) * u_cell_stride;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const int r = r0 + tx * 4 + v;
+    if (r >= q) continue;
+    const double lm = lam[int64_t(c) * n + r];
+    const double inv = lm > 1e-300 ? 1.0 / sqrt(lm) : 0.0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int t = t0 + ty * 4 + u;
+      if (t < T) out[int64_t(t) * q + r] = float(acc[u][v] * inv);
+    }
+  }
+}
+
+// S_d = sum over the d x d diagonal blocks of the token-unfolding Gram.
+__global__ void k_diag_blocks(const double* __restrict__ G, int n, int d, int nblk, double* __restrict__ Sd) {
+  const int c = blockIdx.y;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < d * d; e += gridDim.x * blockDim.x) {
+    const int i = e / d, j = e % d;
+    double a = 0.0;
+    for (int b = 0; b < nblk; ++b) a += G[int64_t(c) * n * n + int64_t(b * d + i) * n + b * d + j];
+    Sd[int64_t(c) * d * d + e] = a;
+  }
+}
+
+int grid1(int64_t n) { return int(std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 148 * 16))); }
+
+int ksplit_for(int64_t tiles, int64_t K) {
+  int64_t want = (2 * 148 + tiles - 1) / tiles;
+  const int64_t kblocks = (K + 63) / 64;
+  want = std::min<int64_t>(want, std::max<int64_t>(1, kblocks / 8));
+  return int(std::max<int64_t>(1, std::min<int64_t>(want, 64)));
+}
+
+struct Ctx {
+  const jolt_shape* s;
+  Plan p;
+  uint8_t* ws;
+  int32_t* err;
+  cudaStream_t st;
+  uint8_t* pass() const { return ws + p.off_pass; }
+  template <typename Tp> Tp* at(size_t rel) const { return reinterpret_cast<Tp*>(pass() + rel); }
+  template <typename Tp> Tp* atc(size_t rel) const { return reinterpret_cast<Tp*>(ws + p.off_cmp + rel); }
+};
+
+Operand plain(const void* ptr, int major, int64_t inner, int64_t outer, int64_t ld, int64_t batch = 1,
+              int64_t bstride = 0) {
+  Operand o;
+  o.ptr = ptr;
+  o.major = major;
+  o.inner = inner;
+  o.outer = outer;
+  o.outer_stride = ld;
+  o.batch = batch;
+  o.batch_stride = bstride;
+  return o;
+}
+
+// X_(T) of a cell batch: rows t, columns (lh, j); folded inner index (lh, j) with fold d.
+Operand xunfold(const void* X, int major, const Plan& p, int C) {
+  Operand o;
+  o.ptr = X;
+  o.major = major;
+  o.inner = p.d;
+  o.fold = p.d;
+  o.nfold = p.LgH;
+  o.fold_stride = int64_t(p.T) * p.d;
+  o.outer = p.T;
+  o.outer_stride = p.d;
+  o.batch = C;
+  o.batch_stride = p.cell_elems;
+  return o;
+}
+
+// Y <- orth(Y), Y fp32 [C][rows][l]; shifted CholeskyQR3 with hi/lo bf16 Grams and products.
+jolt_status orth(const Ctx& c, float* Y, int rows, int C) {
+  const Plan& p = c.p;
+  const int l = p.l;
+  __nv_bfloat16* Yh = c.at<__nv_bfloat16>(p.Yh);
+  __nv_bfloat16* Yl = c.at<__nv_bfloat16>(p.Yl);
+  float* Gm = c.at<float>(p.Gm);
+  __nv_bfloat16* Rh = c.at<__nv_bfloat16>(p.Rh);
+  __nv_bfloat16* Rl = c.at<__nv_bfloat16>(p.Rl);
+  const double shifts[3] = {1e-4, 1e-4, 0.0};
+  for (int pass = 0; pass < 3; ++pass) {
+    jolt_status r = split_bf16(Y, l, rows, l, C, int64_t(rows) * l, Yh, Yl, l, int64_t(rows) * l, c.st);
+    if (r) return r;
+    JOLT_CUDA_TRY(cudaMemsetAsync(Gm, 0, size_t(C) * l * l * 4, c.st));
+    GemmCall g;
+    g.M = l; g.N = l; g.K = rows; g.n_terms = 3;
+    const Operand yh = plain(Yh, kMajorMN, l, rows, l, C, int64_t(rows) * l);
+    const Operand yl = plain(Yl, kMajorMN, l, rows, l, C, int64_t(rows) * l);
+    g.A[0] = yh; g.B[0] = yh;
+    g.A[1] = yh; g.B[1] = yl;
+    g.A[2] = yl; g.B[2] = yh;
+    g.C = Gm; g.ldc = l; g.c_batch_stride = int64_t(l) * l; g.batch = C;
+    g.k_split = ksplit_for(int64_t((l + 127) / 128) * ((l + 255) / 256) * C, rows);
+    g.accumulate = true; g.err = c.err;
+    if ((r = gemm_tc(g, c.st))) return r;
+    if ((r = chol_inverse(Gm, l, C, l, shifts[pass], Rh, Rl, c.pass() + p.chol, c.err, c.st))) return r;
+    GemmCall t;
+    t.M = rows; t.N = l; t.K = l; t.n_terms = 3;
+    const Operand ykh = plain(Yh, kMajorK, l, rows, l, C, int64_t(rows) * l);
+    const Operand ykl = plain(Yl, kMajorK, l, rows, l, C, int64_t(rows) * l);
+    const Operand rh = plain(Rh, kMajorMN, l, l, l, C, int64_t(l) * l);
+    const Operand rl = plain(Rl, kMajorMN, l, l, l, C, int64_t(l) * l);
+    t.A[0] = ykh; t.B[0] = rh;
+    t.A[1] = ykh; t.B[1] = rl;
+    t.A[2] = ykl; t.B[2] = rh;
+    t.C = Y; t.ldc = l; t.c_batch_stride = int64_t(rows) * l; t.batch = C; t.err = c.err;
+    if ((r = gemm_tc(t, c.st))) return r;
+  }
+  return JOLT_OK;
+}
+
+// One pass: cells [bg0, bg0 + C) of kind kv. Writes U_T to the persistent region and the spectra
+// (eigenvalues of W and S_d, ||X||^2) to host arrays.
+jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C, std::vector<double>& evT,
+                         std::vector<double>& evD, std::vector<double>& nrm) {
+  const Plan& p = c.p;
+  const jolt_shape& s = *c.s;
+  const int T = p.T, n = p.n, l = p.l, d = p.d, q = p.qcap;
+  const bool io32 = s.io_dtype == JOLT_F32;
+  const uint8_t* X = static_cast<const uint8_t*>(Xkind) + int64_t(bg0) * p.cell_elems * (io32 ? 4 : 2);
+  jolt_status r;
+  // ||X||^2
+  double* nr = c.at<double>(p.nrm);
+  JOLT_CUDA_TRY(cudaMemsetAsync(nr, 0, C * 8, c.st));
+  if (io32) k_norm2<float><<<dim3(148, C), 256, 0, c.st>>>(reinterpret_cast<const float*>(X), p.cell_elems, nr);
+  else k_norm2<__nv_bfloat16><<<dim3(148, C), 256, 0, c.st>>>(reinterpret_cast<const __nv_bfloat16*>(X), p.cell_elems, nr);
+  // f32 inputs enter the tensor cores as hi + lo bf16 parts (bf16 inputs are exact as they are)
+  const void* Xb = X;
+  const void* Xlo = nullptr;
+  if (io32) {
+    __nv_bfloat16* xh = c.at<__nv_bfloat16>(p.xb);
+    __nv_bfloat16* xl = xh + int64_t(C) * p.cell_elems;
+    if ((r = split_bf16(reinterpret_cast<const float*>(X), 1, int64_t(C) * p.cell_elems, 1, 1, 0, xh, xl, 1, 0, c.st)))
+      return r;
+    Xb = xh;
+    Xlo = xl;
+  }
+  // S_d = sum_lh X_lh^T X_lh
+  float* Sd = c.at<float>(p.Sd);
+  JOLT_CUDA_TRY(cudaMemsetAsync(Sd, 0, size_t(C) * d * d * 4, c.st));
+  {
+    GemmCall g;
+    g.M = d; g.N = d; g.K = T;
+    const Operand xh = plain(Xb, kMajorMN, d, T, d, int64_t(C) * p.LgH, int64_t(T) * d);
+    g.A[0] = xh; g.B[0] = xh;
+    if (Xlo) {
+      const Operand xl = plain(Xlo, kMajorMN, d, T, d, int64_t(C) * p.LgH, int64_t(T) * d);
+      g.n_terms = 3;
+      g.A[1] = xh; g.B[1] = xl;
+      g.A[2] = xl; g.B[2] = xh;
+    }
+    g.C = Sd; g.ldc = d; g.c_batch_stride = int64_t(d) * d; g.c_batch_div = p.LgH;
+    g.batch = C * p.LgH; g.k_split = ksplit_for(int64_t(C) * p.LgH, T); g.accumulate = true; g.err = c.err;
+    if ((r = gemm_tc(g, c.st))) return r;
+  }
+  const bool exact = (p.l == p.n);
+  if (exact && q > 0) {
+    // sketch width == n: the range finder would span all of X_(T); take the exact token-mode
+    // spectrum instead, in fp64: G = X_(T)^T X_(T), eig(G), U_T = X_(T) V / sigma.
+    double* G64 = c.at<double>(p.g64);
+    double* ev64 = c.at<double>(p.ev64);
+    double* evec64 = c.at<double>(p.evec64);
+    JOLT_CUDA_TRY(cudaMemsetAsync(G64, 0, size_t(C) * n * n * 8, c.st));
+    const int nt = (n + 63) / 64;
+    const int ks = std::max(1, std::min(64, int((2 * 148 + int64_t(nt) * nt * C - 1) / (int64_t(nt) * nt * C))));
+    const dim3 gg(nt, nt, C * ks);
+    if (io32) k_gram64<float><<<gg, 256, 0, c.st>>>(reinterpret_cast<const float*>(X), p.cell_elems, T, d, n, ks, G64);
+    else k_gram64<__nv_bfloat16><<<gg, 256, 0, c.st>>>(reinterpret_cast<const __nv_bfloat16*>(X), p.cell_elems, T, d, n, ks, G64);
+    JOLT_CUDA_TRY(cudaGetLastError());
+    if ((r = jacobi_eig64(G64, n, C, n, ev64, evec64, c.pass() + p.jac, 30, 1e-13, c.err, c.st))) return r;
+    float* Ut = reinterpret_cast<float*>(c.ws + p.off_ut) + (int64_t(bg0) * 2 + kv) * int64_t(T) * q;
+    const dim3 gx((q + 63) / 64, (T + 63) / 64, C);
+    if (io32) k_xv64<float><<<gx, 256, 0, c.st>>>(reinterpret_cast<const float*>(X), p.cell_elems, T, d, n, evec64, ev64, q, Ut, 2 * int64_t(T) * q);
+    else k_xv64<__nv_bfloat16><<<gx, 256, 0, c.st>>>(reinterpret_cast<const __nv_bfloat16*>(X), p.cell_elems, T, d, n, evec64, ev64, q, Ut, 2 * int64_t(T) * q);
+    JOLT_CUDA_TRY(cudaGetLastError());
+    std::vector<double> e64(size_t(C) * n);
+    JOLT_CUDA_TRY(cudaMemcpyAsync(e64.data(), ev64, size_t(C) * n * 8, cudaMemcpyDeviceToHost, c.st));
+    // exact feature Gram from the diagonal blocks
+    double* sd64 = c.at<double>(p.sd64);
+    double* evd64 = c.at<double>(p.evd64);
+    double* evecd64 = c.at<double>(p.evecd64);
+    k_diag_blocks<<<dim3(std::max(1, d * d / 256), C), 256, 0, c.st>>>(G64, n, d, p.LgH, sd64);
+    if ((r = jacobi_eig64(sd64, d, C, d, evd64, evecd64, c.pass() + p.jac, 30, 1e-13, c.err, c.st))) return r;
+    std::vector<double> d64(size_t(C) * d);
+    JOLT_CUDA_TRY(cudaMemcpyAsync(d64.data(), evd64, size_t(C) * d * 8, cudaMemcpyDeviceToHost, c.st));
+    nrm.resize(C);
+    JOLT_CUDA_TRY(cudaMemcpyAsync(nrm.data(), nr, size_t(C) * 8, cudaMemcpyDeviceToHost, c.st));
+    JOLT_CUDA_TRY(cudaStreamSynchronize(c.st));
+    evT.assign(e64.begin(), e64.end());
+    evD.assign(d64.begin(), d64.end());
+    return JOLT_OK;
+  }
+  if (q > 0) {
+    float* Y = c.at<float>(p.Y);
+    float* Z = c.at<float>(p.Z);
+    __nv_bfloat16* Yh = c.at<__nv_bfloat16>(p.Yh);
+    __nv_bfloat16* Yl = c.at<__nv_bfloat16>(p.Yl);
+    __nv_bfloat16* Zh = c.at<__nv_bfloat16>(p.Zh);
+    __nv_bfloat16* Zl = c.at<__nv_bfloat16>(p.Zl);
+    const __nv_bfloat16* om = c.at<__nv_bfloat16>(p.om);
+    // Y = X Omega
+    {
+      GemmCall g;
+      g.M = T; g.N = l; g.K = n;
+      g.A[0] = xunfold(Xb, kMajorK, p, C);
+      g.B[0] = plain(om, kMajorK, n, l, n);
+      g.C = Y; g.ldc = l; g.c_batch_stride = int64_t(T) * l; g.batch = C; g.err = c.err;
+      if ((r = gemm_tc(g, c.st))) return r;
+    }
+    for (int it = 0; it < s.power_iters; ++it) {
+      if ((r = orth(c, Y, T, C))) return r;
+      if ((r = split_bf16(Y, l, T, l, C, int64_t(T) * l, Yh, nullptr, l, int64_t(T) * l, c.st))) return r;
+      JOLT_CUDA_TRY(cudaMemsetAsync(Z, 0, size_t(C) * n * l * 4, c.st));
+      GemmCall g;
+      g.M = n; g.N = l; g.K = T;
+      g.A[0] = xunfold(Xb, kMajorMN, p, C);
+      g.B[0] = plain(Yh, kMajorMN, l, T, l, C, int64_t(T) * l);
+      g.C = Z; g.ldc = l; g.c_batch_stride = int64_t(n) * l; g.batch = C;
+      g.k_split = ksplit_for(int64_t((n + 127) / 128) * ((l + 255) / 256) * C, T); g.accumulate = true; g.err = c.err;
+      if ((r = gemm_tc(g, c.st))) return r;
+      if ((r = orth(c, Z, n, C))) return r;
+      if ((r = split_bf16(Z, l, n, l, C, int64_t(n) * l, Zh, nullptr, l, int64_t(n) * l, c.st))) return r;
+      GemmCall h;
+      h.M = T; h.N = l; h.K = n;
+      h.A[0] = xunfold(Xb, kMajorK, p, C);
+      h.B[0] = plain(Zh, kMajorMN, l, n, l, C, int64_t(n) * l);
+      h.C = Y; h.ldc = l; h.c_batch_stride = int64_t(T) * l; h.batch = C; h.err = c.err;
+      if ((r = gemm_tc(h, c.st))) return r;
+    }
+    if ((r = orth(c, Y, T, C))) return r;  // Q
+    if ((r = split_bf16(Y, l, T, l, C, int64_t(T) * l, Yh, Yl, l, int64_t(T) * l, c.st))) return r;
+    // B^T = X^T Q  (n x l), hi/lo terms of Q
+    JOLT_CUDA_TRY(cudaMemsetAsync(Z, 0, size_t(C) * n * l * 4, c.st));
+    {
+      GemmCall g;
+      g.M = n; g.N = l; g.K = T; g.n_terms = 2;
+      g.A[0] = xunfold(Xb, kMajorMN, p, C);
+      g.A[1] = g.A[0];
+      g.B[0] = plain(Yh, kMajorMN, l, T, l, C, int64_t(T) * l);
+      g.B[1] = plain(Yl, kMajorMN, l, T, l, C, int64_t(T) * l);
+      if (Xlo) {
+        g.n_terms = 3;
+        g.A[2] = xunfold(Xlo, kMajorMN, p, C);
+        g.B[2] = g.B[0];
+      }
+      g.C = Z; g.ldc = l; g.c_batch_stride = int64_t(n) * l; g.batch = C;
+      g.k_split = ksplit_for(int64_t((n + 127) / 128) * ((l + 255) / 256) * C, T); g.accumulate = true; g.err = c.err;
+      if ((r = gemm_tc(g, c.st))) return r;
+    }
+    // W = B B^T = (B^T)^T (B^T), hi/lo terms
+    if ((r = split_bf16(Z, l, n, l, C, int64_t(n) * l, Zh, Zl, l, int64_t(n) * l, c.st))) return r;
+    float* W = c.at<float>(p.Gm);
+    JOLT_CUDA_TRY(cudaMemsetAsync(W, 0, size_t(C) * l * l * 4, c.st));
+    {
+      GemmCall g;
+      g.M = l; g.N = l; g.K = n; g.n_terms = 3;
+      const Operand zh = plain(Zh, kMajorMN, l, n, l, C, int64_t(n) * l);
+      const Operand zl = plain(Zl, kMajorMN, l, n, l, C, int64_t(n) * l);
+      g.A[0] = zh; g.B[0] = zh;
+      g.A[1] = zh; g.B[1] = zl;
+      g.A[2] = zl; g.B[2] = zh;
+      g.C = W; g.ldc = l; g.c_batch_stride = int64_t(l) * l; g.batch = C;
+      g.k_split = ksplit_for(int64_t((l + 127) / 128) * ((l + 255) / 256) * C, n); g.accumulate = true; g.err = c.err;
+      if ((r = gemm_tc(g, c.st))) return r;
+    }
+    float* ev = c.at<float>(p.ev);
+    float* evec = c.at<float>(p.evec);
+    if ((r = jacobi_eig(W, l, C, l, ev, evec, c.pass() + p.jac, 30, 1e-10, c.err, c.st))) return r;
+    __nv_bfloat16* Vh = c.at<__nv_bfloat16>(p.Vh);
+    __nv_bfloat16* Vl = c.at<__nv_bfloat16>(p.Vl);
+    if ((r = split_bf16(evec, l, l, l, C, int64_t(l) * l, Vh, Vl, l, int64_t(l) * l, c.st))) return r;
+    // U_T = Q V[:, :q]
+    {
+      float* Ut = reinterpret_cast<float*>(c.ws + p.off_ut) + (int64_t(bg0) * 2 + kv) * int64_t(T) * q;
+      GemmCall g;
+      g.M = T; g.N = q; g.K = l; g.n_terms = 3;
+      const Operand qh = plain(Yh, kMajorK, l, T, l, C, int64_t(T) * l);
+      const Operand ql = plain(Yl, kMajorK, l, T, l, C, int64_t(T) * l);
+      const Operand vh = plain(Vh, kMajorMN, q, l, l, C, int64_t(l) * l);
+      const Operand vl = plain(Vl, kMajorMN, q, l, l, C, int64_t(l) * l);
+      g.A[0] = qh; g.B[0] = vh;
+      g.A[1] = qh; g.B[1] = vl;
+      g.A[2] = ql; g.B[2] = vh;
+      g.C = Ut; g.ldc = q; g.c_batch_stride = 2 * int64_t(T) * q; g.batch = C; g.err = c.err;
+      if ((r = gemm_tc(g, c.st))) return r;
+    }
+    std::vector<float> e32(size_t(C) * l);
+    JOLT_CUDA_TRY(cudaMemcpyAsync(e32.data(), ev, size_t(C) * l * 4, cudaMemcpyDeviceToHost, c.st));
+    JOLT_CUDA_TRY(cudaStreamSynchronize(c.st));
+    evT.assign(e32.begin(), e32.end());
+  }
+  float* evd = c.at<float>(p.evd);
+  float* evecd = c.at<float>(p.evecd);
+  if ((r = jacobi_eig(Sd, d, C, d, evd, evecd, c.pass() + p.jac, 30, 1e-10, c.err, c.st))) return r;
+  std::vector<float> d32(size_t(C) * d);
+  nrm.resize(C);
+  JOLT_CUDA_TRY(cudaMemcpyAsync(d32.data(), evd, size_t(C) * d * 4, cudaMemcpyDeviceToHost, c.st));
+  JOLT_CUDA_TRY(cudaMemcpyAsync(nrm.data(), nr, size_t(C) * 8, cudaMemcpyDeviceToHost, c.st));
+  JOLT_CUDA_TRY(cudaStreamSynchronize(c.st));
+  evD.assign(d32.begin(), d32.end());
+  return JOLT_OK;
+}
+
+jolt_status read_err(const Ctx& c) {
+  int32_t e = 0;
+  JOLT_CUDA_TRY(cudaMemcpyAsync(&e, c.err, 4, cudaMemcpyDeviceToHost, c.st));
+  JOLT_CUDA_TRY(cudaStreamSynchronize(c.st));
+  return static_cast<jolt_status>(e);
+}
+
+}  // namespace
+
+size_t compress_workspace_bytes(const jolt_shape& s) { return make_plan(s).total; }
+
+}  // namespace jolt
+
+using namespace jolt;
+
+extern "C" jolt_status jolt_analyze(const jolt_shape* shape, const void* k, const void* v, double* norm2_out,
+                                    double* tail_T_out, double* tail_d_out, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  if (!shape_ok(shape) || !k || !v || !norm2_out || !tail_T_out || !tail_d_out || !ws) return JOLT_ERR_INVALID_ARG;
+  const jolt_shape& s = *shape;
+  Ctx c;
+  c.s = shape;
+  c.p = make_plan(s);
+  if (ws_bytes < c.p.total) return JOLT_ERR_WORKSPACE;
+  c.ws = static_cast<uint8_t*>(ws);
+  c.err = reinterpret_cast<int32_t*>(ws);
+  c.st = static_cast<cudaStream_t>(stream);
+  const Plan& p = c.p;
+  WsHeader hdr;
+  memset(&hdr, 0, sizeof(hdr));
+  JOLT_CUDA_TRY(cudaMemcpyAsync(ws, &hdr, sizeof(hdr), cudaMemcpyHostToDevice, c.st));
+  if (p.qcap > 0) {
+    k_omega<<<grid1(int64_t(p.l) * p.n), 256, 0, c.st>>>(c.at<__nv_bfloat16>(p.om), p.l, p.n, s.sketch_seed);
+    JOLT_CUDA_TRY(cudaGetLastError());
+  }
+  const int per_kind = s.batch * n_groups(s);
+  const int nrt = n_rt(s), nrd = n_rd(s);
+  const bool exact_path = (p.l == p.n);
+  for (int kv = 0; kv < 2; ++kv) {
+    for (int bg0 = 0; bg0 < per_kind; bg0 += p.C) {
+      const int C = std::min(p.C, per_kind - bg0);
+      std::vector<double> evT, evD;
+      std::vector<double> nrm;
+      jolt_status r = analyze_pass(c, kv ? v : k, kv, bg0, C, evT, evD, nrm);
+      if (r) return r;
+      if ((r = read_err(c))) return r;
+      for (int i = 0; i < C; ++i) {
+        const int cell = (bg0 + i) * 2 + kv;
+        const double n2 = nrm[i];
+        if (!std::isfinite(n2)) return JOLT_ERR_NUMERIC;
+        norm2_out[cell] = n2;
+        double cum = 0.0;
+        for (int kk = 0; kk < nrt; ++kk) {
+          if (kk > 0)
+            for (int j = (kk - 1) * kRankStep; j < kk * kRankStep; ++j) cum += std::max(0.0, evT[size_t(i) * (exact_path ? p.n : p.l) + j]);
+          tail_T_out[size_t(cell) * nrt + kk] = std::max(0.0, n2 - cum);
+        }
+        cum = 0.0;
+        for (int jj = 0; jj < nrd; ++jj) {
+          if (jj > 0)
+            for (int j = (jj - 1) * kRankStep; j < jj * kRankStep; ++j) cum += std::max(0.0, evD[size_t(i) * p.d + j]);
+          tail_d_out[size_t(cell) * nrd + jj] = std::max(0.0, n2 - cum);
+        }
+      }
+    }
+  }
+  hdr.analyze_tag = shape_tag(s);
+  JOLT_CUDA_TRY(cudaMemcpyAsync(&reinterpret_cast<WsHeader*>(ws)->analyze_tag, &hdr.analyze_tag, 8,
+                                cudaMemcpyHostToDevice, c.st));
+  JOLT_CUDA_TRY(cudaStreamSynchronize(c.st));
+  return JOLT_OK;
+}
+
+extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, const void* v,
+                                     const jolt_cell_choice* choices, void* cache, uint64_t cache_bytes, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  if (!shape_ok(shape) || !k || !v || !choices || !cache || !ws) return JOLT_ERR_INVALID_ARG;
+  const jolt_shape& s = *shape;
+  Ctx c;
+  c.s = shape;
+  c.p = make_plan(s);
+  const Plan& p = c.p;
+  if (ws_bytes < p.total) return JOLT_ERR_WORKSPACE;
+  c.ws = static_cast<uint8_t*>(ws);
+  c.err = reinterpret_cast<int32_t*>(ws);
+  c.st = static_cast<cudaStream_t>(stream);
+  uint64_t total = 0;
+  const int nc = n_cells(s);
+  std::vector<uint64_t> offs(size_t(nc) * 5);
+  jolt_status r = jolt_cache_layout(shape, choices, offs.data(), &total);
+  if (r) return r;
+  if (cache_bytes < total) return JOLT_ERR_INVALID_ARG;
+  uint64_t tag = 0;
+  JOLT_CUDA_TRY(cudaMemcpyAsync(&tag, &reinterpret_cast<WsHeader*>(ws)->analyze_tag, 8, cudaMemcpyDeviceToHost, c.st));
+  JOLT_CUDA_TRY(cudaStreamSynchronize(c.st));
+  if (tag != shape_tag(s)) return JOLT_ERR_STATE;
+  const bool io32 = s.io_dtype == JOLT_F32, f32 = s.factor_dtype == JOLT_F32;
+  const int T = p.T, d = p.d, q = p.qcap, LgH = p.LgH;
+  uint8_t* cb = static_cast<uint8_t*>(cache);
+  for (int cell = 0; cell < nc; ++cell) {
+    const int bg = cell / 2, kv = cell % 2;
+    const jolt_cell_choice ch = choices[cell];
+    const uint8_t* Xk = static_cast<const uint8_t*>(kv ? v : k) + int64_t(bg) * p.cell_elems * (io32 ? 4 : 2);
+    float* Xt = nullptr;
+    if (ch.r_T > 0) {
+      const int rT = ch.r_T, rd = ch.r_d;
+      const float* U = reinterpret_cast<const float*>(c.ws + p.off_ut) + int64_t(cell) * T * q;
+      uint8_t* cut = cb + offs[5 * cell + 0];
+      uint8_t* cud = cb + offs[5 * cell + 1];
+      uint8_t* cg = cb + offs[5 * cell + 2];
+      // GEMM parts of U: hi (the stored value for bf16 factors), lo (and mid for fp32 factors)
+      __nv_bfloat16* uh = f32 ? c.atc<__nv_bfloat16>(p.uh) : reinterpret_cast<__nv_bfloat16*>(cut);
+      __nv_bfloat16* ul = c.atc<__nv_bfloat16>(p.ul);
+      __nv_bfloat16* um = f32 ? c.atc<__nv_bfloat16>(p.um) : nullptr;
+      k_store_ut<<<grid1(int64_t(T) * rT), 256, 0, c.st>>>(U, T, q, rT, f32, cut, f32 ? uh : nullptr, um, ul);
+      // the cell's X as bf16 for the tensor cores (f32 inputs: a bf16 copy in the X~ region first)
+      const void* Xb = Xk;
+      const void* Xlo = nullptr;
+      float* xt = c.atc<float>(p.xt);
+      if (io32) {
+        __nv_bfloat16* xh = c.at<__nv_bfloat16>(p.xb);
+        __nv_bfloat16* xl = xh + p.cell_elems;
+        if ((r = split_bf16(reinterpret_cast<const float*>(Xk), 1, p.cell_elems, 1, 1, 0, xh, xl, 1, 0, c.st))) return r;
+        Xb = xh;
+        Xlo = xl;
+      }
+      // Y_lh = U_T^T X_lh  [LgH][rT][d]
+      float* ylh = c.atc<float>(p.ylh);
+      JOLT_CUDA_TRY(cudaMemsetAsync(ylh, 0, size_t(LgH) * rT * d * 4, c.st));
+      {
+        // projection with the unrounded basis: (U_hi, X_hi) + (U_hi, X_lo) + (U_2nd, X_hi)
+        GemmCall g;
+        g.M = rT; g.N = d; g.K = T;
+        const Operand xh = plain(Xb, kMajorMN, d, T, d, LgH, int64_t(T) * d);
+        const Operand uhh = plain(uh, kMajorMN, rT, T, rT, LgH, 0);
+        int nt = 0;
+        g.A[nt] = uhh; g.B[nt] = xh; ++nt;
+        if (Xlo) { g.A[nt] = uhh; g.B[nt] = plain(Xlo, kMajorMN, d, T, d, LgH, int64_t(T) * d); ++nt; }
+        g.A[nt] = plain(f32 ? um : ul, kMajorMN, rT, T, rT, LgH, 0); g.B[nt] = xh; ++nt;
+        g.n_terms = nt;
+        g.C = ylh; g.ldc = d; g.c_batch_stride = int64_t(rT) * d; g.batch = LgH;
+        g.k_split = ksplit_for(int64_t((rT + 127) / 128) * LgH, T); g.accumulate = true; g.err = c.err;
+        if ((r = gemm_tc(g, c.st))) return r;
+      }
+      // S_Y, U_d
+      float* sy = c.atc<float>(p.sy);
+      JOLT_CUDA_TRY(cudaMemsetAsync(sy, 0, size_t(d) * d * 4, c.st));
+      {
+        const int nrows = LgH * rT;
+        const int gx = std::max(1, std::min(64, nrows / 256));
+        k_gram_small<<<dim3(gx, (d + 31) / 32, (d + 31) / 32), 256, 32 * 64 * 4, c.st>>>(ylh, nrows, d, sy);
+      }
+      float* evy = c.atc<float>(p.evy);
+      float* evecy = c.atc<float>(p.evecy);
+      if ((r = jacobi_eig(sy, d, 1, d, evy, evecy, c.ws + p.off_cmp + p.jac2, 30, 1e-10, c.err, c.st))) return r;
+      // U_d = first rd eigenvector columns (stored dtype), then G = Y U_d (stored dtype)
+      k_store_ut<<<grid1(int64_t(d) * rd), 256, 0, c.st>>>(evecy, d, d, rd, f32, cud, nullptr, nullptr, nullptr);
+      k_proj_small<<<grid1(int64_t(LgH) * rT * rd), 256, 0, c.st>>>(ylh, int64_t(LgH) * rT, d, evecy, d, rd, f32, cg);
+      // B_lh = G U_d^T from stored values (hi/lo), then X~ = U_T B_lh
+      // X~ = U^s B with B = G^s U_d^s^T, to fp32 accuracy: 3-way bf16 splits, terms of order <= 2
+      __nv_bfloat16* bh = c.atc<__nv_bfloat16>(p.bh);
+      __nv_bfloat16* bm = c.atc<__nv_bfloat16>(p.bm);
+      __nv_bfloat16* bl = c.atc<__nv_bfloat16>(p.bl);
+      float* blh = c.atc<float>(p.blh);
+      k_recon_b<<<grid1(int64_t(LgH) * rT * d), 256, 0, c.st>>>(cg, cud, int64_t(LgH) * rT, rd, d, f32, blh);
+      if ((r = split3_bf16(blh, int64_t(LgH) * rT * d, bh, bm, bl, c.st))) return r;
+      {
+        GemmCall g;
+        g.M = T; g.N = d; g.K = rT;
+        const Operand Bp[3] = {plain(bh, kMajorMN, d, rT, d, LgH, int64_t(rT) * d),
+                               plain(bm, kMajorMN, d, rT, d, LgH, int64_t(rT) * d),
+                               plain(bl, kMajorMN, d, rT, d, LgH, int64_t(rT) * d)};
+        const Operand Up[3] = {plain(uh, kMajorK, rT, T, rT, LgH, 0), plain(um, kMajorK, rT, T, rT, LgH, 0),
+                               plain(ul, kMajorK, rT, T, rT, LgH, 0)};
+        const int nu = f32 ? 3 : 1;
+        int nt = 0;
+        for (int i = 0; i < nu; ++i)
+          for (int j = 0; j < 3; ++j)
+            if (i + j <= 2) {
+              g.A[nt] = Up[i];
+              g.B[nt] = Bp[j];
+              ++nt;
+            }
+        g.n_terms = nt;
+        g.C = xt; g.ldc = d; g.c_batch_stride = int64_t(T) * d; g.batch = LgH; g.err = c.err;
+        if ((r = gemm_tc(g, c.st))) return r;
+      }
+      Xt = xt;
+    }
+    if (ch.b > 0) {
+      uint8_t* codes = cb + offs[5 * cell + 3];
+      __half2* sz = reinterpret_cast<__half2*>(cb + offs[5 * cell + 4]);
+      const int64_t rows = int64_t(LgH) * T;
+      const int grid = int(std::min<int64_t>((rows + 7) / 8, 148 * 16));
+      if (d == 128) {
+        if (io32) k_residual<4, float><<<grid, 256, 0, c.st>>>(reinterpret_cast<const float*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
+        else k_residual<4, __nv_bfloat16><<<grid, 256, 0, c.st>>>(reinterpret_cast<const __nv_bfloat16*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
+      } else {
+        if (io32) k_residual<2, float><<<grid, 256, 0, c.st>>>(reinterpret_cast<const float*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
+        else k_residual<2, __nv_bfloat16><<<grid, 256, 0, c.st>>>(reinterpret_cast<const __nv_bfloat16*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
+      }
+      JOLT_CUDA_TRY(cudaGetLastError());
+    }
+  }
+  return read_err(c);
+}

@@ -25,14 +25,14 @@ namespace {
 constexpr int BM = 128, BK = 64;
 
 struct TmaPack {
-  CUtensorMap a[3];
-  CUtensorMap b[3];
+  CUtensorMap a[kMaxTerms];
+  CUtensorMap b[kMaxTerms];
 };
 
 struct GemmDev {
   int M, N, K, n_terms, nkb_split, k_split;
-  int a_fold[3], b_fold[3];      // fold length (0 = plain)
-  int a_batch[3], b_batch[3];    // operand batch extents (coordinate = z % extent)
+  int a_fold[kMaxTerms], b_fold[kMaxTerms];    // fold length (0 = plain)
+  int a_batch[kMaxTerms], b_batch[kMaxTerms];  // operand batch extents (coordinate = z % extent)
   float* C;
   int64_t ldc, c_bstride;
   int c_div, accumulate;
@@ -259,7 +259,7 @@ jolt_status launch_bn(int am, int bm, const TmaPack& maps, const GemmDev& d, dim
 
 jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return JOLT_OK;
-  if (g.n_terms < 1 || g.n_terms > 3 || !g.C || g.batch < 1 || g.k_split < 1 || g.c_batch_div < 1)
+  if (g.n_terms < 1 || g.n_terms > kMaxTerms || !g.C || g.batch < 1 || g.k_split < 1 || g.c_batch_div < 1)
     return JOLT_ERR_INVALID_ARG;
   if ((g.k_split > 1 || g.c_batch_div > 1) && !g.accumulate) return JOLT_ERR_INVALID_ARG;
   const int am = g.A[0].major, bm = g.B[0].major;

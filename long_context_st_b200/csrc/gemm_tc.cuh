@@ -26,10 +26,12 @@ struct Operand {
   int64_t batch_stride = 0;   // elements between batch entries
 };
 
+constexpr int kMaxTerms = 6;
+
 struct GemmCall {
   int M = 0, N = 0, K = 0;
   int n_terms = 1;
-  Operand A[3], B[3];
+  Operand A[kMaxTerms], B[kMaxTerms];
   float* C = nullptr;
   int64_t ldc = 0;
   int64_t c_batch_stride = 0;  // elements between C batch entries

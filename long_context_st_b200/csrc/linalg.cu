@@ -1,0 +1,658 @@
+// Batched small dense linear algebra for the compressor.
+//
+// chol_inverse: right-looking blocked Cholesky (64-wide blocks, fp64) of G + shift*I, G = R^T R
+//   with R upper triangular, then the blocked triangular inverse R^{-1}. Every block step is a
+//   separate launch whose grid covers all matrices of the batch and all independent blocks, so
+//   the whole GPU works on a handful of 1152 x 1152 problems.
+// jacobi_eig: two-sided block Jacobi (32-wide blocks; each round diagonalises one cyclic sweep
+//   of 64 x 64 block pairs in shared memory, then applies the rotations to whole block rows and
+//   columns), tournament ordering, fp32, sweeps until the off-diagonal norm is below tol.
+#include <algorithm>
+#include <vector>
+
+#include "linalg.cuh"
+
+namespace jolt {
+
+namespace {
+
+constexpr int NB = 64;     // Cholesky block
+constexpr int JW = 32;     // Jacobi block width (sub-problem is 2*JW)
+constexpr int JS = 2 * JW;
+
+inline int rup(int x, int a) { return (x + a - 1) / a * a; }
+
+struct CholScratch {
+  double* Gd;    // [nb][np][np]
+  double* Xd;    // [nb][np][np]
+  double* mdiag; // [nb]
+};
+
+CholScratch chol_carve(void* scratch, int nb, int n) {
+  const int np = rup(n, NB);
+  CholScratch s;
+  uint8_t* p = static_cast<uint8_t*>(scratch);
+  s.Gd = reinterpret_cast<double*>(p);
+  p += align_up(size_t(nb) * np * np * 8, 256);
+  s.Xd = reinterpret_cast<double*>(p);
+  p += align_up(size_t(nb) * np * np * 8, 256);
+  s.mdiag = reinterpret_cast<double*>(p);
+  return s;
+}
+
+__global__ void k_maxdiag(const float* __restrict__ G, int64_t ldg, int n, double* md) {
+  const int b = blockIdx.x;
+  const float* g = G + int64_t(b) * n * ldg;
+  double m = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmax(m, double(g[int64_t(i) * ldg + i]));
+  __shared__ double red[256];
+  red[threadIdx.x] = m;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] = fmax(red[threadIdx.x], red[threadIdx.x + s]);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) md[b] = red[0];
+}
+
+__global__ void k_chol_init(const float* __restrict__ G, int64_t ldg, int n, int np, double shift_rel,
+                            const double* __restrict__ md, double* __restrict__ Gd, double* __restrict__ Xd) {
+  const int b = blockIdx.z;
+  const int i0 = blockIdx.y * NB, j0 = blockIdx.x * NB;
+  const float* g = G + int64_t(b) * n * ldg;
+  double* gd = Gd + int64_t(b) * np * np;
+  double* xd = Xd + int64_t(b) * np * np;
+  const double sh = shift_rel * md[b];
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+    const int i = i0 + e / NB, j = j0 + e % NB;
+    double v;
+    if (i < n && j < n) v = double(g[int64_t(i) * ldg + j]) + (i == j ? sh : 0.0);
+    else v = (i == j) ? 1.0 : 0.0;
+    gd[int64_t(i) * np + j] = v;
+    xd[int64_t(i) * np + j] = 0.0;
+  }
+}
+
+// 64x64 fp64 tile load/store helpers (row stride np).
+__device__ __forceinline__ void tile_load(double (*S)[NB + 1], const double* src, int np) {
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) S[e / NB][e % NB] = src[int64_t(e / NB) * np + e % NB];
+}
+__device__ __forceinline__ void tile_store(double* dst, double (*S)[NB + 1], int np) {
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) dst[int64_t(e / NB) * np + e % NB] = S[e / NB][e % NB];
+}
+
+// out = op(A)^T-style products on 64x64 tiles: C[a][b] = sum_k A[k][a] * B[k][b]
+__device__ __forceinline__ void tile_atb(double (*C)[NB + 1], double (*A)[NB + 1], double (*B)[NB + 1]) {
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;  // 16x16 threads, 4x4 outputs each
+  double acc[4][4] = {};
+  for (int k = 0; k < NB; ++k) {
+    double a[4], bb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] = A[k][ty * 4 + u];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) bb[v] = B[k][tx * 4 + v];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[u][v] += a[u] * bb[v];
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) C[ty * 4 + u][tx * 4 + v] = acc[u][v];
+}
+// C[a][b] = sum_k A[a][k] * B[k][b]
+__device__ __forceinline__ void tile_ab(double (*C)[NB + 1], double (*A)[NB + 1], double (*B)[NB + 1]) {
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[4][4] = {};
+  for (int k = 0; k < NB; ++k) {
+    double a[4], bb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] = A[ty * 4 + u][k];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) bb[v] = B[k][tx * 4 + v];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[u][v] += a[u] * bb[v];
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) C[ty * 4 + u][tx * 4 + v] = acc[u][v];
+}
+
+// Factor the diagonal block p and invert it.
+__global__ void __launch_bounds__(256) k_chol_diag(double* __restrict__ Gd, double* __restrict__ Xd, int np,
+                                                   int p, int32_t* err) {
+  extern __shared__ double sh[];
+  double(*S)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
+  double(*X)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
+  const int b = blockIdx.x;
+  double* gd = Gd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
+  double* xd = Xd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
+  tile_load(S, gd, np);
+  __syncthreads();
+  for (int j = 0; j < NB; ++j) {
+    if (threadIdx.x == 0) {
+      double d = S[j][j];
+      if (!(d > 0.0)) {
+        report_error(err, JOLT_ERR_NUMERIC);
+        d = 1.0;
+      }
+      S[j][j] = sqrt(d);
+    }
+    __syncthreads();
+    const double piv = S[j][j];
+    for (int k = j + 1 + threadIdx.x; k < NB; k += blockDim.x) S[j][k] /= piv;
+    __syncthreads();
+    const int m = NB - j - 1;
+    for (int e = threadIdx.x; e < m * m; e += blockDim.x) {
+      const int i = j + 1 + e / m, k = j + 1 + e % m;
+      if (i <= k) S[i][k] -= S[j][i] * S[j][k];
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+    const int i = e / NB, k = e % NB;
+    if (i > k) S[i][k] = 0.0;
+    X[i][k] = 0.0;
+  }
+  __syncthreads();
+  if (threadIdx.x < NB) {
+    const int c = threadIdx.x;
+    X[c][c] = 1.0 / S[c][c];
+    for (int i = c - 1; i >= 0; --i) {
+      double a = 0.0;
+      for (int k = i + 1; k <= c; ++k) a += S[i][k] * X[k][c];
+      X[i][c] = -a / S[i][i];
+    }
+  }
+  __syncthreads();
+  tile_store(gd, S, np);
+  tile_store(xd, X, np);
+}
+
+// Panel: R_pj = X_pp^T G_pj for j > p.
+__global__ void __launch_bounds__(256) k_chol_panel(double* __restrict__ Gd, const double* __restrict__ Xd,
+                                                    int np, int p) {
+  extern __shared__ double sh[];
+  double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
+  double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
+  double(*C)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 2 * NB * (NB + 1));
+  const int b = blockIdx.y, j = p + 1 + blockIdx.x;
+  const double* xpp = Xd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
+  double* gpj = Gd + int64_t(b) * np * np + int64_t(p) * NB * np + j * NB;
+  tile_load(A, xpp, np);
+  tile_load(B, gpj, np);
+  __syncthreads();
+  tile_atb(C, A, B);
+  __syncthreads();
+  tile_store(gpj, C, np);
+}
+
+// Trailing update: G_ij -= R_pi^T R_pj for p < i <= j.
+__global__ void __launch_bounds__(256) k_chol_update(double* __restrict__ Gd, int np, int P, int p) {
+  extern __shared__ double sh[];
+  double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
+  double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
+  double(*C)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 2 * NB * (NB + 1));
+  const int b = blockIdx.y;
+  int idx = blockIdx.x, i = p + 1;
+  while (idx >= P - i) {
+    idx -= P - i;
+    ++i;
+  }
+  const int j = i + idx;
+  double* g = Gd + int64_t(b) * np * np;
+  tile_load(A, g + int64_t(p) * NB * np + i * NB, np);
+  tile_load(B, g + int64_t(p) * NB * np + j * NB, np);
+  __syncthreads();
+  tile_atb(C, A, B);
+  __syncthreads();
+  double* gij = g + int64_t(i) * NB * np + j * NB;
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) gij[int64_t(e / NB) * np + e % NB] -= C[e / NB][e % NB];
+}
+
+// Inverse blocks at distance d: X_ij = -X_ii * sum_{k=i+1..j} R_ik X_kj, j = i + d.
+__global__ void __launch_bounds__(256) k_trinv(const double* __restrict__ Gd, double* __restrict__ Xd, int np,
+                                               int d) {
+  extern __shared__ double sh[];
+  double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
+  double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
+  double(*C)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 2 * NB * (NB + 1));
+  double(*Acc)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 3 * NB * (NB + 1));
+  const int b = blockIdx.y, i = blockIdx.x, j = i + d;
+  const double* g = Gd + int64_t(b) * np * np;
+  double* x = Xd + int64_t(b) * np * np;
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) Acc[e / NB][e % NB] = 0.0;
+  for (int k = i + 1; k <= j; ++k) {
+    __syncthreads();
+    tile_load(A, g + int64_t(i) * NB * np + k * NB, np);
+    tile_load(B, x + int64_t(k) * NB * np + j * NB, np);
+    __syncthreads();
+    tile_ab(C, A, B);
+    __syncthreads();
+    for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) Acc[e / NB][e % NB] += C[e / NB][e % NB];
+  }
+  __syncthreads();
+  tile_load(A, x + int64_t(i) * NB * np + i * NB, np);
+  __syncthreads();
+  tile_ab(C, A, Acc);
+  __syncthreads();
+  double* xij = x + int64_t(i) * NB * np + j * NB;
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) xij[int64_t(e / NB) * np + e % NB] = -C[e / NB][e % NB];
+}
+
+__global__ void k_rinv_out(const double* __restrict__ Xd, int np, int n, __nv_bfloat16* hi, __nv_bfloat16* lo) {
+  const int b = blockIdx.y;
+  const int64_t total = int64_t(n) * n;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    const int i = int(e / n), j = int(e % n);
+    const float v = (i <= j) ? float(Xd[int64_t(b) * np * np + int64_t(i) * np + j]) : 0.f;
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[int64_t(b) * total + e] = h;
+    lo[int64_t(b) * total + e] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// ---- block Jacobi (fp64 working precision) -----------------------------------------------------
+
+struct JacScratch {
+  double* A;     // [nb][np][np]
+  double* V;     // [nb][np][np]
+  double* Th;    // [nb][npair][JS][JS]
+  double* norms; // [nb][2] off^2, total^2
+  int* perm;     // [nb][np]
+};
+
+JacScratch jac_carve(void* scratch, int nb, int n) {
+  const int np = rup(n, JS);
+  const int npair = np / JS;
+  JacScratch s;
+  uint8_t* p = static_cast<uint8_t*>(scratch);
+  s.A = reinterpret_cast<double*>(p); p += align_up(size_t(nb) * np * np * 8, 256);
+  s.V = reinterpret_cast<double*>(p); p += align_up(size_t(nb) * np * np * 8, 256);
+  s.Th = reinterpret_cast<double*>(p); p += align_up(size_t(nb) * npair * JS * JS * 8, 256);
+  s.norms = reinterpret_cast<double*>(p); p += align_up(size_t(nb) * 16, 256);
+  s.perm = reinterpret_cast<int*>(p);
+  return s;
+}
+
+template <typename TA>
+__global__ void k_jac_init(const TA* __restrict__ A, int64_t lda, int n, int np, double* __restrict__ Aw,
+                           double* __restrict__ V) {
+  const int b = blockIdx.y;
+  const int64_t total = int64_t(np) * np;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    const int i = int(e / np), j = int(e % np);
+    double v;
+    if (i < n && j < n)
+      v = 0.5 * (double(A[int64_t(b) * n * lda + int64_t(i) * lda + j]) + double(A[int64_t(b) * n * lda + int64_t(j) * lda + i]));
+    else v = (i == j) ? -1.0 : 0.0;
+    Aw[int64_t(b) * total + e] = v;
+    V[int64_t(b) * total + e] = (i == j) ? 1.0 : 0.0;
+  }
+}
+
+// tournament (circle method) pairing of m players in round r: pair k -> (first, second)
+__host__ __device__ __forceinline__ void tour_pair(int m, int r, int k, int* a, int* b) {
+  auto pos = [&](int x) { return x == 0 ? 0 : ((x - 1 + r) % (m - 1)) + 1; };
+  *a = pos(k);
+  *b = pos(m - 1 - k);
+}
+
+typedef double Tile[JS][JS + 1];
+
+__global__ void __launch_bounds__(256) k_jac_solve(const double* __restrict__ Aw, int np, int nblk, int round,
+                                                   double* __restrict__ Th) {
+  extern __shared__ double jsm[];
+  Tile& S = *reinterpret_cast<Tile*>(jsm);
+  Tile& Q = *reinterpret_cast<Tile*>(jsm + JS * (JS + 1));
+  __shared__ double cs[JW], sn[JW];
+  __shared__ int pp[JW], qq[JW];
+  const int b = blockIdx.y, k = blockIdx.x, npair = nblk / 2;
+  int I, J;
+  tour_pair(nblk, round, k, &I, &J);
+  const double* a = Aw + int64_t(b) * np * np;
+  for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) {
+    const int u = e / JS, v = e % JS;
+    const int gu = (u < JW ? I * JW + u : J * JW + u - JW);
+    const int gv = (v < JW ? I * JW + v : J * JW + v - JW);
+    S[u][v] = a[int64_t(gu) * np + gv];
+    Q[u][v] = (u == v) ? 1.0 : 0.0;
+  }
+  __syncthreads();
+  for (int r = 0; r < JS - 1; ++r) {
+    if (threadIdx.x < JW) {
+      int p, q;
+      tour_pair(JS, r, threadIdx.x, &p, &q);
+      if (p > q) { const int t = p; p = q; q = t; }
+      const double apq = S[p][q], app = S[p][p], aqq = S[q][q];
+      double c = 1.0, s = 0.0;
+      if (apq != 0.0 && fabs(apq) > 1e-300) {
+        const double theta = (aqq - app) / (2.0 * apq);
+        const double t = (theta >= 0.0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
+        c = 1.0 / sqrt(t * t + 1.0);
+        s = t * c;
+      }
+      cs[threadIdx.x] = c; sn[threadIdx.x] = s; pp[threadIdx.x] = p; qq[threadIdx.x] = q;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < JW * JS; e += blockDim.x) {  // rows p, q
+      const int kk = e / JS, m = e % JS;
+      const int p = pp[kk], q = qq[kk];
+      const double c = cs[kk], s = sn[kk];
+      const double xp = S[p][m], xq = S[q][m];
+      S[p][m] = c * xp - s * xq;
+      S[q][m] = s * xp + c * xq;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < JW * JS; e += blockDim.x) {  // columns p, q of S and Q
+      const int kk = e / JS, m = e % JS;
+      const int p = pp[kk], q = qq[kk];
+      const double c = cs[kk], s = sn[kk];
+      const double xp = S[m][p], xq = S[m][q];
+      S[m][p] = c * xp - s * xq;
+      S[m][q] = s * xp + c * xq;
+      const double yp = Q[m][p], yq = Q[m][q];
+      Q[m][p] = c * yp - s * yq;
+      Q[m][q] = s * yp + c * yq;
+    }
+    __syncthreads();
+  }
+  double* th = Th + (int64_t(b) * npair + k) * JS * JS;
+  for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) th[e] = Q[e / JS][e % JS];
+}
+
+// columns I u J of A and V (chunk of 64 rows per CTA): X[:, IJ] <- X[:, IJ] * Theta
+__global__ void __launch_bounds__(256) k_jac_cols(double* __restrict__ Aw, double* __restrict__ V, int np,
+                                                  int nblk, int round, const double* __restrict__ Th) {
+  extern __shared__ double jsm[];
+  Tile& T = *reinterpret_cast<Tile*>(jsm);
+  Tile& X = *reinterpret_cast<Tile*>(jsm + JS * (JS + 1));
+  const int b = blockIdx.z, k = blockIdx.x, r0 = blockIdx.y * JS, npair = nblk / 2;
+  int I, J;
+  tour_pair(nblk, round, k, &I, &J);
+  const double* th = Th + (int64_t(b) * npair + k) * JS * JS;
+  for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) T[e / JS][e % JS] = th[e];
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  for (int which = 0; which < 2; ++which) {
+    double* M = (which ? V : Aw) + int64_t(b) * np * np;
+    __syncthreads();
+    for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) {
+      const int u = e / JS, v = e % JS;
+      const int gv = (v < JW ? I * JW + v : J * JW + v - JW);
+      X[u][v] = M[int64_t(r0 + u) * np + gv];
+    }
+    __syncthreads();
+    double acc[4][4] = {};
+    for (int kk = 0; kk < JS; ++kk) {
+      double a[4], bb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) a[u] = X[ty * 4 + u][kk];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) bb[v] = T[kk][tx * 4 + v];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] += a[u] * bb[v];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int col = tx * 4 + v;
+        const int gv = (col < JW ? I * JW + col : J * JW + col - JW);
+        M[int64_t(r0 + ty * 4 + u) * np + gv] = acc[u][v];
+      }
+  }
+}
+
+// rows I u J of A (chunk of 64 columns per CTA): A[IJ, :] <- Theta^T A[IJ, :]
+__global__ void __launch_bounds__(256) k_jac_rows(double* __restrict__ Aw, int np, int nblk, int round,
+                                                  const double* __restrict__ Th) {
+  extern __shared__ double jsm[];
+  Tile& T = *reinterpret_cast<Tile*>(jsm);
+  Tile& X = *reinterpret_cast<Tile*>(jsm + JS * (JS + 1));
+  const int b = blockIdx.z, k = blockIdx.x, c0 = blockIdx.y * JS, npair = nblk / 2;
+  int I, J;
+  tour_pair(nblk, round, k, &I, &J);
+  const double* th = Th + (int64_t(b) * npair + k) * JS * JS;
+  double* M = Aw + int64_t(b) * np * np;
+  for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) {
+    const int u = e / JS, v = e % JS;
+    T[u][v] = th[e];
+    const int gu = (u < JW ? I * JW + u : J * JW + u - JW);
+    X[u][v] = M[int64_t(gu) * np + c0 + v];
+  }
+  __syncthreads();
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[4][4] = {};
+  for (int kk = 0; kk < JS; ++kk) {
+    double a[4], bb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] = T[kk][ty * 4 + u];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) bb[v] = X[kk][tx * 4 + v];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[u][v] += a[u] * bb[v];
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int row = ty * 4 + u;
+    const int gu = (row < JW ? I * JW + row : J * JW + row - JW);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) M[int64_t(gu) * np + c0 + tx * 4 + v] = acc[u][v];
+  }
+}
+
+__global__ void k_jac_norms(const double* __restrict__ Aw, int np, double* norms) {
+  const int b = blockIdx.y;
+  const int64_t total = int64_t(np) * np;
+  double off = 0.0, tot = 0.0;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    const double v = Aw[int64_t(b) * total + e];
+    tot += v * v;
+    if (e / np != e % np) off += v * v;
+  }
+  for (int m = 16; m; m >>= 1) {
+    off += __shfl_xor_sync(0xffffffffu, off, m);
+    tot += __shfl_xor_sync(0xffffffffu, tot, m);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(&norms[2 * b], off);
+    atomicAdd(&norms[2 * b + 1], tot);
+  }
+}
+
+template <typename TO>
+__global__ void k_jac_sort(const double* __restrict__ Aw, int np, int n, TO* evals, int* perm) {
+  const int b = blockIdx.y;
+  const double* a = Aw + int64_t(b) * np * np;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const double di = a[int64_t(i) * np + i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const double dj = a[int64_t(j) * np + j];
+      rank += (dj > di) || (dj == di && j < i);
+    }
+    evals[int64_t(b) * n + rank] = TO(di);
+    perm[int64_t(b) * np + rank] = i;
+  }
+}
+
+template <typename TO>
+__global__ void k_jac_out(const double* __restrict__ V, int np, int n, const int* __restrict__ perm, TO* evecs) {
+  const int b = blockIdx.y;
+  const int64_t total = int64_t(n) * n;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    const int row = int(e / n), col = int(e % n);
+    evecs[int64_t(b) * total + e] = TO(V[int64_t(b) * np * np + int64_t(row) * np + perm[int64_t(b) * np + col]]);
+  }
+}
+
+__global__ void k_split(const float* __restrict__ x, int64_t ldx, int64_t rows, int64_t cols, int64_t bsx,
+                        __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo, int64_t ldo, int64_t bso) {
+  const int b = blockIdx.y;
+  const int64_t total = rows * cols;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = e / cols, c = e % cols;
+    const float v = x[b * bsx + r * ldx + c];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[b * bso + r * ldo + c] = h;
+    if (lo) lo[b * bso + r * ldo + c] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+__global__ void k_split3(const float* __restrict__ x, int64_t n, __nv_bfloat16* __restrict__ hi,
+                         __nv_bfloat16* __restrict__ mid, __nv_bfloat16* __restrict__ lo) {
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
+    const float v = x[e];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(m);
+    hi[e] = h;
+    mid[e] = m;
+    lo[e] = __float2bfloat16_rn(r2);
+  }
+}
+
+int grid_1d(int64_t n, int per = 256) {
+  int64_t g = (n + per - 1) / per;
+  return int(std::max<int64_t>(1, std::min<int64_t>(g, 148 * 8)));
+}
+
+}  // namespace
+
+size_t chol_scratch_bytes(int nb, int n) {
+  const int np = rup(n, NB);
+  return 2 * align_up(size_t(nb) * np * np * 8, 256) + align_up(size_t(nb) * 8, 256);
+}
+
+jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shift_rel,
+                         __nv_bfloat16* rinv_hi, __nv_bfloat16* rinv_lo, void* scratch, int32_t* err,
+                         cudaStream_t st) {
+  if (nb < 1 || n < 1) return JOLT_OK;
+  const int np = rup(n, NB), P = np / NB;
+  CholScratch s = chol_carve(scratch, nb, n);
+  k_maxdiag<<<nb, 256, 0, st>>>(G, ld_g, n, s.mdiag);
+  k_chol_init<<<dim3(P, P, nb), 256, 0, st>>>(G, ld_g, n, np, shift_rel, s.mdiag, s.Gd, s.Xd);
+  const int sm2 = 2 * NB * (NB + 1) * 8, sm3 = 3 * NB * (NB + 1) * 8, sm4 = 4 * NB * (NB + 1) * 8;
+  static bool attr = false;
+  if (!attr) {
+    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_chol_diag, cudaFuncAttributeMaxDynamicSharedMemorySize, sm2));
+    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_chol_panel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm3));
+    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_chol_update, cudaFuncAttributeMaxDynamicSharedMemorySize, sm3));
+    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_trinv, cudaFuncAttributeMaxDynamicSharedMemorySize, sm4));
+    attr = true;
+  }
+  for (int p = 0; p < P; ++p) {
+    k_chol_diag<<<nb, 256, sm2, st>>>(s.Gd, s.Xd, np, p, err);
+    if (p + 1 < P) {
+      k_chol_panel<<<dim3(P - p - 1, nb), 256, sm3, st>>>(s.Gd, s.Xd, np, p);
+      const int npairs = (P - p - 1) * (P - p) / 2;
+      k_chol_update<<<dim3(npairs, nb), 256, sm3, st>>>(s.Gd, np, P, p);
+    }
+  }
+  for (int d = 1; d < P; ++d) k_trinv<<<dim3(P - d, nb), 256, sm4, st>>>(s.Gd, s.Xd, np, d);
+  k_rinv_out<<<dim3(grid_1d(int64_t(n) * n), nb), 256, 0, st>>>(s.Xd, np, n, rinv_hi, rinv_lo);
+  JOLT_CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
+size_t jacobi_scratch_bytes(int nb, int n) {
+  const int np = rup(n, JS), npair = np / JS;
+  return 2 * align_up(size_t(nb) * np * np * 8, 256) + align_up(size_t(nb) * npair * JS * JS * 8, 256) +
+         align_up(size_t(nb) * 16, 256) + align_up(size_t(nb) * np * 4, 256);
+}
+
+template <typename TA, typename TO>
+jolt_status jacobi_impl(const TA* A, int64_t ld_a, int nb, int n, TO* evals, TO* evecs, void* scratch,
+                        int max_sweeps, double tol, int32_t* err, cudaStream_t st) {
+  if (nb < 1 || n < 1) return JOLT_OK;
+  const int np = rup(n, JS), nblk = np / JW, npair = nblk / 2, chunks = np / JS;
+  JacScratch s = jac_carve(scratch, nb, n);
+  const int tsm = 2 * JS * (JS + 1) * 8;
+  static bool attr = false;
+  if (!attr) {
+    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_jac_solve, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm));
+    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_jac_cols, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm));
+    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_jac_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm));
+    attr = true;
+  }
+  k_jac_init<<<dim3(grid_1d(int64_t(np) * np), nb), 256, 0, st>>>(A, ld_a, n, np, s.A, s.V);
+  std::vector<double> h(2 * nb);
+  for (int sweep = 0; sweep < max_sweeps; ++sweep) {
+    for (int r = 0; r < nblk - 1; ++r) {
+      k_jac_solve<<<dim3(npair, nb), 256, tsm, st>>>(s.A, np, nblk, r, s.Th);
+      k_jac_cols<<<dim3(npair, chunks, nb), 256, tsm, st>>>(s.A, s.V, np, nblk, r, s.Th);
+      k_jac_rows<<<dim3(npair, chunks, nb), 256, tsm, st>>>(s.A, np, nblk, r, s.Th);
+    }
+    JOLT_CUDA_TRY(cudaMemsetAsync(s.norms, 0, sizeof(double) * 2 * nb, st));
+    k_jac_norms<<<dim3(grid_1d(int64_t(np) * np), nb), 256, 0, st>>>(s.A, np, s.norms);
+    JOLT_CUDA_TRY(cudaMemcpyAsync(h.data(), s.norms, sizeof(double) * 2 * nb, cudaMemcpyDeviceToHost, st));
+    JOLT_CUDA_TRY(cudaStreamSynchronize(st));
+    bool done = true;
+    for (int b = 0; b < nb; ++b)
+      if (h[2 * b] > tol * tol * h[2 * b + 1]) done = false;
+    if (done) break;
+  }
+  k_jac_sort<<<dim3((n + 255) / 256, nb), 256, 0, st>>>(s.A, np, n, evals, s.perm);
+  k_jac_out<<<dim3(grid_1d(int64_t(n) * n), nb), 256, 0, st>>>(s.V, np, n, s.perm, evecs);
+  JOLT_CUDA_TRY(cudaGetLastError());
+  (void)err;
+  return JOLT_OK;
+}
+
+jolt_status jacobi_eig(const float* A, int64_t ld_a, int nb, int n, float* evals, float* evecs, void* scratch,
+                       int max_sweeps, double tol, int32_t* err, cudaStream_t st) {
+  return jacobi_impl<float, float>(A, ld_a, nb, n, evals, evecs, scratch, max_sweeps, tol, err, st);
+}
+
+jolt_status jacobi_eig64(const double* A, int64_t ld_a, int nb, int n, double* evals, double* evecs, void* scratch,
+                         int max_sweeps, double tol, int32_t* err, cudaStream_t st) {
+  return jacobi_impl<double, double>(A, ld_a, nb, n, evals, evecs, scratch, max_sweeps, tol, err, st);
+}
+
+jolt_status split3_bf16(const float* x, int64_t n, __nv_bfloat16* hi, __nv_bfloat16* mid, __nv_bfloat16* lo,
+                        cudaStream_t st) {
+  if (n <= 0) return JOLT_OK;
+  k_split3<<<grid_1d(n), 256, 0, st>>>(x, n, hi, mid, lo);
+  JOLT_CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
+jolt_status split_bf16(const float* x, int64_t ldx, int64_t rows, int64_t cols, int batch, int64_t bstride_x,
+                       __nv_bfloat16* hi, __nv_bfloat16* lo, int64_t ldo, int64_t bstride_o, cudaStream_t st) {
+  if (rows <= 0 || cols <= 0) return JOLT_OK;
+  k_split<<<dim3(grid_1d(rows * cols), batch), 256, 0, st>>>(x, ldx, rows, cols, bstride_x, hi, lo, ldo, bstride_o);
+  JOLT_CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
+}  // namespace jolt
+
+using namespace jolt;
+
+extern "C" size_t jolt_sym_eig_workspace(int32_t n, int32_t batch) {
+  if (n < 1 || batch < 1) return 0;
+  return sizeof(WsHeader) + jacobi_scratch_bytes(batch, n);
+}
+
+extern "C" jolt_status jolt_sym_eig(const float* A, int32_t n, int32_t batch, float* evals, float* evecs,
+                                    void* ws, size_t ws_bytes, void* stream) {
+  if (n < 1 || batch < 1) return JOLT_ERR_INVALID_ARG;
+  if (!A || !evals || !evecs || !ws) return JOLT_ERR_INVALID_ARG;
+  if (ws_bytes < jolt_sym_eig_workspace(n, batch)) return JOLT_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  JOLT_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(WsHeader), st));
+  jolt_status r = jacobi_eig(A, n, batch, n, evals, evecs, static_cast<uint8_t*>(ws) + sizeof(WsHeader), 30,
+                             1e-10, static_cast<int32_t*>(ws), st);
+  if (r) return r;
+  JOLT_CUDA_TRY(cudaStreamSynchronize(st));
+  return JOLT_OK;
+}

@@ -31,7 +31,7 @@ class Workload:
     seed: int = 0
     q_cap: int = 1024          # token-rank cap of the randomized token-mode SVD
     oversample: int = 128      # extra sketch columns beyond q_cap
-    power_iters: int = 2
+    power_iters: int = 3
     noise: float = 0.05
     outlier_scale: float = 10.0
     tags: dict = field(default_factory=dict, compare=False, hash=False)

@@ -98,3 +98,33 @@ def max_rel_err(out, ref):
     num = np.abs(out - ref).max(axis=-1)
     den = np.abs(ref).max(axis=-1)
     return float(np.max(num / den))
+
+
+def device_to_cells(shape, w, cache, choices, factor_dtype=None):
+    """Read a device cache (jolt layout) back into oracle cell dicts (stored values as float64)."""
+    fdt = _FDT[factor_dtype or w.factor_dtype]
+    esz = 4 if fdt == torch.float32 else 2
+    offs, total = api.cache_layout(shape, choices)
+    buf = cache.cpu()
+    Lg, H, T, d = w.layers_per_group, w.n_kv, shape.T, w.d_h
+    cells = []
+
+    def get(off, count, dtype):
+        raw = buf[int(off):int(off) + count * (torch.finfo(dtype).bits // 8 if dtype.is_floating_point else 1)]
+        return raw.view(dtype)
+
+    for c, (rT, rd, b) in enumerate(choices):
+        cell = {"r_T": rT, "r_d": rd, "b": b, "shape": (Lg, H, T, d)}
+        if rT:
+            cell["U_T"] = get(offs[c, 0], T * rT, fdt).double().numpy().reshape(T, rT)
+            cell["U_d"] = get(offs[c, 1], d * rd, fdt).double().numpy().reshape(d, rd)
+            cell["G"] = get(offs[c, 2], Lg * H * rT * rd, fdt).double().numpy().reshape(Lg, H, rT, rd)
+        else:
+            cell["U_T"] = np.zeros((T, 0)); cell["U_d"] = np.zeros((d, 0)); cell["G"] = np.zeros((Lg, H, 0, 0))
+        if b:
+            cell["codes"] = buf[int(offs[c, 3]):int(offs[c, 3]) + Lg * H * T * d * b // 8].numpy().reshape(Lg, H, T, d * b // 8)
+            sz = get(offs[c, 4], Lg * H * T * 2, torch.float16).numpy().reshape(Lg, H, T, 2)
+            cell["scale"] = sz[..., 0].copy()
+            cell["zero"] = sz[..., 1].copy()
+        cells.append(cell)
+    return cells

@@ -1,0 +1,169 @@
+"""GPU compressor (jolt_analyze + jolt_compress) vs the oracle.
+
+* spectra tails vs the oracle's exact tails;
+* stored U_T and U_d orthonormal to 1e-4 (fp32 factor storage);
+* relative reconstruction error of the GPU cache (decoded by the oracle) within 1% of the
+  oracle's own compression at the same (r_T, r_d, b);
+* allocation on GPU tables; error paths.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.alloc import tables_to_options, allocate as oracle_allocate
+from oracle.bytes_model import raw_sequence_bytes
+from synth import get_workload, make_kv
+from cache_io import oracle_cells, device_to_cells, cell_index
+from long_context_st_b200 import api
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_compress(w, K, V, choices, **over):
+    shape = api.make_shape(w, **over)
+    ws = api.new_workspace(shape, api.JOLT_OP_COMPRESS)
+    n2, tT, td = api.analyze(shape, K, V, ws)
+    _, total = api.cache_layout(shape, choices)
+    cache = torch.zeros(total, dtype=torch.uint8, device="cuda")
+    api.compress(shape, K, V, choices, cache, ws)
+    torch.cuda.synchronize()
+    return shape, (n2, tT, td), cache
+
+
+def cell_tensors(w, K, V):
+    G = w.n_layers // w.layers_per_group
+    out = []
+    for b in range(K.shape[0]):
+        for g in range(G):
+            sl = slice(g * w.layers_per_group, (g + 1) * w.layers_per_group)
+            for X in (K, V):
+                out.append(X[b, sl].double().cpu().numpy())
+    return out
+
+
+# Reading of "relative reconstruction error within 1% of the oracle's": |e_gpu - e_oracle| <=
+# 1% of e_oracle, where e is the squared relative Frobenius error, or both below the fp32 resolution
+# floor (squared relative error 1e-12, i.e. relative error 1e-6): the oracle's float64 result can
+# sit below what any fp32 reconstruction resolves (e.g. full ranks with 8-bit residuals).
+FP32_FLOOR = 1e-12
+
+
+def within(eg, eo, nx, tol):
+    return abs(eg - eo) <= tol * eo + FP32_FLOOR * nx
+
+
+def recon_errors(w, Xs, gcells, ocells, rot_seed):
+    res = []
+    for X, gc, oc in zip(Xs, gcells, ocells):
+        eg = np.sum((oracle.decompress_cell(gc, rot_seed) - X) ** 2)
+        eo = np.sum((oracle.decompress_cell(oc, rot_seed) - X) ** 2)
+        res.append((eg, eo, np.sum(X ** 2)))
+    return res
+
+
+def check_tails(w, shape, K, V, tables, rtol_norm):
+    n2, tT, td = tables
+    for i, X in enumerate(cell_tensors(w, K, V)):
+        on2, otT, otd = oracle.spectra_tails(X, shape.q_cap)
+        assert n2[i] == pytest.approx(on2, rel=1e-6)
+        assert np.max(np.abs(tT[i] - otT)) <= rtol_norm * on2
+        assert np.max(np.abs(td[i] - otd)) <= 1e-5 * on2
+
+
+def check_orthonormal(cells, tol=1e-4):
+    for c in cells:
+        if c["r_T"]:
+            U, Ud = c["U_T"], c["U_d"]
+            assert np.max(np.abs(U.T @ U - np.eye(U.shape[1]))) <= tol
+            assert np.max(np.abs(Ud.T @ Ud - np.eye(Ud.shape[1]))) <= tol
+
+
+def run(w, choices, factor_dtype=None, tail_tol=1e-4, err_tol=0.01, **over):
+    K, V = make_kv(w, device="cuda")
+    fdt = factor_dtype or w.factor_dtype
+    shape, tables, cache = gpu_compress(w, K, V, choices, factor_dtype=fdt, **over)
+    check_tails(w, shape, K, V, tables, tail_tol)
+    gcells = device_to_cells(shape, w, cache, choices, factor_dtype=fdt)
+    ocells = oracle_cells(w, K, V, choices, shape.rot_seed, factor_dtype=fdt)
+    if fdt == "f32":
+        check_orthonormal(gcells)
+    for eg, eo, nx in recon_errors(w, cell_tensors(w, K, V), gcells, ocells, shape.rot_seed):
+        assert within(eg, eo, nx, err_tol), (eg / nx, eo / nx)
+    return shape, tables, gcells
+
+
+def uniform(w, ch):
+    return [ch] * (2 * w.batch * (w.n_layers // w.layers_per_group))
+
+
+def test_toy_fixed(cuda_ok):
+    w = get_workload("toy")
+    run(w, uniform(w, w.fixed_choice))
+
+
+@pytest.mark.parametrize("ch", [(0, 0, 4), (32, 32, 0), (64, 48, 2), (128, 64, 8)])
+def test_toy_choices(cuda_ok, ch):
+    w = get_workload("toy")
+    run(w, uniform(w, ch))
+
+
+def test_toy_ragged_T(cuda_ok):
+    w = get_workload("toy", T=333)
+    run(w, uniform(w, (48, 32, 4)))
+
+
+def test_llama8b_layer_fixed(cuda_ok):
+    w = get_workload("llama8b_layer")
+    run(w, uniform(w, w.fixed_choice))
+
+
+def test_llama8b_layer_fp32_factors_orthonormal(cuda_ok):
+    w = get_workload("llama8b_layer", T=2048)
+    run(w, uniform(w, (512, 96, 4)), factor_dtype="f32")
+
+
+def test_grouped_randomized_allocated(cuda_ok):
+    # one 4-layer group (n = 4096 > l = 1152): the randomized token SVD path, allocator at 3x
+    w = get_workload("llama8b_32k", n_layers=4, T=4096)
+    K, V = make_kv(w, device="cuda")
+    shape = api.make_shape(w)
+    ws = api.new_workspace(shape, api.JOLT_OP_COMPRESS)
+    n2, tT, td = api.analyze(shape, K, V, ws)
+    check_tails(w, shape, K, V, (n2, tT, td), 2e-3)
+    # oracle's exact tables -> oracle allocation; the GPU compresses with those choices
+    phi = oracle.phi_table(w.d_h)
+    tabs = [oracle.spectra_tails(X, shape.q_cap) for X in cell_tensors(w, K, V)]
+    opts = tables_to_options(np.array([t[0] for t in tabs]), np.array([t[1] for t in tabs]),
+                             np.array([t[2] for t in tabs]), phi, w)
+    choices, lam, tot = oracle_allocate(opts, raw_sequence_bytes(w) // 3)
+    _, total = api.cache_layout(shape, choices)
+    cache = torch.zeros(total, dtype=torch.uint8, device="cuda")
+    api.compress(shape, K, V, choices, cache, ws)
+    gcells = device_to_cells(shape, w, cache, choices)
+    ocells = oracle_cells(w, K, V, choices, shape.rot_seed)
+    for eg, eo, nx in recon_errors(w, cell_tensors(w, K, V), gcells, ocells, shape.rot_seed):
+        assert within(eg, eo, nx, 0.01), (eg / nx, eo / nx, choices)
+
+
+def test_compress_without_analyze_is_state_error(cuda_ok):
+    w = get_workload("toy")
+    K, V = make_kv(w, device="cuda")
+    shape = api.make_shape(w)
+    ws = api.new_workspace(shape, api.JOLT_OP_COMPRESS)
+    choices = uniform(w, w.fixed_choice)
+    _, total = api.cache_layout(shape, choices)
+    cache = torch.zeros(total, dtype=torch.uint8, device="cuda")
+    with pytest.raises(api.JoltError) as e:
+        api.compress(shape, K, V, choices, cache, ws)
+    assert e.value.status == -7
+
+
+def test_workspace_too_small(cuda_ok):
+    w = get_workload("toy")
+    K, V = make_kv(w, device="cuda")
+    shape = api.make_shape(w)
+    ws = torch.zeros(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(api.JoltError) as e:
+        api.analyze(shape, K, V, ws)
+    assert e.value.status == -6
