@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Benchmark of the JoLT codec's hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input resident in HBM:
+  jolt_analyze (spectra of every cell) -> jolt_allocate (host, one multiplier per sequence at the
+  workload's byte budget) -> jolt_compress (factors + packed residuals) -> jolt_decode_attn (one
+  query token per (sequence, layer, query head) over every cached token of every layer).
+Throughput unit: context tokens (B*T per rank) through the step per second. The JSON line also
+breaks the step down (compress raw GB/s; decode context tokens/s and HBM GB/s) and carries the
+live roofline of the dominant kernel family and of the decode kernel.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl jolt|reference]
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import get_workload, make_kv, make_queries, make_inv_freq  # noqa: E402
+
+METRIC = ("decode-attn context tokens/s & HBM GB/s over compressed cache; compress raw GB/s")
+DEFAULT_WORKLOAD = "llama70b_128k"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--ratio", type=float, default=None)
+    ap.add_argument("--impl", default="jolt", choices=["jolt", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=4096)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling (200 ms) of SM clock and throttle reasons during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                self.rows.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ---------------------------------------------------------------------------------------------
+# oracle (CPU) leg: bounded sample of the same workload
+# ---------------------------------------------------------------------------------------------
+
+def oracle_sample(w, choices_by_cell, T_s, K=None, V=None):
+    """Time the CPU oracle on one layer group (its K and V cells) over the first T_s tokens:
+    exact ST-HOSVD compression with the given choices, then decode attention for the group's
+    layers. Returns (seconds, description)."""
+    import oracle
+    from oracle.codec import compress_cell, decompress_cell, decode_attention, rope
+    Lg, d = w.layers_per_group, w.d_h
+    T_s = min(T_s, w.T)
+    ws = get_workload(w.name, T=T_s, n_layers=Lg, batch=1)
+    if K is None:
+        Kc, Vc = make_kv(ws, device="cpu", dtype=torch.float32)
+    else:
+        Kc = K[:1, :Lg, :, :T_s].float().cpu()
+        Vc = V[:1, :Lg, :, :T_s].float().cpu()
+    q = make_queries(ws, device="cpu", dtype=torch.float32).double().numpy()
+    inv = make_inv_freq(d, w.rope_theta)
+    t0 = time.perf_counter()
+    cells = []
+    for kv, X in ((0, Kc), (1, Vc)):
+        rT, rd, b = choices_by_cell[kv]
+        rT = min(rT, (min(T_s, Lg * w.n_kv * d) // 16) * 16)
+        rd = rd if rT else 0
+        cells.append(compress_cell(X[0].double().numpy(), rT, rd, b, 1234, w.factor_dtype))
+    for ll in range(Lg):
+        Kh = decompress_cell(cells[0], 1234)[ll]
+        Vh = decompress_cell(cells[1], 1234)[ll]
+        if w.keys_pre_rope:
+            Kh = rope(Kh, np.arange(T_s), inv)
+        decode_attention(Kh, Vh, q[0, ll], 1.0 / math.sqrt(d))
+    dt = time.perf_counter() - t0
+    desc = (f"oracle (float64 NumPy) on one {Lg}-layer group (its K and V cells) of the first {T_s} "
+            f"tokens: exact ST-HOSVD compress + decode of {Lg} layers; full-step time extrapolated "
+            f"linearly in T and in the {w.n_groups} groups x {w.batch} sequences")
+    return dt, desc
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [os.cpu_count()])
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, w, rank, world):
+    """--impl reference: the CPU oracle, as it stands, on bounded samples of the workload."""
+    if rank != 0:
+        return
+    choices = {0: (256, 128, 4), 1: (256, 128, 4)} if not w.fixed_choice else {0: w.fixed_choice, 1: w.fixed_choice}
+    T_s = min(args.cpu_tokens, w.T)
+    for _ in range(args.warmup):
+        oracle_sample(w, choices, T_s)
+    times = []
+    for _ in range(args.steps):
+        dt, desc = oracle_sample(w, choices, T_s)
+        times.append(dt)
+    t_sample = float(np.mean(times))
+    t_full = t_sample * w.n_groups * w.batch * (w.T / T_s)
+    value = w.batch * w.T / t_full
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "context tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_full * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "T": w.T, "n_layers": w.n_layers,
+                       "budget": "fixed sample ranks (256, 128, 4)" if not w.fixed_choice else "fixed"},
+            "cpu_baseline": {"value": value, "unit": "context tokens/s", "cores": cpu_threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "context tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+# GPU leg
+# ---------------------------------------------------------------------------------------------
+
+class Step:
+    def __init__(self, w, ratio, device, seed_shift=0):
+        from long_context_st_b200 import api
+        self.api = api
+        self.w = w
+        self.shape = api.make_shape(w)
+        self.dev = device
+        self.K, self.V = make_kv(w, device=device)
+        self.q = make_queries(w, device=device)
+        self.inv = torch.from_numpy(make_inv_freq(w.d_h, w.rope_theta)).to(device)
+        self.cws = api.new_workspace(self.shape, api.JOLT_OP_COMPRESS, device)
+        self.dws = api.new_workspace(self.shape, api.JOLT_OP_DECODE, device)
+        self.out = torch.empty_like(self.q)
+        self.phi = api.phi(w.d_h)
+        self.ratio = ratio
+        self.cache = None
+        self.choices = None
+        raw = 2 * w.n_layers * w.n_kv * w.d_h * w.T * w.io_bytes
+        self.budget = int(raw / ratio) if ratio else None
+
+    def allocate(self, tables):
+        w, api = self.w, self.api
+        n2, tT, td = tables
+        if w.fixed_choice:
+            return [tuple(w.fixed_choice)] * len(n2)
+        G = w.n_layers // w.layers_per_group
+        out = []
+        for b in range(w.batch):
+            sl = slice(b * 2 * G, (b + 1) * 2 * G)
+            ch, lam, tot = api.allocate(self.shape, n2[sl], tT[sl], td[sl], self.phi, self.budget)
+            out.extend(ch)
+        return out
+
+    def run(self, events=None, K=None, V=None):
+        api = self.api
+        K = self.K if K is None else K
+        V = self.V if V is None else V
+        ev = events or {}
+        if "start" in ev:
+            ev["start"].record()
+        tables = api.analyze(self.shape, K, V, self.cws)
+        if "analyzed" in ev:
+            ev["analyzed"].record()
+        choices = self.allocate(tables)
+        if self.cache is None or choices != self.choices:
+            _, total = api.cache_layout(self.shape, choices)
+            if self.cache is None or self.cache.numel() < total:
+                self.cache = torch.empty(total, dtype=torch.uint8, device=self.dev)
+            self.choices = choices
+            self.choices_c = api.choices_array(choices)
+        if "allocated" in ev:
+            ev["allocated"].record()
+        api.compress(self.shape, K, V, choices, self.cache, self.cws)
+        if "compressed" in ev:
+            ev["compressed"].record()
+        api.decode_attn(self.shape, choices, self.cache, self.q, self.out, self.dws, inv_freq=self.inv,
+                        choices_c=self.choices_c)
+        if "decoded" in ev:
+            ev["decoded"].record()
+        return choices
+
+
+def decode_bytes(w, shape, choices):
+    """Algorithmic bytes one full decode step reads and writes (per-layer schedule)."""
+    sf, io = w.factor_bytes, w.io_bytes
+    G = w.n_layers // w.layers_per_group
+    tot = 0
+    for b in range(w.batch):
+        for l in range(w.n_layers):
+            g = l // w.layers_per_group
+            for kv in range(2):
+                rT, rd, bb = choices[(b * G + g) * 2 + kv]
+                tot += sf * (w.T * rT + w.d_h * rd + w.n_kv * rT * rd)
+                if bb:
+                    tot += w.n_kv * w.T * (w.d_h * bb // 8 + 4)
+            tot += 2 * w.n_q * w.d_h * io
+    return tot
+
+
+def count_kernels(step):
+    """Kernels of this library launched by one step (CUPTI trace of one untimed step)."""
+    try:
+        from torch.profiler import profile, ProfilerActivity
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step.run()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+        ours = [n for n in names if "jolt" in n or n.startswith("k_") or "k_gemm" in n]
+        return len(ours), sorted(set(ours))
+    except Exception as ex:  # profiler unavailable: no claim
+        return None, [f"profiler unavailable: {ex}"]
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = get_workload(args.workload)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() and args.impl == "jolt" else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    # weak scaling: every rank compresses and decodes its own sequences (own seed)
+    w = get_workload(args.workload, seed=w.seed + 1000 * rank) if rank else w
+    ratio = args.ratio if args.ratio else (w.budget_ratios[0] if w.budget_ratios else None)
+    hbm_peak, tc_burst, tc_sust, peak_src = load_peaks()
+    from long_context_st_b200 import api
+
+    step = Step(w, ratio, dev)
+    torch.cuda.synchronize()
+    for _ in range(max(3, args.warmup)):
+        step.run()
+    torch.cuda.synchronize()
+    n_kernels, kernel_names = count_kernels(step)
+
+    names = ["start", "analyzed", "allocated", "compressed", "decoded"]
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    api.stats_read(reset=True)
+    api.stats_enable(True)
+    with Clocks(local) as clk:
+        t_start.record()
+        for i in range(args.steps):
+            step.run(evs[i])
+        t_end.record()
+        torch.cuda.synchronize()
+    api.stats_enable(False)
+    stats = api.stats_read(reset=True)
+    total_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    ms_step = total_ms / args.steps
+    ph = {k: float(np.mean([e["start"].elapsed_time(e[k]) if k != "start" else 0.0 for e in evs]))
+          for k in names}
+    t_an = ph["analyzed"]
+    t_alloc = ph["allocated"] - ph["analyzed"]
+    t_cmp = ph["compressed"] - ph["allocated"]
+    t_dec = ph["decoded"] - ph["compressed"]
+
+    tokens = w.batch * w.T
+    value = tokens * world / (ms_step / 1e3)
+    raw = 2 * w.batch * w.n_layers * w.n_kv * w.T * w.d_h * w.io_bytes
+    dbytes = decode_bytes(w, step.shape, step.choices)
+    _, cache_total = api.cache_layout(step.shape, step.choices)
+
+    def fam_roof(name, bound, peak):
+        s = stats[name]
+        if not s["launches"] or s["ms"] <= 0:
+            return None
+        if bound == "tensor":
+            ach = s["flops"] / s["launches"] / (s["ms"] / s["launches"] / 1e3) / 1e12
+            unit = "TFLOP/s"
+        else:
+            ach = s["bytes"] / s["launches"] / (s["ms"] / s["launches"] / 1e3) / 1e9
+            unit = "GB/s"
+        return {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+                "traffic": None, "kernel": name, "launches_per_step": s["launches"] / args.steps,
+                "ms_per_step": s["ms"] / args.steps, "peak_source": peak_src}
+
+    fams = {"gemm": ("tensor", tc_sust), "decode_main": ("hbm", hbm_peak), "residual": ("hbm", hbm_peak)}
+    dom = max(fams, key=lambda k: stats[k]["ms"])
+    roof = fam_roof(dom, *fams[dom])
+    roof_dec = fam_roof("decode_main", "hbm", hbm_peak)
+
+    line = {"metric": METRIC, "value": value, "unit": "context tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (planted low-rank + noise K/V, seeded)",
+            "config": {"workload": w.name, "batch": w.batch, "n_layers": w.n_layers,
+                       "layers_per_group": w.layers_per_group, "n_kv": w.n_kv, "n_q": w.n_q, "T": w.T,
+                       "d_h": w.d_h, "keys_pre_rope": w.keys_pre_rope, "budget_ratio": ratio,
+                       "q_cap": step.shape.q_cap, "sketch_cols": step.shape.sketch_cols,
+                       "power_iters": step.shape.power_iters, "l2": "inputs larger than L2 (no flush)",
+                       "parallelism": f"dp{world}" if world > 1 else "single-gpu"},
+            "breakdown_ms": {"analyze": t_an, "allocate_host": t_alloc, "compress": t_cmp, "decode": t_dec},
+            "compress": {"raw_gbs": raw / ((t_an + t_alloc + t_cmp) / 1e3) / 1e9,
+                         "raw_bytes": raw, "cache_bytes": cache_total, "ratio": raw / cache_total},
+            "decode": {"context_tokens_per_s": tokens * w.n_layers / (t_dec / 1e3) if t_dec > 0 else None,
+                       "context_tokens_per_s_per_layer_step": tokens / (t_dec / 1e3) if t_dec > 0 else None,
+                       "hbm_gbs": dbytes / (t_dec / 1e3) / 1e9 if t_dec > 0 else None,
+                       "alg_bytes": dbytes, "frac_of_hbm": dbytes / (t_dec / 1e3) / 1e9 / hbm_peak if t_dec > 0 else None},
+            "roofline": roof, "roofline_decode": roof_dec,
+            "kernel_stats": {k: {kk: (float(vv) if isinstance(vv, float) else int(vv)) for kk, vv in v.items()}
+                             for k, v in stats.items()},
+            "gpu_launches": n_kernels * args.steps if n_kernels is not None else None,
+            "kernels": kernel_names, "clocks": clk.summary(), "choices": sorted(set(map(tuple, step.choices)))}
+
+    # e2e: same step through the C ABI with host buffers: H2D of K and V and D2H of the outputs
+    if not args.no_e2e:
+        try:
+            Kh = step.K.cpu().pin_memory()
+            Vh = step.V.cpu().pin_memory()
+            outh = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+            Kd = torch.empty_like(step.K)
+            Vd = torch.empty_like(step.V)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            n_e2e = max(1, min(args.steps, 3))
+            Kd.copy_(Kh, non_blocking=True)
+            Vd.copy_(Vh, non_blocking=True)
+            step.run(K=Kd, V=Vd)
+            outh.copy_(step.out, non_blocking=True)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(n_e2e):
+                Kd.copy_(Kh, non_blocking=True)
+                Vd.copy_(Vh, non_blocking=True)
+                step.run(K=Kd, V=Vd)
+                outh.copy_(step.out, non_blocking=True)
+            e1.record()
+            torch.cuda.synchronize()
+            e_ms = e0.elapsed_time(e1) / n_e2e
+            line["e2e"] = {"value": tokens * world / (e_ms / 1e3), "unit": "context tokens/s",
+                           "h2d_bytes_per_step": Kh.numel() * Kh.element_size() * 2,
+                           "d2h_bytes_per_step": outh.numel() * outh.element_size(), "ms_per_step": e_ms,
+                           "steps": n_e2e}
+            del Kh, Vh, Kd, Vd
+        except (RuntimeError, MemoryError) as ex:
+            line["e2e"] = {"value": None, "unit": "context tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0, "error": str(ex)[:200]}
+
+    # CPU oracle on a bounded sample (rank 0, N = 1 only)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        G = w.n_layers // w.layers_per_group
+        ch = {0: step.choices[0], 1: step.choices[1]}
+        dt, desc = oracle_sample(w, ch, min(args.cpu_tokens, w.T), step.K, step.V)
+        t_full = dt * G * w.batch * (w.T / min(args.cpu_tokens, w.T))
+        line["cpu_baseline"] = {"value": tokens / t_full, "unit": "context tokens/s", "cores": cpu_threads(),
+                                "kind": "oracle", "sample": desc, "sample_seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

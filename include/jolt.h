@@ -231,6 +231,30 @@ size_t jolt_sym_eig_workspace(int32_t n, int32_t batch);
 jolt_status jolt_sym_eig(const float* A, int32_t n, int32_t batch, float* evals, float* evecs,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* Per-kernel-family device timing (off by default). When enabled, the library records a CUDA event
+ * pair on the launching stream around every launch of the families below and accumulates the
+ * elapsed device time together with the launch's algorithmic work (FLOPs of a contraction, or
+ * bytes a streaming kernel must move). Host-global; not for concurrent use from several threads. */
+typedef enum {
+  JOLT_K_GEMM = 0,          /* tcgen05 contractions of the compressor */
+  JOLT_K_DECODE_MAIN = 1,   /* split-T decode attention over the stored factors */
+  JOLT_K_RESIDUAL = 2,      /* residual rotate + quantise + pack */
+  JOLT_K_DECODE_AUX = 3,    /* decode prologue and split merge */
+  JOLT_K_COUNT = 4
+} jolt_kernel_family;
+
+typedef struct {
+  int32_t kernel;       /* jolt_kernel_family */
+  uint64_t launches;
+  double ms;            /* summed device time of the launches */
+  double flops;         /* summed algorithmic FLOPs */
+  double bytes;         /* summed algorithmic bytes */
+} jolt_kernel_stat;
+
+void jolt_stats_enable(int32_t on);
+/* Fills out[JOLT_K_COUNT] (host); synchronises on the pending events; reset != 0 clears. */
+jolt_status jolt_stats_read(jolt_kernel_stat* out, int32_t reset);
+
 #ifdef __cplusplus
 }
 #endif

@@ -32,6 +32,14 @@ class Shape(C.Structure):
                 ("attn_scale", C.c_float), ("rope_attention_scaling", C.c_float)]
 
 
+class KernelStat(C.Structure):
+    _fields_ = [("kernel", C.c_int32), ("launches", C.c_uint64), ("ms", C.c_double),
+                ("flops", C.c_double), ("bytes", C.c_double)]
+
+
+KERNEL_FAMILIES = ["gemm", "decode_main", "residual", "decode_aux"]
+
+
 class CellChoice(C.Structure):
     _fields_ = [("r_T", C.c_int32), ("r_d", C.c_int32), ("b", C.c_int32)]
 
@@ -66,6 +74,8 @@ SIGNATURES = [
                                  C.c_int64, C.c_int64, C.c_int64, C.c_int32, C.c_int64, C.c_int64,
                                  C.c_int64, C.c_int32, C.c_int32, _P]),
     ("jolt_sym_eig_workspace", C.c_size_t, [C.c_int32, C.c_int32]),
+    ("jolt_stats_enable", None, [C.c_int32]),
+    ("jolt_stats_read", C.c_int, [C.POINTER(KernelStat), C.c_int32]),
     ("jolt_sym_eig", C.c_int, [_P, C.c_int32, C.c_int32, _P, _P, _P, C.c_size_t, _P]),
 ]
 

@@ -203,7 +203,20 @@ def sym_eig(A, stream=None):
     return (ev, V) if batched else (ev[0], V[0])
 
 
-__all__ = ["sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
+def stats_enable(on=True):
+    lib().jolt_stats_enable(int(on))
+
+
+def stats_read(reset=True):
+    """Per kernel family: launches, device ms (CUDA events), algorithmic flops and bytes."""
+    from ._lib import KernelStat, KERNEL_FAMILIES
+    arr = (KernelStat * len(KERNEL_FAMILIES))()
+    check(lib().jolt_stats_read(arr, int(reset)), "jolt_stats_read")
+    return {KERNEL_FAMILIES[i]: dict(launches=arr[i].launches, ms=arr[i].ms, flops=arr[i].flops,
+                                     bytes=arr[i].bytes) for i in range(len(KERNEL_FAMILIES))}
+
+
+__all__ = ["stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
            "allocate", "workspace_bytes", "new_workspace", "analyze", "compress", "decode_attn",
            "check_ws", "rotate_rows", "quantize_pack", "unpack_dequant", "JoltError",
            "JOLT_OP_COMPRESS", "JOLT_OP_DECODE"]

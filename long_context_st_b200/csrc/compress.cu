@@ -4,20 +4,23 @@
 //   ||X||^2 (fp64), S_d = sum_lh X_lh^T X_lh (tcgen05), Y = X_(T) Omega (tcgen05, Rademacher Omega),
 //   q power iterations Y <- X_(T) orth(X_(T)^T orth(Y)), Q = orth(Y), B^T = X_(T)^T Q (hi/lo terms),
 //   W = B B^T, eig(W) (block Jacobi), U_T = Q V[:, :q_cap] (hi/lo terms) kept in the workspace.
-//   orth() is shifted CholeskyQR3: three passes of Gram (hi/lo terms) -> fp64 Cholesky of
-//   G + s*I -> Y R^{-1} (hi/lo terms), shifts 1e-4*max(diag), 1e-4*max(diag), 0.
+//   orth() is shifted CholeskyQR: passes of Gram (hi/lo terms) -> fp64 Cholesky of G + s*I ->
+//   Y R^{-1} (hi/lo terms) with s = 1e-4*||G||_F until the Gram is well conditioned, then s = 0.
 // compress, per cell: U_T (first r_T columns) stored; Y_lh = U_T^T X_lh (tcgen05);
 //   S_Y = sum Y_lh^T Y_lh; U_d = top-r_d eigenvectors (block Jacobi); G = Y U_d; X~ = U_T (G U_d^T)
 //   from the stored (rounded) factors (tcgen05, hi/lo terms); residual X - X~ rotated by the
 //   seeded randomized Hadamard, quantised per row and packed.
 #include <algorithm>
 #include <cmath>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <vector>
 
 #include "gemm_tc.cuh"
 #include "linalg.cuh"
 #include "pack.cuh"
+#include "stats.h"
 
 namespace jolt {
 
@@ -386,6 +389,14 @@ struct Ctx {
   template <typename Tp> Tp* atc(size_t rel) const { return reinterpret_cast<Tp*>(ws + p.off_cmp + rel); }
 };
 
+void report_error_host(const Ctx& c, int32_t code) {
+  int32_t cur = 0;
+  cudaMemcpyAsync(&cur, c.err, 4, cudaMemcpyDeviceToHost, c.st);
+  cudaStreamSynchronize(c.st);
+  if (!cur) cudaMemcpyAsync(c.err, &code, 4, cudaMemcpyHostToDevice, c.st);
+  cudaStreamSynchronize(c.st);
+}
+
 Operand plain(const void* ptr, int major, int64_t inner, int64_t outer, int64_t ld, int64_t batch = 1,
               int64_t bstride = 0) {
   Operand o;
@@ -415,7 +426,13 @@ Operand xunfold(const void* X, int major, const Plan& p, int C) {
   return o;
 }
 
-// Y <- orth(Y), Y fp32 [C][rows][l]; shifted CholeskyQR3 with hi/lo bf16 Grams and products.
+// Y <- orth(Y), Y fp32 [C][rows][l]: CholeskyQR passes with hi/lo bf16 Grams and products.
+// Shifted passes (s = 1e-4 * ||G||_F) run until the Cholesky's smallest pivot ratio R_jj^2 / G_jj
+// reaches 0.1; then unshifted passes run until one factors a Gram whose ratio is >= 0.9 (an
+// almost orthonormal input, so the output is orthonormal to the hi/lo precision). A breakdown of
+// an unshifted factorisation falls back to a shifted pass. At most kMaxOrthPasses passes.
+constexpr int kMaxOrthPasses = 8;
+
 jolt_status orth(const Ctx& c, float* Y, int rows, int C) {
   const Plan& p = c.p;
   const int l = p.l;
@@ -424,8 +441,8 @@ jolt_status orth(const Ctx& c, float* Y, int rows, int C) {
   float* Gm = c.at<float>(p.Gm);
   __nv_bfloat16* Rh = c.at<__nv_bfloat16>(p.Rh);
   __nv_bfloat16* Rl = c.at<__nv_bfloat16>(p.Rl);
-  const double shifts[3] = {1e-4, 1e-4, 0.0};
-  for (int pass = 0; pass < 3; ++pass) {
+  bool conditioned = false;
+  for (int pass = 0; pass < kMaxOrthPasses; ++pass) {
     jolt_status r = split_bf16(Y, l, rows, l, C, int64_t(rows) * l, Yh, Yl, l, int64_t(rows) * l, c.st);
     if (r) return r;
     JOLT_CUDA_TRY(cudaMemsetAsync(Gm, 0, size_t(C) * l * l * 4, c.st));
@@ -440,7 +457,42 @@ jolt_status orth(const Ctx& c, float* Y, int rows, int C) {
     g.k_split = ksplit_for(int64_t((l + 127) / 128) * ((l + 255) / 256) * C, rows);
     g.accumulate = true; g.err = c.err;
     if ((r = gemm_tc(g, c.st))) return r;
-    if ((r = chol_inverse(Gm, l, C, l, shifts[pass], Rh, Rl, c.pass() + p.chol, c.err, c.st))) return r;
+    if (std::getenv("JOLT_DEBUG")) {
+      std::vector<float> h(size_t(C) * l * l);
+      cudaMemcpyAsync(h.data(), Gm, h.size() * 4, cudaMemcpyDeviceToHost, c.st);
+      cudaStreamSynchronize(c.st);
+      for (int b = 0; b < C; ++b) {
+        const float* gb = h.data() + size_t(b) * l * l;
+        int bad = 0;
+        float dmn = 1e30f, dmx = 0.f, asym = 0.f;
+        for (int i = 0; i < l; ++i) {
+          dmn = std::min(dmn, gb[size_t(i) * l + i]);
+          dmx = std::max(dmx, gb[size_t(i) * l + i]);
+          for (int j = 0; j < l; ++j) {
+            bad += !std::isfinite(gb[size_t(i) * l + j]);
+            asym = std::max(asym, std::fabs(gb[size_t(i) * l + j] - gb[size_t(j) * l + i]));
+          }
+        }
+        std::fprintf(stderr, "jolt gram: rows %d pass %d cell %d nonfinite %d diag [%g, %g] asym %g\n", rows, pass, b,
+                     bad, dmn, dmx, asym);
+      }
+    }
+    const bool last = pass == kMaxOrthPasses - 1;
+    float ratio = 0.f;
+    double shift = (conditioned || last) ? 0.0 : 1e-4;
+    if ((r = chol_inverse(Gm, l, C, l, shift, Rh, Rl, c.pass() + p.chol, c.err, c.st, &ratio))) return r;
+    if (!(ratio > 0.f)) {
+      if (shift == 0.0 && pass < kMaxOrthPasses - 1) {
+        shift = 1e-4;
+        if ((r = chol_inverse(Gm, l, C, l, shift, Rh, Rl, c.pass() + p.chol, c.err, c.st, &ratio))) return r;
+      }
+      if (!(ratio > 0.f)) {
+        report_error_host(c, JOLT_ERR_NUMERIC);
+        return JOLT_ERR_NUMERIC;
+      }
+    }
+    if (std::getenv("JOLT_DEBUG"))
+      std::fprintf(stderr, "jolt orth: rows %d pass %d shift %g min pivot ratio %g\n", rows, pass, shift, ratio);
     GemmCall t;
     t.M = rows; t.N = l; t.K = l; t.n_terms = 3;
     const Operand ykh = plain(Yh, kMajorK, l, rows, l, C, int64_t(rows) * l);
@@ -452,6 +504,8 @@ jolt_status orth(const Ctx& c, float* Y, int rows, int C) {
     t.A[2] = ykl; t.B[2] = rh;
     t.C = Y; t.ldc = l; t.c_batch_stride = int64_t(rows) * l; t.batch = C; t.err = c.err;
     if ((r = gemm_tc(t, c.st))) return r;
+    if (shift == 0.0 && ratio >= 0.9f) return JOLT_OK;
+    if (ratio >= 0.1f) conditioned = true;
   }
   return JOLT_OK;
 }
@@ -692,12 +746,21 @@ extern "C" jolt_status jolt_analyze(const jolt_shape* shape, const void* k, cons
       std::vector<double> evT, evD;
       std::vector<double> nrm;
       jolt_status r = analyze_pass(c, kv ? v : k, kv, bg0, C, evT, evD, nrm);
-      if (r) return r;
-      if ((r = read_err(c))) return r;
+      if (r) {
+        if (std::getenv("JOLT_DEBUG")) std::fprintf(stderr, "jolt analyze: pass kv %d bg0 %d status %d\n", kv, bg0, int(r));
+        return r;
+      }
+      if ((r = read_err(c))) {
+        if (std::getenv("JOLT_DEBUG")) std::fprintf(stderr, "jolt analyze: device error %d after pass kv %d bg0 %d\n", int(r), kv, bg0);
+        return r;
+      }
       for (int i = 0; i < C; ++i) {
         const int cell = (bg0 + i) * 2 + kv;
         const double n2 = nrm[i];
-        if (!std::isfinite(n2)) return JOLT_ERR_NUMERIC;
+        if (!std::isfinite(n2)) {
+          if (std::getenv("JOLT_DEBUG")) std::fprintf(stderr, "jolt analyze: cell %d norm2 %g\n", cell, n2);
+          return JOLT_ERR_NUMERIC;
+        }
         norm2_out[cell] = n2;
         double cum = 0.0;
         for (int kk = 0; kk < nrt; ++kk) {
@@ -842,6 +905,9 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
       __half2* sz = reinterpret_cast<__half2*>(cb + offs[5 * cell + 4]);
       const int64_t rows = int64_t(LgH) * T;
       const int grid = int(std::min<int64_t>((rows + 7) / 8, 148 * 16));
+      // algorithmic bytes: read X (io dtype) and X~ (fp32, when present), write codes and sz
+      StatScope sc(JOLT_K_RESIDUAL, c.st, 0.0,
+                   double(rows) * d * ((io32 ? 4 : 2) + (Xt ? 4 : 0)) + double(rows) * (d * ch.b / 8 + 4));
       if (d == 128) {
         if (io32) k_residual<4, float><<<grid, 256, 0, c.st>>>(reinterpret_cast<const float*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
         else k_residual<4, __nv_bfloat16><<<grid, 256, 0, c.st>>>(reinterpret_cast<const __nv_bfloat16*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);

@@ -142,6 +142,21 @@ extern "C" jolt_status jolt_decode_attn(const jolt_shape* shape, const jolt_cell
     pc.q = static_cast<const uint8_t*>(q) + size_t(b0) * row * s.d_h * iob;
     pc.out = static_cast<uint8_t*>(out) + size_t(b0) * row * s.d_h * iob;
     pc.lse = lse ? lse + size_t(b0) * row : nullptr;
+    // algorithmic bytes of this launch set: per (b, layer) the U_T rows of K and V (per-layer
+    // re-read), and per KV head the packed codes and scale/zero pairs, plus U_d, G, q and out
+    double ab = 0.0;
+    const int sf = s.factor_dtype == JOLT_F32 ? 4 : 2;
+    for (int bi = 0; bi < nb; ++bi)
+      for (int li = 0; li < Lc; ++li) {
+        const int gi = (layer_begin + li) / s.layers_per_group - g_first;
+        for (int kv = 0; kv < 2; ++kv) {
+          const CellRef& c = pc.cells[(bi * Gc + gi) * 2 + kv];
+          ab += double(sf) * s.T * c.r_T + double(sf) * s.d_h * c.r_d + double(sf) * s.n_kv * c.r_T * c.r_d;
+          if (c.b) ab += double(s.n_kv) * s.T * (double(s.d_h) * c.b / 8 + 4);
+        }
+        ab += 2.0 * s.n_q * s.d_h * iob;
+      }
+    pc.alg_bytes = ab;
     jolt_status st_ = launch_decode_simt(pc, st);
     if (st_ != JOLT_OK) return st_;
   }

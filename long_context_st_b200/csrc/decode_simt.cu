@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "pack.cuh"
+#include "stats.h"
 
 namespace jolt {
 
@@ -390,16 +391,20 @@ size_t decode_simt_main_smem(const DecodeParams& p) {
 jolt_status launch_decode_simt(const DecodeParams& p, cudaStream_t st) {
   if (p.gq > kMaxGq) return JOLT_ERR_INVALID_ARG;
   const dim3 gq_grid(p.n_q, p.Lc, p.B);
-  if (p.d_h == 64) k_prologue_q<2><<<gq_grid, 128, 0, st>>>(p);
-  else k_prologue_q<4><<<gq_grid, 128, 0, st>>>(p);
-  JOLT_CUDA_TRY(cudaGetLastError());
-  if (p.pre_rope) {
-    k_prologue_bh<<<dim3(p.n_kv, p.Lc, p.B), 256, 0, st>>>(p);
+  {
+    StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
+    if (p.d_h == 64) k_prologue_q<2><<<gq_grid, 128, 0, st>>>(p);
+    else k_prologue_q<4><<<gq_grid, 128, 0, st>>>(p);
     JOLT_CUDA_TRY(cudaGetLastError());
+    if (p.pre_rope) {
+      k_prologue_bh<<<dim3(p.n_kv, p.Lc, p.B), 256, 0, st>>>(p);
+      JOLT_CUDA_TRY(cudaGetLastError());
+    }
   }
   const size_t smem = decode_simt_main_smem(p);
   if (smem > 227 * 1024) return JOLT_ERR_INVALID_ARG;
   const dim3 grid(p.S, p.n_kv, p.B * p.Lc);
+  StatScope sc(JOLT_K_DECODE_MAIN, st, 0.0, p.alg_bytes);
   if (p.d_h == 64) {
     JOLT_CUDA_TRY(cudaFuncSetAttribute(k_decode_main<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
     k_decode_main<2><<<grid, 256, smem, st>>>(p);
@@ -408,6 +413,7 @@ jolt_status launch_decode_simt(const DecodeParams& p, cudaStream_t st) {
     k_decode_main<4><<<grid, 256, smem, st>>>(p);
   }
   JOLT_CUDA_TRY(cudaGetLastError());
+  StatScope sc2(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
   const size_t msm = (size_t(p.q_cap) + 128 + p.d_h + p.S) * sizeof(float);
   if (p.d_h == 64) {
     JOLT_CUDA_TRY(cudaFuncSetAttribute(k_decode_merge<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(msm)));

@@ -17,6 +17,7 @@
 
 #include "gemm_tc.cuh"
 #include "sm100.cuh"
+#include "stats.h"
 
 namespace jolt {
 
@@ -288,6 +289,7 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   d.err = g.err;
   const dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM, g.batch * g.k_split);
   if (grid.y > 65535 || grid.z > 65535) return JOLT_ERR_INVALID_ARG;
+  StatScope sc(JOLT_K_GEMM, st, 2.0 * g.M * double(g.N) * g.K * g.batch * g.n_terms, 0.0);
   return BN == 256 ? launch_bn<256>(am, bm, maps, d, grid, st) : launch_bn<128>(am, bm, maps, d, grid, st);
 }
 

@@ -26,6 +26,8 @@ struct CholScratch {
   double* Gd;    // [nb][np][np]
   double* Xd;    // [nb][np][np]
   double* mdiag; // [nb]
+  double* diag0; // [nb][np] diagonal of G + shift
+  float* ratio;  // [nb] min pivot ratio
 };
 
 CholScratch chol_carve(void* scratch, int nb, int n) {
@@ -37,26 +39,39 @@ CholScratch chol_carve(void* scratch, int nb, int n) {
   s.Xd = reinterpret_cast<double*>(p);
   p += align_up(size_t(nb) * np * np * 8, 256);
   s.mdiag = reinterpret_cast<double*>(p);
+  p += align_up(size_t(nb) * 8, 256);
+  s.diag0 = reinterpret_cast<double*>(p);
+  p += align_up(size_t(nb) * np * 8, 256);
+  s.ratio = reinterpret_cast<float*>(p);
   return s;
 }
 
+// Frobenius norm of each matrix (the shift scale: ||G||_2 <= ||G||_F <= sqrt(n) ||G||_2).
 __global__ void k_maxdiag(const float* __restrict__ G, int64_t ldg, int n, double* md) {
   const int b = blockIdx.x;
   const float* g = G + int64_t(b) * n * ldg;
   double m = 0.0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmax(m, double(g[int64_t(i) * ldg + i]));
+  for (int64_t e = threadIdx.x; e < int64_t(n) * n; e += blockDim.x) {
+    const double v = g[(e / n) * ldg + e % n];
+    m += v * v;
+  }
   __shared__ double red[256];
   red[threadIdx.x] = m;
   __syncthreads();
   for (int s = blockDim.x / 2; s; s >>= 1) {
-    if (threadIdx.x < s) red[threadIdx.x] = fmax(red[threadIdx.x], red[threadIdx.x + s]);
+    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
     __syncthreads();
   }
-  if (threadIdx.x == 0) md[b] = red[0];
+  if (threadIdx.x == 0) md[b] = sqrt(red[0]);
+}
+
+__global__ void k_ratio_init(float* ratio, int nb) {
+  if (threadIdx.x < nb) ratio[threadIdx.x] = 1.f;
 }
 
 __global__ void k_chol_init(const float* __restrict__ G, int64_t ldg, int n, int np, double shift_rel,
-                            const double* __restrict__ md, double* __restrict__ Gd, double* __restrict__ Xd) {
+                            const double* __restrict__ md, double* __restrict__ Gd, double* __restrict__ Xd,
+                            double* __restrict__ diag0) {
   const int b = blockIdx.z;
   const int i0 = blockIdx.y * NB, j0 = blockIdx.x * NB;
   const float* g = G + int64_t(b) * n * ldg;
@@ -70,6 +85,7 @@ __global__ void k_chol_init(const float* __restrict__ G, int64_t ldg, int n, int
     else v = (i == j) ? 1.0 : 0.0;
     gd[int64_t(i) * np + j] = v;
     xd[int64_t(i) * np + j] = 0.0;
+    if (i == j) diag0[int64_t(b) * np + i] = v;
   }
 }
 
@@ -124,7 +140,7 @@ __device__ __forceinline__ void tile_ab(double (*C)[NB + 1], double (*A)[NB + 1]
 
 // Factor the diagonal block p and invert it.
 __global__ void __launch_bounds__(256) k_chol_diag(double* __restrict__ Gd, double* __restrict__ Xd, int np,
-                                                   int p, int32_t* err) {
+                                                   int p, const double* __restrict__ diag0, float* ratio) {
   extern __shared__ double sh[];
   double(*S)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*X)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
@@ -133,12 +149,16 @@ __global__ void __launch_bounds__(256) k_chol_diag(double* __restrict__ Gd, doub
   double* xd = Xd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
   tile_load(S, gd, np);
   __syncthreads();
+  float rmin = 1.f;
   for (int j = 0; j < NB; ++j) {
     if (threadIdx.x == 0) {
       double d = S[j][j];
-      if (!(d > 0.0)) {
-        report_error(err, JOLT_ERR_NUMERIC);
+      const double d0 = diag0[int64_t(b) * np + p * NB + j];
+      if (!(d > 0.0) || !(d0 > 0.0)) {
+        rmin = 0.f;  // breakdown: the caller retries with a shift
         d = 1.0;
+      } else {
+        rmin = fminf(rmin, float(d / d0));
       }
       S[j][j] = sqrt(d);
     }
@@ -153,6 +173,7 @@ __global__ void __launch_bounds__(256) k_chol_diag(double* __restrict__ Gd, doub
     }
     __syncthreads();
   }
+  if (threadIdx.x == 0) atomicMin(reinterpret_cast<int*>(ratio + b), __float_as_int(rmin));
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
     const int i = e / NB, k = e % NB;
     if (i > k) S[i][k] = 0.0;
@@ -530,17 +551,19 @@ int grid_1d(int64_t n, int per = 256) {
 
 size_t chol_scratch_bytes(int nb, int n) {
   const int np = rup(n, NB);
-  return 2 * align_up(size_t(nb) * np * np * 8, 256) + align_up(size_t(nb) * 8, 256);
+  return 2 * align_up(size_t(nb) * np * np * 8, 256) + align_up(size_t(nb) * 8, 256) +
+         align_up(size_t(nb) * np * 8, 256) + align_up(size_t(nb) * 4, 256);
 }
 
 jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shift_rel,
                          __nv_bfloat16* rinv_hi, __nv_bfloat16* rinv_lo, void* scratch, int32_t* err,
-                         cudaStream_t st) {
+                         cudaStream_t st, float* min_ratio) {
   if (nb < 1 || n < 1) return JOLT_OK;
   const int np = rup(n, NB), P = np / NB;
   CholScratch s = chol_carve(scratch, nb, n);
   k_maxdiag<<<nb, 256, 0, st>>>(G, ld_g, n, s.mdiag);
-  k_chol_init<<<dim3(P, P, nb), 256, 0, st>>>(G, ld_g, n, np, shift_rel, s.mdiag, s.Gd, s.Xd);
+  k_ratio_init<<<1, 256, 0, st>>>(s.ratio, nb);
+  k_chol_init<<<dim3(P, P, nb), 256, 0, st>>>(G, ld_g, n, np, shift_rel, s.mdiag, s.Gd, s.Xd, s.diag0);
   const int sm2 = 2 * NB * (NB + 1) * 8, sm3 = 3 * NB * (NB + 1) * 8, sm4 = 4 * NB * (NB + 1) * 8;
   static bool attr = false;
   if (!attr) {
@@ -551,7 +574,7 @@ jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shi
     attr = true;
   }
   for (int p = 0; p < P; ++p) {
-    k_chol_diag<<<nb, 256, sm2, st>>>(s.Gd, s.Xd, np, p, err);
+    k_chol_diag<<<nb, 256, sm2, st>>>(s.Gd, s.Xd, np, p, s.diag0, s.ratio);
     if (p + 1 < P) {
       k_chol_panel<<<dim3(P - p - 1, nb), 256, sm3, st>>>(s.Gd, s.Xd, np, p);
       const int npairs = (P - p - 1) * (P - p) / 2;
@@ -561,6 +584,15 @@ jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shi
   for (int d = 1; d < P; ++d) k_trinv<<<dim3(P - d, nb), 256, sm4, st>>>(s.Gd, s.Xd, np, d);
   k_rinv_out<<<dim3(grid_1d(int64_t(n) * n), nb), 256, 0, st>>>(s.Xd, np, n, rinv_hi, rinv_lo);
   JOLT_CUDA_TRY(cudaGetLastError());
+  (void)err;
+  if (min_ratio) {
+    std::vector<float> r(nb);
+    JOLT_CUDA_TRY(cudaMemcpyAsync(r.data(), s.ratio, sizeof(float) * nb, cudaMemcpyDeviceToHost, st));
+    JOLT_CUDA_TRY(cudaStreamSynchronize(st));
+    float m = 1.f;
+    for (float v : r) m = std::min(m, v);
+    *min_ratio = m;
+  }
   return JOLT_OK;
 }
 

@@ -5,12 +5,15 @@
 namespace jolt {
 
 // Blocked upper Cholesky of (G + shift*I) in fp64, G fp32 [nb][n][ld_g] symmetric, followed by the
-// triangular inverse. shift = shift_rel * max_i G_ii per matrix. Outputs R^{-1} split into bf16
+// triangular inverse. shift = shift_rel * ||G||_F per matrix. Outputs R^{-1} split into bf16
 // hi/lo parts [nb][n][n] (ready as a GEMM operand). Scratch: chol_scratch_bytes(nb, n).
+// min_ratio (host, may be null; synchronises): the smallest pivot ratio R_jj^2 / (G_jj + shift)
+// over the batch — 0 when a pivot was not positive (the factor is then unusable), near 1 for a
+// well-conditioned G.
 size_t chol_scratch_bytes(int nb, int n);
 jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shift_rel,
                          __nv_bfloat16* rinv_hi, __nv_bfloat16* rinv_lo, void* scratch,
-                         int32_t* err, cudaStream_t st);
+                         int32_t* err, cudaStream_t st, float* min_ratio = nullptr);
 
 // Symmetric eigendecomposition by block Jacobi (fp32), nb matrices A fp32 [nb][n][ld_a].
 // Outputs eigenvalues descending (fp32 [nb][n]) and eigenvectors as columns of V fp32 [nb][n][n]

@@ -167,3 +167,10 @@ def test_workspace_too_small(cuda_ok):
     with pytest.raises(api.JoltError) as e:
         api.analyze(shape, K, V, ws)
     assert e.value.status == -6
+
+
+def test_randomized_path_fp32_factors_orthonormal(cuda_ok):
+    # sketch narrower than the unfolding (l = 1152 < n = 4096): orthonormality of the stored
+    # fp32 bases and the 1% bar at a fixed choice
+    w = get_workload("llama8b_32k", n_layers=4, T=4096)
+    run(w, uniform(w, (256, 96, 2)), factor_dtype="f32", tail_tol=2e-3)
