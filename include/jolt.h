@@ -231,6 +231,27 @@ size_t jolt_sym_eig_workspace(int32_t n, int32_t batch);
 jolt_status jolt_sym_eig(const float* A, int32_t n, int32_t batch, float* evals, float* evecs,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* Decode attention without a caller-provided workspace: same arguments, results and kernels as
+ * jolt_decode_attn, except that its scratch lives in a fixed 32 MiB device array inside this
+ * library instead of `ws`. The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory when they decode, e.g. a plugin of an inference runtime that is
+ * handed a stream but no allocator, or a serving loop whose device memory is planned up front and
+ * where an allocation would synchronise the device or fail under memory pressure.
+ *   - Every GPU that loads the library reserves the 32 MiB until the process exits.
+ *   - The first call on a device looks up the array's device address (once per device, with that
+ *     device current); make that first call before any stream capture.
+ *   - A call whose scratch would exceed 32 MiB (jolt_workspace_bytes-style sizing for its
+ *     n_layers_call) returns JOLT_ERR_WORKSPACE before launching anything: use smaller
+ *     n_layers_call or jolt_decode_attn with your own workspace.
+ *   - Calls share the array: calls that overlap on the GPU (different streams, or other devices'
+ *     contexts excluded) race and corrupt each other's results. The error word is cleared at the
+ *     start of every call; device errors are not reported back by this call.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
+jolt_status jolt_decode_attn_noalloc(const jolt_shape* shape, const jolt_cell_choice* choices,
+                                     const void* cache, int32_t layer_begin, int32_t n_layers_call,
+                                     const void* q, void* out, float* lse, const float* inv_freq,
+                                     int32_t pos_offset, void* stream);
+
 /* Per-kernel-family device timing (off by default). When enabled, the library records a CUDA event
  * pair on the launching stream around every launch of the families below and accumulates the
  * elapsed device time together with the launch's algorithmic work (FLOPs of a contraction, or

@@ -67,6 +67,8 @@ SIGNATURES = [
     ("jolt_decode_attn", C.c_int, [C.POINTER(Shape), C.POINTER(CellChoice), _P, C.c_int32,
                                    C.c_int32, _P, _P, _P, _P, C.c_int32, _P, C.c_size_t, _P]),
     ("jolt_check", C.c_int, [_P, _P]),
+    ("jolt_decode_attn_noalloc", C.c_int, [C.POINTER(Shape), C.POINTER(CellChoice), _P, C.c_int32,
+                                           C.c_int32, _P, _P, _P, _P, C.c_int32, _P]),
     ("jolt_rotate_rows", C.c_int, [_P, _P, C.c_int64, C.c_int32, C.c_uint64, C.c_int32, _P]),
     ("jolt_quantize_pack", C.c_int, [_P, C.c_int64, C.c_int32, C.c_int32, _P, _P, _P, _P]),
     ("jolt_unpack_dequant", C.c_int, [_P, _P, C.c_int64, C.c_int32, C.c_int32, _P, _P]),

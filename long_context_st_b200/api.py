@@ -137,6 +137,16 @@ def decode_attn(s: Shape, choices, cache, q, out, ws, lse=None, inv_freq=None, l
                                  ws.numel(), _stream(stream)), "jolt_decode_attn")
 
 
+def decode_attn_noalloc(s: Shape, choices, cache, q, out, lse=None, inv_freq=None, layer_begin=0,
+                        n_layers_call=None, pos_offset=0, stream=None):
+    """jolt_decode_attn with the library's built-in 32 MiB scratch instead of a workspace."""
+    if n_layers_call is None:
+        n_layers_call = s.n_layers - layer_begin
+    check(lib().jolt_decode_attn_noalloc(C.byref(s), choices_array(choices), _ptr(cache), layer_begin,
+                                         n_layers_call, _ptr(q), _ptr(out), _ptr(lse), _ptr(inv_freq),
+                                         pos_offset, _stream(stream)), "jolt_decode_attn_noalloc")
+
+
 def check_ws(ws, stream=None):
     check(lib().jolt_check(_ptr(ws), _stream(stream)), "device error")
 
@@ -216,7 +226,7 @@ def stats_read(reset=True):
                                      bytes=arr[i].bytes) for i in range(len(KERNEL_FAMILIES))}
 
 
-__all__ = ["stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
+__all__ = ["decode_attn_noalloc", "stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
            "allocate", "workspace_bytes", "new_workspace", "analyze", "compress", "decode_attn",
            "check_ws", "rotate_rows", "quantize_pack", "unpack_dequant", "JoltError",
            "JOLT_OP_COMPRESS", "JOLT_OP_DECODE"]

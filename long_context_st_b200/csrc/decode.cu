@@ -1,5 +1,6 @@
 // jolt_decode_attn: argument checks, workspace carving, split choice and kernel dispatch.
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include "common.cuh"
@@ -174,4 +175,48 @@ extern "C" jolt_status jolt_check(void* ws, void* stream) {
     JOLT_CUDA_TRY(cudaMemcpy(ws, &zero, sizeof(int32_t), cudaMemcpyHostToDevice));
   }
   return static_cast<jolt_status>(err);
+}
+
+// ---- decode without a caller-provided workspace ------------------------------------------------
+// Scratch of jolt_decode_attn_noalloc: a file-scope device array that every GPU loading this
+// library holds until the process exits. Host code must not pass the array's name to a kernel (on
+// the host it is only a stand-in symbol); its device address is looked up once per device.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+extern "C" jolt_status jolt_decode_attn_noalloc(const jolt_shape* shape, const jolt_cell_choice* choices,
+                                                const void* cache, int32_t layer_begin, int32_t n_layers_call,
+                                                const void* q, void* out, float* lse, const float* inv_freq,
+                                                int32_t pos_offset, void* stream) {
+  if (!shape_ok(shape) || !choices || !cache || !q || !out) return JOLT_ERR_INVALID_ARG;
+  if (layer_begin < 0 || n_layers_call < 1 || layer_begin + n_layers_call > shape->n_layers)
+    return JOLT_ERR_INVALID_ARG;
+  // the scratch this call needs must fit the static array
+  if (decode_ws_layout(*shape, n_layers_call, choose_splits(*shape, n_layers_call)).total > kNoAllocScratchBytes)
+    return JOLT_ERR_WORKSPACE;
+  int dev = 0;
+  JOLT_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return JOLT_ERR_INVALID_ARG;
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void* ptr = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+      if (e != cudaSuccess || !ptr) return JOLT_ERR_CUDA;
+      g_noalloc_ptr[dev] = ptr;
+    }
+    ws = g_noalloc_ptr[dev];
+  }
+  // every call shares the array: the error word must start at zero; everything else the decode
+  // kernels read is written earlier in the same call
+  JOLT_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)));
+  return jolt_decode_attn(shape, choices, cache, layer_begin, n_layers_call, q, out, lse, inv_freq, pos_offset, ws,
+                          kNoAllocScratchBytes, stream);
 }
