@@ -43,6 +43,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=4096)
+    ap.add_argument("--layers", type=int, default=None, help="override n_layers (small profiling cases)")
+    ap.add_argument("--seqlen", type=int, default=None, help="override T (small profiling cases)")
+    ap.add_argument("--nvtx", action="store_true", help="NVTX range 'jolt_step' around each timed step")
+    ap.add_argument("--no-count", action="store_true", help="skip the CUPTI kernel count")
     return ap.parse_args()
 
 
@@ -280,7 +284,12 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    w = get_workload(args.workload)
+    over = {}
+    if args.layers:
+        over["n_layers"] = args.layers
+    if args.seqlen:
+        over["T"] = args.seqlen
+    w = get_workload(args.workload, **over)
     if world > 1:
         import datetime
         import torch.distributed as dist
@@ -296,7 +305,7 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     # weak scaling: every rank compresses and decodes its own sequences (own seed)
-    w = get_workload(args.workload, seed=w.seed + 1000 * rank) if rank else w
+    w = get_workload(args.workload, seed=w.seed + 1000 * rank, **over) if rank else w
     ratio = args.ratio if args.ratio else (w.budget_ratios[0] if w.budget_ratios else None)
     hbm_peak, tc_burst, tc_sust, peak_src = load_peaks()
     from long_context_st_b200 import api
@@ -306,7 +315,7 @@ def main():
     for _ in range(max(3, args.warmup)):
         step.run()
     torch.cuda.synchronize()
-    n_kernels, kernel_names = count_kernels(step)
+    n_kernels, kernel_names = (None, []) if args.no_count else count_kernels(step)
 
     names = ["start", "analyzed", "allocated", "compressed", "decoded"]
     evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
@@ -321,7 +330,11 @@ def main():
     with Clocks(local) as clk:
         t_start.record()
         for i in range(args.steps):
+            if args.nvtx:
+                torch.cuda.nvtx.range_push("jolt_step")
             step.run(evs[i])
+            if args.nvtx:
+                torch.cuda.nvtx.range_pop()
         t_end.record()
         torch.cuda.synchronize()
     api.stats_enable(False)

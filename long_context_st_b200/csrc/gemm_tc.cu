@@ -183,6 +183,26 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
 
 // ---- host: tensor maps ----------------------------------------------------------------------
 
+template <int BN, int AM, int BMJ>
+jolt_status launch(const TmaPack& maps, const GemmDev& d, dim3 grid, cudaStream_t st) {
+  using C = Cfg<BN>;
+  auto kern = k_gemm<BN, AM, BMJ>;
+  JOLT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem));
+  kern<<<grid, 128, C::kSmem, st>>>(maps, d);
+  JOLT_CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
+template <int BN>
+jolt_status launch_bn(int am, int bm, const TmaPack& maps, const GemmDev& d, dim3 grid, cudaStream_t st) {
+  if (am == kMajorK && bm == kMajorK) return launch<BN, kMajorK, kMajorK>(maps, d, grid, st);
+  if (am == kMajorK && bm == kMajorMN) return launch<BN, kMajorK, kMajorMN>(maps, d, grid, st);
+  if (am == kMajorMN && bm == kMajorK) return launch<BN, kMajorMN, kMajorK>(maps, d, grid, st);
+  return launch<BN, kMajorMN, kMajorMN>(maps, d, grid, st);
+}
+
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -201,7 +221,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool make_map(CUtensorMap* m, const Operand& o, int rows) {
+bool make_tensor_map(CUtensorMap* m, const Operand& o, int rows) {
+  constexpr int BK = 64;
   EncodeTiledFn enc = encode_fn();
   if (!enc || !o.ptr) return false;
   if (reinterpret_cast<uintptr_t>(o.ptr) % 16) return false;
@@ -238,26 +259,6 @@ bool make_map(CUtensorMap* m, const Operand& o, int rows) {
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int AM, int BMJ>
-jolt_status launch(const TmaPack& maps, const GemmDev& d, dim3 grid, cudaStream_t st) {
-  using C = Cfg<BN>;
-  auto kern = k_gemm<BN, AM, BMJ>;
-  JOLT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem));
-  kern<<<grid, 128, C::kSmem, st>>>(maps, d);
-  JOLT_CUDA_TRY(cudaGetLastError());
-  return JOLT_OK;
-}
-
-template <int BN>
-jolt_status launch_bn(int am, int bm, const TmaPack& maps, const GemmDev& d, dim3 grid, cudaStream_t st) {
-  if (am == kMajorK && bm == kMajorK) return launch<BN, kMajorK, kMajorK>(maps, d, grid, st);
-  if (am == kMajorK && bm == kMajorMN) return launch<BN, kMajorK, kMajorMN>(maps, d, grid, st);
-  if (am == kMajorMN && bm == kMajorK) return launch<BN, kMajorMN, kMajorK>(maps, d, grid, st);
-  return launch<BN, kMajorMN, kMajorMN>(maps, d, grid, st);
-}
-
-}  // namespace
-
 jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return JOLT_OK;
   if (g.n_terms < 1 || g.n_terms > kMaxTerms || !g.C || g.batch < 1 || g.k_split < 1 || g.c_batch_div < 1)
@@ -273,8 +274,8 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   memset(&maps, 0, sizeof(maps));
   GemmDev d{};
   for (int t = 0; t < g.n_terms; ++t) {
-    if (!make_map(&maps.a[t], g.A[t], BM)) return JOLT_ERR_INVALID_ARG;
-    if (!make_map(&maps.b[t], g.B[t], BN)) return JOLT_ERR_INVALID_ARG;
+    if (!make_tensor_map(&maps.a[t], g.A[t], BM)) return JOLT_ERR_INVALID_ARG;
+    if (!make_tensor_map(&maps.b[t], g.B[t], BN)) return JOLT_ERR_INVALID_ARG;
     d.a_fold[t] = int(g.A[t].fold);
     d.b_fold[t] = int(g.B[t].fold);
     d.a_batch[t] = g.A[t].batch_stride ? int(g.A[t].batch) : 1;

@@ -42,6 +42,10 @@ struct GemmCall {
   int32_t* err = nullptr;
 };
 
+// TMA tensor map (bf16, 128-byte swizzle) for an operand: box = 64 contiguous elements x `rows`
+// (K-major) or 64 x 64 (MN-major). False if the driver rejects it or the pointer is misaligned.
+bool make_tensor_map(CUtensorMap* m, const Operand& o, int rows);
+
 // Launch; validates shapes and alignment (JOLT_ERR_INVALID_ARG) before any launch.
 jolt_status gemm_tc(const GemmCall& g, cudaStream_t st);
 

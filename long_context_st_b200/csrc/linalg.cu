@@ -22,12 +22,52 @@ constexpr int JS = 2 * JW;
 
 inline int rup(int x, int a) { return (x + a - 1) / a * a; }
 
+// Grid-wide barrier for cooperative launches (all blocks co-resident), with a time limit: a block
+// that waits more than ~2 s reports JOLT_ERR_TIMEOUT and stops waiting; once the error word is set,
+// later barriers do not wait at all, so a failure never hangs the GPU.
+struct GridBar {
+  unsigned int* count;
+  unsigned int* gen;
+  int32_t* err;
+};
+
+__device__ __forceinline__ void grid_barrier(const GridBar& gb) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile unsigned int* vgen = gb.gen;
+    const unsigned int g = *vgen;
+    __threadfence();
+    const unsigned int arrived = atomicAdd(gb.count, 1u);
+    if (arrived == gridDim.x - 1) {
+      *gb.count = 0;
+      __threadfence();
+      atomicAdd(gb.gen, 1u);
+    } else {
+      uint64_t t0;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+      while (*vgen == g) {
+        if (*reinterpret_cast<volatile int32_t*>(gb.err) != 0) break;
+        uint64_t t1;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+        if (t1 - t0 > 2000000000ull) {
+          atomicCAS(gb.err, 0, int32_t(JOLT_ERR_TIMEOUT));
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+}
+
 struct CholScratch {
   double* Gd;    // [nb][np][np]
   double* Xd;    // [nb][np][np]
   double* mdiag; // [nb]
   double* diag0; // [nb][np] diagonal of G + shift
   float* ratio;  // [nb] min pivot ratio
+  unsigned int* bar;  // [2] grid barrier count, generation
 };
 
 CholScratch chol_carve(void* scratch, int nb, int n) {
@@ -43,51 +83,13 @@ CholScratch chol_carve(void* scratch, int nb, int n) {
   s.diag0 = reinterpret_cast<double*>(p);
   p += align_up(size_t(nb) * np * 8, 256);
   s.ratio = reinterpret_cast<float*>(p);
+  p += align_up(size_t(nb) * 4, 256);
+  s.bar = reinterpret_cast<unsigned int*>(p);
   return s;
 }
 
-// Frobenius norm of each matrix (the shift scale: ||G||_2 <= ||G||_F <= sqrt(n) ||G||_2).
-__global__ void k_maxdiag(const float* __restrict__ G, int64_t ldg, int n, double* md) {
-  const int b = blockIdx.x;
-  const float* g = G + int64_t(b) * n * ldg;
-  double m = 0.0;
-  for (int64_t e = threadIdx.x; e < int64_t(n) * n; e += blockDim.x) {
-    const double v = g[(e / n) * ldg + e % n];
-    m += v * v;
-  }
-  __shared__ double red[256];
-  red[threadIdx.x] = m;
-  __syncthreads();
-  for (int s = blockDim.x / 2; s; s >>= 1) {
-    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) md[b] = sqrt(red[0]);
-}
 
-__global__ void k_ratio_init(float* ratio, int nb) {
-  if (threadIdx.x < nb) ratio[threadIdx.x] = 1.f;
-}
 
-__global__ void k_chol_init(const float* __restrict__ G, int64_t ldg, int n, int np, double shift_rel,
-                            const double* __restrict__ md, double* __restrict__ Gd, double* __restrict__ Xd,
-                            double* __restrict__ diag0) {
-  const int b = blockIdx.z;
-  const int i0 = blockIdx.y * NB, j0 = blockIdx.x * NB;
-  const float* g = G + int64_t(b) * n * ldg;
-  double* gd = Gd + int64_t(b) * np * np;
-  double* xd = Xd + int64_t(b) * np * np;
-  const double sh = shift_rel * md[b];
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int i = i0 + e / NB, j = j0 + e % NB;
-    double v;
-    if (i < n && j < n) v = double(g[int64_t(i) * ldg + j]) + (i == j ? sh : 0.0);
-    else v = (i == j) ? 1.0 : 0.0;
-    gd[int64_t(i) * np + j] = v;
-    xd[int64_t(i) * np + j] = 0.0;
-    if (i == j) diag0[int64_t(b) * np + i] = v;
-  }
-}
 
 // 64x64 fp64 tile load/store helpers (row stride np).
 __device__ __forceinline__ void tile_load(double (*S)[NB + 1], const double* src, int np) {
@@ -138,13 +140,11 @@ __device__ __forceinline__ void tile_ab(double (*C)[NB + 1], double (*A)[NB + 1]
     for (int v = 0; v < 4; ++v) C[ty * 4 + u][tx * 4 + v] = acc[u][v];
 }
 
-// Factor the diagonal block p and invert it.
-__global__ void __launch_bounds__(256) k_chol_diag(double* __restrict__ Gd, double* __restrict__ Xd, int np,
-                                                   int p, const double* __restrict__ diag0, float* ratio) {
-  extern __shared__ double sh[];
+// Factor the diagonal block p of matrix b and invert it.
+__device__ void dev_chol_diag(double* __restrict__ Gd, double* __restrict__ Xd, int np, int p,
+                              const double* __restrict__ diag0, float* ratio, int b, double* sh) {
   double(*S)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*X)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
-  const int b = blockIdx.x;
   double* gd = Gd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
   double* xd = Xd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
   tile_load(S, gd, np);
@@ -192,16 +192,15 @@ __global__ void __launch_bounds__(256) k_chol_diag(double* __restrict__ Gd, doub
   __syncthreads();
   tile_store(gd, S, np);
   tile_store(xd, X, np);
+  __syncthreads();
 }
 
 // Panel: R_pj = X_pp^T G_pj for j > p.
-__global__ void __launch_bounds__(256) k_chol_panel(double* __restrict__ Gd, const double* __restrict__ Xd,
-                                                    int np, int p) {
-  extern __shared__ double sh[];
+__device__ void dev_chol_panel(double* __restrict__ Gd, const double* __restrict__ Xd, int np, int p, int b,
+                               int j, double* sh) {
   double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
   double(*C)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 2 * NB * (NB + 1));
-  const int b = blockIdx.y, j = p + 1 + blockIdx.x;
   const double* xpp = Xd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
   double* gpj = Gd + int64_t(b) * np * np + int64_t(p) * NB * np + j * NB;
   tile_load(A, xpp, np);
@@ -210,16 +209,15 @@ __global__ void __launch_bounds__(256) k_chol_panel(double* __restrict__ Gd, con
   tile_atb(C, A, B);
   __syncthreads();
   tile_store(gpj, C, np);
+  __syncthreads();
 }
 
-// Trailing update: G_ij -= R_pi^T R_pj for p < i <= j.
-__global__ void __launch_bounds__(256) k_chol_update(double* __restrict__ Gd, int np, int P, int p) {
-  extern __shared__ double sh[];
+// Trailing update: G_ij -= R_pi^T R_pj for p < i <= j (pair number idx).
+__device__ void dev_chol_update(double* __restrict__ Gd, int np, int P, int p, int b, int idx, double* sh) {
   double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
   double(*C)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 2 * NB * (NB + 1));
-  const int b = blockIdx.y;
-  int idx = blockIdx.x, i = p + 1;
+  int i = p + 1;
   while (idx >= P - i) {
     idx -= P - i;
     ++i;
@@ -233,17 +231,17 @@ __global__ void __launch_bounds__(256) k_chol_update(double* __restrict__ Gd, in
   __syncthreads();
   double* gij = g + int64_t(i) * NB * np + j * NB;
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) gij[int64_t(e / NB) * np + e % NB] -= C[e / NB][e % NB];
+  __syncthreads();
 }
 
 // Inverse blocks at distance d: X_ij = -X_ii * sum_{k=i+1..j} R_ik X_kj, j = i + d.
-__global__ void __launch_bounds__(256) k_trinv(const double* __restrict__ Gd, double* __restrict__ Xd, int np,
-                                               int d) {
-  extern __shared__ double sh[];
+__device__ void dev_trinv(const double* __restrict__ Gd, double* __restrict__ Xd, int np, int d, int b, int i,
+                          double* sh) {
   double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
   double(*C)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 2 * NB * (NB + 1));
   double(*Acc)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 3 * NB * (NB + 1));
-  const int b = blockIdx.y, i = blockIdx.x, j = i + d;
+  const int j = i + d;
   const double* g = Gd + int64_t(b) * np * np;
   double* x = Xd + int64_t(b) * np * np;
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) Acc[e / NB][e % NB] = 0.0;
@@ -263,28 +261,103 @@ __global__ void __launch_bounds__(256) k_trinv(const double* __restrict__ Gd, do
   __syncthreads();
   double* xij = x + int64_t(i) * NB * np + j * NB;
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) xij[int64_t(e / NB) * np + e % NB] = -C[e / NB][e % NB];
+  __syncthreads();
 }
 
-__global__ void k_rinv_out(const double* __restrict__ Xd, int np, int n, __nv_bfloat16* hi, __nv_bfloat16* lo) {
-  const int b = blockIdx.y;
-  const int64_t total = int64_t(n) * n;
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
-    const int i = int(e / n), j = int(e % n);
-    const float v = (i <= j) ? float(Xd[int64_t(b) * np * np + int64_t(i) * np + j]) : 0.f;
+struct CholArgs {
+  const float* G;
+  int64_t ldg;
+  int n, np, P, nb;
+  double shift_rel;
+  double *Gd, *Xd, *md, *diag0;
+  float* ratio;
+  __nv_bfloat16 *hi, *lo;
+  GridBar bar;
+};
+
+// The whole blocked Cholesky + triangular inverse of nb matrices in one cooperative launch.
+__global__ void __launch_bounds__(256) k_chol_coop(CholArgs a) {
+  extern __shared__ double sh[];
+  const int nbk = gridDim.x;
+  // norms and ratios
+  for (int b = blockIdx.x; b < a.nb; b += nbk) {
+    const float* g = a.G + int64_t(b) * a.n * a.ldg;
+    double m = 0.0;
+    for (int64_t e = threadIdx.x; e < int64_t(a.n) * a.n; e += blockDim.x) {
+      const double v = g[(e / a.n) * a.ldg + e % a.n];
+      m += v * v;
+    }
+    sh[threadIdx.x] = m;
+    __syncthreads();
+    for (int st = blockDim.x / 2; st; st >>= 1) {
+      if (threadIdx.x < st) sh[threadIdx.x] += sh[threadIdx.x + st];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+      a.md[b] = sqrt(sh[0]);
+      a.ratio[b] = 1.f;
+    }
+    __syncthreads();
+  }
+  grid_barrier(a.bar);
+  // shifted copy into fp64 working storage
+  {
+    const int64_t tot = int64_t(a.nb) * a.np * a.np;
+    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < tot; e += int64_t(nbk) * blockDim.x) {
+      const int b = int(e / (int64_t(a.np) * a.np));
+      const int64_t r = e % (int64_t(a.np) * a.np);
+      const int i = int(r / a.np), j = int(r % a.np);
+      double v;
+      if (i < a.n && j < a.n) v = double(a.G[int64_t(b) * a.n * a.ldg + int64_t(i) * a.ldg + j]) + (i == j ? a.shift_rel * a.md[b] : 0.0);
+      else v = (i == j) ? 1.0 : 0.0;
+      a.Gd[e] = v;
+      a.Xd[e] = 0.0;
+      if (i == j) a.diag0[int64_t(b) * a.np + i] = v;
+    }
+  }
+  grid_barrier(a.bar);
+  for (int p = 0; p < a.P; ++p) {
+    for (int b = blockIdx.x; b < a.nb; b += nbk) dev_chol_diag(a.Gd, a.Xd, a.np, p, a.diag0, a.ratio, b, sh);
+    grid_barrier(a.bar);
+    if (p + 1 < a.P) {
+      const int np1 = a.P - p - 1;
+      for (int it = blockIdx.x; it < a.nb * np1; it += nbk) dev_chol_panel(a.Gd, a.Xd, a.np, p, it / np1, p + 1 + it % np1, sh);
+      grid_barrier(a.bar);
+      const int npairs = np1 * (np1 + 1) / 2;
+      for (int it = blockIdx.x; it < a.nb * npairs; it += nbk) dev_chol_update(a.Gd, a.np, a.P, p, it / npairs, it % npairs, sh);
+      grid_barrier(a.bar);
+    }
+  }
+  for (int d = 1; d < a.P; ++d) {
+    const int cnt = a.P - d;
+    for (int it = blockIdx.x; it < a.nb * cnt; it += nbk) dev_trinv(a.Gd, a.Xd, a.np, d, it / cnt, it % cnt, sh);
+    grid_barrier(a.bar);
+  }
+  const int64_t tot = int64_t(a.n) * a.n;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < tot * a.nb; e += int64_t(nbk) * blockDim.x) {
+    const int b = int(e / tot);
+    const int64_t r = e % tot;
+    const int i = int(r / a.n), j = int(r % a.n);
+    const float v = (i <= j) ? float(a.Xd[int64_t(b) * a.np * a.np + int64_t(i) * a.np + j]) : 0.f;
     const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    hi[int64_t(b) * total + e] = h;
-    lo[int64_t(b) * total + e] = __float2bfloat16_rn(v - __bfloat162float(h));
+    a.hi[e] = h;
+    a.lo[e] = __float2bfloat16_rn(v - __bfloat162float(h));
   }
 }
 
+
 // ---- block Jacobi (fp64 working precision) -----------------------------------------------------
+
+constexpr int kJacMaxSweeps = 40;
 
 struct JacScratch {
   double* A;     // [nb][np][np]
   double* V;     // [nb][np][np]
   double* Th;    // [nb][npair][JS][JS]
-  double* norms; // [nb][2] off^2, total^2
+  double* norms; // [kJacMaxSweeps][nb][2] off^2, total^2
   int* perm;     // [nb][np]
+  unsigned int* bar;  // [2] grid barrier count, generation
+  int* sweeps;   // [1]
 };
 
 JacScratch jac_carve(void* scratch, int nb, int n) {
@@ -295,8 +368,10 @@ JacScratch jac_carve(void* scratch, int nb, int n) {
   s.A = reinterpret_cast<double*>(p); p += align_up(size_t(nb) * np * np * 8, 256);
   s.V = reinterpret_cast<double*>(p); p += align_up(size_t(nb) * np * np * 8, 256);
   s.Th = reinterpret_cast<double*>(p); p += align_up(size_t(nb) * npair * JS * JS * 8, 256);
-  s.norms = reinterpret_cast<double*>(p); p += align_up(size_t(nb) * 16, 256);
-  s.perm = reinterpret_cast<int*>(p);
+  s.norms = reinterpret_cast<double*>(p); p += align_up(size_t(kJacMaxSweeps) * nb * 16, 256);
+  s.perm = reinterpret_cast<int*>(p); p += align_up(size_t(nb) * np * 4, 256);
+  s.bar = reinterpret_cast<unsigned int*>(p); p += 256;
+  s.sweeps = reinterpret_cast<int*>(p);
   return s;
 }
 
@@ -325,14 +400,13 @@ __host__ __device__ __forceinline__ void tour_pair(int m, int r, int k, int* a, 
 
 typedef double Tile[JS][JS + 1];
 
-__global__ void __launch_bounds__(256) k_jac_solve(const double* __restrict__ Aw, int np, int nblk, int round,
-                                                   double* __restrict__ Th) {
-  extern __shared__ double jsm[];
+__device__ void dev_jac_solve(const double* __restrict__ Aw, int np, int nblk, int round, double* __restrict__ Th,
+                              int b, int k, double* jsm) {
   Tile& S = *reinterpret_cast<Tile*>(jsm);
   Tile& Q = *reinterpret_cast<Tile*>(jsm + JS * (JS + 1));
   __shared__ double cs[JW], sn[JW];
   __shared__ int pp[JW], qq[JW];
-  const int b = blockIdx.y, k = blockIdx.x, npair = nblk / 2;
+  const int npair = nblk / 2;
   int I, J;
   tour_pair(nblk, round, k, &I, &J);
   const double* a = Aw + int64_t(b) * np * np;
@@ -384,15 +458,15 @@ __global__ void __launch_bounds__(256) k_jac_solve(const double* __restrict__ Aw
   }
   double* th = Th + (int64_t(b) * npair + k) * JS * JS;
   for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) th[e] = Q[e / JS][e % JS];
+  __syncthreads();
 }
 
 // columns I u J of A and V (chunk of 64 rows per CTA): X[:, IJ] <- X[:, IJ] * Theta
-__global__ void __launch_bounds__(256) k_jac_cols(double* __restrict__ Aw, double* __restrict__ V, int np,
-                                                  int nblk, int round, const double* __restrict__ Th) {
-  extern __shared__ double jsm[];
+__device__ void dev_jac_cols(double* __restrict__ Aw, double* __restrict__ V, int np, int nblk, int round,
+                             const double* __restrict__ Th, int b, int k, int chunk, double* jsm) {
   Tile& T = *reinterpret_cast<Tile*>(jsm);
   Tile& X = *reinterpret_cast<Tile*>(jsm + JS * (JS + 1));
-  const int b = blockIdx.z, k = blockIdx.x, r0 = blockIdx.y * JS, npair = nblk / 2;
+  const int r0 = chunk * JS, npair = nblk / 2;
   int I, J;
   tour_pair(nblk, round, k, &I, &J);
   const double* th = Th + (int64_t(b) * npair + k) * JS * JS;
@@ -428,15 +502,15 @@ __global__ void __launch_bounds__(256) k_jac_cols(double* __restrict__ Aw, doubl
         M[int64_t(r0 + ty * 4 + u) * np + gv] = acc[u][v];
       }
   }
+  __syncthreads();
 }
 
 // rows I u J of A (chunk of 64 columns per CTA): A[IJ, :] <- Theta^T A[IJ, :]
-__global__ void __launch_bounds__(256) k_jac_rows(double* __restrict__ Aw, int np, int nblk, int round,
-                                                  const double* __restrict__ Th) {
-  extern __shared__ double jsm[];
+__device__ void dev_jac_rows(double* __restrict__ Aw, int np, int nblk, int round, const double* __restrict__ Th,
+                             int b, int k, int chunk, double* jsm) {
   Tile& T = *reinterpret_cast<Tile*>(jsm);
   Tile& X = *reinterpret_cast<Tile*>(jsm + JS * (JS + 1));
-  const int b = blockIdx.z, k = blockIdx.x, c0 = blockIdx.y * JS, npair = nblk / 2;
+  const int c0 = chunk * JS, npair = nblk / 2;
   int I, J;
   tour_pair(nblk, round, k, &I, &J);
   const double* th = Th + (int64_t(b) * npair + k) * JS * JS;
@@ -468,24 +542,70 @@ __global__ void __launch_bounds__(256) k_jac_rows(double* __restrict__ Aw, int n
 #pragma unroll
     for (int v = 0; v < 4; ++v) M[int64_t(gu) * np + c0 + tx * 4 + v] = acc[u][v];
   }
+  __syncthreads();
 }
 
-__global__ void k_jac_norms(const double* __restrict__ Aw, int np, double* norms) {
-  const int b = blockIdx.y;
-  const int64_t total = int64_t(np) * np;
-  double off = 0.0, tot = 0.0;
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
-    const double v = Aw[int64_t(b) * total + e];
-    tot += v * v;
-    if (e / np != e % np) off += v * v;
-  }
-  for (int m = 16; m; m >>= 1) {
-    off += __shfl_xor_sync(0xffffffffu, off, m);
-    tot += __shfl_xor_sync(0xffffffffu, tot, m);
-  }
-  if ((threadIdx.x & 31) == 0) {
-    atomicAdd(&norms[2 * b], off);
-    atomicAdd(&norms[2 * b + 1], tot);
+struct JacArgs {
+  double *A, *V, *Th, *norms;  // norms [max_sweeps][nb][2], zeroed before launch
+  int np, nblk, npair, chunks, nb, max_sweeps;
+  double tol;
+  int* sweeps_done;
+  GridBar bar;
+};
+
+// Block-Jacobi sweeps until the off-diagonal norm of every matrix is below tol (one launch).
+__global__ void __launch_bounds__(256) k_jac_coop(JacArgs a) {
+  extern __shared__ double jsm[];
+  const int nbk = gridDim.x;
+  __shared__ int s_done;
+  for (int sweep = 0; sweep < a.max_sweeps; ++sweep) {
+    for (int r = 0; r < a.nblk - 1; ++r) {
+      for (int it = blockIdx.x; it < a.nb * a.npair; it += nbk)
+        dev_jac_solve(a.A, a.np, a.nblk, r, a.Th, it / a.npair, it % a.npair, jsm);
+      grid_barrier(a.bar);
+      const int per = a.npair * a.chunks;
+      for (int it = blockIdx.x; it < a.nb * per; it += nbk)
+        dev_jac_cols(a.A, a.V, a.np, a.nblk, r, a.Th, it / per, (it % per) / a.chunks, (it % per) % a.chunks, jsm);
+      grid_barrier(a.bar);
+      for (int it = blockIdx.x; it < a.nb * per; it += nbk)
+        dev_jac_rows(a.A, a.np, a.nblk, r, a.Th, it / per, (it % per) / a.chunks, (it % per) % a.chunks, jsm);
+      grid_barrier(a.bar);
+    }
+    // off-diagonal and total Frobenius mass of every matrix
+    double* nm = a.norms + int64_t(sweep) * a.nb * 2;
+    const int64_t tot = int64_t(a.np) * a.np;
+    for (int b = 0; b < a.nb; ++b) {
+      double off = 0.0, all = 0.0;
+      for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < tot; e += int64_t(nbk) * blockDim.x) {
+        const double v = a.A[int64_t(b) * tot + e];
+        all += v * v;
+        if (e / a.np != e % a.np) off += v * v;
+      }
+      for (int m = 16; m; m >>= 1) {
+        off += __shfl_xor_sync(0xffffffffu, off, m);
+        all += __shfl_xor_sync(0xffffffffu, all, m);
+      }
+      if ((threadIdx.x & 31) == 0 && (off != 0.0 || all != 0.0)) {
+        atomicAdd(&nm[2 * b], off);
+        atomicAdd(&nm[2 * b + 1], all);
+      }
+    }
+    grid_barrier(a.bar);
+    if (threadIdx.x == 0) {
+      int done = 1;
+      for (int b = 0; b < a.nb; ++b) {
+        const double off = *reinterpret_cast<volatile double*>(&nm[2 * b]);
+        const double all = *reinterpret_cast<volatile double*>(&nm[2 * b + 1]);
+        if (off > a.tol * a.tol * all) done = 0;
+      }
+      s_done = done;
+    }
+    __syncthreads();
+    if (s_done) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) *a.sweeps_done = sweep + 1;
+      break;
+    }
+    if (sweep + 1 == a.max_sweeps && blockIdx.x == 0 && threadIdx.x == 0) *a.sweeps_done = sweep + 1;
   }
 }
 
@@ -552,7 +672,23 @@ int grid_1d(int64_t n, int per = 256) {
 size_t chol_scratch_bytes(int nb, int n) {
   const int np = rup(n, NB);
   return 2 * align_up(size_t(nb) * np * np * 8, 256) + align_up(size_t(nb) * 8, 256) +
-         align_up(size_t(nb) * np * 8, 256) + align_up(size_t(nb) * 4, 256);
+         align_up(size_t(nb) * np * 8, 256) + align_up(size_t(nb) * 4, 256) + 256;
+}
+
+template <typename K, typename A>
+jolt_status launch_coop(K kernel, const A& args, int smem, cudaStream_t st) {
+  static_assert(sizeof(A) < 4000, "kernel arguments must fit the parameter space");
+  int dev = 0, sms = 0, per = 0;
+  JOLT_CUDA_TRY(cudaGetDevice(&dev));
+  JOLT_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  JOLT_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  JOLT_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, 256, smem));
+  if (per < 1) return JOLT_ERR_CUDA;
+  A local = args;
+  void* params[] = {&local};
+  JOLT_CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kernel), dim3(sms * per), dim3(256), params,
+                                            size_t(smem), st));
+  return JOLT_OK;
 }
 
 jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shift_rel,
@@ -561,36 +697,20 @@ jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shi
   if (nb < 1 || n < 1) return JOLT_OK;
   const int np = rup(n, NB), P = np / NB;
   CholScratch s = chol_carve(scratch, nb, n);
-  k_maxdiag<<<nb, 256, 0, st>>>(G, ld_g, n, s.mdiag);
-  k_ratio_init<<<1, 256, 0, st>>>(s.ratio, nb);
-  k_chol_init<<<dim3(P, P, nb), 256, 0, st>>>(G, ld_g, n, np, shift_rel, s.mdiag, s.Gd, s.Xd, s.diag0);
-  const int sm2 = 2 * NB * (NB + 1) * 8, sm3 = 3 * NB * (NB + 1) * 8, sm4 = 4 * NB * (NB + 1) * 8;
-  static bool attr = false;
-  if (!attr) {
-    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_chol_diag, cudaFuncAttributeMaxDynamicSharedMemorySize, sm2));
-    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_chol_panel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm3));
-    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_chol_update, cudaFuncAttributeMaxDynamicSharedMemorySize, sm3));
-    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_trinv, cudaFuncAttributeMaxDynamicSharedMemorySize, sm4));
-    attr = true;
-  }
-  for (int p = 0; p < P; ++p) {
-    k_chol_diag<<<nb, 256, sm2, st>>>(s.Gd, s.Xd, np, p, s.diag0, s.ratio);
-    if (p + 1 < P) {
-      k_chol_panel<<<dim3(P - p - 1, nb), 256, sm3, st>>>(s.Gd, s.Xd, np, p);
-      const int npairs = (P - p - 1) * (P - p) / 2;
-      k_chol_update<<<dim3(npairs, nb), 256, sm3, st>>>(s.Gd, np, P, p);
-    }
-  }
-  for (int d = 1; d < P; ++d) k_trinv<<<dim3(P - d, nb), 256, sm4, st>>>(s.Gd, s.Xd, np, d);
-  k_rinv_out<<<dim3(grid_1d(int64_t(n) * n), nb), 256, 0, st>>>(s.Xd, np, n, rinv_hi, rinv_lo);
-  JOLT_CUDA_TRY(cudaGetLastError());
-  (void)err;
+  JOLT_CUDA_TRY(cudaMemsetAsync(s.bar, 0, 2 * sizeof(unsigned int), st));
+  CholArgs a;
+  a.G = G; a.ldg = ld_g; a.n = n; a.np = np; a.P = P; a.nb = nb; a.shift_rel = shift_rel;
+  a.Gd = s.Gd; a.Xd = s.Xd; a.md = s.mdiag; a.diag0 = s.diag0; a.ratio = s.ratio;
+  a.hi = rinv_hi; a.lo = rinv_lo;
+  a.bar = GridBar{s.bar, s.bar + 1, err};
+  jolt_status r = launch_coop(k_chol_coop, a, 4 * NB * (NB + 1) * 8, st);
+  if (r) return r;
   if (min_ratio) {
-    std::vector<float> r(nb);
-    JOLT_CUDA_TRY(cudaMemcpyAsync(r.data(), s.ratio, sizeof(float) * nb, cudaMemcpyDeviceToHost, st));
+    std::vector<float> h(nb);
+    JOLT_CUDA_TRY(cudaMemcpyAsync(h.data(), s.ratio, sizeof(float) * nb, cudaMemcpyDeviceToHost, st));
     JOLT_CUDA_TRY(cudaStreamSynchronize(st));
     float m = 1.f;
-    for (float v : r) m = std::min(m, v);
+    for (float v : h) m = std::min(m, v);
     *min_ratio = m;
   }
   return JOLT_OK;
@@ -599,7 +719,7 @@ jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shi
 size_t jacobi_scratch_bytes(int nb, int n) {
   const int np = rup(n, JS), npair = np / JS;
   return 2 * align_up(size_t(nb) * np * np * 8, 256) + align_up(size_t(nb) * npair * JS * JS * 8, 256) +
-         align_up(size_t(nb) * 16, 256) + align_up(size_t(nb) * np * 4, 256);
+         align_up(size_t(kJacMaxSweeps) * nb * 16, 256) + align_up(size_t(nb) * np * 4, 256) + 512;
 }
 
 template <typename TA, typename TO>
@@ -608,35 +728,21 @@ jolt_status jacobi_impl(const TA* A, int64_t ld_a, int nb, int n, TO* evals, TO*
   if (nb < 1 || n < 1) return JOLT_OK;
   const int np = rup(n, JS), nblk = np / JW, npair = nblk / 2, chunks = np / JS;
   JacScratch s = jac_carve(scratch, nb, n);
-  const int tsm = 2 * JS * (JS + 1) * 8;
-  static bool attr = false;
-  if (!attr) {
-    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_jac_solve, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm));
-    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_jac_cols, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm));
-    JOLT_CUDA_TRY(cudaFuncSetAttribute(k_jac_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm));
-    attr = true;
-  }
   k_jac_init<<<dim3(grid_1d(int64_t(np) * np), nb), 256, 0, st>>>(A, ld_a, n, np, s.A, s.V);
-  std::vector<double> h(2 * nb);
-  for (int sweep = 0; sweep < max_sweeps; ++sweep) {
-    for (int r = 0; r < nblk - 1; ++r) {
-      k_jac_solve<<<dim3(npair, nb), 256, tsm, st>>>(s.A, np, nblk, r, s.Th);
-      k_jac_cols<<<dim3(npair, chunks, nb), 256, tsm, st>>>(s.A, s.V, np, nblk, r, s.Th);
-      k_jac_rows<<<dim3(npair, chunks, nb), 256, tsm, st>>>(s.A, np, nblk, r, s.Th);
-    }
-    JOLT_CUDA_TRY(cudaMemsetAsync(s.norms, 0, sizeof(double) * 2 * nb, st));
-    k_jac_norms<<<dim3(grid_1d(int64_t(np) * np), nb), 256, 0, st>>>(s.A, np, s.norms);
-    JOLT_CUDA_TRY(cudaMemcpyAsync(h.data(), s.norms, sizeof(double) * 2 * nb, cudaMemcpyDeviceToHost, st));
-    JOLT_CUDA_TRY(cudaStreamSynchronize(st));
-    bool done = true;
-    for (int b = 0; b < nb; ++b)
-      if (h[2 * b] > tol * tol * h[2 * b + 1]) done = false;
-    if (done) break;
-  }
+  JOLT_CUDA_TRY(cudaMemsetAsync(s.norms, 0, size_t(kJacMaxSweeps) * nb * 16, st));
+  JOLT_CUDA_TRY(cudaMemsetAsync(s.bar, 0, 2 * sizeof(unsigned int), st));
+  JacArgs a;
+  a.A = s.A; a.V = s.V; a.Th = s.Th; a.norms = s.norms;
+  a.np = np; a.nblk = nblk; a.npair = npair; a.chunks = chunks; a.nb = nb;
+  a.max_sweeps = std::min(max_sweeps, kJacMaxSweeps);
+  a.tol = tol;
+  a.sweeps_done = s.sweeps;
+  a.bar = GridBar{s.bar, s.bar + 1, err};
+  jolt_status r = launch_coop(k_jac_coop, a, 2 * JS * (JS + 1) * 8, st);
+  if (r) return r;
   k_jac_sort<<<dim3((n + 255) / 256, nb), 256, 0, st>>>(s.A, np, n, evals, s.perm);
   k_jac_out<<<dim3(grid_1d(int64_t(n) * n), nb), 256, 0, st>>>(s.V, np, n, s.perm, evecs);
   JOLT_CUDA_TRY(cudaGetLastError());
-  (void)err;
   return JOLT_OK;
 }
 
