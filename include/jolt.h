@@ -174,7 +174,10 @@ jolt_status jolt_compress(const jolt_shape* shape, const void* k, const void* v,
  * tile and rotated by RoPE at position pos_offset + t before the dot product, cos/sin computed in
  * the kernel from inv_freq ("JoLT: совместное распределение ранга и бит в KV-кэше", section on
  * building cos/sin in the kernel).
- *   cache        device, filled by jolt_compress (or laid out by jolt_cache_layout)
+ * bf16 I/O and factors with d_h = 128 and g_q <= 16 run on the tensor-core path (tcgen05 key
+ * rebuild and value GEMMs, fp32 accumulation); other shapes on the CUDA-core split-T path.
+ *   cache        device, filled by jolt_compress (or laid out by jolt_cache_layout); on the
+ *                tensor-core path it must be 16-byte aligned (JOLT_ERR_INVALID_ARG otherwise)
  *   layer_begin, n_layers_call: layers [layer_begin, layer_begin + n_layers_call)
  *   q            device [B][n_layers_call][n_q][d_h] io dtype
  *   out          device [B][n_layers_call][n_q][d_h] io dtype

@@ -19,13 +19,16 @@ int choose_splits(const jolt_shape& s, int Lc) {
   return S;
 }
 
+// Workspace of one call: header, prologue outputs, then either the CUDA-core path's split
+// partials (ws_Bh, part) or the tensor-core path's buffers (tc).
 struct DecodeWs {
-  size_t qrot, qsum, P, Bh, part, total;
+  size_t qrot, qsum, P, Bh, part, tc, total;
 };
 
 DecodeWs decode_ws_layout(const jolt_shape& s, int Lc, int S) {
   DecodeWs w{};
   const size_t B = s.batch, nq = s.n_q, d = s.d_h, qc = std::max(s.q_cap, 16);
+  const bool tc = decode_tc_supported(s);
   size_t off = sizeof(WsHeader);
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -35,8 +38,9 @@ DecodeWs decode_ws_layout(const jolt_shape& s, int Lc, int S) {
   w.qrot = take(B * Lc * nq * d * 4);
   w.qsum = take(B * Lc * nq * 4);
   w.P = take(s.keys_pre_rope ? 0 : B * Lc * nq * qc * 4);
-  w.Bh = take(s.keys_pre_rope ? B * Lc * s.n_kv * qc * d * 4 : 0);
-  w.part = take(B * Lc * nq * size_t(S) * (2 + qc + d) * 4);
+  w.Bh = take(s.keys_pre_rope && !tc ? B * Lc * s.n_kv * qc * d * 4 : 0);
+  w.part = take(tc ? 0 : B * Lc * nq * size_t(S) * (2 + qc + d) * 4);
+  w.tc = take(tc ? decode_tc_ws_bytes(s, Lc) : 0);
   w.total = off;
   return w;
 }
@@ -66,6 +70,8 @@ extern "C" jolt_status jolt_decode_attn(const jolt_shape* shape, const jolt_cell
   const int nc = n_cells(s);
   for (int c = 0; c < nc; ++c)
     if (!choice_ok(s, choices[c])) return JOLT_ERR_INVALID_ARG;
+  // the tensor-core path reads the cache with 16-byte vector loads and TMA
+  if (decode_tc_supported(s) && reinterpret_cast<uintptr_t>(cache) % 16) return JOLT_ERR_INVALID_ARG;
   const int Lc = n_layers_call;
   const int S = choose_splits(s, Lc);
   const DecodeWs wl = decode_ws_layout(s, Lc, S);
@@ -158,7 +164,27 @@ extern "C" jolt_status jolt_decode_attn(const jolt_shape* shape, const jolt_cell
         ab += 2.0 * s.n_q * s.d_h * iob;
       }
     pc.alg_bytes = ab;
-    jolt_status st_ = launch_decode_simt(pc, st);
+    jolt_status st_;
+    if (decode_tc_supported(s)) {
+      TcCellView views[kMaxCallCells];
+      const uint8_t* cb = static_cast<const uint8_t*>(cache);
+      for (int i = 0; i < 2 * nb * Gc; ++i) {
+        const CellRef& c = pc.cells[i];
+        const SegOffsets so = seg_offsets(s.T, s.d_h, s.layers_per_group, s.n_kv, 2, c.r_T, c.r_d, c.b);
+        const uint8_t* base = cb + c.offset;
+        views[i].Ut = reinterpret_cast<const __nv_bfloat16*>(base + so.ut);
+        views[i].Ud = reinterpret_cast<const __nv_bfloat16*>(base + so.ud);
+        views[i].G = reinterpret_cast<const __nv_bfloat16*>(base + so.g);
+        views[i].codes = base + so.codes;
+        views[i].sz = reinterpret_cast<const __half2*>(base + so.sz);
+        views[i].r_T = c.r_T;
+        views[i].r_d = c.r_d;
+        views[i].bits = c.b;
+      }
+      st_ = launch_decode_tc(pc, views, wsb + wl.tc, s, st);
+    } else {
+      st_ = launch_decode_simt(pc, st);
+    }
     if (st_ != JOLT_OK) return st_;
   }
   return JOLT_OK;

@@ -28,5 +28,24 @@ struct DecodeParams {
 };
 
 jolt_status launch_decode_simt(const DecodeParams& p, cudaStream_t st);
+// First prologue kernel of both paths: q_rot = R q, qsum = sum(q_rot) and (non-RoPE keys) P.
+jolt_status launch_decode_prologue_q(const DecodeParams& p, cudaStream_t st);
+
+// One stored cell as device pointers (bf16 factors), for the tensor-core path.
+struct TcCellView {
+  const __nv_bfloat16* Ut;  // [T][r_T]
+  const __nv_bfloat16* Ud;  // [d_h][r_d]
+  const __nv_bfloat16* G;   // [L_g][n_kv][r_T][r_d]
+  const uint8_t* codes;     // [L_g][n_kv][T][d_h * b / 8]
+  const __half2* sz;        // [L_g][n_kv][T] (scale, zero)
+  int r_T, r_d, bits;
+};
+
+// Tensor-core decode (bf16 I/O and factors, d_h = 128, g_q <= 16).
+bool decode_tc_supported(const jolt_shape& s);
+size_t decode_tc_ws_bytes(const jolt_shape& s, int Lc);
+// views: (b * Gc + (g - g_first)) * 2 + kv for the call's batch range; tcws: the path's workspace.
+jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uint8_t* tcws,
+                             const jolt_shape& s, cudaStream_t st);
 
 }  // namespace jolt

@@ -388,14 +388,21 @@ size_t decode_simt_main_smem(const DecodeParams& p) {
   return f * sizeof(float);
 }
 
+jolt_status launch_decode_prologue_q(const DecodeParams& p, cudaStream_t st) {
+  const dim3 gq_grid(p.n_q, p.Lc, p.B);
+  if (p.d_h == 64) k_prologue_q<2><<<gq_grid, 128, 0, st>>>(p);
+  else k_prologue_q<4><<<gq_grid, 128, 0, st>>>(p);
+  JOLT_CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
 jolt_status launch_decode_simt(const DecodeParams& p, cudaStream_t st) {
   if (p.gq > kMaxGq) return JOLT_ERR_INVALID_ARG;
   const dim3 gq_grid(p.n_q, p.Lc, p.B);
   {
     StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
-    if (p.d_h == 64) k_prologue_q<2><<<gq_grid, 128, 0, st>>>(p);
-    else k_prologue_q<4><<<gq_grid, 128, 0, st>>>(p);
-    JOLT_CUDA_TRY(cudaGetLastError());
+    jolt_status r = launch_decode_prologue_q(p, st);
+    if (r) return r;
     if (p.pre_rope) {
       k_prologue_bh<<<dim3(p.n_kv, p.Lc, p.B), 256, 0, st>>>(p);
       JOLT_CUDA_TRY(cudaGetLastError());

@@ -1,0 +1,771 @@
+// Decode attention over the stored factors with tensor cores (bf16 caches, d_h = 128).
+//
+// The attention of one (sequence, layer group) runs as a short pipeline over the group's layers:
+//   keys     : pre-RoPE keys — k_keys_tc rebuilds each 128-token tile's keys K = U_T^K B_h for every
+//              (layer, KV head) of the group on tcgen05 (B_h = G^K_h U_d^K^T as fp32 split into
+//              bf16 hi + lo terms, fp32 accumulation in TMEM); its epilogue (one thread per token)
+//              adds the inverse-rotated dequantised residual, applies RoPE at the token's position
+//              and writes q . k for the KV head's query heads.
+//              Non-RoPE keys — S = P U_T^K^T on the tcgen05 GEMM (P = G^K U_d^K^T q, hi + lo), then
+//              k_scores_res adds scale * (codes . R q) + zero * sum(R q) per (token, query head).
+//   softmax  : per (layer, query head) row: m = max s, P~ = bf16(exp(s - m)), l = sum P~
+//   values   : W = P~ U_T^V on the tcgen05 GEMM (split-K, atomic fp32) and, on CUDA cores,
+//              acc = sum_t P~_t deq(codes^V_t) in the rotated domain
+//   finalize : out = (U_d^V (G^V_h^T W) + R^T acc) / l,  lse = m + log l
+// Rows of scores and probabilities go through the workspace (n_q * T * 6 bytes per layer, written
+// once and read twice); everything else the attention reads is the compressed cache itself.
+// Method: the JoLT pages' decode-time attention over the stored factors (scores from G q-hat and
+// the U_T rows plus the rotated-query residual term; values from the softmax-weighted U_T, the
+// core and U_d plus the inverse-rotated residual; RoPE re-applied per token for pre-RoPE keys).
+#include <algorithm>
+#include <cstring>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "gemm_tc.cuh"
+#include "pack.cuh"
+#include "sm100.cuh"
+#include "stats.h"
+
+namespace jolt {
+
+namespace {
+
+constexpr int kD = 128;              // head dimension this path serves
+constexpr int kBM = 128, kBK = 64;   // token tile, rank chunk
+constexpr int kMaxG = 16;            // query heads per KV head
+constexpr int kABytes = kBM * kBK * 2;
+constexpr int kBBytes = kBK * kD * 2;
+
+template <int NT>
+struct KeysCfg {
+  static constexpr int kStages = NT == 1 ? 4 : 3;
+  static constexpr int kStageBytes = kABytes + NT * kBBytes;
+  static constexpr int kQsBytes = 2 * kMaxG * kD * 4;      // queries of two pairs, fp32
+  static constexpr int kRopeBytes = kD / 2 * kBM * 8;      // (cos, sin) per frequency and token
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + kQsBytes + kRopeBytes + kD * 4 + 256;
+};
+
+struct KeysMaps {
+  CUtensorMap a;       // U_T^K [T][r_T], K-major, box 64 x 128
+  CUtensorMap b[2];    // B_h hi / lo [pairs][r_T][128], MN-major, box 64 x 64
+};
+
+struct KeysArgs {
+  int T, nkb, n_kv, gq, n_q, nl;
+  uint64_t rot_seed;
+  float attn_scale;
+  int pos0;
+  float rope_scaling;
+  const uint8_t* codes;    // residual codes of layer ll0, head 0: rows (li * n_kv + h) * T + t
+  const __half2* sz;       // scale/zero pairs, same rows
+  const __nv_bfloat16* q;  // queries of (b, li0): [nl][n_q][128]
+  const float* inv_freq;   // [64]
+  float* scores;           // [nl][n_q][T]
+  int32_t* err;
+};
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Residual row of one token: 128 codes of BITS bits (little-endian bit stream) as floats.
+template <int BITS>
+__device__ __forceinline__ void load_codes(const uint8_t* row, float (&v)[kD]) {
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+  uint32_t w[4 * BITS + 1];
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+#pragma unroll
+  for (int i = 0; i < BITS; ++i) {
+    const uint4 x = __ldg(r4 + i);
+    w[4 * i + 0] = x.x;
+    w[4 * i + 1] = x.y;
+    w[4 * i + 2] = x.z;
+    w[4 * i + 3] = x.w;
+  }
+#pragma unroll
+  for (int j = 0; j < kD; ++j) v[j] = float((w[(j * BITS) >> 5] >> ((j * BITS) & 31)) & mask);
+}
+
+// Same row dequantised: code * scale + zero (fp32 fused multiply-add).
+template <int BITS>
+__device__ __forceinline__ void load_dequant(const uint8_t* row, float sc, float zr, float (&v)[kD]) {
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+  uint32_t w[4 * BITS + 1];
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+#pragma unroll
+  for (int i = 0; i < BITS; ++i) {
+    const uint4 x = __ldg(r4 + i);
+    w[4 * i + 0] = x.x;
+    w[4 * i + 1] = x.y;
+    w[4 * i + 2] = x.z;
+    w[4 * i + 3] = x.w;
+  }
+#pragma unroll
+  for (int j = 0; j < kD; ++j) v[j] = dequant((w[(j * BITS) >> 5] >> ((j * BITS) & 31)) & mask, sc, zr);
+}
+
+__device__ __forceinline__ void fwht128(float (&v)[kD]) {
+#pragma unroll
+  for (int s = 1; s < kD; s <<= 1) {
+#pragma unroll
+    for (int i = 0; i < kD; ++i) {
+      if ((i & s) == 0) {
+        const float a = v[i], c = v[i + s];
+        v[i] = a + c;
+        v[i + s] = a - c;
+      }
+    }
+  }
+}
+
+// grid.x = token tiles; 192 threads: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner),
+// warps 2..5 epilogue (warp w reads TMEM lanes 32 * (w % 4) .. +31, i.e. token rows of the tile).
+template <int BITS, int NT>
+__global__ void __launch_bounds__(192, 1) k_keys_tc(const __grid_constant__ KeysMaps maps, const KeysArgs p) {
+  using C = KeysCfg<NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* qs = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);  // [2][kMaxG][kD]
+  float2* rope = reinterpret_cast<float2*>(qs + 2 * kMaxG * kD);            // [64][kBM]
+  float* sgn = reinterpret_cast<float*>(rope + kD / 2 * kBM);                 // [kD]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sgn + kD);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 5);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * kBM;
+  const int npairs = p.nl * p.n_kv;
+  const bool fac = p.nkb > 0;
+
+  const uint32_t bar0 = sm100::smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      sm100::mbar_init(full_bar(s), 1);
+      sm100::mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      sm100::mbar_init(tfull_bar(b), 1);
+      sm100::mbar_init(tempty_bar(b), 128);
+    }
+    sm100::mbar_init(drain_bar, 1);
+    sm100::fence_mbar_init();
+    if (fac) {
+      sm100::prefetch_tmap(&maps.a);
+      for (int t = 0; t < NT; ++t) sm100::prefetch_tmap(&maps.b[t]);
+    }
+  }
+  if (threadIdx.x < kD) sgn[threadIdx.x] = rsqrtf(float(kD)) * rot_sign(p.rot_seed, threadIdx.x);
+  // RoPE of the tile's tokens: cos / sin of (pos0 + t) * inv_freq[f], angle reduced mod 2 pi in
+  // fp64, times the attention scaling
+  for (int e = threadIdx.x; e < kD / 2 * kBM; e += blockDim.x) {
+    const int f = e / kBM, tt = e % kBM;
+    const double ang = double(p.pos0 + t0 + tt) * double(p.inv_freq[f]);
+    const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+    float sn, cs;
+    sincosf(float(red), &sn, &cs);
+    rope[e] = make_float2(cs * p.rope_scaling, sn * p.rope_scaling);
+  }
+  if (warp == 1) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), 256);
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sbase = sm100::smem_u32(smem);
+
+  if (warp == 0) {
+    if (lane == 0 && fac) {
+      // ---- TMA producer: per (layer, head) pair, the U_T tile chunk and the B_h chunk(s) ----
+      int it = 0;
+      bool ok = true;
+      for (int pr = 0; pr < npairs && ok; ++pr) {
+        for (int kb = 0; kb < p.nkb; ++kb) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1;
+          if (!sm100::mbar_wait(empty_bar(s), ph ^ 1, p.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + s * C::kStageBytes;
+          sm100::mbar_expect_tx(full_bar(s), C::kStageBytes);
+          sm100::tma_load_3d(sa, &maps.a, full_bar(s), kb * kBK, t0, 0);
+#pragma unroll
+          for (int t = 0; t < NT; ++t)
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              sm100::tma_load_3d(sa + kABytes + t * kBBytes + c * 8192, &maps.b[t], full_bar(s), c * 64, kb * kBK, pr);
+          ++it;
+        }
+      }
+      // wait (bounded) for the copies still in flight before the block may exit
+      for (int i = max(0, it - C::kStages); i < it; ++i)
+        sm100::mbar_wait(full_bar(i % C::kStages), (i / C::kStages) & 1, p.err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && fac) {
+      // ---- MMA issuer: D[bi] = sum_k U_T[t][k] (B_hi + B_lo)[k][:] ----
+      constexpr uint32_t idesc = sm100::idesc_bf16_f32(kBM, kD, 0, 1);
+      int it = 0;
+      bool ok = true;
+      for (int pr = 0; pr < npairs && ok; ++pr) {
+        const int bi = pr & 1;
+        if (!sm100::mbar_wait(tempty_bar(bi), ((pr >> 1) & 1) ^ 1, p.err)) break;
+        sm100::tc_fence_after();
+        const uint32_t dt = tmem + bi * kD;
+        for (int kb = 0; kb < p.nkb; ++kb, ++it) {
+          const int s = it % C::kStages;
+          if (!sm100::mbar_wait(full_bar(s), (it / C::kStages) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+          const uint32_t sa = sbase + s * C::kStageBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = sm100::smem_desc_sw128(sa + kk * 32, 16, 1024);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+              const uint64_t bd = sm100::smem_desc_sw128(sa + kABytes + t * kBBytes + kk * 2048, 8192, 1024);
+              sm100::mma_bf16(dt, ad, bd, idesc, (kb > 0 || kk > 0 || t > 0) ? 1u : 0u);
+            }
+          }
+          sm100::mma_commit(empty_bar(s));
+        }
+        if (ok) sm100::mma_commit(tfull_bar(bi));
+      }
+      // every MMA this thread issued has completed before TMEM is released
+      sm100::mma_commit(drain_bar);
+      sm100::mbar_wait(drain_bar, 0, p.err);
+    }
+  } else {
+    // ---- epilogue: thread = token row of the tile ----
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int et = threadIdx.x - 64;
+    const int t = t0 + row;
+    const bool valid = t < p.T;
+    bool live = true;
+    for (int pr = 0; pr < npairs; ++pr) {
+      const int li = pr / p.n_kv, h = pr % p.n_kv, bi = pr & 1;
+      float* qb = qs + bi * kMaxG * kD;
+      const __nv_bfloat16* qsrc = p.q + (int64_t(li) * p.n_q + int64_t(h) * p.gq) * kD;
+      for (int e = et; e < p.gq * kD; e += 128) qb[e] = __bfloat162float(qsrc[e]);
+      epi_bar();
+      float v[kD];
+      if (BITS > 0 && valid) {
+        const int64_t rr = (int64_t(li) * p.n_kv + h) * p.T + t;
+        const __half2 szv = p.sz[rr];
+        load_dequant<BITS>(p.codes + rr * (kD * BITS / 8), __low2float(szv), __high2float(szv), v);
+        fwht128(v);
+#pragma unroll
+        for (int j = 0; j < kD; ++j) v[j] *= sgn[j];
+      } else {
+#pragma unroll
+        for (int j = 0; j < kD; ++j) v[j] = 0.f;
+      }
+      if (fac) {
+        if (live) live = sm100::mbar_wait(tfull_bar(bi), (pr >> 1) & 1, p.err);
+        sm100::tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kD / 16; ++c) {
+          uint32_t r[16];
+          sm100::tmem_ld16(tmem + bi * kD + c * 16 + (uint32_t(quarter * 32) << 16), r);
+          sm100::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[c * 16 + j] += __uint_as_float(r[j]);
+        }
+        sm100::tc_fence_before();
+        sm100::mbar_arrive(tempty_bar(bi));
+      }
+      if (valid && live) {
+#pragma unroll
+        for (int f = 0; f < kD / 2; ++f) {
+          const float2 csn = rope[f * kBM + row];
+          const float x1 = v[f], x2 = v[f + kD / 2];
+          v[f] = x1 * csn.x - x2 * csn.y;
+          v[f + kD / 2] = x2 * csn.x + x1 * csn.y;
+        }
+        float* out = p.scores + (int64_t(li) * p.n_q + int64_t(h) * p.gq) * p.T + t;
+#pragma unroll 1
+        for (int g = 0; g < p.gq; ++g) {
+          const float4* qg = reinterpret_cast<const float4*>(qb + g * kD);
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+          for (int j = 0; j < kD; j += 4) {
+            const float4 qq = qg[j >> 2];
+            a0 = fmaf(v[j], qq.x, a0);
+            a1 = fmaf(v[j + 1], qq.y, a1);
+            a2 = fmaf(v[j + 2], qq.z, a2);
+            a3 = fmaf(v[j + 3], qq.w, a3);
+          }
+          out[int64_t(g) * p.T] = ((a0 + a1) + (a2 + a3)) * p.attn_scale;
+        }
+      }
+    }
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) sm100::tmem_dealloc(tmem, 256);
+}
+
+// ---- CUDA-core stages -------------------------------------------------------------------------
+
+// fp32 -> bf16 hi + lo parts (hi = rn(x), lo = rn(x - hi)).
+__global__ void k_split_hilo(const float* __restrict__ x, int64_t n, __nv_bfloat16* __restrict__ hi,
+                             __nv_bfloat16* __restrict__ lo) {
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
+    const float v = x[e];
+    const __nv_bfloat16 hh = __float2bfloat16_rn(v);
+    hi[e] = hh;
+    lo[e] = __float2bfloat16_rn(v - __bfloat162float(hh));
+  }
+}
+
+struct ResArgs {
+  int T, n_kv, gq, n_q, has_fac;
+  float attn_scale;
+  const uint8_t* codes;   // rows (li * n_kv + h) * T + t
+  const __half2* sz;
+  const float* qrot;      // [nl][n_q][128]
+  const float* qsum;      // [nl][n_q]
+  float* scores;          // [nl][n_q][T]
+};
+
+// Non-RoPE keys: s = (s_fac + scale * (codes . q_rot) + zero * qsum) * attn_scale.
+// grid (token tiles, n_kv, nl), thread = token.
+template <int BITS>
+__global__ void __launch_bounds__(128) k_scores_res(const ResArgs a) {
+  __shared__ float qr[kMaxG][kD];
+  __shared__ float qsm[kMaxG];
+  const int h = blockIdx.y, li = blockIdx.z;
+  const int64_t qrow0 = int64_t(li) * a.n_q + int64_t(h) * a.gq;
+  for (int e = threadIdx.x; e < a.gq * kD; e += blockDim.x) qr[e / kD][e % kD] = a.qrot[qrow0 * kD + e];
+  if (threadIdx.x < a.gq) qsm[threadIdx.x] = a.qsum[qrow0 + threadIdx.x];
+  __syncthreads();
+  const int t = blockIdx.x * 128 + threadIdx.x;
+  if (t >= a.T) return;
+  float c[kD];
+  float sc = 0.f, zr = 0.f;
+  if (BITS > 0) {
+    const int64_t rr = (int64_t(li) * a.n_kv + h) * a.T + t;
+    load_codes<BITS>(a.codes + rr * (kD * BITS / 8), c);
+    const __half2 szv = a.sz[rr];
+    sc = __low2float(szv);
+    zr = __high2float(szv);
+  }
+  float* s = a.scores + qrow0 * a.T + t;
+#pragma unroll 1
+  for (int g = 0; g < a.gq; ++g) {
+    float res = 0.f;
+    if (BITS > 0) {
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int j = 0; j < kD; j += 4) {
+        a0 = fmaf(c[j], qr[g][j], a0);
+        a1 = fmaf(c[j + 1], qr[g][j + 1], a1);
+        a2 = fmaf(c[j + 2], qr[g][j + 2], a2);
+        a3 = fmaf(c[j + 3], qr[g][j + 3], a3);
+      }
+      res = sc * ((a0 + a1) + (a2 + a3)) + zr * qsm[g];
+    }
+    const float f = a.has_fac ? s[int64_t(g) * a.T] : 0.f;
+    s[int64_t(g) * a.T] = (f + res) * a.attn_scale;
+  }
+}
+
+// Per row: m = max s, P~ = bf16(exp(s - m)) (row stride ldp), l = sum of the rounded P~.
+__global__ void __launch_bounds__(512) k_softmax_rows(const float* __restrict__ scores, int T, int64_t ldp,
+                                                      float* __restrict__ mrow, float* __restrict__ lrow,
+                                                      __nv_bfloat16* __restrict__ ptil) {
+  const int64_t r = blockIdx.x;
+  const float* s = scores + r * T;
+  __shared__ float red[32];
+  const int nw = blockDim.x >> 5, wid = threadIdx.x >> 5, ln = threadIdx.x & 31;
+  float m = -INFINITY;
+  for (int t = threadIdx.x; t < T; t += blockDim.x) m = fmaxf(m, s[t]);
+  m = warp_max(m);
+  if (ln == 0) red[wid] = m;
+  __syncthreads();
+  if (wid == 0) {
+    float x = ln < nw ? red[ln] : -INFINITY;
+    x = warp_max(x);
+    if (ln == 0) red[0] = x;
+  }
+  __syncthreads();
+  m = red[0];
+  __syncthreads();
+  float l = 0.f;
+  __nv_bfloat16* pr = ptil + r * ldp;
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const __nv_bfloat16 e = __float2bfloat16_rn(__expf(s[t] - m));
+    pr[t] = e;
+    l += __bfloat162float(e);
+  }
+  l = warp_sum(l);
+  if (ln == 0) red[wid] = l;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float x = 0.f;
+    for (int i = 0; i < nw; ++i) x += red[i];
+    mrow[r] = m;
+    lrow[r] = x;
+  }
+}
+
+struct ValArgs {
+  int T, n_kv, gq, n_q, bits, chunk;
+  int64_t ldp;
+  const uint8_t* codes;       // value residual rows (li * n_kv + h) * T + t
+  const __half2* sz;
+  const __nv_bfloat16* ptil;  // [nl][n_q][ldp]
+  float* acc;                 // [nl][n_q][128], rotated domain
+};
+
+// acc[h'][j] += sum_t P~[h'][t] deq(code_t[j]). grid (token chunks, n_kv, nl); thread = feature j.
+__global__ void __launch_bounds__(128) k_values_res(const ValArgs a) {
+  __shared__ float pr[kMaxG][128];
+  __shared__ float2 szs[128];
+  const int h = blockIdx.y, li = blockIdx.z, j = threadIdx.x;
+  const int64_t qrow0 = int64_t(li) * a.n_q + int64_t(h) * a.gq;
+  const int nbytes = kD * a.bits / 8;
+  const int64_t rbase = (int64_t(li) * a.n_kv + h) * a.T;
+  float acc[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
+  const int t_beg = blockIdx.x * a.chunk, t_end = min(a.T, t_beg + a.chunk);
+  for (int tb = t_beg; tb < t_end; tb += 128) {
+    const int nt = min(128, t_end - tb);
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.gq * 128; e += blockDim.x) {
+      const int g = e >> 7, tt = e & 127;
+      pr[g][tt] = tt < nt ? __bfloat162float(a.ptil[(qrow0 + g) * a.ldp + tb + tt]) : 0.f;
+    }
+    if (threadIdx.x < nt) {
+      const __half2 szv = a.sz[rbase + tb + threadIdx.x];
+      szs[threadIdx.x] = make_float2(__low2float(szv), __high2float(szv));
+    }
+    __syncthreads();
+    const uint8_t* crow = a.codes + (rbase + tb) * nbytes;
+    for (int tt = 0; tt < nt; ++tt) {
+      const float2 z = szs[tt];
+      const float dv = dequant(unpack_code(crow + int64_t(tt) * nbytes, j, a.bits), z.x, z.y);
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g)
+        if (g < a.gq) acc[g] = fmaf(pr[g][tt], dv, acc[g]);
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g)
+    if (g < a.gq) atomicAdd(&a.acc[(qrow0 + g) * kD + j], acc[g]);
+}
+
+struct FinArgs {
+  int n_kv, gq, n_q, r_T, r_d, bits, q_cap;
+  uint64_t rot_seed;
+  const __nv_bfloat16* G;    // value core of layer ll0: [nl][n_kv][r_T][r_d]
+  const __nv_bfloat16* Ud;   // [128][r_d]
+  const float* W;            // [nl][n_q][q_cap]
+  const float* acc;          // [nl][n_q][128]
+  const float* mrow;         // [nl][n_q]
+  const float* lrow;
+  __nv_bfloat16* out;        // [nl][n_q][128] rows of (b, li0)
+  float* lse;                // [nl][n_q] or null
+};
+
+// grid (n_kv, nl), 128 threads; dynamic smem: w [gq][r_T] + v [gq][r_d] + x [gq][128] floats.
+__global__ void __launch_bounds__(128) k_finalize(const FinArgs a) {
+  extern __shared__ float fs[];
+  const int h = blockIdx.x, li = blockIdx.y, tid = threadIdx.x;
+  const int64_t qrow0 = int64_t(li) * a.n_q + int64_t(h) * a.gq;
+  float* w = fs;
+  float* v = w + a.gq * a.r_T;
+  float* x = v + a.gq * a.r_d;
+  for (int e = tid; e < a.gq * a.r_T; e += blockDim.x) w[e] = a.W[(qrow0 + e / a.r_T) * a.q_cap + e % a.r_T];
+  for (int e = tid; e < a.gq * kD; e += blockDim.x) x[e] = a.bits ? a.acc[qrow0 * kD + e] : 0.f;
+  __syncthreads();
+  // v[g][j] = sum_r G[r][j] w[g][r]
+  if (a.r_T > 0) {
+    const __nv_bfloat16* G = a.G + (int64_t(li) * a.n_kv + h) * a.r_T * a.r_d;
+    for (int j = tid; j < a.r_d; j += blockDim.x) {
+      float acc[kMaxG];
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
+      for (int r = 0; r < a.r_T; ++r) {
+        const float gv = __bfloat162float(G[int64_t(r) * a.r_d + j]);
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < a.gq) acc[g] = fmaf(gv, w[g * a.r_T + r], acc[g]);
+      }
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g)
+        if (g < a.gq) v[g * a.r_d + j] = acc[g];
+    }
+  }
+  // inverse rotation of the residual accumulators, one warp per query head
+  if (a.bits) {
+    const int wid = tid >> 5, ln = tid & 31;
+    for (int g = wid; g < a.gq; g += 4) {
+      float xv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[i] = x[g * kD + ln * 4 + i];
+      warp_unrotate<4>(xv, a.rot_seed, rsqrtf(float(kD)));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) x[g * kD + ln * 4 + i] = xv[i];
+    }
+  }
+  __syncthreads();
+  const int i = tid;
+  for (int g = 0; g < a.gq; ++g) {
+    float o = x[g * kD + i];
+    if (a.r_T > 0) {
+      const __nv_bfloat16* ud = a.Ud + int64_t(i) * a.r_d;
+      for (int jj = 0; jj < a.r_d; ++jj) o = fmaf(__bfloat162float(ud[jj]), v[g * a.r_d + jj], o);
+    }
+    const int64_t qr = qrow0 + g;
+    a.out[qr * kD + i] = __float2bfloat16_rn(o / a.lrow[qr]);
+    if (i == 0 && a.lse) a.lse[qr] = a.mrow[qr] + logf(a.lrow[qr]);
+  }
+}
+
+int grid1(int64_t n) { return int(std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 148 * 16))); }
+
+Operand op(const void* ptr, int major, int64_t inner, int64_t outer, int64_t ld, int64_t batch = 1,
+           int64_t bstride = 0) {
+  Operand o;
+  o.ptr = ptr;
+  o.major = major;
+  o.inner = inner;
+  o.outer = outer;
+  o.outer_stride = ld;
+  o.batch = batch;
+  o.batch_stride = bstride;
+  return o;
+}
+
+// Workspace regions of the tensor-core path (per-group buffers are reused group after group).
+struct TcWs {
+  size_t hl, bh, scores, ptil, ml, W, acc, total;
+};
+
+TcWs tc_layout(const jolt_shape& s, int Lc) {
+  const size_t B = s.batch, nq = s.n_q, T = s.T, qc = std::max(s.q_cap, 16);
+  const size_t nl = std::min(Lc, s.layers_per_group);
+  const size_t Tp = (T + 7) / 8 * 8;
+  TcWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  w.hl = take(s.keys_pre_rope ? 2 * nl * s.n_kv * qc * kD * 2 : 2 * B * Lc * nq * qc * 2);
+  w.bh = take(s.keys_pre_rope ? nl * s.n_kv * qc * kD * 4 : 0);
+  w.scores = take(nl * nq * T * 4);
+  w.ptil = take(nl * nq * Tp * 2);
+  w.ml = take(2 * nl * nq * 4);
+  w.W = take(nl * nq * qc * 4);
+  w.acc = take(nl * nq * kD * 4);
+  w.total = off;
+  return w;
+}
+
+template <int BITS, int NT>
+jolt_status launch_keys(const KeysMaps& maps, const KeysArgs& a, cudaStream_t st) {
+  auto kern = k_keys_tc<BITS, NT>;
+  JOLT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, KeysCfg<NT>::kSmem));
+  const int ntiles = (a.T + kBM - 1) / kBM;
+  kern<<<ntiles, 192, KeysCfg<NT>::kSmem, st>>>(maps, a);
+  JOLT_CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
+template <int NT>
+jolt_status launch_keys_bits(int bits, const KeysMaps& maps, const KeysArgs& a, cudaStream_t st) {
+  switch (bits) {
+    case 0: return launch_keys<0, NT>(maps, a, st);
+    case 2: return launch_keys<2, NT>(maps, a, st);
+    case 4: return launch_keys<4, NT>(maps, a, st);
+    default: return launch_keys<8, NT>(maps, a, st);
+  }
+}
+
+jolt_status launch_scores_res(int bits, const ResArgs& a, int nl, cudaStream_t st) {
+  const dim3 grid((a.T + 127) / 128, a.n_kv, nl);
+  switch (bits) {
+    case 0: k_scores_res<0><<<grid, 128, 0, st>>>(a); break;
+    case 2: k_scores_res<2><<<grid, 128, 0, st>>>(a); break;
+    case 4: k_scores_res<4><<<grid, 128, 0, st>>>(a); break;
+    default: k_scores_res<8><<<grid, 128, 0, st>>>(a); break;
+  }
+  JOLT_CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
+}  // namespace
+
+bool decode_tc_supported(const jolt_shape& s) {
+  return s.io_dtype == JOLT_BF16 && s.factor_dtype == JOLT_BF16 && s.d_h == kD && s.n_q % s.n_kv == 0 &&
+         s.n_q / s.n_kv <= kMaxG;
+}
+
+size_t decode_tc_ws_bytes(const jolt_shape& s, int Lc) { return tc_layout(s, Lc).total; }
+
+jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uint8_t* tcws,
+                             const jolt_shape& s, cudaStream_t st) {
+  const TcWs wl = tc_layout(s, p.Lc);
+  const int T = p.T, nq = p.n_q, qc = p.q_cap, n_kv = p.n_kv, gq = p.gq;
+  const int64_t Tp = (int64_t(T) + 7) / 8 * 8;
+  __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(tcws + wl.hl);
+  float* bh = reinterpret_cast<float*>(tcws + wl.bh);
+  float* scores = reinterpret_cast<float*>(tcws + wl.scores);
+  __nv_bfloat16* ptil = reinterpret_cast<__nv_bfloat16*>(tcws + wl.ptil);
+  float* mrow = reinterpret_cast<float*>(tcws + wl.ml);
+  float* W = reinterpret_cast<float*>(tcws + wl.W);
+  float* acc = reinterpret_cast<float*>(tcws + wl.acc);
+  const int nlmax = std::min(p.Lc, p.Lg);
+  float* lrow = mrow + size_t(nlmax) * nq;
+  jolt_status r;
+
+  // ---- per-call prologue: R q, sum(R q), P (non-RoPE, as hi + lo) ----
+  const size_t nP = size_t(p.B) * p.Lc * nq * qc;
+  {
+    StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
+    if ((r = launch_decode_prologue_q(p, st))) return r;  // records no scope of its own
+    if (!p.pre_rope) {
+      k_split_hilo<<<grid1(int64_t(nP)), 256, 0, st>>>(p.ws_P, int64_t(nP), hl, hl + nP);
+      JOLT_CUDA_TRY(cudaGetLastError());
+    }
+  }
+  const __nv_bfloat16* qall = static_cast<const __nv_bfloat16*>(p.q);
+  __nv_bfloat16* oall = static_cast<__nv_bfloat16*>(p.out);
+
+  for (int b = 0; b < p.B; ++b) {
+    for (int gi = 0; gi < p.Gc; ++gi) {
+      const int g = p.g_first + gi;
+      const int l_lo = std::max(p.layer_begin, g * p.Lg), l_hi = std::min(p.layer_begin + p.Lc, (g + 1) * p.Lg);
+      const int nl = l_hi - l_lo;
+      if (nl <= 0) continue;
+      const int li0 = l_lo - p.layer_begin, ll0 = l_lo - g * p.Lg;
+      const TcCellView& ck = views[(b * p.Gc + gi) * 2 + 0];
+      const TcCellView& cv = views[(b * p.Gc + gi) * 2 + 1];
+      const int rows = nl * nq;
+      const int64_t row0 = (int64_t(b) * p.Lc + li0) * nq;  // first (b, layer, head) row of the call
+      const int64_t res_off = int64_t(ll0) * n_kv * T;       // first residual row of layer ll0
+
+      // ---- scores ----
+      if (p.pre_rope) {
+        KeysMaps maps;
+        std::memset(&maps, 0, sizeof(maps));
+        KeysArgs ka{};
+        ka.nkb = 0;
+        if (ck.r_T > 0) {
+          // B_h = G_h U_d^T for the group's (layer, head) pairs: exact bf16 products, fp32 sums
+          GemmCall gc;
+          gc.M = ck.r_T; gc.N = kD; gc.K = ck.r_d;
+          gc.A[0] = op(ck.G + int64_t(ll0) * n_kv * ck.r_T * ck.r_d, kMajorK, ck.r_d, ck.r_T, ck.r_d, nl * n_kv,
+                       int64_t(ck.r_T) * ck.r_d);
+          gc.B[0] = op(ck.Ud, kMajorK, ck.r_d, kD, ck.r_d);
+          gc.C = bh; gc.ldc = kD; gc.c_batch_stride = int64_t(qc) * kD; gc.batch = nl * n_kv; gc.err = p.err;
+          if ((r = gemm_tc(gc, st))) return r;
+          const int64_t nb = int64_t(nl) * n_kv * qc * kD;
+          {
+            StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
+            k_split_hilo<<<grid1(nb), 256, 0, st>>>(bh, nb, hl, hl + nb);
+            JOLT_CUDA_TRY(cudaGetLastError());
+          }
+          if (!make_tensor_map(&maps.a, op(ck.Ut, kMajorK, ck.r_T, T, ck.r_T), kBM) ||
+              !make_tensor_map(&maps.b[0], op(hl, kMajorMN, kD, ck.r_T, kD, nl * n_kv, int64_t(qc) * kD), kD) ||
+              !make_tensor_map(&maps.b[1], op(hl + nb, kMajorMN, kD, ck.r_T, kD, nl * n_kv, int64_t(qc) * kD), kD))
+            return JOLT_ERR_INVALID_ARG;
+          ka.nkb = (ck.r_T + kBK - 1) / kBK;
+        }
+        ka.T = T; ka.n_kv = n_kv; ka.gq = gq; ka.n_q = nq; ka.nl = nl;
+        ka.rot_seed = p.rot_seed; ka.attn_scale = p.attn_scale;
+        ka.codes = ck.bits ? ck.codes + res_off * (kD * ck.bits / 8) : nullptr;
+        ka.sz = ck.bits ? ck.sz + res_off : nullptr;
+        ka.q = qall + row0 * kD;
+        ka.pos0 = p.pos_offset; ka.rope_scaling = p.rope_scaling; ka.inv_freq = p.inv_freq;
+        ka.scores = scores; ka.err = p.err;
+        // algorithmic work of the launch: the U_T^K rows once, each pair's residual rows; the
+        // tensor flops of the two B_h terms
+        const double kbytes = 2.0 * T * ck.r_T + (ck.bits ? double(nl) * n_kv * T * (kD * ck.bits / 8 + 4) : 0.0);
+        StatScope sc(JOLT_K_DECODE_MAIN, st, 2.0 * 2.0 * T * ck.r_T * kD * nl * n_kv, kbytes);
+        if ((r = launch_keys_bits<2>(ck.bits, maps, ka, st))) return r;
+      } else {
+        if (ck.r_T > 0) {
+          GemmCall gc;
+          gc.M = rows; gc.N = T; gc.K = ck.r_T; gc.n_terms = 2;
+          gc.A[0] = op(hl + row0 * qc, kMajorK, ck.r_T, rows, qc);
+          gc.A[1] = op(hl + nP + row0 * qc, kMajorK, ck.r_T, rows, qc);
+          gc.B[0] = op(ck.Ut, kMajorK, ck.r_T, T, ck.r_T);
+          gc.B[1] = gc.B[0];
+          gc.C = scores; gc.ldc = T; gc.err = p.err;
+          if ((r = gemm_tc(gc, st))) return r;
+        }
+        ResArgs ra{};
+        ra.T = T; ra.n_kv = n_kv; ra.gq = gq; ra.n_q = nq; ra.has_fac = ck.r_T > 0;
+        ra.attn_scale = p.attn_scale;
+        ra.codes = ck.bits ? ck.codes + res_off * (kD * ck.bits / 8) : nullptr;
+        ra.sz = ck.bits ? ck.sz + res_off : nullptr;
+        ra.qrot = p.ws_qrot + row0 * kD;
+        ra.qsum = p.ws_qsum + row0;
+        ra.scores = scores;
+        const double rbytes = ck.bits ? double(nl) * n_kv * T * (kD * ck.bits / 8 + 4) : 0.0;
+        StatScope sc(JOLT_K_DECODE_MAIN, st, 0.0, rbytes);
+        if ((r = launch_scores_res(ck.bits, ra, nl, st))) return r;
+      }
+
+      // ---- softmax rows ----
+      {
+        StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
+        k_softmax_rows<<<rows, 512, 0, st>>>(scores, T, Tp, mrow, lrow, ptil);
+        JOLT_CUDA_TRY(cudaGetLastError());
+      }
+      // ---- values ----
+      JOLT_CUDA_TRY(cudaMemsetAsync(W, 0, size_t(rows) * qc * 4, st));
+      if (cv.bits) JOLT_CUDA_TRY(cudaMemsetAsync(acc, 0, size_t(rows) * kD * 4, st));
+      if (cv.r_T > 0) {
+        GemmCall gc;
+        gc.M = rows; gc.N = cv.r_T; gc.K = T;
+        gc.A[0] = op(ptil, kMajorK, T, rows, Tp);
+        gc.B[0] = op(cv.Ut, kMajorMN, cv.r_T, T, cv.r_T);
+        gc.C = W; gc.ldc = qc; gc.err = p.err;
+        const int64_t tiles = int64_t((rows + 127) / 128) * ((cv.r_T + 127) / 128);
+        const int64_t nkb = (T + 63) / 64;
+        gc.k_split = int(std::max<int64_t>(1, std::min<int64_t>((2 * 148 + tiles - 1) / tiles, nkb / 8)));
+        gc.accumulate = true;
+        if ((r = gemm_tc(gc, st))) return r;
+      }
+      StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
+      if (cv.bits) {
+        ValArgs va{};
+        va.T = T; va.n_kv = n_kv; va.gq = gq; va.n_q = nq; va.bits = cv.bits; va.ldp = Tp;
+        va.chunk = 512;
+        va.codes = cv.codes + res_off * (kD * cv.bits / 8);
+        va.sz = cv.sz + res_off;
+        va.ptil = ptil; va.acc = acc;
+        k_values_res<<<dim3((T + va.chunk - 1) / va.chunk, n_kv, nl), 128, 0, st>>>(va);
+        JOLT_CUDA_TRY(cudaGetLastError());
+      }
+      // ---- finalize ----
+      FinArgs fa{};
+      fa.n_kv = n_kv; fa.gq = gq; fa.n_q = nq; fa.r_T = cv.r_T; fa.r_d = cv.r_d; fa.bits = cv.bits; fa.q_cap = qc;
+      fa.rot_seed = p.rot_seed;
+      fa.G = cv.r_T ? cv.G + int64_t(ll0) * n_kv * cv.r_T * cv.r_d : nullptr;
+      fa.Ud = cv.Ud;
+      fa.W = W; fa.acc = acc; fa.mrow = mrow; fa.lrow = lrow;
+      fa.out = oall + row0 * kD;
+      fa.lse = p.lse ? p.lse + row0 : nullptr;
+      const size_t fsm = size_t(gq) * (cv.r_T + cv.r_d + kD) * 4;
+      JOLT_CUDA_TRY(cudaFuncSetAttribute(k_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, int(std::max<size_t>(fsm, 1))));
+      k_finalize<<<dim3(n_kv, nl), 128, fsm, st>>>(fa);
+      JOLT_CUDA_TRY(cudaGetLastError());
+    }
+  }
+  return JOLT_OK;
+}
+
+}  // namespace jolt

@@ -96,3 +96,27 @@ def test_grouped_pre_rope_gqa4(cuda_ok):
     ch = [(int(rng.integers(1, 6)) * 16, int(rng.integers(2, 9)) * 16, int(rng.choice([2, 4])))
           for _ in range(2 * 1 * 2)]
     run_case(w, ch, 1e-2, layer_calls=[(0, 2), (2, 2)], pos_offset=5)
+
+
+def test_pre_rope_residual_only_keys_and_calls_across_groups(cuda_ok):
+    # key cells with r_T = 0 (residual only), b = 0 and b = 8 cells, ragged T, a call that spans
+    # two groups and starts mid-group
+    w = get_workload("llama8b_64k_b4", n_layers=8, T=450, batch=2)
+    ch = [(0, 0, 4), (32, 32, 0), (64, 128, 8), (48, 16, 2),
+          (16, 16, 0), (0, 0, 8), (96, 64, 4), (128, 96, 4)]
+    run_case(w, ch, 1e-2, layer_calls=[(1, 5), (6, 2), (0, 1)], pos_offset=3)
+
+
+def test_pre_rope_full_token_rank(cuda_ok):
+    # r_T = q_cap = 1024 > any shared-memory-resident tile, T not a multiple of the 128-token tile
+    w = get_workload("llama8b_layer", keys_pre_rope=True, T=1100)
+    run_case(w, uniform(w, (1024, 128, 4)), 1e-2, pos_offset=70000)
+
+
+def test_70b_shape_gqa8_two_row_tiles(cuda_ok):
+    # 64 query heads x 4 layers = 256 rows: two 128-row tiles in the score and value GEMMs
+    for pre in (False, True):
+        w = get_workload("llama70b_128k", n_layers=4, T=640, keys_pre_rope=pre)
+        rng = np.random.default_rng(7)
+        ch = [(int(rng.integers(1, 9)) * 32, 128, int(rng.choice([2, 4]))) for _ in range(2)]
+        run_case(w, ch, 1e-2, layer_calls=[(0, 4)], pos_offset=11)
