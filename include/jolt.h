@@ -260,11 +260,14 @@ jolt_status jolt_decode_attn_noalloc(const jolt_shape* shape, const jolt_cell_ch
  * elapsed device time together with the launch's algorithmic work (FLOPs of a contraction, or
  * bytes a streaming kernel must move). Host-global; not for concurrent use from several threads. */
 typedef enum {
-  JOLT_K_GEMM = 0,          /* tcgen05 contractions of the compressor */
-  JOLT_K_DECODE_MAIN = 1,   /* split-T decode attention over the stored factors */
+  JOLT_K_GEMM = 0,          /* tcgen05 contractions (compressor, and the decode's value GEMMs) */
+  JOLT_K_DECODE_MAIN = 1,   /* decode scores: tcgen05 key rebuild (pre-RoPE) or residual scores,
+                               or the CUDA-core split-T kernel */
   JOLT_K_RESIDUAL = 2,      /* residual rotate + quantise + pack */
-  JOLT_K_DECODE_AUX = 3,    /* decode prologue and split merge */
-  JOLT_K_COUNT = 4
+  JOLT_K_DECODE_AUX = 3,    /* decode prologue, softmax, value residual, finalize, split merge */
+  JOLT_K_CHOL = 4,          /* fp64 Cholesky + triangular inverse (CholeskyQR) */
+  JOLT_K_EIG = 5,           /* fp64 block-Jacobi symmetric eigensolver */
+  JOLT_K_COUNT = 6
 } jolt_kernel_family;
 
 typedef struct {

@@ -37,7 +37,7 @@ class KernelStat(C.Structure):
                 ("flops", C.c_double), ("bytes", C.c_double)]
 
 
-KERNEL_FAMILIES = ["gemm", "decode_main", "residual", "decode_aux"]
+KERNEL_FAMILIES = ["gemm", "decode_main", "residual", "decode_aux", "chol", "eig"]
 
 
 class CellChoice(C.Structure):

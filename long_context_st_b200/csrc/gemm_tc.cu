@@ -40,13 +40,17 @@ struct GemmDev {
   int32_t* err;
 };
 
-template <int BN>
+// MT: 128-row M tiles per CTA; with MT = 2 two accumulators share every B tile (half the B
+// bytes per flop, and each stage covers twice the MMA time).
+template <int BN, int MT>
 struct Cfg {
-  static constexpr int kStages = BN >= 256 ? 4 : 6;
-  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kABytes1 = BM * BK * 2;
+  static constexpr int kABytes = MT * kABytes1;
   static constexpr int kBBytes = BN * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kTmemCols = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
+  static constexpr int kStages = (192 * 1024) / kStageBytes < 6 ? (192 * 1024) / kStageBytes : 6;
+  static constexpr int kCols = MT * BN;
+  static constexpr int kTmemCols = kCols <= 32 ? 32 : (kCols <= 64 ? 64 : (kCols <= 128 ? 128 : (kCols <= 256 ? 256 : 512)));
   static constexpr int kEpiBytes = 4 * 32 * 33 * 4;
   static constexpr int kSmem = 1024 + kStages * kStageBytes + kEpiBytes + 256;
 };
@@ -68,9 +72,9 @@ __device__ __forceinline__ void load_operand(const CUtensorMap* map, int major, 
   }
 }
 
-template <int BN, int AMAJ, int BMAJ>
+template <int BN, int AMAJ, int BMAJ, int MT>
 __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack maps, GemmDev p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, MT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* epi = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
@@ -78,7 +82,7 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM * MT;
   const int z = blockIdx.z / p.k_split, kz = blockIdx.z % p.k_split;
   const int nkb_total = (p.K + BK - 1) / BK;
   const int kb_begin = kz * p.nkb_split;
@@ -121,7 +125,10 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
         const uint32_t sa = smem_base + s * C::kStageBytes;
         const uint32_t sb = sa + C::kABytes;
         sm100::mbar_expect_tx(full_bar(s), C::kStageBytes);
-        load_operand(&maps.a[t], AMAJ, p.a_fold[t], p.a_batch[t], sa, full_bar(s), m0, BM, k0, z);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+          load_operand(&maps.a[t], AMAJ, p.a_fold[t], p.a_batch[t], sa + mt * C::kABytes1, full_bar(s), m0 + mt * BM,
+                       BM, k0, z);
         load_operand(&maps.b[t], BMAJ, p.b_fold[t], p.b_batch[t], sb, full_bar(s), n0, BN, k0, z);
       }
     } else if (warp == 1 && lane == 0) {
@@ -136,12 +143,17 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
         const uint32_t sb = sa + C::kABytes;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          uint64_t ad, bd;
-          if (AMAJ == kMajorK) ad = sm100::smem_desc_sw128(sa + kk * 32, 16, 1024);
-          else ad = sm100::smem_desc_sw128(sa + kk * 2048, 64 * BK * 2, 1024);
+          uint64_t bd;
           if (BMAJ == kMajorK) bd = sm100::smem_desc_sw128(sb + kk * 32, 16, 1024);
           else bd = sm100::smem_desc_sw128(sb + kk * 2048, 64 * BK * 2, 1024);
-          sm100::mma_bf16(tmem, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            const uint32_t sam = sa + mt * C::kABytes1;
+            uint64_t ad;
+            if (AMAJ == kMajorK) ad = sm100::smem_desc_sw128(sam + kk * 32, 16, 1024);
+            else ad = sm100::smem_desc_sw128(sam + kk * 2048, 64 * BK * 2, 1024);
+            sm100::mma_bf16(tmem + mt * BN, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         sm100::mma_commit(empty_bar(s));
       }
@@ -154,9 +166,10 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
     if (ok) {
       float* st = epi + warp * 32 * 33;
       float* Cz = p.C + int64_t(z / p.c_div) * p.c_bstride;
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int cc = 0; cc < MT * BN; cc += 32) {
+        const int mt = cc / BN, c0 = cc % BN;
         uint32_t r[32];
-        sm100::tmem_ld32(tmem + (uint32_t(warp * 32) << 16) + c0, r);
+        sm100::tmem_ld32(tmem + (uint32_t(warp * 32) << 16) + cc, r);
         sm100::tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; ++i) st[lane * 33 + i] = __uint_as_float(r[i]);
@@ -164,7 +177,7 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
         const int col = n0 + c0 + lane;
 #pragma unroll 4
         for (int i = 0; i < 32; ++i) {
-          const int row = m0 + warp * 32 + i;
+          const int row = m0 + mt * BM + warp * 32 + i;
           if (row < p.M && col < p.N) {
             float* dst = Cz + int64_t(row) * p.ldc + col;
             const float v = st[i * 33 + lane];
@@ -183,22 +196,22 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
 
 // ---- host: tensor maps ----------------------------------------------------------------------
 
-template <int BN, int AM, int BMJ>
+template <int BN, int AM, int BMJ, int MT>
 jolt_status launch(const TmaPack& maps, const GemmDev& d, dim3 grid, cudaStream_t st) {
-  using C = Cfg<BN>;
-  auto kern = k_gemm<BN, AM, BMJ>;
+  using C = Cfg<BN, MT>;
+  auto kern = k_gemm<BN, AM, BMJ, MT>;
   JOLT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem));
   kern<<<grid, 128, C::kSmem, st>>>(maps, d);
   JOLT_CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
 
-template <int BN>
+template <int BN, int MT>
 jolt_status launch_bn(int am, int bm, const TmaPack& maps, const GemmDev& d, dim3 grid, cudaStream_t st) {
-  if (am == kMajorK && bm == kMajorK) return launch<BN, kMajorK, kMajorK>(maps, d, grid, st);
-  if (am == kMajorK && bm == kMajorMN) return launch<BN, kMajorK, kMajorMN>(maps, d, grid, st);
-  if (am == kMajorMN && bm == kMajorK) return launch<BN, kMajorMN, kMajorK>(maps, d, grid, st);
-  return launch<BN, kMajorMN, kMajorMN>(maps, d, grid, st);
+  if (am == kMajorK && bm == kMajorK) return launch<BN, kMajorK, kMajorK, MT>(maps, d, grid, st);
+  if (am == kMajorK && bm == kMajorMN) return launch<BN, kMajorK, kMajorMN, MT>(maps, d, grid, st);
+  if (am == kMajorMN && bm == kMajorK) return launch<BN, kMajorMN, kMajorK, MT>(maps, d, grid, st);
+  return launch<BN, kMajorMN, kMajorMN, MT>(maps, d, grid, st);
 }
 
 }  // namespace
@@ -267,9 +280,9 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   const int am = g.A[0].major, bm = g.B[0].major;
   for (int t = 0; t < g.n_terms; ++t)
     if (g.A[t].major != am || g.B[t].major != bm) return JOLT_ERR_INVALID_ARG;
-  // BN: the tile width with the least padding of N, preferring the wider one
-  const int pad256 = (g.N + 255) / 256 * 256 - g.N, pad128 = (g.N + 127) / 128 * 128 - g.N;
-  const int BN = (g.N >= 256 && pad256 <= pad128) ? 256 : 128;
+  // BN: 256 whenever N exceeds one 128-wide tile — a 128 x 256 tile runs ~1.5x more flops per
+  // cycle than 128 x 128 (half the operand bytes per flop), which outweighs the padding of N
+  const int BN = g.N > 128 ? 256 : 128;
   TmaPack maps;
   memset(&maps, 0, sizeof(maps));
   GemmDev d{};
@@ -288,10 +301,14 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   d.C = g.C; d.ldc = g.ldc; d.c_bstride = g.c_batch_stride; d.c_div = g.c_batch_div;
   d.accumulate = g.accumulate ? 1 : 0;
   d.err = g.err;
-  const dim3 grid((g.N + BN - 1) / BN, (g.M + BM - 1) / BM, g.batch * g.k_split);
+  // two 128-row tiles per CTA when that still leaves at least two CTAs per SM
+  const int64_t ntile = (g.N + BN - 1) / BN, zc = int64_t(g.batch) * g.k_split;
+  const int MT = (g.M > BM && ntile * ((g.M + 2 * BM - 1) / (2 * BM)) * zc >= 2 * 148) ? 2 : 1;
+  const dim3 grid(unsigned(ntile), unsigned((g.M + BM * MT - 1) / (BM * MT)), unsigned(zc));
   if (grid.y > 65535 || grid.z > 65535) return JOLT_ERR_INVALID_ARG;
   StatScope sc(JOLT_K_GEMM, st, 2.0 * g.M * double(g.N) * g.K * g.batch * g.n_terms, 0.0);
-  return BN == 256 ? launch_bn<256>(am, bm, maps, d, grid, st) : launch_bn<128>(am, bm, maps, d, grid, st);
+  if (MT == 2) return BN == 256 ? launch_bn<256, 2>(am, bm, maps, d, grid, st) : launch_bn<128, 2>(am, bm, maps, d, grid, st);
+  return BN == 256 ? launch_bn<256, 1>(am, bm, maps, d, grid, st) : launch_bn<128, 1>(am, bm, maps, d, grid, st);
 }
 
 }  // namespace jolt

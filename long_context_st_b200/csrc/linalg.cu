@@ -1,16 +1,20 @@
 // Batched small dense linear algebra for the compressor.
 //
 // chol_inverse: right-looking blocked Cholesky (64-wide blocks, fp64) of G + shift*I, G = R^T R
-//   with R upper triangular, then the blocked triangular inverse R^{-1}. Every block step is a
-//   separate launch whose grid covers all matrices of the batch and all independent blocks, so
-//   the whole GPU works on a handful of 1152 x 1152 problems.
+//   with R upper triangular, then the blocked triangular inverse R^{-1} by block diagonals (the
+//   products of one diagonal spread over all CTAs, summed with fp64 atomics). One cooperative
+//   launch; block steps are separated by bounded grid barriers, and every step's grid covers all
+//   matrices of the batch and all independent blocks.
 // jacobi_eig: two-sided block Jacobi (32-wide blocks; each round diagonalises one cyclic sweep
 //   of 64 x 64 block pairs in shared memory, then applies the rotations to whole block rows and
 //   columns), tournament ordering, fp32, sweeps until the off-diagonal norm is below tol.
 #include <algorithm>
+#include <cstdio>
+#include <cstdlib>
 #include <vector>
 
 #include "linalg.cuh"
+#include "stats.h"
 
 namespace jolt {
 
@@ -91,107 +95,87 @@ CholScratch chol_carve(void* scratch, int nb, int n) {
 
 
 
-// 64x64 fp64 tile load/store helpers (row stride np).
+// 64x64 fp64 tile load (row stride np) into shared memory; a warp reads half a row per access.
 __device__ __forceinline__ void tile_load(double (*S)[NB + 1], const double* src, int np) {
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) S[e / NB][e % NB] = src[int64_t(e / NB) * np + e % NB];
-}
-__device__ __forceinline__ void tile_store(double* dst, double (*S)[NB + 1], int np) {
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) dst[int64_t(e / NB) * np + e % NB] = S[e / NB][e % NB];
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) S[e >> 6][e & 63] = src[int64_t(e >> 6) * np + (e & 63)];
 }
 
-// out = op(A)^T-style products on 64x64 tiles: C[a][b] = sum_k A[k][a] * B[k][b]
-__device__ __forceinline__ void tile_atb(double (*C)[NB + 1], double (*A)[NB + 1], double (*B)[NB + 1]) {
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;  // 16x16 threads, 4x4 outputs each
-  double acc[4][4] = {};
+// 64x64x64 tile product held in registers: thread (ty, tx) of a 16 x 16 grid owns the strided
+// 4 x 4 set C[ty + 16u][tx + 16v] (a warp reads 16 consecutive B elements and broadcasts two A
+// elements per step: no shared-memory bank conflicts). TA: C = A^T B when true, else C = A B.
+template <bool TA, int LD>
+__device__ __forceinline__ void tile_mm(double (&acc)[4][4], const double (*A)[LD], const double (*B)[LD]) {
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll 4
   for (int k = 0; k < NB; ++k) {
     double a[4], bb[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) a[u] = A[k][ty * 4 + u];
+    for (int u = 0; u < 4; ++u) a[u] = TA ? A[k][ty + 16 * u] : A[ty + 16 * u][k];
 #pragma unroll
-    for (int v = 0; v < 4; ++v) bb[v] = B[k][tx * 4 + v];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int v = 0; v < 4; ++v) acc[u][v] += a[u] * bb[v];
-  }
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-#pragma unroll
-    for (int v = 0; v < 4; ++v) C[ty * 4 + u][tx * 4 + v] = acc[u][v];
-}
-// C[a][b] = sum_k A[a][k] * B[k][b]
-__device__ __forceinline__ void tile_ab(double (*C)[NB + 1], double (*A)[NB + 1], double (*B)[NB + 1]) {
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
-  double acc[4][4] = {};
-  for (int k = 0; k < NB; ++k) {
-    double a[4], bb[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) a[u] = A[ty * 4 + u][k];
-#pragma unroll
-    for (int v = 0; v < 4; ++v) bb[v] = B[k][tx * 4 + v];
+    for (int v = 0; v < 4; ++v) bb[v] = B[k][tx + 16 * v];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
-      for (int v = 0; v < 4; ++v) acc[u][v] += a[u] * bb[v];
+      for (int v = 0; v < 4; ++v) acc[u][v] = fma(a[u], bb[v], acc[u][v]);
   }
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-#pragma unroll
-    for (int v = 0; v < 4; ++v) C[ty * 4 + u][tx * 4 + v] = acc[u][v];
 }
 
-// Factor the diagonal block p of matrix b and invert it.
+// Factor the diagonal block p of matrix b (right-looking, one barrier per column: the trailing
+// update uses the unscaled pivot row, S_ik -= S_ji S_jk / d_j, and rows are scaled by 1/sqrt(d_j)
+// at the end), then invert the upper-triangular factor row by row from the bottom.
 __device__ void dev_chol_diag(double* __restrict__ Gd, double* __restrict__ Xd, int np, int p,
                               const double* __restrict__ diag0, float* ratio, int b, double* sh) {
   double(*S)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*X)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
+  __shared__ double dpiv[NB];
+  __shared__ double part[4][NB];
   double* gd = Gd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
   double* xd = Xd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
   tile_load(S, gd, np);
   __syncthreads();
-  float rmin = 1.f;
   for (int j = 0; j < NB; ++j) {
-    if (threadIdx.x == 0) {
-      double d = S[j][j];
-      const double d0 = diag0[int64_t(b) * np + p * NB + j];
-      if (!(d > 0.0) || !(d0 > 0.0)) {
-        rmin = 0.f;  // breakdown: the caller retries with a shift
-        d = 1.0;
-      } else {
-        rmin = fminf(rmin, float(d / d0));
-      }
-      S[j][j] = sqrt(d);
-    }
-    __syncthreads();
-    const double piv = S[j][j];
-    for (int k = j + 1 + threadIdx.x; k < NB; k += blockDim.x) S[j][k] /= piv;
-    __syncthreads();
+    double d = S[j][j];
+    if (!(d > 0.0)) d = 1.0;  // breakdown: recorded below, the caller retries with a shift
+    const double inv = 1.0 / d;
     const int m = NB - j - 1;
     for (int e = threadIdx.x; e < m * m; e += blockDim.x) {
       const int i = j + 1 + e / m, k = j + 1 + e % m;
-      if (i <= k) S[i][k] -= S[j][i] * S[j][k];
+      if (i <= k) S[i][k] -= S[j][i] * S[j][k] * inv;
     }
+    if (threadIdx.x == 0) dpiv[j] = S[j][j];
     __syncthreads();
   }
-  if (threadIdx.x == 0) atomicMin(reinterpret_cast<int*>(ratio + b), __float_as_int(rmin));
+  if (threadIdx.x == 0) {
+    float rmin = 1.f;
+    for (int j = 0; j < NB; ++j) {
+      const double d = dpiv[j], d0 = diag0[int64_t(b) * np + p * NB + j];
+      rmin = (d > 0.0 && d0 > 0.0) ? fminf(rmin, float(d / d0)) : 0.f;
+    }
+    atomicMin(reinterpret_cast<int*>(ratio + b), __float_as_int(rmin));
+  }
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int i = e / NB, k = e % NB;
-    if (i > k) S[i][k] = 0.0;
+    const int i = e >> 6, k = e & 63;
+    const bool ok = dpiv[i] > 0.0;  // a broken-down pivot becomes 1 (the result is discarded)
+    S[i][k] = (i > k) ? 0.0 : (i == k ? (ok ? sqrt(dpiv[i]) : 1.0) : S[i][k] / (ok ? sqrt(dpiv[i]) : 1.0));
     X[i][k] = 0.0;
   }
   __syncthreads();
-  if (threadIdx.x < NB) {
-    const int c = threadIdx.x;
-    X[c][c] = 1.0 / S[c][c];
-    for (int i = c - 1; i >= 0; --i) {
-      double a = 0.0;
-      for (int k = i + 1; k <= c; ++k) a += S[i][k] * X[k][c];
-      X[i][c] = -a / S[i][i];
-    }
+  // X = R^-1: X_ic = (delta_ic - sum_{i<k<=c} R_ik X_kc) / R_ii, rows from the bottom; thread
+  // (q, c) sums the k-quarter q of column c
+  const int c = threadIdx.x & 63, q = threadIdx.x >> 6;
+  for (int i = NB - 1; i >= 0; --i) {
+    double a = 0.0;
+    if (c > i)
+      for (int k = i + 1 + q; k <= c; k += 4) a = fma(S[i][k], X[k][c], a);
+    part[q][c] = a;
+    __syncthreads();
+    if (q == 0 && c >= i) X[i][c] = ((c == i ? 1.0 : 0.0) - (part[0][c] + part[1][c] + part[2][c] + part[3][c])) / S[i][i];
+    __syncthreads();
   }
-  __syncthreads();
-  tile_store(gd, S, np);
-  tile_store(xd, X, np);
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+    gd[int64_t(e >> 6) * np + (e & 63)] = S[e >> 6][e & 63];
+    xd[int64_t(e >> 6) * np + (e & 63)] = X[e >> 6][e & 63];
+  }
   __syncthreads();
 }
 
@@ -200,15 +184,18 @@ __device__ void dev_chol_panel(double* __restrict__ Gd, const double* __restrict
                                int j, double* sh) {
   double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
-  double(*C)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 2 * NB * (NB + 1));
   const double* xpp = Xd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
   double* gpj = Gd + int64_t(b) * np * np + int64_t(p) * NB * np + j * NB;
   tile_load(A, xpp, np);
   tile_load(B, gpj, np);
   __syncthreads();
-  tile_atb(C, A, B);
-  __syncthreads();
-  tile_store(gpj, C, np);
+  double acc[4][4] = {};
+  tile_mm<true, NB + 1>(acc, A, B);
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) gpj[int64_t(ty + 16 * u) * np + tx + 16 * v] = acc[u][v];
   __syncthreads();
 }
 
@@ -216,7 +203,6 @@ __device__ void dev_chol_panel(double* __restrict__ Gd, const double* __restrict
 __device__ void dev_chol_update(double* __restrict__ Gd, int np, int P, int p, int b, int idx, double* sh) {
   double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
-  double(*C)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 2 * NB * (NB + 1));
   int i = p + 1;
   while (idx >= P - i) {
     idx -= P - i;
@@ -227,40 +213,55 @@ __device__ void dev_chol_update(double* __restrict__ Gd, int np, int P, int p, i
   tile_load(A, g + int64_t(p) * NB * np + i * NB, np);
   tile_load(B, g + int64_t(p) * NB * np + j * NB, np);
   __syncthreads();
-  tile_atb(C, A, B);
-  __syncthreads();
+  double acc[4][4] = {};
+  tile_mm<true, NB + 1>(acc, A, B);
   double* gij = g + int64_t(i) * NB * np + j * NB;
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) gij[int64_t(e / NB) * np + e % NB] -= C[e / NB][e % NB];
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) gij[int64_t(ty + 16 * u) * np + tx + 16 * v] -= acc[u][v];
   __syncthreads();
 }
 
-// Inverse blocks at distance d: X_ij = -X_ii * sum_{k=i+1..j} R_ik X_kj, j = i + d.
-__device__ void dev_trinv(const double* __restrict__ Gd, double* __restrict__ Xd, int np, int d, int b, int i,
-                          double* sh) {
+// Triangular inverse, diagonal d, step 1: S_ij += R_ik X_kj for one k in (i, j], j = i + d,
+// accumulated (fp64 atomics) into the still-zero block X_ij.
+__device__ void dev_trinv_sum(const double* __restrict__ Gd, double* __restrict__ Xd, int np, int i, int j, int k,
+                              int b, double* sh) {
   double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
-  double(*C)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 2 * NB * (NB + 1));
-  double(*Acc)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + 3 * NB * (NB + 1));
-  const int j = i + d;
   const double* g = Gd + int64_t(b) * np * np;
   double* x = Xd + int64_t(b) * np * np;
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) Acc[e / NB][e % NB] = 0.0;
-  for (int k = i + 1; k <= j; ++k) {
-    __syncthreads();
-    tile_load(A, g + int64_t(i) * NB * np + k * NB, np);
-    tile_load(B, x + int64_t(k) * NB * np + j * NB, np);
-    __syncthreads();
-    tile_ab(C, A, B);
-    __syncthreads();
-    for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) Acc[e / NB][e % NB] += C[e / NB][e % NB];
-  }
+  tile_load(A, g + int64_t(i) * NB * np + k * NB, np);
+  tile_load(B, x + int64_t(k) * NB * np + j * NB, np);
   __syncthreads();
-  tile_load(A, x + int64_t(i) * NB * np + i * NB, np);
-  __syncthreads();
-  tile_ab(C, A, Acc);
-  __syncthreads();
+  double acc[4][4] = {};
+  tile_mm<false, NB + 1>(acc, A, B);
   double* xij = x + int64_t(i) * NB * np + j * NB;
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) xij[int64_t(e / NB) * np + e % NB] = -C[e / NB][e % NB];
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) atomicAdd(&xij[int64_t(ty + 16 * u) * np + tx + 16 * v], acc[u][v]);
+  __syncthreads();
+}
+
+// Step 2: X_ij = -X_ii S_ij.
+__device__ void dev_trinv_fin(double* __restrict__ Xd, int np, int i, int j, int b, double* sh) {
+  double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
+  double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
+  double* x = Xd + int64_t(b) * np * np;
+  tile_load(A, x + int64_t(i) * NB * np + i * NB, np);
+  double* xij = x + int64_t(i) * NB * np + j * NB;
+  tile_load(B, xij, np);
+  __syncthreads();
+  double acc[4][4] = {};
+  tile_mm<false, NB + 1>(acc, A, B);
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) xij[int64_t(ty + 16 * u) * np + tx + 16 * v] = -acc[u][v];
   __syncthreads();
 }
 
@@ -269,7 +270,7 @@ struct CholArgs {
   int64_t ldg;
   int n, np, P, nb;
   double shift_rel;
-  double *Gd, *Xd, *md, *diag0;
+  double *Gd, *Xd, *md, *diag0;  // md: sums of squares, zeroed before the launch
   float* ratio;
   __nv_bfloat16 *hi, *lo;
   GridBar bar;
@@ -279,39 +280,36 @@ struct CholArgs {
 __global__ void __launch_bounds__(256) k_chol_coop(CholArgs a) {
   extern __shared__ double sh[];
   const int nbk = gridDim.x;
-  // norms and ratios
-  for (int b = blockIdx.x; b < a.nb; b += nbk) {
-    const float* g = a.G + int64_t(b) * a.n * a.ldg;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int64_t gw = int64_t(blockIdx.x) * nw + wid, nwt = int64_t(nbk) * nw;
+  // Frobenius norms (a warp per row), pivot ratios reset
+  for (int64_t row = gw; row < int64_t(a.nb) * a.n; row += nwt) {
+    const int b = int(row / a.n), i = int(row % a.n);
+    const float* g = a.G + int64_t(b) * a.n * a.ldg + int64_t(i) * a.ldg;
     double m = 0.0;
-    for (int64_t e = threadIdx.x; e < int64_t(a.n) * a.n; e += blockDim.x) {
-      const double v = g[(e / a.n) * a.ldg + e % a.n];
-      m += v * v;
+    for (int j = lane; j < a.n; j += 32) {
+      const double v = g[j];
+      m = fma(v, v, m);
     }
-    sh[threadIdx.x] = m;
-    __syncthreads();
-    for (int st = blockDim.x / 2; st; st >>= 1) {
-      if (threadIdx.x < st) sh[threadIdx.x] += sh[threadIdx.x + st];
-      __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-      a.md[b] = sqrt(sh[0]);
-      a.ratio[b] = 1.f;
-    }
-    __syncthreads();
+    for (int o = 16; o; o >>= 1) m += __shfl_xor_sync(0xffffffffu, m, o);
+    if (lane == 0) atomicAdd(a.md + b, m);
   }
+  if (blockIdx.x == 0)
+    for (int b = threadIdx.x; b < a.nb; b += blockDim.x) a.ratio[b] = 1.f;
   grid_barrier(a.bar);
-  // shifted copy into fp64 working storage
-  {
-    const int64_t tot = int64_t(a.nb) * a.np * a.np;
-    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < tot; e += int64_t(nbk) * blockDim.x) {
-      const int b = int(e / (int64_t(a.np) * a.np));
-      const int64_t r = e % (int64_t(a.np) * a.np);
-      const int i = int(r / a.np), j = int(r % a.np);
+  // shifted copy into fp64 working storage (padding: identity), X zeroed
+  for (int64_t row = gw; row < int64_t(a.nb) * a.np; row += nwt) {
+    const int b = int(row / a.np), i = int(row % a.np);
+    const double shift = a.shift_rel * sqrt(a.md[b]);
+    const float* g = a.G + int64_t(b) * a.n * a.ldg + int64_t(i) * a.ldg;
+    double* gd = a.Gd + row * a.np;
+    double* xd = a.Xd + row * a.np;
+    for (int j = lane; j < a.np; j += 32) {
       double v;
-      if (i < a.n && j < a.n) v = double(a.G[int64_t(b) * a.n * a.ldg + int64_t(i) * a.ldg + j]) + (i == j ? a.shift_rel * a.md[b] : 0.0);
+      if (i < a.n && j < a.n) v = double(g[j]) + (i == j ? shift : 0.0);
       else v = (i == j) ? 1.0 : 0.0;
-      a.Gd[e] = v;
-      a.Xd[e] = 0.0;
+      gd[j] = v;
+      xd[j] = 0.0;
       if (i == j) a.diag0[int64_t(b) * a.np + i] = v;
     }
   }
@@ -328,20 +326,29 @@ __global__ void __launch_bounds__(256) k_chol_coop(CholArgs a) {
       grid_barrier(a.bar);
     }
   }
+  // X = R^-1 by block diagonals: X_ij = -X_ii sum_{k=i+1..j} R_ik X_kj
   for (int d = 1; d < a.P; ++d) {
-    const int cnt = a.P - d;
-    for (int it = blockIdx.x; it < a.nb * cnt; it += nbk) dev_trinv(a.Gd, a.Xd, a.np, d, it / cnt, it % cnt, sh);
+    const int cnt = a.P - d;  // blocks on the diagonal
+    const int items = a.nb * cnt * d;
+    for (int it = blockIdx.x; it < items; it += nbk) {
+      const int b = it / (cnt * d), r = it % (cnt * d);
+      const int i = r / d, k = i + 1 + r % d;
+      dev_trinv_sum(a.Gd, a.Xd, a.np, i, i + d, k, b, sh);
+    }
+    grid_barrier(a.bar);
+    for (int it = blockIdx.x; it < a.nb * cnt; it += nbk) dev_trinv_fin(a.Xd, a.np, it % cnt, it % cnt + d, it / cnt, sh);
     grid_barrier(a.bar);
   }
-  const int64_t tot = int64_t(a.n) * a.n;
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < tot * a.nb; e += int64_t(nbk) * blockDim.x) {
-    const int b = int(e / tot);
-    const int64_t r = e % tot;
-    const int i = int(r / a.n), j = int(r % a.n);
-    const float v = (i <= j) ? float(a.Xd[int64_t(b) * a.np * a.np + int64_t(i) * a.np + j]) : 0.f;
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    a.hi[e] = h;
-    a.lo[e] = __float2bfloat16_rn(v - __bfloat162float(h));
+  // R^-1 (upper triangle) as bf16 hi + lo, a warp per row
+  for (int64_t row = gw; row < int64_t(a.nb) * a.n; row += nwt) {
+    const int b = int(row / a.n), i = int(row % a.n);
+    const double* x = a.Xd + (int64_t(b) * a.np + i) * a.np;
+    for (int j = lane; j < a.n; j += 32) {
+      const float v = (i <= j) ? float(x[j]) : 0.f;
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      a.hi[row * a.n + j] = h;
+      a.lo[row * a.n + j] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
   }
 }
 
@@ -482,24 +489,14 @@ __device__ void dev_jac_cols(double* __restrict__ Aw, double* __restrict__ V, in
     }
     __syncthreads();
     double acc[4][4] = {};
-    for (int kk = 0; kk < JS; ++kk) {
-      double a[4], bb[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) a[u] = X[ty * 4 + u][kk];
-#pragma unroll
-      for (int v = 0; v < 4; ++v) bb[v] = T[kk][tx * 4 + v];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] += a[u] * bb[v];
-    }
+    tile_mm<false, JS + 1>(acc, X, T);
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
-        const int col = tx * 4 + v;
+        const int col = tx + 16 * v;
         const int gv = (col < JW ? I * JW + col : J * JW + col - JW);
-        M[int64_t(r0 + ty * 4 + u) * np + gv] = acc[u][v];
+        M[int64_t(r0 + ty + 16 * u) * np + gv] = acc[u][v];
       }
   }
   __syncthreads();
@@ -524,23 +521,13 @@ __device__ void dev_jac_rows(double* __restrict__ Aw, int np, int nblk, int roun
   __syncthreads();
   const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
   double acc[4][4] = {};
-  for (int kk = 0; kk < JS; ++kk) {
-    double a[4], bb[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) a[u] = T[kk][ty * 4 + u];
-#pragma unroll
-    for (int v = 0; v < 4; ++v) bb[v] = X[kk][tx * 4 + v];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int v = 0; v < 4; ++v) acc[u][v] += a[u] * bb[v];
-  }
+  tile_mm<true, JS + 1>(acc, T, X);
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
-    const int row = ty * 4 + u;
+    const int row = ty + 16 * u;
     const int gu = (row < JW ? I * JW + row : J * JW + row - JW);
 #pragma unroll
-    for (int v = 0; v < 4; ++v) M[int64_t(gu) * np + c0 + tx * 4 + v] = acc[u][v];
+    for (int v = 0; v < 4; ++v) M[int64_t(gu) * np + c0 + tx + 16 * v] = acc[u][v];
   }
   __syncthreads();
 }
@@ -573,21 +560,27 @@ __global__ void __launch_bounds__(256) k_jac_coop(JacArgs a) {
     }
     // off-diagonal and total Frobenius mass of every matrix
     double* nm = a.norms + int64_t(sweep) * a.nb * 2;
-    const int64_t tot = int64_t(a.np) * a.np;
-    for (int b = 0; b < a.nb; ++b) {
-      double off = 0.0, all = 0.0;
-      for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < tot; e += int64_t(nbk) * blockDim.x) {
-        const double v = a.A[int64_t(b) * tot + e];
-        all += v * v;
-        if (e / a.np != e % a.np) off += v * v;
-      }
-      for (int m = 16; m; m >>= 1) {
-        off += __shfl_xor_sync(0xffffffffu, off, m);
-        all += __shfl_xor_sync(0xffffffffu, all, m);
-      }
-      if ((threadIdx.x & 31) == 0 && (off != 0.0 || all != 0.0)) {
-        atomicAdd(&nm[2 * b], off);
-        atomicAdd(&nm[2 * b + 1], all);
+    {
+      // a warp per row of every matrix
+      const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+      for (int64_t row = int64_t(blockIdx.x) * nw + (threadIdx.x >> 5); row < int64_t(a.nb) * a.np;
+           row += int64_t(nbk) * nw) {
+        const int b = int(row / a.np), i = int(row % a.np);
+        const double* ar = a.A + row * a.np;
+        double off = 0.0, all = 0.0;
+        for (int j = lane; j < a.np; j += 32) {
+          const double v = ar[j];
+          all = fma(v, v, all);
+          if (j != i) off = fma(v, v, off);
+        }
+        for (int m = 16; m; m >>= 1) {
+          off += __shfl_xor_sync(0xffffffffu, off, m);
+          all += __shfl_xor_sync(0xffffffffu, all, m);
+        }
+        if (lane == 0 && (off != 0.0 || all != 0.0)) {
+          atomicAdd(&nm[2 * b], off);
+          atomicAdd(&nm[2 * b + 1], all);
+        }
       }
     }
     grid_barrier(a.bar);
@@ -698,12 +691,18 @@ jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shi
   const int np = rup(n, NB), P = np / NB;
   CholScratch s = chol_carve(scratch, nb, n);
   JOLT_CUDA_TRY(cudaMemsetAsync(s.bar, 0, 2 * sizeof(unsigned int), st));
+  JOLT_CUDA_TRY(cudaMemsetAsync(s.mdiag, 0, size_t(nb) * sizeof(double), st));
   CholArgs a;
   a.G = G; a.ldg = ld_g; a.n = n; a.np = np; a.P = P; a.nb = nb; a.shift_rel = shift_rel;
   a.Gd = s.Gd; a.Xd = s.Xd; a.md = s.mdiag; a.diag0 = s.diag0; a.ratio = s.ratio;
   a.hi = rinv_hi; a.lo = rinv_lo;
   a.bar = GridBar{s.bar, s.bar + 1, err};
-  jolt_status r = launch_coop(k_chol_coop, a, 4 * NB * (NB + 1) * 8, st);
+  jolt_status r;
+  {
+    // fp64 work: factor n^3/3 plus triangular inverse n^3/3 per matrix
+    StatScope sc(JOLT_K_CHOL, st, nb * 2.0 * double(n) * n * n / 3.0, 0.0);
+    r = launch_coop(k_chol_coop, a, 2 * NB * (NB + 1) * 8, st);
+  }
   if (r) return r;
   if (min_ratio) {
     std::vector<float> h(nb);
@@ -738,8 +737,18 @@ jolt_status jacobi_impl(const TA* A, int64_t ld_a, int nb, int n, TO* evals, TO*
   a.tol = tol;
   a.sweeps_done = s.sweeps;
   a.bar = GridBar{s.bar, s.bar + 1, err};
-  jolt_status r = launch_coop(k_jac_coop, a, 2 * JS * (JS + 1) * 8, st);
+  jolt_status r;
+  {
+    StatScope sc(JOLT_K_EIG, st, 0.0, 0.0);
+    r = launch_coop(k_jac_coop, a, 2 * JS * (JS + 1) * 8, st);
+  }
   if (r) return r;
+  if (std::getenv("JOLT_DEBUG")) {
+    int sw = 0;
+    JOLT_CUDA_TRY(cudaMemcpyAsync(&sw, s.sweeps, sizeof(int), cudaMemcpyDeviceToHost, st));
+    JOLT_CUDA_TRY(cudaStreamSynchronize(st));
+    std::fprintf(stderr, "jolt jacobi: n %d batch %d sweeps %d\n", n, nb, sw);
+  }
   k_jac_sort<<<dim3((n + 255) / 256, nb), 256, 0, st>>>(s.A, np, n, evals, s.perm);
   k_jac_out<<<dim3(grid_1d(int64_t(n) * n), nb), 256, 0, st>>>(s.V, np, n, s.perm, evecs);
   JOLT_CUDA_TRY(cudaGetLastError());

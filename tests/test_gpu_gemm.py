@@ -17,7 +17,9 @@ def ref_mm(A, B, a_mn, b_mn):
 
 @pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
 @pytest.mark.parametrize("M,N,K", [(128, 128, 64), (1000, 1152, 1000), (304, 96, 4160),
-                                   (4096, 256, 128), (64, 384, 200)])
+                                   (4096, 256, 128), (64, 384, 200),
+                                   # grids large enough for two 128-row tiles per CTA, ragged M/N/K
+                                   (16000, 1152, 192), (80000, 200, 72)])
 def test_gemm_majors_and_ragged(cuda_ok, a_mn, b_mn, M, N, K):
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K + a_mn * 2 + b_mn)
     A = torch.randn((K, M) if a_mn else (M, K), generator=g, device="cuda").to(torch.bfloat16)
