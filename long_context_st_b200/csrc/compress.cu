@@ -666,7 +666,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
     }
     float* ev = c.at<float>(p.ev);
     float* evec = c.at<float>(p.evec);
-    if ((r = jacobi_eig(W, l, C, l, ev, evec, c.pass() + p.jac, 30, 1e-10, c.err, c.st))) return r;
+    if ((r = jacobi_eig(W, l, C, l, ev, evec, c.pass() + p.jac, 30, 1e-8, c.err, c.st))) return r;
     __nv_bfloat16* Vh = c.at<__nv_bfloat16>(p.Vh);
     __nv_bfloat16* Vl = c.at<__nv_bfloat16>(p.Vl);
     if ((r = split_bf16(evec, l, l, l, C, int64_t(l) * l, Vh, Vl, l, int64_t(l) * l, c.st))) return r;
@@ -692,7 +692,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
   }
   float* evd = c.at<float>(p.evd);
   float* evecd = c.at<float>(p.evecd);
-  if ((r = jacobi_eig(Sd, d, C, d, evd, evecd, c.pass() + p.jac, 30, 1e-10, c.err, c.st))) return r;
+  if ((r = jacobi_eig(Sd, d, C, d, evd, evecd, c.pass() + p.jac, 30, 1e-8, c.err, c.st))) return r;
   std::vector<float> d32(size_t(C) * d);
   nrm.resize(C);
   JOLT_CUDA_TRY(cudaMemcpyAsync(d32.data(), evd, size_t(C) * d * 4, cudaMemcpyDeviceToHost, c.st));
@@ -865,7 +865,7 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
       }
       float* evy = c.atc<float>(p.evy);
       float* evecy = c.atc<float>(p.evecy);
-      if ((r = jacobi_eig(sy, d, 1, d, evy, evecy, c.ws + p.off_cmp + p.jac2, 30, 1e-10, c.err, c.st))) return r;
+      if ((r = jacobi_eig(sy, d, 1, d, evy, evecy, c.ws + p.off_cmp + p.jac2, 30, 1e-8, c.err, c.st))) return r;
       // U_d = first rd eigenvector columns (stored dtype), then G = Y U_d (stored dtype)
       k_store_ut<<<grid1(int64_t(d) * rd), 256, 0, c.st>>>(evecy, d, d, rd, f32, cud, nullptr, nullptr, nullptr);
       k_proj_small<<<grid1(int64_t(LgH) * rT * rd), 256, 0, c.st>>>(ylh, int64_t(LgH) * rT, d, evecy, d, rd, f32, cg);

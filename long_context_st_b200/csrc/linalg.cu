@@ -5,9 +5,11 @@
 //   products of one diagonal spread over all CTAs, summed with fp64 atomics). One cooperative
 //   launch; block steps are separated by bounded grid barriers, and every step's grid covers all
 //   matrices of the batch and all independent blocks.
-// jacobi_eig: two-sided block Jacobi (32-wide blocks; each round diagonalises one cyclic sweep
-//   of 64 x 64 block pairs in shared memory, then applies the rotations to whole block rows and
-//   columns), tournament ordering, fp32, sweeps until the off-diagonal norm is below tol.
+// jacobi_eig: two-sided block Jacobi (32-wide blocks, tournament ordering, fp64 working storage):
+//   each round runs one cyclic sweep on every 64 x 64 pair subproblem in shared memory (writing
+//   the rotated diagonal pair-block back), then, in one pass, applies Theta1^T . Theta2 to every
+//   off-diagonal pair-block of A and Theta to the block columns of V; sweeps until the
+//   off-diagonal norm is below tol.
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
@@ -120,30 +122,54 @@ __device__ __forceinline__ void tile_mm(double (&acc)[4][4], const double (*A)[L
   }
 }
 
-// Factor the diagonal block p of matrix b (right-looking, one barrier per column: the trailing
-// update uses the unscaled pivot row, S_ik -= S_ji S_jk / d_j, and rows are scaled by 1/sqrt(d_j)
-// at the end), then invert the upper-triangular factor row by row from the bottom.
+// Factor the diagonal block p of matrix b (right-looking; the trailing update uses the unscaled
+// pivot row, S_ic -= S_ji S_jc / d_j, and rows are scaled by 1/sqrt(d_j) at the end), then invert
+// the upper-triangular factor row by row from the bottom. Thread t: column t & 63 and row group
+// t >> 6 in the factorisation; column t >> 2 and k-residue t & 3 in the inverse.
 __device__ void dev_chol_diag(double* __restrict__ Gd, double* __restrict__ Xd, int np, int p,
                               const double* __restrict__ diag0, float* ratio, int b, double* sh) {
   double(*S)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*X)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
-  __shared__ double dpiv[NB];
-  __shared__ double part[4][NB];
+  __shared__ double dpiv[NB], pinv[NB], rs[NB];
   double* gd = Gd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
   double* xd = Xd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
   tile_load(S, gd, np);
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) X[e >> 6][e & 63] = 0.0;
   __syncthreads();
-  for (int j = 0; j < NB; ++j) {
-    double d = S[j][j];
-    if (!(d > 0.0)) d = 1.0;  // breakdown: recorded below, the caller retries with a shift
-    const double inv = 1.0 / d;
-    const int m = NB - j - 1;
-    for (int e = threadIdx.x; e < m * m; e += blockDim.x) {
-      const int i = j + 1 + e / m, k = j + 1 + e % m;
-      if (i <= k) S[i][k] -= S[j][i] * S[j][k] * inv;
+  if (threadIdx.x == 0) {
+    const double d = S[0][0];
+    dpiv[0] = d;
+    pinv[0] = d > 0.0 ? 1.0 / d : 1.0;  // breakdown: recorded below, the caller retries with a shift
+  }
+  __syncthreads();
+  {
+    const int c = threadIdx.x & 63, rg = threadIdx.x >> 6;
+    for (int j = 0; j < NB; ++j) {
+      if (c > j) {
+        const double f = S[j][c] * pinv[j];
+        int i = j + 1 + rg;
+        for (; i + 12 <= c; i += 16) {  // four independent read-modify-writes in flight
+          const double s0 = S[j][i], s1 = S[j][i + 4], s2 = S[j][i + 8], s3 = S[j][i + 12];
+          const double t0 = S[i][c], t1 = S[i + 4][c], t2 = S[i + 8][c], t3 = S[i + 12][c];
+          S[i][c] = fma(-s0, f, t0);
+          S[i + 4][c] = fma(-s1, f, t1);
+          S[i + 8][c] = fma(-s2, f, t2);
+          S[i + 12][c] = fma(-s3, f, t3);
+        }
+        for (; i <= c; i += 4) S[i][c] = fma(-S[j][i], f, S[i][c]);
+        // the owner of the next pivot has just finalised it: publish its reciprocal
+        if (c == j + 1 && rg == 0) {
+          const double d = S[c][c];
+          dpiv[c] = d;
+          pinv[c] = d > 0.0 ? 1.0 / d : 1.0;
+        }
+      }
+      __syncthreads();
     }
-    if (threadIdx.x == 0) dpiv[j] = S[j][j];
-    __syncthreads();
+  }
+  if (threadIdx.x < NB) {
+    const double d = dpiv[threadIdx.x];
+    rs[threadIdx.x] = d > 0.0 ? 1.0 / sqrt(d) : 1.0;  // a broken-down pivot becomes 1 (result discarded)
   }
   if (threadIdx.x == 0) {
     float rmin = 1.f;
@@ -153,24 +179,30 @@ __device__ void dev_chol_diag(double* __restrict__ Gd, double* __restrict__ Xd, 
     }
     atomicMin(reinterpret_cast<int*>(ratio + b), __float_as_int(rmin));
   }
+  __syncthreads();
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
     const int i = e >> 6, k = e & 63;
-    const bool ok = dpiv[i] > 0.0;  // a broken-down pivot becomes 1 (the result is discarded)
-    S[i][k] = (i > k) ? 0.0 : (i == k ? (ok ? sqrt(dpiv[i]) : 1.0) : S[i][k] / (ok ? sqrt(dpiv[i]) : 1.0));
-    X[i][k] = 0.0;
+    S[i][k] = (i > k) ? 0.0 : (i == k ? (dpiv[i] > 0.0 ? dpiv[i] * rs[i] : 1.0) : S[i][k] * rs[i]);
   }
   __syncthreads();
-  // X = R^-1: X_ic = (delta_ic - sum_{i<k<=c} R_ik X_kc) / R_ii, rows from the bottom; thread
-  // (q, c) sums the k-quarter q of column c
-  const int c = threadIdx.x & 63, q = threadIdx.x >> 6;
-  for (int i = NB - 1; i >= 0; --i) {
-    double a = 0.0;
-    if (c > i)
-      for (int k = i + 1 + q; k <= c; k += 4) a = fma(S[i][k], X[k][c], a);
-    part[q][c] = a;
-    __syncthreads();
-    if (q == 0 && c >= i) X[i][c] = ((c == i ? 1.0 : 0.0) - (part[0][c] + part[1][c] + part[2][c] + part[3][c])) / S[i][i];
-    __syncthreads();
+  // X = R^-1: X_ic = (delta_ic - sum_{i<k<=c} R_ik X_kc) / R_ii, one barrier per row
+  {
+    const int c = threadIdx.x >> 2, q = threadIdx.x & 3;
+    for (int i = NB - 1; i >= 0; --i) {
+      double a0 = 0.0, a1 = 0.0;
+      int k = i + 1 + q;
+      for (; k + 4 <= c; k += 8) {
+        a0 = fma(S[i][k], X[k][c], a0);
+        a1 = fma(S[i][k + 4], X[k + 4][c], a1);
+      }
+      if (k <= c) a0 = fma(S[i][k], X[k][c], a0);
+      double a = a0 + a1;
+      a += __shfl_xor_sync(0xffffffffu, a, 1);
+      a += __shfl_xor_sync(0xffffffffu, a, 2);
+      // 1 / R_ii = rs[i] (R_ii = sqrt(d_i), or 1 after a breakdown)
+      if (q == 0 && c >= i) X[i][c] = ((c == i ? 1.0 : 0.0) - a) * rs[i];
+      __syncthreads();
+    }
   }
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
     gd[int64_t(e >> 6) * np + (e & 63)] = S[e >> 6][e & 63];
@@ -179,23 +211,36 @@ __device__ void dev_chol_diag(double* __restrict__ Gd, double* __restrict__ Xd, 
   __syncthreads();
 }
 
-// Panel: R_pj = X_pp^T G_pj for j > p.
+// Panel: R_pj = X_pp^T G_pj for j > p, and W_pj = X_pp R_pj (kept in the unused lower block
+// (j, p) of Gd for the triangular inverse).
 __device__ void dev_chol_panel(double* __restrict__ Gd, const double* __restrict__ Xd, int np, int p, int b,
                                int j, double* sh) {
   double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
   const double* xpp = Xd + int64_t(b) * np * np + int64_t(p) * NB * np + p * NB;
   double* gpj = Gd + int64_t(b) * np * np + int64_t(p) * NB * np + j * NB;
+  double* wjp = Gd + int64_t(b) * np * np + int64_t(j) * NB * np + p * NB;
   tile_load(A, xpp, np);
   tile_load(B, gpj, np);
   __syncthreads();
   double acc[4][4] = {};
   tile_mm<true, NB + 1>(acc, A, B);
   const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  __syncthreads();
 #pragma unroll
   for (int u = 0; u < 4; ++u)
 #pragma unroll
-    for (int v = 0; v < 4; ++v) gpj[int64_t(ty + 16 * u) * np + tx + 16 * v] = acc[u][v];
+    for (int v = 0; v < 4; ++v) {
+      gpj[int64_t(ty + 16 * u) * np + tx + 16 * v] = acc[u][v];
+      B[ty + 16 * u][tx + 16 * v] = acc[u][v];
+    }
+  __syncthreads();
+  double w[4][4] = {};
+  tile_mm<false, NB + 1>(w, A, B);
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) wjp[int64_t(ty + 16 * u) * np + tx + 16 * v] = w[u][v];
   __syncthreads();
 }
 
@@ -224,15 +269,16 @@ __device__ void dev_chol_update(double* __restrict__ Gd, int np, int P, int p, i
   __syncthreads();
 }
 
-// Triangular inverse, diagonal d, step 1: S_ij += R_ik X_kj for one k in (i, j], j = i + d,
-// accumulated (fp64 atomics) into the still-zero block X_ij.
-__device__ void dev_trinv_sum(const double* __restrict__ Gd, double* __restrict__ Xd, int np, int i, int j, int k,
-                              int b, double* sh) {
+// Triangular inverse, block diagonal d: X_ij -= W_ik X_kj for one k in (i, j], j = i + d, with
+// W_ik = X_ii R_ik (so X_ij = -X_ii sum_k R_ik X_kj), accumulated with fp64 atomics into the
+// still-zero block X_ij.
+__device__ void dev_trinv(const double* __restrict__ Gd, double* __restrict__ Xd, int np, int i, int j, int k,
+                          int b, double* sh) {
   double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
   double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
   const double* g = Gd + int64_t(b) * np * np;
   double* x = Xd + int64_t(b) * np * np;
-  tile_load(A, g + int64_t(i) * NB * np + k * NB, np);
+  tile_load(A, g + int64_t(k) * NB * np + i * NB, np);  // W_ik, stored in block (k, i)
   tile_load(B, x + int64_t(k) * NB * np + j * NB, np);
   __syncthreads();
   double acc[4][4] = {};
@@ -242,26 +288,7 @@ __device__ void dev_trinv_sum(const double* __restrict__ Gd, double* __restrict_
 #pragma unroll
   for (int u = 0; u < 4; ++u)
 #pragma unroll
-    for (int v = 0; v < 4; ++v) atomicAdd(&xij[int64_t(ty + 16 * u) * np + tx + 16 * v], acc[u][v]);
-  __syncthreads();
-}
-
-// Step 2: X_ij = -X_ii S_ij.
-__device__ void dev_trinv_fin(double* __restrict__ Xd, int np, int i, int j, int b, double* sh) {
-  double(*A)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh);
-  double(*B)[NB + 1] = reinterpret_cast<double(*)[NB + 1]>(sh + NB * (NB + 1));
-  double* x = Xd + int64_t(b) * np * np;
-  tile_load(A, x + int64_t(i) * NB * np + i * NB, np);
-  double* xij = x + int64_t(i) * NB * np + j * NB;
-  tile_load(B, xij, np);
-  __syncthreads();
-  double acc[4][4] = {};
-  tile_mm<false, NB + 1>(acc, A, B);
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-#pragma unroll
-    for (int v = 0; v < 4; ++v) xij[int64_t(ty + 16 * u) * np + tx + 16 * v] = -acc[u][v];
+    for (int v = 0; v < 4; ++v) atomicAdd(&xij[int64_t(ty + 16 * u) * np + tx + 16 * v], -acc[u][v]);
   __syncthreads();
 }
 
@@ -274,12 +301,30 @@ struct CholArgs {
   float* ratio;
   __nv_bfloat16 *hi, *lo;
   GridBar bar;
+  unsigned long long* stamps;  // optional (diagnostics): globaltimer after each phase, block 0
 };
+
+__device__ __forceinline__ void stamp(unsigned long long* st, int& k) {
+  if (st && blockIdx.x == 0 && threadIdx.x == 0) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    st[k] = t;
+  }
+  ++k;
+}
 
 // The whole blocked Cholesky + triangular inverse of nb matrices in one cooperative launch.
 __global__ void __launch_bounds__(256) k_chol_coop(CholArgs a) {
   extern __shared__ double sh[];
   const int nbk = gridDim.x;
+  int sk = 0;
+  if (a.stamps) {  // diagnostics: cost of 100 empty grid barriers, in stamps[4000..4001]
+    int s2 = 4000;
+    stamp(a.stamps, s2);
+    for (int i = 0; i < 100; ++i) grid_barrier(a.bar);
+    stamp(a.stamps, s2);
+  }
+  stamp(a.stamps, sk);
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int64_t gw = int64_t(blockIdx.x) * nw + wid, nwt = int64_t(nbk) * nw;
   // Frobenius norms (a warp per row), pivot ratios reset
@@ -314,30 +359,37 @@ __global__ void __launch_bounds__(256) k_chol_coop(CholArgs a) {
     }
   }
   grid_barrier(a.bar);
-  for (int p = 0; p < a.P; ++p) {
-    for (int b = blockIdx.x; b < a.nb; b += nbk) dev_chol_diag(a.Gd, a.Xd, a.np, p, a.diag0, a.ratio, b, sh);
+  stamp(a.stamps, sk);
+  // block 0's diagonal factor, then per step: panel, and the trailing update in which the CTA that
+  // updates block (p+1, p+1) (its last update) factors it right away
+  for (int b = blockIdx.x; b < a.nb; b += nbk) dev_chol_diag(a.Gd, a.Xd, a.np, 0, a.diag0, a.ratio, b, sh);
+  grid_barrier(a.bar);
+  stamp(a.stamps, sk);
+  for (int p = 0; p + 1 < a.P; ++p) {
+    const int np1 = a.P - p - 1;
+    for (int it = blockIdx.x; it < a.nb * np1; it += nbk) dev_chol_panel(a.Gd, a.Xd, a.np, p, it / np1, p + 1 + it % np1, sh);
     grid_barrier(a.bar);
-    if (p + 1 < a.P) {
-      const int np1 = a.P - p - 1;
-      for (int it = blockIdx.x; it < a.nb * np1; it += nbk) dev_chol_panel(a.Gd, a.Xd, a.np, p, it / np1, p + 1 + it % np1, sh);
-      grid_barrier(a.bar);
-      const int npairs = np1 * (np1 + 1) / 2;
-      for (int it = blockIdx.x; it < a.nb * npairs; it += nbk) dev_chol_update(a.Gd, a.np, a.P, p, it / npairs, it % npairs, sh);
-      grid_barrier(a.bar);
+    stamp(a.stamps, sk);
+    const int npairs = np1 * (np1 + 1) / 2;
+    for (int it = blockIdx.x; it < a.nb * npairs; it += nbk) {
+      const int b = it / npairs, w = it % npairs;
+      dev_chol_update(a.Gd, a.np, a.P, p, b, w, sh);
+      if (w == 0) dev_chol_diag(a.Gd, a.Xd, a.np, p + 1, a.diag0, a.ratio, b, sh);
     }
+    grid_barrier(a.bar);
+    stamp(a.stamps, sk);
   }
-  // X = R^-1 by block diagonals: X_ij = -X_ii sum_{k=i+1..j} R_ik X_kj
+  // X = R^-1 by block diagonals
   for (int d = 1; d < a.P; ++d) {
     const int cnt = a.P - d;  // blocks on the diagonal
     const int items = a.nb * cnt * d;
     for (int it = blockIdx.x; it < items; it += nbk) {
       const int b = it / (cnt * d), r = it % (cnt * d);
       const int i = r / d, k = i + 1 + r % d;
-      dev_trinv_sum(a.Gd, a.Xd, a.np, i, i + d, k, b, sh);
+      dev_trinv(a.Gd, a.Xd, a.np, i, i + d, k, b, sh);
     }
     grid_barrier(a.bar);
-    for (int it = blockIdx.x; it < a.nb * cnt; it += nbk) dev_trinv_fin(a.Xd, a.np, it % cnt, it % cnt + d, it / cnt, sh);
-    grid_barrier(a.bar);
+    stamp(a.stamps, sk);
   }
   // R^-1 (upper triangle) as bf16 hi + lo, a warp per row
   for (int64_t row = gw; row < int64_t(a.nb) * a.n; row += nwt) {
@@ -350,6 +402,7 @@ __global__ void __launch_bounds__(256) k_chol_coop(CholArgs a) {
       a.lo[row * a.n + j] = __float2bfloat16_rn(v - __bfloat162float(h));
     }
   }
+  stamp(a.stamps, sk);
 }
 
 
@@ -363,6 +416,7 @@ struct JacScratch {
   double* Th;    // [nb][npair][JS][JS]
   double* norms; // [kJacMaxSweeps][nb][2] off^2, total^2
   int* perm;     // [nb][np]
+  int* skip;     // [nb][npair] this round's pair was already diagonal (rotation = identity)
   unsigned int* bar;  // [2] grid barrier count, generation
   int* sweeps;   // [1]
 };
@@ -377,6 +431,7 @@ JacScratch jac_carve(void* scratch, int nb, int n) {
   s.Th = reinterpret_cast<double*>(p); p += align_up(size_t(nb) * npair * JS * JS * 8, 256);
   s.norms = reinterpret_cast<double*>(p); p += align_up(size_t(kJacMaxSweeps) * nb * 16, 256);
   s.perm = reinterpret_cast<int*>(p); p += align_up(size_t(nb) * np * 4, 256);
+  s.skip = reinterpret_cast<int*>(p); p += align_up(size_t(nb) * npair * 4, 256);
   s.bar = reinterpret_cast<unsigned int*>(p); p += 256;
   s.sweeps = reinterpret_cast<int*>(p);
   return s;
@@ -407,16 +462,20 @@ __host__ __device__ __forceinline__ void tour_pair(int m, int r, int k, int* a, 
 
 typedef double Tile[JS][JS + 1];
 
-__device__ void dev_jac_solve(const double* __restrict__ Aw, int np, int nblk, int round, double* __restrict__ Th,
-                              int b, int k, double* jsm) {
+// thr: off-diagonal mass of the 64 x 64 subproblem at or below which the pair is left as it is
+// (its rotation recorded as the identity); negative in the first sweep.
+__device__ void dev_jac_solve(double* __restrict__ Aw, int np, int nblk, int round, double* __restrict__ Th,
+                              int* __restrict__ skip, double thr, int b, int k, double* jsm) {
   Tile& S = *reinterpret_cast<Tile*>(jsm);
   Tile& Q = *reinterpret_cast<Tile*>(jsm + JS * (JS + 1));
   __shared__ double cs[JW], sn[JW];
   __shared__ int pp[JW], qq[JW];
+  __shared__ double red[8];
+  __shared__ int s_skip;
   const int npair = nblk / 2;
   int I, J;
   tour_pair(nblk, round, k, &I, &J);
-  const double* a = Aw + int64_t(b) * np * np;
+  double* a = Aw + int64_t(b) * np * np;
   for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) {
     const int u = e / JS, v = e % JS;
     const int gu = (u < JW ? I * JW + u : J * JW + u - JW);
@@ -425,6 +484,28 @@ __device__ void dev_jac_solve(const double* __restrict__ Aw, int np, int nblk, i
     Q[u][v] = (u == v) ? 1.0 : 0.0;
   }
   __syncthreads();
+  {
+    double off = 0.0;
+    for (int e = threadIdx.x; e < JS * JS; e += blockDim.x)
+      if (e / JS != e % JS) off = fma(S[e / JS][e % JS], S[e / JS][e % JS], off);
+    for (int m = 16; m; m >>= 1) off += __shfl_xor_sync(0xffffffffu, off, m);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = off;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double t = 0.0;
+      for (int w = 0; w < int(blockDim.x >> 5); ++w) t += red[w];
+      s_skip = (thr >= 0.0 && t <= thr) ? 1 : 0;
+    }
+    __syncthreads();
+  }
+  double* th = Th + (int64_t(b) * npair + k) * JS * JS;
+  if (s_skip) {
+    for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) th[e] = (e / JS == e % JS) ? 1.0 : 0.0;
+    if (threadIdx.x == 0) skip[b * npair + k] = 1;
+    __syncthreads();
+    return;
+  }
+  if (threadIdx.x == 0) skip[b * npair + k] = 0;
   for (int r = 0; r < JS - 1; ++r) {
     if (threadIdx.x < JW) {
       int p, q;
@@ -463,13 +544,83 @@ __device__ void dev_jac_solve(const double* __restrict__ Aw, int np, int nblk, i
     }
     __syncthreads();
   }
-  double* th = Th + (int64_t(b) * npair + k) * JS * JS;
-  for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) th[e] = Q[e / JS][e % JS];
+  // the pair's diagonal block is now Theta^T S Theta: write it back (pairs of a round are disjoint)
+  for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) {
+    const int u = e / JS, v = e % JS;
+    const int gu = (u < JW ? I * JW + u : J * JW + u - JW);
+    const int gv = (v < JW ? I * JW + v : J * JW + v - JW);
+    th[e] = Q[u][v];
+    a[int64_t(gu) * np + gv] = S[u][v];
+  }
   __syncthreads();
 }
 
-// columns I u J of A and V (chunk of 64 rows per CTA): X[:, IJ] <- X[:, IJ] * Theta
-__device__ void dev_jac_cols(double* __restrict__ Aw, double* __restrict__ V, int np, int nblk, int round,
+// Off-diagonal pair-block (k1 < k2) of A: A[R1, C2] <- Theta1^T A[R1, C2] Theta2 and its mirror
+// A[C2, R1] <- the transpose (R1, C2: the 64 indices of pairs k1 and k2 in this round).
+__device__ void dev_jac_off(double* __restrict__ Aw, int np, int nblk, int round, const double* __restrict__ Th,
+                            const int* __restrict__ skip, int b, int idx, double* jsm) {
+  Tile& X = *reinterpret_cast<Tile*>(jsm);
+  Tile& T1 = *reinterpret_cast<Tile*>(jsm + JS * (JS + 1));
+  Tile& T2 = *reinterpret_cast<Tile*>(jsm + 2 * JS * (JS + 1));
+  const int npair = nblk / 2;
+  int k1 = 0;
+  while (idx >= npair - 1 - k1) {
+    idx -= npair - 1 - k1;
+    ++k1;
+  }
+  const int k2 = k1 + 1 + idx;
+  if (skip[b * npair + k1] && skip[b * npair + k2]) return;  // both rotations are the identity
+  int I1, J1, I2, J2;
+  tour_pair(nblk, round, k1, &I1, &J1);
+  tour_pair(nblk, round, k2, &I2, &J2);
+  double* a = Aw + int64_t(b) * np * np;
+  const double* th1 = Th + (int64_t(b) * npair + k1) * JS * JS;
+  const double* th2 = Th + (int64_t(b) * npair + k2) * JS * JS;
+  for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) {
+    const int u = e / JS, v = e % JS;
+    const int gu = (u < JW ? I1 * JW + u : J1 * JW + u - JW);
+    const int gv = (v < JW ? I2 * JW + v : J2 * JW + v - JW);
+    X[u][v] = a[int64_t(gu) * np + gv];
+    T1[u][v] = th1[e];
+    T2[u][v] = th2[e];
+  }
+  __syncthreads();
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[4][4] = {};
+  tile_mm<true, JS + 1>(acc, T1, X);  // Z = Theta1^T X
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) X[ty + 16 * u][tx + 16 * v] = acc[u][v];
+  __syncthreads();
+  double y[4][4] = {};
+  tile_mm<false, JS + 1>(y, X, T2);   // Y = Z Theta2
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int row = ty + 16 * u;
+    const int gu = (row < JW ? I1 * JW + row : J1 * JW + row - JW);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int col = tx + 16 * v;
+      const int gv = (col < JW ? I2 * JW + col : J2 * JW + col - JW);
+      a[int64_t(gu) * np + gv] = y[u][v];
+      X[row][col] = y[u][v];
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) {  // mirror, coalesced along R1
+    const int r = e / JS, c = e % JS;
+    const int gr = (r < JW ? I2 * JW + r : J2 * JW + r - JW);
+    const int gc = (c < JW ? I1 * JW + c : J1 * JW + c - JW);
+    a[int64_t(gr) * np + gc] = X[c][r];
+  }
+  __syncthreads();
+}
+
+// columns I u J of V (chunk of 64 rows per CTA): V[:, IJ] <- V[:, IJ] * Theta
+__device__ void dev_jac_cols(double* __restrict__ V, int np, int nblk, int round,
                              const double* __restrict__ Th, int b, int k, int chunk, double* jsm) {
   Tile& T = *reinterpret_cast<Tile*>(jsm);
   Tile& X = *reinterpret_cast<Tile*>(jsm + JS * (JS + 1));
@@ -479,8 +630,8 @@ __device__ void dev_jac_cols(double* __restrict__ Aw, double* __restrict__ V, in
   const double* th = Th + (int64_t(b) * npair + k) * JS * JS;
   for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) T[e / JS][e % JS] = th[e];
   const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
-  for (int which = 0; which < 2; ++which) {
-    double* M = (which ? V : Aw) + int64_t(b) * np * np;
+  {
+    double* M = V + int64_t(b) * np * np;
     __syncthreads();
     for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) {
       const int u = e / JS, v = e % JS;
@@ -502,38 +653,9 @@ __device__ void dev_jac_cols(double* __restrict__ Aw, double* __restrict__ V, in
   __syncthreads();
 }
 
-// rows I u J of A (chunk of 64 columns per CTA): A[IJ, :] <- Theta^T A[IJ, :]
-__device__ void dev_jac_rows(double* __restrict__ Aw, int np, int nblk, int round, const double* __restrict__ Th,
-                             int b, int k, int chunk, double* jsm) {
-  Tile& T = *reinterpret_cast<Tile*>(jsm);
-  Tile& X = *reinterpret_cast<Tile*>(jsm + JS * (JS + 1));
-  const int c0 = chunk * JS, npair = nblk / 2;
-  int I, J;
-  tour_pair(nblk, round, k, &I, &J);
-  const double* th = Th + (int64_t(b) * npair + k) * JS * JS;
-  double* M = Aw + int64_t(b) * np * np;
-  for (int e = threadIdx.x; e < JS * JS; e += blockDim.x) {
-    const int u = e / JS, v = e % JS;
-    T[u][v] = th[e];
-    const int gu = (u < JW ? I * JW + u : J * JW + u - JW);
-    X[u][v] = M[int64_t(gu) * np + c0 + v];
-  }
-  __syncthreads();
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
-  double acc[4][4] = {};
-  tile_mm<true, JS + 1>(acc, T, X);
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int row = ty + 16 * u;
-    const int gu = (row < JW ? I * JW + row : J * JW + row - JW);
-#pragma unroll
-    for (int v = 0; v < 4; ++v) M[int64_t(gu) * np + c0 + tx + 16 * v] = acc[u][v];
-  }
-  __syncthreads();
-}
-
 struct JacArgs {
   double *A, *V, *Th, *norms;  // norms [max_sweeps][nb][2], zeroed before launch
+  int* skip;
   int np, nblk, npair, chunks, nb, max_sweeps;
   double tol;
   int* sweeps_done;
@@ -547,15 +669,25 @@ __global__ void __launch_bounds__(256) k_jac_coop(JacArgs a) {
   __shared__ int s_done;
   for (int sweep = 0; sweep < a.max_sweeps; ++sweep) {
     for (int r = 0; r < a.nblk - 1; ++r) {
-      for (int it = blockIdx.x; it < a.nb * a.npair; it += nbk)
-        dev_jac_solve(a.A, a.np, a.nblk, r, a.Th, it / a.npair, it % a.npair, jsm);
+      for (int it = blockIdx.x; it < a.nb * a.npair; it += nbk) {
+        const int b = it / a.npair;
+        // a subproblem whose off-diagonal mass is below tol^2 |A|^2 / nblk^2 is left alone: the
+        // sum over all of them stays below the convergence bound tol^2 |A|^2
+        const double thr = sweep > 0 ? a.tol * a.tol * a.norms[int64_t(sweep - 1) * a.nb * 2 + 2 * b + 1] /
+                                           (double(a.nblk) * a.nblk)
+                                     : -1.0;
+        dev_jac_solve(a.A, a.np, a.nblk, r, a.Th, a.skip, thr, b, it % a.npair, jsm);
+      }
       grid_barrier(a.bar);
+      // one pass over A (off-diagonal pair-blocks, two-sided) and V (block columns)
+      const int noff = a.npair * (a.npair - 1) / 2;
       const int per = a.npair * a.chunks;
-      for (int it = blockIdx.x; it < a.nb * per; it += nbk)
-        dev_jac_cols(a.A, a.V, a.np, a.nblk, r, a.Th, it / per, (it % per) / a.chunks, (it % per) % a.chunks, jsm);
-      grid_barrier(a.bar);
-      for (int it = blockIdx.x; it < a.nb * per; it += nbk)
-        dev_jac_rows(a.A, a.np, a.nblk, r, a.Th, it / per, (it % per) / a.chunks, (it % per) % a.chunks, jsm);
+      for (int it = blockIdx.x; it < a.nb * (noff + per); it += nbk) {
+        const int b = it / (noff + per), w = it % (noff + per);
+        if (w < noff) dev_jac_off(a.A, a.np, a.nblk, r, a.Th, a.skip, b, w, jsm);
+        else if (!a.skip[b * a.npair + (w - noff) / a.chunks])
+          dev_jac_cols(a.V, a.np, a.nblk, r, a.Th, b, (w - noff) / a.chunks, (w - noff) % a.chunks, jsm);
+      }
       grid_barrier(a.bar);
     }
     // off-diagonal and total Frobenius mass of every matrix
@@ -668,8 +800,9 @@ size_t chol_scratch_bytes(int nb, int n) {
          align_up(size_t(nb) * np * 8, 256) + align_up(size_t(nb) * 4, 256) + 256;
 }
 
+// per_sm_cap: at most this many resident CTAs per SM (fewer CTAs make each grid barrier cheaper)
 template <typename K, typename A>
-jolt_status launch_coop(K kernel, const A& args, int smem, cudaStream_t st) {
+jolt_status launch_coop(K kernel, const A& args, int smem, cudaStream_t st, int per_sm_cap = 64) {
   static_assert(sizeof(A) < 4000, "kernel arguments must fit the parameter space");
   int dev = 0, sms = 0, per = 0;
   JOLT_CUDA_TRY(cudaGetDevice(&dev));
@@ -677,6 +810,7 @@ jolt_status launch_coop(K kernel, const A& args, int smem, cudaStream_t st) {
   JOLT_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   JOLT_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kernel, 256, smem));
   if (per < 1) return JOLT_ERR_CUDA;
+  per = std::min(per, per_sm_cap);
   A local = args;
   void* params[] = {&local};
   JOLT_CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kernel), dim3(sms * per), dim3(256), params,
@@ -697,6 +831,11 @@ jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shi
   a.Gd = s.Gd; a.Xd = s.Xd; a.md = s.mdiag; a.diag0 = s.diag0; a.ratio = s.ratio;
   a.hi = rinv_hi; a.lo = rinv_lo;
   a.bar = GridBar{s.bar, s.bar + 1, err};
+  // diagnostics (JOLT_DEBUG): per-phase device timestamps of block 0
+  static unsigned long long* dbg_stamps = nullptr;
+  const bool dbg = std::getenv("JOLT_DEBUG") != nullptr;
+  if (dbg && !dbg_stamps) JOLT_CUDA_TRY(cudaMalloc(&dbg_stamps, 4096 * sizeof(unsigned long long)));
+  a.stamps = dbg ? dbg_stamps : nullptr;
   jolt_status r;
   {
     // fp64 work: factor n^3/3 plus triangular inverse n^3/3 per matrix
@@ -704,6 +843,23 @@ jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shi
     r = launch_coop(k_chol_coop, a, 2 * NB * (NB + 1) * 8, st);
   }
   if (r) return r;
+  if (dbg) {
+    std::vector<unsigned long long> h(4096);
+    JOLT_CUDA_TRY(cudaMemcpyAsync(h.data(), dbg_stamps, h.size() * 8, cudaMemcpyDeviceToHost, st));
+    JOLT_CUDA_TRY(cudaStreamSynchronize(st));
+    // stamps: start, after copy, diag 0, per step (panel, update + next diag), per diagonal, end
+    const int ns = 3 + 2 * (P - 1) + (P - 1) + 1;
+    double fac[2] = {0, 0}, inv = 0;
+    int k = 3;
+    for (int p = 0; p + 1 < P; ++p)
+      for (int ph = 0; ph < 2; ++ph, ++k) fac[ph] += (h[k] - h[k - 1]) * 1e-3;
+    for (int d = 1; d < P; ++d, ++k) inv += (h[k] - h[k - 1]) * 1e-3;
+    std::fprintf(stderr,
+                 "jolt chol: n %d batch %d total %.1f us | norm+copy %.1f | diag0 %.1f panel %.1f update+diag %.1f | "
+                 "trinv %.1f | out %.1f (stamps %d) | empty grid barrier %.2f us\n",
+                 n, nb, (h[ns - 1] - h[0]) * 1e-3, (h[1] - h[0]) * 1e-3, (h[2] - h[1]) * 1e-3, fac[0], fac[1], inv,
+                 (h[ns - 1] - h[ns - 2]) * 1e-3, ns, (h[4001] - h[4000]) * 1e-5);
+  }
   if (min_ratio) {
     std::vector<float> h(nb);
     JOLT_CUDA_TRY(cudaMemcpyAsync(h.data(), s.ratio, sizeof(float) * nb, cudaMemcpyDeviceToHost, st));
@@ -718,7 +874,8 @@ jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shi
 size_t jacobi_scratch_bytes(int nb, int n) {
   const int np = rup(n, JS), npair = np / JS;
   return 2 * align_up(size_t(nb) * np * np * 8, 256) + align_up(size_t(nb) * npair * JS * JS * 8, 256) +
-         align_up(size_t(kJacMaxSweeps) * nb * 16, 256) + align_up(size_t(nb) * np * 4, 256) + 512;
+         align_up(size_t(kJacMaxSweeps) * nb * 16, 256) + align_up(size_t(nb) * np * 4, 256) +
+         align_up(size_t(nb) * npair * 4, 256) + 512;
 }
 
 template <typename TA, typename TO>
@@ -731,7 +888,7 @@ jolt_status jacobi_impl(const TA* A, int64_t ld_a, int nb, int n, TO* evals, TO*
   JOLT_CUDA_TRY(cudaMemsetAsync(s.norms, 0, size_t(kJacMaxSweeps) * nb * 16, st));
   JOLT_CUDA_TRY(cudaMemsetAsync(s.bar, 0, 2 * sizeof(unsigned int), st));
   JacArgs a;
-  a.A = s.A; a.V = s.V; a.Th = s.Th; a.norms = s.norms;
+  a.A = s.A; a.V = s.V; a.Th = s.Th; a.norms = s.norms; a.skip = s.skip;
   a.np = np; a.nblk = nblk; a.npair = npair; a.chunks = chunks; a.nb = nb;
   a.max_sweeps = std::min(max_sweeps, kJacMaxSweeps);
   a.tol = tol;
@@ -740,7 +897,7 @@ jolt_status jacobi_impl(const TA* A, int64_t ld_a, int nb, int n, TO* evals, TO*
   jolt_status r;
   {
     StatScope sc(JOLT_K_EIG, st, 0.0, 0.0);
-    r = launch_coop(k_jac_coop, a, 2 * JS * (JS + 1) * 8, st);
+    r = launch_coop(k_jac_coop, a, 3 * JS * (JS + 1) * 8, st);
   }
   if (r) return r;
   if (std::getenv("JOLT_DEBUG")) {
