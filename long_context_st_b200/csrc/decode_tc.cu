@@ -18,6 +18,8 @@
 // the U_T rows plus the rotated-query residual term; values from the softmax-weighted U_T, the
 // core and U_d plus the inverse-rotated residual; RoPE re-applied per token for pre-RoPE keys).
 #include <algorithm>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -41,9 +43,10 @@ template <int NT>
 struct KeysCfg {
   static constexpr int kStages = NT == 1 ? 4 : 3;
   static constexpr int kStageBytes = kABytes + NT * kBBytes;
-  static constexpr int kQsBytes = 2 * kMaxG * kD * 4;      // queries of two pairs, fp32
-  static constexpr int kRopeBytes = kD / 2 * kBM * 8;      // (cos, sin) per frequency and token
+  static constexpr int kQsBytes = 2 * kMaxG * kD * 4;      // queries of each epilogue group's pair, fp32
+  static constexpr int kRopeBytes = kD / 4 * kBM * 16;     // (cos, cos, sin, sin) of frequency pairs
   static constexpr int kSmem = 1024 + kStages * kStageBytes + kQsBytes + kRopeBytes + kD * 4 + 256;
+  static constexpr int kThreads = 320;                     // producer, MMA, two groups of four epilogue warps
 };
 
 struct KeysMaps {
@@ -65,7 +68,8 @@ struct KeysArgs {
   int32_t* err;
 };
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier of one epilogue group (ids 1 and 2; 0 is __syncthreads).
+__device__ __forceinline__ void group_bar(int g) { asm volatile("bar.sync %0, 128;" ::"r"(1 + g) : "memory"); }
 
 // Residual row of one token: 128 codes of BITS bits (little-endian bit stream) as floats.
 template <int BITS>
@@ -85,9 +89,10 @@ __device__ __forceinline__ void load_codes(const uint8_t* row, float (&v)[kD]) {
   for (int j = 0; j < kD; ++j) v[j] = float((w[(j * BITS) >> 5] >> ((j * BITS) & 31)) & mask);
 }
 
-// Same row dequantised: code * scale + zero (fp32 fused multiply-add).
+// Same row dequantised (code * scale + zero, one fp32 fused multiply-add per code), as 64 packed
+// pairs of consecutive features.
 template <int BITS>
-__device__ __forceinline__ void load_dequant(const uint8_t* row, float sc, float zr, float (&v)[kD]) {
+__device__ __forceinline__ void load_dequant2(const uint8_t* row, float sc, float zr, float2 (&v)[kD / 2]) {
   constexpr uint32_t mask = (1u << BITS) - 1u;
   uint32_t w[4 * BITS + 1];
   const uint4* r4 = reinterpret_cast<const uint4*>(row);
@@ -99,35 +104,53 @@ __device__ __forceinline__ void load_dequant(const uint8_t* row, float sc, float
     w[4 * i + 2] = x.z;
     w[4 * i + 3] = x.w;
   }
+  const float2 sc2 = make_float2(sc, sc), zr2 = make_float2(zr, zr);
 #pragma unroll
-  for (int j = 0; j < kD; ++j) v[j] = dequant((w[(j * BITS) >> 5] >> ((j * BITS) & 31)) & mask, sc, zr);
+  for (int m = 0; m < kD / 2; ++m) {
+    const int j0 = 2 * m, j1 = 2 * m + 1;
+    const float c0 = float((w[(j0 * BITS) >> 5] >> ((j0 * BITS) & 31)) & mask);
+    const float c1 = float((w[(j1 * BITS) >> 5] >> ((j1 * BITS) & 31)) & mask);
+    v[m] = __ffma2_rn(make_float2(c0, c1), sc2, zr2);
+  }
 }
 
-__device__ __forceinline__ void fwht128(float (&v)[kD]) {
+// Unnormalised Walsh-Hadamard transform of 128 values held as 64 packed pairs: the stride-1
+// butterflies inside each pair, the wider strides pair-wise (a - b computed as b * -1 + a, exact
+// in both forms), stages in increasing stride as in the scalar form.
+__device__ __forceinline__ void fwht128x2(float2 (&v)[kD / 2]) {
 #pragma unroll
-  for (int s = 1; s < kD; s <<= 1) {
+  for (int m = 0; m < kD / 2; ++m) {
+    const float a = v[m].x, c = v[m].y;
+    v[m] = make_float2(a + c, a - c);
+  }
+  const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
-    for (int i = 0; i < kD; ++i) {
-      if ((i & s) == 0) {
-        const float a = v[i], c = v[i + s];
-        v[i] = a + c;
-        v[i + s] = a - c;
+  for (int sm = 1; sm < kD / 2; sm <<= 1) {
+#pragma unroll
+    for (int m = 0; m < kD / 2; ++m) {
+      if ((m & sm) == 0) {
+        const float2 a = v[m], c = v[m + sm];
+        v[m] = __fadd2_rn(a, c);
+        v[m + sm] = __ffma2_rn(c, neg1, a);
       }
     }
   }
 }
 
-// grid.x = token tiles; 192 threads: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner),
-// warps 2..5 epilogue (warp w reads TMEM lanes 32 * (w % 4) .. +31, i.e. token rows of the tile).
+// grid.x = token tiles; 320 threads (three warps share some SM sub-partitions, whose register files
+// hold 16384 registers each, so at most 168 registers a thread): warp 0 TMA producer, warp 1 MMA
+// issuer (+ TMEM owner),
+// warps 2..5 and 6..9 two epilogue groups taking alternate (layer, head) pairs and TMEM buffers
+// (warp w reads TMEM lanes 32 * (w % 4) .. +31, i.e. token rows of the tile).
 template <int BITS, int NT>
-__global__ void __launch_bounds__(192, 1) k_keys_tc(const __grid_constant__ KeysMaps maps, const KeysArgs p) {
+__global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ KeysMaps maps, const KeysArgs p) {
   using C = KeysCfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* qs = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);  // [2][kMaxG][kD]
-  float2* rope = reinterpret_cast<float2*>(qs + 2 * kMaxG * kD);            // [64][kBM]
-  float* sgn = reinterpret_cast<float*>(rope + kD / 2 * kBM);                 // [kD]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sgn + kD);
+  float* qs = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);  // [2 groups][kMaxG][kD]
+  float4* rope = reinterpret_cast<float4*>(qs + 2 * kMaxG * kD);            // [32][kBM]
+  float2* sgn = reinterpret_cast<float2*>(rope + kD / 4 * kBM);               // [64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sgn + kD / 2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 5);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -158,16 +181,22 @@ __global__ void __launch_bounds__(192, 1) k_keys_tc(const __grid_constant__ Keys
       for (int t = 0; t < NT; ++t) sm100::prefetch_tmap(&maps.b[t]);
     }
   }
-  if (threadIdx.x < kD) sgn[threadIdx.x] = rsqrtf(float(kD)) * rot_sign(p.rot_seed, threadIdx.x);
+  if (threadIdx.x < kD / 2) {
+    const float isd = rsqrtf(float(kD));
+    sgn[threadIdx.x] = make_float2(isd * rot_sign(p.rot_seed, 2 * threadIdx.x), isd * rot_sign(p.rot_seed, 2 * threadIdx.x + 1));
+  }
   // RoPE of the tile's tokens: cos / sin of (pos0 + t) * inv_freq[f], angle reduced mod 2 pi in
-  // fp64, times the attention scaling
-  for (int e = threadIdx.x; e < kD / 2 * kBM; e += blockDim.x) {
-    const int f = e / kBM, tt = e % kBM;
-    const double ang = double(p.pos0 + t0 + tt) * double(p.inv_freq[f]);
-    const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
-    float sn, cs;
-    sincosf(float(red), &sn, &cs);
-    rope[e] = make_float2(cs * p.rope_scaling, sn * p.rope_scaling);
+  // fp64, times the attention scaling; frequencies 2m and 2m + 1 side by side
+  for (int e = threadIdx.x; e < kD / 4 * kBM; e += blockDim.x) {
+    const int m = e / kBM, tt = e % kBM;
+    float cs[2], sn[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const double ang = double(p.pos0 + t0 + tt) * double(p.inv_freq[2 * m + u]);
+      const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+      sincosf(float(red), &sn[u], &cs[u]);
+    }
+    rope[e] = make_float4(cs[0] * p.rope_scaling, cs[1] * p.rope_scaling, sn[0] * p.rope_scaling, sn[1] * p.rope_scaling);
   }
   if (warp == 1) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), 256);
   sm100::tc_fence_before();
@@ -206,7 +235,7 @@ __global__ void __launch_bounds__(192, 1) k_keys_tc(const __grid_constant__ Keys
     }
   } else if (warp == 1) {
     if (lane == 0 && fac) {
-      // ---- MMA issuer: D[bi] = sum_k U_T[t][k] (B_hi + B_lo)[k][:] ----
+      // ---- MMA issuer: D[pr % 2] = sum_k U_T[t][k] (B_hi + B_lo)[k][:] ----
       constexpr uint32_t idesc = sm100::idesc_bf16_f32(kBM, kD, 0, 1);
       int it = 0;
       bool ok = true;
@@ -241,69 +270,72 @@ __global__ void __launch_bounds__(192, 1) k_keys_tc(const __grid_constant__ Keys
       sm100::mbar_wait(drain_bar, 0, p.err);
     }
   } else {
-    // ---- epilogue: thread = token row of the tile ----
+    // ---- epilogue: group g takes pairs g, g + 2, ... (TMEM buffer g); thread = token row ----
+    const int g = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int et = threadIdx.x - 64;
+    const int et = threadIdx.x - 64 - 128 * g;
     const int t = t0 + row;
     const bool valid = t < p.T;
+    float* qb = qs + g * kMaxG * kD;
     bool live = true;
-    for (int pr = 0; pr < npairs; ++pr) {
-      const int li = pr / p.n_kv, h = pr % p.n_kv, bi = pr & 1;
-      float* qb = qs + bi * kMaxG * kD;
+    for (int pr = g; pr < npairs; pr += 2) {
+      const int li = pr / p.n_kv, h = pr % p.n_kv;
       const __nv_bfloat16* qsrc = p.q + (int64_t(li) * p.n_q + int64_t(h) * p.gq) * kD;
       for (int e = et; e < p.gq * kD; e += 128) qb[e] = __bfloat162float(qsrc[e]);
-      epi_bar();
-      float v[kD];
+      group_bar(g);
+      float2 v[kD / 2];
       if (BITS > 0 && valid) {
         const int64_t rr = (int64_t(li) * p.n_kv + h) * p.T + t;
         const __half2 szv = p.sz[rr];
-        load_dequant<BITS>(p.codes + rr * (kD * BITS / 8), __low2float(szv), __high2float(szv), v);
-        fwht128(v);
+        load_dequant2<BITS>(p.codes + rr * (kD * BITS / 8), __low2float(szv), __high2float(szv), v);
+        fwht128x2(v);
 #pragma unroll
-        for (int j = 0; j < kD; ++j) v[j] *= sgn[j];
+        for (int m = 0; m < kD / 2; ++m) v[m] = __fmul2_rn(v[m], sgn[m]);
       } else {
 #pragma unroll
-        for (int j = 0; j < kD; ++j) v[j] = 0.f;
+        for (int m = 0; m < kD / 2; ++m) v[m] = make_float2(0.f, 0.f);
       }
       if (fac) {
-        if (live) live = sm100::mbar_wait(tfull_bar(bi), (pr >> 1) & 1, p.err);
+        if (live) live = sm100::mbar_wait(tfull_bar(g), (pr >> 1) & 1, p.err);
         sm100::tc_fence_after();
 #pragma unroll
         for (int c = 0; c < kD / 16; ++c) {
           uint32_t r[16];
-          sm100::tmem_ld16(tmem + bi * kD + c * 16 + (uint32_t(quarter * 32) << 16), r);
+          sm100::tmem_ld16(tmem + g * kD + c * 16 + (uint32_t(quarter * 32) << 16), r);
           sm100::tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[c * 16 + j] += __uint_as_float(r[j]);
+          for (int k = 0; k < 8; ++k)
+            v[c * 8 + k] = __fadd2_rn(v[c * 8 + k], make_float2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])));
         }
         sm100::tc_fence_before();
-        sm100::mbar_arrive(tempty_bar(bi));
+        sm100::mbar_arrive(tempty_bar(g));
       }
       if (valid && live) {
 #pragma unroll
-        for (int f = 0; f < kD / 2; ++f) {
-          const float2 csn = rope[f * kBM + row];
-          const float x1 = v[f], x2 = v[f + kD / 2];
-          v[f] = x1 * csn.x - x2 * csn.y;
-          v[f + kD / 2] = x2 * csn.x + x1 * csn.y;
+        for (int m = 0; m < kD / 4; ++m) {  // features (2m, 2m+1) with (2m+64, 2m+65)
+          const float4 r4 = rope[m * kBM + row];
+          const float2 cs = make_float2(r4.x, r4.y), sn = make_float2(r4.z, r4.w);
+          const float2 x1 = v[m], x2 = v[m + kD / 4];
+          const float2 a = __fmul2_rn(x2, sn), b = __fmul2_rn(x1, sn);
+          v[m] = __ffma2_rn(x1, cs, make_float2(-a.x, -a.y));
+          v[m + kD / 4] = __ffma2_rn(x2, cs, b);
         }
         float* out = p.scores + (int64_t(li) * p.n_q + int64_t(h) * p.gq) * p.T + t;
 #pragma unroll 1
-        for (int g = 0; g < p.gq; ++g) {
-          const float4* qg = reinterpret_cast<const float4*>(qb + g * kD);
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        for (int gg = 0; gg < p.gq; ++gg) {
+          const float4* qg = reinterpret_cast<const float4*>(qb + gg * kD);
+          float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int j = 0; j < kD; j += 4) {
-            const float4 qq = qg[j >> 2];
-            a0 = fmaf(v[j], qq.x, a0);
-            a1 = fmaf(v[j + 1], qq.y, a1);
-            a2 = fmaf(v[j + 2], qq.z, a2);
-            a3 = fmaf(v[j + 3], qq.w, a3);
+          for (int k = 0; k < kD / 4; ++k) {
+            const float4 qq = qg[k];
+            a0 = __ffma2_rn(v[2 * k], make_float2(qq.x, qq.y), a0);
+            a1 = __ffma2_rn(v[2 * k + 1], make_float2(qq.z, qq.w), a1);
           }
-          out[int64_t(g) * p.T] = ((a0 + a1) + (a2 + a3)) * p.attn_scale;
+          out[int64_t(gg) * p.T] = ((a0.x + a0.y) + (a1.x + a1.y)) * p.attn_scale;
         }
       }
+      group_bar(g);  // every thread is done with this pair's queries
     }
   }
   sm100::tc_fence_before();
@@ -575,10 +607,22 @@ TcWs tc_layout(const jolt_shape& s, int Lc) {
 template <int BITS, int NT>
 jolt_status launch_keys(const KeysMaps& maps, const KeysArgs& a, cudaStream_t st) {
   auto kern = k_keys_tc<BITS, NT>;
+  cudaFuncAttributes fa;
+  JOLT_CUDA_TRY(cudaFuncGetAttributes(&fa, kern));
+  if (fa.maxThreadsPerBlock < KeysCfg<NT>::kThreads) {  // the block would not fit the register file
+    if (std::getenv("JOLT_DEBUG"))
+      std::fprintf(stderr, "jolt: k_keys_tc needs %d threads, registers allow %d (%d per thread)\n",
+                   KeysCfg<NT>::kThreads, fa.maxThreadsPerBlock, fa.numRegs);
+    return JOLT_ERR_CUDA;
+  }
   JOLT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, KeysCfg<NT>::kSmem));
   const int ntiles = (a.T + kBM - 1) / kBM;
-  kern<<<ntiles, 192, KeysCfg<NT>::kSmem, st>>>(maps, a);
-  JOLT_CUDA_TRY(cudaGetLastError());
+  kern<<<ntiles, KeysCfg<NT>::kThreads, KeysCfg<NT>::kSmem, st>>>(maps, a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    if (std::getenv("JOLT_DEBUG")) std::fprintf(stderr, "jolt: k_keys_tc launch: %s\n", cudaGetErrorString(e));
+    return JOLT_ERR_CUDA;
+  }
   return JOLT_OK;
 }
 
