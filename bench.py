@@ -248,21 +248,29 @@ class Step:
         return choices
 
 
-def decode_bytes(w, shape, choices):
-    """Algorithmic bytes one full decode step reads and writes (per-layer schedule)."""
-    sf, io = w.factor_bytes, w.io_bytes
+def decode_work(w, shape, choices):
+    """Algorithmic work of one decode step over every layer: (bytes, tensor flops).
+
+    Bytes: the compressed cache read once (each cell's U_T, U_d, cores, codes and scale/zero
+    pairs) plus q and the output. Flops: the dense contractions the attention cannot avoid on the
+    tensor-core path — per (layer, KV head) the pre-RoPE key rebuild U_T^K B_h (two bf16 terms of
+    B_h) or the non-RoPE score product P U_T^K^T (two terms of P), and P~ U_T^V per layer."""
+    from long_context_st_b200 import api
     G = w.n_layers // w.layers_per_group
-    tot = 0
+    nbytes = sum(api.cell_bytes(shape, tuple(c)) for c in choices)
+    nbytes += w.batch * w.n_layers * 2 * w.n_q * w.d_h * w.io_bytes
+    flops = 0.0
     for b in range(w.batch):
-        for l in range(w.n_layers):
-            g = l // w.layers_per_group
-            for kv in range(2):
-                rT, rd, bb = choices[(b * G + g) * 2 + kv]
-                tot += sf * (w.T * rT + w.d_h * rd + w.n_kv * rT * rd)
-                if bb:
-                    tot += w.n_kv * w.T * (w.d_h * bb // 8 + 4)
-            tot += 2 * w.n_q * w.d_h * io
-    return tot
+        for g in range(G):
+            rk = choices[(b * G + g) * 2][0]
+            rv = choices[(b * G + g) * 2 + 1][0]
+            for _ in range(w.layers_per_group):
+                if w.keys_pre_rope:
+                    flops += 2 * 2.0 * w.T * rk * w.d_h * w.n_kv
+                else:
+                    flops += 2 * 2.0 * w.n_q * w.T * rk
+                flops += 2.0 * w.n_q * w.T * rv
+    return nbytes, flops
 
 
 def count_kernels(step):
@@ -357,7 +365,7 @@ def main():
     tokens = w.batch * w.T
     value = tokens * world / (ms_step / 1e3)
     raw = 2 * w.batch * w.n_layers * w.n_kv * w.T * w.d_h * w.io_bytes
-    dbytes = decode_bytes(w, step.shape, step.choices)
+    dbytes, dflops = decode_work(w, step.shape, step.choices)
     _, cache_total = api.cache_layout(step.shape, step.choices)
 
     def fam_roof(name, bound, peak):
@@ -408,7 +416,13 @@ def main():
             "decode": {"context_tokens_per_s": tokens * w.n_layers / (t_dec / 1e3) if t_dec > 0 else None,
                        "context_tokens_per_s_per_layer_step": tokens / (t_dec / 1e3) if t_dec > 0 else None,
                        "hbm_gbs": dbytes / (t_dec / 1e3) / 1e9 if t_dec > 0 else None,
-                       "alg_bytes": dbytes, "frac_of_hbm": dbytes / (t_dec / 1e3) / 1e9 / hbm_peak if t_dec > 0 else None},
+                       "alg_bytes": dbytes, "frac_of_hbm": dbytes / (t_dec / 1e3) / 1e9 / hbm_peak if t_dec > 0 else None,
+                       "tensor_flops": dflops,
+                       "tensor_tflops": dflops / (t_dec / 1e3) / 1e12 if t_dec > 0 else None,
+                       # the step's own roofline: the slower of its HBM bytes and its tensor flops
+                       "roofline_ms": max(dbytes / hbm_peak / 1e6, dflops / tc_sust / 1e9),
+                       "bound": "tensor" if dflops / tc_sust / 1e9 > dbytes / hbm_peak / 1e6 else "hbm",
+                       "frac_of_roofline": max(dbytes / hbm_peak / 1e6, dflops / tc_sust / 1e9) / t_dec if t_dec > 0 else None},
             "roofline": roof, "roofline_decode": roof_dec,
             "kernel_stats": {k: {kk: (float(vv) if isinstance(vv, float) else int(vv)) for kk, vv in v.items()}
                              for k, v in stats.items()},
