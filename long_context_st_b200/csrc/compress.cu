@@ -456,6 +456,7 @@ jolt_status orth(const Ctx& c, float* Y, int rows, int C) {
     g.C = Gm; g.ldc = l; g.c_batch_stride = int64_t(l) * l; g.batch = C;
     g.k_split = ksplit_for(int64_t((l + 127) / 128) * ((l + 255) / 256) * C, rows);
     g.accumulate = true; g.err = c.err;
+    g.c_upper = true;  // symmetric: the Cholesky reads the upper triangle
     if ((r = gemm_tc(g, c.st))) return r;
     if (std::getenv("JOLT_DEBUG")) {
       std::vector<float> h(size_t(C) * l * l);
@@ -503,6 +504,7 @@ jolt_status orth(const Ctx& c, float* Y, int rows, int C) {
     t.A[1] = ykh; t.B[1] = rl;
     t.A[2] = ykl; t.B[2] = rh;
     t.C = Y; t.ldc = l; t.c_batch_stride = int64_t(rows) * l; t.batch = C; t.err = c.err;
+    t.b_upper = true;  // R^-1 is upper triangular
     if ((r = gemm_tc(t, c.st))) return r;
     if (shift == 0.0 && ratio >= 0.9f) return JOLT_OK;
     if (ratio >= 0.1f) conditioned = true;
@@ -662,6 +664,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       g.A[2] = zl; g.B[2] = zh;
       g.C = W; g.ldc = l; g.c_batch_stride = int64_t(l) * l; g.batch = C;
       g.k_split = ksplit_for(int64_t((l + 127) / 128) * ((l + 255) / 256) * C, n); g.accumulate = true; g.err = c.err;
+      g.c_upper = true;  // symmetric: the eigensolver reads the upper triangle
       if ((r = gemm_tc(g, c.st))) return r;
     }
     float* ev = c.at<float>(p.ev);

@@ -456,13 +456,17 @@ struct ValArgs {
   float* acc;                 // [nl][n_q][128], rotated domain
 };
 
-// acc[h'][j] += sum_t P~[h'][t] deq(code_t[j]). grid (token chunks, n_kv, nl); thread = feature j.
+// acc[h'][j] += sum_t P~[h'][t] deq(code_t[j]) (rotated domain). grid (token chunks, n_kv, nl),
+// thread = feature j; every 128-token sub-tile stages its code rows (16-byte loads), scale/zero
+// pairs and probabilities in shared memory first.
+template <int BITS>
 __global__ void __launch_bounds__(128) k_values_res(const ValArgs a) {
-  __shared__ float pr[kMaxG][128];
+  constexpr int RB = kD * BITS / 8;  // bytes of one code row
+  __shared__ __align__(16) uint8_t cs[128][RB];
+  __shared__ __align__(16) float pr[128][kMaxG];
   __shared__ float2 szs[128];
   const int h = blockIdx.y, li = blockIdx.z, j = threadIdx.x;
   const int64_t qrow0 = int64_t(li) * a.n_q + int64_t(h) * a.gq;
-  const int nbytes = kD * a.bits / 8;
   const int64_t rbase = (int64_t(li) * a.n_kv + h) * a.T;
   float acc[kMaxG];
 #pragma unroll
@@ -471,22 +475,34 @@ __global__ void __launch_bounds__(128) k_values_res(const ValArgs a) {
   for (int tb = t_beg; tb < t_end; tb += 128) {
     const int nt = min(128, t_end - tb);
     __syncthreads();
-    for (int e = threadIdx.x; e < a.gq * 128; e += blockDim.x) {
-      const int g = e >> 7, tt = e & 127;
-      pr[g][tt] = tt < nt ? __bfloat162float(a.ptil[(qrow0 + g) * a.ldp + tb + tt]) : 0.f;
-    }
     if (threadIdx.x < nt) {
-      const __half2 szv = a.sz[rbase + tb + threadIdx.x];
+      const int64_t rr = rbase + tb + threadIdx.x;
+      const uint4* src = reinterpret_cast<const uint4*>(a.codes + rr * RB);
+#pragma unroll
+      for (int q = 0; q < RB / 16; ++q) reinterpret_cast<uint4*>(cs[threadIdx.x])[q] = __ldg(src + q);
+      const __half2 szv = a.sz[rr];
       szs[threadIdx.x] = make_float2(__low2float(szv), __high2float(szv));
-    }
-    __syncthreads();
-    const uint8_t* crow = a.codes + (rbase + tb) * nbytes;
-    for (int tt = 0; tt < nt; ++tt) {
-      const float2 z = szs[tt];
-      const float dv = dequant(unpack_code(crow + int64_t(tt) * nbytes, j, a.bits), z.x, z.y);
 #pragma unroll
       for (int g = 0; g < kMaxG; ++g)
-        if (g < a.gq) acc[g] = fmaf(pr[g][tt], dv, acc[g]);
+        pr[threadIdx.x][g] = g < a.gq ? __bfloat162float(a.ptil[(qrow0 + g) * a.ldp + tb + threadIdx.x]) : 0.f;
+    }
+    __syncthreads();
+    const int byte = (j * BITS) >> 3, shift = (j * BITS) & 7;
+    for (int tt = 0; tt < nt; ++tt) {
+      const uint32_t code = (uint32_t(cs[tt][byte]) >> shift) & ((1u << BITS) - 1u);
+      const float2 z = szs[tt];
+      const float dv = dequant(code, z.x, z.y);
+      const float4* p4 = reinterpret_cast<const float4*>(pr[tt]);
+#pragma unroll
+      for (int g4 = 0; g4 < kMaxG / 4; ++g4) {
+        if (4 * g4 < a.gq) {
+          const float4 w = p4[g4];
+          acc[4 * g4 + 0] = fmaf(w.x, dv, acc[4 * g4 + 0]);
+          acc[4 * g4 + 1] = fmaf(w.y, dv, acc[4 * g4 + 1]);
+          acc[4 * g4 + 2] = fmaf(w.z, dv, acc[4 * g4 + 2]);
+          acc[4 * g4 + 3] = fmaf(w.w, dv, acc[4 * g4 + 3]);
+        }
+      }
     }
   }
 #pragma unroll
@@ -507,59 +523,48 @@ struct FinArgs {
   float* lse;                // [nl][n_q] or null
 };
 
-// grid (n_kv, nl), 128 threads; dynamic smem: w [gq][r_T] + v [gq][r_d] + x [gq][128] floats.
+// out = (U_d^V (G_h^V^T w) + R^T acc) / l, lse = m + log l for one query head.
+// grid (n_kv, nl, g_q), 128 threads; dynamic smem: w [r_T] floats.
 __global__ void __launch_bounds__(128) k_finalize(const FinArgs a) {
-  extern __shared__ float fs[];
-  const int h = blockIdx.x, li = blockIdx.y, tid = threadIdx.x;
-  const int64_t qrow0 = int64_t(li) * a.n_q + int64_t(h) * a.gq;
-  float* w = fs;
-  float* v = w + a.gq * a.r_T;
-  float* x = v + a.gq * a.r_d;
-  for (int e = tid; e < a.gq * a.r_T; e += blockDim.x) w[e] = a.W[(qrow0 + e / a.r_T) * a.q_cap + e % a.r_T];
-  for (int e = tid; e < a.gq * kD; e += blockDim.x) x[e] = a.bits ? a.acc[qrow0 * kD + e] : 0.f;
+  extern __shared__ float w[];
+  __shared__ float v[kD];
+  __shared__ float x[kD];
+  const int h = blockIdx.x, li = blockIdx.y, g = blockIdx.z, tid = threadIdx.x;
+  const int64_t qr = int64_t(li) * a.n_q + int64_t(h) * a.gq + g;
+  for (int r = tid; r < a.r_T; r += blockDim.x) w[r] = a.W[qr * a.q_cap + r];
+  x[tid] = a.bits ? a.acc[qr * kD + tid] : 0.f;
   __syncthreads();
-  // v[g][j] = sum_r G[r][j] w[g][r]
+  // v[j] = sum_r G[r][j] w[r]
+  if (tid < a.r_d) {
+    const __nv_bfloat16* G = a.G + (int64_t(li) * a.n_kv + h) * a.r_T * a.r_d + tid;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    int r = 0;
+    for (; r + 4 <= a.r_T; r += 4) {
+      s0 = fmaf(__bfloat162float(G[int64_t(r) * a.r_d]), w[r], s0);
+      s1 = fmaf(__bfloat162float(G[int64_t(r + 1) * a.r_d]), w[r + 1], s1);
+      s2 = fmaf(__bfloat162float(G[int64_t(r + 2) * a.r_d]), w[r + 2], s2);
+      s3 = fmaf(__bfloat162float(G[int64_t(r + 3) * a.r_d]), w[r + 3], s3);
+    }
+    for (; r < a.r_T; ++r) s0 = fmaf(__bfloat162float(G[int64_t(r) * a.r_d]), w[r], s0);
+    v[tid] = (s0 + s1) + (s2 + s3);
+  }
+  // inverse rotation of the residual accumulator (one warp)
+  if (a.bits && tid < 32) {
+    float xv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xv[i] = x[tid * 4 + i];
+    warp_unrotate<4>(xv, a.rot_seed, rsqrtf(float(kD)));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[tid * 4 + i] = xv[i];
+  }
+  __syncthreads();
+  float o = x[tid];
   if (a.r_T > 0) {
-    const __nv_bfloat16* G = a.G + (int64_t(li) * a.n_kv + h) * a.r_T * a.r_d;
-    for (int j = tid; j < a.r_d; j += blockDim.x) {
-      float acc[kMaxG];
-#pragma unroll
-      for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
-      for (int r = 0; r < a.r_T; ++r) {
-        const float gv = __bfloat162float(G[int64_t(r) * a.r_d + j]);
-#pragma unroll
-        for (int g = 0; g < kMaxG; ++g)
-          if (g < a.gq) acc[g] = fmaf(gv, w[g * a.r_T + r], acc[g]);
-      }
-#pragma unroll
-      for (int g = 0; g < kMaxG; ++g)
-        if (g < a.gq) v[g * a.r_d + j] = acc[g];
-    }
+    const __nv_bfloat16* ud = a.Ud + int64_t(tid) * a.r_d;
+    for (int jj = 0; jj < a.r_d; ++jj) o = fmaf(__bfloat162float(ud[jj]), v[jj], o);
   }
-  // inverse rotation of the residual accumulators, one warp per query head
-  if (a.bits) {
-    const int wid = tid >> 5, ln = tid & 31;
-    for (int g = wid; g < a.gq; g += 4) {
-      float xv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) xv[i] = x[g * kD + ln * 4 + i];
-      warp_unrotate<4>(xv, a.rot_seed, rsqrtf(float(kD)));
-#pragma unroll
-      for (int i = 0; i < 4; ++i) x[g * kD + ln * 4 + i] = xv[i];
-    }
-  }
-  __syncthreads();
-  const int i = tid;
-  for (int g = 0; g < a.gq; ++g) {
-    float o = x[g * kD + i];
-    if (a.r_T > 0) {
-      const __nv_bfloat16* ud = a.Ud + int64_t(i) * a.r_d;
-      for (int jj = 0; jj < a.r_d; ++jj) o = fmaf(__bfloat162float(ud[jj]), v[g * a.r_d + jj], o);
-    }
-    const int64_t qr = qrow0 + g;
-    a.out[qr * kD + i] = __float2bfloat16_rn(o / a.lrow[qr]);
-    if (i == 0 && a.lse) a.lse[qr] = a.mrow[qr] + logf(a.lrow[qr]);
-  }
+  a.out[qr * kD + tid] = __float2bfloat16_rn(o / a.lrow[qr]);
+  if (tid == 0 && a.lse) a.lse[qr] = a.mrow[qr] + logf(a.lrow[qr]);
 }
 
 int grid1(int64_t n) { return int(std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 148 * 16))); }
@@ -791,7 +796,10 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
         va.codes = cv.codes + res_off * (kD * cv.bits / 8);
         va.sz = cv.sz + res_off;
         va.ptil = ptil; va.acc = acc;
-        k_values_res<<<dim3((T + va.chunk - 1) / va.chunk, n_kv, nl), 128, 0, st>>>(va);
+        const dim3 vg((T + va.chunk - 1) / va.chunk, n_kv, nl);
+        if (cv.bits == 2) k_values_res<2><<<vg, 128, 0, st>>>(va);
+        else if (cv.bits == 4) k_values_res<4><<<vg, 128, 0, st>>>(va);
+        else k_values_res<8><<<vg, 128, 0, st>>>(va);
         JOLT_CUDA_TRY(cudaGetLastError());
       }
       // ---- finalize ----
@@ -803,9 +811,7 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
       fa.W = W; fa.acc = acc; fa.mrow = mrow; fa.lrow = lrow;
       fa.out = oall + row0 * kD;
       fa.lse = p.lse ? p.lse + row0 : nullptr;
-      const size_t fsm = size_t(gq) * (cv.r_T + cv.r_d + kD) * 4;
-      JOLT_CUDA_TRY(cudaFuncSetAttribute(k_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, int(std::max<size_t>(fsm, 1))));
-      k_finalize<<<dim3(n_kv, nl), 128, fsm, st>>>(fa);
+      k_finalize<<<dim3(n_kv, nl, gq), 128, size_t(std::max(cv.r_T, 1)) * 4, st>>>(fa);
       JOLT_CUDA_TRY(cudaGetLastError());
     }
   }

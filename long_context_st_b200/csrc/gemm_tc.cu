@@ -36,7 +36,7 @@ struct GemmDev {
   int a_batch[kMaxTerms], b_batch[kMaxTerms];  // operand batch extents (coordinate = z % extent)
   float* C;
   int64_t ldc, c_bstride;
-  int c_div, accumulate;
+  int c_div, accumulate, c_upper, b_upper;
   int32_t* err;
 };
 
@@ -83,8 +83,10 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM * MT;
+  if (p.c_upper && m0 >= n0 + BN) return;  // whole tile below the diagonal (uniform per CTA)
   const int z = blockIdx.z / p.k_split, kz = blockIdx.z % p.k_split;
-  const int nkb_total = (p.K + BK - 1) / BK;
+  const int nkb_all = (p.K + BK - 1) / BK;
+  const int nkb_total = p.b_upper ? min(nkb_all, (n0 + BN + BK - 1) / BK) : nkb_all;
   const int kb_begin = kz * p.nkb_split;
   const int nkb = max(0, min(p.nkb_split, nkb_total - kb_begin));
   const int n_iters = nkb * p.n_terms;
@@ -300,13 +302,17 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   d.nkb_split = (nkb + g.k_split - 1) / g.k_split;
   d.C = g.C; d.ldc = g.ldc; d.c_bstride = g.c_batch_stride; d.c_div = g.c_batch_div;
   d.accumulate = g.accumulate ? 1 : 0;
+  d.c_upper = g.c_upper ? 1 : 0;
+  d.b_upper = g.b_upper ? 1 : 0;
   d.err = g.err;
   // two 128-row tiles per CTA when that still leaves at least two CTAs per SM
   const int64_t ntile = (g.N + BN - 1) / BN, zc = int64_t(g.batch) * g.k_split;
   const int MT = (g.M > BM && ntile * ((g.M + 2 * BM - 1) / (2 * BM)) * zc >= 2 * 148) ? 2 : 1;
   const dim3 grid(unsigned(ntile), unsigned((g.M + BM * MT - 1) / (BM * MT)), unsigned(zc));
   if (grid.y > 65535 || grid.z > 65535) return JOLT_ERR_INVALID_ARG;
-  StatScope sc(JOLT_K_GEMM, st, 2.0 * g.M * double(g.N) * g.K * g.batch * g.n_terms, 0.0);
+  // algorithmic flops: a triangular B or a wanted upper triangle of C halves the product
+  const double tri = (g.b_upper || g.c_upper) ? 0.5 : 1.0;
+  StatScope sc(JOLT_K_GEMM, st, tri * 2.0 * g.M * double(g.N) * g.K * g.batch * g.n_terms, 0.0);
   if (MT == 2) return BN == 256 ? launch_bn<256, 2>(am, bm, maps, d, grid, st) : launch_bn<128, 2>(am, bm, maps, d, grid, st);
   return BN == 256 ? launch_bn<256, 1>(am, bm, maps, d, grid, st) : launch_bn<128, 1>(am, bm, maps, d, grid, st);
 }

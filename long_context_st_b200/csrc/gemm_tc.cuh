@@ -39,6 +39,8 @@ struct GemmCall {
   int batch = 1;               // operand batch entries (grid z)
   int k_split = 1;             // split-K factor; > 1 (or c_batch_div > 1) requires accumulate
   bool accumulate = false;     // atomically add into C instead of storing
+  bool c_upper = false;        // only C[m][n] with m <= n is wanted: skip tiles entirely below the diagonal
+  bool b_upper = false;        // B[k][n] = 0 for k > n (upper triangular): K stops at the tile's last column
   int32_t* err = nullptr;
 };
 

@@ -332,9 +332,9 @@ __global__ void __launch_bounds__(256) k_chol_coop(CholArgs a) {
     const int b = int(row / a.n), i = int(row % a.n);
     const float* g = a.G + int64_t(b) * a.n * a.ldg + int64_t(i) * a.ldg;
     double m = 0.0;
-    for (int j = lane; j < a.n; j += 32) {
+    for (int j = i + lane; j < a.n; j += 32) {  // upper triangle, off-diagonal entries twice
       const double v = g[j];
-      m = fma(v, v, m);
+      m = fma(j > i ? 2.0 * v : v, v, m);
     }
     for (int o = 16; o; o >>= 1) m += __shfl_xor_sync(0xffffffffu, m, o);
     if (lane == 0) atomicAdd(a.md + b, m);
@@ -351,7 +351,8 @@ __global__ void __launch_bounds__(256) k_chol_coop(CholArgs a) {
     double* xd = a.Xd + row * a.np;
     for (int j = lane; j < a.np; j += 32) {
       double v;
-      if (i < a.n && j < a.n) v = double(g[j]) + (i == j ? shift : 0.0);
+      if (i < a.n && j < a.n)  // symmetric input: only its upper triangle is read
+        v = double(j >= i ? g[j] : a.G[int64_t(b) * a.n * a.ldg + int64_t(j) * a.ldg + i]) + (i == j ? shift : 0.0);
       else v = (i == j) ? 1.0 : 0.0;
       gd[j] = v;
       xd[j] = 0.0;
@@ -446,7 +447,7 @@ __global__ void k_jac_init(const TA* __restrict__ A, int64_t lda, int n, int np,
     const int i = int(e / np), j = int(e % np);
     double v;
     if (i < n && j < n)
-      v = 0.5 * (double(A[int64_t(b) * n * lda + int64_t(i) * lda + j]) + double(A[int64_t(b) * n * lda + int64_t(j) * lda + i]));
+      v = double(i <= j ? A[int64_t(b) * n * lda + int64_t(i) * lda + j] : A[int64_t(b) * n * lda + int64_t(j) * lda + i]);
     else v = (i == j) ? -1.0 : 0.0;
     Aw[int64_t(b) * total + e] = v;
     V[int64_t(b) * total + e] = (i == j) ? 1.0 : 0.0;
