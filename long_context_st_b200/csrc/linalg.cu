@@ -761,16 +761,38 @@ __global__ void k_jac_out(const double* __restrict__ V, int np, int n, const int
   }
 }
 
+// Strided rows: a warp per row.
 __global__ void k_split(const float* __restrict__ x, int64_t ldx, int64_t rows, int64_t cols, int64_t bsx,
                         __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo, int64_t ldo, int64_t bso) {
+  const int b = blockIdx.y, lane = threadIdx.x & 31;
+  const int64_t nw = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += nw) {
+    const float* xr = x + b * bsx + r * ldx;
+    __nv_bfloat16* hr = hi + b * bso + r * ldo;
+    __nv_bfloat16* lr = lo ? lo + b * bso + r * ldo : nullptr;
+    for (int64_t c = lane; c < cols; c += 32) {
+      const float v = xr[c];
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      hr[c] = h;
+      if (lr) lr[c] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
+  }
+}
+
+// Contiguous rows (ldx = ldo = cols), 4 values per thread: one 16-byte load, two 8-byte stores.
+__global__ void k_split_vec(const float4* __restrict__ x, int64_t n4, int64_t bsx4, uint2* __restrict__ hi,
+                            uint2* __restrict__ lo, int64_t bso4) {
   const int b = blockIdx.y;
-  const int64_t total = rows * cols;
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = e / cols, c = e % cols;
-    const float v = x[b * bsx + r * ldx + c];
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    hi[b * bso + r * ldo + c] = h;
-    if (lo) lo[b * bso + r * ldo + c] = __float2bfloat16_rn(v - __bfloat162float(h));
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n4; e += int64_t(gridDim.x) * blockDim.x) {
+    const float4 v = x[b * bsx4 + e];
+    const __nv_bfloat162 h01 = __floats2bfloat162_rn(v.x, v.y), h23 = __floats2bfloat162_rn(v.z, v.w);
+    hi[b * bso4 + e] = make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+    if (lo) {
+      const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+      const __nv_bfloat162 l01 = __floats2bfloat162_rn(v.x - f01.x, v.y - f01.y);
+      const __nv_bfloat162 l23 = __floats2bfloat162_rn(v.z - f23.x, v.w - f23.y);
+      lo[b * bso4 + e] = make_uint2(*reinterpret_cast<const uint32_t*>(&l01), *reinterpret_cast<const uint32_t*>(&l23));
+    }
   }
 }
 
@@ -934,7 +956,18 @@ jolt_status split3_bf16(const float* x, int64_t n, __nv_bfloat16* hi, __nv_bfloa
 jolt_status split_bf16(const float* x, int64_t ldx, int64_t rows, int64_t cols, int batch, int64_t bstride_x,
                        __nv_bfloat16* hi, __nv_bfloat16* lo, int64_t ldo, int64_t bstride_o, cudaStream_t st) {
   if (rows <= 0 || cols <= 0) return JOLT_OK;
-  k_split<<<dim3(grid_1d(rows * cols), batch), 256, 0, st>>>(x, ldx, rows, cols, bstride_x, hi, lo, ldo, bstride_o);
+  const int64_t n = rows * cols;
+  const bool vec = ldx == cols && ldo == cols && n % 4 == 0 && bstride_x % 4 == 0 && bstride_o % 4 == 0 &&
+                   reinterpret_cast<uintptr_t>(x) % 16 == 0 && reinterpret_cast<uintptr_t>(hi) % 8 == 0 &&
+                   (!lo || reinterpret_cast<uintptr_t>(lo) % 8 == 0);
+  if (vec) {
+    const int gx = int(std::max<int64_t>(1, std::min<int64_t>((n / 4 + 255) / 256, 148 * 8 / std::max(1, batch) + 1)));
+    k_split_vec<<<dim3(gx, batch), 256, 0, st>>>(reinterpret_cast<const float4*>(x), n / 4, bstride_x / 4,
+                                                 reinterpret_cast<uint2*>(hi), reinterpret_cast<uint2*>(lo), bstride_o / 4);
+  } else {
+    const int gx = int(std::max<int64_t>(1, std::min<int64_t>((rows + 7) / 8, 148 * 8)));
+    k_split<<<dim3(gx, batch), 256, 0, st>>>(x, ldx, rows, cols, bstride_x, hi, lo, ldo, bstride_o);
+  }
   JOLT_CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
 }
