@@ -433,7 +433,10 @@ Operand xunfold(const void* X, int major, const Plan& p, int C) {
 // an unshifted factorisation falls back to a shifted pass. At most kMaxOrthPasses passes.
 constexpr int kMaxOrthPasses = 8;
 
-jolt_status orth(const Ctx& c, float* Y, int rows, int C) {
+// polish = false (inside the power iterations): stop after the first pass whose pivots show a
+// well-conditioned input (ratio >= 0.1); its output is orthonormal to within the shift's effect,
+// which is all the next product needs. The final basis (polish = true) gets the unshifted passes.
+jolt_status orth(const Ctx& c, float* Y, int rows, int C, bool polish = true) {
   const Plan& p = c.p;
   const int l = p.l;
   __nv_bfloat16* Yh = c.at<__nv_bfloat16>(p.Yh);
@@ -507,6 +510,7 @@ jolt_status orth(const Ctx& c, float* Y, int rows, int C) {
     t.b_upper = true;  // R^-1 is upper triangular
     if ((r = gemm_tc(t, c.st))) return r;
     if (shift == 0.0 && ratio >= 0.9f) return JOLT_OK;
+    if (!polish && ratio >= 0.1f) return JOLT_OK;
     if (ratio >= 0.1f) conditioned = true;
   }
   return JOLT_OK;
@@ -611,7 +615,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       if ((r = gemm_tc(g, c.st))) return r;
     }
     for (int it = 0; it < s.power_iters; ++it) {
-      if ((r = orth(c, Y, T, C))) return r;
+      if ((r = orth(c, Y, T, C, false))) return r;
       if ((r = split_bf16(Y, l, T, l, C, int64_t(T) * l, Yh, nullptr, l, int64_t(T) * l, c.st))) return r;
       JOLT_CUDA_TRY(cudaMemsetAsync(Z, 0, size_t(C) * n * l * 4, c.st));
       GemmCall g;
@@ -621,7 +625,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       g.C = Z; g.ldc = l; g.c_batch_stride = int64_t(n) * l; g.batch = C;
       g.k_split = ksplit_for(int64_t((n + 127) / 128) * ((l + 255) / 256) * C, T); g.accumulate = true; g.err = c.err;
       if ((r = gemm_tc(g, c.st))) return r;
-      if ((r = orth(c, Z, n, C))) return r;
+      if ((r = orth(c, Z, n, C, false))) return r;
       if ((r = split_bf16(Z, l, n, l, C, int64_t(n) * l, Zh, nullptr, l, int64_t(n) * l, c.st))) return r;
       GemmCall h;
       h.M = T; h.N = l; h.K = n;
