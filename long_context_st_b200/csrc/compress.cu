@@ -371,13 +371,6 @@ __global__ void k_diag_blocks(const double* __restrict__ G, int n, int d, int nb
 
 int grid1(int64_t n) { return int(std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 148 * 16))); }
 
-int ksplit_for(int64_t tiles, int64_t K) {
-  int64_t want = (2 * 148 + tiles - 1) / tiles;
-  const int64_t kblocks = (K + 63) / 64;
-  want = std::min<int64_t>(want, std::max<int64_t>(1, kblocks / 8));
-  return int(std::max<int64_t>(1, std::min<int64_t>(want, 64)));
-}
-
 struct Ctx {
   const jolt_shape* s;
   Plan p;
@@ -457,7 +450,7 @@ jolt_status orth(const Ctx& c, float* Y, int rows, int C, bool polish = true) {
     g.A[1] = yh; g.B[1] = yl;
     g.A[2] = yl; g.B[2] = yh;
     g.C = Gm; g.ldc = l; g.c_batch_stride = int64_t(l) * l; g.batch = C;
-    g.k_split = ksplit_for(int64_t((l + 127) / 128) * ((l + 255) / 256) * C, rows);
+    g.k_split = 0;
     g.accumulate = true; g.err = c.err;
     g.c_upper = true;  // symmetric: the Cholesky reads the upper triangle
     if ((r = gemm_tc(g, c.st))) return r;
@@ -557,7 +550,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       g.A[2] = xl; g.B[2] = xh;
     }
     g.C = Sd; g.ldc = d; g.c_batch_stride = int64_t(d) * d; g.c_batch_div = p.LgH;
-    g.batch = C * p.LgH; g.k_split = ksplit_for(int64_t(C) * p.LgH, T); g.accumulate = true; g.err = c.err;
+    g.batch = C * p.LgH; g.k_split = 0; g.accumulate = true; g.err = c.err;
     if ((r = gemm_tc(g, c.st))) return r;
   }
   const bool exact = (p.l == p.n);
@@ -623,7 +616,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       g.A[0] = xunfold(Xb, kMajorMN, p, C);
       g.B[0] = plain(Yh, kMajorMN, l, T, l, C, int64_t(T) * l);
       g.C = Z; g.ldc = l; g.c_batch_stride = int64_t(n) * l; g.batch = C;
-      g.k_split = ksplit_for(int64_t((n + 127) / 128) * ((l + 255) / 256) * C, T); g.accumulate = true; g.err = c.err;
+      g.k_split = 0; g.accumulate = true; g.err = c.err;
       if ((r = gemm_tc(g, c.st))) return r;
       if ((r = orth(c, Z, n, C, false))) return r;
       if ((r = split_bf16(Z, l, n, l, C, int64_t(n) * l, Zh, nullptr, l, int64_t(n) * l, c.st))) return r;
@@ -651,7 +644,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
         g.B[2] = g.B[0];
       }
       g.C = Z; g.ldc = l; g.c_batch_stride = int64_t(n) * l; g.batch = C;
-      g.k_split = ksplit_for(int64_t((n + 127) / 128) * ((l + 255) / 256) * C, T); g.accumulate = true; g.err = c.err;
+      g.k_split = 0; g.accumulate = true; g.err = c.err;
       if ((r = gemm_tc(g, c.st))) return r;
     }
     // W = B B^T = (B^T)^T (B^T), hi/lo terms
@@ -667,7 +660,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       g.A[1] = zh; g.B[1] = zl;
       g.A[2] = zl; g.B[2] = zh;
       g.C = W; g.ldc = l; g.c_batch_stride = int64_t(l) * l; g.batch = C;
-      g.k_split = ksplit_for(int64_t((l + 127) / 128) * ((l + 255) / 256) * C, n); g.accumulate = true; g.err = c.err;
+      g.k_split = 0; g.accumulate = true; g.err = c.err;
       g.c_upper = true;  // symmetric: the eigensolver reads the upper triangle
       if ((r = gemm_tc(g, c.st))) return r;
     }
@@ -859,7 +852,7 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
         g.A[nt] = plain(f32 ? um : ul, kMajorMN, rT, T, rT, LgH, 0); g.B[nt] = xh; ++nt;
         g.n_terms = nt;
         g.C = ylh; g.ldc = d; g.c_batch_stride = int64_t(rT) * d; g.batch = LgH;
-        g.k_split = ksplit_for(int64_t((rT + 127) / 128) * LgH, T); g.accumulate = true; g.err = c.err;
+        g.k_split = 0; g.accumulate = true; g.err = c.err;
         if ((r = gemm_tc(g, c.st))) return r;
       }
       // S_Y, U_d

@@ -782,9 +782,7 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
         gc.A[0] = op(ptil, kMajorK, T, rows, Tp);
         gc.B[0] = op(cv.Ut, kMajorMN, cv.r_T, T, cv.r_T);
         gc.C = W; gc.ldc = qc; gc.err = p.err;
-        const int64_t tiles = int64_t((rows + 127) / 128) * ((cv.r_T + 127) / 128);
-        const int64_t nkb = (T + 63) / 64;
-        gc.k_split = int(std::max<int64_t>(1, std::min<int64_t>((2 * 148 + tiles - 1) / tiles, nkb / 8)));
+        gc.k_split = 0;  // split K to fill whole waves
         gc.accumulate = true;
         if ((r = gemm_tc(gc, st))) return r;
       }

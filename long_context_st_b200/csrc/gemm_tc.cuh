@@ -37,7 +37,8 @@ struct GemmCall {
   int64_t c_batch_stride = 0;  // elements between C batch entries
   int c_batch_div = 1;         // C entry of operand batch z is z / c_batch_div
   int batch = 1;               // operand batch entries (grid z)
-  int k_split = 1;             // split-K factor; > 1 (or c_batch_div > 1) requires accumulate
+  int k_split = 1;             // split-K factor; 0 = chosen to fill whole waves; != 1 (or
+                               // c_batch_div > 1) requires accumulate
   bool accumulate = false;     // atomically add into C instead of storing
   bool c_upper = false;        // only C[m][n] with m <= n is wanted: skip tiles entirely below the diagonal
   bool b_upper = false;        // B[k][n] = 0 for k > n (upper triangular): K stops at the tile's last column
