@@ -666,7 +666,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
     }
     float* ev = c.at<float>(p.ev);
     float* evec = c.at<float>(p.evec);
-    if ((r = jacobi_eig(W, l, C, l, ev, evec, c.pass() + p.jac, 30, 1e-8, c.err, c.st))) return r;
+    if ((r = jacobi_eig(W, l, C, l, ev, evec, c.pass() + p.jac, 30, 1e-6, c.err, c.st))) return r;
     __nv_bfloat16* Vh = c.at<__nv_bfloat16>(p.Vh);
     __nv_bfloat16* Vl = c.at<__nv_bfloat16>(p.Vl);
     if ((r = split_bf16(evec, l, l, l, C, int64_t(l) * l, Vh, Vl, l, int64_t(l) * l, c.st))) return r;

@@ -514,11 +514,21 @@ __device__ void dev_jac_solve(double* __restrict__ Aw, int np, int nblk, int rou
       if (p > q) { const int t = p; p = q; q = t; }
       const double apq = S[p][q], app = S[p][p], aqq = S[q][q];
       double c = 1.0, s = 0.0;
-      if (apq != 0.0 && fabs(apq) > 1e-300) {
-        const double theta = (aqq - app) / (2.0 * apq);
-        const double t = (theta >= 0.0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
-        c = 1.0 / sqrt(t * t + 1.0);
-        s = t * c;
+      // Rotation angle in fp32 (tan t of the annihilating angle, small-angle form for huge
+      // cot 2phi), then (c, s) renormalised in fp64 by one Newton step of 1/sqrt(c^2 + s^2) so the
+      // rotation is orthogonal to fp64 rounding; an fp32 angle only leaves ~1e-7 of a_pq behind,
+      // which later rotations remove. (The fp64 divide/sqrt chain was the solve's critical path.)
+      const float af = float(apq);
+      if (af != 0.f) {
+        const float th = float(aqq - app) / (2.f * af);
+        const float at = fabsf(th);
+        const float tt = at > 1e18f ? 0.5f / at : 1.f / (at + sqrtf(fmaf(at, at, 1.f)));
+        const float t = th >= 0.f ? tt : -tt;
+        const float c32 = rsqrtf(fmaf(t, t, 1.f));
+        const double cd = c32, sd = double(t * c32);
+        const double corr = 1.5 - 0.5 * fma(cd, cd, sd * sd);
+        c = cd * corr;
+        s = sd * corr;
       }
       cs[threadIdx.x] = c; sn[threadIdx.x] = s; pp[threadIdx.x] = p; qq[threadIdx.x] = q;
     }
@@ -657,6 +667,7 @@ __device__ void dev_jac_cols(double* __restrict__ V, int np, int nblk, int round
 struct JacArgs {
   double *A, *V, *Th, *norms;  // norms [max_sweeps][nb][2], zeroed before launch
   int* skip;
+  unsigned long long* stamps;  // optional (diagnostics): [0] solve ns, [1] update ns, [2] norm ns
   int np, nblk, npair, chunks, nb, max_sweeps;
   double tol;
   int* sweeps_done;
@@ -670,6 +681,8 @@ __global__ void __launch_bounds__(256) k_jac_coop(JacArgs a) {
   __shared__ int s_done;
   for (int sweep = 0; sweep < a.max_sweeps; ++sweep) {
     for (int r = 0; r < a.nblk - 1; ++r) {
+      unsigned long long tr0 = 0, tr1 = 0, tr2 = 0;
+      if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tr0));
       for (int it = blockIdx.x; it < a.nb * a.npair; it += nbk) {
         const int b = it / a.npair;
         // a subproblem whose off-diagonal mass is below tol^2 |A|^2 / nblk^2 is left alone: the
@@ -680,6 +693,7 @@ __global__ void __launch_bounds__(256) k_jac_coop(JacArgs a) {
         dev_jac_solve(a.A, a.np, a.nblk, r, a.Th, a.skip, thr, b, it % a.npair, jsm);
       }
       grid_barrier(a.bar);
+      if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tr1));
       // one pass over A (off-diagonal pair-blocks, two-sided) and V (block columns)
       const int noff = a.npair * (a.npair - 1) / 2;
       const int per = a.npair * a.chunks;
@@ -690,6 +704,11 @@ __global__ void __launch_bounds__(256) k_jac_coop(JacArgs a) {
           dev_jac_cols(a.V, a.np, a.nblk, r, a.Th, b, (w - noff) / a.chunks, (w - noff) % a.chunks, jsm);
       }
       grid_barrier(a.bar);
+      if (a.stamps && blockIdx.x == 0 && threadIdx.x == 0) {
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tr2));
+        a.stamps[0] += tr1 - tr0;
+        a.stamps[1] += tr2 - tr1;
+      }
     }
     // off-diagonal and total Frobenius mass of every matrix
     double* nm = a.norms + int64_t(sweep) * a.nb * 2;
@@ -917,6 +936,11 @@ jolt_status jacobi_impl(const TA* A, int64_t ld_a, int nb, int n, TO* evals, TO*
   a.tol = tol;
   a.sweeps_done = s.sweeps;
   a.bar = GridBar{s.bar, s.bar + 1, err};
+  static unsigned long long* jdbg = nullptr;
+  const bool dbg = std::getenv("JOLT_DEBUG") != nullptr;
+  if (dbg && !jdbg) JOLT_CUDA_TRY(cudaMalloc(&jdbg, 4 * sizeof(unsigned long long)));
+  if (dbg) JOLT_CUDA_TRY(cudaMemsetAsync(jdbg, 0, 4 * sizeof(unsigned long long), st));
+  a.stamps = dbg ? jdbg : nullptr;
   jolt_status r;
   {
     StatScope sc(JOLT_K_EIG, st, 0.0, 0.0);
@@ -927,7 +951,10 @@ jolt_status jacobi_impl(const TA* A, int64_t ld_a, int nb, int n, TO* evals, TO*
     int sw = 0;
     JOLT_CUDA_TRY(cudaMemcpyAsync(&sw, s.sweeps, sizeof(int), cudaMemcpyDeviceToHost, st));
     JOLT_CUDA_TRY(cudaStreamSynchronize(st));
-    std::fprintf(stderr, "jolt jacobi: n %d batch %d sweeps %d\n", n, nb, sw);
+    unsigned long long h[4] = {0, 0, 0, 0};
+    JOLT_CUDA_TRY(cudaMemcpy(h, jdbg, sizeof(h), cudaMemcpyDeviceToHost));
+    std::fprintf(stderr, "jolt jacobi: n %d batch %d sweeps %d | solve %.1f us update %.1f us\n", n, nb, sw,
+                 h[0] * 1e-3, h[1] * 1e-3);
   }
   k_jac_sort<<<dim3((n + 255) / 256, nb), 256, 0, st>>>(s.A, np, n, evals, s.perm);
   k_jac_out<<<dim3(grid_1d(int64_t(n) * n), nb), 256, 0, st>>>(s.V, np, n, s.perm, evecs);
