@@ -47,6 +47,10 @@ struct Plan {
   size_t uh, ul, um, ylh, sy, evy, evecy, ud, blh, bh, bm, bl, xt, jac2;
 };
 
+// jolt_compress handles cells in chunks of this many: per chunk one batched eigensolver launch for
+// the feature-mode Grams S_Y of all its cells.
+constexpr int kCmpChunk = 8;
+
 Plan make_plan(const jolt_shape& s) {
   Plan p{};
   p.T = s.T;
@@ -105,17 +109,17 @@ Plan make_plan(const jolt_shape& s) {
   p.uh = relc(T * q * 2);
   p.ul = relc(T * q * 2);
   p.um = relc(T * q * 2);
-  p.ylh = relc(size_t(p.LgH) * q * d * 4);
-  p.sy = relc(d * d * 4);
-  p.evy = relc(d * 4);
-  p.evecy = relc(d * d * 4);
+  p.ylh = relc(size_t(kCmpChunk) * p.LgH * q * d * 4);
+  p.sy = relc(size_t(kCmpChunk) * d * d * 4);
+  p.evy = relc(size_t(kCmpChunk) * d * 4);
+  p.evecy = relc(size_t(kCmpChunk) * d * d * 4);
   p.ud = relc(d * d * 4);
   p.blh = relc(size_t(p.LgH) * q * d * 4);
   p.bh = relc(size_t(p.LgH) * q * d * 2);
   p.bm = relc(size_t(p.LgH) * q * d * 2);
   p.bl = relc(size_t(p.LgH) * q * d * 2);
   p.xt = relc(size_t(p.LgH) * T * d * 4);
-  p.jac2 = relc(jacobi_scratch_bytes(1, int(d)));
+  p.jac2 = relc(jacobi_scratch_bytes(kCmpChunk, int(d)));
   p.total = off;
   return p;
 }
@@ -810,26 +814,34 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
   const bool io32 = s.io_dtype == JOLT_F32, f32 = s.factor_dtype == JOLT_F32;
   const int T = p.T, d = p.d, q = p.qcap, LgH = p.LgH;
   uint8_t* cb = static_cast<uint8_t*>(cache);
-  for (int cell = 0; cell < nc; ++cell) {
-    const int bg = cell / 2, kv = cell % 2;
-    const jolt_cell_choice ch = choices[cell];
-    const uint8_t* Xk = static_cast<const uint8_t*>(kv ? v : k) + int64_t(bg) * p.cell_elems * (io32 ? 4 : 2);
-    float* Xt = nullptr;
-    if (ch.r_T > 0) {
-      const int rT = ch.r_T, rd = ch.r_d;
-      const float* U = reinterpret_cast<const float*>(c.ws + p.off_ut) + int64_t(cell) * T * q;
-      uint8_t* cut = cb + offs[5 * cell + 0];
-      uint8_t* cud = cb + offs[5 * cell + 1];
-      uint8_t* cg = cb + offs[5 * cell + 2];
-      // GEMM parts of U: hi (the stored value for bf16 factors), lo (and mid for fp32 factors)
-      __nv_bfloat16* uh = f32 ? c.atc<__nv_bfloat16>(p.uh) : reinterpret_cast<__nv_bfloat16*>(cut);
-      __nv_bfloat16* ul = c.atc<__nv_bfloat16>(p.ul);
-      __nv_bfloat16* um = f32 ? c.atc<__nv_bfloat16>(p.um) : nullptr;
-      k_store_ut<<<grid1(int64_t(T) * rT), 256, 0, c.st>>>(U, T, q, rT, f32, cut, f32 ? uh : nullptr, um, ul);
-      // the cell's X as bf16 for the tensor cores (f32 inputs: a bf16 copy in the X~ region first)
+  // U's GEMM parts for one cell: hi (the stored value for bf16 factors), lo (and mid for fp32 factors)
+  auto store_u = [&](int cell, int rT, __nv_bfloat16*& uh, __nv_bfloat16*& ul, __nv_bfloat16*& um) {
+    const float* U = reinterpret_cast<const float*>(c.ws + p.off_ut) + int64_t(cell) * T * q;
+    uint8_t* cut = cb + offs[5 * cell + 0];
+    uh = f32 ? c.atc<__nv_bfloat16>(p.uh) : reinterpret_cast<__nv_bfloat16*>(cut);
+    ul = c.atc<__nv_bfloat16>(p.ul);
+    um = f32 ? c.atc<__nv_bfloat16>(p.um) : nullptr;
+    k_store_ut<<<grid1(int64_t(T) * rT), 256, 0, c.st>>>(U, T, q, rT, f32, cut, f32 ? uh : nullptr, um, ul);
+  };
+  for (int c0 = 0; c0 < nc; c0 += kCmpChunk) {
+    const int c1 = std::min(nc, c0 + kCmpChunk);
+    // ---- per cell: Y_lh = U_T^T X_lh [LgH][rT][d] and S_Y (slot = rank among the chunk's
+    // cells with r_T > 0) ----
+    int nact = 0;
+    int slot_of[kCmpChunk];
+    for (int cell = c0; cell < c1; ++cell) {
+      const jolt_cell_choice ch = choices[cell];
+      slot_of[cell - c0] = -1;
+      if (ch.r_T <= 0) continue;
+      const int slot = nact++;
+      slot_of[cell - c0] = slot;
+      const int bg = cell / 2, kv = cell % 2, rT = ch.r_T;
+      const uint8_t* Xk = static_cast<const uint8_t*>(kv ? v : k) + int64_t(bg) * p.cell_elems * (io32 ? 4 : 2);
+      __nv_bfloat16 *uh, *ul, *um;
+      store_u(cell, rT, uh, ul, um);
+      // the cell's X as bf16 for the tensor cores (f32 inputs: hi + lo copies first)
       const void* Xb = Xk;
       const void* Xlo = nullptr;
-      float* xt = c.atc<float>(p.xt);
       if (io32) {
         __nv_bfloat16* xh = c.at<__nv_bfloat16>(p.xb);
         __nv_bfloat16* xl = xh + p.cell_elems;
@@ -837,8 +849,7 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
         Xb = xh;
         Xlo = xl;
       }
-      // Y_lh = U_T^T X_lh  [LgH][rT][d]
-      float* ylh = c.atc<float>(p.ylh);
+      float* ylh = c.atc<float>(p.ylh) + int64_t(slot) * LgH * q * d;
       JOLT_CUDA_TRY(cudaMemsetAsync(ylh, 0, size_t(LgH) * rT * d * 4, c.st));
       {
         // projection with the unrounded basis: (U_hi, X_hi) + (U_hi, X_lo) + (U_2nd, X_hi)
@@ -855,67 +866,89 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
         g.k_split = 0; g.accumulate = true; g.err = c.err;
         if ((r = gemm_tc(g, c.st))) return r;
       }
-      // S_Y, U_d
-      float* sy = c.atc<float>(p.sy);
+      float* sy = c.atc<float>(p.sy) + int64_t(slot) * d * d;
       JOLT_CUDA_TRY(cudaMemsetAsync(sy, 0, size_t(d) * d * 4, c.st));
       {
         const int nrows = LgH * rT;
         const int gx = std::max(1, std::min(64, nrows / 256));
         k_gram_small<<<dim3(gx, (d + 31) / 32, (d + 31) / 32), 256, 32 * 64 * 4, c.st>>>(ylh, nrows, d, sy);
       }
-      float* evy = c.atc<float>(p.evy);
-      float* evecy = c.atc<float>(p.evecy);
-      if ((r = jacobi_eig(sy, d, 1, d, evy, evecy, c.ws + p.off_cmp + p.jac2, 30, 1e-8, c.err, c.st))) return r;
-      // U_d = first rd eigenvector columns (stored dtype), then G = Y U_d (stored dtype)
-      k_store_ut<<<grid1(int64_t(d) * rd), 256, 0, c.st>>>(evecy, d, d, rd, f32, cud, nullptr, nullptr, nullptr);
-      k_proj_small<<<grid1(int64_t(LgH) * rT * rd), 256, 0, c.st>>>(ylh, int64_t(LgH) * rT, d, evecy, d, rd, f32, cg);
-      // B_lh = G U_d^T from stored values (hi/lo), then X~ = U_T B_lh
-      // X~ = U^s B with B = G^s U_d^s^T, to fp32 accuracy: 3-way bf16 splits, terms of order <= 2
-      __nv_bfloat16* bh = c.atc<__nv_bfloat16>(p.bh);
-      __nv_bfloat16* bm = c.atc<__nv_bfloat16>(p.bm);
-      __nv_bfloat16* bl = c.atc<__nv_bfloat16>(p.bl);
-      float* blh = c.atc<float>(p.blh);
-      k_recon_b<<<grid1(int64_t(LgH) * rT * d), 256, 0, c.st>>>(cg, cud, int64_t(LgH) * rT, rd, d, f32, blh);
-      if ((r = split3_bf16(blh, int64_t(LgH) * rT * d, bh, bm, bl, c.st))) return r;
-      {
-        GemmCall g;
-        g.M = T; g.N = d; g.K = rT;
-        const Operand Bp[3] = {plain(bh, kMajorMN, d, rT, d, LgH, int64_t(rT) * d),
-                               plain(bm, kMajorMN, d, rT, d, LgH, int64_t(rT) * d),
-                               plain(bl, kMajorMN, d, rT, d, LgH, int64_t(rT) * d)};
-        const Operand Up[3] = {plain(uh, kMajorK, rT, T, rT, LgH, 0), plain(um, kMajorK, rT, T, rT, LgH, 0),
-                               plain(ul, kMajorK, rT, T, rT, LgH, 0)};
-        const int nu = f32 ? 3 : 1;
-        int nt = 0;
-        for (int i = 0; i < nu; ++i)
-          for (int j = 0; j < 3; ++j)
-            if (i + j <= 2) {
-              g.A[nt] = Up[i];
-              g.B[nt] = Bp[j];
-              ++nt;
-            }
-        g.n_terms = nt;
-        g.C = xt; g.ldc = d; g.c_batch_stride = int64_t(T) * d; g.batch = LgH; g.err = c.err;
-        if ((r = gemm_tc(g, c.st))) return r;
-      }
-      Xt = xt;
     }
-    if (ch.b > 0) {
-      uint8_t* codes = cb + offs[5 * cell + 3];
-      __half2* sz = reinterpret_cast<__half2*>(cb + offs[5 * cell + 4]);
-      const int64_t rows = int64_t(LgH) * T;
-      const int grid = int(std::min<int64_t>((rows + 7) / 8, 148 * 16));
-      // algorithmic bytes: read X (io dtype) and X~ (fp32, when present), write codes and sz
-      StatScope sc(JOLT_K_RESIDUAL, c.st, 0.0,
-                   double(rows) * d * ((io32 ? 4 : 2) + (Xt ? 4 : 0)) + double(rows) * (d * ch.b / 8 + 4));
-      if (d == 128) {
-        if (io32) k_residual<4, float><<<grid, 256, 0, c.st>>>(reinterpret_cast<const float*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
-        else k_residual<4, __nv_bfloat16><<<grid, 256, 0, c.st>>>(reinterpret_cast<const __nv_bfloat16*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
-      } else {
-        if (io32) k_residual<2, float><<<grid, 256, 0, c.st>>>(reinterpret_cast<const float*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
-        else k_residual<2, __nv_bfloat16><<<grid, 256, 0, c.st>>>(reinterpret_cast<const __nv_bfloat16*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
+    // ---- the chunk's S_Y eigenproblems in one launch ----
+    float* evy = c.atc<float>(p.evy);
+    float* evecy = c.atc<float>(p.evecy);
+    if (nact > 0 &&
+        (r = jacobi_eig(c.atc<float>(p.sy), d, nact, d, evy, evecy, c.ws + p.off_cmp + p.jac2, 30, 1e-8, c.err, c.st)))
+      return r;
+    // ---- per cell: U_d, G, X~, residual ----
+    for (int cell = c0; cell < c1; ++cell) {
+      const int bg = cell / 2, kv = cell % 2;
+      const jolt_cell_choice ch = choices[cell];
+      const uint8_t* Xk = static_cast<const uint8_t*>(kv ? v : k) + int64_t(bg) * p.cell_elems * (io32 ? 4 : 2);
+      float* Xt = nullptr;
+      if (ch.r_T > 0) {
+        const int rT = ch.r_T, rd = ch.r_d, slot = slot_of[cell - c0];
+        uint8_t* cud = cb + offs[5 * cell + 1];
+        uint8_t* cg = cb + offs[5 * cell + 2];
+        __nv_bfloat16 *uh, *ul, *um;
+        if (f32) store_u(cell, rT, uh, ul, um);  // the scratch parts were overwritten by later cells
+        else {
+          uh = reinterpret_cast<__nv_bfloat16*>(cb + offs[5 * cell + 0]);
+          ul = um = nullptr;
+        }
+        const float* ylh = c.atc<float>(p.ylh) + int64_t(slot) * LgH * q * d;
+        const float* evs = evecy + int64_t(slot) * d * d;
+        float* xt = c.atc<float>(p.xt);
+        // U_d = first rd eigenvector columns (stored dtype), then G = Y U_d (stored dtype)
+        k_store_ut<<<grid1(int64_t(d) * rd), 256, 0, c.st>>>(evs, d, d, rd, f32, cud, nullptr, nullptr, nullptr);
+        k_proj_small<<<grid1(int64_t(LgH) * rT * rd), 256, 0, c.st>>>(ylh, int64_t(LgH) * rT, d, evs, d, rd, f32, cg);
+        // X~ = U^s B with B = G^s U_d^s^T, to fp32 accuracy: 3-way bf16 splits, terms of order <= 2
+        __nv_bfloat16* bh = c.atc<__nv_bfloat16>(p.bh);
+        __nv_bfloat16* bm = c.atc<__nv_bfloat16>(p.bm);
+        __nv_bfloat16* bl = c.atc<__nv_bfloat16>(p.bl);
+        float* blh = c.atc<float>(p.blh);
+        k_recon_b<<<grid1(int64_t(LgH) * rT * d), 256, 0, c.st>>>(cg, cud, int64_t(LgH) * rT, rd, d, f32, blh);
+        if ((r = split3_bf16(blh, int64_t(LgH) * rT * d, bh, bm, bl, c.st))) return r;
+        {
+          GemmCall g;
+          g.M = T; g.N = d; g.K = rT;
+          const Operand Bp[3] = {plain(bh, kMajorMN, d, rT, d, LgH, int64_t(rT) * d),
+                                 plain(bm, kMajorMN, d, rT, d, LgH, int64_t(rT) * d),
+                                 plain(bl, kMajorMN, d, rT, d, LgH, int64_t(rT) * d)};
+          const Operand Up[3] = {plain(uh, kMajorK, rT, T, rT, LgH, 0), plain(um, kMajorK, rT, T, rT, LgH, 0),
+                                 plain(ul, kMajorK, rT, T, rT, LgH, 0)};
+          const int nu = f32 ? 3 : 1;
+          int nt = 0;
+          for (int i = 0; i < nu; ++i)
+            for (int jj = 0; jj < 3; ++jj)
+              if (i + jj <= 2) {
+                g.A[nt] = Up[i];
+                g.B[nt] = Bp[jj];
+                ++nt;
+              }
+          g.n_terms = nt;
+          g.C = xt; g.ldc = d; g.c_batch_stride = int64_t(T) * d; g.batch = LgH; g.err = c.err;
+          if ((r = gemm_tc(g, c.st))) return r;
+        }
+        Xt = xt;
       }
-      JOLT_CUDA_TRY(cudaGetLastError());
+      if (ch.b > 0) {
+        uint8_t* codes = cb + offs[5 * cell + 3];
+        __half2* sz = reinterpret_cast<__half2*>(cb + offs[5 * cell + 4]);
+        const int64_t rows = int64_t(LgH) * T;
+        const int grid = int(std::min<int64_t>((rows + 7) / 8, 148 * 16));
+        // algorithmic bytes: read X (io dtype) and X~ (fp32, when present), write codes and sz
+        StatScope sc(JOLT_K_RESIDUAL, c.st, 0.0,
+                     double(rows) * d * ((io32 ? 4 : 2) + (Xt ? 4 : 0)) + double(rows) * (d * ch.b / 8 + 4));
+        if (d == 128) {
+          if (io32) k_residual<4, float><<<grid, 256, 0, c.st>>>(reinterpret_cast<const float*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
+          else k_residual<4, __nv_bfloat16><<<grid, 256, 0, c.st>>>(reinterpret_cast<const __nv_bfloat16*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
+        } else {
+          if (io32) k_residual<2, float><<<grid, 256, 0, c.st>>>(reinterpret_cast<const float*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
+          else k_residual<2, __nv_bfloat16><<<grid, 256, 0, c.st>>>(reinterpret_cast<const __nv_bfloat16*>(Xk), Xt, rows, ch.b, s.rot_seed, codes, sz, c.err);
+        }
+        JOLT_CUDA_TRY(cudaGetLastError());
+      }
     }
   }
   return read_err(c);
