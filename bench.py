@@ -287,6 +287,21 @@ def count_kernels(step):
         return None, [f"profiler unavailable: {ex}"]
 
 
+def rank_workload(name, rank, over):
+    """Weak scaling: every rank compresses and decodes its own sequences — the same shape, its own
+    seed (no data-path collective)."""
+    w = get_workload(name, **over)
+    return get_workload(name, seed=w.seed + 1000 * rank, **over) if rank else w
+
+
+def max_over_ranks(ms, device):
+    """The step time of the slowest rank (every rank calls this at the same point)."""
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -312,8 +327,7 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    # weak scaling: every rank compresses and decodes its own sequences (own seed)
-    w = get_workload(args.workload, seed=w.seed + 1000 * rank, **over) if rank else w
+    w = rank_workload(args.workload, rank, over)
     ratio = args.ratio if args.ratio else (w.budget_ratios[0] if w.budget_ratios else None)
     hbm_peak, tc_burst, tc_sust, peak_src = load_peaks()
     from long_context_st_b200 import api
@@ -350,9 +364,7 @@ def main():
     total_ms = t_start.elapsed_time(t_end)
     if world > 1:
         import torch.distributed as dist
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(total_ms, dev)
         dist.barrier()
     ms_step = total_ms / args.steps
     ph = {k: float(np.mean([e["start"].elapsed_time(e[k]) if k != "start" else 0.0 for e in evs]))
