@@ -408,16 +408,27 @@ __global__ void __launch_bounds__(128) k_scores_res(const ResArgs a) {
   }
 }
 
-// Per row: m = max s, P~ = bf16(exp(s - m)) (row stride ldp), l = sum of the rounded P~.
+// Per row: m = max s, P~ = bf16(exp(s - m)) (row stride ldp), l = sum of the rounded P~. Rows of a
+// multiple of 4 scores are read as float4 and written as four bf16 at a time.
 __global__ void __launch_bounds__(512) k_softmax_rows(const float* __restrict__ scores, int T, int64_t ldp,
                                                       float* __restrict__ mrow, float* __restrict__ lrow,
                                                       __nv_bfloat16* __restrict__ ptil) {
   const int64_t r = blockIdx.x;
   const float* s = scores + r * T;
+  __nv_bfloat16* pr = ptil + r * ldp;
   __shared__ float red[32];
   const int nw = blockDim.x >> 5, wid = threadIdx.x >> 5, ln = threadIdx.x & 31;
+  const bool vec = (T % 4) == 0 && (ldp % 4) == 0;
   float m = -INFINITY;
-  for (int t = threadIdx.x; t < T; t += blockDim.x) m = fmaxf(m, s[t]);
+  if (vec) {
+    const float4* s4 = reinterpret_cast<const float4*>(s);
+    for (int t = threadIdx.x; t < T / 4; t += blockDim.x) {
+      const float4 x = s4[t];
+      m = fmaxf(m, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
+    }
+  } else {
+    for (int t = threadIdx.x; t < T; t += blockDim.x) m = fmaxf(m, s[t]);
+  }
   m = warp_max(m);
   if (ln == 0) red[wid] = m;
   __syncthreads();
@@ -430,11 +441,23 @@ __global__ void __launch_bounds__(512) k_softmax_rows(const float* __restrict__ 
   m = red[0];
   __syncthreads();
   float l = 0.f;
-  __nv_bfloat16* pr = ptil + r * ldp;
-  for (int t = threadIdx.x; t < T; t += blockDim.x) {
-    const __nv_bfloat16 e = __float2bfloat16_rn(__expf(s[t] - m));
-    pr[t] = e;
-    l += __bfloat162float(e);
+  if (vec) {
+    const float4* s4 = reinterpret_cast<const float4*>(s);
+    uint2* p4 = reinterpret_cast<uint2*>(pr);
+    for (int t = threadIdx.x; t < T / 4; t += blockDim.x) {
+      const float4 x = s4[t];
+      const __nv_bfloat162 e01 = __floats2bfloat162_rn(__expf(x.x - m), __expf(x.y - m));
+      const __nv_bfloat162 e23 = __floats2bfloat162_rn(__expf(x.z - m), __expf(x.w - m));
+      p4[t] = make_uint2(*reinterpret_cast<const uint32_t*>(&e01), *reinterpret_cast<const uint32_t*>(&e23));
+      const float2 f01 = __bfloat1622float2(e01), f23 = __bfloat1622float2(e23);
+      l += (f01.x + f01.y) + (f23.x + f23.y);
+    }
+  } else {
+    for (int t = threadIdx.x; t < T; t += blockDim.x) {
+      const __nv_bfloat16 e = __float2bfloat16_rn(__expf(s[t] - m));
+      pr[t] = e;
+      l += __bfloat162float(e);
+    }
   }
   l = warp_sum(l);
   if (ln == 0) red[wid] = l;
@@ -457,20 +480,26 @@ struct ValArgs {
 };
 
 // acc[h'][j] += sum_t P~[h'][t] deq(code_t[j]) (rotated domain). grid (token chunks, n_kv, nl),
-// thread = feature j; every 128-token sub-tile stages its code rows (16-byte loads), scale/zero
-// pairs and probabilities in shared memory first.
+// 128 threads: lane l owns features 4l .. 4l+3 (one 4-code word per token), warp w the tokens
+// w, w+4, ... of every 128-token sub-tile, whose code rows (16-byte loads), scale/zero pairs and
+// probabilities are staged in shared memory first; the four warps' partial sums are added in
+// shared memory before one atomic add per (query head, feature).
 template <int BITS>
 __global__ void __launch_bounds__(128) k_values_res(const ValArgs a) {
-  constexpr int RB = kD * BITS / 8;  // bytes of one code row
+  constexpr int RB = kD * BITS / 8;        // bytes of one code row
+  constexpr uint32_t mask = (1u << BITS) - 1u;
   __shared__ __align__(16) uint8_t cs[128][RB];
   __shared__ __align__(16) float pr[128][kMaxG];
   __shared__ float2 szs[128];
-  const int h = blockIdx.y, li = blockIdx.z, j = threadIdx.x;
+  __shared__ __align__(16) float red[2][kMaxG][kD];
+  const int h = blockIdx.y, li = blockIdx.z, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int64_t qrow0 = int64_t(li) * a.n_q + int64_t(h) * a.gq;
   const int64_t rbase = (int64_t(li) * a.n_kv + h) * a.T;
-  float acc[kMaxG];
+  float acc[kMaxG][4];
 #pragma unroll
-  for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
+  for (int g = 0; g < kMaxG; ++g)
+#pragma unroll
+    for (int f = 0; f < 4; ++f) acc[g][f] = 0.f;
   const int t_beg = blockIdx.x * a.chunk, t_end = min(a.T, t_beg + a.chunk);
   for (int tb = t_beg; tb < t_end; tb += 128) {
     const int nt = min(128, t_end - tb);
@@ -487,27 +516,60 @@ __global__ void __launch_bounds__(128) k_values_res(const ValArgs a) {
         pr[threadIdx.x][g] = g < a.gq ? __bfloat162float(a.ptil[(qrow0 + g) * a.ldp + tb + threadIdx.x]) : 0.f;
     }
     __syncthreads();
-    const int byte = (j * BITS) >> 3, shift = (j * BITS) & 7;
-    for (int tt = 0; tt < nt; ++tt) {
-      const uint32_t code = (uint32_t(cs[tt][byte]) >> shift) & ((1u << BITS) - 1u);
+    for (int tt = w; tt < nt; tt += 4) {
+      uint32_t word;
+      if (BITS == 2) word = cs[tt][lane];
+      else if (BITS == 4) word = reinterpret_cast<const uint16_t*>(cs[tt])[lane];
+      else word = reinterpret_cast<const uint32_t*>(cs[tt])[lane];
       const float2 z = szs[tt];
-      const float dv = dequant(code, z.x, z.y);
+      float dv[4];
+#pragma unroll
+      for (int f = 0; f < 4; ++f) dv[f] = dequant((word >> (f * BITS)) & mask, z.x, z.y);
       const float4* p4 = reinterpret_cast<const float4*>(pr[tt]);
 #pragma unroll
       for (int g4 = 0; g4 < kMaxG / 4; ++g4) {
         if (4 * g4 < a.gq) {
-          const float4 w = p4[g4];
-          acc[4 * g4 + 0] = fmaf(w.x, dv, acc[4 * g4 + 0]);
-          acc[4 * g4 + 1] = fmaf(w.y, dv, acc[4 * g4 + 1]);
-          acc[4 * g4 + 2] = fmaf(w.z, dv, acc[4 * g4 + 2]);
-          acc[4 * g4 + 3] = fmaf(w.w, dv, acc[4 * g4 + 3]);
+          const float4 pw = p4[g4];
+          const float pv[4] = {pw.x, pw.y, pw.z, pw.w};
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg)
+#pragma unroll
+            for (int f = 0; f < 4; ++f) acc[4 * g4 + gg][f] = fmaf(pv[gg], dv[f], acc[4 * g4 + gg][f]);
         }
       }
     }
   }
+  // warps 2, 3 -> shared; warps 0, 1 add; warp 1 -> shared; warp 0 adds and commits
+  __syncthreads();
+  if (w >= 2)
 #pragma unroll
-  for (int g = 0; g < kMaxG; ++g)
-    if (g < a.gq) atomicAdd(&a.acc[(qrow0 + g) * kD + j], acc[g]);
+    for (int g = 0; g < kMaxG; ++g)
+      if (g < a.gq) *reinterpret_cast<float4*>(&red[w - 2][g][4 * lane]) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
+  __syncthreads();
+  if (w < 2)
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g)
+      if (g < a.gq) {
+        const float4 o = *reinterpret_cast<const float4*>(&red[w][g][4 * lane]);
+        acc[g][0] += o.x; acc[g][1] += o.y; acc[g][2] += o.z; acc[g][3] += o.w;
+      }
+  __syncthreads();
+  if (w == 1)
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g)
+      if (g < a.gq) *reinterpret_cast<float4*>(&red[0][g][4 * lane]) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
+  __syncthreads();
+  if (w == 0)
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g)
+      if (g < a.gq) {
+        const float4 o = *reinterpret_cast<const float4*>(&red[0][g][4 * lane]);
+        float* dst = &a.acc[(qrow0 + g) * kD + 4 * lane];
+        atomicAdd(dst + 0, acc[g][0] + o.x);
+        atomicAdd(dst + 1, acc[g][1] + o.y);
+        atomicAdd(dst + 2, acc[g][2] + o.z);
+        atomicAdd(dst + 3, acc[g][3] + o.w);
+      }
 }
 
 struct FinArgs {
