@@ -430,9 +430,11 @@ Operand xunfold(const void* X, int major, const Plan& p, int C) {
 // an unshifted factorisation falls back to a shifted pass. At most kMaxOrthPasses passes.
 constexpr int kMaxOrthPasses = 8;
 
-// polish = false (inside the power iterations): stop after the first pass whose pivots show a
-// well-conditioned input (ratio >= 0.1); its output is orthonormal to within the shift's effect,
-// which is all the next product needs. The final basis (polish = true) gets the unshifted passes.
+// polish = false (inside the power iterations): the basis only feeds the next product, which reads
+// its bf16 part, so the passes orthonormalise the bf16-rounded matrix itself — Gram Y_hi^T Y_hi
+// (one term, exact), Q = Y_hi (R^-1 hi + lo) — and stop after the first pass whose pivots show a
+// well-conditioned input (ratio >= 0.1). The final basis (polish = true) uses hi/lo terms
+// throughout and gets the unshifted passes.
 jolt_status orth(const Ctx& c, float* Y, int rows, int C, bool polish = true) {
   const Plan& p = c.p;
   const int l = p.l;
@@ -443,11 +445,11 @@ jolt_status orth(const Ctx& c, float* Y, int rows, int C, bool polish = true) {
   __nv_bfloat16* Rl = c.at<__nv_bfloat16>(p.Rl);
   bool conditioned = false;
   for (int pass = 0; pass < kMaxOrthPasses; ++pass) {
-    jolt_status r = split_bf16(Y, l, rows, l, C, int64_t(rows) * l, Yh, Yl, l, int64_t(rows) * l, c.st);
+    jolt_status r = split_bf16(Y, l, rows, l, C, int64_t(rows) * l, Yh, polish ? Yl : nullptr, l, int64_t(rows) * l, c.st);
     if (r) return r;
     JOLT_CUDA_TRY(cudaMemsetAsync(Gm, 0, size_t(C) * l * l * 4, c.st));
     GemmCall g;
-    g.M = l; g.N = l; g.K = rows; g.n_terms = 3;
+    g.M = l; g.N = l; g.K = rows; g.n_terms = polish ? 3 : 1;
     const Operand yh = plain(Yh, kMajorMN, l, rows, l, C, int64_t(rows) * l);
     const Operand yl = plain(Yl, kMajorMN, l, rows, l, C, int64_t(rows) * l);
     g.A[0] = yh; g.B[0] = yh;
@@ -495,7 +497,7 @@ jolt_status orth(const Ctx& c, float* Y, int rows, int C, bool polish = true) {
     if (std::getenv("JOLT_DEBUG"))
       std::fprintf(stderr, "jolt orth: rows %d pass %d shift %g min pivot ratio %g\n", rows, pass, shift, ratio);
     GemmCall t;
-    t.M = rows; t.N = l; t.K = l; t.n_terms = 3;
+    t.M = rows; t.N = l; t.K = l; t.n_terms = polish ? 3 : 2;
     const Operand ykh = plain(Yh, kMajorK, l, rows, l, C, int64_t(rows) * l);
     const Operand ykl = plain(Yl, kMajorK, l, rows, l, C, int64_t(rows) * l);
     const Operand rh = plain(Rh, kMajorMN, l, l, l, C, int64_t(l) * l);
