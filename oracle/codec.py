@@ -82,6 +82,21 @@ def decompress_cell(cell, rot_seed: int) -> np.ndarray:
     return Xt + residual_hat(cell, rot_seed)
 
 
+def decompress_slice(cell, l: int, h: int, rot_seed: int) -> np.ndarray:
+    """X^[l, h] of one cell (layer l of the group, KV head h) without rebuilding the rest:
+    U_T (G[l, h] U_d^T) + rotation^T deq(codes[l, h]) — the same stored values as decompress_cell."""
+    L, H, T, d = cell["shape"]
+    if cell["r_T"] > 0:
+        Xt = cell["U_T"] @ (cell["G"][l, h] @ cell["U_d"].T)
+    else:
+        Xt = np.zeros((T, d))
+    if cell["b"] == 0:
+        return Xt
+    code = unpack_codes(cell["codes"][l, h], cell["b"], d)
+    deq = dequantize_rows(code, cell["scale"][l, h], cell["zero"][l, h]).astype(np.float64)
+    return Xt + deq @ rotation_matrix(d, rot_seed)
+
+
 def rope(x: np.ndarray, positions: np.ndarray, inv_freq: np.ndarray) -> np.ndarray:
     """x [..., T, d] float64, positions [T] ints, inv_freq [d/2] float32 -> rotated float64."""
     d = x.shape[-1]

@@ -128,3 +128,29 @@ def device_to_cells(shape, w, cache, choices, factor_dtype=None):
             cell["zero"] = sz[..., 1].copy()
         cells.append(cell)
     return cells
+
+
+def device_cell(shape, w, cache, choices, c, factor_dtype=None):
+    """One cell of a device cache as an oracle cell dict (only that cell's bytes are copied)."""
+    fdt = _FDT[factor_dtype or w.factor_dtype]
+    offs, _ = api.cache_layout(shape, choices)
+    Lg, H, T, d = w.layers_per_group, w.n_kv, shape.T, w.d_h
+    rT, rd, b = choices[c]
+
+    def get(off, count, dtype):
+        nb = count * (torch.finfo(dtype).bits // 8 if dtype.is_floating_point else 1)
+        return cache[int(off):int(off) + nb].cpu().view(dtype)
+
+    cell = {"r_T": rT, "r_d": rd, "b": b, "shape": (Lg, H, T, d)}
+    if rT:
+        cell["U_T"] = get(offs[c, 0], T * rT, fdt).double().numpy().reshape(T, rT)
+        cell["U_d"] = get(offs[c, 1], d * rd, fdt).double().numpy().reshape(d, rd)
+        cell["G"] = get(offs[c, 2], Lg * H * rT * rd, fdt).double().numpy().reshape(Lg, H, rT, rd)
+    else:
+        cell["U_T"] = np.zeros((T, 0)); cell["U_d"] = np.zeros((d, 0)); cell["G"] = np.zeros((Lg, H, 0, 0))
+    if b:
+        cell["codes"] = get(offs[c, 3], Lg * H * T * d * b // 8, torch.uint8).numpy().reshape(Lg, H, T, d * b // 8)
+        sz = get(offs[c, 4], Lg * H * T * 2, torch.float16).numpy().reshape(Lg, H, T, 2)
+        cell["scale"] = sz[..., 0].copy()
+        cell["zero"] = sz[..., 1].copy()
+    return cell

@@ -3,7 +3,7 @@ import numpy as np
 import torch
 import pytest
 
-from oracle.codec import compress_cell, decompress_cell, rope, decode_attention
+from oracle.codec import compress_cell, decompress_cell, decompress_slice, rope, decode_attention
 from oracle.hosvd import st_hosvd, reconstruct
 from synth import get_workload, make_kv_cell, make_inv_freq
 
@@ -69,3 +69,16 @@ def test_rope_complex_form_and_relative_position():
     a = rope(q[None], np.array([10]), inv) @ rope(k[None], np.array([3]), inv).T
     b = rope(q[None], np.array([1007]), inv) @ rope(k[None], np.array([1000]), inv).T
     assert abs(a - b).max() < 1e-9
+
+
+@pytest.mark.parametrize("ch", [(32, 32, 4), (0, 0, 2), (48, 16, 0), (16, 64, 8)])
+def test_decompress_slice_is_the_cells_slice(ch):
+    # every (layer, head) slice of the whole-cell reconstruction, for factor-only, residual-only
+    # and mixed cells (an index or transpose slip in the slice path breaks it)
+    w = get_workload("toy", n_layers=2, layers_per_group=2)
+    X = make_kv_cell(w, "K", 0, 0, dtype=torch.float64).numpy()
+    cell = compress_cell(X, *ch, 7, "bf16")
+    full = decompress_cell(cell, 7)
+    for l in range(X.shape[0]):
+        for h in range(X.shape[1]):
+            assert np.allclose(decompress_slice(cell, l, h, 7), full[l, h], rtol=0, atol=1e-12)
