@@ -115,6 +115,37 @@ uint64_t jolt_cell_bytes(const jolt_shape* shape, jolt_cell_choice choice);
 jolt_status jolt_cache_layout(const jolt_shape* shape, const jolt_cell_choice* choices,
                               uint64_t* offsets, uint64_t* total_bytes);
 
+/* ---- Stored cache as a host blob (persisting a compressed cache, moving it between processes).
+ * The pages store the factors, codes and scales per group ("A JoLT for the KV cache", §3, the
+ * stored cache); the blob adds a header so a reader can check what it holds:
+ *   bytes 0..7   magic "JOLTCACH"; 8..11 format version (1); 12..15 header bytes (h)
+ *   16..         jolt_shape (as in this header), int32 n_cells, n_cells jolt_cell_choice,
+ *                uint64 cache bytes (c), zero padding up to h (a multiple of 256)
+ *   h .. h+c     the cache exactly as jolt_cache_layout places it (device bytes copied verbatim)
+ * All fields little-endian. */
+
+/* Blob bytes for a shape and its choices (0 if either is invalid). */
+uint64_t jolt_cache_blob_bytes(const jolt_shape* shape, const jolt_cell_choice* choices);
+
+/* Copies the device cache (laid out for `choices`) into the host blob and writes the header.
+ *   cache  device, >= the jolt_cache_layout total;  blob  host, >= jolt_cache_blob_bytes
+ * Synchronises `stream`. JOLT_ERR_INVALID_ARG on a bad shape, choice or short blob. */
+jolt_status jolt_cache_serialize(const jolt_shape* shape, const jolt_cell_choice* choices, const void* cache,
+                                 void* blob, uint64_t blob_bytes, void* stream);
+
+/* Reads and checks a blob's header (host only, no device work): magic, version, shape, choices,
+ * and that the blob holds the cache bytes the layout needs.
+ *   shape_out (host, may be NULL), n_cells_out (host, may be NULL), cache_bytes_out (host, may
+ *   be NULL). JOLT_ERR_INVALID_ARG on a malformed or truncated blob. */
+jolt_status jolt_cache_blob_info(const void* blob, uint64_t blob_bytes, jolt_shape* shape_out, int32_t* n_cells_out,
+                                 uint64_t* cache_bytes_out);
+
+/* Checks the blob as jolt_cache_blob_info does, then writes its choices (host, n_cells entries
+ * from jolt_cache_blob_info) and copies the cache into device memory `cache` (>= cache bytes).
+ * Synchronises `stream`. */
+jolt_status jolt_cache_deserialize(const void* blob, uint64_t blob_bytes, jolt_cell_choice* choices_out,
+                                   int32_t n_cells, void* cache, uint64_t cache_bytes, void* stream);
+
 /* Error fraction phi(b) of the rotated b-bit quantiser for b = 0, 2, 4, 8 (phi(0) = 1), measured
  * on n_rows Gaussian rows of dimension d_h drawn from `seed` (host computation). The allocator's
  * surrogate multiplies the discarded mass by it ("A JoLT for the KV cache", §3). */

@@ -52,6 +52,13 @@ SIGNATURES = [
     ("jolt_shape_check", C.c_int, [C.POINTER(Shape)]),
     ("jolt_kv_bytes", C.c_uint64, [C.c_int32, C.c_int32, C.c_int32, C.c_int64, C.c_int32]),
     ("jolt_cell_bytes", C.c_uint64, [C.POINTER(Shape), CellChoice]),
+    ("jolt_cache_blob_bytes", C.c_uint64, [C.POINTER(Shape), C.POINTER(CellChoice)]),
+    ("jolt_cache_serialize", C.c_int, [C.POINTER(Shape), C.POINTER(CellChoice), C.c_void_p, C.c_void_p,
+                                       C.c_uint64, C.c_void_p]),
+    ("jolt_cache_blob_info", C.c_int, [C.c_void_p, C.c_uint64, C.POINTER(Shape), C.POINTER(C.c_int32),
+                                       C.POINTER(C.c_uint64)]),
+    ("jolt_cache_deserialize", C.c_int, [C.c_void_p, C.c_uint64, C.POINTER(CellChoice), C.c_int32, C.c_void_p,
+                                         C.c_uint64, C.c_void_p]),
     ("jolt_cache_layout", C.c_int, [C.POINTER(Shape), C.POINTER(CellChoice), C.POINTER(C.c_uint64),
                                     C.POINTER(C.c_uint64)]),
     ("jolt_phi", C.c_int, [C.c_int32, C.c_int32, C.c_uint64, C.POINTER(C.c_double)]),

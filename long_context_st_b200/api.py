@@ -78,6 +78,43 @@ def cache_layout(s: Shape, choices):
     return np.array(offs, dtype=np.uint64).reshape(nc, 5), int(tot.value)
 
 
+def cache_blob_bytes(s: Shape, choices) -> int:
+    return int(lib().jolt_cache_blob_bytes(C.byref(s), choices_array(choices)))
+
+
+def serialize_cache(s: Shape, choices, cache, stream=None) -> np.ndarray:
+    """The stored cache (device uint8 tensor) as a host blob with a checked header."""
+    n = cache_blob_bytes(s, choices)
+    if n == 0:
+        raise JoltError(-1, "jolt_cache_blob_bytes")
+    blob = np.empty(n, dtype=np.uint8)
+    check(lib().jolt_cache_serialize(C.byref(s), choices_array(choices), _ptr(cache), blob.ctypes.data, n,
+                                     _stream(stream)), "jolt_cache_serialize")
+    return blob
+
+
+def cache_blob_info(blob):
+    """(shape, n_cells, cache_bytes) of a blob; raises on a malformed or truncated blob."""
+    b = np.ascontiguousarray(blob, dtype=np.uint8)
+    s = Shape()
+    nc = C.c_int32(0)
+    cb = C.c_uint64(0)
+    check(lib().jolt_cache_blob_info(b.ctypes.data, b.size, C.byref(s), C.byref(nc), C.byref(cb)),
+          "jolt_cache_blob_info")
+    return s, int(nc.value), int(cb.value)
+
+
+def deserialize_cache(blob, device="cuda", stream=None):
+    """(shape, choices, cache device tensor) from a blob written by serialize_cache."""
+    b = np.ascontiguousarray(blob, dtype=np.uint8)
+    s, nc, cb = cache_blob_info(b)
+    out = (CellChoice * nc)()
+    cache = torch.empty(max(cb, 1), dtype=torch.uint8, device=device)
+    check(lib().jolt_cache_deserialize(b.ctypes.data, b.size, out, nc, _ptr(cache), cache.numel(),
+                                       _stream(stream)), "jolt_cache_deserialize")
+    return s, [(c.r_T, c.r_d, c.b) for c in out], cache
+
+
 def phi(d_h: int, n_rows: int = 1 << 16, seed: int = 1):
     out = (C.c_double * 4)()
     check(lib().jolt_phi(d_h, n_rows, seed, out), "jolt_phi")
@@ -226,7 +263,7 @@ def stats_read(reset=True):
                                      bytes=arr[i].bytes) for i in range(len(KERNEL_FAMILIES))}
 
 
-__all__ = ["decode_attn_noalloc", "stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
+__all__ = ["serialize_cache", "deserialize_cache", "cache_blob_info", "cache_blob_bytes", "decode_attn_noalloc", "stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
            "allocate", "workspace_bytes", "new_workspace", "analyze", "compress", "decode_attn",
            "check_ws", "rotate_rows", "quantize_pack", "unpack_dequant", "JoltError",
            "JOLT_OP_COMPRESS", "JOLT_OP_DECODE"]

@@ -125,3 +125,36 @@ def test_allocator_zero_budget_stores_nothing():
     n2, tT, td = make_random_tables(2, s.q_cap // 16 + 1, w.d_h // 16 + 1, 1)
     ch, lam, tot = api.allocate(s, n2, tT, td, [1.0, 0.1, 0.01, 0.0001], 0)
     assert ch == [(0, 0, 0), (0, 0, 0)] and tot == 0 and lam > 0
+
+
+def test_cache_blob_header_checks():
+    # host-only paths of the blob format: size arithmetic and rejection of malformed blobs
+    import ctypes as C
+    from long_context_st_b200._lib import Shape
+    w = get_workload("llama8b_32k", n_layers=8, T=1000)
+    shape = api.make_shape(w)
+    choices = [(64, 32, 4), (0, 0, 2)] * (api.n_cells(shape) // 2)
+    _, total = api.cache_layout(shape, choices)
+    n = api.cache_blob_bytes(shape, choices)
+    hdr = n - total
+    assert hdr % 256 == 0 and hdr >= 16 + C.sizeof(Shape) + 4 + 12 * len(choices) + 8
+    with pytest.raises(api.JoltError):
+        api.cache_blob_info(np.zeros(n, dtype=np.uint8))           # no magic
+    with pytest.raises(api.JoltError):
+        api.cache_blob_info(np.frombuffer(b"JOLTCACH", dtype=np.uint8))  # truncated
+    # a header written by hand to the documented layout is accepted; one byte short is not
+    blob = np.zeros(n, dtype=np.uint8)
+    raw = bytearray(b"JOLTCACH") + (1).to_bytes(4, "little") + hdr.to_bytes(4, "little")
+    raw += bytes(shape) + len(choices).to_bytes(4, "little", signed=True)
+    for c in choices:
+        raw += b"".join(int(v).to_bytes(4, "little", signed=True) for v in c)
+    raw += total.to_bytes(8, "little")
+    blob[:len(raw)] = np.frombuffer(bytes(raw), dtype=np.uint8)
+    s2, nc, cb = api.cache_blob_info(blob)
+    assert nc == len(choices) and cb == total and s2.T == shape.T and s2.rot_seed == shape.rot_seed
+    with pytest.raises(api.JoltError):
+        api.cache_blob_info(blob[:-1])
+    bad = blob.copy()
+    bad[8] = 2                                                   # unknown version
+    with pytest.raises(api.JoltError):
+        api.cache_blob_info(bad)
