@@ -227,6 +227,7 @@ class Step:
         if "start" in ev:
             ev["start"].record()
         tables = api.analyze(self.shape, K, V, self.cws)
+        self.tables = tables
         if "analyzed" in ev:
             ev["analyzed"].record()
         choices = self.allocate(tables)
@@ -246,6 +247,37 @@ class Step:
         if "decoded" in ev:
             ev["decoded"].record()
         return choices
+
+
+def surrogate_error(tables, choices, phi):
+    """The allocator's summed error model for a choice vector: phi(b) times the discarded mass."""
+    n2, tT, td = tables
+    bits = {0: 0, 2: 1, 4: 2, 8: 3}
+    e = 0.0
+    for c, (rT, rd, b) in enumerate(choices):
+        D = n2[c] if rT == 0 else min(n2[c], tT[c][rT // 16] + td[c][rd // 16])
+        e += phi[bits[b]] * D
+    return e
+
+
+def allocator_ablation(step):
+    """The pages' allocation ablations on this step's own tables at its budget (first sequence):
+    joint (one multiplier), K/V-decoupled, uniform ranks — summed surrogate error / ||X||^2."""
+    api, w = step.api, step.w
+    if w.fixed_choice or step.budget is None:
+        return None
+    G = w.n_layers // w.layers_per_group
+    n2, tT, td = (np.asarray(a)[:2 * G] for a in step.tables)
+    out = {"budget_bytes": step.budget}
+    for name, mode in (("joint", api.JOLT_ALLOC_JOINT), ("kv_split", api.JOLT_ALLOC_KV_SPLIT),
+                       ("uniform", api.JOLT_ALLOC_UNIFORM)):
+        try:
+            ch, tot = api.allocate_variant(step.shape, n2, tT, td, step.phi, step.budget, mode)
+            out[name] = {"rel_error": surrogate_error((n2, tT, td), ch, step.phi) / float(np.sum(n2)),
+                         "bytes": tot}
+        except api.JoltError as e:
+            out[name] = {"error": str(e)}
+    return out
 
 
 def decode_work(w, shape, choices):
@@ -438,6 +470,7 @@ def main():
             "roofline": roof, "roofline_decode": roof_dec,
             "kernel_stats": {k: {kk: (float(vv) if isinstance(vv, float) else int(vv)) for kk, vv in v.items()}
                              for k, v in stats.items()},
+            "allocator_ablation": allocator_ablation(step),
             "gpu_launches": n_kernels * args.steps if n_kernels is not None else None,
             "kernels": kernel_names, "clocks": clk.summary(), "choices": sorted(set(map(tuple, step.choices)))}
 

@@ -166,6 +166,23 @@ jolt_status jolt_allocate(const jolt_shape* shape, int32_t n_cells, const double
                           const double phi[4], uint64_t budget, jolt_cell_choice* choices_out,
                           double* lambda_out, uint64_t* total_bytes_out);
 
+/* Allocation variants of the pages' ablations ("A JoLT for the KV cache", §4.4 Ablations and
+ * App. D Tables 12-13), same inputs and error model as jolt_allocate, cells ordered (sequence,
+ * group, K|V) so even cells are keys and odd cells values:
+ *   JOLT_ALLOC_JOINT     jolt_allocate itself;
+ *   JOLT_ALLOC_KV_SPLIT  K/V-decoupled: keys and values each allocated jointly on their own, with
+ *                        budget/2 (rounded down) for keys and the rest for values;
+ *   JOLT_ALLOC_UNIFORM   uniform ranks: one (r_T, r_d, b) for every key cell and one for every
+ *                        value cell, the pair of least summed error whose bytes fit (ties: fewer
+ *                        bytes, then the earlier key choice, then the earlier value choice, choices
+ *                        ordered by r_T, r_d, b).
+ * Host-only. JOLT_ERR_BUDGET if nothing fits; JOLT_ERR_INVALID_ARG for an odd n_cells or bad mode. */
+typedef enum { JOLT_ALLOC_JOINT = 0, JOLT_ALLOC_KV_SPLIT = 1, JOLT_ALLOC_UNIFORM = 2 } jolt_alloc_mode;
+jolt_status jolt_allocate_variant(const jolt_shape* shape, int32_t n_cells, const double* norm2,
+                                  const double* tail_T, int32_t n_rt, const double* tail_d, int32_t n_rd,
+                                  const double phi[4], uint64_t budget, int32_t mode,
+                                  jolt_cell_choice* choices_out, uint64_t* total_bytes_out);
+
 /* Workspace bytes for an operation (device memory the caller allocates and passes as `ws`).
  * JOLT_OP_COMPRESS covers jolt_analyze followed by jolt_compress on the same ws;
  * JOLT_OP_DECODE covers jolt_decode_attn with any n_layers_call <= n_layers. 0 on bad shape. */

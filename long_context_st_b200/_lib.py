@@ -66,6 +66,10 @@ SIGNATURES = [
                                 C.POINTER(C.c_double), C.c_int32, C.POINTER(C.c_double), C.c_int32,
                                 C.POINTER(C.c_double), C.c_uint64, C.POINTER(CellChoice),
                                 C.POINTER(C.c_double), C.POINTER(C.c_uint64)]),
+    ("jolt_allocate_variant", C.c_int, [C.POINTER(Shape), C.c_int32, C.POINTER(C.c_double),
+                                        C.POINTER(C.c_double), C.c_int32, C.POINTER(C.c_double), C.c_int32,
+                                        C.POINTER(C.c_double), C.c_uint64, C.c_int32, C.POINTER(CellChoice),
+                                        C.POINTER(C.c_uint64)]),
     ("jolt_workspace_bytes", C.c_size_t, [C.POINTER(Shape), C.c_int32]),
     ("jolt_analyze", C.c_int, [C.POINTER(Shape), _P, _P, C.POINTER(C.c_double),
                                C.POINTER(C.c_double), C.POINTER(C.c_double), _P, C.c_size_t, _P]),

@@ -121,6 +121,26 @@ def phi(d_h: int, n_rows: int = 1 << 16, seed: int = 1):
     return list(out)
 
 
+JOLT_ALLOC_JOINT, JOLT_ALLOC_KV_SPLIT, JOLT_ALLOC_UNIFORM = 0, 1, 2
+
+
+def allocate_variant(s: Shape, norm2, tail_T, tail_d, phi4, budget: int, mode: int):
+    """The allocator's ablation variants (joint, K/V-decoupled, uniform ranks). Returns
+    (choices [(r_T, r_d, b)], bytes)."""
+    norm2 = np.ascontiguousarray(norm2, dtype=np.float64)
+    tT = np.ascontiguousarray(tail_T, dtype=np.float64)
+    td = np.ascontiguousarray(tail_d, dtype=np.float64)
+    nc = norm2.shape[0]
+    out = (CellChoice * nc)()
+    tot = C.c_uint64(0)
+    dp = C.POINTER(C.c_double)
+    ph = (C.c_double * 4)(*phi4)
+    check(lib().jolt_allocate_variant(C.byref(s), nc, norm2.ctypes.data_as(dp), tT.ctypes.data_as(dp),
+                                      tT.shape[1], td.ctypes.data_as(dp), td.shape[1], ph, int(budget),
+                                      int(mode), out, C.byref(tot)), "jolt_allocate_variant")
+    return [(c.r_T, c.r_d, c.b) for c in out], int(tot.value)
+
+
 def allocate(s: Shape, norm2, tail_T, tail_d, phi4, budget: int):
     """One allocation over the given cells. Returns (choices [(r_T, r_d, b)], lambda, bytes)."""
     norm2 = np.ascontiguousarray(norm2, dtype=np.float64)
@@ -263,7 +283,7 @@ def stats_read(reset=True):
                                      bytes=arr[i].bytes) for i in range(len(KERNEL_FAMILIES))}
 
 
-__all__ = ["serialize_cache", "deserialize_cache", "cache_blob_info", "cache_blob_bytes", "decode_attn_noalloc", "stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
+__all__ = ["allocate_variant", "JOLT_ALLOC_JOINT", "JOLT_ALLOC_KV_SPLIT", "JOLT_ALLOC_UNIFORM", "serialize_cache", "deserialize_cache", "cache_blob_info", "cache_blob_bytes", "decode_attn_noalloc", "stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
            "allocate", "workspace_bytes", "new_workspace", "analyze", "compress", "decode_attn",
            "check_ws", "rotate_rows", "quantize_pack", "unpack_dequant", "JoltError",
            "JOLT_OP_COMPRESS", "JOLT_OP_DECODE"]

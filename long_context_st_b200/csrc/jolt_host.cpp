@@ -303,6 +303,88 @@ jolt_status jolt_allocate(const jolt_shape* s, int32_t nc, const double* norm2,
   return JOLT_OK;
 }
 
+jolt_status jolt_allocate_variant(const jolt_shape* s, int32_t nc, const double* norm2, const double* tail_T,
+                                  int32_t nrt, const double* tail_d, int32_t nrd, const double phi[4],
+                                  uint64_t budget, int32_t mode, jolt_cell_choice* out, uint64_t* total_out) {
+  if (mode == JOLT_ALLOC_JOINT)
+    return jolt_allocate(s, nc, norm2, tail_T, nrt, tail_d, nrd, phi, budget, out, nullptr, total_out);
+  if (!shape_ok(s) || nc < 2 || nc % 2 || !norm2 || !tail_T || !tail_d || !phi || !out) return JOLT_ERR_INVALID_ARG;
+  if (nrt < 1 || nrd < 1 || (nrt - 1) * kRankStep > s->q_cap || (nrd - 1) * kRankStep > s->d_h)
+    return JOLT_ERR_INVALID_ARG;
+  for (int i = 0; i < 4; ++i)
+    if (!(phi[i] >= 0.0) || !std::isfinite(phi[i])) return JOLT_ERR_INVALID_ARG;
+  const int half = nc / 2;
+  if (mode == JOLT_ALLOC_KV_SPLIT) {
+    uint64_t total = 0;
+    for (int kind = 0; kind < 2; ++kind) {
+      std::vector<double> n2(half), tT(size_t(half) * nrt), td(size_t(half) * nrd);
+      for (int i = 0; i < half; ++i) {
+        const int c = 2 * i + kind;
+        n2[i] = norm2[c];
+        std::copy(tail_T + size_t(c) * nrt, tail_T + size_t(c + 1) * nrt, tT.begin() + size_t(i) * nrt);
+        std::copy(tail_d + size_t(c) * nrd, tail_d + size_t(c + 1) * nrd, td.begin() + size_t(i) * nrd);
+      }
+      std::vector<jolt_cell_choice> ch(half);
+      uint64_t tot = 0;
+      const uint64_t bud = kind == 0 ? budget / 2 : budget - budget / 2;
+      const jolt_status r = jolt_allocate(s, half, n2.data(), tT.data(), nrt, td.data(), nrd, phi, bud, ch.data(),
+                                          nullptr, &tot);
+      if (r != JOLT_OK) return r;
+      for (int i = 0; i < half; ++i) out[2 * i + kind] = ch[i];
+      total += tot;
+    }
+    if (total_out) *total_out = total;
+    return JOLT_OK;
+  }
+  if (mode != JOLT_ALLOC_UNIFORM) return JOLT_ERR_INVALID_ARG;
+  // every choice in (r_T, r_d, b) order with its bytes and its summed error over each kind's cells
+  const int bits[4] = {0, 2, 4, 8};
+  std::vector<jolt_cell_choice> grid;
+  for (int k = 0; k < nrt; ++k)
+    for (int j = 0; j < nrd; ++j) {
+      if ((k == 0) != (j == 0)) continue;
+      for (int bi = 0; bi < 4; ++bi) grid.push_back(jolt_cell_choice{k * kRankStep, j * kRankStep, bits[bi]});
+    }
+  const size_t ng = grid.size();
+  std::vector<uint64_t> gb(ng);
+  std::vector<double> ge[2] = {std::vector<double>(ng, 0.0), std::vector<double>(ng, 0.0)};
+  for (size_t o = 0; o < ng; ++o) {
+    const jolt_cell_choice& ch = grid[o];
+    gb[o] = jolt_cell_bytes(s, ch);
+    const int k = ch.r_T / kRankStep, j = ch.r_d / kRankStep;
+    const int bi = ch.b == 0 ? 0 : ch.b == 2 ? 1 : ch.b == 4 ? 2 : 3;
+    for (int c = 0; c < nc; ++c) {
+      const double D = k == 0 ? norm2[c] : std::min(norm2[c], tail_T[size_t(c) * nrt + k] + tail_d[size_t(c) * nrd + j]);
+      if (!std::isfinite(D)) return JOLT_ERR_NUMERIC;
+      ge[c % 2][o] += D * phi[bi];
+    }
+  }
+  bool found = false;
+  double bestE = 0.0;
+  uint64_t bestB = 0;
+  size_t bk = 0, bv = 0;
+  for (size_t ok = 0; ok < ng; ++ok) {
+    const uint64_t bK = uint64_t(half) * gb[ok];
+    if (bK > budget) continue;
+    for (size_t ov = 0; ov < ng; ++ov) {
+      const uint64_t B = bK + uint64_t(half) * gb[ov];
+      if (B > budget) continue;
+      const double E = ge[0][ok] + ge[1][ov];
+      if (!found || E < bestE || (E == bestE && B < bestB)) {
+        found = true;
+        bestE = E;
+        bestB = B;
+        bk = ok;
+        bv = ov;
+      }
+    }
+  }
+  if (!found) return JOLT_ERR_BUDGET;
+  for (int c = 0; c < nc; ++c) out[c] = grid[c % 2 ? bv : bk];
+  if (total_out) *total_out = bestB;
+  return JOLT_OK;
+}
+
 size_t jolt_workspace_bytes(const jolt_shape* s, int32_t op) {
   if (!shape_ok(s)) return 0;
   if (op == JOLT_OP_COMPRESS) return compress_workspace_bytes(*s);

@@ -121,6 +121,42 @@ def brute_force_allocate(cell_options, budget: int):
     return best
 
 
+def allocate_kv_split(cell_options, budget: int):
+    """K/V-decoupled allocation ([v4] §4.4 Ablations, App. D Table 12): keys (even cells) and
+    values (odd cells) each allocated jointly on their own; reading: budget // 2 for keys, the
+    rest for values. Returns (choices, total bytes)."""
+    ck, tk = allocate(cell_options[0::2], budget // 2)[0::2]
+    cv, tv = allocate(cell_options[1::2], budget - budget // 2)[0::2]
+    choices = [None] * len(cell_options)
+    choices[0::2] = ck
+    choices[1::2] = cv
+    return choices, tk + tv
+
+
+def allocate_uniform(cell_options, budget: int):
+    """Uniform ranks ([v4] §4.4 Ablations, App. D Table 13); reading: one (r_T, r_d, b) for all
+    key cells and one for all value cells, the pair with the least summed error whose bytes fit.
+    Ties: fewer bytes, then the earlier key option, then the earlier value option (options in
+    build_options order). Returns (choices, total bytes); BudgetError if nothing fits."""
+    n = len(cell_options)
+    half = n // 2
+    ng = len(cell_options[0])
+    Bo = np.array([o[0] for o in cell_options[0]], dtype=np.int64)
+    E = [np.zeros(ng), np.zeros(ng)]
+    for c in range(n):
+        E[c % 2] = E[c % 2] + np.array([o[1] for o in cell_options[c]])
+    Et = E[0][:, None] + E[1][None, :]
+    Bt = half * Bo[:, None] + half * Bo[None, :]
+    ok = Bt <= budget
+    if not ok.any():
+        raise BudgetError(f"budget {budget} below the cheapest uniform pair")
+    ki, vi = np.nonzero(ok)
+    order = np.lexsort((vi, ki, Bt[ki, vi], Et[ki, vi]))
+    k, v = int(ki[order[0]]), int(vi[order[0]])
+    choices = [tuple(cell_options[c][k if c % 2 == 0 else v][2:5]) for c in range(n)]
+    return choices, int(Bt[k, v])
+
+
 def evaluate(cell_options, choices):
     """(total bytes, total E) of a choice vector."""
     B = E = 0

@@ -117,6 +117,27 @@ def test_allocator_bit_exact_vs_oracle(seed):
         assert lam_g == lam_o and tot_g == tot_o
 
 
+@pytest.mark.parametrize("seed", range(3))
+def test_allocator_variants_bit_exact_vs_oracle(seed):
+    from oracle.alloc import allocate_kv_split, allocate_uniform
+    w = get_workload(["llama8b_32k", "llama70b_128k", "llama8b_64k_b4"][seed])
+    s = api.make_shape(w)
+    nc = 2 * (w.n_layers // w.layers_per_group)
+    nrt, nrd = s.q_cap // 16 + 1, w.d_h // 16 + 1
+    n2, tT, td = make_random_tables(nc, nrt, nrd, 200 + seed)
+    phi = oracle.phi_table(w.d_h, 1 << 12, 1)
+    raw = raw_sequence_bytes(w)
+    opts = tables_to_options(n2, tT, td, phi, w)
+    for ratio in (2.0, 3.0, 5.0):
+        budget = int(raw / ratio)
+        for mode, fn in ((api.JOLT_ALLOC_KV_SPLIT, allocate_kv_split), (api.JOLT_ALLOC_UNIFORM, allocate_uniform)):
+            want, tot_o = fn(opts, budget)
+            got, tot_g = api.allocate_variant(s, n2, tT, td, phi, budget, mode)
+            assert [tuple(c) for c in got] == [tuple(c) for c in want] and tot_g == tot_o
+        got, tot = api.allocate_variant(s, n2, tT, td, phi, budget, api.JOLT_ALLOC_JOINT)
+        assert got == api.allocate(s, n2, tT, td, phi, budget)[0]
+
+
 def test_allocator_zero_budget_stores_nothing():
     # The empty choice (r_T = r_d = b = 0) costs no bytes, so every budget is feasible; at a
     # zero budget every cell keeps nothing and its error is its whole mass.

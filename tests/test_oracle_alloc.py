@@ -77,3 +77,40 @@ def test_zero_rank_pairs_with_zero_rank():
     opts = small_instance(1, 2)[0]
     for B, E, rT, rd, b in opts:
         assert (rT == 0) == (rd == 0)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_uniform_equals_brute_force_with_one_cell_per_kind(seed):
+    # with one key and one value cell every joint choice is uniform: the uniform allocator must
+    # reach the exhaustive minimum over all joint choices (a different search)
+    from oracle.alloc import allocate_uniform
+    opts = small_instance(2, seed)
+    lo = sum(min(o[0] for o in c) for c in opts)
+    hi = sum(max(o[0] for o in c) for c in opts)
+    for frac in np.linspace(0.0, 1.0, 7):
+        budget = int(lo + frac * (hi - lo))
+        ch, total = allocate_uniform(opts, budget)
+        B, E = evaluate(opts, ch)
+        assert B == total <= budget
+        assert E == pytest.approx(brute_force_allocate(opts, budget)[0], rel=1e-12, abs=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_ablation_allocations_are_feasible_and_never_beat_the_joint_optimum(seed):
+    # both ablations are feasible allocations, so neither goes below the exhaustive joint minimum;
+    # uniform shares one choice per kind; the decoupled split keeps keys within half the budget
+    from oracle.alloc import allocate_uniform, allocate_kv_split
+    opts = small_instance(4, seed)
+    lo = sum(min(o[0] for o in c) for c in opts)
+    hi = sum(max(o[0] for o in c) for c in opts)
+    for frac in (0.3, 0.6, 0.9):
+        budget = int(lo + frac * (hi - lo)) + 2 * max(max(o[0] for o in c) for c in opts)
+        best = brute_force_allocate(opts, budget)[0]
+        cu, tu = allocate_uniform(opts, budget)
+        assert len(set(cu[0::2])) == 1 and len(set(cu[1::2])) == 1
+        Bu, Eu = evaluate(opts, cu)
+        assert Bu == tu <= budget and Eu >= best * (1 - 1e-12)
+        ck, tk = allocate_kv_split(opts, budget)
+        Bk, Ek = evaluate(opts, ck)
+        assert Bk == tk <= budget and Ek >= best * (1 - 1e-12)
+        assert evaluate(opts[0::2], ck[0::2])[0] <= budget // 2
