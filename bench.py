@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--seqlen", type=int, default=None, help="override T (small profiling cases)")
     ap.add_argument("--nvtx", action="store_true", help="NVTX range 'jolt_step' around each timed step")
     ap.add_argument("--no-count", action="store_true", help="skip the CUPTI kernel count")
+    ap.add_argument("--cells-per-pass", type=int, default=0,
+                    help="cells jolt_analyze batches per pass (0: every cell of a kind in one pass)")
     ap.add_argument("--exact", action="store_true",
                     help="exact token-mode SVD (sketch width = L_g*n_kv*d_h: the JoLT backbone FlashJoLT replaces)")
     return ap.parse_args()
@@ -189,11 +191,14 @@ def run_reference(args, w, rank, world):
 # ---------------------------------------------------------------------------------------------
 
 class Step:
-    def __init__(self, w, ratio, device, seed_shift=0, exact=False):
+    def __init__(self, w, ratio, device, seed_shift=0, exact=False, cells_per_pass=0):
         from long_context_st_b200 import api
         self.api = api
         self.w = w
-        self.shape = api.make_shape(w, sketch_cols=w.n_cols) if exact else api.make_shape(w)
+        over = {"cells_per_pass": cells_per_pass or w.batch * w.n_groups}
+        if exact:
+            over["sketch_cols"] = w.n_cols
+        self.shape = api.make_shape(w, **over)
         self.dev = device
         self.K, self.V = make_kv(w, device=device)
         self.q = make_queries(w, device=device)
@@ -366,7 +371,7 @@ def main():
     hbm_peak, tc_burst, tc_sust, peak_src = load_peaks()
     from long_context_st_b200 import api
 
-    step = Step(w, ratio, dev, exact=args.exact)
+    step = Step(w, ratio, dev, exact=args.exact, cells_per_pass=args.cells_per_pass)
     torch.cuda.synchronize()
     for _ in range(max(3, args.warmup)):
         step.run()
@@ -456,6 +461,7 @@ def main():
                        "q_cap": step.shape.q_cap, "sketch_cols": step.shape.sketch_cols,
                        "power_iters": step.shape.power_iters, "l2": "inputs larger than L2 (no flush)",
                        "token_svd": "exact" if step.shape.sketch_cols == w.n_cols else "randomized",
+                       "cells_per_pass": step.shape.cells_per_pass,
                        "parallelism": f"dp{world}" if world > 1 else "single-gpu"},
             "breakdown_ms": {"analyze": t_an, "allocate_host": t_alloc, "compress": t_cmp, "decode": t_dec},
             "compress": {"raw_gbs": raw / ((t_an + t_alloc + t_cmp) / 1e3) / 1e9,
