@@ -5,6 +5,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstdio>
+#include <cstdlib>
+
 #include "jolt_internal.h"
 
 namespace jolt {
@@ -23,10 +26,19 @@ __device__ __forceinline__ void report_error(int32_t* err, int32_t code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// With JOLT_DEBUG set in the environment, a failing CUDA call is printed with its location.
+inline void jolt_note_cuda_error(cudaError_t e, const char* what, const char* file, int line) {
+  if (std::getenv("JOLT_DEBUG"))
+    std::fprintf(stderr, "jolt: %s:%d: %s -> %s\n", file, line, what, cudaGetErrorString(e));
+}
+
 #define JOLT_CUDA_TRY(expr)                                       \
   do {                                                            \
     cudaError_t e_ = (expr);                                      \
-    if (e_ != cudaSuccess) return JOLT_ERR_CUDA;                  \
+    if (e_ != cudaSuccess) {                                      \
+      jolt_note_cuda_error(e_, #expr, __FILE__, __LINE__);        \
+      return JOLT_ERR_CUDA;                                       \
+    }                                                             \
   } while (0)
 
 // ---- counter-based randomness (SplitMix64 as a hash of a 64-bit counter) --------------------

@@ -1,10 +1,13 @@
 // tcgen05 GEMM for sm_100a: TMA (128-byte swizzle) streams bf16 A/B tiles into a ring of shared-
-// memory stages; one thread issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM accumulator; four
-// warps drain TMEM with tcgen05.ld and store (or atomically add) fp32 C with coalesced writes.
+// memory stages; one thread issues tcgen05.mma into TMEM accumulators; epilogue warps drain TMEM
+// with tcgen05.ld and store (or atomically add) fp32 C.
 //
-// Warp roles (128 threads): warp 0 lane 0 = TMA producer, warp 1 lane 0 = MMA issuer, warp 2 =
-// TMEM allocator; all four warps run the epilogue. Every mbarrier wait is bounded (2 s) and
-// reports JOLT_ERR_TIMEOUT instead of hanging.
+// Two kernels. k_gemm: one output tile per CTA (128 threads: warp 0 lane 0 = TMA producer, warp
+// 1 lane 0 = MMA issuer, warp 2 = TMEM allocator, all four warps run the epilogue), used for
+// N <= 128 or a single 128-row tile. k_gemm_p: persistent, by default as CTA pairs
+// (cta_group::2, M = 256 per MMA, each SM stages half of B) with two TMEM accumulators so the
+// epilogue of one tile overlaps the main loop of the next. Every mbarrier wait is bounded (2 s)
+// and reports JOLT_ERR_TIMEOUT instead of hanging.
 //
 // Several (A_t, B_t) "terms" can accumulate into one tile: a fp32 operand split as hi + lo bf16
 // parts gives x*y ~ hi*hi + hi*lo + lo*hi with ~2^-16 relative error at bf16 tensor-core speed.
@@ -13,6 +16,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "gemm_tc.cuh"
@@ -38,7 +42,49 @@ struct GemmDev {
   int64_t ldc, c_bstride;
   int c_div, accumulate, c_upper, b_upper;
   int32_t* err;
+  int ntile, mtiles, n_tiles;  // persistent kernels: tile grid (N tiles fastest, then M, then z)
+  int c_vec;                   // C rows start 16-byte aligned (C, ldc, batch stride multiples of 4 floats)
 };
+
+// Store one 32-row x 32-column slice of an accumulator: lane = row (row0 + lane), r[i] = column
+// col0 + i. Plain stores of whole 32-column slices go straight from registers, 16 bytes at a
+// time along each lane's row; atomic accumulation (and ragged or unaligned slices) is transposed
+// through shared memory first, so that each instruction covers 32 consecutive columns of a row.
+__device__ __forceinline__ void store_chunk(const GemmDev& p, float* Cz, const uint32_t (&r)[32],
+                                            float* st, int row0, int col0, int lane) {
+  if (!p.accumulate && p.c_vec && col0 + 32 <= p.N) {
+    const int row = row0 + lane;
+    if (row < p.M) {
+      float4* dst = reinterpret_cast<float4*>(Cz + int64_t(row) * p.ldc + col0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                             __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+    }
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) st[lane * 33 + i] = __uint_as_float(r[i]);
+  __syncwarp();
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = st[i * 33 + lane];
+  __syncwarp();
+  const int col = col0 + lane;
+  const int nrow = min(32, p.M - row0);
+  if (col < p.N && nrow > 0) {
+    float* base = Cz + int64_t(row0) * p.ldc + col;
+    if (p.accumulate) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < nrow) atomicAdd(base + int64_t(i) * p.ldc, v[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < nrow) base[int64_t(i) * p.ldc] = v[i];
+    }
+  }
+}
 
 // MT: 128-row M tiles per CTA; with MT = 2 two accumulators share every B tile (half the B
 // bytes per flop, and each stage covers twice the MMA time).
@@ -55,19 +101,59 @@ struct Cfg {
   static constexpr int kSmem = 1024 + kStages * kStageBytes + kEpiBytes + 256;
 };
 
-__device__ __forceinline__ void load_operand(const CUtensorMap* map, int major, int fold, int bext,
-                                             uint32_t dst, uint32_t bar, int mn0, int rows, int k0,
-                                             int z) {
-  const int zb = bext > 1 ? z % bext : 0;
-  if (major == kMajorK) {
-    if (fold) sm100::tma_load_4d(dst, map, bar, k0 % fold, mn0, k0 / fold, zb);
-    else sm100::tma_load_3d(dst, map, bar, k0, mn0, zb);
+// TMA coordinates of one operand for one (tile, term), precomputed so that the producer's
+// per-k-block work is a few adds (its scalar address arithmetic, not memory, otherwise bounds the
+// stage rate). K-major: row mn0, k advanced by 64 per k-block (folded: k % fold, k / fold kept
+// incrementally). MN-major: per 64-wide chunk the (mn % fold, mn / fold) pair, k as given.
+struct OpCoord {
+  int fold, zb, mn0, kf, kq;
+  int c0[4], c2[4];
+};
+
+template <int MAJ>
+__device__ __forceinline__ void op_coord(OpCoord& o, int fold, int bext, int z, int mn0, int rows, int k0) {
+  o.fold = fold;
+  o.zb = bext > 1 ? z % bext : 0;
+  o.mn0 = mn0;
+  if (MAJ == kMajorK) {
+    o.kf = fold ? k0 % fold : k0;
+    o.kq = fold ? k0 / fold : 0;
   } else {
-    for (int i = 0; i < rows / 64; ++i) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
       const int mn = mn0 + 64 * i;
+      o.c0[i] = (i < rows / 64) ? (fold ? mn % fold : mn) : 0;
+      o.c2[i] = (i < rows / 64 && fold) ? mn / fold : 0;
+    }
+  }
+}
+
+template <int MAJ, int ROWS, bool PAIRLOAD>
+__device__ __forceinline__ void op_issue(const CUtensorMap* map, OpCoord& o, uint32_t dst, uint32_t bar, int k0) {
+  if (MAJ == kMajorK) {
+    if (o.fold) {
+      if (PAIRLOAD) sm100::tma_load_4d_pair(dst, map, bar, o.kf, o.mn0, o.kq, o.zb);
+      else sm100::tma_load_4d(dst, map, bar, o.kf, o.mn0, o.kq, o.zb);
+      o.kf += BK;
+      if (o.kf >= o.fold) {
+        o.kf -= o.fold;
+        ++o.kq;
+      }
+    } else {
+      if (PAIRLOAD) sm100::tma_load_3d_pair(dst, map, bar, k0, o.mn0, o.zb);
+      else sm100::tma_load_3d(dst, map, bar, k0, o.mn0, o.zb);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < ROWS / 64; ++i) {
       const uint32_t d = dst + i * (64 * BK * 2);
-      if (fold) sm100::tma_load_4d(d, map, bar, mn % fold, k0, mn / fold, zb);
-      else sm100::tma_load_3d(d, map, bar, mn, k0, zb);
+      if (o.fold) {
+        if (PAIRLOAD) sm100::tma_load_4d_pair(d, map, bar, o.c0[i], k0, o.c2[i], o.zb);
+        else sm100::tma_load_4d(d, map, bar, o.c0[i], k0, o.c2[i], o.zb);
+      } else {
+        if (PAIRLOAD) sm100::tma_load_3d_pair(d, map, bar, o.c0[i], k0, o.zb);
+        else sm100::tma_load_3d(d, map, bar, o.c0[i], k0, o.zb);
+      }
     }
   }
 }
@@ -116,22 +202,38 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
   const uint32_t smem_base = sm100::smem_u32(smem);
 
   if (n_iters > 0) {
-    if (warp == 0 && lane == 0) {
-      // ---- TMA producer ----
-      for (int it = 0; it < n_iters; ++it) {
-        const int s = it % C::kStages;
-        const uint32_t ph = (it / C::kStages) & 1;
-        if (!sm100::mbar_wait(empty_bar(s), ph ^ 1, p.err)) break;
-        const int t = it / nkb, kb = it % nkb;
-        const int k0 = (kb_begin + kb) * BK;
-        const uint32_t sa = smem_base + s * C::kStageBytes;
-        const uint32_t sb = sa + C::kABytes;
-        sm100::mbar_expect_tx(full_bar(s), C::kStageBytes);
+    if ((warp == 0 || warp == 2) && lane == 0) {
+      // ---- TMA producers: warp 0 streams A (and posts the stage's byte count), warp 2 streams
+      // B; both wait for the same free stage ----
+      const bool is_a = warp == 0;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = 0; ok && t < p.n_terms; ++t) {
+        int k0 = kb_begin * BK;
+        OpCoord o[MT];
+        if (is_a) {
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-          load_operand(&maps.a[t], AMAJ, p.a_fold[t], p.a_batch[t], sa + mt * C::kABytes1, full_bar(s), m0 + mt * BM,
-                       BM, k0, z);
-        load_operand(&maps.b[t], BMAJ, p.b_fold[t], p.b_batch[t], sb, full_bar(s), n0, BN, k0, z);
+          for (int mt = 0; mt < MT; ++mt) op_coord<AMAJ>(o[mt], p.a_fold[t], p.a_batch[t], z, m0 + mt * BM, BM, k0);
+        } else {
+          op_coord<BMAJ>(o[0], p.b_fold[t], p.b_batch[t], z, n0, BN, k0);
+        }
+        for (int kb = 0; kb < nkb; ++kb, k0 += BK) {
+          if (!sm100::mbar_wait(empty_bar(stage), phase ^ 1, p.err)) { ok = false; break; }
+          const uint32_t sa = smem_base + stage * C::kStageBytes;
+          if (is_a) {
+            sm100::mbar_expect_tx(full_bar(stage), C::kStageBytes);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+              op_issue<AMAJ, BM, false>(&maps.a[t], o[mt], sa + mt * C::kABytes1, full_bar(stage), k0);
+          } else {
+            op_issue<BMAJ, BN, false>(&maps.b[t], o[0], sa + C::kABytes, full_bar(stage), k0);
+          }
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
       }
     } else if (warp == 1 && lane == 0) {
       // ---- MMA issuer ----
@@ -173,27 +275,244 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
         uint32_t r[32];
         sm100::tmem_ld32(tmem + (uint32_t(warp * 32) << 16) + cc, r);
         sm100::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) st[lane * 33 + i] = __uint_as_float(r[i]);
-        __syncwarp();
-        const int col = n0 + c0 + lane;
-#pragma unroll 4
-        for (int i = 0; i < 32; ++i) {
-          const int row = m0 + mt * BM + warp * 32 + i;
-          if (row < p.M && col < p.N) {
-            float* dst = Cz + int64_t(row) * p.ldc + col;
-            const float v = st[i * 33 + lane];
-            if (p.accumulate) atomicAdd(dst, v);
-            else *dst = v;
-          }
-        }
-        __syncwarp();
+        store_chunk(p, Cz, r, st, m0 + mt * BM + warp * 32, n0 + c0, lane);
       }
     }
   }
   sm100::tc_fence_before();
   __syncthreads();
   if (warp == 2) sm100::tmem_dealloc(tmem, C::kTmemCols);
+}
+
+// ---- persistent variant: double-buffered accumulators -----------------------------------------
+// Each CTA (or CTA pair) walks tiles t = cluster, cluster + clusters, ... with the N tile fastest
+// (CTAs running at the same time share rows of A in L2). Two 128 x 256 fp32 accumulators live
+// in TMEM (all 512 columns), so four epilogue warps drain tile i while the MMA warp fills tile
+// i + 1 and two TMA warps stream its stages. 224 threads: warp 0 TMA for A, warp 6 TMA for B,
+// warp 1 MMA (+ TMEM allocation), warps 2..5 epilogue (TMEM lane quarter = warp % 4).
+// PAIR = 1 is the cta_group::2 form: a tile is 256 x 256, each CTA stages its 128 rows of A and
+// 128 columns of B, the even CTA issues the MMAs and owns the stage "full" barriers and the
+// accumulator "empty" barriers (the odd CTA's epilogue arrives there remotely).
+template <int PAIR>
+struct CfgP {
+  static constexpr int BN = 256;
+  static constexpr int kBCols = PAIR ? 128 : 256;
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = kBCols * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (192 * 1024) / kStageBytes < 8 ? (192 * 1024) / kStageBytes : 8;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kEpiBytes = 4 * 32 * 33 * 4;
+  static constexpr int kThreads = 224;
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + kEpiBytes + 256;
+};
+
+struct TileP {
+  int n0, m0, z, kb_begin, nkb;
+};
+
+// Tile t of the persistent walk; false if it has no work (below a c_upper diagonal, or a split-K
+// slice past a b_upper triangle). Every role calls this with the same t and gets the same answer.
+template <int ROWS>
+__device__ __forceinline__ bool tile_p(const GemmDev& p, int t, TileP& ti) {
+  constexpr int BN = 256;
+  const int nt = t % p.ntile;
+  const int r = t / p.ntile;
+  const int mt = r % p.mtiles;
+  const int zz = r / p.mtiles;
+  ti.n0 = nt * BN;
+  ti.m0 = mt * ROWS;
+  ti.z = zz / p.k_split;
+  const int kz = zz % p.k_split;
+  if (p.c_upper && ti.m0 >= ti.n0 + BN) return false;
+  const int nkb_all = (p.K + BK - 1) / BK;
+  const int nkb_total = p.b_upper ? min(nkb_all, (ti.n0 + BN + BK - 1) / BK) : nkb_all;
+  ti.kb_begin = kz * p.nkb_split;
+  ti.nkb = max(0, min(p.nkb_split, nkb_total - ti.kb_begin));
+  return ti.nkb > 0;
+}
+
+template <int PAIR, int AMAJ, int BMAJ>
+__global__ void __launch_bounds__(224, 1) k_gemm_p(const __grid_constant__ TmaPack maps, GemmDev p) {
+  using C = CfgP<PAIR>;
+  constexpr int BN = C::BN;
+  constexpr int ROWS = PAIR ? 2 * BM : BM;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* epi = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes + C::kEpiBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? sm100::cluster_ctarank() : 0u;
+  const int cluster = PAIR ? int(blockIdx.x >> 1) : int(blockIdx.x);
+  const int n_clusters = PAIR ? int(gridDim.x >> 1) : int(gridDim.x);
+
+  const uint32_t bar0 = sm100::smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+  auto accf_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };
+  auto acce_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 + b); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      sm100::mbar_init(full_bar(s), 1);
+      sm100::mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      sm100::mbar_init(accf_bar(b), 1);
+      sm100::mbar_init(acce_bar(b), PAIR ? 8 : 4);
+    }
+    *abort_flag = 0;
+    sm100::fence_mbar_init();
+    for (int t = 0; t < p.n_terms; ++t) {
+      sm100::prefetch_tmap(&maps.a[t]);
+      sm100::prefetch_tmap(&maps.b[t]);
+    }
+  }
+  if (warp == 1) {
+    if (PAIR) sm100::tmem_alloc_pair(sm100::smem_u32(tmem_slot), C::kTmemCols);
+    else sm100::tmem_alloc(sm100::smem_u32(tmem_slot), C::kTmemCols);
+  }
+  sm100::tc_fence_before();
+  if (PAIR) sm100::cluster_sync();
+  else __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t smem_base = sm100::smem_u32(smem);
+  auto aborted = [&]() { return *abort_flag != 0 || (p.err && *reinterpret_cast<volatile int32_t*>(p.err) != 0); };
+  auto fail = [&]() { *abort_flag = 1; };
+
+  if (warp == 0 || warp == 6) {
+    if (lane == 0) {
+      // ---- TMA producers: warp 0 streams A (and posts the stage's byte count), warp 6 streams
+      // B; both wait for the same free stage ----
+      const bool is_a = warp == 0;
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t full_own = full_bar(0);
+      const uint32_t full_lead = PAIR ? sm100::mapa_shared(full_bar(0), 0) : full_bar(0);
+      const uint32_t tx = PAIR ? 2 * C::kStageBytes : C::kStageBytes;
+      TileP ti;
+      bool ok = true;
+      for (int t = cluster; ok && t < p.n_tiles && !aborted(); t += n_clusters) {
+        if (!tile_p<ROWS>(p, t, ti)) continue;
+        const int arow = ti.m0 + int(rank) * BM;
+        const int bcol = ti.n0 + int(rank) * C::kBCols;
+        for (int term = 0; ok && term < p.n_terms; ++term) {
+          int k0 = ti.kb_begin * BK;
+          OpCoord o;
+          if (is_a) op_coord<AMAJ>(o, p.a_fold[term], p.a_batch[term], ti.z, arow, BM, k0);
+          else op_coord<BMAJ>(o, p.b_fold[term], p.b_batch[term], ti.z, bcol, C::kBCols, k0);
+          const CUtensorMap* m = is_a ? &maps.a[term] : &maps.b[term];
+          for (int kb = 0; kb < ti.nkb; ++kb, k0 += BK) {
+            if (!sm100::mbar_wait(empty_bar(stage), phase ^ 1, p.err)) { ok = false; break; }
+            const uint32_t sa = smem_base + stage * C::kStageBytes;
+            const uint32_t fb = (PAIR ? full_lead : full_own) + 8u * stage;
+            if (is_a) {
+              if (rank == 0) sm100::mbar_expect_tx(full_bar(stage), tx);
+              op_issue<AMAJ, BM, PAIR != 0>(m, o, sa, fb, k0);
+            } else {
+              op_issue<BMAJ, C::kBCols, PAIR != 0>(m, o, sa + C::kABytes, fb, k0);
+            }
+            if (++stage == C::kStages) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+        }
+      }
+      if (!ok) fail();
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---- MMA issuer ----
+      constexpr uint32_t idesc = sm100::idesc_bf16_f32(ROWS, BN, AMAJ, BMAJ);
+      // descriptor of stage 0's A / B tiles; per K16 step the start address advances by 32 bytes
+      // (K-major) or 2048 bytes (MN-major), per stage by kStageBytes (encoded >> 4)
+      const uint64_t a0 = AMAJ == kMajorK ? sm100::smem_desc_sw128(smem_base, 16, 1024)
+                                          : sm100::smem_desc_sw128(smem_base, 64 * BK * 2, 1024);
+      const uint64_t b0 = BMAJ == kMajorK ? sm100::smem_desc_sw128(smem_base + C::kABytes, 16, 1024)
+                                          : sm100::smem_desc_sw128(smem_base + C::kABytes, 64 * BK * 2, 1024);
+      constexpr uint32_t a_step = (AMAJ == kMajorK ? 32 : 2048) >> 4;
+      constexpr uint32_t b_step = (BMAJ == kMajorK ? 32 : 2048) >> 4;
+      int stage = 0, lt = 0;
+      uint32_t phase = 0;
+      TileP ti;
+      for (int t = cluster; t < p.n_tiles && !aborted(); t += n_clusters) {
+        if (!tile_p<ROWS>(p, t, ti)) continue;
+        const int b = lt & 1;
+        const uint32_t aph = (lt >> 1) & 1;
+        ++lt;
+        if (!sm100::mbar_wait(acce_bar(b), aph ^ 1, p.err)) { fail(); break; }
+        sm100::tc_fence_after();
+        const uint32_t dt = tmem + uint32_t(b * BN);
+        const int n_it = ti.nkb * p.n_terms;
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+          if (!sm100::mbar_wait(full_bar(stage), phase, p.err)) { ok = false; break; }
+          sm100::tc_fence_after();
+          const uint64_t soff = uint64_t((uint32_t(stage) * C::kStageBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = a0 + soff + kk * a_step;
+            const uint64_t bd = b0 + soff + kk * b_step;
+            const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+            if (PAIR) sm100::mma_bf16_pair(dt, ad, bd, idesc, acc);
+            else sm100::mma_bf16(dt, ad, bd, idesc, acc);
+          }
+          if (PAIR) sm100::mma_commit_pair(empty_bar(stage), 0x3);
+          else sm100::mma_commit(empty_bar(stage));
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) { fail(); break; }
+        if (PAIR) sm100::mma_commit_pair(accf_bar(b), 0x3);
+        else sm100::mma_commit(accf_bar(b));
+      }
+    }
+  } else if (warp >= 2 && warp <= 5) {
+    // ---- epilogue: TMEM -> registers -> smem transpose -> coalesced global ----
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    float* st = epi + (warp - 2) * 32 * 33;
+    const uint32_t acce_target = PAIR ? sm100::mapa_shared(acce_bar(0), 0) : acce_bar(0);
+    int lt = 0;
+    TileP ti;
+    for (int t = cluster; t < p.n_tiles && !aborted(); t += n_clusters) {
+      if (!tile_p<ROWS>(p, t, ti)) continue;
+      const int b = lt & 1;
+      const uint32_t aph = (lt >> 1) & 1;
+      ++lt;
+      if (!sm100::mbar_wait(accf_bar(b), aph, p.err)) { fail(); break; }
+      sm100::tc_fence_after();
+      float* Cz = p.C + int64_t(ti.z / p.c_div) * p.c_bstride;
+      const int rbase = ti.m0 + int(rank) * BM + q * 32;
+      for (int cc = 0; cc < BN; cc += 32) {
+        uint32_t r[32];
+        sm100::tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(b * BN + cc), r);
+        sm100::tmem_ld_wait();
+        store_chunk(p, Cz, r, st, rbase, ti.n0 + cc, lane);
+      }
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (PAIR) sm100::mbar_arrive_cluster(acce_target + 8u * b);
+        else sm100::mbar_arrive(acce_bar(b));
+      }
+    }
+  }
+  __syncwarp();
+  sm100::tc_fence_before();
+  if (PAIR) sm100::cluster_sync();
+  else __syncthreads();
+  sm100::tc_fence_after();
+  if (warp == 1) {
+    if (PAIR) sm100::tmem_dealloc_pair(tmem, C::kTmemCols);
+    else sm100::tmem_dealloc(tmem, C::kTmemCols);
+  }
 }
 
 // ---- host: tensor maps ----------------------------------------------------------------------
@@ -206,6 +525,35 @@ jolt_status launch(const TmaPack& maps, const GemmDev& d, dim3 grid, cudaStream_
   kern<<<grid, 128, C::kSmem, st>>>(maps, d);
   JOLT_CUDA_TRY(cudaGetLastError());
   return JOLT_OK;
+}
+
+template <int PAIR, int AM, int BMJ>
+jolt_status launch_p(const TmaPack& maps, const GemmDev& d, dim3 grid, cudaStream_t st) {
+  using C = CfgP<PAIR>;
+  auto kern = k_gemm_p<PAIR, AM, BMJ>;
+  JOLT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = PAIR ? 2 : 1;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  JOLT_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, maps, d));
+  return JOLT_OK;
+}
+
+template <int PAIR>
+jolt_status launch_pers(int am, int bm, const TmaPack& maps, const GemmDev& d, dim3 grid, cudaStream_t st) {
+  if (am == kMajorK && bm == kMajorK) return launch_p<PAIR, kMajorK, kMajorK>(maps, d, grid, st);
+  if (am == kMajorK && bm == kMajorMN) return launch_p<PAIR, kMajorK, kMajorMN>(maps, d, grid, st);
+  if (am == kMajorMN && bm == kMajorK) return launch_p<PAIR, kMajorMN, kMajorK>(maps, d, grid, st);
+  return launch_p<PAIR, kMajorMN, kMajorMN>(maps, d, grid, st);
 }
 
 template <int BN, int MT>
@@ -276,37 +624,56 @@ bool make_tensor_map(CUtensorMap* m, const Operand& o, int rows) {
 
 namespace {
 
-// Tile plan: 128-row tiles per CTA (MT) and split-K factor. Estimated time = whole waves of one
-// CTA per SM x the k-blocks one CTA runs (+1 for its epilogue), with two-accumulator CTAs ~1.2x
-// faster per flop (measured); tiles a symmetric (c_upper) output skips are not counted.
+// Tile plan: the one-tile-per-CTA kernel with MT 128-row accumulators and the split-K factor that
+// minimise the estimated time, i.e. whole waves of one CTA per SM x (k-blocks per CTA + 1 for
+// its epilogue) over the relative per-SM speed (two accumulators sharing B run ~1.2x the flops
+// per cycle of one). Tiles a symmetric (c_upper) output skips are not counted.
+// The persistent forms (JOLT_GEMM_PLAN=p1: single CTAs, p2: CTA pairs; N > 128 and more than one
+// 128-row tile) are faster in isolation at a fixed clock, but in a whole compression pass under
+// the board's power cap they lower the clock the rest of the pass runs at by more than they
+// gain, so the one-tile kernel is the default (JOLT_GEMM_PLAN=1sm names it explicitly).
 struct TilePlan {
-  int MT, k_split;
+  int kind, MT, k_split;  // kind: 0 one tile per CTA, 2 persistent single CTA, 3 persistent pair
 };
 
 TilePlan plan_tiles(const GemmCall& g, int BN) {
   constexpr int kSMs = 148;
+  const char* force = std::getenv("JOLT_GEMM_PLAN");
+  int only = -1;
+  if (force) {
+    if (!std::strcmp(force, "1sm")) only = 0;
+    else if (!std::strcmp(force, "p1")) only = 2;
+    else if (!std::strcmp(force, "p2")) only = 3;
+  }
+  const bool pers_ok = BN == 256 && g.M > BM;
+  if (only < 0 || !pers_ok) only = 0;
   const int64_t ntile = (g.N + BN - 1) / BN, kb = (g.K + BK - 1) / BK;
-  auto active = [&](int MT) {
-    const int64_t mt = (g.M + BM * MT - 1) / (BM * MT);
+  // tiles with work when one CTA (or pair) covers `rows` rows
+  auto active = [&](int rows) {
+    const int64_t mt = (g.M + rows - 1) / rows;
     int64_t a = 0;
     for (int64_t i = 0; i < mt; ++i)
-      for (int64_t j = 0; j < ntile; ++j) a += (g.c_upper && i * BM * MT >= j * BN + BN) ? 0 : 1;
+      for (int64_t j = 0; j < ntile; ++j) a += (g.c_upper && i * rows >= j * BN + BN) ? 0 : 1;
     return a * g.batch;
   };
   const int kmax = g.k_split == 0 ? int(std::max<int64_t>(1, std::min<int64_t>(64, kb / 2))) : g.k_split;
   const int kmin = g.k_split == 0 ? 1 : g.k_split;
-  TilePlan best{1, kmin};
+  TilePlan best{only, 1, kmin};
   double best_t = 1e300;
-  for (int MT = 2; MT >= 1; --MT) {
+  for (int MT = (only == 0 ? 2 : 1); MT >= 1; --MT) {
     if (MT == 2 && g.M <= BM) continue;
-    const int64_t act = active(MT);
+    const bool pair = only == 3;
+    const int slots = pair ? kSMs / 2 : kSMs;  // tiles in flight at once
+    const int64_t act = active((pair ? 2 : 1) * BM * MT);
     for (int k = kmin; k <= kmax; ++k) {
-      const int64_t ctas = act * k;
-      const double waves = double((ctas + kSMs - 1) / kSMs);
-      const double t = waves * MT * (double((kb + k - 1) / k) + 1.0) / (MT == 2 ? 1.2 : 1.0);
+      const int64_t tiles = act * k;
+      const double rounds = double((tiles + slots - 1) / slots);
+      const double per = double((kb + k - 1) / k);
+      // one-tile kernel: two accumulators sharing B run ~1.2x the flops per cycle of one
+      const double t = only == 0 ? rounds * MT * (per + 1.0) / (MT == 2 ? 1.2 : 1.0) : rounds * (per + 2.0);
       if (t < best_t * 0.999) {
         best_t = t;
-        best = TilePlan{MT, k};
+        best = TilePlan{only, MT, k};
       }
     }
   }
@@ -326,20 +693,20 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   // BN: 256 whenever N exceeds one 128-wide tile — a 128 x 256 tile runs ~1.5x more flops per
   // cycle than 128 x 128 (half the operand bytes per flop), which outweighs the padding of N
   const int BN = g.N > 128 ? 256 : 128;
+  const TilePlan tp = plan_tiles(g, BN);
+  const int MT = tp.MT;
   TmaPack maps;
   memset(&maps, 0, sizeof(maps));
   GemmDev d{};
   for (int t = 0; t < g.n_terms; ++t) {
     if (!make_tensor_map(&maps.a[t], g.A[t], BM)) return JOLT_ERR_INVALID_ARG;
-    if (!make_tensor_map(&maps.b[t], g.B[t], BN)) return JOLT_ERR_INVALID_ARG;
+    if (!make_tensor_map(&maps.b[t], g.B[t], tp.kind == 3 ? BN / 2 : BN)) return JOLT_ERR_INVALID_ARG;
     d.a_fold[t] = int(g.A[t].fold);
     d.b_fold[t] = int(g.B[t].fold);
     d.a_batch[t] = g.A[t].batch_stride ? int(g.A[t].batch) : 1;
     d.b_batch[t] = g.B[t].batch_stride ? int(g.B[t].batch) : 1;
     if ((g.A[t].fold && g.A[t].fold % 64) || (g.B[t].fold && g.B[t].fold % 64)) return JOLT_ERR_INVALID_ARG;
   }
-  const TilePlan tp = plan_tiles(g, BN);
-  const int MT = tp.MT;
   d.M = g.M; d.N = g.N; d.K = g.K; d.n_terms = g.n_terms; d.k_split = tp.k_split;
   const int nkb = (g.K + BK - 1) / BK;
   d.nkb_split = (nkb + tp.k_split - 1) / tp.k_split;
@@ -348,12 +715,31 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   d.c_upper = g.c_upper ? 1 : 0;
   d.b_upper = g.b_upper ? 1 : 0;
   d.err = g.err;
+  d.c_vec = (reinterpret_cast<uintptr_t>(g.C) % 16 == 0 && g.ldc % 4 == 0 && g.c_batch_stride % 4 == 0) ? 1 : 0;
   const int64_t ntile = (g.N + BN - 1) / BN, zc = int64_t(g.batch) * tp.k_split;
-  const dim3 grid(unsigned(ntile), unsigned((g.M + BM * MT - 1) / (BM * MT)), unsigned(zc));
-  if (grid.y > 65535 || grid.z > 65535) return JOLT_ERR_INVALID_ARG;
+  // single CTAs: (N tile, M tile); pairs: (2 x N tile + CTA of the pair, pair tile), so that
+  // consecutive CTAs share the rows of A
+  const bool pair = tp.kind == 3;
+  const int64_t rows = int64_t(pair ? 2 : 1) * BM * MT;
+  const int64_t gy = (g.M + rows - 1) / rows;
+  dim3 grid{unsigned(ntile * (pair ? 2 : 1)), unsigned(gy), unsigned(zc)};
+  if (tp.kind >= 2) {
+    // persistent: one CTA (pair) per SM (pair of SMs), tiles walked in-kernel
+    const int64_t n_tiles = ntile * gy * zc;
+    if (n_tiles > INT32_MAX) return JOLT_ERR_INVALID_ARG;
+    d.ntile = int(ntile);
+    d.mtiles = int(gy);
+    d.n_tiles = int(n_tiles);
+    const int64_t slots = pair ? 74 : 148;
+    grid = dim3{unsigned(std::min(n_tiles, slots) * (pair ? 2 : 1)), 1u, 1u};
+  } else if (gy > 65535 || zc > 65535) {
+    return JOLT_ERR_INVALID_ARG;
+  }
   // algorithmic flops: a triangular B or a wanted upper triangle of C halves the product
   const double tri = (g.b_upper || g.c_upper) ? 0.5 : 1.0;
   StatScope sc(JOLT_K_GEMM, st, tri * 2.0 * g.M * double(g.N) * g.K * g.batch * g.n_terms, 0.0);
+  if (tp.kind == 3) return launch_pers<1>(am, bm, maps, d, grid, st);
+  if (tp.kind == 2) return launch_pers<0>(am, bm, maps, d, grid, st);
   if (MT == 2) return BN == 256 ? launch_bn<256, 2>(am, bm, maps, d, grid, st) : launch_bn<128, 2>(am, bm, maps, d, grid, st);
   return BN == 256 ? launch_bn<256, 1>(am, bm, maps, d, grid, st) : launch_bn<128, 1>(am, bm, maps, d, grid, st);
 }

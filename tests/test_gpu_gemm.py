@@ -20,7 +20,10 @@ def ref_mm(A, B, a_mn, b_mn):
                                    (4096, 256, 128), (64, 384, 200),
                                    # grids large enough for two 128-row tiles per CTA, ragged M/N/K
                                    (16000, 1152, 192), (80000, 200, 72)])
-def test_gemm_majors_and_ragged(cuda_ok, a_mn, b_mn, M, N, K):
+@pytest.mark.parametrize("plan", ["auto", "1sm", "p1", "p2"])
+def test_gemm_majors_and_ragged(cuda_ok, monkeypatch, plan, a_mn, b_mn, M, N, K):
+    # restrict the tile plan to the one-tile kernel or the persistent single-CTA / CTA-pair forms
+    monkeypatch.setenv("JOLT_GEMM_PLAN", plan)
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K + a_mn * 2 + b_mn)
     A = torch.randn((K, M) if a_mn else (M, K), generator=g, device="cuda").to(torch.bfloat16)
     B = torch.randn((K, N) if b_mn else (N, K), generator=g, device="cuda").to(torch.bfloat16)
@@ -36,7 +39,9 @@ def tol(K):
     return 2e-7 * K ** 0.5 + 1e-6
 
 
-def test_gemm_split_k_and_batch(cuda_ok):
+@pytest.mark.parametrize("plan", ["1sm", "p1", "p2"])
+def test_gemm_split_k_and_batch(cuda_ok, monkeypatch, plan):
+    monkeypatch.setenv("JOLT_GEMM_PLAN", plan)
     g = torch.Generator(device="cuda").manual_seed(1)
     bt, M, N, K = 3, 384, 256, 8192
     A = torch.randn(bt, K, M, generator=g, device="cuda").to(torch.bfloat16)
