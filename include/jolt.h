@@ -274,6 +274,15 @@ jolt_status jolt_gemm_bf16(const void* A, int32_t a_mn_major, const void* B, int
                            int64_t ldc, int32_t batch, int64_t stride_a, int64_t stride_b,
                            int64_t stride_c, int32_t k_split, int32_t accumulate, void* stream);
 
+/* The same product with the fp32 result split into bf16 parts by the GEMM's epilogue instead of
+ * being stored: Ch = bf16_rn(c), and when Cl is not NULL, Cl = bf16_rn(c - Ch), for every result c
+ * (the hi / lo split the compressor's CholeskyQR passes feed back into the tensor cores). Ch, Cl
+ * (device, bf16) use C's layout (ldc, stride_c). No split-K and no accumulation. */
+jolt_status jolt_gemm_bf16_hilo(const void* A, int32_t a_mn_major, const void* B, int32_t b_mn_major,
+                                void* Ch, void* Cl, int32_t M, int32_t N, int32_t K, int64_t lda,
+                                int64_t ldb, int64_t ldc, int32_t batch, int64_t stride_a,
+                                int64_t stride_b, int64_t stride_c, void* stream);
+
 /* Symmetric eigendecomposition of `batch` fp32 matrices A [batch][n][n] (device) by block Jacobi
  * (the solver the compressor uses for the Rayleigh-Ritz and feature-mode steps): eigenvalues
  * descending into evals [batch][n], eigenvectors as the columns of evecs [batch][n][n] (device).

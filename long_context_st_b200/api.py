@@ -256,6 +256,27 @@ def gemm_bf16(A, B, a_mn_major=False, b_mn_major=False, C=None, k_split=1, accum
     return C3 if batched else C3[0]
 
 
+def gemm_bf16_hilo(A, B, a_mn_major=False, b_mn_major=False, lo=True, stream=None):
+    """The product of gemm_bf16 returned as its bf16 hi / lo split (hi = bf16(c), lo =
+    bf16(c - hi)) written by the GEMM epilogue. Returns (hi, lo or None), bf16 [batch?, M, N]."""
+    batched = A.dim() == 3
+    A3 = A if batched else A[None]
+    B3 = B if batched else B[None]
+    bt = A3.shape[0]
+    M = A3.shape[2] if a_mn_major else A3.shape[1]
+    K = A3.shape[1] if a_mn_major else A3.shape[2]
+    N = B3.shape[2] if b_mn_major else B3.shape[1]
+    hi = torch.empty(bt, M, N, dtype=torch.bfloat16, device=A.device)
+    lo_t = torch.empty_like(hi) if lo else None
+    check(lib().jolt_gemm_bf16_hilo(_ptr(A3), int(a_mn_major), _ptr(B3), int(b_mn_major), _ptr(hi),
+                                    _ptr(lo_t) if lo else None, M, N, K, A3.stride(1), B3.stride(1),
+                                    hi.stride(1), bt, A3.stride(0), B3.stride(0), hi.stride(0),
+                                    _stream(stream)), "jolt_gemm_bf16_hilo")
+    if batched:
+        return hi, lo_t
+    return hi[0], (lo_t[0] if lo else None)
+
+
 def sym_eig(A, stream=None):
     """Eigen-decomposition of symmetric fp32 matrices [batch?, n, n] on the GPU (block Jacobi).
     Returns (evals descending [batch?, n], evecs [batch?, n, n] with eigenvectors as columns)."""

@@ -41,7 +41,7 @@ struct Plan {
   int64_t cell_elems;
   size_t off_ut, off_pass, off_cmp, total;
   // pass scratch offsets (relative to off_pass)
-  size_t om, Y, Yh, Yl, Gm, Rh, Rl, Z, Zh, Zl, ev, evec, Vh, Vl, Sd, evd, evecd, nrm, chol, jac, xb;
+  size_t om, Yh2, Yl2, Yh, Yl, Gm, Rh, Rl, Z, Zh, Zl, ev, evec, Vh, Vl, Sd, evd, evecd, nrm, chol, jac, xb;
   size_t g64, ev64, evec64, sd64, evd64, evecd64;  // exact path (sketch width == n)
   // compress scratch (relative to off_cmp)
   size_t uh, ul, um, ylh, sy, evy, evecy, ud, blh, bh, bm, bl, xt, jac2;
@@ -75,7 +75,8 @@ Plan make_plan(const jolt_shape& s) {
   p.off_pass = pass0;
   const size_t rowsmax = std::max(T, n);
   p.om = rel(l * n * 2);
-  p.Y = rel(C * rowsmax * l * 4);
+  p.Yh2 = rel(C * rowsmax * l * 2);  // second hi / lo buffer: orthonormalisation passes ping-pong
+  p.Yl2 = rel(C * rowsmax * l * 2);
   p.Yh = rel(C * rowsmax * l * 2);
   p.Yl = rel(C * rowsmax * l * 2);
   p.Gm = rel(C * l * l * 4);
@@ -147,11 +148,6 @@ __global__ void k_norm2(const T* __restrict__ X, int64_t cell_elems, double* out
   }
   for (int m = 16; m; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
   if ((threadIdx.x & 31) == 0) atomicAdd(&out[c], acc);
-}
-
-__global__ void k_f32_to_bf16(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, int64_t n) {
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x)
-    y[e] = __float2bfloat16_rn(x[e]);
 }
 
 // Copy the first r columns of U [T][q] (fp32) to the stored cache (dtype) and to bf16 GEMM operands
@@ -423,7 +419,11 @@ Operand xunfold(const void* X, int major, const Plan& p, int C) {
   return o;
 }
 
-// Y <- orth(Y), Y fp32 [C][rows][l]: CholeskyQR passes with hi/lo bf16 Grams and products.
+// Orthonormalise the columns of Y [C][rows][l] by CholeskyQR passes with bf16 hi/lo Grams and
+// products. Two forms of Y:
+//  - fp32 (Yf != nullptr, updated in place): each pass splits Yf into hi/lo buffer 0 first;
+//  - bf16 parts already in hi/lo buffer *cur (Yf == nullptr): each pass writes its product's hi/lo
+//    split straight from the GEMM epilogue into the other buffer, and *cur follows the result.
 // Shifted passes (s = 1e-4 * ||G||_F) run until the Cholesky's smallest pivot ratio R_jj^2 / G_jj
 // reaches 0.1; then unshifted passes run until one factors a Gram whose ratio is >= 0.9 (an
 // almost orthonormal input, so the output is orthonormal to the hi/lo precision). A breakdown of
@@ -435,18 +435,22 @@ constexpr int kMaxOrthPasses = 8;
 // (one term, exact), Q = Y_hi (R^-1 hi + lo) — and stop after the first pass whose pivots show a
 // well-conditioned input (ratio >= 0.1). The final basis (polish = true) uses hi/lo terms
 // throughout and gets the unshifted passes.
-jolt_status orth(const Ctx& c, float* Y, int rows, int C, bool polish = true) {
+jolt_status orth(const Ctx& c, float* Yf, int* cur, int rows, int C, bool polish = true) {
   const Plan& p = c.p;
   const int l = p.l;
-  __nv_bfloat16* Yh = c.at<__nv_bfloat16>(p.Yh);
-  __nv_bfloat16* Yl = c.at<__nv_bfloat16>(p.Yl);
+  __nv_bfloat16* Yh_b[2] = {c.at<__nv_bfloat16>(p.Yh), c.at<__nv_bfloat16>(p.Yh2)};
+  __nv_bfloat16* Yl_b[2] = {c.at<__nv_bfloat16>(p.Yl), c.at<__nv_bfloat16>(p.Yl2)};
   float* Gm = c.at<float>(p.Gm);
   __nv_bfloat16* Rh = c.at<__nv_bfloat16>(p.Rh);
   __nv_bfloat16* Rl = c.at<__nv_bfloat16>(p.Rl);
+  int b = Yf ? 0 : *cur;
   bool conditioned = false;
   for (int pass = 0; pass < kMaxOrthPasses; ++pass) {
-    jolt_status r = split_bf16(Y, l, rows, l, C, int64_t(rows) * l, Yh, polish ? Yl : nullptr, l, int64_t(rows) * l, c.st);
-    if (r) return r;
+    __nv_bfloat16* Yh = Yh_b[b];
+    __nv_bfloat16* Yl = Yl_b[b];
+    jolt_status r;
+    if (Yf && (r = split_bf16(Yf, l, rows, l, C, int64_t(rows) * l, Yh, polish ? Yl : nullptr, l, int64_t(rows) * l, c.st)))
+      return r;
     JOLT_CUDA_TRY(cudaMemsetAsync(Gm, 0, size_t(C) * l * l * 4, c.st));
     GemmCall g;
     g.M = l; g.N = l; g.K = rows; g.n_terms = polish ? 3 : 1;
@@ -464,20 +468,17 @@ jolt_status orth(const Ctx& c, float* Y, int rows, int C, bool polish = true) {
       std::vector<float> h(size_t(C) * l * l);
       cudaMemcpyAsync(h.data(), Gm, h.size() * 4, cudaMemcpyDeviceToHost, c.st);
       cudaStreamSynchronize(c.st);
-      for (int b = 0; b < C; ++b) {
-        const float* gb = h.data() + size_t(b) * l * l;
+      for (int bb = 0; bb < C; ++bb) {
+        const float* gb = h.data() + size_t(bb) * l * l;
         int bad = 0;
-        float dmn = 1e30f, dmx = 0.f, asym = 0.f;
+        float dmn = 1e30f, dmx = 0.f;
         for (int i = 0; i < l; ++i) {
           dmn = std::min(dmn, gb[size_t(i) * l + i]);
           dmx = std::max(dmx, gb[size_t(i) * l + i]);
-          for (int j = 0; j < l; ++j) {
-            bad += !std::isfinite(gb[size_t(i) * l + j]);
-            asym = std::max(asym, std::fabs(gb[size_t(i) * l + j] - gb[size_t(j) * l + i]));
-          }
+          for (int j = i; j < l; ++j) bad += !std::isfinite(gb[size_t(i) * l + j]);
         }
-        std::fprintf(stderr, "jolt gram: rows %d pass %d cell %d nonfinite %d diag [%g, %g] asym %g\n", rows, pass, b,
-                     bad, dmn, dmx, asym);
+        std::fprintf(stderr, "jolt gram: rows %d pass %d cell %d nonfinite %d diag [%g, %g]\n", rows, pass, bb, bad,
+                     dmn, dmx);
       }
     }
     const bool last = pass == kMaxOrthPasses - 1;
@@ -505,9 +506,18 @@ jolt_status orth(const Ctx& c, float* Y, int rows, int C, bool polish = true) {
     t.A[0] = ykh; t.B[0] = rh;
     t.A[1] = ykh; t.B[1] = rl;
     t.A[2] = ykl; t.B[2] = rh;
-    t.C = Y; t.ldc = l; t.c_batch_stride = int64_t(rows) * l; t.batch = C; t.err = c.err;
+    if (Yf) {
+      t.C = Yf;
+    } else {
+      // the product cannot overwrite the parts it reads: write the other buffer
+      b ^= 1;
+      t.Ch = Yh_b[b];
+      t.Cl = polish ? Yl_b[b] : nullptr;
+    }
+    t.ldc = l; t.c_batch_stride = int64_t(rows) * l; t.batch = C; t.err = c.err;
     t.b_upper = true;  // R^-1 is upper triangular
     if ((r = gemm_tc(t, c.st))) return r;
+    if (cur) *cur = b;
     if (shift == 0.0 && ratio >= 0.9f) return JOLT_OK;
     if (!polish && ratio >= 0.1f) return JOLT_OK;
     if (ratio >= 0.1f) conditioned = true;
@@ -597,44 +607,52 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
     return JOLT_OK;
   }
   if (q > 0) {
-    float* Y = c.at<float>(p.Y);
     float* Z = c.at<float>(p.Z);
-    __nv_bfloat16* Yh = c.at<__nv_bfloat16>(p.Yh);
-    __nv_bfloat16* Yl = c.at<__nv_bfloat16>(p.Yl);
+    __nv_bfloat16* Yh_b[2] = {c.at<__nv_bfloat16>(p.Yh), c.at<__nv_bfloat16>(p.Yh2)};
+    __nv_bfloat16* Yl_b[2] = {c.at<__nv_bfloat16>(p.Yl), c.at<__nv_bfloat16>(p.Yl2)};
     __nv_bfloat16* Zh = c.at<__nv_bfloat16>(p.Zh);
     __nv_bfloat16* Zl = c.at<__nv_bfloat16>(p.Zl);
     const __nv_bfloat16* om = c.at<__nv_bfloat16>(p.om);
+    // The sketch Y lives only as bf16 hi (/ lo) parts written by the GEMM epilogues (its fp32 value
+    // is never needed beyond its split). The lo part is kept where the next step reads it: before
+    // the final (polished) orthonormalisation.
+    int cur = 0;
     // Y = X Omega
     {
       GemmCall g;
       g.M = T; g.N = l; g.K = n;
       g.A[0] = xunfold(Xb, kMajorK, p, C);
       g.B[0] = plain(om, kMajorK, n, l, n);
-      g.C = Y; g.ldc = l; g.c_batch_stride = int64_t(T) * l; g.batch = C; g.err = c.err;
+      g.Ch = Yh_b[0];
+      g.Cl = s.power_iters == 0 ? Yl_b[0] : nullptr;
+      g.ldc = l; g.c_batch_stride = int64_t(T) * l; g.batch = C; g.err = c.err;
       if ((r = gemm_tc(g, c.st))) return r;
     }
     for (int it = 0; it < s.power_iters; ++it) {
-      if ((r = orth(c, Y, T, C, false))) return r;
-      if ((r = split_bf16(Y, l, T, l, C, int64_t(T) * l, Yh, nullptr, l, int64_t(T) * l, c.st))) return r;
+      if ((r = orth(c, nullptr, &cur, T, C, false))) return r;
       JOLT_CUDA_TRY(cudaMemsetAsync(Z, 0, size_t(C) * n * l * 4, c.st));
       GemmCall g;
       g.M = n; g.N = l; g.K = T;
       g.A[0] = xunfold(Xb, kMajorMN, p, C);
-      g.B[0] = plain(Yh, kMajorMN, l, T, l, C, int64_t(T) * l);
+      g.B[0] = plain(Yh_b[cur], kMajorMN, l, T, l, C, int64_t(T) * l);
       g.C = Z; g.ldc = l; g.c_batch_stride = int64_t(n) * l; g.batch = C;
       g.k_split = 0; g.accumulate = true; g.err = c.err;
       if ((r = gemm_tc(g, c.st))) return r;
-      if ((r = orth(c, Z, n, C, false))) return r;
+      if ((r = orth(c, Z, nullptr, n, C, false))) return r;
       if ((r = split_bf16(Z, l, n, l, C, int64_t(n) * l, Zh, nullptr, l, int64_t(n) * l, c.st))) return r;
       GemmCall h;
       h.M = T; h.N = l; h.K = n;
       h.A[0] = xunfold(Xb, kMajorK, p, C);
       h.B[0] = plain(Zh, kMajorMN, l, n, l, C, int64_t(n) * l);
-      h.C = Y; h.ldc = l; h.c_batch_stride = int64_t(T) * l; h.batch = C; h.err = c.err;
+      cur = 0;
+      h.Ch = Yh_b[0];
+      h.Cl = it + 1 == s.power_iters ? Yl_b[0] : nullptr;
+      h.ldc = l; h.c_batch_stride = int64_t(T) * l; h.batch = C; h.err = c.err;
       if ((r = gemm_tc(h, c.st))) return r;
     }
-    if ((r = orth(c, Y, T, C))) return r;  // Q
-    if ((r = split_bf16(Y, l, T, l, C, int64_t(T) * l, Yh, Yl, l, int64_t(T) * l, c.st))) return r;
+    if ((r = orth(c, nullptr, &cur, T, C, true))) return r;  // Q, as hi / lo parts in buffer cur
+    __nv_bfloat16* Yh = Yh_b[cur];
+    __nv_bfloat16* Yl = Yl_b[cur];
     // B^T = X^T Q  (n x l), hi/lo terms of Q
     JOLT_CUDA_TRY(cudaMemsetAsync(Z, 0, size_t(C) * n * l * 4, c.st));
     {

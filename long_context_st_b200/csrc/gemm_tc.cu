@@ -43,15 +43,73 @@ struct GemmDev {
   int c_div, accumulate, c_upper, b_upper;
   int32_t* err;
   int ntile, mtiles, n_tiles;  // persistent kernels: tile grid (N tiles fastest, then M, then z)
-  int c_vec;                   // C rows start 16-byte aligned (C, ldc, batch stride multiples of 4 floats)
+  int c_vec;                   // output rows start 16-byte aligned (pointer, ldc, batch stride)
+  __nv_bfloat16* Ch;           // bf16 hi (and lo) outputs instead of fp32 C
+  __nv_bfloat16* Cl;
 };
+
+__device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// bf16 hi / lo split of one fp32 value (lo = rounding of the exact remainder).
+__device__ __forceinline__ void split_hl(float v, __nv_bfloat16& h, __nv_bfloat16& l) {
+  h = __float2bfloat16_rn(v);
+  l = __float2bfloat16_rn(v - __bfloat162float(h));
+}
 
 // Store one 32-row x 32-column slice of an accumulator: lane = row (row0 + lane), r[i] = column
 // col0 + i. Plain stores of whole 32-column slices go straight from registers, 16 bytes at a
 // time along each lane's row; atomic accumulation (and ragged or unaligned slices) is transposed
 // through shared memory first, so that each instruction covers 32 consecutive columns of a row.
-__device__ __forceinline__ void store_chunk(const GemmDev& p, float* Cz, const uint32_t (&r)[32],
+// zoff: element offset of this tile's batch entry in the output.
+__device__ __forceinline__ void store_chunk(const GemmDev& p, int64_t zoff, const uint32_t (&r)[32],
                                             float* st, int row0, int col0, int lane) {
+  if (p.Ch) {
+    if (p.c_vec && col0 + 32 <= p.N) {
+      const int row = row0 + lane;
+      if (row < p.M) {
+        const int64_t o = zoff + int64_t(row) * p.ldc + col0;
+        uint4* dh = reinterpret_cast<uint4*>(p.Ch + o);
+        uint4* dl = p.Cl ? reinterpret_cast<uint4*>(p.Cl + o) : nullptr;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat16 h0, l0, h1, l1;
+            split_hl(__uint_as_float(r[8 * j + 2 * e]), h0, l0);
+            split_hl(__uint_as_float(r[8 * j + 2 * e + 1]), h1, l1);
+            hw[e] = bf2_bits(__halves2bfloat162(h0, h1));
+            lw[e] = bf2_bits(__halves2bfloat162(l0, l1));
+          }
+          dh[j] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          if (dl) dl[j] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+      }
+      return;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) st[lane * 33 + i] = __uint_as_float(r[i]);
+    __syncwarp();
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = st[i * 33 + lane];
+    __syncwarp();
+    const int col = col0 + lane;
+    const int nrow = min(32, p.M - row0);
+    if (col < p.N && nrow > 0) {
+      const int64_t o = zoff + int64_t(row0) * p.ldc + col;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < nrow) {
+          __nv_bfloat16 h, l;
+          split_hl(v[i], h, l);
+          p.Ch[o + int64_t(i) * p.ldc] = h;
+          if (p.Cl) p.Cl[o + int64_t(i) * p.ldc] = l;
+        }
+    }
+    return;
+  }
+  float* Cz = p.C + zoff;
   if (!p.accumulate && p.c_vec && col0 + 32 <= p.N) {
     const int row = row0 + lane;
     if (row < p.M) {
@@ -269,13 +327,13 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
     sm100::tc_fence_after();
     if (ok) {
       float* st = epi + warp * 32 * 33;
-      float* Cz = p.C + int64_t(z / p.c_div) * p.c_bstride;
+      const int64_t zoff = int64_t(z / p.c_div) * p.c_bstride;
       for (int cc = 0; cc < MT * BN; cc += 32) {
         const int mt = cc / BN, c0 = cc % BN;
         uint32_t r[32];
         sm100::tmem_ld32(tmem + (uint32_t(warp * 32) << 16) + cc, r);
         sm100::tmem_ld_wait();
-        store_chunk(p, Cz, r, st, m0 + mt * BM + warp * 32, n0 + c0, lane);
+        store_chunk(p, zoff, r, st, m0 + mt * BM + warp * 32, n0 + c0, lane);
       }
     }
   }
@@ -488,13 +546,13 @@ __global__ void __launch_bounds__(224, 1) k_gemm_p(const __grid_constant__ TmaPa
       ++lt;
       if (!sm100::mbar_wait(accf_bar(b), aph, p.err)) { fail(); break; }
       sm100::tc_fence_after();
-      float* Cz = p.C + int64_t(ti.z / p.c_div) * p.c_bstride;
+      const int64_t zoff = int64_t(ti.z / p.c_div) * p.c_bstride;
       const int rbase = ti.m0 + int(rank) * BM + q * 32;
       for (int cc = 0; cc < BN; cc += 32) {
         uint32_t r[32];
         sm100::tmem_ld32(tmem + (uint32_t(q * 32) << 16) + uint32_t(b * BN + cc), r);
         sm100::tmem_ld_wait();
-        store_chunk(p, Cz, r, st, rbase, ti.n0 + cc, lane);
+        store_chunk(p, zoff, r, st, rbase, ti.n0 + cc, lane);
       }
       sm100::tc_fence_before();
       __syncwarp();
@@ -656,7 +714,7 @@ TilePlan plan_tiles(const GemmCall& g, int BN) {
       for (int64_t j = 0; j < ntile; ++j) a += (g.c_upper && i * rows >= j * BN + BN) ? 0 : 1;
     return a * g.batch;
   };
-  const int kmax = g.k_split == 0 ? int(std::max<int64_t>(1, std::min<int64_t>(64, kb / 2))) : g.k_split;
+  const int kmax = g.Ch ? 1 : (g.k_split == 0 ? int(std::max<int64_t>(1, std::min<int64_t>(64, kb / 2))) : g.k_split);
   const int kmin = g.k_split == 0 ? 1 : g.k_split;
   TilePlan best{only, 1, kmin};
   double best_t = 1e300;
@@ -684,8 +742,11 @@ TilePlan plan_tiles(const GemmCall& g, int BN) {
 
 jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return JOLT_OK;
-  if (g.n_terms < 1 || g.n_terms > kMaxTerms || !g.C || g.batch < 1 || g.k_split < 0 || g.c_batch_div < 1)
+  if (g.n_terms < 1 || g.n_terms > kMaxTerms || (!g.C && !g.Ch) || (g.C && g.Ch) || g.batch < 1 || g.k_split < 0 ||
+      g.c_batch_div < 1)
     return JOLT_ERR_INVALID_ARG;
+  if (g.Ch && (g.accumulate || g.k_split > 1 || g.c_batch_div > 1)) return JOLT_ERR_INVALID_ARG;
+  if (g.Cl && !g.Ch) return JOLT_ERR_INVALID_ARG;
   if ((g.k_split != 1 || g.c_batch_div > 1) && !g.accumulate) return JOLT_ERR_INVALID_ARG;
   const int am = g.A[0].major, bm = g.B[0].major;
   for (int t = 0; t < g.n_terms; ++t)
@@ -715,7 +776,13 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   d.c_upper = g.c_upper ? 1 : 0;
   d.b_upper = g.b_upper ? 1 : 0;
   d.err = g.err;
-  d.c_vec = (reinterpret_cast<uintptr_t>(g.C) % 16 == 0 && g.ldc % 4 == 0 && g.c_batch_stride % 4 == 0) ? 1 : 0;
+  d.Ch = g.Ch;
+  d.Cl = g.Cl;
+  if (g.Ch)
+    d.c_vec = (reinterpret_cast<uintptr_t>(g.Ch) % 16 == 0 && reinterpret_cast<uintptr_t>(g.Cl) % 16 == 0 &&
+               g.ldc % 8 == 0 && g.c_batch_stride % 8 == 0) ? 1 : 0;
+  else
+    d.c_vec = (reinterpret_cast<uintptr_t>(g.C) % 16 == 0 && g.ldc % 4 == 0 && g.c_batch_stride % 4 == 0) ? 1 : 0;
   const int64_t ntile = (g.N + BN - 1) / BN, zc = int64_t(g.batch) * tp.k_split;
   // single CTAs: (N tile, M tile); pairs: (2 x N tile + CTA of the pair, pair tile), so that
   // consecutive CTAs share the rows of A
@@ -771,5 +838,31 @@ extern "C" jolt_status jolt_gemm_bf16(const void* A, int32_t a_mn_major, const v
   g.C = C; g.ldc = ldc; g.c_batch_stride = stride_c; g.batch = batch;
   g.k_split = k_split; g.accumulate = accumulate != 0;
   if (k_split > 1 && !accumulate) return JOLT_ERR_INVALID_ARG;
+  return gemm_tc(g, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" jolt_status jolt_gemm_bf16_hilo(const void* A, int32_t a_mn_major, const void* B,
+                                           int32_t b_mn_major, void* Ch, void* Cl, int32_t M, int32_t N,
+                                           int32_t K, int64_t lda, int64_t ldb, int64_t ldc, int32_t batch,
+                                           int64_t stride_a, int64_t stride_b, int64_t stride_c,
+                                           void* stream) {
+  if (M < 0 || N < 0 || K < 0 || batch < 1) return JOLT_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return JOLT_OK;
+  if (!A || !B || !Ch || ldc < N || K == 0) return JOLT_ERR_INVALID_ARG;
+  GemmCall g;
+  g.M = M; g.N = N; g.K = K;
+  Operand& a = g.A[0];
+  a.ptr = A; a.major = a_mn_major ? kMajorMN : kMajorK;
+  a.inner = a_mn_major ? M : K; a.outer = a_mn_major ? K : M; a.outer_stride = lda;
+  a.batch = batch; a.batch_stride = stride_a;
+  Operand& b = g.B[0];
+  b.ptr = B; b.major = b_mn_major ? kMajorMN : kMajorK;
+  b.inner = b_mn_major ? N : K; b.outer = b_mn_major ? K : N; b.outer_stride = ldb;
+  b.batch = batch; b.batch_stride = stride_b;
+  if (lda < a.inner || ldb < b.inner) return JOLT_ERR_INVALID_ARG;
+  g.Ch = static_cast<__nv_bfloat16*>(Ch);
+  g.Cl = static_cast<__nv_bfloat16*>(Cl);
+  g.ldc = ldc; g.c_batch_stride = stride_c; g.batch = batch;
+  g.k_split = 1;
   return gemm_tc(g, static_cast<cudaStream_t>(stream));
 }

@@ -2,6 +2,7 @@
 // memory described by TMA tensor maps, fp32 accumulation in TMEM, fp32 output.
 #pragma once
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 #include "common.cuh"
 
@@ -33,6 +34,11 @@ struct GemmCall {
   int n_terms = 1;
   Operand A[kMaxTerms], B[kMaxTerms];
   float* C = nullptr;
+  // Instead of fp32 C (C = nullptr): the bf16 rounding of each result to Ch and, when Cl is given,
+  // the bf16 rounding of the remainder to Cl (the hi/lo split of the fp32 result), with C's
+  // ldc / batch layout. Requires accumulate = false and no split-K.
+  __nv_bfloat16* Ch = nullptr;
+  __nv_bfloat16* Cl = nullptr;
   int64_t ldc = 0;
   int64_t c_batch_stride = 0;  // elements between C batch entries
   int c_batch_div = 1;         // C entry of operand batch z is z / c_batch_div

@@ -52,3 +52,23 @@ def test_gemm_split_k_and_batch(cuda_ok, monkeypatch, plan):
     R = ref_mm(A, B, True, True)
     err = (C.double() - R).abs().max().item() / R.abs().max().item()
     assert err < tol(K), err
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 1)])
+@pytest.mark.parametrize("M,N,K", [(1000, 1152, 1000), (16000, 1152, 192), (304, 200, 72), (4096, 96, 640)])
+def test_gemm_hilo_outputs_split_the_fp32_result(cuda_ok, a_mn, b_mn, M, N, K):
+    """The epilogue's bf16 hi / lo outputs are exactly the split of the fp32 result the same
+    kernel stores (same tile plan, same accumulation order)."""
+    g = torch.Generator(device="cuda").manual_seed(M + 5 * N + 7 * K + a_mn + 2 * b_mn)
+    A = torch.randn((K, M) if a_mn else (M, K), generator=g, device="cuda").to(torch.bfloat16)
+    B = torch.randn((K, N) if b_mn else (N, K), generator=g, device="cuda").to(torch.bfloat16)
+    C = api.gemm_bf16(A, B, a_mn, b_mn)
+    hi, lo = api.gemm_bf16_hilo(A, B, a_mn, b_mn)
+    hi_only, none = api.gemm_bf16_hilo(A, B, a_mn, b_mn, lo=False)
+    torch.cuda.synchronize()
+    h_ref = C.to(torch.bfloat16)
+    l_ref = (C - h_ref.float()).to(torch.bfloat16)
+    assert none is None
+    assert torch.equal(hi.view(torch.int16), h_ref.view(torch.int16))
+    assert torch.equal(hi_only.view(torch.int16), h_ref.view(torch.int16))
+    assert torch.equal(lo.view(torch.int16), l_ref.view(torch.int16))
