@@ -283,6 +283,17 @@ jolt_status jolt_gemm_bf16_hilo(const void* A, int32_t a_mn_major, const void* B
                                 int64_t ldb, int64_t ldc, int32_t batch, int64_t stride_a,
                                 int64_t stride_b, int64_t stride_c, void* stream);
 
+/* The same product with N = 128 coded as residual rows instead of stored (the compressor's fused
+ * reconstruction + residual step): for each output row c = C[z][m][:], x = X[z*M + m][:] - c is
+ * rotated as jolt_rotate_rows does, quantised to b bits and packed as jolt_quantize_pack does,
+ * into codes [batch*M][16*b] and sz (fp16 pairs) [batch*M][2]. A K-major (lda), B N-major (ldb);
+ * X (device) bf16, or fp32 when x_f32, [batch*M][128]. codes, X 16-byte aligned. err (device
+ * int32, may be NULL) gets JOLT_ERR_NUMERIC for a non-finite row, scale or zero. b in {2,4,8}. */
+jolt_status jolt_gemm_bf16_residual(const void* A, const void* B, int32_t M, int32_t K, int64_t lda,
+                                    int64_t ldb, int32_t batch, int64_t stride_a, int64_t stride_b,
+                                    const void* X, int32_t x_f32, uint64_t seed, int32_t b,
+                                    uint8_t* codes, void* sz, int32_t* err, void* stream);
+
 /* Symmetric eigendecomposition of `batch` fp32 matrices A [batch][n][n] (device) by block Jacobi
  * (the solver the compressor uses for the Rayleigh-Ritz and feature-mode steps): eigenvalues
  * descending into evals [batch][n], eigenvectors as the columns of evecs [batch][n][n] (device).

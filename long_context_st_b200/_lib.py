@@ -89,6 +89,9 @@ SIGNATURES = [
     ("jolt_gemm_bf16_hilo", C.c_int, [_P, C.c_int32, _P, C.c_int32, _P, _P, C.c_int32, C.c_int32,
                                       C.c_int32, C.c_int64, C.c_int64, C.c_int64, C.c_int32, C.c_int64,
                                       C.c_int64, C.c_int64, _P]),
+    ("jolt_gemm_bf16_residual", C.c_int, [_P, _P, C.c_int32, C.c_int32, C.c_int64, C.c_int64, C.c_int32,
+                                          C.c_int64, C.c_int64, _P, C.c_int32, C.c_uint64, C.c_int32, _P,
+                                          _P, _P, _P]),
     ("jolt_sym_eig_workspace", C.c_size_t, [C.c_int32, C.c_int32]),
     ("jolt_stats_enable", None, [C.c_int32]),
     ("jolt_stats_read", C.c_int, [C.POINTER(KernelStat), C.c_int32]),

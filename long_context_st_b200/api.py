@@ -277,6 +277,25 @@ def gemm_bf16_hilo(A, B, a_mn_major=False, b_mn_major=False, lo=True, stream=Non
     return hi[0], (lo_t[0] if lo else None)
 
 
+def gemm_bf16_residual(A, B, X, seed, b, stream=None):
+    """Fused reconstruction + residual coding: rows of X - A @ B (A [batch?, M, K] bf16 K-major,
+    B [batch?, K, 128] bf16, X [batch?, M, 128] bf16 or fp32) rotated, quantised to b bits and
+    packed. Returns (codes uint8 [batch?*M, 16*b], sz fp16 [batch?*M, 2], err int32 [1])."""
+    batched = A.dim() == 3
+    A3 = A if batched else A[None]
+    B3 = B if batched else B[None]
+    bt, M, K = A3.shape
+    X2 = X.reshape(bt * M, 128)
+    codes = torch.empty(bt * M, 16 * b, dtype=torch.uint8, device=A.device)
+    sz = torch.empty(bt * M, 2, dtype=torch.float16, device=A.device)
+    err = torch.zeros(1, dtype=torch.int32, device=A.device)
+    check(lib().jolt_gemm_bf16_residual(_ptr(A3), _ptr(B3), M, K, A3.stride(1), B3.stride(1), bt,
+                                        A3.stride(0), B3.stride(0), _ptr(X2),
+                                        int(X2.dtype == torch.float32), seed, b, _ptr(codes), _ptr(sz),
+                                        _ptr(err), _stream(stream)), "jolt_gemm_bf16_residual")
+    return codes, sz, err
+
+
 def sym_eig(A, stream=None):
     """Eigen-decomposition of symmetric fp32 matrices [batch?, n, n] on the GPU (block Jacobi).
     Returns (evals descending [batch?, n], evecs [batch?, n, n] with eigenvectors as columns)."""

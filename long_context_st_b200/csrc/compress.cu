@@ -221,16 +221,44 @@ __device__ __forceinline__ float ld_fac_any(const uint8_t* p, int64_t i, int f32
   return f32 ? reinterpret_cast<const float*>(p)[i] : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
 }
 
-// B[lh][r][i] = sum_j G[lh][r][j] * U_d[i][j] from the stored values (fp32 out).
-__global__ void k_recon_b(const uint8_t* __restrict__ G, const uint8_t* __restrict__ Ud, int64_t nrows, int rd,
-                          int d, int f32, float* __restrict__ B) {
-  const int64_t total = nrows * d;
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total; e += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = e / d;
-    const int i = int(e % d);
-    float a = 0.f;
-    for (int j = 0; j < rd; ++j) a += ld_fac_any(G, r * rd + j, f32) * ld_fac_any(Ud, int64_t(i) * rd + j, f32);
-    B[e] = a;
+// B[lh][r][i] = sum_j G[lh][r][j] * U_d[i][j] from the stored values (fp32 out), with rows r of
+// all (lh, r) pairs flattened. A block covers 32 rows x all D columns; G and U_d pass through
+// shared memory 32 values of j at a time; each sum runs over j in order (one fused multiply-add
+// per term).
+template <int D>
+__global__ void __launch_bounds__(256) k_recon_b(const uint8_t* __restrict__ G, const uint8_t* __restrict__ Ud,
+                                                 int64_t nrows, int rd, int f32, float* __restrict__ B) {
+  constexpr int kGroups = 256 / D, kRows = 32 / kGroups;
+  __shared__ float Gs[32][33];
+  __shared__ float Us[32][D];
+  const int i = threadIdx.x % D, g = threadIdx.x / D;
+  const int64_t r0 = int64_t(blockIdx.x) * 32;
+  float a[kRows];
+#pragma unroll
+  for (int k = 0; k < kRows; ++k) a[k] = 0.f;
+  for (int j0 = 0; j0 < rd; j0 += 32) {
+    const int nj = min(32, rd - j0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < 32 * 32; e += 256) {
+      const int rr = e / 32, jj = e % 32;
+      const int64_t r = r0 + rr;
+      Gs[rr][jj] = (r < nrows && jj < nj) ? ld_fac_any(G, r * rd + j0 + jj, f32) : 0.f;
+    }
+    for (int e = threadIdx.x; e < 32 * D; e += 256) {
+      const int jj = e / D, ii = e % D;
+      Us[jj][ii] = jj < nj ? ld_fac_any(Ud, int64_t(ii) * rd + j0 + jj, f32) : 0.f;
+    }
+    __syncthreads();
+    for (int jj = 0; jj < nj; ++jj) {
+      const float u = Us[jj][i];
+#pragma unroll
+      for (int k = 0; k < kRows; ++k) a[k] += Gs[g + kGroups * k][jj] * u;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kRows; ++k) {
+    const int64_t r = r0 + g + kGroups * k;
+    if (r < nrows) B[r * D + i] = a[k];
   }
 }
 
@@ -906,8 +934,21 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
       const jolt_cell_choice ch = choices[cell];
       const uint8_t* Xk = static_cast<const uint8_t*>(kv ? v : k) + int64_t(bg) * p.cell_elems * (io32 ? 4 : 2);
       float* Xt = nullptr;
+      bool coded = false;  // residual already coded by the fused X~ GEMM
       if (ch.r_T > 0) {
         const int rT = ch.r_T, rd = ch.r_d, slot = slot_of[cell - c0];
+        uint8_t* cud = cb + offs[5 * cell + 1];
+        uint8_t* cg = cb + offs[5 * cell + 2];
+        const float* ylh = c.atc<float>(p.ylh) + int64_t(slot) * LgH * q * d;
+        const float* evs = evecy + int64_t(slot) * d * d;
+        // U_d = first rd eigenvector columns (stored dtype), then G = Y U_d (stored dtype)
+        k_store_ut<<<grid1(int64_t(d) * rd), 256, 0, c.st>>>(evs, d, d, rd, f32, cud, nullptr, nullptr, nullptr);
+        k_proj_small<<<grid1(int64_t(LgH) * rT * rd), 256, 0, c.st>>>(ylh, int64_t(LgH) * rT, d, evs, d, rd, f32, cg);
+      }
+      if (ch.r_T > 0 && ch.b > 0) {
+        // X~ = U^s B with B = G^s U_d^s^T, to fp32 accuracy: 3-way bf16 splits, terms of order <= 2
+        // (only the residual needs it: a cell without one stores the factors alone)
+        const int rT = ch.r_T, rd = ch.r_d;
         uint8_t* cud = cb + offs[5 * cell + 1];
         uint8_t* cg = cb + offs[5 * cell + 2];
         __nv_bfloat16 *uh, *ul, *um;
@@ -916,18 +957,17 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
           uh = reinterpret_cast<__nv_bfloat16*>(cb + offs[5 * cell + 0]);
           ul = um = nullptr;
         }
-        const float* ylh = c.atc<float>(p.ylh) + int64_t(slot) * LgH * q * d;
-        const float* evs = evecy + int64_t(slot) * d * d;
         float* xt = c.atc<float>(p.xt);
-        // U_d = first rd eigenvector columns (stored dtype), then G = Y U_d (stored dtype)
-        k_store_ut<<<grid1(int64_t(d) * rd), 256, 0, c.st>>>(evs, d, d, rd, f32, cud, nullptr, nullptr, nullptr);
-        k_proj_small<<<grid1(int64_t(LgH) * rT * rd), 256, 0, c.st>>>(ylh, int64_t(LgH) * rT, d, evs, d, rd, f32, cg);
-        // X~ = U^s B with B = G^s U_d^s^T, to fp32 accuracy: 3-way bf16 splits, terms of order <= 2
         __nv_bfloat16* bh = c.atc<__nv_bfloat16>(p.bh);
         __nv_bfloat16* bm = c.atc<__nv_bfloat16>(p.bm);
         __nv_bfloat16* bl = c.atc<__nv_bfloat16>(p.bl);
         float* blh = c.atc<float>(p.blh);
-        k_recon_b<<<grid1(int64_t(LgH) * rT * d), 256, 0, c.st>>>(cg, cud, int64_t(LgH) * rT, rd, d, f32, blh);
+        {
+          const int64_t nrows = int64_t(LgH) * rT;
+          const unsigned gb = unsigned((nrows + 31) / 32);
+          if (d == 128) k_recon_b<128><<<gb, 256, 0, c.st>>>(cg, cud, nrows, rd, f32, blh);
+          else k_recon_b<64><<<gb, 256, 0, c.st>>>(cg, cud, nrows, rd, f32, blh);
+        }
         if ((r = split3_bf16(blh, int64_t(LgH) * rT * d, bh, bm, bl, c.st))) return r;
         {
           GemmCall g;
@@ -947,12 +987,30 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
                 ++nt;
               }
           g.n_terms = nt;
-          g.C = xt; g.ldc = d; g.c_batch_stride = int64_t(T) * d; g.batch = LgH; g.err = c.err;
-          if ((r = gemm_tc(g, c.st))) return r;
+          g.batch = LgH; g.err = c.err;
+          // d = 128: the GEMM's epilogue codes the residual rows X - X~ directly (X~ never
+          // reaches memory); otherwise X~ is stored and coded by k_residual
+          uint8_t* codes = cb + offs[5 * cell + 3];
+          void* szp = cb + offs[5 * cell + 4];
+          ResidualEpi e;
+          e.X = Xk; e.x_f32 = io32 ? 1 : 0; e.T = T; e.seed = s.rot_seed; e.b = ch.b;
+          e.codes = codes; e.sz = szp;
+          const bool fuse = d == 128 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
+                            reinterpret_cast<uintptr_t>(Xk) % 16 == 0 && reinterpret_cast<uintptr_t>(szp) % 4 == 0;
+          if (fuse) {
+            g.res = &e;
+            const int64_t rows = int64_t(LgH) * T;
+            StatScope sc(JOLT_K_RESIDUAL, c.st, 0.0, double(rows) * d * (io32 ? 4 : 2) + double(rows) * (d * ch.b / 8 + 4));
+            if ((r = gemm_tc(g, c.st))) return r;
+            coded = true;
+          } else {
+            g.C = xt; g.ldc = d; g.c_batch_stride = int64_t(T) * d;
+            if ((r = gemm_tc(g, c.st))) return r;
+            Xt = xt;
+          }
         }
-        Xt = xt;
       }
-      if (ch.b > 0) {
+      if (ch.b > 0 && !coded) {
         uint8_t* codes = cb + offs[5 * cell + 3];
         __half2* sz = reinterpret_cast<__half2*>(cb + offs[5 * cell + 4]);
         const int64_t rows = int64_t(LgH) * T;

@@ -46,6 +46,7 @@ struct GemmDev {
   int c_vec;                   // output rows start 16-byte aligned (pointer, ldc, batch stride)
   __nv_bfloat16* Ch;           // bf16 hi (and lo) outputs instead of fp32 C
   __nv_bfloat16* Cl;
+  ResidualEpi res;             // fused residual coding (k_gemm<..., EPI = 1>)
 };
 
 __device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 h) { return *reinterpret_cast<uint32_t*>(&h); }
@@ -146,16 +147,18 @@ __device__ __forceinline__ void store_chunk(const GemmDev& p, int64_t zoff, cons
 
 // MT: 128-row M tiles per CTA; with MT = 2 two accumulators share every B tile (half the B
 // bytes per flop, and each stage covers twice the MMA time).
-template <int BN, int MT>
+// EPI = 1 (fused residual coding, compute-heavy epilogue): three stages and no transpose buffer,
+// so that two CTAs fit on an SM and one's epilogue overlaps the other's main loop.
+template <int BN, int MT, int EPI = 0>
 struct Cfg {
   static constexpr int kABytes1 = BM * BK * 2;
   static constexpr int kABytes = MT * kABytes1;
   static constexpr int kBBytes = BN * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (192 * 1024) / kStageBytes < 6 ? (192 * 1024) / kStageBytes : 6;
+  static constexpr int kStages = EPI ? 3 : ((192 * 1024) / kStageBytes < 6 ? (192 * 1024) / kStageBytes : 6);
   static constexpr int kCols = MT * BN;
   static constexpr int kTmemCols = kCols <= 32 ? 32 : (kCols <= 64 ? 64 : (kCols <= 128 ? 128 : (kCols <= 256 ? 256 : 512)));
-  static constexpr int kEpiBytes = 4 * 32 * 33 * 4;
+  static constexpr int kEpiBytes = EPI ? 0 : 4 * 32 * 33 * 4;
   static constexpr int kSmem = 1024 + kStages * kStageBytes + kEpiBytes + 256;
 };
 
@@ -216,14 +219,124 @@ __device__ __forceinline__ void op_issue(const CUtensorMap* map, OpCoord& o, uin
   }
 }
 
-template <int BN, int AMAJ, int BMAJ, int MT>
-__global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack maps, GemmDev p) {
-  using C = Cfg<BN, MT>;
+// ---- fused residual coding epilogue (one thread per token row of 128 features) ---------------
+// The arithmetic is the stand-alone coder's, operation for operation: x = X - x~ (fp32), signs,
+// fast Walsh-Hadamard butterflies with strides 1, 2, ..., 64 ((lo, hi) -> (lo + hi, lo - hi)),
+// x rsqrt(128); min / max; step = (max - min) / (2^b - 1) and zero = min rounded to fp16;
+// code = clip(rint((x - zero) / scale)), packed little-endian.
+template <int B>
+__device__ __forceinline__ void res_pack_store(const float (&v)[128], float s, float zf, uint8_t* dst) {
+  constexpr int kPer = 32 / B;
+  const float levels = float((1 << B) - 1);
+#pragma unroll
+  for (int q = 0; q < B; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t acc = 0;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int i = (q * 4 + e) * kPer + k;
+        float c = 0.f;
+        if (s != 0.f) {
+          c = rintf(__fdiv_rn(__fsub_rn(v[i], zf), s));
+          c = fminf(fmaxf(c, 0.f), levels);
+        }
+        acc |= uint32_t(c) << (k * B);
+      }
+      w[e] = acc;
+    }
+    reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+template <int MT, int BN>
+__device__ __forceinline__ void residual_epilogue(const GemmDev& p, uint32_t tmem, int warp, int lane, int m0, int z,
+                                                  const uint32_t* smask) {
+  const float isd = rsqrtf(128.f);
+  for (int mt = 0; mt < MT; ++mt) {
+    float v[128];
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      uint32_t r[32];
+      sm100::tmem_ld32(tmem + (uint32_t(warp * 32) << 16) + uint32_t(mt * BN + ch * 32), r);
+      sm100::tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[ch * 32 + i] = __uint_as_float(r[i]);
+    }
+    const int t = m0 + mt * BM + warp * 32 + lane;
+    if (t >= p.M) continue;
+    const int64_t rr = int64_t(z) * p.res.T + t;
+    if (p.res.x_f32) {
+      const float4* xr = reinterpret_cast<const float4*>(static_cast<const float*>(p.res.X) + rr * 128);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float4 x = xr[j];
+        v[4 * j] = x.x - v[4 * j];
+        v[4 * j + 1] = x.y - v[4 * j + 1];
+        v[4 * j + 2] = x.z - v[4 * j + 2];
+        v[4 * j + 3] = x.w - v[4 * j + 3];
+      }
+    } else {
+      const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.res.X) + rr * 128);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint4 x = xr[j];
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+          v[8 * j + 2 * e] = f.x - v[8 * j + 2 * e];
+          v[8 * j + 2 * e + 1] = f.y - v[8 * j + 2 * e + 1];
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 128; ++i)
+      if ((smask[i >> 5] >> (i & 31)) & 1u) v[i] = -v[i];
+#pragma unroll
+    for (int st = 1; st < 128; st <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        if ((i & st) == 0) {
+          const float a = v[i], b = v[i + st];
+          v[i] = a + b;
+          v[i + st] = a - b;
+        }
+      }
+    }
+    bool ok = true;
+    float mn, mx;
+#pragma unroll
+    for (int i = 0; i < 128; ++i) {
+      v[i] *= isd;
+      ok &= isfinite(v[i]);
+      mn = i ? fminf(mn, v[i]) : v[i];
+      mx = i ? fmaxf(mx, v[i]) : v[i];
+    }
+    const float levels = float((1 << p.res.b) - 1);
+    const float step = __fdiv_rn(__fsub_rn(mx, mn), levels);
+    const __half hs = __float2half_rn(step);
+    const __half hz = __float2half_rn(mn);
+    const float sc = __half2float(hs), zf = __half2float(hz);
+    if (!(ok && isfinite(sc) && isfinite(zf))) report_error(p.err, JOLT_ERR_NUMERIC);
+    uint8_t* dst = p.res.codes + rr * (16 * p.res.b);
+    if (p.res.b == 2) res_pack_store<2>(v, sc, zf, dst);
+    else if (p.res.b == 4) res_pack_store<4>(v, sc, zf, dst);
+    else res_pack_store<8>(v, sc, zf, dst);
+    static_cast<__half2*>(p.res.sz)[rr] = __halves2half2(hs, hz);
+  }
+}
+
+template <int BN, int AMAJ, int BMAJ, int MT, int EPI = 0>
+__global__ void __launch_bounds__(128, EPI ? 2 : 1) k_gemm(const __grid_constant__ TmaPack maps, GemmDev p) {
+  using C = Cfg<BN, MT, EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* epi = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes + C::kEpiBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 1);
+  uint32_t* smask = tmem_slot + 1;  // EPI = 1: rotation signs of the 128 features, one bit each
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM * MT;
@@ -253,6 +366,13 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
     }
   }
   if (warp == 2) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), C::kTmemCols);
+  if (EPI == 1 && warp == 3) {
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint32_t m = __ballot_sync(0xffffffffu, rot_sign(p.res.seed, w * 32 + lane) < 0.f);
+      if (lane == 0) smask[w] = m;
+    }
+  }
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
@@ -325,7 +445,9 @@ __global__ void __launch_bounds__(128, 1) k_gemm(const __grid_constant__ TmaPack
     // ---- epilogue: TMEM -> registers -> smem transpose -> coalesced global ----
     const bool ok = sm100::mbar_wait(done_bar, 0, p.err);
     sm100::tc_fence_after();
-    if (ok) {
+    if (ok && EPI == 1) {
+      residual_epilogue<MT, BN>(p, tmem, warp, lane, m0, z, smask);
+    } else if (ok) {
       float* st = epi + warp * 32 * 33;
       const int64_t zoff = int64_t(z / p.c_div) * p.c_bstride;
       for (int cc = 0; cc < MT * BN; cc += 32) {
@@ -614,6 +736,16 @@ jolt_status launch_pers(int am, int bm, const TmaPack& maps, const GemmDev& d, d
   return launch_p<PAIR, kMajorMN, kMajorMN>(maps, d, grid, st);
 }
 
+template <int MT>
+jolt_status launch_res(const TmaPack& maps, const GemmDev& d, dim3 grid, cudaStream_t st) {
+  using C = Cfg<128, MT, 1>;
+  auto kern = k_gemm<128, kMajorK, kMajorMN, MT, 1>;
+  JOLT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem));
+  kern<<<grid, 128, C::kSmem, st>>>(maps, d);
+  JOLT_CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
+}
+
 template <int BN, int MT>
 jolt_status launch_bn(int am, int bm, const TmaPack& maps, const GemmDev& d, dim3 grid, cudaStream_t st) {
   if (am == kMajorK && bm == kMajorK) return launch<BN, kMajorK, kMajorK, MT>(maps, d, grid, st);
@@ -714,11 +846,12 @@ TilePlan plan_tiles(const GemmCall& g, int BN) {
       for (int64_t j = 0; j < ntile; ++j) a += (g.c_upper && i * rows >= j * BN + BN) ? 0 : 1;
     return a * g.batch;
   };
-  const int kmax = g.Ch ? 1 : (g.k_split == 0 ? int(std::max<int64_t>(1, std::min<int64_t>(64, kb / 2))) : g.k_split);
+  const int kmax = (g.Ch || g.res) ? 1 : (g.k_split == 0 ? int(std::max<int64_t>(1, std::min<int64_t>(64, kb / 2))) : g.k_split);
   const int kmin = g.k_split == 0 ? 1 : g.k_split;
   TilePlan best{only, 1, kmin};
   double best_t = 1e300;
-  for (int MT = (only == 0 ? 2 : 1); MT >= 1; --MT) {
+  // the fused residual epilogue runs with one accumulator, two CTAs per SM
+  for (int MT = (only == 0 && !g.res ? 2 : 1); MT >= 1; --MT) {
     if (MT == 2 && g.M <= BM) continue;
     const bool pair = only == 3;
     const int slots = pair ? kSMs / 2 : kSMs;  // tiles in flight at once
@@ -742,11 +875,19 @@ TilePlan plan_tiles(const GemmCall& g, int BN) {
 
 jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return JOLT_OK;
-  if (g.n_terms < 1 || g.n_terms > kMaxTerms || (!g.C && !g.Ch) || (g.C && g.Ch) || g.batch < 1 || g.k_split < 0 ||
+  if (g.n_terms < 1 || g.n_terms > kMaxTerms || (!g.C && !g.Ch && !g.res) || (g.C && g.Ch) || g.batch < 1 || g.k_split < 0 ||
       g.c_batch_div < 1)
     return JOLT_ERR_INVALID_ARG;
   if (g.Ch && (g.accumulate || g.k_split > 1 || g.c_batch_div > 1)) return JOLT_ERR_INVALID_ARG;
   if (g.Cl && !g.Ch) return JOLT_ERR_INVALID_ARG;
+  if (g.res) {
+    const ResidualEpi& e = *g.res;
+    if (g.C || g.Ch || g.accumulate || g.k_split > 1 || g.c_batch_div > 1 || g.N != 128 || !e.X || !e.codes ||
+        !e.sz || e.T != g.M || !(e.b == 2 || e.b == 4 || e.b == 8) ||
+        reinterpret_cast<uintptr_t>(e.codes) % 16 || reinterpret_cast<uintptr_t>(e.X) % 16 ||
+        reinterpret_cast<uintptr_t>(e.sz) % 4 || g.A[0].major != kMajorK || g.B[0].major != kMajorMN)
+      return JOLT_ERR_INVALID_ARG;
+  }
   if ((g.k_split != 1 || g.c_batch_div > 1) && !g.accumulate) return JOLT_ERR_INVALID_ARG;
   const int am = g.A[0].major, bm = g.B[0].major;
   for (int t = 0; t < g.n_terms; ++t)
@@ -778,6 +919,7 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   d.err = g.err;
   d.Ch = g.Ch;
   d.Cl = g.Cl;
+  if (g.res) d.res = *g.res;
   if (g.Ch)
     d.c_vec = (reinterpret_cast<uintptr_t>(g.Ch) % 16 == 0 && reinterpret_cast<uintptr_t>(g.Cl) % 16 == 0 &&
                g.ldc % 8 == 0 && g.c_batch_stride % 8 == 0) ? 1 : 0;
@@ -804,7 +946,8 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   }
   // algorithmic flops: a triangular B or a wanted upper triangle of C halves the product
   const double tri = (g.b_upper || g.c_upper) ? 0.5 : 1.0;
-  StatScope sc(JOLT_K_GEMM, st, tri * 2.0 * g.M * double(g.N) * g.K * g.batch * g.n_terms, 0.0);
+  StatScope sc(g.res ? -1 : JOLT_K_GEMM, st, tri * 2.0 * g.M * double(g.N) * g.K * g.batch * g.n_terms, 0.0);
+  if (g.res) return launch_res<1>(maps, d, grid, st);
   if (tp.kind == 3) return launch_pers<1>(am, bm, maps, d, grid, st);
   if (tp.kind == 2) return launch_pers<0>(am, bm, maps, d, grid, st);
   if (MT == 2) return BN == 256 ? launch_bn<256, 2>(am, bm, maps, d, grid, st) : launch_bn<128, 2>(am, bm, maps, d, grid, st);
@@ -864,5 +1007,28 @@ extern "C" jolt_status jolt_gemm_bf16_hilo(const void* A, int32_t a_mn_major, co
   g.Cl = static_cast<__nv_bfloat16*>(Cl);
   g.ldc = ldc; g.c_batch_stride = stride_c; g.batch = batch;
   g.k_split = 1;
+  return gemm_tc(g, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" jolt_status jolt_gemm_bf16_residual(const void* A, const void* B, int32_t M, int32_t K, int64_t lda,
+                                               int64_t ldb, int32_t batch, int64_t stride_a, int64_t stride_b,
+                                               const void* X, int32_t x_f32, uint64_t seed, int32_t b,
+                                               uint8_t* codes, void* sz, int32_t* err, void* stream) {
+  if (M < 0 || K < 1 || batch < 1) return JOLT_ERR_INVALID_ARG;
+  if (M == 0) return JOLT_OK;
+  if (!A || !B || !X || !codes || !sz || lda < K || ldb < 128) return JOLT_ERR_INVALID_ARG;
+  GemmCall g;
+  g.M = M; g.N = 128; g.K = K;
+  Operand& a = g.A[0];
+  a.ptr = A; a.major = kMajorK; a.inner = K; a.outer = M; a.outer_stride = lda;
+  a.batch = batch; a.batch_stride = stride_a;
+  Operand& bo = g.B[0];
+  bo.ptr = B; bo.major = kMajorMN; bo.inner = 128; bo.outer = K; bo.outer_stride = ldb;
+  bo.batch = batch; bo.batch_stride = stride_b;
+  ResidualEpi e;
+  e.X = X; e.x_f32 = x_f32 ? 1 : 0; e.T = M; e.seed = seed; e.b = b; e.codes = codes; e.sz = sz;
+  g.res = &e;
+  g.batch = batch;
+  g.err = err;
   return gemm_tc(g, static_cast<cudaStream_t>(stream));
 }

@@ -29,6 +29,20 @@ struct Operand {
 
 constexpr int kMaxTerms = 6;
 
+// Fused residual coding: with N = 128 output columns (the features of one token row), each
+// output row x~ = C[z][t][:] is not stored; the epilogue forms x = X[z*T + t][:] - x~, rotates it by
+// (1/sqrt(128)) H diag(s) (s the seeded signs), quantises it per row to b bits (fp16 scale and
+// zero) and packs the codes, exactly as the stand-alone residual coder does.
+struct ResidualEpi {
+  const void* X = nullptr;   // [batch][T][128] input rows (bf16, or fp32 when x_f32)
+  int x_f32 = 0;
+  int64_t T = 0;             // rows per batch entry (= M)
+  uint64_t seed = 0;         // rotation sign seed
+  int b = 0;                 // 2, 4 or 8
+  uint8_t* codes = nullptr;  // [batch*T][128*b/8], 16-byte aligned
+  void* sz = nullptr;        // __half2 [batch*T]: (scale, zero)
+};
+
 struct GemmCall {
   int M = 0, N = 0, K = 0;
   int n_terms = 1;
@@ -48,6 +62,7 @@ struct GemmCall {
   bool accumulate = false;     // atomically add into C instead of storing
   bool c_upper = false;        // only C[m][n] with m <= n is wanted: skip tiles entirely below the diagonal
   bool b_upper = false;        // B[k][n] = 0 for k > n (upper triangular): K stops at the tile's last column
+  const ResidualEpi* res = nullptr;  // fused residual coding instead of any C output (see above)
   int32_t* err = nullptr;
 };
 

@@ -42,7 +42,7 @@ bool stats_on() {
 StatScope::StatScope(int family, cudaStream_t st, double flops, double bytes)
     : fam_(family), st_(st), flops_(flops), bytes_(bytes) {
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_on) return;
+  if (!g_on || family < 0) return;  // family < 0: not recorded (the caller's own scope covers it)
   e0_ = take_event();
   e1_ = take_event();
   if (e0_) cudaEventRecord(e0_, st_);

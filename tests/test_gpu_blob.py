@@ -1,4 +1,5 @@
-"""A compressed cache written to a host blob and read back decodes to the same outputs."""
+"""A compressed cache written to a host blob and read back is byte-identical and decodes to the
+same outputs (up to the summation order of the decode's atomic partial sums)."""
 import numpy as np
 import pytest
 import torch
@@ -31,4 +32,7 @@ def test_blob_round_trip_decodes_identically(cuda_ok):
     api.decode_attn(shape, choices, cache, q, o1, dws, inv_freq=inv)
     api.decode_attn(s2, ch2, cache2, q, o2, dws, inv_freq=inv)
     torch.cuda.synchronize()
-    assert torch.equal(o1, o2)
+    # the bytes are identical (above); decode sums split-K partials with float atomics, whose
+    # order (hence last-bit rounding) may differ from one call to the next
+    scale = o1.float().abs().max().item()
+    assert (o1.float() - o2.float()).abs().max().item() <= 1e-5 * scale

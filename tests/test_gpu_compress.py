@@ -174,3 +174,4 @@ def test_randomized_path_fp32_factors_orthonormal(cuda_ok):
     # fp32 bases and the 1% bar at a fixed choice
     w = get_workload("llama8b_32k", n_layers=4, T=4096)
     run(w, uniform(w, (256, 96, 2)), factor_dtype="f32", tail_tol=2e-3)
+

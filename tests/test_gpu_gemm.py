@@ -72,3 +72,25 @@ def test_gemm_hilo_outputs_split_the_fp32_result(cuda_ok, a_mn, b_mn, M, N, K):
     assert torch.equal(hi.view(torch.int16), h_ref.view(torch.int16))
     assert torch.equal(hi_only.view(torch.int16), h_ref.view(torch.int16))
     assert torch.equal(lo.view(torch.int16), l_ref.view(torch.int16))
+
+
+@pytest.mark.parametrize("b", [2, 4, 8])
+@pytest.mark.parametrize("M,K,bt,xf32", [(1000, 448, 2, False), (333, 1344, 1, True), (4096, 96, 3, False)])
+def test_gemm_residual_epilogue_matches_standalone_coder(cuda_ok, M, K, bt, xf32, b):
+    """The fused epilogue codes X - A @ B exactly as the stand-alone path does: the fp32 product
+    stored by the same kernel, subtracted, rotated (jolt_rotate_rows) and quantised
+    (jolt_quantize_pack)."""
+    g = torch.Generator(device="cuda").manual_seed(M + K + 11 * b + bt)
+    A = torch.randn(bt, M, K, generator=g, device="cuda").to(torch.bfloat16)
+    B = (0.05 * torch.randn(bt, K, 128, generator=g, device="cuda")).to(torch.bfloat16)
+    X = torch.randn(bt, M, 128, generator=g, device="cuda")
+    X = X if xf32 else X.to(torch.bfloat16)
+    seed = 0x1234ABCD + b
+    codes, sz, err = api.gemm_bf16_residual(A, B, X, seed, b)
+    C = api.gemm_bf16(A, B, False, True)
+    x = (X.float() - C).reshape(bt * M, 128)
+    rc, rsz, rerr = api.quantize_pack(api.rotate_rows(x, seed), b)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and int(rerr.item()) == 0
+    assert torch.equal(codes, rc)
+    assert torch.equal(sz.view(torch.int16), rsz.view(torch.int16))
