@@ -56,6 +56,7 @@ struct KeysMaps {
 
 struct KeysArgs {
   int T, nkb, n_kv, gq, n_q, nl;
+  int b_one;               // maps.b[0] loads both chunks of every term at once (5-D map)
   uint64_t rot_seed;
   float attn_scale;
   int pos0;
@@ -221,11 +222,15 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
           const uint32_t sa = sbase + s * C::kStageBytes;
           sm100::mbar_expect_tx(full_bar(s), C::kStageBytes);
           sm100::tma_load_3d(sa, &maps.a, full_bar(s), kb * kBK, t0, 0);
+          if (p.b_one) {
+            sm100::tma_load_5d(sa + kABytes, &maps.b[0], full_bar(s), 0, kb * kBK, 0, pr, 0);
+          } else {
 #pragma unroll
-          for (int t = 0; t < NT; ++t)
+            for (int t = 0; t < NT; ++t)
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-              sm100::tma_load_3d(sa + kABytes + t * kBBytes + c * 8192, &maps.b[t], full_bar(s), c * 64, kb * kBK, pr);
+              for (int c = 0; c < 2; ++c)
+                sm100::tma_load_3d(sa + kABytes + t * kBBytes + c * 8192, &maps.b[t], full_bar(s), c * 64, kb * kBK, pr);
+          }
           ++it;
         }
       }
@@ -489,7 +494,7 @@ __global__ void __launch_bounds__(128) k_values_res(const ValArgs a) {
   constexpr int RB = kD * BITS / 8;        // bytes of one code row
   constexpr uint32_t mask = (1u << BITS) - 1u;
   __shared__ __align__(16) uint8_t cs[128][RB];
-  __shared__ __align__(16) float pr[128][kMaxG];
+  __shared__ __align__(16) __nv_bfloat16 pr[128][kMaxG];  // P~ as stored (bf16): 8 heads per 16-byte load
   __shared__ float2 szs[128];
   __shared__ __align__(16) float red[2][kMaxG][kD];
   const int h = blockIdx.y, li = blockIdx.z, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -513,7 +518,7 @@ __global__ void __launch_bounds__(128) k_values_res(const ValArgs a) {
       szs[threadIdx.x] = make_float2(__low2float(szv), __high2float(szv));
 #pragma unroll
       for (int g = 0; g < kMaxG; ++g)
-        pr[threadIdx.x][g] = g < a.gq ? __bfloat162float(a.ptil[(qrow0 + g) * a.ldp + tb + threadIdx.x]) : 0.f;
+        pr[threadIdx.x][g] = g < a.gq ? a.ptil[(qrow0 + g) * a.ldp + tb + threadIdx.x] : __float2bfloat16_rn(0.f);
     }
     __syncthreads();
     for (int tt = w; tt < nt; tt += 4) {
@@ -525,16 +530,21 @@ __global__ void __launch_bounds__(128) k_values_res(const ValArgs a) {
       float dv[4];
 #pragma unroll
       for (int f = 0; f < 4; ++f) dv[f] = dequant((word >> (f * BITS)) & mask, z.x, z.y);
-      const float4* p4 = reinterpret_cast<const float4*>(pr[tt]);
+      const uint4* p8 = reinterpret_cast<const uint4*>(pr[tt]);
 #pragma unroll
-      for (int g4 = 0; g4 < kMaxG / 4; ++g4) {
-        if (4 * g4 < a.gq) {
-          const float4 pw = p4[g4];
-          const float pv[4] = {pw.x, pw.y, pw.z, pw.w};
+      for (int g8 = 0; g8 < kMaxG / 8; ++g8) {
+        if (8 * g8 < a.gq) {
+          const uint4 pw = p8[g8];
+          const uint32_t pb[4] = {pw.x, pw.y, pw.z, pw.w};
 #pragma unroll
-          for (int gg = 0; gg < 4; ++gg)
+          for (int e = 0; e < 4; ++e) {
+            const float2 pv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pb[e]));
 #pragma unroll
-            for (int f = 0; f < 4; ++f) acc[4 * g4 + gg][f] = fmaf(pv[gg], dv[f], acc[4 * g4 + gg][f]);
+            for (int f = 0; f < 4; ++f) {
+              acc[8 * g8 + 2 * e][f] = fmaf(pv.x, dv[f], acc[8 * g8 + 2 * e][f]);
+              acc[8 * g8 + 2 * e + 1][f] = fmaf(pv.y, dv[f], acc[8 * g8 + 2 * e + 1][f]);
+            }
+          }
         }
       }
     }
@@ -787,9 +797,14 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
             k_split_hilo<<<grid1(nb), 256, 0, st>>>(bh, nb, hl, hl + nb);
             JOLT_CUDA_TRY(cudaGetLastError());
           }
-          if (!make_tensor_map(&maps.a, op(ck.Ut, kMajorK, ck.r_T, T, ck.r_T), kBM) ||
-              !make_tensor_map(&maps.b[0], op(hl, kMajorMN, kD, ck.r_T, kD, nl * n_kv, int64_t(qc) * kD), kD) ||
-              !make_tensor_map(&maps.b[1], op(hl + nb, kMajorMN, kD, ck.r_T, kD, nl * n_kv, int64_t(qc) * kD), kD))
+          if (!make_tensor_map(&maps.a, op(ck.Ut, kMajorK, ck.r_T, T, ck.r_T), kBM)) return JOLT_ERR_INVALID_ARG;
+          // both terms' two 64-wide chunks in one copy per k-block when the driver takes the
+          // 5-D layout (hi and lo parts are nb elements apart); else four copies
+          ka.b_one = make_tensor_map_mn_chunks(&maps.b[0], hl, ck.r_T, kD, 2, int64_t(nl) * n_kv, int64_t(qc) * kD, 2, nb)
+                         ? 1 : 0;
+          if (!ka.b_one &&
+              (!make_tensor_map(&maps.b[0], op(hl, kMajorMN, kD, ck.r_T, kD, nl * n_kv, int64_t(qc) * kD), kD) ||
+               !make_tensor_map(&maps.b[1], op(hl + nb, kMajorMN, kD, ck.r_T, kD, nl * n_kv, int64_t(qc) * kD), kD)))
             return JOLT_ERR_INVALID_ARG;
           ka.nkb = (ck.r_T + kBK - 1) / kBK;
         }

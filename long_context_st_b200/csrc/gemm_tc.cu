@@ -812,6 +812,25 @@ bool make_tensor_map(CUtensorMap* m, const Operand& o, int rows) {
   return r == CUDA_SUCCESS;
 }
 
+bool make_tensor_map_mn_chunks(CUtensorMap* m, const void* ptr, int64_t K, int64_t ld, int chunks, int64_t batch,
+                               int64_t batch_stride, int terms, int64_t term_stride) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || !ptr || reinterpret_cast<uintptr_t>(ptr) % 16) return false;
+  cuuint64_t dims[5] = {64, cuuint64_t(K), cuuint64_t(chunks), cuuint64_t(std::max<int64_t>(1, batch)),
+                        cuuint64_t(terms)};
+  cuuint64_t strides[4] = {cuuint64_t(ld) * 2, 128, cuuint64_t(batch_stride) * 2, cuuint64_t(term_stride) * 2};
+  cuuint32_t box[5] = {64, 64, cuuint32_t(chunks), 1, cuuint32_t(terms)};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  for (int i = 0; i < 4; ++i)
+    if (strides[i] % 16 || strides[i] == 0) return false;
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && std::getenv("JOLT_DEBUG"))
+    std::fprintf(stderr, "jolt: chunked MN tensor map rejected (CUresult %d)\n", int(r));
+  return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 // Tile plan: the one-tile-per-CTA kernel with MT 128-row accumulators and the split-K factor that

@@ -70,6 +70,13 @@ struct GemmCall {
 // (K-major) or 64 x 64 (MN-major). False if the driver rejects it or the pointer is misaligned.
 bool make_tensor_map(CUtensorMap* m, const Operand& o, int rows);
 
+// TMA tensor map that loads `chunks` 64-wide MN chunks x 64 k rows of `terms` equally spaced
+// MN-major bf16 operands in one copy: dims (64, K, chunks, batch, terms), element strides
+// (ld, 64, batch_stride, term_stride), box (64, 64, chunks, 1, terms), 128-byte swizzle; the
+// shared-memory tile is [term][chunk][64 k rows][64]. False if the driver rejects the layout.
+bool make_tensor_map_mn_chunks(CUtensorMap* m, const void* ptr, int64_t K, int64_t ld, int chunks, int64_t batch,
+                               int64_t batch_stride, int terms, int64_t term_stride);
+
 // Launch; validates shapes and alignment (JOLT_ERR_INVALID_ARG) before any launch.
 jolt_status gemm_tc(const GemmCall& g, cudaStream_t st);
 
