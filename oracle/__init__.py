@@ -21,3 +21,4 @@ from .hosvd import token_unfolding, st_hosvd, spectra_tails, reconstruct  # noqa
 from .quant import quantize_rows, dequantize_rows, pack_codes, unpack_codes, phi_table  # noqa: F401
 from .alloc import build_options, allocate, brute_force_allocate, allocate_kv_split, allocate_uniform  # noqa: F401
 from .codec import compress_cell, decompress_cell, decompress_slice, decode_attention, rope  # noqa: F401
+from .grouping import layer_token_basis, subspace_alignment, layer_alignment, group_layers, uniform_group  # noqa: F401
