@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--seqlen", type=int, default=None, help="override T (small profiling cases)")
     ap.add_argument("--nvtx", action="store_true", help="NVTX range 'jolt_step' around each timed step")
     ap.add_argument("--no-count", action="store_true", help="skip the CUPTI kernel count")
+    ap.add_argument("--no-grouping", action="store_true", help="skip the layer-grouping report")
     ap.add_argument("--cells-per-pass", type=int, default=0,
                     help="cells jolt_analyze batches per pass (0: every cell of a kind in one pass)")
     ap.add_argument("--exact", action="store_true",
@@ -287,6 +288,33 @@ def allocator_ablation(step):
     return out
 
 
+def layer_grouping(step, rank=32, tau=0.5):
+    """The pages' layer-grouping step ([v4] §3) on this step's own K/V, outside the timed step:
+    alignment of consecutive layers' top-`rank` token subspaces (jolt_layer_align, averaged over
+    the sequences), the consecutive groups at tau, the uniform group size a fixed-L_g shape could
+    use, and the device time of one call."""
+    api, w = step.api, step.w
+    if w.n_layers < 2:
+        return None
+    try:
+        ws = torch.zeros(api.layer_align_workspace(step.shape, rank), dtype=torch.uint8, device=step.K.device)
+        api.layer_align(step.shape, step.K, step.V, rank, ws=ws)  # warm-up
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        a = api.layer_align(step.shape, step.K, step.V, rank, ws=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        del ws
+        mean = a.mean(axis=0)
+        groups = api.group_layers(mean, tau)
+        return {"rank": rank, "tau": tau, "ms": e0.elapsed_time(e1), "align_min": float(mean.min()),
+                "align_max": float(mean.max()), "n_groups": len(groups), "groups": groups,
+                "uniform_L_g": api.uniform_group(mean, tau)}
+    except Exception as e:  # reported, not fatal: the step's own numbers stand
+        return {"error": str(e)}
+
+
 def decode_work(w, shape, choices):
     """Algorithmic work of one decode step over every layer: (bytes, tensor flops).
 
@@ -480,6 +508,7 @@ def main():
             "kernel_stats": {k: {kk: (float(vv) if isinstance(vv, float) else int(vv)) for kk, vv in v.items()}
                              for k, v in stats.items()},
             "allocator_ablation": allocator_ablation(step),
+            "layer_grouping": None if args.no_grouping else layer_grouping(step),
             "gpu_launches": n_kernels * args.steps if n_kernels is not None else None,
             "kernels": kernel_names, "clocks": clk.summary(), "choices": sorted(set(map(tuple, step.choices)))}
 

@@ -202,6 +202,35 @@ jolt_status jolt_analyze(const jolt_shape* shape, const void* k, const void* v, 
                          double* tail_T_out, double* tail_d_out, void* ws, size_t ws_bytes,
                          void* stream);
 
+/* Layer alignment for grouping ("A JoLT for the KV cache", §3: JoLT groups consecutive layers
+ * whose token-mode singular vectors align, from the cache being compressed). The pages give no
+ * measure; the one computed here: for every sequence b and layer l, U^X_{b,l} = the top-k token
+ * directions of layer l's own cache X in {K, V} (token unfolding [T][n_kv*d_h]), found by the
+ * compressor's randomized token SVD (sketch width k + 16 capped at min(T, n_kv*d_h), two power
+ * iterations, Rayleigh-Ritz); then
+ *   align[b*(L-1) + l] = ( ||U^K_l^T U^K_{l+1}||_F^2 + ||U^V_l^T U^V_{l+1}||_F^2 ) / (2k),
+ * the mean squared cosine of the principal angles, in [0, 1], for l < L-1.
+ *   shape   the codec's shape (layers_per_group, q_cap, sketch_cols, power_iters are ignored)
+ *   k       multiple of 16, 16 <= k <= min(T, n_kv*d_h)
+ *   K, V    device, [B][L][n_kv][T][d_h] io dtype
+ *   align   host [B][L-1]
+ *   ws      device, >= jolt_layer_align_workspace(shape, k)
+ * Synchronises `stream`. JOLT_ERR_INVALID_ARG for a bad shape or k. */
+size_t jolt_layer_align_workspace(const jolt_shape* shape, int32_t k);
+jolt_status jolt_layer_align(const jolt_shape* shape, int32_t k, const void* K, const void* V, double* align,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Consecutive layer groups from alignments (host): layer l+1 joins the current group when
+ * align[l] >= tau and, if max_group > 0, the group has fewer than max_group layers.
+ *   align        host [n_layers - 1];  group_sizes host [n_layers] (first *n_groups entries set)
+ * JOLT_ERR_INVALID_ARG for n_layers < 1 or NULL outputs. */
+jolt_status jolt_group_layers(const double* align, int32_t n_layers, double tau, int32_t max_group,
+                              int32_t* group_sizes, int32_t* n_groups);
+
+/* Largest group size L_g dividing n_layers whose uniform groups keep every consecutive alignment
+ * inside a group >= tau (1 always qualifies): the grouping a fixed-L_g shape can use (host). */
+jolt_status jolt_uniform_group(const double* align, int32_t n_layers, double tau, int32_t* L_g);
+
 /* Compress every cell with its choice ("A JoLT for the KV cache", §3): U_T = the first r_T token
  * directions found by jolt_analyze, U_d = top-r_d eigenvectors of the feature Gram of U_T^T X,
  * G = U_T^T X U_d, residual R = X - U_T G U_d^T against the stored (rounded) factors, rotated by

@@ -179,6 +179,44 @@ def analyze(s: Shape, k, v, ws, stream=None):
     return norm2, tT, td
 
 
+def layer_align_workspace(s: Shape, rank=32):
+    return lib().jolt_layer_align_workspace(C.byref(s), rank)
+
+
+def layer_align(s: Shape, k, v, rank=32, ws=None, stream=None):
+    """Alignment of consecutive layers' top-`rank` token subspaces (mean squared cosine of the
+    principal angles, K and V averaged), per sequence: float64 [B, L-1]."""
+    nb = lib().jolt_layer_align_workspace(C.byref(s), rank)
+    if nb == 0:
+        raise JoltError(-1, "jolt_layer_align_workspace")
+    if ws is None or ws.numel() < nb:
+        ws = torch.zeros(nb, dtype=torch.uint8, device=k.device)
+    out = np.zeros((s.batch, max(0, s.n_layers - 1)))
+    check(lib().jolt_layer_align(C.byref(s), rank, _ptr(k), _ptr(v), out.ctypes.data_as(C.POINTER(C.c_double)),
+                                 _ptr(ws), ws.numel(), _stream(stream)), "jolt_layer_align")
+    return out
+
+
+def group_layers(align, tau, max_group=0):
+    """Consecutive layer groups (sizes) from one sequence's alignments [L-1]."""
+    a = np.ascontiguousarray(np.asarray(align, dtype=np.float64))
+    L = a.size + 1
+    sizes = np.zeros(L, dtype=np.int32)
+    ng = C.c_int32(0)
+    check(lib().jolt_group_layers(a.ctypes.data_as(C.c_void_p), L, float(tau), int(max_group),
+                                  sizes.ctypes.data_as(C.c_void_p), C.byref(ng)), "jolt_group_layers")
+    return [int(x) for x in sizes[:ng.value]]
+
+
+def uniform_group(align, tau):
+    """Largest uniform group size dividing L that keeps every in-group alignment >= tau."""
+    a = np.ascontiguousarray(np.asarray(align, dtype=np.float64))
+    out = C.c_int32(0)
+    check(lib().jolt_uniform_group(a.ctypes.data_as(C.c_void_p), a.size + 1, float(tau), C.byref(out)),
+          "jolt_uniform_group")
+    return out.value
+
+
 def compress(s: Shape, k, v, choices, cache, ws, stream=None):
     check(lib().jolt_compress(C.byref(s), _ptr(k), _ptr(v), choices_array(choices), _ptr(cache),
                               cache.numel(), _ptr(ws), ws.numel(), _stream(stream)), "jolt_compress")
@@ -323,7 +361,7 @@ def stats_read(reset=True):
                                      bytes=arr[i].bytes) for i in range(len(KERNEL_FAMILIES))}
 
 
-__all__ = ["allocate_variant", "JOLT_ALLOC_JOINT", "JOLT_ALLOC_KV_SPLIT", "JOLT_ALLOC_UNIFORM", "serialize_cache", "deserialize_cache", "cache_blob_info", "cache_blob_bytes", "decode_attn_noalloc", "stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
+__all__ = ["layer_align_workspace", "layer_align", "group_layers", "uniform_group", "gemm_bf16_hilo", "gemm_bf16_residual", "allocate_variant", "JOLT_ALLOC_JOINT", "JOLT_ALLOC_KV_SPLIT", "JOLT_ALLOC_UNIFORM", "serialize_cache", "deserialize_cache", "cache_blob_info", "cache_blob_bytes", "decode_attn_noalloc", "stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
            "allocate", "workspace_bytes", "new_workspace", "analyze", "compress", "decode_attn",
            "check_ws", "rotate_rows", "quantize_pack", "unpack_dequant", "JoltError",
            "JOLT_OP_COMPRESS", "JOLT_OP_DECODE"]

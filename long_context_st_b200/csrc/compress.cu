@@ -836,6 +836,117 @@ extern "C" jolt_status jolt_analyze(const jolt_shape* shape, const void* k, cons
   return JOLT_OK;
 }
 
+// ---- layer alignment (grouping) ----------------------------------------------------------------
+
+namespace jolt {
+namespace {
+
+// The single-layer shape whose cells are the layers of `s`: its analyze pass finds each layer's
+// top-k token directions (sketch width k + 16 capped at min(T, n_kv*d_h), two power iterations).
+bool layer_shape(const jolt_shape& s, int k, jolt_shape* o) {
+  if (!shape_ok(&s)) return false;
+  *o = s;
+  o->layers_per_group = 1;
+  const int64_t lim = std::min<int64_t>(int64_t(s.n_kv) * s.d_h, s.T);
+  if (k < 16 || k % kRankStep || k > lim) return false;
+  int64_t l = std::min<int64_t>(lim, int64_t(k) + 16);
+  l -= l % kRankStep;
+  o->q_cap = k;
+  o->sketch_cols = int(l);
+  o->power_iters = 2;
+  o->cells_per_pass = std::max(1, std::min(s.batch * s.n_layers, 32));
+  return shape_ok(o);
+}
+
+// M[pair] += sum_t U1[t][i] U2[t][j] over this block's rows, pair = (b * (L-1) + l) * 2 + kv with
+// U1, U2 the token bases (fp32 [T][k]) of layers l and l + 1 of sequence b, kind kv.
+constexpr int kAlignMaxK = 128;
+__global__ void __launch_bounds__(256) k_align(const float* __restrict__ Ut, int64_t cell_elems, int T, int k,
+                                               int L, int rows_per_block, double* __restrict__ M) {
+  constexpr int kMaxE = kAlignMaxK * kAlignMaxK / 256;
+  __shared__ float s1[32][kAlignMaxK + 1], s2[32][kAlignMaxK + 1];
+  const int pair = blockIdx.y;
+  const int kv = pair & 1, bl = pair >> 1;
+  const int b = bl / (L - 1), l = bl % (L - 1);
+  const float* U1 = Ut + int64_t((b * L + l) * 2 + kv) * cell_elems;
+  const float* U2 = Ut + int64_t((b * L + l + 1) * 2 + kv) * cell_elems;
+  const int t0 = blockIdx.x * rows_per_block, t1 = min(T, t0 + rows_per_block);
+  float acc[kMaxE];
+#pragma unroll
+  for (int j = 0; j < kMaxE; ++j) acc[j] = 0.f;
+  for (int r0 = t0; r0 < t1; r0 += 32) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < 32 * k; e += 256) {
+      const int rr = e / k, c = e % k, t = r0 + rr;
+      s1[rr][c] = t < t1 ? U1[int64_t(t) * k + c] : 0.f;
+      s2[rr][c] = t < t1 ? U2[int64_t(t) * k + c] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kMaxE; ++j) {
+      const int e = threadIdx.x + 256 * j;
+      if (e < k * k) {
+        const int i = e / k, c = e % k;
+        float a = acc[j];
+#pragma unroll 8
+        for (int rr = 0; rr < 32; ++rr) a = fmaf(s1[rr][i], s2[rr][c], a);
+        acc[j] = a;
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kMaxE; ++j) {
+    const int e = threadIdx.x + 256 * j;
+    if (e < k * k) atomicAdd(&M[int64_t(pair) * k * k + e], double(acc[j]));
+  }
+}
+
+}  // namespace
+}  // namespace jolt
+
+extern "C" size_t jolt_layer_align_workspace(const jolt_shape* shape, int32_t k) {
+  jolt_shape s1;
+  if (!shape || !layer_shape(*shape, k, &s1) || k > kAlignMaxK) return 0;
+  const size_t npairs = size_t(shape->batch) * std::max(0, shape->n_layers - 1) * 2;
+  return align_up(make_plan(s1).total, 256) + npairs * size_t(k) * k * 8;
+}
+
+extern "C" jolt_status jolt_layer_align(const jolt_shape* shape, int32_t k, const void* K, const void* V,
+                                        double* align, void* ws, size_t ws_bytes, void* stream) {
+  jolt_shape s1;
+  if (!shape || !layer_shape(*shape, k, &s1) || k > kAlignMaxK || !K || !V || !align || !ws)
+    return JOLT_ERR_INVALID_ARG;
+  const jolt_shape& s = *shape;
+  if (s.n_layers < 2) return JOLT_OK;
+  if (ws_bytes < jolt_layer_align_workspace(shape, k)) return JOLT_ERR_WORKSPACE;
+  const Plan p = make_plan(s1);
+  const int ncell = n_cells(s1);
+  std::vector<double> n2(ncell), tT(size_t(ncell) * n_rt(s1)), td(size_t(ncell) * n_rd(s1));
+  jolt_status r = jolt_analyze(&s1, K, V, n2.data(), tT.data(), td.data(), ws, p.total, stream);
+  if (r) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int npairs = s.batch * (s.n_layers - 1) * 2;
+  double* M = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + align_up(p.total, 256));
+  JOLT_CUDA_TRY(cudaMemsetAsync(M, 0, size_t(npairs) * k * k * 8, st));
+  const float* Ut = reinterpret_cast<const float*>(static_cast<uint8_t*>(ws) + p.off_ut);
+  const int rows_per_block = 2048;
+  const dim3 grid(unsigned((s.T + rows_per_block - 1) / rows_per_block), unsigned(npairs));
+  k_align<<<grid, 256, 0, st>>>(Ut, int64_t(s.T) * k, s.T, k, s.n_layers, rows_per_block, M);
+  JOLT_CUDA_TRY(cudaGetLastError());
+  std::vector<double> h(size_t(npairs) * k * k);
+  JOLT_CUDA_TRY(cudaMemcpyAsync(h.data(), M, h.size() * 8, cudaMemcpyDeviceToHost, st));
+  JOLT_CUDA_TRY(cudaStreamSynchronize(st));
+  for (int bl = 0; bl < s.batch * (s.n_layers - 1); ++bl) {
+    double f[2] = {0.0, 0.0};
+    for (int kv = 0; kv < 2; ++kv) {
+      const double* m = h.data() + size_t(bl * 2 + kv) * k * k;
+      for (int e = 0; e < k * k; ++e) f[kv] += m[e] * m[e];
+    }
+    align[bl] = (f[0] + f[1]) / (2.0 * k);
+  }
+  return JOLT_OK;
+}
+
 extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, const void* v,
                                      const jolt_cell_choice* choices, void* cache, uint64_t cache_bytes, void* ws,
                                      size_t ws_bytes, void* stream) {

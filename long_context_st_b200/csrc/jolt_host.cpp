@@ -393,3 +393,33 @@ size_t jolt_workspace_bytes(const jolt_shape* s, int32_t op) {
 }
 
 }  // extern "C"
+
+extern "C" jolt_status jolt_group_layers(const double* align, int32_t n_layers, double tau, int32_t max_group,
+                                         int32_t* group_sizes, int32_t* n_groups) {
+  if (n_layers < 1 || !group_sizes || !n_groups || (n_layers > 1 && !align)) return JOLT_ERR_INVALID_ARG;
+  int ng = 1;
+  group_sizes[0] = 1;
+  for (int l = 0; l + 1 < n_layers; ++l) {
+    if (align[l] >= tau && (max_group <= 0 || group_sizes[ng - 1] < max_group)) {
+      ++group_sizes[ng - 1];
+    } else {
+      group_sizes[ng++] = 1;
+    }
+  }
+  *n_groups = ng;
+  return JOLT_OK;
+}
+
+extern "C" jolt_status jolt_uniform_group(const double* align, int32_t n_layers, double tau, int32_t* L_g) {
+  if (n_layers < 1 || !L_g || (n_layers > 1 && !align)) return JOLT_ERR_INVALID_ARG;
+  int best = 1;
+  for (int g = 1; g <= n_layers; ++g) {
+    if (n_layers % g) continue;
+    bool ok = true;
+    for (int l = 0; l + 1 < n_layers && ok; ++l)
+      if ((l + 1) % g != 0 && !(align[l] >= tau)) ok = false;
+    if (ok) best = g;
+  }
+  *L_g = best;
+  return JOLT_OK;
+}

@@ -179,3 +179,19 @@ def test_cache_blob_header_checks():
     bad[8] = 2                                                   # unknown version
     with pytest.raises(api.JoltError):
         api.cache_blob_info(bad)
+
+
+def test_group_layers_matches_oracle():
+    """Host grouping (jolt_group_layers / jolt_uniform_group) equals the oracle's on random and
+    boundary alignments."""
+    import numpy as np
+    from oracle.grouping import group_layers as o_group, uniform_group as o_uniform
+    from long_context_st_b200 import api
+    rng = np.random.default_rng(7)
+    cases = [rng.uniform(0, 1, size=n) for n in (0, 1, 5, 11, 79)]
+    cases.append(np.array([0.5, 0.49999999, 0.5, 1.0, 0.0]))
+    for a in cases:
+        for tau in (0.3, 0.5, 0.8):
+            for mg in (0, 2, 3):
+                assert api.group_layers(a, tau, mg) == o_group(list(a), tau, mg)
+            assert api.uniform_group(a, tau) == o_uniform(list(a), a.size + 1, tau)
