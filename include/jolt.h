@@ -323,6 +323,14 @@ jolt_status jolt_gemm_bf16_residual(const void* A, const void* B, int32_t M, int
                                     const void* X, int32_t x_f32, uint64_t seed, int32_t b,
                                     uint8_t* codes, void* sz, int32_t* err, void* stream);
 
+/* Failure-detection self-test: launches a kernel whose wait nothing will end — which = 0: an
+ * mbarrier no thread arrives on (the bounded wait of every TMA / tensor-core pipeline); which = 1:
+ * a two-CTA cooperative grid whose second CTA never reaches the grid barrier (the barrier of the
+ * Cholesky and Jacobi kernels). The wait gives up after limit_ns (1 ns .. 2 s) and the kernel
+ * returns with JOLT_ERR_TIMEOUT in ws's error word, which jolt_check then reports; the context
+ * stays usable. ws device, >= 512 bytes (zeroed here). Does not synchronise. */
+jolt_status jolt_selftest_timeout(int32_t which, uint64_t limit_ns, void* ws, size_t ws_bytes, void* stream);
+
 /* Symmetric eigendecomposition of `batch` fp32 matrices A [batch][n][n] (device) by block Jacobi
  * (the solver the compressor uses for the Rayleigh-Ritz and feature-mode steps): eigenvalues
  * descending into evals [batch][n], eigenvectors as the columns of evecs [batch][n][n] (device).

@@ -96,6 +96,7 @@ SIGNATURES = [
     ("jolt_layer_align", C.c_int, [C.POINTER(Shape), C.c_int32, _P, _P, _P, _P, C.c_size_t, _P]),
     ("jolt_group_layers", C.c_int, [_P, C.c_int32, C.c_double, C.c_int32, _P, _P]),
     ("jolt_uniform_group", C.c_int, [_P, C.c_int32, C.c_double, _P]),
+    ("jolt_selftest_timeout", C.c_int, [C.c_int32, C.c_uint64, _P, C.c_size_t, _P]),
     ("jolt_sym_eig_workspace", C.c_size_t, [C.c_int32, C.c_int32]),
     ("jolt_stats_enable", None, [C.c_int32]),
     ("jolt_stats_read", C.c_int, [C.POINTER(KernelStat), C.c_int32]),

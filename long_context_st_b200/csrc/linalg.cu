@@ -16,6 +16,7 @@
 #include <vector>
 
 #include "linalg.cuh"
+#include "sm100.cuh"
 #include "stats.h"
 
 namespace jolt {
@@ -37,7 +38,7 @@ struct GridBar {
   int32_t* err;
 };
 
-__device__ __forceinline__ void grid_barrier(const GridBar& gb) {
+__device__ __forceinline__ void grid_barrier(const GridBar& gb, uint64_t limit_ns = 2000000000ull) {
   __syncthreads();
   if (threadIdx.x == 0) {
     volatile unsigned int* vgen = gb.gen;
@@ -55,7 +56,7 @@ __device__ __forceinline__ void grid_barrier(const GridBar& gb) {
         if (*reinterpret_cast<volatile int32_t*>(gb.err) != 0) break;
         uint64_t t1;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
-        if (t1 - t0 > 2000000000ull) {
+        if (t1 - t0 > limit_ns) {
           atomicCAS(gb.err, 0, int32_t(JOLT_ERR_TIMEOUT));
           break;
         }
@@ -860,6 +861,31 @@ jolt_status launch_coop(K kernel, const A& args, int smem, cudaStream_t st, int 
   return JOLT_OK;
 }
 
+// ---- failure-detection self-tests: a wait that nothing will end must give up and report ----------
+
+// An mbarrier no thread arrives on: the bounded wait (the one every TMA / MMA pipeline uses)
+// returns false after limit_ns and sets JOLT_ERR_TIMEOUT in the error word.
+__global__ void k_selftest_mbar(int32_t* err, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(sm100::smem_u32(&bar), 1);
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  sm100::mbar_wait(sm100::smem_u32(&bar), 0, err, limit_ns);
+}
+
+// A cooperative grid whose last CTA returns without arriving: the others' grid barrier (the one
+// the Cholesky and Jacobi kernels use) gives up after limit_ns with JOLT_ERR_TIMEOUT.
+struct SelftestGridArgs {
+  GridBar bar;
+  uint64_t limit_ns;
+};
+__global__ void k_selftest_grid(SelftestGridArgs a) {
+  if (blockIdx.x == gridDim.x - 1) return;
+  grid_barrier(a.bar, a.limit_ns);
+}
+
 jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shift_rel,
                          __nv_bfloat16* rinv_hi, __nv_bfloat16* rinv_lo, void* scratch, int32_t* err,
                          cudaStream_t st, float* min_ratio) {
@@ -1002,6 +1028,29 @@ jolt_status split_bf16(const float* x, int64_t ldx, int64_t rows, int64_t cols, 
 }  // namespace jolt
 
 using namespace jolt;
+
+extern "C" jolt_status jolt_selftest_timeout(int32_t which, uint64_t limit_ns, void* ws, size_t ws_bytes,
+                                             void* stream) {
+  if (!ws || ws_bytes < 512 || limit_ns == 0 || limit_ns > 2000000000ull || (which != 0 && which != 1))
+    return JOLT_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* err = static_cast<int32_t*>(ws);
+  JOLT_CUDA_TRY(cudaMemsetAsync(ws, 0, 512, st));
+  if (which == 0) {
+    k_selftest_mbar<<<1, 32, 0, st>>>(err, limit_ns);
+    JOLT_CUDA_TRY(cudaGetLastError());
+    return JOLT_OK;
+  }
+  SelftestGridArgs a;
+  unsigned int* bar = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + 256);
+  a.bar.count = bar;
+  a.bar.gen = bar + 1;
+  a.bar.err = err;
+  a.limit_ns = limit_ns;
+  void* params[] = {&a};
+  JOLT_CUDA_TRY(cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k_selftest_grid), dim3(2), dim3(32), params, 0, st));
+  return JOLT_OK;
+}
 
 extern "C" size_t jolt_sym_eig_workspace(int32_t n, int32_t batch) {
   if (n < 1 || batch < 1) return 0;
