@@ -37,6 +37,7 @@ struct TmaPack {
 struct GemmDev {
   int M, N, K, n_terms, nkb_split, k_split;
   int a_fold[kMaxTerms], b_fold[kMaxTerms];    // fold length (0 = plain)
+  int a_chunk[kMaxTerms], b_chunk[kMaxTerms];  // MN-major operand loaded by one chunked copy
   int a_batch[kMaxTerms], b_batch[kMaxTerms];  // operand batch extents (coordinate = z % extent)
   float* C;
   int64_t ldc, c_bstride;
@@ -169,13 +170,21 @@ struct Cfg {
 struct OpCoord {
   int fold, zb, mn0, kf, kq;
   int c0[4], c2[4];
+  int chunked, cs, cf;  // chunked MN-major map: sub-chunk and fold (or chunk) coordinates of the tile
 };
 
 template <int MAJ>
-__device__ __forceinline__ void op_coord(OpCoord& o, int fold, int bext, int z, int mn0, int rows, int k0) {
+__device__ __forceinline__ void op_coord(OpCoord& o, int fold, int bext, int z, int mn0, int rows, int k0,
+                                         int chunked = 0) {
   o.fold = fold;
   o.zb = bext > 1 ? z % bext : 0;
   o.mn0 = mn0;
+  o.chunked = (MAJ == kMajorMN) ? chunked : 0;
+  if (o.chunked) {
+    // plain: chunk index mn0 / 64; folded: (sub-chunk within the fold, fold index)
+    o.cs = fold ? (mn0 % fold) / 64 : mn0 / 64;
+    o.cf = fold ? mn0 / fold : 0;
+  }
   if (MAJ == kMajorK) {
     o.kf = fold ? k0 % fold : k0;
     o.kq = fold ? k0 / fold : 0;
@@ -204,6 +213,10 @@ __device__ __forceinline__ void op_issue(const CUtensorMap* map, OpCoord& o, uin
       if (PAIRLOAD) sm100::tma_load_3d_pair(dst, map, bar, k0, o.mn0, o.zb);
       else sm100::tma_load_3d(dst, map, bar, k0, o.mn0, o.zb);
     }
+  } else if (!PAIRLOAD && o.chunked) {
+    // every 64-wide chunk of the tile in one copy: [chunk][64 k rows][64]
+    if (o.fold) sm100::tma_load_5d(dst, map, bar, 0, k0, o.cs, o.cf, o.zb);
+    else sm100::tma_load_4d(dst, map, bar, 0, k0, o.cs, o.zb);
   } else {
 #pragma unroll
     for (int i = 0; i < ROWS / 64; ++i) {
@@ -390,20 +403,27 @@ __global__ void __launch_bounds__(128, EPI ? 2 : 1) k_gemm(const __grid_constant
       for (int t = 0; ok && t < p.n_terms; ++t) {
         int k0 = kb_begin * BK;
         OpCoord o[MT];
+        // a chunked MN-major A covers all MT row tiles (consecutive in shared memory) in one copy
+        const bool a_one = AMAJ == kMajorMN && p.a_chunk[t];
         if (is_a) {
 #pragma unroll
-          for (int mt = 0; mt < MT; ++mt) op_coord<AMAJ>(o[mt], p.a_fold[t], p.a_batch[t], z, m0 + mt * BM, BM, k0);
+          for (int mt = 0; mt < MT; ++mt)
+            op_coord<AMAJ>(o[mt], p.a_fold[t], p.a_batch[t], z, m0 + mt * BM, BM, k0, p.a_chunk[t]);
         } else {
-          op_coord<BMAJ>(o[0], p.b_fold[t], p.b_batch[t], z, n0, BN, k0);
+          op_coord<BMAJ>(o[0], p.b_fold[t], p.b_batch[t], z, n0, BN, k0, p.b_chunk[t]);
         }
         for (int kb = 0; kb < nkb; ++kb, k0 += BK) {
           if (!sm100::mbar_wait(empty_bar(stage), phase ^ 1, p.err)) { ok = false; break; }
           const uint32_t sa = smem_base + stage * C::kStageBytes;
           if (is_a) {
             sm100::mbar_expect_tx(full_bar(stage), C::kStageBytes);
+            if (a_one) {
+              op_issue<AMAJ, BM, false>(&maps.a[t], o[0], sa, full_bar(stage), k0);
+            } else {
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-              op_issue<AMAJ, BM, false>(&maps.a[t], o[mt], sa + mt * C::kABytes1, full_bar(stage), k0);
+              for (int mt = 0; mt < MT; ++mt)
+                op_issue<AMAJ, BM, false>(&maps.a[t], o[mt], sa + mt * C::kABytes1, full_bar(stage), k0);
+            }
           } else {
             op_issue<BMAJ, BN, false>(&maps.b[t], o[0], sa + C::kABytes, full_bar(stage), k0);
           }
@@ -812,6 +832,44 @@ bool make_tensor_map(CUtensorMap* m, const Operand& o, int rows) {
   return r == CUDA_SUCCESS;
 }
 
+// MN-major operand tile of `rows` MN elements (a multiple of 64, starting at a multiple of rows) in
+// one copy: plain (64, K, inner/64, batch) with box (64, 64, rows/64, 1); folded (64, K, fold/64,
+// nfold, batch) with box (64, 64, min(rows, fold)/64, max(1, rows/fold), 1). The chunk stride is
+// 128 bytes (the next 64 elements of a row). False where the layout does not fit (the caller then
+// copies chunk by chunk).
+bool make_tensor_map_chunked(CUtensorMap* m, const Operand& o, int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || !o.ptr || o.major != kMajorMN || rows % 64) return false;
+  if (reinterpret_cast<uintptr_t>(o.ptr) % 16) return false;
+  const int64_t bext = std::max<int64_t>(1, o.batch_stride ? o.batch : 1);
+  cuuint64_t dims[5], strides[4];
+  cuuint32_t box[5], estr[5] = {1, 1, 1, 1, 1};
+  int rank;
+  if (o.fold) {
+    if (o.fold % 64) return false;
+    if (o.fold >= rows ? (o.fold % rows) : (rows % o.fold)) return false;
+    rank = 5;
+    dims[0] = 64; dims[1] = o.outer; dims[2] = o.fold / 64; dims[3] = o.nfold; dims[4] = bext;
+    strides[0] = o.outer_stride * 2; strides[1] = 128; strides[2] = o.fold_stride * 2;
+    strides[3] = (o.batch_stride ? o.batch_stride : o.fold_stride * o.nfold) * 2;
+    box[0] = 64; box[1] = 64; box[2] = uint32_t(std::min<int64_t>(rows, o.fold) / 64);
+    box[3] = uint32_t(std::max<int64_t>(1, rows / o.fold)); box[4] = 1;
+  } else {
+    if (o.inner % 64) return false;  // the last chunk must end at the row's end
+    rank = 4;
+    dims[0] = 64; dims[1] = o.outer; dims[2] = o.inner / 64; dims[3] = bext;
+    strides[0] = o.outer_stride * 2; strides[1] = 128;
+    strides[2] = (o.batch_stride ? o.batch_stride : o.outer_stride * o.outer) * 2;
+    box[0] = 64; box[1] = 64; box[2] = uint32_t(rows / 64); box[3] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i)
+    if (strides[i] % 16 || strides[i] == 0) return false;
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(o.ptr), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tensor_map_mn_chunks(CUtensorMap* m, const void* ptr, int64_t K, int64_t ld, int chunks, int64_t batch,
                                int64_t batch_stride, int terms, int64_t term_stride) {
   EncodeTiledFn enc = encode_fn();
@@ -919,9 +977,13 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   TmaPack maps;
   memset(&maps, 0, sizeof(maps));
   GemmDev d{};
+  const char* nochunk = std::getenv("JOLT_GEMM_NO_CHUNKED");  // per-chunk copies only (tests compare both)
+  const bool try_chunk = tp.kind == 0 && !(nochunk && nochunk[0] == '1');
   for (int t = 0; t < g.n_terms; ++t) {
-    if (!make_tensor_map(&maps.a[t], g.A[t], BM)) return JOLT_ERR_INVALID_ARG;
-    if (!make_tensor_map(&maps.b[t], g.B[t], tp.kind == 3 ? BN / 2 : BN)) return JOLT_ERR_INVALID_ARG;
+    d.a_chunk[t] = try_chunk && g.A[t].major == kMajorMN && make_tensor_map_chunked(&maps.a[t], g.A[t], BM * tp.MT);
+    d.b_chunk[t] = try_chunk && g.B[t].major == kMajorMN && make_tensor_map_chunked(&maps.b[t], g.B[t], BN);
+    if (!d.a_chunk[t] && !make_tensor_map(&maps.a[t], g.A[t], BM)) return JOLT_ERR_INVALID_ARG;
+    if (!d.b_chunk[t] && !make_tensor_map(&maps.b[t], g.B[t], tp.kind == 3 ? BN / 2 : BN)) return JOLT_ERR_INVALID_ARG;
     d.a_fold[t] = int(g.A[t].fold);
     d.b_fold[t] = int(g.B[t].fold);
     d.a_batch[t] = g.A[t].batch_stride ? int(g.A[t].batch) : 1;

@@ -20,10 +20,14 @@ def ref_mm(A, B, a_mn, b_mn):
                                    (4096, 256, 128), (64, 384, 200),
                                    # grids large enough for two 128-row tiles per CTA, ragged M/N/K
                                    (16000, 1152, 192), (80000, 200, 72)])
-@pytest.mark.parametrize("plan", ["auto", "1sm", "p1", "p2"])
+@pytest.mark.parametrize("plan", ["auto", "1sm", "p1", "p2", "perchunk"])
 def test_gemm_majors_and_ragged(cuda_ok, monkeypatch, plan, a_mn, b_mn, M, N, K):
-    # restrict the tile plan to the one-tile kernel or the persistent single-CTA / CTA-pair forms
-    monkeypatch.setenv("JOLT_GEMM_PLAN", plan)
+    # restrict the tile plan to the one-tile kernel or the persistent single-CTA / CTA-pair forms;
+    # perchunk: the one-tile kernel copying MN-major operands one 64-wide chunk at a time
+    if plan == "perchunk":
+        monkeypatch.setenv("JOLT_GEMM_NO_CHUNKED", "1")
+    else:
+        monkeypatch.setenv("JOLT_GEMM_PLAN", plan)
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K + a_mn * 2 + b_mn)
     A = torch.randn((K, M) if a_mn else (M, K), generator=g, device="cuda").to(torch.bfloat16)
     B = torch.randn((K, N) if b_mn else (N, K), generator=g, device="cuda").to(torch.bfloat16)
