@@ -227,14 +227,19 @@ class Step:
             out.extend(ch)
         return out
 
-    def run(self, events=None, K=None, V=None):
+    def run(self, events=None, K=None, V=None, host=None):
+        """One step. host = (K_host, V_host): the inputs are copied from (pinned) host memory into
+        K, V inside the analyze call (the value copy overlapping the key cells' analysis)."""
         api = self.api
         K = self.K if K is None else K
         V = self.V if V is None else V
         ev = events or {}
         if "start" in ev:
             ev["start"].record()
-        tables = api.analyze(self.shape, K, V, self.cws)
+        if host is not None:
+            tables = api.analyze_from_host(self.shape, host[0], host[1], K, V, self.cws)
+        else:
+            tables = api.analyze(self.shape, K, V, self.cws)
         self.tables = tables
         if "analyzed" in ev:
             ev["analyzed"].record()
@@ -523,16 +528,13 @@ def main():
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             n_e2e = max(1, min(args.steps, 3))
-            Kd.copy_(Kh, non_blocking=True)
-            Vd.copy_(Vh, non_blocking=True)
-            step.run(K=Kd, V=Vd)
+            step.run(K=Kd, V=Vd, host=(Kh, Vh))
             outh.copy_(step.out, non_blocking=True)
             torch.cuda.synchronize()
             e0.record()
             for _ in range(n_e2e):
-                Kd.copy_(Kh, non_blocking=True)
-                Vd.copy_(Vh, non_blocking=True)
-                step.run(K=Kd, V=Vd)
+                # the H2D copies of K and V run inside the analyze call (jolt_analyze_from_host)
+                step.run(K=Kd, V=Vd, host=(Kh, Vh))
                 outh.copy_(step.out, non_blocking=True)
             e1.record()
             torch.cuda.synchronize()

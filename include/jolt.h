@@ -202,6 +202,17 @@ jolt_status jolt_analyze(const jolt_shape* shape, const void* k, const void* v, 
                          double* tail_T_out, double* tail_d_out, void* ws, size_t ws_bytes,
                          void* stream);
 
+/* jolt_analyze with the inputs streamed from host memory: K crosses the bus into k_dev, then V
+ * into v_dev on a copy stream of the library's own while the key cells are analysed (each kind's
+ * passes wait only for that kind's copy). The copies start after the work already queued on
+ * `stream` (which may still be reading k_dev / v_dev). k_host, v_host: page-locked host
+ * memory [B][L][n_kv][T][d_h] io dtype (pageable memory works but does not overlap); k_dev, v_dev:
+ * device buffers of the same size, left holding the inputs for jolt_compress. Otherwise as
+ * jolt_analyze. Synchronises `stream`. */
+jolt_status jolt_analyze_from_host(const jolt_shape* shape, const void* k_host, const void* v_host,
+                                   void* k_dev, void* v_dev, double* norm2_out, double* tail_T_out,
+                                   double* tail_d_out, void* ws, size_t ws_bytes, void* stream);
+
 /* Layer alignment for grouping ("A JoLT for the KV cache", §3: JoLT groups consecutive layers
  * whose token-mode singular vectors align, from the cache being compressed). The pages give no
  * measure; the one computed here: for every sequence b and layer l, U^X_{b,l} = the top-k token

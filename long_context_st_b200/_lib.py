@@ -92,6 +92,7 @@ SIGNATURES = [
     ("jolt_gemm_bf16_residual", C.c_int, [_P, _P, C.c_int32, C.c_int32, C.c_int64, C.c_int64, C.c_int32,
                                           C.c_int64, C.c_int64, _P, C.c_int32, C.c_uint64, C.c_int32, _P,
                                           _P, _P, _P]),
+    ("jolt_analyze_from_host", C.c_int, [C.POINTER(Shape), _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     ("jolt_layer_align_workspace", C.c_size_t, [C.POINTER(Shape), C.c_int32]),
     ("jolt_layer_align", C.c_int, [C.POINTER(Shape), C.c_int32, _P, _P, _P, _P, C.c_size_t, _P]),
     ("jolt_group_layers", C.c_int, [_P, C.c_int32, C.c_double, C.c_int32, _P, _P]),

@@ -217,6 +217,22 @@ def uniform_group(align, tau):
     return out.value
 
 
+def analyze_from_host(s: Shape, k_host, v_host, k_dev, v_dev, ws, stream=None):
+    """analyze() with K and V copied from (pinned) host tensors into k_dev / v_dev inside the
+    call, the value copy overlapping the key cells' analysis."""
+    nc = n_cells(s)
+    nrt, nrd = s.q_cap // 16 + 1, s.d_h // 16 + 1
+    norm2 = np.zeros(nc)
+    tT = np.zeros((nc, nrt))
+    td = np.zeros((nc, nrd))
+    dp = C.POINTER(C.c_double)
+    check(lib().jolt_analyze_from_host(C.byref(s), C.c_void_p(k_host.data_ptr()), C.c_void_p(v_host.data_ptr()),
+                                       _ptr(k_dev), _ptr(v_dev), norm2.ctypes.data_as(dp), tT.ctypes.data_as(dp),
+                                       td.ctypes.data_as(dp), _ptr(ws), ws.numel(), _stream(stream)),
+          "jolt_analyze_from_host")
+    return norm2, tT, td
+
+
 def compress(s: Shape, k, v, choices, cache, ws, stream=None):
     check(lib().jolt_compress(C.byref(s), _ptr(k), _ptr(v), choices_array(choices), _ptr(cache),
                               cache.numel(), _ptr(ws), ws.numel(), _stream(stream)), "jolt_compress")
@@ -361,7 +377,7 @@ def stats_read(reset=True):
                                      bytes=arr[i].bytes) for i in range(len(KERNEL_FAMILIES))}
 
 
-__all__ = ["layer_align_workspace", "layer_align", "group_layers", "uniform_group", "gemm_bf16_hilo", "gemm_bf16_residual", "allocate_variant", "JOLT_ALLOC_JOINT", "JOLT_ALLOC_KV_SPLIT", "JOLT_ALLOC_UNIFORM", "serialize_cache", "deserialize_cache", "cache_blob_info", "cache_blob_bytes", "decode_attn_noalloc", "stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
+__all__ = ["analyze_from_host", "layer_align_workspace", "layer_align", "group_layers", "uniform_group", "gemm_bf16_hilo", "gemm_bf16_residual", "allocate_variant", "JOLT_ALLOC_JOINT", "JOLT_ALLOC_KV_SPLIT", "JOLT_ALLOC_UNIFORM", "serialize_cache", "deserialize_cache", "cache_blob_info", "cache_blob_bytes", "decode_attn_noalloc", "stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
            "allocate", "workspace_bytes", "new_workspace", "analyze", "compress", "decode_attn",
            "check_ws", "rotate_rows", "quantize_pack", "unpack_dequant", "JoltError",
            "JOLT_OP_COMPRESS", "JOLT_OP_DECODE"]

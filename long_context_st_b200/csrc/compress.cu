@@ -769,9 +769,64 @@ size_t compress_workspace_bytes(const jolt_shape& s) { return make_plan(s).total
 
 using namespace jolt;
 
+namespace jolt {
+namespace {
+// ready[kv] (optional): an event the stream waits on before the first pass over kind kv's cells
+// (the host-to-device copy of that kind, when the inputs are streamed in).
+jolt_status analyze_impl(const jolt_shape* shape, const void* k, const void* v, double* norm2_out,
+                         double* tail_T_out, double* tail_d_out, void* ws, size_t ws_bytes, void* stream,
+                         const cudaEvent_t* ready);
+}  // namespace
+}  // namespace jolt
+
 extern "C" jolt_status jolt_analyze(const jolt_shape* shape, const void* k, const void* v, double* norm2_out,
                                     double* tail_T_out, double* tail_d_out, void* ws, size_t ws_bytes,
                                     void* stream) {
+  return analyze_impl(shape, k, v, norm2_out, tail_T_out, tail_d_out, ws, ws_bytes, stream, nullptr);
+}
+
+extern "C" jolt_status jolt_analyze_from_host(const jolt_shape* shape, const void* k_host, const void* v_host,
+                                              void* k_dev, void* v_dev, double* norm2_out, double* tail_T_out,
+                                              double* tail_d_out, void* ws, size_t ws_bytes, void* stream) {
+  if (!shape_ok(shape) || !k_host || !v_host || !k_dev || !v_dev) return JOLT_ERR_INVALID_ARG;
+  const jolt_shape& s = *shape;
+  const size_t bytes = size_t(s.batch) * s.n_layers * s.n_kv * size_t(s.T) * s.d_h * (s.io_dtype == JOLT_F32 ? 4 : 2);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t cs = nullptr;
+  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+  auto cleanup = [&]() {
+    for (cudaEvent_t& e : ev)
+      if (e) cudaEventDestroy(e);
+    if (cs) cudaStreamDestroy(cs);
+  };
+  jolt_status r = JOLT_OK;
+  do {
+    if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) { r = JOLT_ERR_CUDA; break; }
+    bool ok = true;
+    for (cudaEvent_t& e : ev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) { r = JOLT_ERR_CUDA; break; }
+    // the copies wait for earlier work on `stream` (which may still read k_dev / v_dev), then K and
+    // V cross the bus one after the other while the key cells are being analysed
+    if (cudaEventRecord(ev[0], st) != cudaSuccess || cudaStreamWaitEvent(cs, ev[0], 0) != cudaSuccess ||
+        cudaMemcpyAsync(k_dev, k_host, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaEventRecord(ev[1], cs) != cudaSuccess ||
+        cudaMemcpyAsync(v_dev, v_host, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaEventRecord(ev[2], cs) != cudaSuccess) {
+      r = JOLT_ERR_CUDA;
+      break;
+    }
+    r = analyze_impl(shape, k_dev, v_dev, norm2_out, tail_T_out, tail_d_out, ws, ws_bytes, stream, ev + 1);
+    if (cudaStreamSynchronize(cs) != cudaSuccess && r == JOLT_OK) r = JOLT_ERR_CUDA;
+  } while (false);
+  cleanup();
+  return r;
+}
+
+namespace jolt {
+namespace {
+jolt_status analyze_impl(const jolt_shape* shape, const void* k, const void* v, double* norm2_out,
+                         double* tail_T_out, double* tail_d_out, void* ws, size_t ws_bytes, void* stream,
+                         const cudaEvent_t* ready) {
   if (!shape_ok(shape) || !k || !v || !norm2_out || !tail_T_out || !tail_d_out || !ws) return JOLT_ERR_INVALID_ARG;
   const jolt_shape& s = *shape;
   Ctx c;
@@ -793,6 +848,7 @@ extern "C" jolt_status jolt_analyze(const jolt_shape* shape, const void* k, cons
   const int nrt = n_rt(s), nrd = n_rd(s);
   const bool exact_path = (p.l == p.n);
   for (int kv = 0; kv < 2; ++kv) {
+    if (ready) JOLT_CUDA_TRY(cudaStreamWaitEvent(c.st, ready[kv], 0));
     for (int bg0 = 0; bg0 < per_kind; bg0 += p.C) {
       const int C = std::min(p.C, per_kind - bg0);
       std::vector<double> evT, evD;
@@ -835,6 +891,8 @@ extern "C" jolt_status jolt_analyze(const jolt_shape* shape, const void* k, cons
   JOLT_CUDA_TRY(cudaStreamSynchronize(c.st));
   return JOLT_OK;
 }
+}  // namespace
+}  // namespace jolt
 
 // ---- layer alignment (grouping) ----------------------------------------------------------------
 

@@ -175,3 +175,26 @@ def test_randomized_path_fp32_factors_orthonormal(cuda_ok):
     w = get_workload("llama8b_32k", n_layers=4, T=4096)
     run(w, uniform(w, (256, 96, 2)), factor_dtype="f32", tail_tol=2e-3)
 
+
+
+def test_analyze_from_host_matches_device_inputs(cuda_ok):
+    """jolt_analyze_from_host copies K and V from pinned host memory inside the call (the value
+    copy overlapping the key cells' passes): the device buffers end up holding the inputs and the
+    spectra agree with jolt_analyze on device inputs (up to the split-K summation order)."""
+    w = get_workload("llama8b_32k", n_layers=8, T=3000)
+    K, V = make_kv(w, device="cuda")
+    s = api.make_shape(w)
+    ws = api.new_workspace(s, api.JOLT_OP_COMPRESS)
+    ref = api.analyze(s, K, V, ws)
+    Kh, Vh = K.cpu().pin_memory(), V.cpu().pin_memory()
+    Kd, Vd = torch.zeros_like(K), torch.zeros_like(V)
+    got = api.analyze_from_host(s, Kh, Vh, Kd, Vd, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(Kd, K) and torch.equal(Vd, V)
+    for a, b in zip(got, ref):
+        assert np.allclose(a, b, rtol=1e-5, atol=1e-6 * float(np.max(np.abs(b)))), np.max(np.abs(a - b))
+    # the stored tag lets jolt_compress run on the streamed-in buffers
+    choices = [(256, 64, 4)] * (2 * w.batch * (w.n_layers // w.layers_per_group))
+    _, total = api.cache_layout(s, choices)
+    cache = torch.zeros(total, dtype=torch.uint8, device="cuda")
+    api.compress(s, Kd, Vd, choices, cache, ws)
