@@ -37,6 +37,7 @@ uint64_t shape_tag(const jolt_shape& s) {
 
 struct Plan {
   int C;          // cells per pass
+  int cc;         // cells per compress chunk
   int T, d, LgH, n, l, qcap;
   int64_t cell_elems;
   size_t off_ut, off_pass, off_cmp, total;
@@ -49,7 +50,7 @@ struct Plan {
 
 // jolt_compress handles cells in chunks of this many: per chunk one batched eigensolver launch for
 // the feature-mode Grams S_Y of all its cells.
-constexpr int kCmpChunk = 8;
+constexpr int kCmpChunk = 40;  // at most this many cells per chunk (one eigensolver launch each)
 
 Plan make_plan(const jolt_shape& s) {
   Plan p{};
@@ -110,17 +111,18 @@ Plan make_plan(const jolt_shape& s) {
   p.uh = relc(T * q * 2);
   p.ul = relc(T * q * 2);
   p.um = relc(T * q * 2);
-  p.ylh = relc(size_t(kCmpChunk) * p.LgH * q * d * 4);
-  p.sy = relc(size_t(kCmpChunk) * d * d * 4);
-  p.evy = relc(size_t(kCmpChunk) * d * 4);
-  p.evecy = relc(size_t(kCmpChunk) * d * d * 4);
+  p.cc = std::max(1, std::min(kCmpChunk, n_cells(s)));
+  p.ylh = relc(size_t(p.cc) * p.LgH * q * d * 4);
+  p.sy = relc(size_t(p.cc) * d * d * 4);
+  p.evy = relc(size_t(p.cc) * d * 4);
+  p.evecy = relc(size_t(p.cc) * d * d * 4);
   p.ud = relc(d * d * 4);
   p.blh = relc(size_t(p.LgH) * q * d * 4);
   p.bh = relc(size_t(p.LgH) * q * d * 2);
   p.bm = relc(size_t(p.LgH) * q * d * 2);
   p.bl = relc(size_t(p.LgH) * q * d * 2);
   p.xt = relc(size_t(p.LgH) * T * d * 4);
-  p.jac2 = relc(jacobi_scratch_bytes(kCmpChunk, int(d)));
+  p.jac2 = relc(jacobi_scratch_bytes(p.cc, int(d)));
   p.total = off;
   return p;
 }
@@ -1040,8 +1042,8 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
     um = f32 ? c.atc<__nv_bfloat16>(p.um) : nullptr;
     k_store_ut<<<grid1(int64_t(T) * rT), 256, 0, c.st>>>(U, T, q, rT, f32, cut, f32 ? uh : nullptr, um, ul);
   };
-  for (int c0 = 0; c0 < nc; c0 += kCmpChunk) {
-    const int c1 = std::min(nc, c0 + kCmpChunk);
+  for (int c0 = 0; c0 < nc; c0 += p.cc) {
+    const int c1 = std::min(nc, c0 + p.cc);
     // ---- per cell: Y_lh = U_T^T X_lh [LgH][rT][d] and S_Y (slot = rank among the chunk's
     // cells with r_T > 0) ----
     int nact = 0;
