@@ -90,12 +90,9 @@ __device__ __forceinline__ void load_codes(const uint8_t* row, float (&v)[kD]) {
   for (int j = 0; j < kD; ++j) v[j] = float((w[(j * BITS) >> 5] >> ((j * BITS) & 31)) & mask);
 }
 
-// Same row dequantised (code * scale + zero, one fp32 fused multiply-add per code), as 64 packed
-// pairs of consecutive features.
+// The same row's packed code words (issued early: the loads are consumed later by dequant2).
 template <int BITS>
-__device__ __forceinline__ void load_dequant2(const uint8_t* row, float sc, float zr, float2 (&v)[kD / 2]) {
-  constexpr uint32_t mask = (1u << BITS) - 1u;
-  uint32_t w[4 * BITS + 1];
+__device__ __forceinline__ void load_codes_raw(const uint8_t* row, uint32_t (&w)[4 * BITS + 1]) {
   const uint4* r4 = reinterpret_cast<const uint4*>(row);
 #pragma unroll
   for (int i = 0; i < BITS; ++i) {
@@ -105,6 +102,14 @@ __device__ __forceinline__ void load_dequant2(const uint8_t* row, float sc, floa
     w[4 * i + 2] = x.z;
     w[4 * i + 3] = x.w;
   }
+  w[4 * BITS] = 0u;
+}
+
+// The row dequantised (code * scale + zero, one fp32 fused multiply-add per code), as 64 packed
+// pairs of consecutive features.
+template <int BITS>
+__device__ __forceinline__ void dequant2(const uint32_t (&w)[4 * BITS + 1], float sc, float zr, float2 (&v)[kD / 2]) {
+  constexpr uint32_t mask = (1u << BITS) - 1u;
   const float2 sc2 = make_float2(sc, sc), zr2 = make_float2(zr, zr);
 #pragma unroll
   for (int m = 0; m < kD / 2; ++m) {
@@ -284,16 +289,51 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
     const bool valid = t < p.T;
     float* qb = qs + g * kMaxG * kD;
     bool live = true;
+    // a pair's g_q query rows (g_q * 128 bf16): thread et holds 8 consecutive values of each 1024,
+    // loaded one pair ahead of their use
+    const int nq8 = p.gq * kD / 8;
+    uint4 qn[kMaxG * kD / 1024];
+    auto q_issue = [&](int prq) {
+      const uint4* src = reinterpret_cast<const uint4*>(
+          p.q + (int64_t(prq / p.n_kv) * p.n_q + int64_t(prq % p.n_kv) * p.gq) * kD);
+#pragma unroll
+      for (int j = 0; j < kMaxG * kD / 1024; ++j)
+        qn[j] = et + 128 * j < nq8 ? __ldg(src + et + 128 * j) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    if (g < npairs) q_issue(g);
     for (int pr = g; pr < npairs; pr += 2) {
       const int li = pr / p.n_kv, h = pr % p.n_kv;
-      const __nv_bfloat16* qsrc = p.q + (int64_t(li) * p.n_q + int64_t(h) * p.gq) * kD;
-      for (int e = et; e < p.gq * kD; e += 128) qb[e] = __bfloat162float(qsrc[e]);
-      group_bar(g);
-      float2 v[kD / 2];
+      // this pair's residual row first: its loads overlap the query staging below
+      uint32_t cw[4 * BITS + 1];
+      float scv = 0.f, zrv = 0.f;
       if (BITS > 0 && valid) {
         const int64_t rr = (int64_t(li) * p.n_kv + h) * p.T + t;
         const __half2 szv = p.sz[rr];
-        load_dequant2<BITS>(p.codes + rr * (kD * BITS / 8), __low2float(szv), __high2float(szv), v);
+        load_codes_raw<BITS>(p.codes + rr * (kD * BITS / 8), cw);
+        scv = __low2float(szv);
+        zrv = __high2float(szv);
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxG * kD / 1024; ++j) {
+        const int e0 = (et + 128 * j) * 8;
+        if (e0 < p.gq * kD) {
+          const uint32_t wq[4] = {qn[j].x, qn[j].y, qn[j].z, qn[j].w};
+          float f[8];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 ff = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wq[u]));
+            f[2 * u] = ff.x;
+            f[2 * u + 1] = ff.y;
+          }
+          *reinterpret_cast<float4*>(qb + e0) = make_float4(f[0], f[1], f[2], f[3]);
+          *reinterpret_cast<float4*>(qb + e0 + 4) = make_float4(f[4], f[5], f[6], f[7]);
+        }
+      }
+      if (pr + 2 < npairs) q_issue(pr + 2);
+      group_bar(g);
+      float2 v[kD / 2];
+      if (BITS > 0 && valid) {
+        dequant2<BITS>(cw, scv, zrv, v);
         fwht128x2(v);
 #pragma unroll
         for (int m = 0; m < kD / 2; ++m) v[m] = __fmul2_rn(v[m], sgn[m]);
