@@ -463,7 +463,8 @@ __global__ void __launch_bounds__(128, EPI ? 2 : 1) k_gemm(const __grid_constant
     }
     __syncwarp();
     // ---- epilogue: TMEM -> registers -> smem transpose -> coalesced global ----
-    const bool ok = sm100::mbar_wait(done_bar, 0, p.err);
+    // warp-uniform (the TMEM loads below are warp-collective)
+    const bool ok = __all_sync(0xffffffffu, sm100::mbar_wait(done_bar, 0, p.err));
     sm100::tc_fence_after();
     if (ok && EPI == 1) {
       residual_epilogue<MT, BN>(p, tmem, warp, lane, m0, z, smask);
@@ -686,7 +687,7 @@ __global__ void __launch_bounds__(224, 1) k_gemm_p(const __grid_constant__ TmaPa
       const int b = lt & 1;
       const uint32_t aph = (lt >> 1) & 1;
       ++lt;
-      if (!sm100::mbar_wait(accf_bar(b), aph, p.err)) { fail(); break; }
+      if (!__all_sync(0xffffffffu, sm100::mbar_wait(accf_bar(b), aph, p.err))) { fail(); break; }
       sm100::tc_fence_after();
       const int64_t zoff = int64_t(ti.z / p.c_div) * p.c_bstride;
       const int rbase = ti.m0 + int(rank) * BM + q * 32;

@@ -33,6 +33,9 @@ def test_blob_round_trip_decodes_identically(cuda_ok):
     api.decode_attn(s2, ch2, cache2, q, o2, dws, inv_freq=inv)
     torch.cuda.synchronize()
     # the bytes are identical (above); decode sums split-K partials with float atomics, whose
-    # order (hence last-bit rounding) may differ from one call to the next
-    scale = o1.float().abs().max().item()
-    assert (o1.float() - o2.float()).abs().max().item() <= 1e-5 * scale
+    # order (hence last-bit rounding) may differ from one call to the next: the bf16 outputs agree
+    # to one unit in the last place
+    a, b = o1.float(), o2.float()
+    ulp = torch.maximum(a.abs(), b.abs()) * 2.0 ** -7 + 1e-30
+    assert bool(((a - b).abs() <= ulp).all())
+    assert (a - b).abs().max().item() <= 2.0 ** -7 * a.abs().max().item()
