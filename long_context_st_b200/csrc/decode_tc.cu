@@ -40,16 +40,12 @@ constexpr int kABytes = kBM * kBK * 2;
 constexpr int kBBytes = kBK * kD * 2;
 
 template <int NT>
-// The tile's RoPE factors live in TMEM columns kRopeCol.. (one lane per token row: cos of the 64
-// frequencies, then their sin, times the attention scaling), which leaves shared memory for four
-// TMA stages of the two-term operand instead of three.
 struct KeysCfg {
-  static constexpr int kStages = 4;
+  static constexpr int kStages = NT == 1 ? 4 : 3;
   static constexpr int kStageBytes = kABytes + NT * kBBytes;
   static constexpr int kQsBytes = 2 * kMaxG * kD * 4;      // queries of each epilogue group's pair, fp32
-  static constexpr int kSmem = 1024 + kStages * kStageBytes + kQsBytes + kD * 4 + 256;
-  static constexpr int kRopeCol = 256;                     // accumulators use columns 0 .. 255
-  static constexpr int kTmemCols = 512;
+  static constexpr int kRopeBytes = kD / 4 * kBM * 16;     // (cos, cos, sin, sin) of frequency pairs
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + kQsBytes + kRopeBytes + kD * 4 + 256;
   static constexpr int kThreads = 320;                     // producer, MMA, two groups of four epilogue warps
 };
 
@@ -158,7 +154,8 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* qs = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);  // [2 groups][kMaxG][kD]
-  float2* sgn = reinterpret_cast<float2*>(qs + 2 * kMaxG * kD);               // [64]
+  float4* rope = reinterpret_cast<float4*>(qs + 2 * kMaxG * kD);            // [32][kBM]
+  float2* sgn = reinterpret_cast<float2*>(rope + kD / 4 * kBM);               // [64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sgn + kD / 2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 5);
 
@@ -194,39 +191,25 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
     const float isd = rsqrtf(float(kD));
     sgn[threadIdx.x] = make_float2(isd * rot_sign(p.rot_seed, 2 * threadIdx.x), isd * rot_sign(p.rot_seed, 2 * threadIdx.x + 1));
   }
-  if (warp == 1) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), C::kTmemCols);
+  // RoPE of the tile's tokens: cos / sin of (pos0 + t) * inv_freq[f], angle reduced mod 2 pi in
+  // fp64, times the attention scaling; frequencies 2m and 2m + 1 side by side
+  for (int e = threadIdx.x; e < kD / 4 * kBM; e += blockDim.x) {
+    const int m = e / kBM, tt = e % kBM;
+    float cs[2], sn[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const double ang = double(p.pos0 + t0 + tt) * double(p.inv_freq[2 * m + u]);
+      const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+      sincosf(float(red), &sn[u], &cs[u]);
+    }
+    rope[e] = make_float4(cs[0] * p.rope_scaling, cs[1] * p.rope_scaling, sn[0] * p.rope_scaling, sn[1] * p.rope_scaling);
+  }
+  if (warp == 1) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), 256);
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = sm100::smem_u32(smem);
-  // RoPE of the tile's tokens into TMEM: the first epilogue group (warps 2..5, TMEM lane quarter
-  // warp % 4, one token row per thread) writes cos of (pos0 + t) * inv_freq[f] to column
-  // kRopeCol + f and its sin to kRopeCol + 64 + f, the angle reduced mod 2 pi in fp64, times
-  // the attention scaling
-  if (warp >= 2 && warp < 6) {
-    const int tt = (warp & 3) * 32 + lane;
-    const uint32_t base = tmem + C::kRopeCol + (uint32_t((warp & 3) * 32) << 16);
-#pragma unroll 1
-    for (int f0 = 0; f0 < kD / 2; f0 += 8) {
-      uint32_t cw[8], sw[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const double ang = double(p.pos0 + t0 + tt) * double(p.inv_freq[f0 + u]);
-        const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
-        float sn, cs;
-        sincosf(float(red), &sn, &cs);
-        cw[u] = __float_as_uint(cs * p.rope_scaling);
-        sw[u] = __float_as_uint(sn * p.rope_scaling);
-      }
-      sm100::tmem_st8(base + f0, cw);
-      sm100::tmem_st8(base + kD / 2 + f0, sw);
-    }
-    sm100::tmem_st_wait();
-  }
-  sm100::tc_fence_before();
-  __syncthreads();
-  sm100::tc_fence_after();
 
   if (warp == 0) {
     if (lane == 0 && fac) {
@@ -359,6 +342,7 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
         for (int m = 0; m < kD / 2; ++m) v[m] = make_float2(0.f, 0.f);
       }
       if (fac) {
+        // warp-uniform: the TMEM loads below are warp-collective
         if (live) live = __all_sync(0xffffffffu, sm100::mbar_wait(tfull_bar(g), (pr >> 1) & 1, p.err));
         sm100::tc_fence_after();
 #pragma unroll
@@ -373,30 +357,16 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
         sm100::tc_fence_before();
         sm100::mbar_arrive(tempty_bar(g));
       }
-      {
-        // features (2m, 2m+1) with (2m+64, 2m+65): frequencies 2m, 2m+1, 8 at a time from TMEM.
-        // tcgen05.ld is warp-collective, so every row of the tile rotates (rows past T or after
-        // a failed wait rotate values nobody stores)
-        const uint32_t rbase = tmem + C::kRopeCol + (uint32_t(quarter * 32) << 16);
-#pragma unroll
-        for (int f0 = 0; f0 < kD / 2; f0 += 8) {
-          uint32_t cr[8], sr[8];
-          sm100::tmem_ld8(rbase + f0, cr);
-          sm100::tmem_ld8(rbase + kD / 2 + f0, sr);
-          sm100::tmem_ld_wait();
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int m = f0 / 2 + u;
-            const float2 cs = make_float2(__uint_as_float(cr[2 * u]), __uint_as_float(cr[2 * u + 1]));
-            const float2 sn = make_float2(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1]));
-            const float2 x1 = v[m], x2 = v[m + kD / 4];
-            const float2 a = __fmul2_rn(x2, sn), b = __fmul2_rn(x1, sn);
-            v[m] = __ffma2_rn(x1, cs, make_float2(-a.x, -a.y));
-            v[m + kD / 4] = __ffma2_rn(x2, cs, b);
-          }
-        }
-      }
       if (valid && live) {
+#pragma unroll
+        for (int m = 0; m < kD / 4; ++m) {  // features (2m, 2m+1) with (2m+64, 2m+65)
+          const float4 r4 = rope[m * kBM + row];
+          const float2 cs = make_float2(r4.x, r4.y), sn = make_float2(r4.z, r4.w);
+          const float2 x1 = v[m], x2 = v[m + kD / 4];
+          const float2 a = __fmul2_rn(x2, sn), b = __fmul2_rn(x1, sn);
+          v[m] = __ffma2_rn(x1, cs, make_float2(-a.x, -a.y));
+          v[m + kD / 4] = __ffma2_rn(x2, cs, b);
+        }
         float* out = p.scores + (int64_t(li) * p.n_q + int64_t(h) * p.gq) * p.T + t;
 #pragma unroll 1
         for (int gg = 0; gg < p.gq; ++gg) {
@@ -416,7 +386,7 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
   }
   sm100::tc_fence_before();
   __syncthreads();
-  if (warp == 1) sm100::tmem_dealloc(tmem, C::kTmemCols);
+  if (warp == 1) sm100::tmem_dealloc(tmem, 256);
 }
 
 // ---- CUDA-core stages -------------------------------------------------------------------------
