@@ -195,3 +195,25 @@ def test_group_layers_matches_oracle():
             for mg in (0, 2, 3):
                 assert api.group_layers(a, tau, mg) == o_group(list(a), tau, mg)
             assert api.uniform_group(a, tau) == o_uniform(list(a), a.size + 1, tau)
+
+
+def test_argument_checks_before_any_device_work():
+    """Entry points added for streaming, grouping and failure detection reject bad arguments on
+    the host (no device needed)."""
+    import ctypes as C
+    from long_context_st_b200 import api
+    from long_context_st_b200._lib import lib
+    w = get_workload("toy", n_layers=2)
+    s = api.make_shape(w)
+    L = lib()
+    # streamed analyze: null host or device buffers
+    assert L.jolt_analyze_from_host(C.byref(s), None, None, None, None, None, None, None, None, 0, None) == -1
+    # layer alignment: rank not a multiple of 16, or above min(T, n_kv*d_h)
+    assert L.jolt_layer_align_workspace(C.byref(s), 24) == 0
+    assert L.jolt_layer_align_workspace(C.byref(s), 16 * 1000) == 0
+    assert L.jolt_layer_align_workspace(C.byref(s), 16) > 0
+    # grouping: no layers, null outputs
+    assert L.jolt_group_layers(None, 0, 0.5, 0, None, None) == -1
+    # self-test: unbounded or zero limits, unknown test, too small a workspace
+    assert L.jolt_selftest_timeout(0, 0, None, 512, None) == -1
+    assert L.jolt_selftest_timeout(3, 1000, None, 512, None) == -1
