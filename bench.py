@@ -483,6 +483,12 @@ def main():
     dom = max(fams, key=lambda k: stats[k]["ms"])
     roof = binding(dom)
     roof_dec = binding("decode_main")
+    # DRAM traffic of the key kernel from one ncu capture (profiles/k_keys_tc_k_values_res_*:
+    # one 4-layer group of the 70B shape at T = 65536, r_T = 464, b = 4: 225.7 MB read + 58.7 MB
+    # written), scaled to a full launch by the tokens it processes; other workloads: not measured
+    if roof_dec is not None and w.name == "llama70b_128k" and w.keys_pre_rope:
+        roof_dec["traffic"] = (225.711616e6 + 58.666752e6) * (w.T / 65536)
+        roof_dec["traffic_source"] = "ncu capture at T = 65536 scaled by T (one layer group per launch)"
 
     line = {"metric": METRIC, "value": value, "unit": "context tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
