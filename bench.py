@@ -523,36 +523,53 @@ def main():
             "gpu_launches": n_kernels * args.steps if n_kernels is not None else None,
             "kernels": kernel_names, "clocks": clk.summary(), "choices": sorted(set(map(tuple, step.choices)))}
 
-    # e2e: same step through the C ABI with host buffers: H2D of K and V and D2H of the outputs
+    # e2e: same step through the C ABI with host buffers: H2D of K and V and D2H of the outputs.
+    # Every rank takes the same collective steps whether or not its own leg worked.
     if not args.no_e2e:
+        e_ms, err, h2d, d2h = None, None, 0, 0
+        n_e2e = max(1, min(args.steps, 3))
         try:
             Kh = step.K.cpu().pin_memory()
             Vh = step.V.cpu().pin_memory()
             outh = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
             Kd = torch.empty_like(step.K)
             Vd = torch.empty_like(step.V)
+            h2d = Kh.numel() * Kh.element_size() * 2
+            d2h = outh.numel() * outh.element_size()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
-            n_e2e = max(1, min(args.steps, 3))
             step.run(K=Kd, V=Vd, host=(Kh, Vh))
             outh.copy_(step.out, non_blocking=True)
             torch.cuda.synchronize()
-            e0.record()
-            for _ in range(n_e2e):
-                # the H2D copies of K and V run inside the analyze call (jolt_analyze_from_host)
-                step.run(K=Kd, V=Vd, host=(Kh, Vh))
-                outh.copy_(step.out, non_blocking=True)
-            e1.record()
-            torch.cuda.synchronize()
-            e_ms = e0.elapsed_time(e1) / n_e2e
-            line["e2e"] = {"value": tokens * world / (e_ms / 1e3), "unit": "context tokens/s",
-                           "h2d_bytes_per_step": Kh.numel() * Kh.element_size() * 2,
-                           "d2h_bytes_per_step": outh.numel() * outh.element_size(), "ms_per_step": e_ms,
-                           "steps": n_e2e}
-            del Kh, Vh, Kd, Vd
         except (RuntimeError, MemoryError) as ex:
+            err = str(ex)[:200]
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        if err is None:
+            try:
+                e0.record()
+                for _ in range(n_e2e):
+                    # the H2D copies of K and V run inside the analyze call (jolt_analyze_from_host)
+                    step.run(K=Kd, V=Vd, host=(Kh, Vh))
+                    outh.copy_(step.out, non_blocking=True)
+                e1.record()
+                torch.cuda.synchronize()
+                e_ms = e0.elapsed_time(e1) / n_e2e
+            except (RuntimeError, MemoryError) as ex:
+                err = str(ex)[:200]
+        if world > 1:
+            e_ms = max_over_ranks(e_ms if e_ms is not None else float("inf"), dev)
+            if not math.isfinite(e_ms):
+                e_ms, err = None, err or "the end-to-end leg failed on another rank"
+        if e_ms is not None:
+            line["e2e"] = {"value": tokens * world / (e_ms / 1e3), "unit": "context tokens/s",
+                           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+                           "steps": n_e2e}
+        else:
             line["e2e"] = {"value": None, "unit": "context tokens/s", "h2d_bytes_per_step": 0,
-                           "d2h_bytes_per_step": 0, "error": str(ex)[:200]}
+                           "d2h_bytes_per_step": 0, "error": err}
+        Kh = Vh = Kd = Vd = None
 
     # CPU oracle on a bounded sample (rank 0, N = 1 only)
     if rank == 0 and world == 1 and not args.no_cpu:
