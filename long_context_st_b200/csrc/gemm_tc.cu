@@ -2,12 +2,13 @@
 // memory stages; one thread issues tcgen05.mma into TMEM accumulators; epilogue warps drain TMEM
 // with tcgen05.ld and store (or atomically add) fp32 C.
 //
-// Two kernels. k_gemm: one output tile per CTA (128 threads: warp 0 lane 0 = TMA producer, warp
-// 1 lane 0 = MMA issuer, warp 2 = TMEM allocator, all four warps run the epilogue), used for
-// N <= 128 or a single 128-row tile. k_gemm_p: persistent, by default as CTA pairs
-// (cta_group::2, M = 256 per MMA, each SM stages half of B) with two TMEM accumulators so the
-// epilogue of one tile overlaps the main loop of the next. Every mbarrier wait is bounded (2 s)
-// and reports JOLT_ERR_TIMEOUT instead of hanging.
+// Two kernels. k_gemm (the default): one output tile per CTA of 128 threads — lane 0 of warp 0
+// streams A and lane 0 of warp 2 streams B by TMA, lane 0 of warp 1 issues the MMAs, warp 2 owns
+// the TMEM allocation, all four warps run the epilogue (fp32 stores or atomics, the bf16 hi/lo
+// split of the result, or the fused residual coder). k_gemm_p (selected with JOLT_GEMM_PLAN):
+// persistent, as single CTAs or CTA pairs (cta_group::2, M = 256 per MMA, each SM stages half of
+// B), with two TMEM accumulators so the epilogue of one tile overlaps the main loop of the next.
+// Every mbarrier wait is bounded (2 s) and reports JOLT_ERR_TIMEOUT instead of hanging.
 //
 // Several (A_t, B_t) "terms" can accumulate into one tile: a fp32 operand split as hi + lo bf16
 // parts gives x*y ~ hi*hi + hi*lo + lo*hi with ~2^-16 relative error at bf16 tensor-core speed.
