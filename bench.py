@@ -374,6 +374,15 @@ def max_over_ranks(ms, device):
     return float(t.item())
 
 
+def e2e_over_ranks(e_ms, err, device):
+    """Slowest rank's end-to-end step time; None (with a reason) when any rank's leg failed.
+    Every rank calls this at the same point, whatever happened to its own leg."""
+    t = max_over_ranks(e_ms if e_ms is not None else float("inf"), device)
+    if not math.isfinite(t):
+        return None, err or "the end-to-end leg failed on another rank"
+    return t, err
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -559,9 +568,7 @@ def main():
             except (RuntimeError, MemoryError) as ex:
                 err = str(ex)[:200]
         if world > 1:
-            e_ms = max_over_ranks(e_ms if e_ms is not None else float("inf"), dev)
-            if not math.isfinite(e_ms):
-                e_ms, err = None, err or "the end-to-end leg failed on another rank"
+            e_ms, err = e2e_over_ranks(e_ms, err, dev)
         if e_ms is not None:
             line["e2e"] = {"value": tokens * world / (e_ms / 1e3), "unit": "context tokens/s",
                            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,

@@ -32,6 +32,35 @@ def _rank_main(rank, world, port, q):
     dist.destroy_process_group()
 
 
+def _e2e_rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    dev = torch.device("cpu")
+    ok = bench.e2e_over_ranks(100.0 + rank, None, dev)                       # both legs worked
+    one_failed = bench.e2e_over_ranks(None if rank == 1 else 50.0,
+                                      "out of pinned memory" if rank == 1 else None, dev)
+    q.put((rank, ok, one_failed))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_e2e_leg_reduces_over_ranks_even_when_one_fails():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_e2e_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [(101.0, None), (101.0, None)]  # the slowest rank's time
+    assert res[0][2] == (None, "the end-to-end leg failed on another rank")
+    assert res[1][2] == (None, "out of pinned memory")
+
+
 def test_max_over_ranks_and_weak_scaling_workloads():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
