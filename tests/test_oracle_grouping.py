@@ -93,3 +93,25 @@ def test_planted_groups_recovered():
     assert np.all(a[inside] > 0.99)
     assert np.all(np.delete(a, inside) < 0.2)
     assert group_layers(a, 0.5) == sizes
+
+
+def test_grouping_properties_random():
+    """group sizes partition the layers; every in-group link is >= tau and every boundary link
+    is < tau (without a size cap); the uniform size divides L and respects tau inside groups."""
+    rng = np.random.default_rng(11)
+    for _ in range(200):
+        L = int(rng.integers(1, 40))
+        a = rng.uniform(0, 1, size=L - 1)
+        tau = float(rng.uniform(0.1, 0.9))
+        sizes = group_layers(a, tau)
+        assert sum(sizes) == L and min(sizes) >= 1
+        edge = np.cumsum(sizes)[:-1] - 1          # last layer of each group but the final one
+        inside = np.setdiff1d(np.arange(L - 1), edge)
+        assert np.all(a[inside] >= tau) and np.all(a[edge] < tau)
+        Lg = uniform_group(a, L, tau)
+        assert L % Lg == 0
+        assert all(a[l] >= tau for l in range(L - 1) if (l + 1) % Lg)
+        # no larger divisor qualifies
+        for g in range(Lg + 1, L + 1):
+            if L % g == 0:
+                assert not all(a[l] >= tau for l in range(L - 1) if (l + 1) % g)
