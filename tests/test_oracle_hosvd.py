@@ -73,3 +73,55 @@ def test_spectra_tails():
     # tails agree with the ST-HOSVD spectra at the same ranks
     _, _, _, sig2, _ = st_hosvd(X, 16, 16)
     assert tT[1] == pytest.approx(sig2[16:].sum(), rel=1e-9)
+
+
+def _known_spectrum_tensor(L, H, T, d, sig, seed):
+    """X[l,h] = A_lh diag(sig) W^T with every A_lh [T, d] having orthonormal columns and W an
+    orthogonal d x d basis: X[l,h]^T X[l,h] = W diag(sig^2) W^T for every (l, h), so the feature
+    Gram sum_lh X_lh^T X_lh has the eigenvalues L*H*sig_j^2 exactly (up to rounding)."""
+    rng = np.random.default_rng(seed)
+    W = np.linalg.qr(rng.standard_normal((d, d)))[0]
+    X = np.empty((L, H, T, d))
+    for l in range(L):
+        for h in range(H):
+            A = np.linalg.qr(rng.standard_normal((T, d)))[0]
+            X[l, h] = (A * sig[None, :]) @ W.T
+    return X
+
+
+@pytest.mark.parametrize("L,H", [(1, 1), (2, 3)])
+def test_spectra_tails_feature_closed_form(L, H):
+    # [v4 §3] the feature-mode tail is the discarded energy sum_{j > r_d} lambda_j(S_d), lambda in
+    # decreasing order. Singular values given in a shuffled order: a tail summed from the
+    # smallest eigenvalue first, or over the wrong end, misses the closed form below.
+    d, T = 64, 160
+    rng = np.random.default_rng(11)
+    sig = rng.permutation(np.linspace(5.0, 0.1, d) ** 1.5)
+    X = _known_spectrum_tensor(L, H, T, d, sig, seed=12)
+    n2, tT, td = spectra_tails(X, 64)
+    lam = np.sort(L * H * sig ** 2)[::-1]
+    assert n2 == pytest.approx(lam.sum(), rel=1e-12)
+    for j in range(d // 16 + 1):
+        assert td[j] == pytest.approx(lam[16 * j:].sum(), rel=1e-9, abs=1e-9 * n2), j
+    if L * H == 1:
+        # one slice: X = A diag(sig) W^T is its own SVD, so the token tail is the same closed form
+        for k in range(len(tT)):
+            assert tT[k] == pytest.approx(lam[16 * k:].sum(), rel=1e-9, abs=1e-9 * n2), k
+
+
+def test_spectra_tails_token_closed_form_grouped():
+    # token-mode tail of a grouped cell: columns of X_(T) spanned by the orthonormal token basis P
+    # with X[l,h] = P diag(s) C_lh^T where the stacked C_lh [n_heads*d, r] has orthonormal columns:
+    # X_(T) = P diag(s) C^T is an SVD, so t_T(16k) = sum_{i > 16k} s_i^2 (s in decreasing order).
+    L, H, T, d, r = 2, 2, 300, 32, 48
+    rng = np.random.default_rng(13)
+    P = np.linalg.qr(rng.standard_normal((T, r)))[0]
+    C = np.linalg.qr(rng.standard_normal((L * H * d, r)))[0]
+    s = rng.permutation(np.geomspace(30.0, 0.5, r))
+    XT = (P * s[None, :]) @ C.T                                  # [T, L*H*d], columns (l, h, j)
+    X = XT.reshape(T, L, H, d).transpose(1, 2, 0, 3)
+    assert np.allclose(token_unfolding(X), XT)
+    n2, tT, td = spectra_tails(X, 64)
+    s2 = np.sort(s ** 2)[::-1]
+    for k in range(len(tT)):
+        assert tT[k] == pytest.approx(s2[16 * k:].sum(), rel=1e-9, abs=1e-9 * n2), k
