@@ -275,7 +275,9 @@ def surrogate_error(tables, choices, phi):
 
 def allocator_ablation(step):
     """The pages' allocation ablations on this step's own tables at its budget (first sequence):
-    joint (one multiplier), K/V-decoupled, uniform ranks — summed surrogate error / ||X||^2."""
+    joint (one multiplier, exact per-cell search), K/V-decoupled, uniform ranks, and the pages'
+    coordinate-wise rank search under the same multiplier — summed surrogate error / ||X||^2, bytes
+    used and the share of the budget they use."""
     api, w = step.api, step.w
     if w.fixed_choice or step.budget is None:
         return None
@@ -283,11 +285,13 @@ def allocator_ablation(step):
     n2, tT, td = (np.asarray(a)[:2 * G] for a in step.tables)
     out = {"budget_bytes": step.budget}
     for name, mode in (("joint", api.JOLT_ALLOC_JOINT), ("kv_split", api.JOLT_ALLOC_KV_SPLIT),
-                       ("uniform", api.JOLT_ALLOC_UNIFORM)):
+                       ("uniform", api.JOLT_ALLOC_UNIFORM), ("coordinate", api.JOLT_ALLOC_COORD)):
         try:
+            t0 = time.perf_counter()
             ch, tot = api.allocate_variant(step.shape, n2, tT, td, step.phi, step.budget, mode)
             out[name] = {"rel_error": surrogate_error((n2, tT, td), ch, step.phi) / float(np.sum(n2)),
-                         "bytes": tot}
+                         "bytes": tot, "budget_use": tot / step.budget,
+                         "host_ms": (time.perf_counter() - t0) * 1e3}
         except api.JoltError as e:
             out[name] = {"error": str(e)}
     return out

@@ -175,9 +175,18 @@ jolt_status jolt_allocate(const jolt_shape* shape, int32_t n_cells, const double
  *   JOLT_ALLOC_UNIFORM   uniform ranks: one (r_T, r_d, b) for every key cell and one for every
  *                        value cell, the pair of least summed error whose bytes fit (ties: fewer
  *                        bytes, then the earlier key choice, then the earlier value choice, choices
- *                        ordered by r_T, r_d, b).
+ *                        ordered by r_T, r_d, b);
+ *   JOLT_ALLOC_COORD     the pages' coordinate-wise rank search ("A JoLT for the KV cache", §3: a
+ *                        heuristic over the two truncated modes) under the same single multiplier:
+ *                        for a multiplier lam each cell starts at full ranks and alternates the best
+ *                        r_T with r_d held (r_T = 0 takes the residual-only choices) and the best r_d
+ *                        with r_T held, b chosen with each move, by E + lam * bytes (ties: fewer
+ *                        bytes, smaller r_T, r_d, b) until a round changes nothing (at most 32);
+ *                        lam is the fitting end of a geometric bisection of [1e-30, 1e30] (200
+ *                        halvings, midpoint sqrt(lo * hi)). Never better than jolt_allocate at equal
+ *                        bytes; reported beside it to show what the exact search gains.
  * Host-only. JOLT_ERR_BUDGET if nothing fits; JOLT_ERR_INVALID_ARG for an odd n_cells or bad mode. */
-typedef enum { JOLT_ALLOC_JOINT = 0, JOLT_ALLOC_KV_SPLIT = 1, JOLT_ALLOC_UNIFORM = 2 } jolt_alloc_mode;
+typedef enum { JOLT_ALLOC_JOINT = 0, JOLT_ALLOC_KV_SPLIT = 1, JOLT_ALLOC_UNIFORM = 2, JOLT_ALLOC_COORD = 3 } jolt_alloc_mode;
 jolt_status jolt_allocate_variant(const jolt_shape* shape, int32_t n_cells, const double* norm2,
                                   const double* tail_T, int32_t n_rt, const double* tail_d, int32_t n_rd,
                                   const double phi[4], uint64_t budget, int32_t mode,

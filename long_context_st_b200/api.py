@@ -121,7 +121,7 @@ def phi(d_h: int, n_rows: int = 1 << 16, seed: int = 1):
     return list(out)
 
 
-JOLT_ALLOC_JOINT, JOLT_ALLOC_KV_SPLIT, JOLT_ALLOC_UNIFORM = 0, 1, 2
+JOLT_ALLOC_JOINT, JOLT_ALLOC_KV_SPLIT, JOLT_ALLOC_UNIFORM, JOLT_ALLOC_COORD = 0, 1, 2, 3
 
 
 def allocate_variant(s: Shape, norm2, tail_T, tail_d, phi4, budget: int, mode: int):

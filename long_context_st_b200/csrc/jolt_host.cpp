@@ -303,6 +303,104 @@ jolt_status jolt_allocate(const jolt_shape* s, int32_t nc, const double* norm2,
   return JOLT_OK;
 }
 
+namespace {
+
+// One option of a cell: bytes, modelled error and the choice.
+struct CoordOpt {
+  uint64_t B;
+  double E;
+  int32_t rT, rd, b;
+};
+
+// Ordering of the coordinate search: E + lam * bytes, then bytes, r_T, r_d, b.
+bool coord_less(const CoordOpt& x, const CoordOpt& y, double lam) {
+  const double vx = x.E + lam * double(x.B), vy = y.E + lam * double(y.B);
+  if (vx != vy) return vx < vy;
+  if (x.B != y.B) return x.B < y.B;
+  if (x.rT != y.rT) return x.rT < y.rT;
+  if (x.rd != y.rd) return x.rd < y.rd;
+  return x.b < y.b;
+}
+
+// The coordinate-wise rank search of one cell at multiplier lam: from full ranks, the best r_T
+// with r_d held (a zero token rank takes the residual-only options), then the best r_d with r_T
+// held, b chosen with each move, until a round changes nothing (at most 32 rounds).
+CoordOpt coord_cell(const std::vector<CoordOpt>& opts, int32_t rTmax, int32_t rdmax, double lam) {
+  const CoordOpt* cur = nullptr;
+  for (const CoordOpt& o : opts)
+    if (o.rT == rTmax && o.rd == rdmax && (!cur || coord_less(o, *cur, lam))) cur = &o;
+  for (int round = 0; round < 32; ++round) {
+    const CoordOpt* start = cur;
+    const CoordOpt* best = nullptr;
+    for (const CoordOpt& o : opts)
+      if ((o.rd == cur->rd || o.rT == 0) && (!best || coord_less(o, *best, lam))) best = &o;
+    cur = best;
+    best = nullptr;
+    for (const CoordOpt& o : opts)
+      if (o.rT == cur->rT && (!best || coord_less(o, *best, lam))) best = &o;
+    cur = best;
+    if (cur == start) break;
+  }
+  return *cur;
+}
+
+// Coordinate-wise allocation: the multiplier from a geometric bisection of [1e-30, 1e30] (200
+// halvings, midpoint sqrt(lo * hi)); the allocation of the bracket end that fits the budget.
+jolt_status allocate_coord(const jolt_shape* s, int32_t nc, const double* norm2, const double* tail_T, int32_t nrt,
+                           const double* tail_d, int32_t nrd, const double phi[4], uint64_t budget,
+                           jolt_cell_choice* out, uint64_t* total_out) {
+  const int bits[4] = {0, 2, 4, 8};
+  std::vector<std::vector<CoordOpt>> cells(nc);
+  for (int c = 0; c < nc; ++c) {
+    if (!std::isfinite(norm2[c])) return JOLT_ERR_NUMERIC;
+    for (int k = 0; k < nrt; ++k)
+      for (int j = 0; j < nrd; ++j) {
+        if ((k == 0) != (j == 0)) continue;
+        const double D = k == 0 ? norm2[c] : std::min(norm2[c], tail_T[size_t(c) * nrt + k] + tail_d[size_t(c) * nrd + j]);
+        if (!std::isfinite(D)) return JOLT_ERR_NUMERIC;
+        for (int bi = 0; bi < 4; ++bi) {
+          const jolt_cell_choice ch{k * kRankStep, j * kRankStep, bits[bi]};
+          cells[c].push_back(CoordOpt{jolt_cell_bytes(s, ch), D * phi[bi], ch.r_T, ch.r_d, ch.b});
+        }
+      }
+  }
+  const int32_t rTmax = (nrt - 1) * kRankStep, rdmax = (nrd - 1) * kRankStep;
+  std::vector<CoordOpt> pick(nc), best(nc);
+  auto at = [&](double lam, std::vector<CoordOpt>& dst) {
+    uint64_t tot = 0;
+    for (int c = 0; c < nc; ++c) {
+      dst[c] = coord_cell(cells[c], rTmax, rdmax, lam);
+      tot += dst[c].B;
+    }
+    return tot;
+  };
+  double lo = 1e-30, hi = 1e30;
+  uint64_t b_hi = at(hi, best);
+  if (b_hi > budget) return JOLT_ERR_BUDGET;
+  uint64_t b_lo = at(lo, pick);
+  if (b_lo <= budget) {
+    best = pick;
+    b_hi = b_lo;
+  } else {
+    for (int it = 0; it < 200; ++it) {
+      const double mid = std::sqrt(lo * hi);
+      const uint64_t b = at(mid, pick);
+      if (b <= budget) {
+        hi = mid;
+        best = pick;
+        b_hi = b;
+      } else {
+        lo = mid;
+      }
+    }
+  }
+  for (int c = 0; c < nc; ++c) out[c] = jolt_cell_choice{best[c].rT, best[c].rd, best[c].b};
+  if (total_out) *total_out = b_hi;
+  return JOLT_OK;
+}
+
+}  // namespace
+
 jolt_status jolt_allocate_variant(const jolt_shape* s, int32_t nc, const double* norm2, const double* tail_T,
                                   int32_t nrt, const double* tail_d, int32_t nrd, const double phi[4],
                                   uint64_t budget, int32_t mode, jolt_cell_choice* out, uint64_t* total_out) {
@@ -336,6 +434,7 @@ jolt_status jolt_allocate_variant(const jolt_shape* s, int32_t nc, const double*
     if (total_out) *total_out = total;
     return JOLT_OK;
   }
+  if (mode == JOLT_ALLOC_COORD) return allocate_coord(s, nc, norm2, tail_T, nrt, tail_d, nrd, phi, budget, out, total_out);
   if (mode != JOLT_ALLOC_UNIFORM) return JOLT_ERR_INVALID_ARG;
   // every choice in (r_T, r_d, b) order with its bytes and its summed error over each kind's cells
   const int bits[4] = {0, 2, 4, 8};

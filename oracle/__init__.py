@@ -19,6 +19,6 @@ from .rotation import hadamard, rotation_matrix  # noqa: F401
 from .bytes_model import kv_cache_bytes, cell_bytes, raw_sequence_bytes  # noqa: F401
 from .hosvd import token_unfolding, st_hosvd, spectra_tails, reconstruct  # noqa: F401
 from .quant import quantize_rows, dequantize_rows, pack_codes, unpack_codes, phi_table  # noqa: F401
-from .alloc import build_options, allocate, brute_force_allocate, allocate_kv_split, allocate_uniform  # noqa: F401
+from .alloc import build_options, allocate, brute_force_allocate, allocate_kv_split, allocate_uniform, allocate_coord  # noqa: F401
 from .codec import compress_cell, decompress_cell, decompress_slice, decode_attention, rope  # noqa: F401
 from .grouping import layer_token_basis, subspace_alignment, layer_alignment, group_layers, uniform_group  # noqa: F401

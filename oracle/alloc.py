@@ -157,6 +157,58 @@ def allocate_uniform(cell_options, budget: int):
     return choices, int(Bt[k, v])
 
 
+def _coord_cell(opts, lam, max_rounds=32):
+    """One cell's choice for multiplier lam by the coordinate-wise rank search: from full ranks,
+    alternately the best r_T with r_d held (r_T = 0 forces r_d = 0) and the best r_d with r_T held,
+    b chosen with each move, until a round changes nothing. The current option is always a
+    candidate, so E + lam * bytes never rises. Ordering key: (E + lam * bytes, bytes, r_T, r_d, b)."""
+    def key(o):
+        return (o[1] + lam * o[0], o[0], o[2], o[3], o[4])
+
+    kmax = max(o[2] for o in opts)
+    jmax = max(o[3] for o in opts)
+    cur = min((o for o in opts if o[2] == kmax and o[3] == jmax), key=key)
+    for _ in range(max_rounds):
+        start = cur
+        # token-mode move: r_d held (a zero token rank takes the residual-only option)
+        cand = [o for o in opts if o[3] == cur[3] or o[2] == 0]
+        cur = min(cand, key=key)
+        # feature-mode move: r_T held
+        cand = [o for o in opts if o[2] == cur[2]]
+        cur = min(cand, key=key)
+        if cur == start:
+            break
+    return cur
+
+
+def allocate_coord(cell_options, budget: int, iters: int = 200):
+    """The pages' coordinate-wise rank search ([v4] §3: a heuristic over the two truncated modes)
+    under the same single multiplier and error model. Reading: each cell's choice for a given lam
+    comes from _coord_cell; lam is the bracket end of a geometric bisection over [1e-30, 1e30]
+    (iters halvings of the bracket, midpoint sqrt(lo * hi)) with the largest total bytes that still
+    fit. Returns (choices, lam, total bytes); BudgetError if even the sparsest allocation does not
+    fit."""
+    def at(lam):
+        ch = [_coord_cell(o, lam) for o in cell_options]
+        return ch, sum(o[0] for o in ch)
+
+    lo, hi = 1e-30, 1e30
+    ch_hi, b_hi = at(hi)
+    if b_hi > budget:
+        raise BudgetError(f"budget {budget} below the sparsest coordinate allocation {b_hi}")
+    ch_lo, b_lo = at(lo)
+    if b_lo <= budget:
+        return [tuple(o[2:5]) for o in ch_lo], lo, b_lo
+    for _ in range(iters):
+        mid = float(np.sqrt(lo * hi))
+        ch, b = at(mid)
+        if b <= budget:
+            hi, ch_hi, b_hi = mid, ch, b
+        else:
+            lo = mid
+    return [tuple(o[2:5]) for o in ch_hi], hi, b_hi
+
+
 def evaluate(cell_options, choices):
     """(total bytes, total E) of a choice vector."""
     B = E = 0

@@ -217,3 +217,27 @@ def test_argument_checks_before_any_device_work():
     # self-test: unbounded or zero limits, unknown test, too small a workspace
     assert L.jolt_selftest_timeout(0, 0, None, 512, None) == -1
     assert L.jolt_selftest_timeout(3, 1000, None, 512, None) == -1
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_coordinate_allocator_bit_exact_vs_oracle(seed):
+    # the pages' coordinate-wise rank search: host library and oracle agree bit for bit (choices,
+    # bytes) on random tables; small grids keep the pure-Python oracle fast
+    from oracle.alloc import allocate_coord
+    w = get_workload("toy")
+    s = api.make_shape(w)
+    nc = 8
+    nrt, nrd = s.q_cap // 16 + 1, w.d_h // 16 + 1
+    n2, tT, td = make_random_tables(nc, nrt, nrd, 300 + seed)
+    phi = oracle.phi_table(w.d_h, 1 << 12, 1)
+    opts = tables_to_options(n2, tT, td, phi, w)
+    hi = sum(max(o[0] for o in c) for c in opts)
+    for frac in (0.05, 0.2, 0.45, 0.8):
+        budget = int(frac * hi)
+        want, lam, tot_o = allocate_coord(opts, budget)
+        got, tot_g = api.allocate_variant(s, n2, tT, td, phi, budget, api.JOLT_ALLOC_COORD)
+        assert [tuple(c) for c in got] == [tuple(c) for c in want] and tot_g == tot_o
+        # never better than the exact single-multiplier allocation at its own bytes
+        ex, _, tot_e = api.allocate(s, n2, tT, td, phi, budget)
+        from oracle.alloc import evaluate
+        assert evaluate(opts, got)[1] >= evaluate(opts, ex)[1] * (1 - 1e-12) or tot_g > tot_e

@@ -114,3 +114,59 @@ def test_ablation_allocations_are_feasible_and_never_beat_the_joint_optimum(seed
         Bk, Ek = evaluate(opts, ck)
         assert Bk == tk <= budget and Ek >= best * (1 - 1e-12)
         assert evaluate(opts[0::2], ck[0::2])[0] <= budget // 2
+
+
+# ---- the pages' coordinate-wise rank search (a heuristic under the same multiplier) ----------
+
+@pytest.mark.parametrize("seed", range(5))
+def test_coord_never_beats_the_exhaustive_optimum(seed):
+    # Everett's bound: no allocation using at most B bytes has less summed error than the best
+    # one found by brute force within B; the coordinate search must respect it and the budget.
+    from oracle.alloc import allocate_coord
+    opts = small_instance(3, 40 + seed, n_rt=4, n_rd=3)
+    lo = sum(min(o[0] for o in c) for c in opts)
+    hi = sum(max(o[0] for o in c) for c in opts)
+    for frac in np.linspace(0.0, 1.0, 7):
+        budget = int(lo + frac * (hi - lo))
+        ch, lam, total = allocate_coord(opts, budget, iters=80)
+        B, E = evaluate(opts, ch)
+        assert B == total <= budget
+        best = brute_force_allocate(opts, B)
+        assert E >= best[0] * (1 - 1e-12) - 1e-12
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_coord_cell_with_one_feature_rank_is_the_exhaustive_argmin(seed):
+    # with a single nonzero r_d the token-mode move already ranges over every option, so the
+    # search returns the exact minimiser of E + lam * bytes (ties: bytes, r_T, r_d, b)
+    from oracle.alloc import _coord_cell
+    opts = small_instance(1, 60 + seed, n_rt=6, n_rd=2)[0]
+    for lam in (0.0, 1e-9, 1e-6, 1e-4, 1e-2, 1.0, 1e3):
+        got = _coord_cell(opts, lam)
+        want = min(opts, key=lambda o: (o[1] + lam * o[0], o[0], o[2], o[3], o[4]))
+        assert got == want
+
+
+def test_coord_descent_can_stop_short_of_the_optimum():
+    # a hand-built cell (bytes, error) over r_T in {0, 16, 32}, r_d in {0, 16, 32}, b = 0 only
+    # (other b priced out): from full ranks (32, 32) the token move keeps r_T = 32 and the
+    # feature move keeps r_d = 32, although (16, 16) has the smaller E + lam * bytes.
+    lam = 1.0
+    grid = {(0, 0): (0, 100.0), (16, 16): (10, 20.0), (16, 32): (40, 19.0), (32, 16): (40, 19.0),
+            (32, 32): (45, 0.0)}
+    opts = [(B, E, rT, rd, 0) for (rT, rd), (B, E) in grid.items()]
+    from oracle.alloc import _coord_cell
+    got = _coord_cell(opts, lam)
+    assert got[2:4] == (32, 32)                     # stuck: 45 + 0 < 40 + 19 and < 100
+    best = min(opts, key=lambda o: o[1] + lam * o[0])
+    assert best[2:4] == (16, 16) and best[1] + lam * best[0] < got[1] + lam * got[0]
+
+
+def test_coord_infeasible_and_unbounded_budgets():
+    from oracle.alloc import allocate_coord
+    opts = small_instance(2, 3)
+    # the sparsest coordinate choice of every cell is residual-only with b = 0 (zero bytes)
+    ch, lam, total = allocate_coord(opts, 0, iters=40)
+    assert total == 0 and all(c == (0, 0, 0) for c in ch)
+    ch, lam, total = allocate_coord(opts, 10 ** 15, iters=40)
+    assert lam == 1e-30
