@@ -878,10 +878,16 @@ jolt_status analyze_impl(const jolt_shape* shape, const void* k, const void* v, 
             for (int j = (kk - 1) * kRankStep; j < kk * kRankStep; ++j) cum += std::max(0.0, evT[size_t(i) * (exact_path ? p.n : p.l) + j]);
           tail_T_out[size_t(cell) * nrt + kk] = std::max(0.0, n2 - cum);
         }
+        // The eigenvalues of S_d sum to trace(S_d) = ||X||^2. The tensor-core Gram accumulates in
+        // fp32 and comes out short by a near-uniform factor (~2e-5 at T = 128K), so the spectrum is
+        // rescaled to the fp64 norm before the tail is taken.
+        double tr = 0.0;
+        for (int j = 0; j < p.d; ++j) tr += std::max(0.0, evD[size_t(i) * p.d + j]);
+        const double dsc = (tr > 0.0 && n2 > 0.0) ? n2 / tr : 1.0;
         cum = 0.0;
         for (int jj = 0; jj < nrd; ++jj) {
           if (jj > 0)
-            for (int j = (jj - 1) * kRankStep; j < jj * kRankStep; ++j) cum += std::max(0.0, evD[size_t(i) * p.d + j]);
+            for (int j = (jj - 1) * kRankStep; j < jj * kRankStep; ++j) cum += dsc * std::max(0.0, evD[size_t(i) * p.d + j]);
           tail_d_out[size_t(cell) * nrd + jj] = std::max(0.0, n2 - cum);
         }
       }
