@@ -40,7 +40,7 @@ DecodeWs decode_ws_layout(const jolt_shape& s, int Lc, int S) {
   w.P = take(s.keys_pre_rope ? 0 : B * Lc * nq * qc * 4);
   w.Bh = take(s.keys_pre_rope && !tc ? B * Lc * s.n_kv * qc * d * 4 : 0);
   w.part = take(tc ? 0 : B * Lc * nq * size_t(S) * (2 + qc + d) * 4);
-  w.tc = take(tc ? decode_tc_ws_bytes(s, Lc) : 0);
+  w.tc = take(decode_fused_supported(s) ? decode_fused_ws_bytes(s, Lc) : tc ? decode_tc_ws_bytes(s, Lc) : 0);
   w.total = off;
   return w;
 }
@@ -126,7 +126,9 @@ extern "C" jolt_status jolt_decode_attn(const jolt_shape* shape, const jolt_cell
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   // one launch set per batch range whose cells fit the parameter table
-  const int bchunk = std::max(1, kMaxCallCells / (2 * Gc));
+  const bool fused = decode_fused_supported(s);
+  const int bchunk = fused ? std::max(1, std::min(decode_fused_max_cells() / (2 * Gc), 512 / Lc))
+                           : std::max(1, kMaxCallCells / (2 * Gc));
   for (int b0 = 0; b0 < s.batch; b0 += bchunk) {
     const int nb = std::min(bchunk, s.batch - b0);
     DecodeParams pc = p;
@@ -181,7 +183,7 @@ extern "C" jolt_status jolt_decode_attn(const jolt_shape* shape, const jolt_cell
         views[i].r_d = c.r_d;
         views[i].bits = c.b;
       }
-      st_ = launch_decode_tc(pc, views, wsb + wl.tc, s, st);
+      st_ = fused ? launch_decode_fused(pc, views, wsb + wl.tc, s, st) : launch_decode_tc(pc, views, wsb + wl.tc, s, st);
     } else {
       st_ = launch_decode_simt(pc, st);
     }

@@ -30,6 +30,8 @@ struct DecodeParams {
 jolt_status launch_decode_simt(const DecodeParams& p, cudaStream_t st);
 // First prologue kernel of both paths: q_rot = R q, qsum = sum(q_rot) and (non-RoPE keys) P.
 jolt_status launch_decode_prologue_q(const DecodeParams& p, cudaStream_t st);
+// Log-sum-exp merge of p.S split partials (p.ws_part) and the output projection.
+jolt_status launch_decode_merge(const DecodeParams& p, cudaStream_t st);
 
 // One stored cell as device pointers (bf16 factors), for the tensor-core path.
 struct TcCellView {
@@ -47,5 +49,13 @@ size_t decode_tc_ws_bytes(const jolt_shape& s, int Lc);
 // views: (b * Gc + (g - g_first)) * 2 + kv for the call's batch range; tcws: the path's workspace.
 jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uint8_t* tcws,
                              const jolt_shape& s, cudaStream_t st);
+
+// Fused split-T decode for bf16 caches with non-RoPE keys (n_q = 32, n_kv = 4 or 8): one kernel
+// for scores, online softmax and values per (sequence, layer, split), then the split merge.
+bool decode_fused_supported(const jolt_shape& s);
+size_t decode_fused_ws_bytes(const jolt_shape& s, int Lc);
+int decode_fused_max_cells();
+jolt_status launch_decode_fused(const DecodeParams& p, const TcCellView* views, uint8_t* ws,
+                                const jolt_shape& s, cudaStream_t st);
 
 }  // namespace jolt

@@ -1,0 +1,885 @@
+// Fused split-T decode attention over the stored factors: bf16 caches, keys stored after RoPE
+// (no per-token rotation), d_h = 128, 32 query heads over 4 or 8 KV heads.
+//
+// One CTA per (sequence, layer, token split) walks its 128-token tiles once and reads every byte
+// of the layer's compressed cache it needs exactly once from HBM (the group's U_T tiles are shared
+// through L2 by the CTAs of the group's layers, which run side by side):
+//   scores   s[t][j] = U_T^K[t] . P[:, j] + scale_t (codes^K_t . R q_j) + zero_t sum(R q_j), with
+//            P = G^K (U_d^K^T q) ("A JoLT for the KV cache", §4.5: attention evaluated directly
+//            over the stored factors; §3: the residual stored after a seeded rotation R)
+//   softmax  online, per query head, in registers (exp2 domain; the reference maximum moves only
+//            when a tile exceeds it by more than 2^8, so rescaling the accumulators is rare)
+//   values   W[r][j] += sum_t U_T^V[t][r] p~[t][j] and acc[d][j] += sum_t p~[t][j] deq(codes^V_t)[d]
+//   partials (m, l, W, acc) per split go to the workspace; k_decode_merge combines the splits and
+//            applies U_d^V G^V^T and the inverse rotation.
+// Where each contraction runs:
+//   * U_T^K P (M = 128 tokens, N = 64: the 32 query heads' P as bf16 hi + lo columns, K = r_T) and
+//     W (M = 128 rank rows per chunk, N = 32 heads, K = tokens; U_T^V read MN-major, P~ K-major) on
+//     tcgen05 with TMEM accumulators, operands staged by TMA;
+//   * both residual contractions (codes . R q and P~-weighted codes) on mma.sync m16n8k16 with
+//     the f16 operands built in registers straight from the packed codes in shared memory (each
+//     b-bit field becomes an exact f16 integer with one mask-and-or and one add): the codes are
+//     never expanded to 16 bits in memory, which would cost four times their size in shared-memory
+//     traffic per contraction.
+// Warp roles (320 threads): 0 TMA producer, 1 MMA issuer (owns TMEM), 2-5 score warps (thread =
+// token of the tile for the softmax; the same warps run the key-residual MMAs for their 32 tokens),
+// 6-9 value warps (value-residual MMAs, 32 features each).
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <type_traits>
+#include <vector>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "gemm_tc.cuh"
+#include "sm100.cuh"
+#include "stats.h"
+
+namespace jolt {
+
+namespace {
+
+constexpr int kD = 128;           // head dimension
+constexpr int kBM = 128;          // tokens per tile
+constexpr int kBK = 64;           // rank chunk of the score MMA
+constexpr int kNQ = 32;           // query heads per layer this kernel serves
+constexpr int kMaxFusedCells = 64;   // cells one launch references (tensor-map table)
+constexpr int kMaxFusedRows = 512;   // (sequence, layer) rows one launch serves
+constexpr int kKStages = 2, kVStages = 3, kCStages = 2;
+constexpr int kKStageBytes = kBM * kBK * 2 + 2 * kNQ * kBK * 2;  // U_T^K chunk + P hi/lo chunk
+constexpr int kVStageBytes = 2 * 64 * 64 * 2;                    // U_T^V: 128 ranks x 64 tokens
+constexpr int kCStageBytes = 16384;                              // codes of 8/b heads x 128 tokens
+constexpr int kPtBytes = kNQ * kBM * 2;                          // P~ (bf16, K-major, 32 rows)
+constexpr int kWbBytes = kNQ * 256;                              // value weights (f16 fragments)
+constexpr int kScrStride = kNQ + 4;                              // floats per token row of the exchange
+constexpr int kScrBytes = 4 * 32 * kScrStride * 4;
+constexpr int kQfBytes = kNQ * 256;                              // query fragments (f16)
+
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kKStages * kKStageBytes;
+constexpr int kOffPt = kOffV + kVStages * kVStageBytes;
+constexpr int kOffCK = kOffPt + 2 * kPtBytes;
+constexpr int kOffCV = kOffCK + kCStages * kCStageBytes;
+constexpr int kOffWb = kOffCV + kCStages * kCStageBytes;
+constexpr int kOffScr = kOffWb + 2 * kWbBytes;
+constexpr int kOffQf = kOffScr + kScrBytes;
+constexpr int kOffRed = kOffQf + kQfBytes;          // [2][4][32] floats
+constexpr int kOffAlpha = kOffRed + 2 * 4 * 32 * 4; // [2][64] floats: alpha[32], flag
+constexpr int kOffFin = kOffAlpha + 2 * 64 * 4;     // [4][32] float2
+constexpr int kOffZf = kOffFin + 4 * 32 * 8;        // [32]
+constexpr int kOffQs = kOffZf + 32 * 4;             // [32]
+constexpr int kOffBars = kOffQs + 32 * 4;
+constexpr int kNumBars = 32;
+constexpr int kSmemUsed = kOffBars + kNumBars * 8 + 16;
+constexpr int kSmem = kSmemUsed + 1024;             // 1024-byte alignment of the swizzled tiles
+static_assert(kSmem <= 232448, "fused decode shared memory");
+static_assert(kOffV % 1024 == 0 && kOffPt % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.f;  // log2 units: p~ <= 2^8 between rescales
+
+struct FusedCell {
+  const uint8_t* codes;  // [L_g][n_kv][T][16 b] or null
+  const __half2* sz;     // [L_g][n_kv][T] or null
+  int r_T, b;
+};
+
+struct FusedMaps {
+  CUtensorMap p;                      // P hi/lo [B*Lc][2*32][q_cap] bf16, K-major, box 64 x 64
+  CUtensorMap ut[kMaxFusedCells];     // key cells: U_T [T][r_T] K-major box 64 x 128; value cells: MN-major box 64 x 64
+};
+
+struct FusedArgs {
+  int T, nt, tps, S, Lc, Lg, layer_begin, g_first, Gc, n_kv, gq, q_cap;
+  float attn_scale;
+  const float* qrot;   // [B][Lc][32][128] of this launch set
+  const float* qsum;   // [B][Lc][32]
+  float* part;         // [B][Lc][32][S][2 + q_cap + 128]
+  int32_t* err;
+  FusedCell cells[kMaxFusedCells];  // (b * Gc + g - g_first) * 2 + kv
+};
+
+__device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// b-bit code fields of a word as exact f16 pairs. The mask-and-or puts each field into the
+// mantissa of 1024 (f16 0x6400), scaled by 2^shift; one fused multiply-add removes both.
+__device__ __forceinline__ uint32_t f16pair_field(uint32_t x, uint32_t mask, float inv, float off) {
+  const uint32_t v = (x & mask) | 0x64006400u;
+  __half2 h = *reinterpret_cast<const __half2*>(&v);
+  h = __hfma2(h, __float2half2_rn(inv), __float2half2_rn(off));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// 4-bit fields at bits 0-3 / 16-19 (lo) or 4-7 / 20-23 (hi)
+__device__ __forceinline__ uint32_t nib_lo(uint32_t x) { return f16pair_field(x, 0x000F000Fu, 1.f, -1024.f); }
+__device__ __forceinline__ uint32_t nib_hi(uint32_t x) { return f16pair_field(x, 0x00F000F0u, 0.0625f, -64.f); }
+// 2-bit fields at bit 2s / 16 + 2s
+__device__ __forceinline__ uint32_t crumb(uint32_t x, int s) {
+  switch (s) {
+    case 0: return f16pair_field(x, 0x00030003u, 1.f, -1024.f);
+    case 1: return f16pair_field(x, 0x000C000Cu, 0.25f, -256.f);
+    case 2: return f16pair_field(x, 0x00300030u, 0.0625f, -64.f);
+    default: return f16pair_field(x, 0x00C000C0u, 0.015625f, -16.f);
+  }
+}
+// bytes i and k of x -> f16 pair (x.byte_i, x.byte_k)
+__device__ __forceinline__ uint32_t byte_pair(uint32_t x, uint32_t sel) {
+  const uint32_t v = __byte_perm(x, 0x64646464u, sel);
+  __half2 h = *reinterpret_cast<const __half2*>(&v);
+  h = __hsub2(h, __float2half2_rn(1024.f));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Within a lane's 32-code segment of a key-residual row, pair p (16 pairs, in the order the
+// conversion produces them) holds the codes at offsets (lo, lo + gap).
+__device__ __forceinline__ int pair_lo(int bits, int p) {
+  return bits == 4 ? 8 * (p >> 2) + (p & 3) : bits == 2 ? 16 * (p >> 3) + (p & 7) : 4 * (p >> 1) + (p & 1);
+}
+__device__ __forceinline__ int pair_gap(int bits) { return bits == 4 ? 4 : bits == 2 ? 8 : 2; }
+
+// Warp reduce-scatter over 32 values: afterwards v[0] of lane l combines value index l of all lanes.
+template <bool MAX>
+__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool up = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float keep = up ? v[i + w] : v[i];
+      const float send = up ? v[i] : v[i + w];
+      const float got = __shfl_xor_sync(0xffffffffu, send, w);
+      v[i] = MAX ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  return v[0];
+}
+
+// Key residual of KV head h (codes in slot k of the stage at cs) for the 32 tokens of quarter q:
+// scr[token][h g_q + j] = scale (codes . R q_j) + zero sum(R q_j). zkh: lane i holds the
+// (scale, zero) pair of token 32 q + i.
+template <int BITS, int GQ>
+__device__ __forceinline__ void kres_head(const uint8_t* cs, int k, int h, int q, int lane, const uint2* qf,
+                                          const float* qs, float* scr, uint32_t zkh) {
+  constexpr int RB = 16 * BITS;
+  const int gr = lane >> 2, m4 = lane & 3;
+#pragma unroll
+  for (int mb = 0; mb < 2; ++mb) {
+    const int rA = 32 * q + 16 * mb + gr;  // tile rows of fragment rows g and g + 8
+    const uint8_t* rowA = cs + (k * kBM + rA) * RB;
+    const uint8_t* rowB = rowA + 8 * RB;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t xa[8], xb[8];
+    if (BITS == 4) {
+      const uint4 u = *reinterpret_cast<const uint4*>(rowA + 16 * m4), v = *reinterpret_cast<const uint4*>(rowB + 16 * m4);
+      xa[0] = u.x; xa[1] = u.y; xa[2] = u.z; xa[3] = u.w;
+      xb[0] = v.x; xb[1] = v.y; xb[2] = v.z; xb[3] = v.w;
+    } else if (BITS == 2) {
+      const uint2 u = *reinterpret_cast<const uint2*>(rowA + 8 * m4), v = *reinterpret_cast<const uint2*>(rowB + 8 * m4);
+      xa[0] = u.x; xa[1] = u.y;
+      xb[0] = v.x; xb[1] = v.y;
+    } else {
+      const uint4 u0 = *reinterpret_cast<const uint4*>(rowA + 32 * m4), u1 = *reinterpret_cast<const uint4*>(rowA + 32 * m4 + 16);
+      const uint4 v0 = *reinterpret_cast<const uint4*>(rowB + 32 * m4), v1 = *reinterpret_cast<const uint4*>(rowB + 32 * m4 + 16);
+      xa[0] = u0.x; xa[1] = u0.y; xa[2] = u0.z; xa[3] = u0.w; xa[4] = u1.x; xa[5] = u1.y; xa[6] = u1.z; xa[7] = u1.w;
+      xb[0] = v0.x; xb[1] = v0.y; xb[2] = v0.z; xb[3] = v0.w; xb[4] = v1.x; xb[5] = v1.y; xb[6] = v1.z; xb[7] = v1.w;
+    }
+#pragma unroll
+    for (int kc = 0; kc < 8; ++kc) {
+      uint32_t af[4];
+      if (BITS == 4) {
+        const uint32_t wa = xa[kc >> 1] >> ((kc & 1) * 8), wb = xb[kc >> 1] >> ((kc & 1) * 8);
+        af[0] = nib_lo(wa); af[2] = nib_hi(wa);
+        af[1] = nib_lo(wb); af[3] = nib_hi(wb);
+      } else if (BITS == 2) {
+        const int sft = ((kc & 3) >= 2) ? 8 : 0, s0 = (2 * (kc & 3)) & 3;
+        const uint32_t wa = xa[kc >> 2] >> sft, wb = xb[kc >> 2] >> sft;
+        af[0] = crumb(wa, s0); af[2] = crumb(wa, s0 + 1);
+        af[1] = crumb(wb, s0); af[3] = crumb(wb, s0 + 1);
+      } else {
+        af[0] = byte_pair(xa[kc], 0x4240); af[2] = byte_pair(xa[kc], 0x4341);
+        af[1] = byte_pair(xb[kc], 0x4240); af[3] = byte_pair(xb[kc], 0x4341);
+      }
+      uint2 bq = make_uint2(0u, 0u);
+      if (gr < GQ) bq = qf[((h * 8 + kc) * GQ + gr) * 4 + m4];
+      mma_f16(acc, af, bq.x, bq.y);
+    }
+    // rows g (tile row rA) and g + 8, query heads 2 m4, 2 m4 + 1 of KV head h
+    const uint32_t zA = __shfl_sync(0xffffffffu, zkh, 16 * mb + gr);
+    const uint32_t zB = __shfl_sync(0xffffffffu, zkh, 16 * mb + gr + 8);
+    const float2 fA = __half22float2(*reinterpret_cast<const __half2*>(&zA));
+    const float2 fB = __half22float2(*reinterpret_cast<const __half2*>(&zB));
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int j = 2 * m4 + e;
+      if (j < GQ) {
+        const float qsj = qs[h * GQ + j];
+        scr[(16 * mb + gr) * kScrStride + h * GQ + j] = fA.x * acc[e] + fA.y * qsj;
+        scr[(16 * mb + gr + 8) * kScrStride + h * GQ + j] = fB.x * acc[2 + e] + fB.y * qsj;
+      }
+    }
+  }
+}
+
+// Value residual of KV head h (codes in slot k of the stage at cs) for one tile: eight chunks of 16
+// tokens, feature pairs (d, d+1) and (d+2, d+3) with d = 16 g + 4 vw; ac[0], ac[1] the fragments.
+template <int BITS, int GQ>
+__device__ __forceinline__ void vres_head(float (&ac)[2][4], const uint8_t* cs, int k, const uint2* wbp, int h,
+                                          int vw, int lane) {
+  constexpr int RB = 16 * BITS;
+  const int gr = lane >> 2, m4 = lane & 3;
+  const uint8_t* base = cs + k * kBM * RB;
+#pragma unroll
+  for (int kc = 0; kc < 8; ++kc) {
+    const int r0 = 16 * kc + m4;  // tile rows of tokens e = 0..3: r0 + 4 e
+    uint32_t f0[4], f1[4];
+    if (BITS == 4) {
+      const uint8_t* p = base + 8 * gr + 2 * vw;
+      const uint32_t xA = *reinterpret_cast<const uint16_t*>(p + (r0 + 0) * RB);
+      const uint32_t xB = *reinterpret_cast<const uint16_t*>(p + (r0 + 4) * RB);
+      const uint32_t xC = *reinterpret_cast<const uint16_t*>(p + (r0 + 8) * RB);
+      const uint32_t xD = *reinterpret_cast<const uint16_t*>(p + (r0 + 12) * RB);
+      const uint32_t u = xA | (xB << 16), w = xC | (xD << 16);
+      f0[0] = nib_lo(u); f0[1] = nib_hi(u); f0[2] = nib_lo(w); f0[3] = nib_hi(w);
+      f1[0] = nib_lo(u >> 8); f1[1] = nib_hi(u >> 8); f1[2] = nib_lo(w >> 8); f1[3] = nib_hi(w >> 8);
+    } else if (BITS == 2) {
+      const uint8_t* p = base + 4 * gr + vw;
+      const uint32_t xA = p[(r0 + 0) * RB], xB = p[(r0 + 4) * RB];
+      const uint32_t xC = p[(r0 + 8) * RB], xD = p[(r0 + 12) * RB];
+      const uint32_t u = xA | (xB << 16), w = xC | (xD << 16);
+      f0[0] = crumb(u, 0); f0[1] = crumb(u, 1); f0[2] = crumb(w, 0); f0[3] = crumb(w, 1);
+      f1[0] = crumb(u, 2); f1[1] = crumb(u, 3); f1[2] = crumb(w, 2); f1[3] = crumb(w, 3);
+    } else {
+      const uint8_t* p = base + 16 * gr + 4 * vw;
+      const uint32_t xA = *reinterpret_cast<const uint32_t*>(p + (r0 + 0) * RB);
+      const uint32_t xB = *reinterpret_cast<const uint32_t*>(p + (r0 + 4) * RB);
+      const uint32_t xC = *reinterpret_cast<const uint32_t*>(p + (r0 + 8) * RB);
+      const uint32_t xD = *reinterpret_cast<const uint32_t*>(p + (r0 + 12) * RB);
+      const uint32_t u0 = __byte_perm(xA, xB, 0x5140), u1 = __byte_perm(xA, xB, 0x7362);
+      const uint32_t w0 = __byte_perm(xC, xD, 0x5140), w1 = __byte_perm(xC, xD, 0x7362);
+      f0[0] = byte_pair(u0, 0x4140); f0[1] = byte_pair(u0, 0x4342);
+      f0[2] = byte_pair(w0, 0x4140); f0[3] = byte_pair(w0, 0x4342);
+      f1[0] = byte_pair(u1, 0x4140); f1[1] = byte_pair(u1, 0x4342);
+      f1[2] = byte_pair(w1, 0x4140); f1[3] = byte_pair(w1, 0x4342);
+    }
+    uint2 bw = make_uint2(0u, 0u);
+    if (gr < GQ) bw = wbp[((h * 8 + kc) * 4 + m4) * GQ + gr];
+    mma_f16(ac[0], f0, bw.x, bw.y);
+    mma_f16(ac[1], f1, bw.x, bw.y);
+  }
+}
+
+template <int GQ>
+__global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_constant__ FusedMaps maps, const FusedArgs a) {
+  constexpr int NKV = kNQ / GQ;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = sm100::smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  const uint32_t bar0 = sm100::smem_u32(bars);
+  auto BK_FULL = [&](int s) { return bar0 + 8u * (0 + s); };
+  auto BK_EMPTY = [&](int s) { return bar0 + 8u * (2 + s); };
+  auto BV_FULL = [&](int s) { return bar0 + 8u * (4 + s); };
+  auto BV_EMPTY = [&](int s) { return bar0 + 8u * (7 + s); };
+  auto BCK_FULL = [&](int s) { return bar0 + 8u * (10 + s); };
+  auto BCK_EMPTY = [&](int s) { return bar0 + 8u * (12 + s); };
+  auto BCV_FULL = [&](int s) { return bar0 + 8u * (14 + s); };
+  auto BCV_EMPTY = [&](int s) { return bar0 + 8u * (16 + s); };
+  auto BS_FULL = [&](int s) { return bar0 + 8u * (18 + s); };
+  auto BS_EMPTY = [&](int s) { return bar0 + 8u * (20 + s); };
+  auto BP_FULL = [&](int s) { return bar0 + 8u * (22 + s); };
+  auto BP_EMPTY = [&](int s) { return bar0 + 8u * (24 + s); };
+  auto BW_DONE = [&](int s) { return bar0 + 8u * (26 + s); };
+  const uint32_t BDRAIN = bar0 + 8u * 28;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // this CTA's (sequence, split, layer): layers fastest, so the CTAs of one layer group that share
+  // U_T tiles run side by side
+  const int li = blockIdx.x % a.Lc;
+  const int sp = (blockIdx.x / a.Lc) % a.S;
+  const int bi = blockIdx.x / (a.Lc * a.S);
+  const int layer = a.layer_begin + li, g = layer / a.Lg, ll = layer % a.Lg;
+  const int ci = (bi * a.Gc + (g - a.g_first)) * 2;
+  const FusedCell ck = a.cells[ci], cv = a.cells[ci + 1];
+  const int tile0 = sp * a.tps;
+  const int ntl = max(0, min(a.nt, tile0 + a.tps) - tile0);  // tiles of this CTA
+  const int bl = bi * a.Lc + li;                              // (sequence, layer) row of the call
+  const int nkb = ck.r_T > 0 ? (ck.r_T + kBK - 1) / kBK : 0;
+  const int nmc = cv.r_T > 0 ? (cv.r_T + 127) / 128 : 0;
+  const int bK = ck.b, bV = cv.b;
+  const int rbK = 16 * bK, rbV = 16 * bV;                    // bytes per code row
+  const int hpsK = bK ? 8 / bK : 1, hpsV = bV ? 8 / bV : 1;  // heads per code stage
+  const int njK = bK ? (NKV + hpsK - 1) / hpsK : 0;
+  const int njV = bV ? (NKV + hpsV - 1) / hpsV : 0;
+  const size_t prow = size_t(2 + a.q_cap + kD);
+
+  if (threadIdx.x == 0) {
+    // arrival counts: TMA / MMA-commit barriers 1; code-stage releases and score-warp hand-offs 4
+    // (one per consuming warp); a P~ buffer is free after the value products (1 commit) and the
+    // four value warps
+    for (int i = 0; i < 29; ++i) {
+      uint32_t cnt = 1;
+      if ((i >= 12 && i < 14) || (i >= 16 && i < 18) || (i >= 20 && i < 24)) cnt = 4;
+      if (i >= 24 && i < 26) cnt = 5;
+      sm100::mbar_init(bar0 + 8u * i, cnt);
+    }
+    sm100::fence_mbar_init();
+    sm100::prefetch_tmap(&maps.p);
+    if (nkb) sm100::prefetch_tmap(&maps.ut[ci]);
+    if (nmc) sm100::prefetch_tmap(&maps.ut[ci + 1]);
+  }
+  if (warp == 1) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), kTmemCols);
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tW = tmem + 2 * 2 * kNQ;  // S: two buffers of 64 columns; W after them
+
+  if (warp == 0) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      int kit = 0, vit = 0, ckit = 0, cvit = 0;
+      bool ok = true;
+      const uint8_t* codesK = ck.codes ? ck.codes + int64_t(ll) * NKV * a.T * rbK : nullptr;
+      const uint8_t* codesV = cv.codes ? cv.codes + int64_t(ll) * NKV * a.T * rbV : nullptr;
+      auto issue_codes = [&](const uint8_t* codes, int rb, int hps, int nj, int t0, int nv, int& cit, bool kside) {
+        for (int jb = 0; jb < nj && ok; ++jb, ++cit) {
+          const int s = cit % kCStages;
+          const uint32_t full = kside ? BCK_FULL(s) : BCV_FULL(s);
+          const uint32_t empty = kside ? BCK_EMPTY(s) : BCV_EMPTY(s);
+          if (!(ok = sm100::mbar_wait(empty, ((cit / kCStages) & 1) ^ 1, a.err))) break;
+          const int h0 = jb * hps, nh = min(hps, NKV - h0);
+          sm100::mbar_expect_tx(full, uint32_t(nh * nv * rb));
+          const uint32_t dst = sb + (kside ? kOffCK : kOffCV) + s * kCStageBytes;
+          for (int k = 0; k < nh; ++k)
+            sm100::bulk_load(dst + k * kBM * rb, codes + (int64_t(h0 + k) * a.T + t0) * rb, uint32_t(nv * rb), full);
+        }
+      };
+      auto issue_v = [&](int it) {
+        const int t0 = (tile0 + it) * kBM, nv = min(kBM, a.T - t0);
+        for (int mc = 0; mc < nmc && ok; ++mc)
+          for (int h2 = 0; h2 < 2 && ok; ++h2, ++vit) {
+            const int s = vit % kVStages;
+            if (!(ok = sm100::mbar_wait(BV_EMPTY(s), ((vit / kVStages) & 1) ^ 1, a.err))) break;
+            sm100::mbar_expect_tx(BV_FULL(s), kVStageBytes);
+            const uint32_t dst = sb + kOffV + s * kVStageBytes;
+            sm100::tma_load_3d(dst, &maps.ut[ci + 1], BV_FULL(s), mc * 128, t0 + 64 * h2, 0);
+            sm100::tma_load_3d(dst + 8192, &maps.ut[ci + 1], BV_FULL(s), mc * 128 + 64, t0 + 64 * h2, 0);
+          }
+        if (ok) issue_codes(codesV, rbV, hpsV, njV, t0, nv, cvit, false);
+      };
+      for (int it = 0; it < ntl && ok; ++it) {
+        const int t0 = (tile0 + it) * kBM, nv = min(kBM, a.T - t0);
+        for (int kb = 0; kb < nkb && ok; ++kb, ++kit) {
+          const int s = kit % kKStages;
+          if (!(ok = sm100::mbar_wait(BK_EMPTY(s), ((kit / kKStages) & 1) ^ 1, a.err))) break;
+          sm100::mbar_expect_tx(BK_FULL(s), kKStageBytes);
+          const uint32_t dst = sb + kOffK + s * kKStageBytes;
+          sm100::tma_load_3d(dst, &maps.ut[ci], BK_FULL(s), kb * kBK, t0, 0);
+          sm100::tma_load_3d(dst + kBM * kBK * 2, &maps.p, BK_FULL(s), kb * kBK, 0, bl);
+        }
+        if (ok) issue_codes(codesK, rbK, hpsK, njK, t0, nv, ckit, true);
+        if (it >= 1 && ok) issue_v(it - 1);
+      }
+      if (ntl > 0 && ok) issue_v(ntl - 1);
+      // the copies still in flight complete before the block may exit
+      for (int i = max(0, kit - kKStages); i < kit; ++i) sm100::mbar_wait(BK_FULL(i % kKStages), (i / kKStages) & 1, a.err);
+      for (int i = max(0, vit - kVStages); i < vit; ++i) sm100::mbar_wait(BV_FULL(i % kVStages), (i / kVStages) & 1, a.err);
+      for (int i = max(0, ckit - kCStages); i < ckit; ++i) sm100::mbar_wait(BCK_FULL(i % kCStages), (i / kCStages) & 1, a.err);
+      for (int i = max(0, cvit - kCStages); i < cvit; ++i) sm100::mbar_wait(BCV_FULL(i % kCStages), (i / kCStages) & 1, a.err);
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      constexpr uint32_t idK = sm100::idesc_bf16_f32(kBM, 2 * kNQ, 0, 0);
+      constexpr uint32_t idW = sm100::idesc_bf16_f32(128, kNQ, 1, 0);
+      int kit = 0, vit = 0;
+      bool ok = true;
+      auto issue_w = [&](int it) {
+        if (!(ok = sm100::mbar_wait(BP_FULL(it & 1), (it >> 1) & 1, a.err))) return;
+        sm100::tc_fence_after();
+        const uint32_t pt = sb + kOffPt + (it & 1) * kPtBytes;
+        for (int mc = 0; mc < nmc && ok; ++mc)
+          for (int h2 = 0; h2 < 2 && ok; ++h2, ++vit) {
+            const int s = vit % kVStages;
+            if (!(ok = sm100::mbar_wait(BV_FULL(s), (vit / kVStages) & 1, a.err))) break;
+            sm100::tc_fence_after();
+            const uint32_t va = sb + kOffV + s * kVStageBytes;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sm100::smem_desc_sw128(va + kk * 2048, 8192, 1024);
+              const uint64_t bd = sm100::smem_desc_sw128(pt + h2 * (kNQ * 128) + kk * 32, 16, 1024);
+              sm100::mma_bf16(tW + mc * kNQ, ad, bd, idW, (it > 0 || h2 > 0 || kk > 0) ? 1u : 0u);
+            }
+            sm100::mma_commit(BV_EMPTY(s));
+          }
+        sm100::mma_commit(BW_DONE(it & 1));
+        sm100::mma_commit(BP_EMPTY(it & 1));
+      };
+      for (int it = 0; it < ntl && ok; ++it) {
+        if (nkb) {
+          if (!(ok = sm100::mbar_wait(BS_EMPTY(it & 1), ((it >> 1) & 1) ^ 1, a.err))) break;
+          sm100::tc_fence_after();
+          const uint32_t dt = tS + (it & 1) * 2 * kNQ;
+          for (int kb = 0; kb < nkb && ok; ++kb, ++kit) {
+            const int s = kit % kKStages;
+            if (!(ok = sm100::mbar_wait(BK_FULL(s), (kit / kKStages) & 1, a.err))) break;
+            sm100::tc_fence_after();
+            const uint32_t ka = sb + kOffK + s * kKStageBytes;
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = sm100::smem_desc_sw128(ka + kk * 32, 16, 1024);
+              const uint64_t bd = sm100::smem_desc_sw128(ka + kBM * kBK * 2 + kk * 32, 16, 1024);
+              sm100::mma_bf16(dt, ad, bd, idK, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
+            sm100::mma_commit(BK_EMPTY(s));
+          }
+          if (ok) sm100::mma_commit(BS_FULL(it & 1));
+        }
+        if (it >= 1 && ok) issue_w(it - 1);
+      }
+      if (ntl > 0 && ok) issue_w(ntl - 1);
+      sm100::mma_commit(BDRAIN);
+      sm100::mbar_wait(BDRAIN, 0, a.err);
+    }
+  } else if (warp < 6) {
+    // ================= score warps: key residual, scores, online softmax =================
+    const int q = warp & 3;            // TMEM lane quarter = tokens 32q .. 32q+31 of the tile
+    const int gr = lane >> 2, m4 = lane & 3;
+    const int tid = threadIdx.x - 64;  // 0..127
+    float* scr = reinterpret_cast<float*>(smem + kOffScr) + q * 32 * kScrStride;
+    float* red = reinterpret_cast<float*>(smem + kOffRed);
+    float* alph = reinterpret_cast<float*>(smem + kOffAlpha);
+    float2* fin = reinterpret_cast<float2*>(smem + kOffFin);
+    float* zf = reinterpret_cast<float*>(smem + kOffZf);
+    float* qs = reinterpret_cast<float*>(smem + kOffQs);
+    uint2* qf = reinterpret_cast<uint2*>(smem + kOffQf);
+    // query-side operands of the key residual: f16 fragments of R q in the pair order of this
+    // cell's code width ([h][chunk][g < g_q][m]), and sum(R q)
+    const float* qr = a.qrot + int64_t(bl) * kNQ * kD;
+    if (bK) {
+      const int gap = pair_gap(bK);
+      for (int e = tid; e < NKV * 8 * GQ * 4; e += 128) {
+        const int mm = e & 3, gg = (e >> 2) % GQ, kc = (e / (4 * GQ)) & 7, h = e / (32 * GQ);
+        const float* qj = qr + (h * GQ + gg) * kD + 32 * mm;
+        const int p0 = pair_lo(bK, 2 * kc), p1 = pair_lo(bK, 2 * kc + 1);
+        const __half2 w0 = __floats2half2_rn(qj[p0], qj[p0 + gap]);
+        const __half2 w1 = __floats2half2_rn(qj[p1], qj[p1 + gap]);
+        qf[e] = make_uint2(*reinterpret_cast<const uint32_t*>(&w0), *reinterpret_cast<const uint32_t*>(&w1));
+      }
+    }
+    if (tid < kNQ) qs[tid] = a.qsum[int64_t(bl) * kNQ + tid];
+    named_bar(1, 128);
+    float mref = -INFINITY, ell = 0.f, zac = 0.f;  // of query head `lane`
+    int ckit = 0;
+    bool ok = true;
+    const __half2* szK = ck.sz ? ck.sz + int64_t(ll) * NKV * a.T : nullptr;
+    const __half2* szV = cv.sz ? cv.sz + int64_t(ll) * NKV * a.T : nullptr;
+
+    for (int it = 0; it < ntl; ++it) {
+      __syncwarp();  // every lane has read its row of the exchange buffer before it is rewritten
+      const int t0 = (tile0 + it) * kBM;
+      const int tl = 32 * q + lane, t = t0 + tl;
+      const bool valid = t < a.T;
+      // this token's scale / zero pairs (the key ones reach the MMA lanes by shuffles)
+      uint32_t zk[NKV], zv[NKV];
+#pragma unroll
+      for (int h = 0; h < NKV; ++h) {
+        zk[h] = (bK && valid) ? __ldg(reinterpret_cast<const uint32_t*>(szK + int64_t(h) * a.T + t)) : 0u;
+        zv[h] = (bV && valid) ? __ldg(reinterpret_cast<const uint32_t*>(szV + int64_t(h) * a.T + t)) : 0u;
+      }
+      // ---- key residual: jobs of 8 / b heads per code stage ----
+      if (bK) {
+        const int hps = 8 / bK;
+        int s = 0;
+#pragma unroll
+        for (int h = 0; h < NKV; ++h) {
+          const int k = h % hps;
+          if (k == 0) {
+            s = ckit % kCStages;
+            if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BCK_FULL(s), (ckit / kCStages) & 1, a.err));
+          }
+          const uint8_t* cs = smem + kOffCK + s * kCStageBytes;
+          if (bK == 4) kres_head<4, GQ>(cs, k, h, q, lane, qf, qs, scr, zk[h]);
+          else if (bK == 2) kres_head<2, GQ>(cs, k, h, q, lane, qf, qs, scr, zk[h]);
+          else kres_head<8, GQ>(cs, k, h, q, lane, qf, qs, scr, zk[h]);
+          if (k == hps - 1 || h == NKV - 1) {
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(BCK_EMPTY(s));
+            ++ckit;
+          }
+        }
+      }
+      // ---- scores of token t for the 32 query heads ----
+      float sv[kNQ];
+      if (nkb) {
+        if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BS_FULL(it & 1), (it >> 1) & 1, a.err));
+        sm100::tc_fence_after();
+        uint32_t hi[32], lo[32];
+        const uint32_t ta = tS + (it & 1) * 2 * kNQ + (uint32_t(32 * q) << 16);
+        sm100::tmem_ld32(ta, hi);
+        sm100::tmem_ld32(ta + kNQ, lo);
+        sm100::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < kNQ; ++j) sv[j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
+        sm100::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(BS_EMPTY(it & 1));
+      } else {
+#pragma unroll
+        for (int j = 0; j < kNQ; ++j) sv[j] = 0.f;
+      }
+      __syncwarp();
+      const float sc2 = a.attn_scale * kLog2e;
+#pragma unroll
+      for (int j = 0; j < kNQ; ++j) {
+        const float r = bK ? scr[lane * kScrStride + j] : 0.f;
+        sv[j] = valid ? (sv[j] + r) * sc2 : -INFINITY;
+      }
+      // ---- tile maximum per query head; the reference maximum moves only by more than 2^8 ----
+      float tmp[kNQ];
+#pragma unroll
+      for (int j = 0; j < kNQ; ++j) tmp[j] = sv[j];
+      const float wmax = reduce_scatter32<true>(tmp, lane);
+      float* rd = red + (it & 1) * 128;
+      rd[q * 32 + lane] = wmax;
+      named_bar(1, 128);
+      const float tmax = fmaxf(fmaxf(rd[lane], rd[32 + lane]), fmaxf(rd[64 + lane], rd[96 + lane]));
+      const float mnew = (tmax > mref + kRescaleThreshold || mref == -INFINITY) ? fmaxf(tmax, mref) : mref;
+      const float al = (mnew == mref) ? 1.f : exp2f(mref - mnew);
+      const bool resc = __any_sync(0xffffffffu, mnew != mref);
+      mref = mnew;
+      ell *= al;
+      zac *= al;
+      // the P~ / weight buffer of this tile is free once tile it - 2's value products are done
+      if (it >= 2 && ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BP_EMPTY(it & 1), ((it >> 1) & 1) ^ 1, a.err));
+      if (resc && it > 0 && nmc > 0) {
+        // W (TMEM) holds tiles 0 .. it-1 at the old reference: rescale its columns once the last of
+        // those products is done
+        if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BW_DONE((it - 1) & 1), ((it - 1) >> 1) & 1, a.err));
+        sm100::tc_fence_after();
+        for (int mc = 0; mc < nmc; ++mc) {
+          uint32_t w[32];
+          const uint32_t ta = tW + mc * kNQ + (uint32_t(32 * q) << 16);
+          sm100::tmem_ld32(ta, w);
+          sm100::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < kNQ; ++j) w[j] = __float_as_uint(__uint_as_float(w[j]) * __shfl_sync(0xffffffffu, al, j));
+          sm100::tmem_st32(ta, w);
+        }
+        sm100::tmem_st_wait();
+        sm100::tc_fence_before();
+      }
+      // ---- probabilities: P~ (bf16) for the U_T^V product, f16 weights for the value residual ----
+      uint8_t* pt = smem + kOffPt + (it & 1) * kPtBytes;
+      uint8_t* wbp = smem + kOffWb + (it & 1) * kWbBytes;
+      float zsum[kNQ];
+      const int kcT = tl >> 4, rT = tl & 15, eT = rT >> 2, mT = rT & 3;
+      const int pc = tl >> 6, pu = (tl & 63) >> 3;
+#pragma unroll
+      for (int j = 0; j < kNQ; ++j) {
+        const float mj = __shfl_sync(0xffffffffu, mref, j);
+        const __nv_bfloat16 pb = __float2bfloat16_rn(valid ? exp2f(sv[j] - mj) : 0.f);
+        const float pf = __bfloat162float(pb);
+        tmp[j] = pf;
+        // K-major, 128-byte swizzle: row j, tokens in two 64-token chunks
+        *reinterpret_cast<__nv_bfloat16*>(pt + pc * (kNQ * 128) + j * 128 + ((pu ^ (j & 7)) << 4) + (tl & 7) * 2) = pb;
+        const int h = j / GQ, gg = j % GQ;
+        float zz = 0.f;
+        if (bV) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&zv[h]));
+          zz = f.y * pf;
+          const __half w = __float2half_rn(pf * f.x * 0.00390625f);
+          *reinterpret_cast<__half*>(wbp + ((((h * 8 + kcT) * 4 + mT) * GQ + gg) * 2 + (eT >> 1)) * 4 + (eT & 1) * 2) = w;
+        }
+        zsum[j] = zz;
+      }
+      if (q == 0) {
+        alph[(it & 1) * 64 + lane] = al;
+        if (lane == 0) alph[(it & 1) * 64 + 32] = resc ? 1.f : 0.f;
+      }
+      sm100::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(BP_FULL(it & 1));
+      ell += reduce_scatter32<false>(tmp, lane);
+      zac += reduce_scatter32<false>(zsum, lane);
+    }
+    // ---- partials of this split: m (natural log), l; W from TMEM ----
+    fin[q * 32 + lane] = make_float2(ell, zac);
+    named_bar(1, 128);
+    if (q == 0) {
+      float L = 0.f, Z = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        L += fin[w * 32 + lane].x;
+        Z += fin[w * 32 + lane].y;
+      }
+      zf[lane] = Z;
+      float* pr = a.part + ((size_t(bl) * kNQ + lane) * a.S + sp) * prow;
+      pr[0] = mref == -INFINITY ? -INFINITY : mref * kLn2;
+      pr[1] = L;
+    }
+    if (nmc > 0 && ntl > 0) {
+      if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BW_DONE((ntl - 1) & 1), ((ntl - 1) >> 1) & 1, a.err));
+      sm100::tc_fence_after();
+      for (int mc = 0; mc < nmc; ++mc) {
+        uint32_t w[32];
+        sm100::tmem_ld32(tW + mc * kNQ + (uint32_t(32 * q) << 16), w);
+        sm100::tmem_ld_wait();
+        const int r = mc * 128 + 32 * q + lane;
+        if (r < cv.r_T)
+#pragma unroll
+          for (int j = 0; j < kNQ; ++j) a.part[((size_t(bl) * kNQ + j) * a.S + sp) * prow + 2 + r] = __uint_as_float(w[j]);
+      }
+      sm100::tc_fence_before();
+    }
+    named_bar(2, 256);  // zf ready for the value warps
+  } else {
+    // ================= value warps: acc[d][j] += sum_t weight[t][j] codes^V[t][d] =================
+    const int vw = warp - 6;  // features 16 g + 4 vw .. + 3
+    const int gr = lane >> 2, m4 = lane & 3;
+    const float* alph = reinterpret_cast<const float*>(smem + kOffAlpha);
+    const float* zf = reinterpret_cast<const float*>(smem + kOffZf);
+    float acc[NKV][2][4];
+#pragma unroll
+    for (int h = 0; h < NKV; ++h)
+#pragma unroll
+      for (int mb = 0; mb < 2; ++mb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[h][mb][e] = 0.f;
+    int cvit = 0;
+    bool ok = true;
+    for (int it = 0; it < ntl; ++it) {
+      if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BP_FULL(it & 1), (it >> 1) & 1, a.err));
+      if (bV) {
+        if (alph[(it & 1) * 64 + 32] != 0.f) {
+          const float* al = alph + (it & 1) * 64;
+#pragma unroll
+          for (int h = 0; h < NKV; ++h) {
+            const int j0 = h * GQ + 2 * m4;
+            const float a0 = (2 * m4 < GQ) ? al[j0] : 0.f;
+            const float a1 = (2 * m4 + 1 < GQ) ? al[j0 + 1] : 0.f;
+#pragma unroll
+            for (int mb = 0; mb < 2; ++mb) {
+              acc[h][mb][0] *= a0; acc[h][mb][1] *= a1; acc[h][mb][2] *= a0; acc[h][mb][3] *= a1;
+            }
+          }
+        }
+        const uint2* wbp = reinterpret_cast<const uint2*>(smem + kOffWb + (it & 1) * kWbBytes);
+        const int hps = 8 / bV;
+        int s = 0;
+#pragma unroll
+        for (int h = 0; h < NKV; ++h) {
+          const int k = h % hps;
+          if (k == 0) {
+            s = cvit % kCStages;
+            if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BCV_FULL(s), (cvit / kCStages) & 1, a.err));
+          }
+          const uint8_t* cs = smem + kOffCV + s * kCStageBytes;
+          if (bV == 4) vres_head<4, GQ>(acc[h], cs, k, wbp, h, vw, lane);
+          else if (bV == 2) vres_head<2, GQ>(acc[h], cs, k, wbp, h, vw, lane);
+          else vres_head<8, GQ>(acc[h], cs, k, wbp, h, vw, lane);
+          if (k == hps - 1 || h == NKV - 1) {
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(BCV_EMPTY(s));
+            ++cvit;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(BP_EMPTY(it & 1));
+    }
+    named_bar(2, 256);
+    // acc entries: features d = 16 g + 4 vw + 2 mb + (0 | 1), query heads h g_q + 2 m4 + (0 | 1);
+    // the stored value is 256 acc (the weights carry 2^-8) + sum_t p~ zero
+#pragma unroll
+    for (int h = 0; h < NKV; ++h) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int jj = 2 * m4 + e;
+        if (jj >= GQ) continue;
+        const int j = h * GQ + jj;
+        float* pr = a.part + ((size_t(bl) * kNQ + j) * a.S + sp) * prow + 2 + a.q_cap;
+        const float z = zf[j];
+#pragma unroll
+        for (int mb = 0; mb < 2; ++mb) {
+          const int d = 16 * gr + 4 * vw + 2 * mb;
+          pr[d] = 256.f * acc[h][mb][e] + z;
+          pr[d + 1] = 256.f * acc[h][mb][2 + e] + z;
+        }
+      }
+    }
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) sm100::tmem_dealloc(tmem, kTmemCols);
+}
+
+// Key-cell token rank of every (sequence, layer) row of a launch set.
+struct RankTab {
+  int r_T[kMaxFusedRows];
+};
+
+// P (fp32, [B*Lc][32][q_cap]) -> bf16 hi rows then lo rows per (sequence, layer): [B*Lc][64][q_cap],
+// zero beyond the key cell's r_T (those columns meet the zero fill of U_T's tensor map)
+__global__ void k_split_p(const float* __restrict__ P, int q_cap, const RankTab rt, __nv_bfloat16* __restrict__ out) {
+  const int bl = blockIdx.y;
+  const int r_T = rt.r_T[bl];
+  const int64_t n = int64_t(kNQ) * q_cap;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
+    const int r = int(e % q_cap);
+    const float v = r < r_T ? P[int64_t(bl) * n + e] : 0.f;
+    const __nv_bfloat16 hh = __float2bfloat16_rn(v);
+    out[int64_t(bl) * 2 * n + e] = hh;
+    out[int64_t(bl) * 2 * n + n + e] = __float2bfloat16_rn(v - __bfloat162float(hh));
+  }
+}
+
+constexpr int kSMs = 148;
+
+// Token tiles per split: the fewest whole-wave rounds of one CTA per SM times tiles per CTA, plus
+// the partials each extra split writes and the merge reads (about 0.75 of a tile's bytes per layer).
+int fused_tps(int units, int nt) {
+  int best = nt;
+  double best_c = 1e300;
+  for (int tps = 1; tps <= nt; ++tps) {
+    const int S = (nt + tps - 1) / tps;
+    if (tps > 1 && (nt + tps - 2) / (tps - 1) == S) continue;  // the same split count with fewer tiles
+    const double waves = double((int64_t(units) * S + kSMs - 1) / kSMs);
+    const double c = waves * tps + 0.75 * double(units) * S / kSMs;
+    if (c < best_c - 1e-9) {
+      best_c = c;
+      best = tps;
+    }
+  }
+  return best;
+}
+
+struct FusedWs {
+  size_t hl, part, total;
+  int tps, S;
+};
+
+FusedWs fused_layout(const jolt_shape& s, int Lc) {
+  FusedWs w{};
+  const size_t BL = size_t(s.batch) * Lc, qc = std::max(s.q_cap, 16);
+  const int nt = (s.T + kBM - 1) / kBM;
+  w.tps = fused_tps(int(std::min<size_t>(BL, kMaxFusedRows)), nt);
+  w.S = (nt + w.tps - 1) / w.tps;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  w.hl = take(BL * 2 * kNQ * qc * 2);
+  w.part = take(BL * kNQ * size_t(w.S) * (2 + qc + kD) * 4);
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+bool decode_fused_supported(const jolt_shape& s) {
+  return decode_tc_supported(s) && !s.keys_pre_rope && s.n_q == kNQ && (s.n_kv == 4 || s.n_kv == 8);
+}
+
+size_t decode_fused_ws_bytes(const jolt_shape& s, int Lc) { return fused_layout(s, Lc).total; }
+
+int decode_fused_max_cells() { return kMaxFusedCells; }
+
+jolt_status launch_decode_fused(const DecodeParams& p, const TcCellView* views, uint8_t* ws, const jolt_shape& s,
+                                cudaStream_t st) {
+  // the workspace is laid out for the whole call; this launch set's rows start at its first sequence
+  const FusedWs wl = fused_layout(s, p.Lc);
+  const int BL = p.B * p.Lc, qc = p.q_cap;
+  const int ncell = 2 * p.B * p.Gc;
+  if (ncell > kMaxFusedCells || BL > kMaxFusedRows) return JOLT_ERR_INVALID_ARG;
+  __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(ws + wl.hl);
+  float* part = reinterpret_cast<float*>(ws + wl.part);
+  jolt_status r;
+  // ---- prologue: R q, sum(R q), P = G^K (U_d^K^T q); P as bf16 hi + lo rows ----
+  {
+    StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
+    if ((r = launch_decode_prologue_q(p, st))) return r;
+    RankTab rt{};
+    for (int b = 0; b < p.B; ++b)
+      for (int li = 0; li < p.Lc; ++li) {
+        const int g = (p.layer_begin + li) / p.Lg;
+        rt.r_T[b * p.Lc + li] = views[(b * p.Gc + (g - p.g_first)) * 2].r_T;
+      }
+    k_split_p<<<dim3(std::max(1, std::min(64, (kNQ * qc + 255) / 256)), BL), 256, 0, st>>>(p.ws_P, qc, rt, hl);
+    JOLT_CUDA_TRY(cudaGetLastError());
+  }
+  // ---- tensor maps and per-cell arguments ----
+  FusedMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  FusedArgs fa{};
+  {
+    Operand o;
+    o.ptr = hl; o.major = kMajorK; o.inner = qc; o.outer = 2 * kNQ; o.outer_stride = qc;
+    o.batch = BL; o.batch_stride = int64_t(2) * kNQ * qc;
+    if (!make_tensor_map(&maps.p, o, 2 * kNQ)) return JOLT_ERR_INVALID_ARG;
+  }
+  for (int c = 0; c < ncell; ++c) {
+    const TcCellView& v = views[c];
+    const bool is_k = (c & 1) == 0;
+    fa.cells[c].codes = v.bits ? v.codes : nullptr;
+    fa.cells[c].sz = v.bits ? v.sz : nullptr;
+    fa.cells[c].r_T = v.r_T;
+    fa.cells[c].b = v.bits;
+    if (v.r_T > 0) {
+      Operand o;
+      o.ptr = v.Ut; o.major = is_k ? kMajorK : kMajorMN; o.inner = v.r_T; o.outer = p.T; o.outer_stride = v.r_T;
+      if (!make_tensor_map(&maps.ut[c], o, is_k ? kBM : 64)) return JOLT_ERR_INVALID_ARG;
+    }
+  }
+  fa.T = p.T; fa.nt = (p.T + kBM - 1) / kBM; fa.tps = wl.tps; fa.S = wl.S;
+  fa.Lc = p.Lc; fa.Lg = p.Lg; fa.layer_begin = p.layer_begin; fa.g_first = p.g_first; fa.Gc = p.Gc;
+  fa.n_kv = p.n_kv; fa.gq = p.gq; fa.q_cap = qc; fa.attn_scale = p.attn_scale;
+  fa.qrot = p.ws_qrot; fa.qsum = p.ws_qsum; fa.part = part; fa.err = p.err;
+  // algorithmic work of the launch: the compressed bytes the call must read (p.alg_bytes) and each
+  // contraction once: 2 T r_T per query head for the key and value factors, 2 T d_h per query head
+  // for each residual
+  double flops = 0.0;
+  for (int b = 0; b < p.B; ++b)
+    for (int li = 0; li < p.Lc; ++li) {
+      const int g = (p.layer_begin + li) / p.Lg;
+      const TcCellView& k = views[(b * p.Gc + (g - p.g_first)) * 2];
+      const TcCellView& v = views[(b * p.Gc + (g - p.g_first)) * 2 + 1];
+      flops += 2.0 * p.T * kNQ * (double(k.r_T) + v.r_T) + 2.0 * p.T * kNQ * kD * ((k.bits ? 1 : 0) + (v.bits ? 1 : 0));
+    }
+  {
+    StatScope sc(JOLT_K_DECODE_MAIN, st, flops, p.alg_bytes);
+    const int grid = BL * wl.S;
+    if (p.gq == 4) {
+      JOLT_CUDA_TRY(cudaFuncSetAttribute(k_decode_fused<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
+      k_decode_fused<4><<<grid, kThreads, kSmem, st>>>(maps, fa);
+    } else {
+      JOLT_CUDA_TRY(cudaFuncSetAttribute(k_decode_fused<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
+      k_decode_fused<8><<<grid, kThreads, kSmem, st>>>(maps, fa);
+    }
+    JOLT_CUDA_TRY(cudaGetLastError());
+  }
+  // ---- merge of the splits and finalize ----
+  DecodeParams pm = p;
+  pm.S = wl.S;
+  pm.ws_part = part;
+  StatScope sc2(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
+  return launch_decode_merge(pm, st);
+}
+
+}  // namespace jolt

@@ -398,7 +398,6 @@ jolt_status launch_decode_prologue_q(const DecodeParams& p, cudaStream_t st) {
 
 jolt_status launch_decode_simt(const DecodeParams& p, cudaStream_t st) {
   if (p.gq > kMaxGq) return JOLT_ERR_INVALID_ARG;
-  const dim3 gq_grid(p.n_q, p.Lc, p.B);
   {
     StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
     jolt_status r = launch_decode_prologue_q(p, st);
@@ -421,6 +420,11 @@ jolt_status launch_decode_simt(const DecodeParams& p, cudaStream_t st) {
   }
   JOLT_CUDA_TRY(cudaGetLastError());
   StatScope sc2(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
+  return launch_decode_merge(p, st);
+}
+
+jolt_status launch_decode_merge(const DecodeParams& p, cudaStream_t st) {
+  const dim3 gq_grid(p.n_q, p.Lc, p.B);
   const size_t msm = (size_t(p.q_cap) + 128 + p.d_h + p.S) * sizeof(float);
   if (p.d_h == 64) {
     JOLT_CUDA_TRY(cudaFuncSetAttribute(k_decode_merge<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(msm)));
