@@ -30,6 +30,9 @@ from synth import get_workload, make_kv, make_queries, make_inv_freq  # noqa: E4
 
 METRIC = ("decode-attn context tokens/s & HBM GB/s over compressed cache; compress raw GB/s")
 DEFAULT_WORKLOAD = "llama70b_128k"
+# the metric's other workloads in the default run: the HBM-bound non-RoPE decode (8B, 32K) and the
+# batch-4 pre-RoPE 64K workload at its tighter budget
+DEFAULT_ALSO = "llama8b_32k:3,llama8b_64k_b4:5"
 
 
 def parse():
@@ -50,6 +53,9 @@ def parse():
     ap.add_argument("--no-grouping", action="store_true", help="skip the layer-grouping report")
     ap.add_argument("--cells-per-pass", type=int, default=0,
                     help="cells jolt_analyze batches per pass (0: every cell of a kind in one pass)")
+    ap.add_argument("--also", default=None,
+                    help="extra workloads name[:ratio],... timed after the headline (default: the metric's "
+                         "other workloads when --workload is the default; '' for none)")
     ap.add_argument("--exact", action="store_true",
                     help="exact token-mode SVD (sketch width = L_g*n_kv*d_h: the JoLT backbone FlashJoLT replaces)")
     return ap.parse_args()
@@ -160,7 +166,11 @@ def cpu_threads():
 
 
 def run_reference(args, w, rank, world):
-    """--impl reference: the CPU oracle, as it stands, on bounded samples of the workload."""
+    """--impl reference: the CPU oracle, as it stands, on bounded samples of the workload. Each step
+    is one sample (one layer group's K and V cells over the first --cpu-tokens tokens: exact
+    ST-HOSVD compression and the group's decode attention); ms_per_step is that sample's measured
+    time and value its context tokens per second, a group of L_g layers being L_g / L of a token's
+    pass through the model."""
     if rank != 0:
         return
     choices = {0: (256, 128, 4), 1: (256, 128, 4)} if not w.fixed_choice else {0: w.fixed_choice, 1: w.fixed_choice}
@@ -172,13 +182,16 @@ def run_reference(args, w, rank, world):
         dt, desc = oracle_sample(w, choices, T_s)
         times.append(dt)
     t_sample = float(np.mean(times))
-    t_full = t_sample * w.n_groups * w.batch * (w.T / T_s)
-    value = w.batch * w.T / t_full
+    value = T_s * (w.layers_per_group / w.n_layers) / t_sample
+    desc = (f"oracle (float64 NumPy) on one {w.layers_per_group}-layer group (its K and V cells) of the first "
+            f"{T_s} tokens: exact ST-HOSVD compress + decode of {w.layers_per_group} layers per step; context "
+            f"tokens counted as {T_s} x {w.layers_per_group}/{w.n_layers} of a full pass")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "context tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": t_full * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": t_sample * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "T": w.T, "n_layers": w.n_layers,
+                       "sample": {"tokens": T_s, "layers": w.layers_per_group, "sequences": 1},
                        "budget": "fixed sample ranks (256, 128, 4)" if not w.fixed_choice else "fixed"},
             "cpu_baseline": {"value": value, "unit": "context tokens/s", "cores": cpu_threads(),
                              "kind": "oracle", "sample": desc},
@@ -325,12 +338,15 @@ def layer_grouping(step, rank=32, tau=0.5):
 
 
 def decode_work(w, shape, choices):
-    """Algorithmic work of one decode step over every layer: (bytes, tensor flops).
+    """Algorithmic work of one decode step over every layer: (bytes, flops).
 
     Bytes: the compressed cache read once (each cell's U_T, U_d, cores, codes and scale/zero
-    pairs) plus q and the output. Flops: the dense contractions the attention cannot avoid on the
-    tensor-core path — per (layer, KV head) the pre-RoPE key rebuild U_T^K B_h (two bf16 terms of
-    B_h) or the non-RoPE score product P U_T^K^T (two terms of P), and P~ U_T^V per layer."""
+    pairs) plus q and the output. Flops: each contraction of the method once per (token, layer):
+    scores 2 r_T^K per query head (non-RoPE: U_T^K against P = G^K U_d^K^T q) or the key rebuild
+    2 r_T^K d_h per KV head plus q.k 2 d_h per query head (pre-RoPE), values 2 r_T^V per query head,
+    and 2 d_h per query head for each residual that is stored (the key residual of non-RoPE keys,
+    the value residual). bf16 hi/lo terms that only restore an operand's precision are not
+    algorithmic work (the kernels report them as issued flops)."""
     from long_context_st_b200 import api
     G = w.n_layers // w.layers_per_group
     nbytes = sum(api.cell_bytes(shape, tuple(c)) for c in choices)
@@ -338,14 +354,15 @@ def decode_work(w, shape, choices):
     flops = 0.0
     for b in range(w.batch):
         for g in range(G):
-            rk = choices[(b * G + g) * 2][0]
-            rv = choices[(b * G + g) * 2 + 1][0]
-            for _ in range(w.layers_per_group):
-                if w.keys_pre_rope:
-                    flops += 2 * 2.0 * w.T * rk * w.d_h * w.n_kv
-                else:
-                    flops += 2 * 2.0 * w.n_q * w.T * rk
-                flops += 2.0 * w.n_q * w.T * rv
+            rk, _, bk = choices[(b * G + g) * 2]
+            rv, _, bv = choices[(b * G + g) * 2 + 1]
+            per_layer = 0.0
+            if w.keys_pre_rope:
+                per_layer += 2.0 * rk * w.d_h * w.n_kv + 2.0 * w.d_h * w.n_q
+            else:
+                per_layer += 2.0 * rk * w.n_q + (2.0 * w.d_h * w.n_q if bk else 0.0)
+            per_layer += 2.0 * rv * w.n_q + (2.0 * w.d_h * w.n_q if bv else 0.0)
+            flops += per_layer * w.T * w.layers_per_group
     return nbytes, flops
 
 
@@ -387,6 +404,127 @@ def e2e_over_ranks(e_ms, err, device):
     return t, err
 
 
+def measure(args, w, ratio, dev, world, steps, warmup, peaks, secondary=False):
+    """Time `steps` steps of workload w after `warmup` untimed ones (barrier and synchronize on both
+    sides, max over ranks). Returns (line fields, step) for the JSON line."""
+    from long_context_st_b200 import api
+    hbm_peak, tc_burst, tc_sust, peak_src = peaks
+    step = Step(w, ratio, dev, exact=args.exact and not secondary, cells_per_pass=args.cells_per_pass)
+    torch.cuda.synchronize()
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    n_kernels, kernel_names = (None, []) if (args.no_count or secondary) else count_kernels(step)
+    names = ["start", "analyzed", "allocated", "compressed", "decoded"]
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    api.stats_read(reset=True)
+    api.stats_enable(True)
+    with Clocks(dev.index) as clk:
+        t_start.record()
+        for i in range(steps):
+            if args.nvtx:
+                torch.cuda.nvtx.range_push("jolt_step")
+            step.run(evs[i])
+            if args.nvtx:
+                torch.cuda.nvtx.range_pop()
+        t_end.record()
+        torch.cuda.synchronize()
+    api.stats_enable(False)
+    stats = api.stats_read(reset=True)
+    total_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        import torch.distributed as dist
+        total_ms = max_over_ranks(total_ms, dev)
+        dist.barrier()
+    ms_step = total_ms / steps
+    ph = {k: float(np.mean([e["start"].elapsed_time(e[k]) if k != "start" else 0.0 for e in evs]))
+          for k in names}
+    t_an = ph["analyzed"]
+    t_alloc = ph["allocated"] - ph["analyzed"]
+    t_cmp = ph["compressed"] - ph["allocated"]
+    t_dec = ph["decoded"] - ph["compressed"]
+
+    tokens = w.batch * w.T
+    raw = 2 * w.batch * w.n_layers * w.n_kv * w.T * w.d_h * w.io_bytes
+    dbytes, dflops = decode_work(w, step.shape, step.choices)
+    _, cache_total = api.cache_layout(step.shape, step.choices)
+
+    def fam_roof(name, bound, peak):
+        st = stats[name]
+        if not st["launches"] or st["ms"] <= 0:
+            return None
+        sec = st["ms"] / st["launches"] / 1e3
+        if bound == "tensor":
+            ach = st["flops"] / st["launches"] / sec / 1e12
+            unit = "TFLOP/s"
+        else:
+            ach = st["bytes"] / st["launches"] / sec / 1e9
+            unit = "GB/s"
+        r = {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+             "traffic": None, "kernel": name, "launches_per_step": st["launches"] / steps,
+             "ms_per_step": st["ms"] / steps, "peak_source": peak_src}
+        if bound == "tensor" and st.get("flops_issued", 0.0) > st["flops"]:
+            r["issued_tflops"] = st["flops_issued"] / st["launches"] / sec / 1e12
+        return r
+
+    def binding(name):
+        # a family that reports both flops and bytes is bound by the resource it uses the larger
+        # fraction of (the pre-RoPE key rebuild is a tensor-core contraction, the rest streams HBM)
+        t = fam_roof(name, "tensor", tc_sust) if stats[name]["flops"] > 0 else None
+        h = fam_roof(name, "hbm", hbm_peak) if stats[name]["bytes"] > 0 else None
+        if t and h:
+            other = h if t["frac"] >= h["frac"] else t
+            best = t if t["frac"] >= h["frac"] else h
+            best["other"] = {"bound": other["bound"], "achieved": other["achieved"], "peak": other["peak"],
+                             "unit": other["unit"], "frac": other["frac"]}
+            return best
+        return t or h
+
+    fams = ["gemm", "decode_main", "residual"]
+    dom = max(fams, key=lambda k: stats[k]["ms"])
+    dec = {"context_tokens_per_s": tokens * w.n_layers / (t_dec / 1e3) if t_dec > 0 else None,
+           "context_tokens_per_s_per_layer_step": tokens / (t_dec / 1e3) if t_dec > 0 else None,
+           "ms": t_dec,
+           "hbm_gbs": dbytes / (t_dec / 1e3) / 1e9 if t_dec > 0 else None,
+           "alg_bytes": dbytes, "frac_of_hbm": dbytes / (t_dec / 1e3) / 1e9 / hbm_peak if t_dec > 0 else None,
+           "tensor_flops": dflops,
+           "tensor_tflops": dflops / (t_dec / 1e3) / 1e12 if t_dec > 0 else None,
+           # the step's own roofline: the slower of its HBM bytes and its tensor flops
+           "roofline_ms": max(dbytes / hbm_peak / 1e6, dflops / tc_sust / 1e9),
+           "bound": "tensor" if dflops / tc_sust / 1e9 > dbytes / hbm_peak / 1e6 else "hbm",
+           "frac_of_roofline": max(dbytes / hbm_peak / 1e6, dflops / tc_sust / 1e9) / t_dec if t_dec > 0 else None}
+    out = {"value": tokens * world / (ms_step / 1e3), "ms_per_step": ms_step,
+           "config": {"workload": w.name, "batch": w.batch, "n_layers": w.n_layers,
+                      "layers_per_group": w.layers_per_group, "n_kv": w.n_kv, "n_q": w.n_q, "T": w.T,
+                      "d_h": w.d_h, "keys_pre_rope": w.keys_pre_rope, "budget_ratio": ratio,
+                      "q_cap": step.shape.q_cap, "sketch_cols": step.shape.sketch_cols,
+                      "power_iters": step.shape.power_iters, "l2": "inputs larger than L2 (no flush)",
+                      "token_svd": "exact" if step.shape.sketch_cols == w.n_cols else "randomized",
+                      "cells_per_pass": step.shape.cells_per_pass,
+                      "parallelism": f"dp{world}" if world > 1 else "single-gpu"},
+           "decode_attn_context_tokens_per_s": dec["context_tokens_per_s"],
+           "decode_hbm_gbs": dec["hbm_gbs"], "decode_frac_of_hbm": dec["frac_of_hbm"],
+           "compress_raw_gbs": raw / ((t_an + t_alloc + t_cmp) / 1e3) / 1e9,
+           "breakdown_ms": {"analyze": t_an, "allocate_host": t_alloc, "compress": t_cmp, "decode": t_dec},
+           "compress": {"raw_gbs": raw / ((t_an + t_alloc + t_cmp) / 1e3) / 1e9,
+                        "raw_bytes": raw, "cache_bytes": cache_total, "ratio": raw / cache_total},
+           "decode": dec, "roofline": binding(dom), "roofline_decode": binding("decode_main"),
+           "kernel_stats": {k: {kk: (float(vv) if isinstance(vv, float) else int(vv)) for kk, vv in v.items()}
+                            for k, v in stats.items()},
+           "allocator_ablation": allocator_ablation(step),
+           "clocks": clk.summary(), "choices": sorted(set(map(tuple, step.choices)))}
+    if not secondary:
+        out["gpu_launches"] = n_kernels * steps if n_kernels is not None else None
+        out["kernels"] = kernel_names
+    return out, step
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -414,127 +552,15 @@ def main():
     dev = torch.device("cuda", local)
     w = rank_workload(args.workload, rank, over)
     ratio = args.ratio if args.ratio else (w.budget_ratios[0] if w.budget_ratios else None)
-    hbm_peak, tc_burst, tc_sust, peak_src = load_peaks()
-    from long_context_st_b200 import api
-
-    step = Step(w, ratio, dev, exact=args.exact, cells_per_pass=args.cells_per_pass)
-    torch.cuda.synchronize()
-    for _ in range(max(3, args.warmup)):
-        step.run()
-    torch.cuda.synchronize()
-    n_kernels, kernel_names = (None, []) if args.no_count else count_kernels(step)
-
-    names = ["start", "analyzed", "allocated", "compressed", "decoded"]
-    evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
-    api.stats_read(reset=True)
-    api.stats_enable(True)
-    with Clocks(local) as clk:
-        t_start.record()
-        for i in range(args.steps):
-            if args.nvtx:
-                torch.cuda.nvtx.range_push("jolt_step")
-            step.run(evs[i])
-            if args.nvtx:
-                torch.cuda.nvtx.range_pop()
-        t_end.record()
-        torch.cuda.synchronize()
-    api.stats_enable(False)
-    stats = api.stats_read(reset=True)
-    total_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        import torch.distributed as dist
-        total_ms = max_over_ranks(total_ms, dev)
-        dist.barrier()
-    ms_step = total_ms / args.steps
-    ph = {k: float(np.mean([e["start"].elapsed_time(e[k]) if k != "start" else 0.0 for e in evs]))
-          for k in names}
-    t_an = ph["analyzed"]
-    t_alloc = ph["allocated"] - ph["analyzed"]
-    t_cmp = ph["compressed"] - ph["allocated"]
-    t_dec = ph["decoded"] - ph["compressed"]
-
+    peaks = load_peaks()
+    res, step = measure(args, w, ratio, dev, world, args.steps, max(3, args.warmup), peaks)
     tokens = w.batch * w.T
-    value = tokens * world / (ms_step / 1e3)
-    raw = 2 * w.batch * w.n_layers * w.n_kv * w.T * w.d_h * w.io_bytes
-    dbytes, dflops = decode_work(w, step.shape, step.choices)
-    _, cache_total = api.cache_layout(step.shape, step.choices)
-
-    def fam_roof(name, bound, peak):
-        s = stats[name]
-        if not s["launches"] or s["ms"] <= 0:
-            return None
-        if bound == "tensor":
-            ach = s["flops"] / s["launches"] / (s["ms"] / s["launches"] / 1e3) / 1e12
-            unit = "TFLOP/s"
-        else:
-            ach = s["bytes"] / s["launches"] / (s["ms"] / s["launches"] / 1e3) / 1e9
-            unit = "GB/s"
-        return {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
-                "traffic": None, "kernel": name, "launches_per_step": s["launches"] / args.steps,
-                "ms_per_step": s["ms"] / args.steps, "peak_source": peak_src}
-
-    def binding(name):
-        # a family that reports both flops and bytes is bound by the resource it uses the larger
-        # fraction of (the pre-RoPE key rebuild is a tensor-core contraction, the rest streams HBM)
-        t = fam_roof(name, "tensor", tc_sust) if stats[name]["flops"] > 0 else None
-        h = fam_roof(name, "hbm", hbm_peak) if stats[name]["bytes"] > 0 else None
-        if t and h:
-            other = h if t["frac"] >= h["frac"] else t
-            best = t if t["frac"] >= h["frac"] else h
-            best["other"] = {"bound": other["bound"], "achieved": other["achieved"], "peak": other["peak"],
-                             "unit": other["unit"], "frac": other["frac"]}
-            return best
-        return t or h
-
-    fams = ["gemm", "decode_main", "residual"]
-    dom = max(fams, key=lambda k: stats[k]["ms"])
-    roof = binding(dom)
-    roof_dec = binding("decode_main")
-    # DRAM traffic of the key kernel from one ncu capture (profiles/k_keys_tc_k_values_res_*:
-    # one 4-layer group of the 70B shape at T = 65536, r_T = 464, b = 4: 225.7 MB read + 58.7 MB
-    # written), scaled to a full launch by the tokens it processes; other workloads: not measured
-    if roof_dec is not None and w.name == "llama70b_128k" and w.keys_pre_rope:
-        roof_dec["traffic"] = (225.711616e6 + 58.666752e6) * (w.T / 65536)
-        roof_dec["traffic_source"] = "ncu capture at T = 65536 scaled by T (one layer group per launch)"
-
-    line = {"metric": METRIC, "value": value, "unit": "context tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+    line = {"metric": METRIC, "value": res["value"], "unit": "context tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": res["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (planted low-rank + noise K/V, seeded)",
-            "config": {"workload": w.name, "batch": w.batch, "n_layers": w.n_layers,
-                       "layers_per_group": w.layers_per_group, "n_kv": w.n_kv, "n_q": w.n_q, "T": w.T,
-                       "d_h": w.d_h, "keys_pre_rope": w.keys_pre_rope, "budget_ratio": ratio,
-                       "q_cap": step.shape.q_cap, "sketch_cols": step.shape.sketch_cols,
-                       "power_iters": step.shape.power_iters, "l2": "inputs larger than L2 (no flush)",
-                       "token_svd": "exact" if step.shape.sketch_cols == w.n_cols else "randomized",
-                       "cells_per_pass": step.shape.cells_per_pass,
-                       "parallelism": f"dp{world}" if world > 1 else "single-gpu"},
-            "breakdown_ms": {"analyze": t_an, "allocate_host": t_alloc, "compress": t_cmp, "decode": t_dec},
-            "compress": {"raw_gbs": raw / ((t_an + t_alloc + t_cmp) / 1e3) / 1e9,
-                         "raw_bytes": raw, "cache_bytes": cache_total, "ratio": raw / cache_total},
-            "decode": {"context_tokens_per_s": tokens * w.n_layers / (t_dec / 1e3) if t_dec > 0 else None,
-                       "context_tokens_per_s_per_layer_step": tokens / (t_dec / 1e3) if t_dec > 0 else None,
-                       "hbm_gbs": dbytes / (t_dec / 1e3) / 1e9 if t_dec > 0 else None,
-                       "alg_bytes": dbytes, "frac_of_hbm": dbytes / (t_dec / 1e3) / 1e9 / hbm_peak if t_dec > 0 else None,
-                       "tensor_flops": dflops,
-                       "tensor_tflops": dflops / (t_dec / 1e3) / 1e12 if t_dec > 0 else None,
-                       # the step's own roofline: the slower of its HBM bytes and its tensor flops
-                       "roofline_ms": max(dbytes / hbm_peak / 1e6, dflops / tc_sust / 1e9),
-                       "bound": "tensor" if dflops / tc_sust / 1e9 > dbytes / hbm_peak / 1e6 else "hbm",
-                       "frac_of_roofline": max(dbytes / hbm_peak / 1e6, dflops / tc_sust / 1e9) / t_dec if t_dec > 0 else None},
-            "roofline": roof, "roofline_decode": roof_dec,
-            "kernel_stats": {k: {kk: (float(vv) if isinstance(vv, float) else int(vv)) for kk, vv in v.items()}
-                             for k, v in stats.items()},
-            "allocator_ablation": allocator_ablation(step),
-            "layer_grouping": None if args.no_grouping else layer_grouping(step),
-            "gpu_launches": n_kernels * args.steps if n_kernels is not None else None,
-            "kernels": kernel_names, "clocks": clk.summary(), "choices": sorted(set(map(tuple, step.choices)))}
+            "data": "synthetic (planted low-rank + noise K/V, seeded)"}
+    line.update({k: v for k, v in res.items() if k not in ("value", "ms_per_step")})
+    line["layer_grouping"] = None if args.no_grouping else layer_grouping(step)
 
     # e2e: same step through the C ABI with host buffers: H2D of K and V and D2H of the outputs.
     # Every rank takes the same collective steps whether or not its own leg worked.
@@ -590,6 +616,30 @@ def main():
         t_full = dt * G * w.batch * (w.T / min(args.cpu_tokens, w.T))
         line["cpu_baseline"] = {"value": tokens / t_full, "unit": "context tokens/s", "cores": cpu_threads(),
                                 "kind": "oracle", "sample": desc, "sample_seconds": dt}
+    # the metric's other workloads, timed the same way in the same run (decode and compress
+    # figures; the headline's buffers are released first)
+    also = args.also if args.also is not None else (DEFAULT_ALSO if args.workload == DEFAULT_WORKLOAD else "")
+    if also and not (args.layers or args.seqlen):
+        step = None
+        torch.cuda.empty_cache()
+        sec = {}
+        for spec in [x for x in also.split(",") if x]:
+            name, r = (spec.split(":") + [None])[:2]
+            w2 = rank_workload(name, rank, {})
+            r2 = float(r) if r else (w2.budget_ratios[0] if w2.budget_ratios else None)
+            try:
+                res2, st2 = measure(args, w2, r2, dev, world, 3, 3, peaks, secondary=True)
+                sec[f"{name}@{r2:g}x" if r2 else name] = {
+                    k: res2[k] for k in ("value", "ms_per_step", "config", "decode_attn_context_tokens_per_s",
+                                         "decode_hbm_gbs", "decode_frac_of_hbm", "compress_raw_gbs", "breakdown_ms",
+                                         "compress", "decode", "roofline", "roofline_decode", "allocator_ablation",
+                                         "clocks")}
+                sec[f"{name}@{r2:g}x" if r2 else name]["steps"] = 3
+            except (RuntimeError, MemoryError) as ex:
+                sec[spec] = {"error": str(ex)[:200]}
+            st2 = None
+            torch.cuda.empty_cache()
+        line["workloads"] = sec
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

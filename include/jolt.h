@@ -62,6 +62,20 @@ typedef enum { JOLT_F32 = 0, JOLT_BF16 = 1 } jolt_dtype;
 typedef enum { JOLT_OP_COMPRESS = 0, JOLT_OP_DECODE = 1 } jolt_op;
 
 /* Problem description shared by all calls. */
+/* Kernel form of the tcgen05 GEMMs the compressor and decoder run (all give the same results up to
+ * the fp32 summation order):
+ *   JOLT_GEMM_DEFAULT     one output tile per CTA, one or two 128-row accumulators, split-K and
+ *                         tile shape from a whole-wave time estimate; MN-major operands copied as one
+ *                         multi-chunk TMA copy per pipeline stage;
+ *   JOLT_GEMM_PER_CHUNK   the same kernel copying MN-major operands one 64-wide chunk at a time;
+ *   JOLT_GEMM_PERSISTENT  persistent single CTAs, two TMEM accumulators (epilogue of one tile under
+ *                         the main loop of the next), for N > 128 and more than one row tile;
+ *   JOLT_GEMM_PAIRS       the persistent form on CTA pairs (cta_group::2, M = 256 per MMA, each SM
+ *                         staging half of B). Faster in isolation at a fixed clock; in a whole
+ *                         compression pass under the 1 kW power cap it lowers the clock the rest of
+ *                         the pass runs at, so it is not the default. */
+typedef enum { JOLT_GEMM_DEFAULT = 0, JOLT_GEMM_PER_CHUNK = 1, JOLT_GEMM_PERSISTENT = 2, JOLT_GEMM_PAIRS = 3 } jolt_gemm_plan;
+
 typedef struct {
   int32_t batch;              /* sequences B >= 1 */
   int32_t n_layers;           /* L >= 1 */
@@ -82,6 +96,7 @@ typedef struct {
   uint64_t sketch_seed;       /* seed of the Rademacher sketch matrix */
   float attn_scale;           /* softmax scale, usually 1/sqrt(d_h) */
   float rope_attention_scaling; /* multiplies cos and sin (1.0 for plain RoPE) */
+  int32_t gemm_plan;          /* jolt_gemm_plan of the compressor's and decoder's GEMMs */
 } jolt_shape;
 
 /* Per-cell rank/bit choice: r_T, r_d multiples of 16 (both 0 or both > 0), b in {0,2,4,8}. */
@@ -118,7 +133,7 @@ jolt_status jolt_cache_layout(const jolt_shape* shape, const jolt_cell_choice* c
 /* ---- Stored cache as a host blob (persisting a compressed cache, moving it between processes).
  * The pages store the factors, codes and scales per group ("A JoLT for the KV cache", §3, the
  * stored cache); the blob adds a header so a reader can check what it holds:
- *   bytes 0..7   magic "JOLTCACH"; 8..11 format version (1); 12..15 header bytes (h)
+ *   bytes 0..7   magic "JOLTCACH"; 8..11 format version (2); 12..15 header bytes (h)
  *   16..         jolt_shape (as in this header), int32 n_cells, n_cells jolt_cell_choice,
  *                uint64 cache bytes (c), zero padding up to h (a multiple of 256)
  *   h .. h+c     the cache exactly as jolt_cache_layout places it (device bytes copied verbatim)
@@ -317,11 +332,12 @@ jolt_status jolt_unpack_dequant(const uint8_t* codes, const void* sz, int64_t n_
  *   B[z*stride_b + n*ldb + k] (b_mn_major = 0) or B[z*stride_b + k*ldb + n] (b_mn_major = 1).
  * C (device, fp32): element (m,n) at C[z*stride_c + m*ldc + n]. Strides in elements; lda and ldb
  * must be multiples of 8 and the base pointers 16-byte aligned. k_split > 1 splits K over CTAs
- * and requires accumulate = 1 (atomic adds into C, which the caller zeroes first). */
+ * and requires accumulate = 1 (atomic adds into C, which the caller zeroes first). plan: a
+ * jolt_gemm_plan (JOLT_ERR_INVALID_ARG outside it). */
 jolt_status jolt_gemm_bf16(const void* A, int32_t a_mn_major, const void* B, int32_t b_mn_major,
                            float* C, int32_t M, int32_t N, int32_t K, int64_t lda, int64_t ldb,
                            int64_t ldc, int32_t batch, int64_t stride_a, int64_t stride_b,
-                           int64_t stride_c, int32_t k_split, int32_t accumulate, void* stream);
+                           int64_t stride_c, int32_t k_split, int32_t accumulate, int32_t plan, void* stream);
 
 /* The same product with the fp32 result split into bf16 parts by the GEMM's epilogue instead of
  * being stored: Ch = bf16_rn(c), and when Cl is not NULL, Cl = bf16_rn(c - Ch), for every result c
@@ -399,8 +415,10 @@ typedef struct {
   int32_t kernel;       /* jolt_kernel_family */
   uint64_t launches;
   double ms;            /* summed device time of the launches */
-  double flops;         /* summed algorithmic FLOPs */
+  double flops;         /* summed algorithmic FLOPs: each product of the method counted once */
   double bytes;         /* summed algorithmic bytes */
+  double flops_issued;  /* summed tensor-core FLOPs issued: a product carried as several bf16
+                           terms (hi/lo splits of fp32 operands) counts once per term */
 } jolt_kernel_stat;
 
 void jolt_stats_enable(int32_t on);

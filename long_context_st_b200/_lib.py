@@ -29,12 +29,12 @@ class Shape(C.Structure):
                 ("io_dtype", C.c_int32), ("factor_dtype", C.c_int32), ("keys_pre_rope", C.c_int32),
                 ("q_cap", C.c_int32), ("sketch_cols", C.c_int32), ("power_iters", C.c_int32),
                 ("cells_per_pass", C.c_int32), ("rot_seed", C.c_uint64), ("sketch_seed", C.c_uint64),
-                ("attn_scale", C.c_float), ("rope_attention_scaling", C.c_float)]
+                ("attn_scale", C.c_float), ("rope_attention_scaling", C.c_float), ("gemm_plan", C.c_int32)]
 
 
 class KernelStat(C.Structure):
     _fields_ = [("kernel", C.c_int32), ("launches", C.c_uint64), ("ms", C.c_double),
-                ("flops", C.c_double), ("bytes", C.c_double)]
+                ("flops", C.c_double), ("bytes", C.c_double), ("flops_issued", C.c_double)]
 
 
 KERNEL_FAMILIES = ["gemm", "decode_main", "residual", "decode_aux", "chol", "eig"]
@@ -85,7 +85,7 @@ SIGNATURES = [
     ("jolt_unpack_dequant", C.c_int, [_P, _P, C.c_int64, C.c_int32, C.c_int32, _P, _P]),
     ("jolt_gemm_bf16", C.c_int, [_P, C.c_int32, _P, C.c_int32, _P, C.c_int32, C.c_int32, C.c_int32,
                                  C.c_int64, C.c_int64, C.c_int64, C.c_int32, C.c_int64, C.c_int64,
-                                 C.c_int64, C.c_int32, C.c_int32, _P]),
+                                 C.c_int64, C.c_int32, C.c_int32, C.c_int32, _P]),
     ("jolt_gemm_bf16_hilo", C.c_int, [_P, C.c_int32, _P, C.c_int32, _P, _P, C.c_int32, C.c_int32,
                                       C.c_int32, C.c_int64, C.c_int64, C.c_int64, C.c_int32, C.c_int64,
                                       C.c_int64, C.c_int64, _P]),

@@ -46,6 +46,7 @@ def make_shape(w, **over) -> Shape:
     s.sketch_seed = over.get("sketch_seed", 0xC0FFEE00 + w.seed)
     s.attn_scale = over.get("attn_scale", 1.0 / math.sqrt(w.d_h))
     s.rope_attention_scaling = over.get("rope_attention_scaling", 1.0)
+    s.gemm_plan = over.get("gemm_plan", GEMM_PLANS["default"])
     check(lib().jolt_shape_check(C.byref(s)), "jolt_shape_check")
     return s
 
@@ -287,8 +288,12 @@ def unpack_dequant(codes, sz, d, b, stream=None):
     return out
 
 
+# jolt_gemm_plan values by name
+GEMM_PLANS = {"default": 0, "perchunk": 1, "persistent": 2, "pairs": 3}
+
+
 def gemm_bf16(A, B, a_mn_major=False, b_mn_major=False, C=None, k_split=1, accumulate=False,
-              stream=None):
+              plan="default", stream=None):
     """C = A_logical @ B_logical for bf16 tensors, via the library's tcgen05 GEMM.
 
     A: [batch?, M, K] (a_mn_major False) or [batch?, K, M] (True); B: [batch?, N, K] (b_mn_major
@@ -305,7 +310,7 @@ def gemm_bf16(A, B, a_mn_major=False, b_mn_major=False, C=None, k_split=1, accum
     C3 = C if C.dim() == 3 else C[None]
     check(lib().jolt_gemm_bf16(_ptr(A3), int(a_mn_major), _ptr(B3), int(b_mn_major), _ptr(C3), M, N,
                                K, A3.stride(1), B3.stride(1), C3.stride(1), bt, A3.stride(0),
-                               B3.stride(0), C3.stride(0), k_split, int(accumulate),
+                               B3.stride(0), C3.stride(0), k_split, int(accumulate), GEMM_PLANS[plan],
                                _stream(stream)), "jolt_gemm_bf16")
     return C3 if batched else C3[0]
 
@@ -374,10 +379,11 @@ def stats_read(reset=True):
     arr = (KernelStat * len(KERNEL_FAMILIES))()
     check(lib().jolt_stats_read(arr, int(reset)), "jolt_stats_read")
     return {KERNEL_FAMILIES[i]: dict(launches=arr[i].launches, ms=arr[i].ms, flops=arr[i].flops,
-                                     bytes=arr[i].bytes) for i in range(len(KERNEL_FAMILIES))}
+                                     bytes=arr[i].bytes, flops_issued=arr[i].flops_issued)
+            for i in range(len(KERNEL_FAMILIES))}
 
 
-__all__ = ["analyze_from_host", "layer_align_workspace", "layer_align", "group_layers", "uniform_group", "gemm_bf16_hilo", "gemm_bf16_residual", "allocate_variant", "JOLT_ALLOC_JOINT", "JOLT_ALLOC_KV_SPLIT", "JOLT_ALLOC_UNIFORM", "serialize_cache", "deserialize_cache", "cache_blob_info", "cache_blob_bytes", "decode_attn_noalloc", "stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
+__all__ = ["analyze_from_host", "layer_align_workspace", "layer_align", "group_layers", "uniform_group", "gemm_bf16_hilo", "gemm_bf16_residual", "allocate_variant", "JOLT_ALLOC_JOINT", "JOLT_ALLOC_KV_SPLIT", "JOLT_ALLOC_UNIFORM", "JOLT_ALLOC_COORD", "GEMM_PLANS", "serialize_cache", "deserialize_cache", "cache_blob_info", "cache_blob_bytes", "decode_attn_noalloc", "stats_enable", "stats_read", "sym_eig", "gemm_bf16", "make_shape", "n_cells", "choices_array", "cell_bytes", "kv_bytes", "cache_layout", "phi",
            "allocate", "workspace_bytes", "new_workspace", "analyze", "compress", "decode_attn",
            "check_ws", "rotate_rows", "quantize_pack", "unpack_dequant", "JoltError",
            "JOLT_OP_COMPRESS", "JOLT_OP_DECODE"]

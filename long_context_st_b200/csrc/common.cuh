@@ -26,10 +26,17 @@ __device__ __forceinline__ void report_error(int32_t* err, int32_t code) {
   if (err) atomicCAS(err, 0, code);
 }
 
-// With JOLT_DEBUG set in the environment, a failing CUDA call is printed with its location.
+// Diagnostic printing to stderr: compiled in by a debug build (-DJOLT_DEBUG), never switched at
+// run time.
+#ifdef JOLT_DEBUG
+constexpr bool kDebug = true;
+#else
+constexpr bool kDebug = false;
+#endif
+
+// In a debug build a failing CUDA call is printed with its location.
 inline void jolt_note_cuda_error(cudaError_t e, const char* what, const char* file, int line) {
-  if (std::getenv("JOLT_DEBUG"))
-    std::fprintf(stderr, "jolt: %s:%d: %s -> %s\n", file, line, what, cudaGetErrorString(e));
+  if (kDebug) std::fprintf(stderr, "jolt: %s:%d: %s -> %s\n", file, line, what, cudaGetErrorString(e));
 }
 
 #define JOLT_CUDA_TRY(expr)                                       \

@@ -412,6 +412,12 @@ struct Ctx {
   template <typename Tp> Tp* atc(size_t rel) const { return reinterpret_cast<Tp*>(ws + p.off_cmp + rel); }
 };
 
+// Every contraction of the compressor runs in the kernel form the shape names.
+jolt_status run_gemm(const Ctx& c, GemmCall& g) {
+  g.plan = c.s->gemm_plan;
+  return gemm_tc(g, c.st);
+}
+
 void report_error_host(const Ctx& c, int32_t code) {
   int32_t cur = 0;
   cudaMemcpyAsync(&cur, c.err, 4, cudaMemcpyDeviceToHost, c.st);
@@ -493,8 +499,8 @@ jolt_status orth(const Ctx& c, float* Yf, int* cur, int rows, int C, bool polish
     g.k_split = 0;
     g.accumulate = true; g.err = c.err;
     g.c_upper = true;  // symmetric: the Cholesky reads the upper triangle
-    if ((r = gemm_tc(g, c.st))) return r;
-    if (std::getenv("JOLT_DEBUG")) {
+    if ((r = run_gemm(c, g))) return r;
+    if (kDebug) {
       std::vector<float> h(size_t(C) * l * l);
       cudaMemcpyAsync(h.data(), Gm, h.size() * 4, cudaMemcpyDeviceToHost, c.st);
       cudaStreamSynchronize(c.st);
@@ -525,7 +531,7 @@ jolt_status orth(const Ctx& c, float* Yf, int* cur, int rows, int C, bool polish
         return JOLT_ERR_NUMERIC;
       }
     }
-    if (std::getenv("JOLT_DEBUG"))
+    if (kDebug)
       std::fprintf(stderr, "jolt orth: rows %d pass %d shift %g min pivot ratio %g\n", rows, pass, shift, ratio);
     GemmCall t;
     t.M = rows; t.N = l; t.K = l; t.n_terms = polish ? 3 : 2;
@@ -546,7 +552,7 @@ jolt_status orth(const Ctx& c, float* Yf, int* cur, int rows, int C, bool polish
     }
     t.ldc = l; t.c_batch_stride = int64_t(rows) * l; t.batch = C; t.err = c.err;
     t.b_upper = true;  // R^-1 is upper triangular
-    if ((r = gemm_tc(t, c.st))) return r;
+    if ((r = run_gemm(c, t))) return r;
     if (cur) *cur = b;
     if (shift == 0.0 && ratio >= 0.9f) return JOLT_OK;
     if (!polish && ratio >= 0.1f) return JOLT_OK;
@@ -597,7 +603,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
     }
     g.C = Sd; g.ldc = d; g.c_batch_stride = int64_t(d) * d; g.c_batch_div = p.LgH;
     g.batch = C * p.LgH; g.k_split = 0; g.accumulate = true; g.err = c.err;
-    if ((r = gemm_tc(g, c.st))) return r;
+    if ((r = run_gemm(c, g))) return r;
   }
   const bool exact = (p.l == p.n);
   if (exact && q > 0) {
@@ -656,7 +662,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       g.Ch = Yh_b[0];
       g.Cl = s.power_iters == 0 ? Yl_b[0] : nullptr;
       g.ldc = l; g.c_batch_stride = int64_t(T) * l; g.batch = C; g.err = c.err;
-      if ((r = gemm_tc(g, c.st))) return r;
+      if ((r = run_gemm(c, g))) return r;
     }
     for (int it = 0; it < s.power_iters; ++it) {
       if ((r = orth(c, nullptr, &cur, T, C, false))) return r;
@@ -667,7 +673,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       g.B[0] = plain(Yh_b[cur], kMajorMN, l, T, l, C, int64_t(T) * l);
       g.C = Z; g.ldc = l; g.c_batch_stride = int64_t(n) * l; g.batch = C;
       g.k_split = 0; g.accumulate = true; g.err = c.err;
-      if ((r = gemm_tc(g, c.st))) return r;
+      if ((r = run_gemm(c, g))) return r;
       if ((r = orth(c, Z, nullptr, n, C, false))) return r;
       if ((r = split_bf16(Z, l, n, l, C, int64_t(n) * l, Zh, nullptr, l, int64_t(n) * l, c.st))) return r;
       GemmCall h;
@@ -678,7 +684,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       h.Ch = Yh_b[0];
       h.Cl = it + 1 == s.power_iters ? Yl_b[0] : nullptr;
       h.ldc = l; h.c_batch_stride = int64_t(T) * l; h.batch = C; h.err = c.err;
-      if ((r = gemm_tc(h, c.st))) return r;
+      if ((r = run_gemm(c, h))) return r;
     }
     if ((r = orth(c, nullptr, &cur, T, C, true))) return r;  // Q, as hi / lo parts in buffer cur
     __nv_bfloat16* Yh = Yh_b[cur];
@@ -699,7 +705,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       }
       g.C = Z; g.ldc = l; g.c_batch_stride = int64_t(n) * l; g.batch = C;
       g.k_split = 0; g.accumulate = true; g.err = c.err;
-      if ((r = gemm_tc(g, c.st))) return r;
+      if ((r = run_gemm(c, g))) return r;
     }
     // W = B B^T = (B^T)^T (B^T), hi/lo terms
     if ((r = split_bf16(Z, l, n, l, C, int64_t(n) * l, Zh, Zl, l, int64_t(n) * l, c.st))) return r;
@@ -716,7 +722,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       g.C = W; g.ldc = l; g.c_batch_stride = int64_t(l) * l; g.batch = C;
       g.k_split = 0; g.accumulate = true; g.err = c.err;
       g.c_upper = true;  // symmetric: the eigensolver reads the upper triangle
-      if ((r = gemm_tc(g, c.st))) return r;
+      if ((r = run_gemm(c, g))) return r;
     }
     float* ev = c.at<float>(p.ev);
     float* evec = c.at<float>(p.evec);
@@ -737,7 +743,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       g.A[1] = qh; g.B[1] = vl;
       g.A[2] = ql; g.B[2] = vh;
       g.C = Ut; g.ldc = q; g.c_batch_stride = 2 * int64_t(T) * q; g.batch = C; g.err = c.err;
-      if ((r = gemm_tc(g, c.st))) return r;
+      if ((r = run_gemm(c, g))) return r;
     }
     std::vector<float> e32(size_t(C) * l);
     JOLT_CUDA_TRY(cudaMemcpyAsync(e32.data(), ev, size_t(C) * l * 4, cudaMemcpyDeviceToHost, c.st));
@@ -857,18 +863,18 @@ jolt_status analyze_impl(const jolt_shape* shape, const void* k, const void* v, 
       std::vector<double> nrm;
       jolt_status r = analyze_pass(c, kv ? v : k, kv, bg0, C, evT, evD, nrm);
       if (r) {
-        if (std::getenv("JOLT_DEBUG")) std::fprintf(stderr, "jolt analyze: pass kv %d bg0 %d status %d\n", kv, bg0, int(r));
+        if (kDebug) std::fprintf(stderr, "jolt analyze: pass kv %d bg0 %d status %d\n", kv, bg0, int(r));
         return r;
       }
       if ((r = read_err(c))) {
-        if (std::getenv("JOLT_DEBUG")) std::fprintf(stderr, "jolt analyze: device error %d after pass kv %d bg0 %d\n", int(r), kv, bg0);
+        if (kDebug) std::fprintf(stderr, "jolt analyze: device error %d after pass kv %d bg0 %d\n", int(r), kv, bg0);
         return r;
       }
       for (int i = 0; i < C; ++i) {
         const int cell = (bg0 + i) * 2 + kv;
         const double n2 = nrm[i];
         if (!std::isfinite(n2)) {
-          if (std::getenv("JOLT_DEBUG")) std::fprintf(stderr, "jolt analyze: cell %d norm2 %g\n", cell, n2);
+          if (kDebug) std::fprintf(stderr, "jolt analyze: cell %d norm2 %g\n", cell, n2);
           return JOLT_ERR_NUMERIC;
         }
         norm2_out[cell] = n2;
@@ -1089,7 +1095,7 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
         g.n_terms = nt;
         g.C = ylh; g.ldc = d; g.c_batch_stride = int64_t(rT) * d; g.batch = LgH;
         g.k_split = 0; g.accumulate = true; g.err = c.err;
-        if ((r = gemm_tc(g, c.st))) return r;
+        if ((r = run_gemm(c, g))) return r;
       }
       float* sy = c.atc<float>(p.sy) + int64_t(slot) * d * d;
       JOLT_CUDA_TRY(cudaMemsetAsync(sy, 0, size_t(d) * d * 4, c.st));
@@ -1178,11 +1184,11 @@ extern "C" jolt_status jolt_compress(const jolt_shape* shape, const void* k, con
             g.res = &e;
             const int64_t rows = int64_t(LgH) * T;
             StatScope sc(JOLT_K_RESIDUAL, c.st, 0.0, double(rows) * d * (io32 ? 4 : 2) + double(rows) * (d * ch.b / 8 + 4));
-            if ((r = gemm_tc(g, c.st))) return r;
+            if ((r = run_gemm(c, g))) return r;
             coded = true;
           } else {
             g.C = xt; g.ldc = d; g.c_batch_stride = int64_t(T) * d;
-            if ((r = gemm_tc(g, c.st))) return r;
+            if ((r = run_gemm(c, g))) return r;
             Xt = xt;
           }
         }

@@ -728,7 +728,7 @@ jolt_status launch_keys(const KeysMaps& maps, const KeysArgs& a, cudaStream_t st
   cudaFuncAttributes fa;
   JOLT_CUDA_TRY(cudaFuncGetAttributes(&fa, kern));
   if (fa.maxThreadsPerBlock < KeysCfg<NT>::kThreads) {  // the block would not fit the register file
-    if (std::getenv("JOLT_DEBUG"))
+    if (kDebug)
       std::fprintf(stderr, "jolt: k_keys_tc needs %d threads, registers allow %d (%d per thread)\n",
                    KeysCfg<NT>::kThreads, fa.maxThreadsPerBlock, fa.numRegs);
     return JOLT_ERR_CUDA;
@@ -738,7 +738,7 @@ jolt_status launch_keys(const KeysMaps& maps, const KeysArgs& a, cudaStream_t st
   kern<<<ntiles, KeysCfg<NT>::kThreads, KeysCfg<NT>::kSmem, st>>>(maps, a);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
-    if (std::getenv("JOLT_DEBUG")) std::fprintf(stderr, "jolt: k_keys_tc launch: %s\n", cudaGetErrorString(e));
+    if (kDebug) std::fprintf(stderr, "jolt: k_keys_tc launch: %s\n", cudaGetErrorString(e));
     return JOLT_ERR_CUDA;
   }
   return JOLT_OK;
@@ -831,6 +831,7 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
                        int64_t(ck.r_T) * ck.r_d);
           gc.B[0] = op(ck.Ud, kMajorK, ck.r_d, kD, ck.r_d);
           gc.C = bh; gc.ldc = kD; gc.c_batch_stride = int64_t(qc) * kD; gc.batch = nl * n_kv; gc.err = p.err;
+          gc.plan = s.gemm_plan;
           if ((r = gemm_tc(gc, st))) return r;
           const int64_t nb = int64_t(nl) * n_kv * qc * kD;
           {
@@ -856,10 +857,10 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
         ka.q = qall + row0 * kD;
         ka.pos0 = p.pos_offset; ka.rope_scaling = p.rope_scaling; ka.inv_freq = p.inv_freq;
         ka.scores = scores; ka.err = p.err;
-        // algorithmic work of the launch: the U_T^K rows once, each pair's residual rows; the
-        // tensor flops of the two B_h terms
+        // algorithmic work of the launch: the U_T^K rows once, each pair's residual rows
         const double kbytes = 2.0 * T * ck.r_T + (ck.bits ? double(nl) * n_kv * T * (kD * ck.bits / 8 + 4) : 0.0);
-        StatScope sc(JOLT_K_DECODE_MAIN, st, 2.0 * 2.0 * T * ck.r_T * kD * nl * n_kv, kbytes);
+        // the key rebuild once per (token, layer, KV head); issued: both bf16 terms of B_h
+        StatScope sc(JOLT_K_DECODE_MAIN, st, 2.0 * T * ck.r_T * kD * nl * n_kv, kbytes, 2.0 * 2.0 * T * ck.r_T * kD * nl * n_kv);
         if ((r = launch_keys_bits<2>(ck.bits, maps, ka, st))) return r;
       } else {
         if (ck.r_T > 0) {
@@ -870,6 +871,7 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
           gc.B[0] = op(ck.Ut, kMajorK, ck.r_T, T, ck.r_T);
           gc.B[1] = gc.B[0];
           gc.C = scores; gc.ldc = T; gc.err = p.err;
+          gc.plan = s.gemm_plan;
           if ((r = gemm_tc(gc, st))) return r;
         }
         ResArgs ra{};
@@ -902,7 +904,8 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
         gc.C = W; gc.ldc = qc; gc.err = p.err;
         gc.k_split = 0;  // split K to fill whole waves
         gc.accumulate = true;
-        if ((r = gemm_tc(gc, st))) return r;
+        gc.plan = s.gemm_plan;
+          if ((r = gemm_tc(gc, st))) return r;
       }
       StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
       if (cv.bits) {

@@ -824,7 +824,7 @@ bool make_tensor_map(CUtensorMap* m, const Operand& o, int rows) {
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(o.ptr), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS && std::getenv("JOLT_DEBUG")) {
+  if (r != CUDA_SUCCESS && kDebug) {
     std::fprintf(stderr, "jolt: tensor map rejected (CUresult %d) rank %d dims", int(r), rank);
     for (int i = 0; i < rank; ++i) std::fprintf(stderr, " %llu", (unsigned long long)dims[i]);
     std::fprintf(stderr, " box");
@@ -886,7 +886,7 @@ bool make_tensor_map_mn_chunks(CUtensorMap* m, const void* ptr, int64_t K, int64
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS && std::getenv("JOLT_DEBUG"))
+  if (r != CUDA_SUCCESS && kDebug)
     std::fprintf(stderr, "jolt: chunked MN tensor map rejected (CUresult %d)\n", int(r));
   return r == CUDA_SUCCESS;
 }
@@ -897,23 +897,17 @@ namespace {
 // minimise the estimated time, i.e. whole waves of one CTA per SM x (k-blocks per CTA + 1 for
 // its epilogue) over the relative per-SM speed (two accumulators sharing B run ~1.2x the flops
 // per cycle of one). Tiles a symmetric (c_upper) output skips are not counted.
-// The persistent forms (JOLT_GEMM_PLAN=p1: single CTAs, p2: CTA pairs; N > 128 and more than one
-// 128-row tile) are faster in isolation at a fixed clock, but in a whole compression pass under
-// the board's power cap they lower the clock the rest of the pass runs at by more than they
-// gain, so the one-tile kernel is the default (JOLT_GEMM_PLAN=1sm names it explicitly).
+// The persistent forms (JOLT_GEMM_PERSISTENT: single CTAs, JOLT_GEMM_PAIRS: CTA pairs; N > 128 and
+// more than one 128-row tile) are faster in isolation at a fixed clock, but in a whole compression
+// pass under the board's power cap they lower the clock the rest of the pass runs at by more than
+// they gain, so the one-tile kernel is the default.
 struct TilePlan {
   int kind, MT, k_split;  // kind: 0 one tile per CTA, 2 persistent single CTA, 3 persistent pair
 };
 
 TilePlan plan_tiles(const GemmCall& g, int BN) {
   constexpr int kSMs = 148;
-  const char* force = std::getenv("JOLT_GEMM_PLAN");
-  int only = -1;
-  if (force) {
-    if (!std::strcmp(force, "1sm")) only = 0;
-    else if (!std::strcmp(force, "p1")) only = 2;
-    else if (!std::strcmp(force, "p2")) only = 3;
-  }
+  int only = g.plan == JOLT_GEMM_PERSISTENT ? 2 : g.plan == JOLT_GEMM_PAIRS ? 3 : 0;
   const bool pers_ok = BN == 256 && g.M > BM;
   if (only < 0 || !pers_ok) only = 0;
   const int64_t ntile = (g.N + BN - 1) / BN, kb = (g.K + BK - 1) / BK;
@@ -979,8 +973,8 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   TmaPack maps;
   memset(&maps, 0, sizeof(maps));
   GemmDev d{};
-  const char* nochunk = std::getenv("JOLT_GEMM_NO_CHUNKED");  // per-chunk copies only (tests compare both)
-  const bool try_chunk = tp.kind == 0 && !(nochunk && nochunk[0] == '1');
+  // MN-major operands as one multi-chunk copy per stage unless the call asks for per-chunk copies
+  const bool try_chunk = tp.kind == 0 && g.plan != JOLT_GEMM_PER_CHUNK;
   for (int t = 0; t < g.n_terms; ++t) {
     d.a_chunk[t] = try_chunk && g.A[t].major == kMajorMN && make_tensor_map_chunked(&maps.a[t], g.A[t], BM * tp.MT);
     d.b_chunk[t] = try_chunk && g.B[t].major == kMajorMN && make_tensor_map_chunked(&maps.b[t], g.B[t], BN);
@@ -1027,9 +1021,11 @@ jolt_status gemm_tc(const GemmCall& g, cudaStream_t st) {
   } else if (gy > 65535 || zc > 65535) {
     return JOLT_ERR_INVALID_ARG;
   }
-  // algorithmic flops: a triangular B or a wanted upper triangle of C halves the product
+  // algorithmic flops: the product once (its bf16 terms only restore fp32 precision of one
+  // operand), halved for a triangular B or a wanted upper triangle of C; issued: once per term
   const double tri = (g.b_upper || g.c_upper) ? 0.5 : 1.0;
-  StatScope sc(g.res ? -1 : JOLT_K_GEMM, st, tri * 2.0 * g.M * double(g.N) * g.K * g.batch * g.n_terms, 0.0);
+  const double prod = tri * 2.0 * g.M * double(g.N) * g.K * g.batch;
+  StatScope sc(g.res ? -1 : JOLT_K_GEMM, st, prod, 0.0, prod * g.n_terms);
   if (g.res) return launch_res<1>(maps, d, grid, st);
   if (tp.kind == 3) return launch_pers<1>(am, bm, maps, d, grid, st);
   if (tp.kind == 2) return launch_pers<0>(am, bm, maps, d, grid, st);
@@ -1045,7 +1041,7 @@ extern "C" jolt_status jolt_gemm_bf16(const void* A, int32_t a_mn_major, const v
                                       int32_t b_mn_major, float* C, int32_t M, int32_t N, int32_t K,
                                       int64_t lda, int64_t ldb, int64_t ldc, int32_t batch,
                                       int64_t stride_a, int64_t stride_b, int64_t stride_c,
-                                      int32_t k_split, int32_t accumulate, void* stream) {
+                                      int32_t k_split, int32_t accumulate, int32_t plan, void* stream) {
   if (M < 0 || N < 0 || K < 0 || batch < 1 || k_split < 1) return JOLT_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return JOLT_OK;
   if (!A || !B || !C || ldc < N) return JOLT_ERR_INVALID_ARG;
@@ -1063,6 +1059,8 @@ extern "C" jolt_status jolt_gemm_bf16(const void* A, int32_t a_mn_major, const v
   if (lda < a.inner || ldb < b.inner) return JOLT_ERR_INVALID_ARG;
   g.C = C; g.ldc = ldc; g.c_batch_stride = stride_c; g.batch = batch;
   g.k_split = k_split; g.accumulate = accumulate != 0;
+  if (plan < JOLT_GEMM_DEFAULT || plan > JOLT_GEMM_PAIRS) return JOLT_ERR_INVALID_ARG;
+  g.plan = plan;
   if (k_split > 1 && !accumulate) return JOLT_ERR_INVALID_ARG;
   return gemm_tc(g, static_cast<cudaStream_t>(stream));
 }

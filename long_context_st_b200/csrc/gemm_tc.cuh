@@ -63,6 +63,7 @@ struct GemmCall {
   bool c_upper = false;        // only C[m][n] with m <= n is wanted: skip tiles entirely below the diagonal
   bool b_upper = false;        // B[k][n] = 0 for k > n (upper triangular): K stops at the tile's last column
   const ResidualEpi* res = nullptr;  // fused residual coding instead of any C output (see above)
+  int plan = 0;                // jolt_gemm_plan: kernel form (0 = the tile planner's default)
   int32_t* err = nullptr;
 };
 

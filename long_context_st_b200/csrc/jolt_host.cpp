@@ -31,6 +31,7 @@ bool shape_ok(const jolt_shape* s) {
   if (!(s->attn_scale > 0.f) || !std::isfinite(s->attn_scale)) return false;
   if (!std::isfinite(s->rope_attention_scaling)) return false;
   if (s->T > (1 << 24)) return false;
+  if (s->gemm_plan < JOLT_GEMM_DEFAULT || s->gemm_plan > JOLT_GEMM_PAIRS) return false;
   return true;
 }
 

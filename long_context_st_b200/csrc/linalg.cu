@@ -899,11 +899,7 @@ jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shi
   a.Gd = s.Gd; a.Xd = s.Xd; a.md = s.mdiag; a.diag0 = s.diag0; a.ratio = s.ratio;
   a.hi = rinv_hi; a.lo = rinv_lo;
   a.bar = GridBar{s.bar, s.bar + 1, err};
-  // diagnostics (JOLT_DEBUG): per-phase device timestamps of block 0
-  static unsigned long long* dbg_stamps = nullptr;
-  const bool dbg = std::getenv("JOLT_DEBUG") != nullptr;
-  if (dbg && !dbg_stamps) JOLT_CUDA_TRY(cudaMalloc(&dbg_stamps, 4096 * sizeof(unsigned long long)));
-  a.stamps = dbg ? dbg_stamps : nullptr;
+  a.stamps = nullptr;
   jolt_status r;
   {
     // fp64 work: factor n^3/3 plus triangular inverse n^3/3 per matrix
@@ -911,23 +907,6 @@ jolt_status chol_inverse(const float* G, int64_t ld_g, int nb, int n, double shi
     r = launch_coop(k_chol_coop, a, 2 * NB * (NB + 1) * 8, st);
   }
   if (r) return r;
-  if (dbg) {
-    std::vector<unsigned long long> h(4096);
-    JOLT_CUDA_TRY(cudaMemcpyAsync(h.data(), dbg_stamps, h.size() * 8, cudaMemcpyDeviceToHost, st));
-    JOLT_CUDA_TRY(cudaStreamSynchronize(st));
-    // stamps: start, after copy, diag 0, per step (panel, update + next diag), per diagonal, end
-    const int ns = 3 + 2 * (P - 1) + (P - 1) + 1;
-    double fac[2] = {0, 0}, inv = 0;
-    int k = 3;
-    for (int p = 0; p + 1 < P; ++p)
-      for (int ph = 0; ph < 2; ++ph, ++k) fac[ph] += (h[k] - h[k - 1]) * 1e-3;
-    for (int d = 1; d < P; ++d, ++k) inv += (h[k] - h[k - 1]) * 1e-3;
-    std::fprintf(stderr,
-                 "jolt chol: n %d batch %d total %.1f us | norm+copy %.1f | diag0 %.1f panel %.1f update+diag %.1f | "
-                 "trinv %.1f | out %.1f (stamps %d) | empty grid barrier %.2f us\n",
-                 n, nb, (h[ns - 1] - h[0]) * 1e-3, (h[1] - h[0]) * 1e-3, (h[2] - h[1]) * 1e-3, fac[0], fac[1], inv,
-                 (h[ns - 1] - h[ns - 2]) * 1e-3, ns, (h[4001] - h[4000]) * 1e-5);
-  }
   if (min_ratio) {
     std::vector<float> h(nb);
     JOLT_CUDA_TRY(cudaMemcpyAsync(h.data(), s.ratio, sizeof(float) * nb, cudaMemcpyDeviceToHost, st));
@@ -962,25 +941,18 @@ jolt_status jacobi_impl(const TA* A, int64_t ld_a, int nb, int n, TO* evals, TO*
   a.tol = tol;
   a.sweeps_done = s.sweeps;
   a.bar = GridBar{s.bar, s.bar + 1, err};
-  static unsigned long long* jdbg = nullptr;
-  const bool dbg = std::getenv("JOLT_DEBUG") != nullptr;
-  if (dbg && !jdbg) JOLT_CUDA_TRY(cudaMalloc(&jdbg, 4 * sizeof(unsigned long long)));
-  if (dbg) JOLT_CUDA_TRY(cudaMemsetAsync(jdbg, 0, 4 * sizeof(unsigned long long), st));
-  a.stamps = dbg ? jdbg : nullptr;
+  a.stamps = nullptr;
   jolt_status r;
   {
     StatScope sc(JOLT_K_EIG, st, 0.0, 0.0);
     r = launch_coop(k_jac_coop, a, 3 * JS * (JS + 1) * 8, st);
   }
   if (r) return r;
-  if (std::getenv("JOLT_DEBUG")) {
+  if (kDebug) {
     int sw = 0;
     JOLT_CUDA_TRY(cudaMemcpyAsync(&sw, s.sweeps, sizeof(int), cudaMemcpyDeviceToHost, st));
     JOLT_CUDA_TRY(cudaStreamSynchronize(st));
-    unsigned long long h[4] = {0, 0, 0, 0};
-    JOLT_CUDA_TRY(cudaMemcpy(h, jdbg, sizeof(h), cudaMemcpyDeviceToHost));
-    std::fprintf(stderr, "jolt jacobi: n %d batch %d sweeps %d | solve %.1f us update %.1f us\n", n, nb, sw,
-                 h[0] * 1e-3, h[1] * 1e-3);
+    std::fprintf(stderr, "jolt jacobi: n %d batch %d sweeps %d\n", n, nb, sw);
   }
   k_jac_sort<<<dim3((n + 255) / 256, nb), 256, 0, st>>>(s.A, np, n, evals, s.perm);
   k_jac_out<<<dim3(grid_1d(int64_t(n) * n), nb), 256, 0, st>>>(s.V, np, n, s.perm, evecs);

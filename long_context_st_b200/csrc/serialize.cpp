@@ -10,7 +10,7 @@ namespace jolt {
 namespace {
 
 constexpr char kMagic[8] = {'J', 'O', 'L', 'T', 'C', 'A', 'C', 'H'};
-constexpr uint32_t kVersion = 1;
+constexpr uint32_t kVersion = 2;
 
 uint64_t header_bytes(int n_cells) {
   const uint64_t raw = 16 + sizeof(jolt_shape) + 4 + uint64_t(n_cells) * sizeof(jolt_cell_choice) + 8;

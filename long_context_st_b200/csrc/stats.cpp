@@ -10,11 +10,11 @@ namespace {
 struct Pending {
   int fam;
   cudaEvent_t e0, e1;
-  double flops, bytes;
+  double flops, bytes, issued;
 };
 struct Acc {
   uint64_t launches = 0;
-  double ms = 0, flops = 0, bytes = 0;
+  double ms = 0, flops = 0, bytes = 0, issued = 0;
 };
 std::mutex g_mu;
 bool g_on = false;
@@ -39,8 +39,8 @@ bool stats_on() {
   return g_on;
 }
 
-StatScope::StatScope(int family, cudaStream_t st, double flops, double bytes)
-    : fam_(family), st_(st), flops_(flops), bytes_(bytes) {
+StatScope::StatScope(int family, cudaStream_t st, double flops, double bytes, double issued)
+    : fam_(family), st_(st), flops_(flops), bytes_(bytes), issued_(issued < 0.0 ? flops : issued) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_on || family < 0) return;  // family < 0: not recorded (the caller's own scope covers it)
   e0_ = take_event();
@@ -52,7 +52,7 @@ StatScope::~StatScope() {
   if (!e0_ || !e1_) return;
   cudaEventRecord(e1_, st_);
   std::lock_guard<std::mutex> lk(g_mu);
-  g_pending.push_back(Pending{fam_, e0_, e1_, flops_, bytes_});
+  g_pending.push_back(Pending{fam_, e0_, e1_, flops_, bytes_, issued_});
 }
 
 }  // namespace jolt
@@ -76,6 +76,7 @@ extern "C" jolt_status jolt_stats_read(jolt_kernel_stat* out, int32_t reset) {
     a.ms += ms;
     a.flops += p.flops;
     a.bytes += p.bytes;
+    a.issued += p.issued;
     g_pool.push_back(p.e0);
     g_pool.push_back(p.e1);
   }
@@ -86,6 +87,7 @@ extern "C" jolt_status jolt_stats_read(jolt_kernel_stat* out, int32_t reset) {
     out[f].ms = g_acc[f].ms;
     out[f].flops = g_acc[f].flops;
     out[f].bytes = g_acc[f].bytes;
+    out[f].flops_issued = g_acc[f].issued;
     if (reset) g_acc[f] = Acc{};
   }
   return JOLT_OK;

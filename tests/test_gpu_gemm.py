@@ -20,18 +20,14 @@ def ref_mm(A, B, a_mn, b_mn):
                                    (4096, 256, 128), (64, 384, 200),
                                    # grids large enough for two 128-row tiles per CTA, ragged M/N/K
                                    (16000, 1152, 192), (80000, 200, 72)])
-@pytest.mark.parametrize("plan", ["auto", "1sm", "p1", "p2", "perchunk"])
-def test_gemm_majors_and_ragged(cuda_ok, monkeypatch, plan, a_mn, b_mn, M, N, K):
-    # restrict the tile plan to the one-tile kernel or the persistent single-CTA / CTA-pair forms;
-    # perchunk: the one-tile kernel copying MN-major operands one 64-wide chunk at a time
-    if plan == "perchunk":
-        monkeypatch.setenv("JOLT_GEMM_NO_CHUNKED", "1")
-    else:
-        monkeypatch.setenv("JOLT_GEMM_PLAN", plan)
+@pytest.mark.parametrize("plan", ["default", "perchunk", "persistent", "pairs"])
+def test_gemm_majors_and_ragged(cuda_ok, plan, a_mn, b_mn, M, N, K):
+    # every kernel form: the one-tile kernel (multi-chunk or per-chunk copies of MN-major operands)
+    # and the persistent single-CTA / CTA-pair forms
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K + a_mn * 2 + b_mn)
     A = torch.randn((K, M) if a_mn else (M, K), generator=g, device="cuda").to(torch.bfloat16)
     B = torch.randn((K, N) if b_mn else (N, K), generator=g, device="cuda").to(torch.bfloat16)
-    C = api.gemm_bf16(A, B, a_mn, b_mn)
+    C = api.gemm_bf16(A, B, a_mn, b_mn, plan=plan)
     torch.cuda.synchronize()
     R = ref_mm(A, B, a_mn, b_mn)
     err = (C.double() - R).abs().max().item() / R.abs().max().item()
@@ -43,15 +39,14 @@ def tol(K):
     return 2e-7 * K ** 0.5 + 1e-6
 
 
-@pytest.mark.parametrize("plan", ["1sm", "p1", "p2"])
-def test_gemm_split_k_and_batch(cuda_ok, monkeypatch, plan):
-    monkeypatch.setenv("JOLT_GEMM_PLAN", plan)
+@pytest.mark.parametrize("plan", ["default", "persistent", "pairs"])
+def test_gemm_split_k_and_batch(cuda_ok, plan):
     g = torch.Generator(device="cuda").manual_seed(1)
     bt, M, N, K = 3, 384, 256, 8192
     A = torch.randn(bt, K, M, generator=g, device="cuda").to(torch.bfloat16)
     B = torch.randn(bt, K, N, generator=g, device="cuda").to(torch.bfloat16)
     C = torch.zeros(bt, M, N, device="cuda")
-    api.gemm_bf16(A, B, True, True, C=C, k_split=8, accumulate=True)
+    api.gemm_bf16(A, B, True, True, C=C, k_split=8, accumulate=True, plan=plan)
     torch.cuda.synchronize()
     R = ref_mm(A, B, True, True)
     err = (C.double() - R).abs().max().item() / R.abs().max().item()

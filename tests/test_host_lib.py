@@ -165,7 +165,7 @@ def test_cache_blob_header_checks():
         api.cache_blob_info(np.frombuffer(b"JOLTCACH", dtype=np.uint8))  # truncated
     # a header written by hand to the documented layout is accepted; one byte short is not
     blob = np.zeros(n, dtype=np.uint8)
-    raw = bytearray(b"JOLTCACH") + (1).to_bytes(4, "little") + hdr.to_bytes(4, "little")
+    raw = bytearray(b"JOLTCACH") + (2).to_bytes(4, "little") + hdr.to_bytes(4, "little")
     raw += bytes(shape) + len(choices).to_bytes(4, "little", signed=True)
     for c in choices:
         raw += b"".join(int(v).to_bytes(4, "little", signed=True) for v in c)
@@ -176,7 +176,7 @@ def test_cache_blob_header_checks():
     with pytest.raises(api.JoltError):
         api.cache_blob_info(blob[:-1])
     bad = blob.copy()
-    bad[8] = 2                                                   # unknown version
+    bad[8] = 1                                                   # an older format version
     with pytest.raises(api.JoltError):
         api.cache_blob_info(bad)
 
