@@ -467,10 +467,13 @@ Operand xunfold(const void* X, int major, const Plan& p, int C) {
 constexpr int kMaxOrthPasses = 8;
 
 // polish = false (inside the power iterations): the basis only feeds the next product, which reads
-// its bf16 part, so the passes orthonormalise the bf16-rounded matrix itself — Gram Y_hi^T Y_hi
-// (one term, exact), Q = Y_hi (R^-1 hi + lo) — and stop after the first pass whose pivots show a
-// well-conditioned input (ratio >= 0.1). The final basis (polish = true) uses hi/lo terms
-// throughout and gets the unshifted passes.
+// its bf16 part. Rounding is harmless once the basis is well conditioned — every direction is then
+// kept to 2^-9 of itself — but not before: the product's columns are dominated by the top singular
+// directions, and those ~1e-4 of the top one in singular value fall below bf16's resolution of the
+// column. So the passes read the product's hi/lo parts (Gram and Y R^-1 in hi/lo terms, as for
+// the final basis), and stop after the first unshifted pass, i.e. once a shifted pass has made the
+// input well conditioned (ratio >= 0.1) and one more pass has orthonormalised it. The final basis
+// (polish = true) gets unshifted passes until the input was nearly orthonormal (ratio >= 0.9).
 jolt_status orth(const Ctx& c, float* Yf, int* cur, int rows, int C, bool polish = true) {
   const Plan& p = c.p;
   const int l = p.l;
@@ -485,11 +488,11 @@ jolt_status orth(const Ctx& c, float* Yf, int* cur, int rows, int C, bool polish
     __nv_bfloat16* Yh = Yh_b[b];
     __nv_bfloat16* Yl = Yl_b[b];
     jolt_status r;
-    if (Yf && (r = split_bf16(Yf, l, rows, l, C, int64_t(rows) * l, Yh, polish ? Yl : nullptr, l, int64_t(rows) * l, c.st)))
+    if (Yf && (r = split_bf16(Yf, l, rows, l, C, int64_t(rows) * l, Yh, Yl, l, int64_t(rows) * l, c.st)))
       return r;
     JOLT_CUDA_TRY(cudaMemsetAsync(Gm, 0, size_t(C) * l * l * 4, c.st));
     GemmCall g;
-    g.M = l; g.N = l; g.K = rows; g.n_terms = polish ? 3 : 1;
+    g.M = l; g.N = l; g.K = rows; g.n_terms = 3;
     const Operand yh = plain(Yh, kMajorMN, l, rows, l, C, int64_t(rows) * l);
     const Operand yl = plain(Yl, kMajorMN, l, rows, l, C, int64_t(rows) * l);
     g.A[0] = yh; g.B[0] = yh;
@@ -534,7 +537,7 @@ jolt_status orth(const Ctx& c, float* Yf, int* cur, int rows, int C, bool polish
     if (kDebug)
       std::fprintf(stderr, "jolt orth: rows %d pass %d shift %g min pivot ratio %g\n", rows, pass, shift, ratio);
     GemmCall t;
-    t.M = rows; t.N = l; t.K = l; t.n_terms = polish ? 3 : 2;
+    t.M = rows; t.N = l; t.K = l; t.n_terms = 3;
     const Operand ykh = plain(Yh, kMajorK, l, rows, l, C, int64_t(rows) * l);
     const Operand ykl = plain(Yl, kMajorK, l, rows, l, C, int64_t(rows) * l);
     const Operand rh = plain(Rh, kMajorMN, l, l, l, C, int64_t(l) * l);
@@ -548,14 +551,14 @@ jolt_status orth(const Ctx& c, float* Yf, int* cur, int rows, int C, bool polish
       // the product cannot overwrite the parts it reads: write the other buffer
       b ^= 1;
       t.Ch = Yh_b[b];
-      t.Cl = polish ? Yl_b[b] : nullptr;
+      t.Cl = Yl_b[b];
     }
     t.ldc = l; t.c_batch_stride = int64_t(rows) * l; t.batch = C; t.err = c.err;
     t.b_upper = true;  // R^-1 is upper triangular
     if ((r = run_gemm(c, t))) return r;
     if (cur) *cur = b;
     if (shift == 0.0 && ratio >= 0.9f) return JOLT_OK;
-    if (!polish && ratio >= 0.1f) return JOLT_OK;
+    if (!polish && shift == 0.0) return JOLT_OK;
     if (ratio >= 0.1f) conditioned = true;
   }
   return JOLT_OK;
@@ -649,9 +652,8 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
     __nv_bfloat16* Zh = c.at<__nv_bfloat16>(p.Zh);
     __nv_bfloat16* Zl = c.at<__nv_bfloat16>(p.Zl);
     const __nv_bfloat16* om = c.at<__nv_bfloat16>(p.om);
-    // The sketch Y lives only as bf16 hi (/ lo) parts written by the GEMM epilogues (its fp32 value
-    // is never needed beyond its split). The lo part is kept where the next step reads it: before
-    // the final (polished) orthonormalisation.
+    // The sketch Y lives only as bf16 hi and lo parts written by the GEMM epilogues (its fp32 value
+    // is never needed beyond its split); every orthonormalisation reads both.
     int cur = 0;
     // Y = X Omega
     {
@@ -660,7 +662,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       g.A[0] = xunfold(Xb, kMajorK, p, C);
       g.B[0] = plain(om, kMajorK, n, l, n);
       g.Ch = Yh_b[0];
-      g.Cl = s.power_iters == 0 ? Yl_b[0] : nullptr;
+      g.Cl = Yl_b[0];
       g.ldc = l; g.c_batch_stride = int64_t(T) * l; g.batch = C; g.err = c.err;
       if ((r = run_gemm(c, g))) return r;
     }
@@ -682,7 +684,7 @@ jolt_status analyze_pass(const Ctx& c, const void* Xkind, int kv, int bg0, int C
       h.B[0] = plain(Zh, kMajorMN, l, n, l, C, int64_t(n) * l);
       cur = 0;
       h.Ch = Yh_b[0];
-      h.Cl = it + 1 == s.power_iters ? Yl_b[0] : nullptr;
+      h.Cl = Yl_b[0];
       h.ldc = l; h.c_batch_stride = int64_t(T) * l; h.batch = C; h.err = c.err;
       if ((r = run_gemm(c, h))) return r;
     }
