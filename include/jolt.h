@@ -382,8 +382,12 @@ jolt_status jolt_sym_eig(const float* A, int32_t n, int32_t batch, float* evals,
  * handed a stream but no allocator, or a serving loop whose device memory is planned up front and
  * where an allocation would synchronise the device or fail under memory pressure.
  *   - Every GPU that loads the library reserves the 32 MiB until the process exits.
- *   - The first call on a device looks up the array's device address (once per device, with that
- *     device current); make that first call before any stream capture.
+ *   - The first call on a device looks up the array's device address (once per device and
+ *     context, with that device current); make that first call before any stream capture. A
+ *     context the device gets later (after cudaDeviceReset, say) is noticed and the address looked
+ *     up again on the next call, which then must also come before any capture.
+ *   - Arguments are checked as jolt_decode_attn checks them (JOLT_ERR_INVALID_ARG) before the
+ *     scratch size.
  *   - A call whose scratch would exceed 32 MiB (jolt_workspace_bytes-style sizing for its
  *     n_layers_call) returns JOLT_ERR_WORKSPACE before launching anything: use smaller
  *     n_layers_call or jolt_decode_attn with your own workspace.

@@ -1,4 +1,6 @@
 // jolt_decode_attn: argument checks, workspace carving, split choice and kernel dispatch.
+#include <cuda.h>
+
 #include <algorithm>
 #include <mutex>
 #include <vector>
@@ -57,21 +59,34 @@ size_t decode_workspace_bytes(const jolt_shape& s) {
 
 using namespace jolt;
 
+namespace {
+
+// The argument checks every decode entry makes before it looks at workspaces.
+bool decode_args_ok(const jolt_shape* shape, const jolt_cell_choice* choices, const void* cache, int32_t layer_begin,
+                    int32_t n_layers_call, const void* q, const void* out, const float* inv_freq, int32_t pos_offset) {
+  if (!shape_ok(shape) || !choices || !cache || !q || !out) return false;
+  const jolt_shape& s = *shape;
+  if (layer_begin < 0 || n_layers_call < 1 || layer_begin + n_layers_call > s.n_layers) return false;
+  if (s.keys_pre_rope && !inv_freq) return false;
+  if (pos_offset < 0 || int64_t(pos_offset) + s.T > (int64_t(1) << 24)) return false;
+  const int nc = n_cells(s);
+  for (int c = 0; c < nc; ++c)
+    if (!choice_ok(s, choices[c])) return false;
+  // the tensor-core paths read the cache with 16-byte vector loads and TMA
+  if (decode_tc_supported(s) && reinterpret_cast<uintptr_t>(cache) % 16) return false;
+  return true;
+}
+
+}  // namespace
+
 extern "C" jolt_status jolt_decode_attn(const jolt_shape* shape, const jolt_cell_choice* choices,
                                         const void* cache, int32_t layer_begin, int32_t n_layers_call,
                                         const void* q, void* out, float* lse, const float* inv_freq,
                                         int32_t pos_offset, void* ws, size_t ws_bytes, void* stream) {
-  if (!shape_ok(shape) || !choices || !cache || !q || !out || !ws) return JOLT_ERR_INVALID_ARG;
-  const jolt_shape& s = *shape;
-  if (layer_begin < 0 || n_layers_call < 1 || layer_begin + n_layers_call > s.n_layers)
+  if (!ws || !decode_args_ok(shape, choices, cache, layer_begin, n_layers_call, q, out, inv_freq, pos_offset))
     return JOLT_ERR_INVALID_ARG;
-  if (s.keys_pre_rope && !inv_freq) return JOLT_ERR_INVALID_ARG;
-  if (pos_offset < 0 || int64_t(pos_offset) + s.T > (int64_t(1) << 24)) return JOLT_ERR_INVALID_ARG;
+  const jolt_shape& s = *shape;
   const int nc = n_cells(s);
-  for (int c = 0; c < nc; ++c)
-    if (!choice_ok(s, choices[c])) return JOLT_ERR_INVALID_ARG;
-  // the tensor-core path reads the cache with 16-byte vector loads and TMA
-  if (decode_tc_supported(s) && reinterpret_cast<uintptr_t>(cache) % 16) return JOLT_ERR_INVALID_ARG;
   const int Lc = n_layers_call;
   const int S = choose_splits(s, Lc);
   const DecodeWs wl = decode_ws_layout(s, Lc, S);
@@ -214,6 +229,21 @@ constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
+CUcontext g_noalloc_ctx[kMaxDevices] = {};  // the context the address was looked up in
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  return fn;
+}
 }  // namespace
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
@@ -222,8 +252,7 @@ extern "C" jolt_status jolt_decode_attn_noalloc(const jolt_shape* shape, const j
                                                 const void* cache, int32_t layer_begin, int32_t n_layers_call,
                                                 const void* q, void* out, float* lse, const float* inv_freq,
                                                 int32_t pos_offset, void* stream) {
-  if (!shape_ok(shape) || !choices || !cache || !q || !out) return JOLT_ERR_INVALID_ARG;
-  if (layer_begin < 0 || n_layers_call < 1 || layer_begin + n_layers_call > shape->n_layers)
+  if (!decode_args_ok(shape, choices, cache, layer_begin, n_layers_call, q, out, inv_freq, pos_offset))
     return JOLT_ERR_INVALID_ARG;
   // the scratch this call needs must fit the static array
   if (decode_ws_layout(*shape, n_layers_call, choose_splits(*shape, n_layers_call)).total > kNoAllocScratchBytes)
@@ -233,12 +262,17 @@ extern "C" jolt_status jolt_decode_attn_noalloc(const jolt_shape* shape, const j
   if (dev < 0 || dev >= kMaxDevices) return JOLT_ERR_INVALID_ARG;
   void* ws = nullptr;
   {
+    // the address is looked up once per device and context: a context the device got since (after
+    // cudaDeviceReset, say) holds the array at a new address
+    CUcontext ctx = nullptr;
+    if (CtxGetCurrentFn get = ctx_get_current_fn()) get(&ctx);
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    if (!g_noalloc_ptr[dev] || g_noalloc_ctx[dev] != ctx) {
       void* ptr = nullptr;
       const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
       if (e != cudaSuccess || !ptr) return JOLT_ERR_CUDA;
       g_noalloc_ptr[dev] = ptr;
+      g_noalloc_ctx[dev] = ctx;
     }
     ws = g_noalloc_ptr[dev];
   }

@@ -241,3 +241,23 @@ def test_coordinate_allocator_bit_exact_vs_oracle(seed):
         ex, _, tot_e = api.allocate(s, n2, tT, td, phi, budget)
         from oracle.alloc import evaluate
         assert evaluate(opts, got)[1] >= evaluate(opts, ex)[1] * (1 - 1e-12) or tot_g > tot_e
+
+
+def test_noalloc_decode_checks_arguments_before_scratch_size():
+    # host-only paths: a malformed call is JOLT_ERR_INVALID_ARG even when its scratch would also
+    # exceed the built-in array; a well-formed oversized call is JOLT_ERR_WORKSPACE. Neither
+    # reaches the device (fake, non-null pointers).
+    import ctypes as C
+    from long_context_st_b200._lib import lib
+    w = get_workload("llama70b_128k")
+    s = api.make_shape(w)
+    good = api.choices_array([(256, 128, 4)] * api.n_cells(s))
+    bad = api.choices_array([(250, 128, 4)] * api.n_cells(s))   # r_T not a multiple of 16
+    fake = C.c_void_p(0x1000)
+    inv = C.c_void_p(0x2000)
+    r_bad = lib().jolt_decode_attn_noalloc(C.byref(s), bad, fake, 0, w.n_layers, fake, fake, None, inv, 0, None)
+    assert r_bad == -1
+    r_big = lib().jolt_decode_attn_noalloc(C.byref(s), good, fake, 0, w.n_layers, fake, fake, None, inv, 0, None)
+    assert r_big == -6
+    r_pos = lib().jolt_decode_attn_noalloc(C.byref(s), good, fake, 0, w.n_layers, fake, fake, None, inv, -1, None)
+    assert r_pos == -1
