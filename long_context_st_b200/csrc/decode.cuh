@@ -23,6 +23,7 @@ struct DecodeParams {
   int B, Lg, n_kv, n_q, gq, T, d_h, Lc, layer_begin, S, q_cap, pos_offset;
   int io_f32, fac_f32, pre_rope;
   int g_first, Gc;  // first group of the call and number of groups it touches
+  int skip_p;       // the query prologue leaves P to the caller (the fused path forms it itself)
   double alg_bytes; // algorithmic bytes the main kernel must read (stats only)
   CellRef cells[kMaxCallCells];  // (b * Gc + (g - g_first)) * 2 + kv
 };

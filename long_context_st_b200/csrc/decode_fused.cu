@@ -21,7 +21,7 @@
 //     b-bit field becomes an exact f16 integer with one mask-and-or and one add): the codes are
 //     never expanded to 16 bits in memory, which would cost four times their size in shared-memory
 //     traffic per contraction.
-// Warp roles (320 threads): 0 TMA producer, 1 MMA issuer (owns TMEM), 2-5 score warps (thread =
+// Warp roles (320 threads): 0 TMA producers (one lane per operand ring), 1 MMA issuer (owns TMEM), 2-5 score warps (thread =
 // token of the tile for the softmax; the same warps run the key-residual MMAs for their 32 tokens),
 // 6-9 value warps (value-residual MMAs, 32 features each).
 #include <algorithm>
@@ -349,109 +349,144 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
   const uint32_t tS = tmem, tW = tmem + 2 * 2 * kNQ;  // S: two buffers of 64 columns; W after them
 
   if (warp == 0) {
-    // ================= TMA producer =================
-    if (lane == 0) {
-      int kit = 0, vit = 0, ckit = 0, cvit = 0;
+    // ================= TMA producers: one lane per ring, each running ahead on its own =========
+    // lane 0: U_T^K + P chunks, lane 1: key code stages, lane 2: U_T^V chunks, lane 3: value code
+    // stages; a lane waits only for its own ring's free slots
+    if (lane < 4) {
       bool ok = true;
-      const uint8_t* codesK = ck.codes ? ck.codes + int64_t(ll) * NKV * a.T * rbK : nullptr;
-      const uint8_t* codesV = cv.codes ? cv.codes + int64_t(ll) * NKV * a.T * rbV : nullptr;
-      auto issue_codes = [&](const uint8_t* codes, int rb, int hps, int nj, int t0, int nv, int& cit, bool kside) {
-        for (int jb = 0; jb < nj && ok; ++jb, ++cit) {
-          const int s = cit % kCStages;
-          const uint32_t full = kside ? BCK_FULL(s) : BCV_FULL(s);
-          const uint32_t empty = kside ? BCK_EMPTY(s) : BCV_EMPTY(s);
-          if (!(ok = sm100::mbar_wait(empty, ((cit / kCStages) & 1) ^ 1, a.err))) break;
-          const int h0 = jb * hps, nh = min(hps, NKV - h0);
-          sm100::mbar_expect_tx(full, uint32_t(nh * nv * rb));
-          const uint32_t dst = sb + (kside ? kOffCK : kOffCV) + s * kCStageBytes;
-          for (int k = 0; k < nh; ++k)
-            sm100::bulk_load(dst + k * kBM * rb, codes + (int64_t(h0 + k) * a.T + t0) * rb, uint32_t(nv * rb), full);
-        }
-      };
-      auto issue_v = [&](int it) {
-        const int t0 = (tile0 + it) * kBM, nv = min(kBM, a.T - t0);
-        for (int mc = 0; mc < nmc && ok; ++mc)
-          for (int h2 = 0; h2 < 2 && ok; ++h2, ++vit) {
-            const int s = vit % kVStages;
-            if (!(ok = sm100::mbar_wait(BV_EMPTY(s), ((vit / kVStages) & 1) ^ 1, a.err))) break;
-            sm100::mbar_expect_tx(BV_FULL(s), kVStageBytes);
-            const uint32_t dst = sb + kOffV + s * kVStageBytes;
-            sm100::tma_load_3d(dst, &maps.ut[ci + 1], BV_FULL(s), mc * 128, t0 + 64 * h2, 0);
-            sm100::tma_load_3d(dst + 8192, &maps.ut[ci + 1], BV_FULL(s), mc * 128 + 64, t0 + 64 * h2, 0);
-          }
-        if (ok) issue_codes(codesV, rbV, hpsV, njV, t0, nv, cvit, false);
-      };
+      int cnt = 0;
+      const bool kside = lane < 2;
+      const FusedCell& cell = kside ? ck : cv;
+      const int rb = kside ? rbK : rbV, hps = kside ? hpsK : hpsV, nj = kside ? njK : njV;
+      const uint8_t* codes = cell.codes ? cell.codes + int64_t(ll) * NKV * a.T * rb : nullptr;
       for (int it = 0; it < ntl && ok; ++it) {
         const int t0 = (tile0 + it) * kBM, nv = min(kBM, a.T - t0);
-        for (int kb = 0; kb < nkb && ok; ++kb, ++kit) {
-          const int s = kit % kKStages;
-          if (!(ok = sm100::mbar_wait(BK_EMPTY(s), ((kit / kKStages) & 1) ^ 1, a.err))) break;
-          sm100::mbar_expect_tx(BK_FULL(s), kKStageBytes);
-          const uint32_t dst = sb + kOffK + s * kKStageBytes;
-          sm100::tma_load_3d(dst, &maps.ut[ci], BK_FULL(s), kb * kBK, t0, 0);
-          sm100::tma_load_3d(dst + kBM * kBK * 2, &maps.p, BK_FULL(s), kb * kBK, 0, bl);
+        if (lane == 0) {
+          for (int kb = 0; kb < nkb && ok; ++kb, ++cnt) {
+            const int s = cnt % kKStages;
+            if (!(ok = sm100::mbar_wait(BK_EMPTY(s), ((cnt / kKStages) & 1) ^ 1, a.err))) break;
+            sm100::mbar_expect_tx(BK_FULL(s), kKStageBytes);
+            const uint32_t dst = sb + kOffK + s * kKStageBytes;
+            sm100::tma_load_3d(dst, &maps.ut[ci], BK_FULL(s), kb * kBK, t0, 0);
+            sm100::tma_load_3d(dst + kBM * kBK * 2, &maps.p, BK_FULL(s), kb * kBK, 0, bl);
+          }
+        } else if (lane == 2) {
+          for (int mc = 0; mc < nmc && ok; ++mc)
+            for (int h2 = 0; h2 < 2 && ok; ++h2, ++cnt) {
+              const int s = cnt % kVStages;
+              if (!(ok = sm100::mbar_wait(BV_EMPTY(s), ((cnt / kVStages) & 1) ^ 1, a.err))) break;
+              sm100::mbar_expect_tx(BV_FULL(s), kVStageBytes);
+              const uint32_t dst = sb + kOffV + s * kVStageBytes;
+              sm100::tma_load_3d(dst, &maps.ut[ci + 1], BV_FULL(s), mc * 128, t0 + 64 * h2, 0);
+              sm100::tma_load_3d(dst + 8192, &maps.ut[ci + 1], BV_FULL(s), mc * 128 + 64, t0 + 64 * h2, 0);
+            }
+        } else {
+          for (int jb = 0; jb < nj && ok; ++jb, ++cnt) {
+            const int s = cnt % kCStages;
+            const uint32_t full = kside ? BCK_FULL(s) : BCV_FULL(s);
+            const uint32_t empty = kside ? BCK_EMPTY(s) : BCV_EMPTY(s);
+            if (!(ok = sm100::mbar_wait(empty, ((cnt / kCStages) & 1) ^ 1, a.err))) break;
+            const int h0 = jb * hps, nh = min(hps, NKV - h0);
+            sm100::mbar_expect_tx(full, uint32_t(nh * nv * rb));
+            const uint32_t dst = sb + (kside ? kOffCK : kOffCV) + s * kCStageBytes;
+            for (int k = 0; k < nh; ++k)
+              sm100::bulk_load(dst + k * kBM * rb, codes + (int64_t(h0 + k) * a.T + t0) * rb, uint32_t(nv * rb), full);
+          }
         }
-        if (ok) issue_codes(codesK, rbK, hpsK, njK, t0, nv, ckit, true);
-        if (it >= 1 && ok) issue_v(it - 1);
       }
-      if (ntl > 0 && ok) issue_v(ntl - 1);
       // the copies still in flight complete before the block may exit
-      for (int i = max(0, kit - kKStages); i < kit; ++i) sm100::mbar_wait(BK_FULL(i % kKStages), (i / kKStages) & 1, a.err);
-      for (int i = max(0, vit - kVStages); i < vit; ++i) sm100::mbar_wait(BV_FULL(i % kVStages), (i / kVStages) & 1, a.err);
-      for (int i = max(0, ckit - kCStages); i < ckit; ++i) sm100::mbar_wait(BCK_FULL(i % kCStages), (i / kCStages) & 1, a.err);
-      for (int i = max(0, cvit - kCStages); i < cvit; ++i) sm100::mbar_wait(BCV_FULL(i % kCStages), (i / kCStages) & 1, a.err);
+      const int depth = lane == 0 ? kKStages : lane == 2 ? kVStages : kCStages;
+      for (int i = max(0, cnt - depth); i < cnt; ++i) {
+        const int s = i % depth;
+        const uint32_t full = lane == 0 ? BK_FULL(s) : lane == 2 ? BV_FULL(s) : lane == 1 ? BCK_FULL(s) : BCV_FULL(s);
+        sm100::mbar_wait(full, (i / depth) & 1, a.err);
+      }
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
+    // Two chains share the thread: the score products S(it) (key ring) and the value products
+    // W += U_T^V^T P~(it') for the tile whose probabilities are ready (value ring). Whichever ring
+    // has a stage ready is served, so the two rings' copies overlap instead of adding up.
     if (lane == 0) {
       constexpr uint32_t idK = sm100::idesc_bf16_f32(kBM, 2 * kNQ, 0, 0);
       constexpr uint32_t idW = sm100::idesc_bf16_f32(128, kNQ, 1, 0);
       int kit = 0, vit = 0;
+      int itK = 0, kb = 0, itW = 0, wst = 0;  // score tile / chunk, value tile / stage within it
+      bool sfree = false, pready = false;
+      const int nws = 2 * nmc;                // value stages per tile
       bool ok = true;
-      auto issue_w = [&](int it) {
-        if (!(ok = sm100::mbar_wait(BP_FULL(it & 1), (it >> 1) & 1, a.err))) return;
-        sm100::tc_fence_after();
-        const uint32_t pt = sb + kOffPt + (it & 1) * kPtBytes;
-        for (int mc = 0; mc < nmc && ok; ++mc)
-          for (int h2 = 0; h2 < 2 && ok; ++h2, ++vit) {
-            const int s = vit % kVStages;
-            if (!(ok = sm100::mbar_wait(BV_FULL(s), (vit / kVStages) & 1, a.err))) break;
-            sm100::tc_fence_after();
-            const uint32_t va = sb + kOffV + s * kVStageBytes;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sm100::smem_desc_sw128(va + kk * 2048, 8192, 1024);
-              const uint64_t bd = sm100::smem_desc_sw128(pt + h2 * (kNQ * 128) + kk * 32, 16, 1024);
-              sm100::mma_bf16(tW + mc * kNQ, ad, bd, idW, (it > 0 || h2 > 0 || kk > 0) ? 1u : 0u);
-            }
-            sm100::mma_commit(BV_EMPTY(s));
-          }
-        sm100::mma_commit(BW_DONE(it & 1));
-        sm100::mma_commit(BP_EMPTY(it & 1));
-      };
-      for (int it = 0; it < ntl && ok; ++it) {
-        if (nkb) {
-          if (!(ok = sm100::mbar_wait(BS_EMPTY(it & 1), ((it >> 1) & 1) ^ 1, a.err))) break;
-          sm100::tc_fence_after();
-          const uint32_t dt = tS + (it & 1) * 2 * kNQ;
-          for (int kb = 0; kb < nkb && ok; ++kb, ++kit) {
+      uint64_t idle0 = sm100::global_ns();
+      while (ok && (itK < ntl || itW < ntl)) {
+        bool progressed = false;
+        if (itK < ntl) {
+          if (nkb == 0) {
+            ++itK;
+            progressed = true;
+          } else {
+            if (!sfree) sfree = sm100::mbar_test_wait(BS_EMPTY(itK & 1), ((itK >> 1) & 1) ^ 1);
             const int s = kit % kKStages;
-            if (!(ok = sm100::mbar_wait(BK_FULL(s), (kit / kKStages) & 1, a.err))) break;
-            sm100::tc_fence_after();
-            const uint32_t ka = sb + kOffK + s * kKStageBytes;
+            if (sfree && sm100::mbar_test_wait(BK_FULL(s), (kit / kKStages) & 1)) {
+              sm100::tc_fence_after();
+              const uint32_t dt = tS + (itK & 1) * 2 * kNQ;
+              const uint32_t ka = sb + kOffK + s * kKStageBytes;
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk) {
-              const uint64_t ad = sm100::smem_desc_sw128(ka + kk * 32, 16, 1024);
-              const uint64_t bd = sm100::smem_desc_sw128(ka + kBM * kBK * 2 + kk * 32, 16, 1024);
-              sm100::mma_bf16(dt, ad, bd, idK, (kb > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < kBK / 16; ++kk) {
+                const uint64_t ad = sm100::smem_desc_sw128(ka + kk * 32, 16, 1024);
+                const uint64_t bd = sm100::smem_desc_sw128(ka + kBM * kBK * 2 + kk * 32, 16, 1024);
+                sm100::mma_bf16(dt, ad, bd, idK, (kb > 0 || kk > 0) ? 1u : 0u);
+              }
+              sm100::mma_commit(BK_EMPTY(s));
+              ++kit;
+              if (++kb == nkb) {
+                sm100::mma_commit(BS_FULL(itK & 1));
+                kb = 0;
+                ++itK;
+                sfree = false;
+              }
+              progressed = true;
             }
-            sm100::mma_commit(BK_EMPTY(s));
           }
-          if (ok) sm100::mma_commit(BS_FULL(it & 1));
         }
-        if (it >= 1 && ok) issue_w(it - 1);
+        if (itW < ntl) {
+          if (!pready) pready = sm100::mbar_test_wait(BP_FULL(itW & 1), (itW >> 1) & 1);
+          if (pready) {
+            if (wst < nws) {
+              const int s = vit % kVStages;
+              if (sm100::mbar_test_wait(BV_FULL(s), (vit / kVStages) & 1)) {
+                sm100::tc_fence_after();
+                const int mc = wst >> 1, h2 = wst & 1;
+                const uint32_t va = sb + kOffV + s * kVStageBytes;
+                const uint32_t pt = sb + kOffPt + (itW & 1) * kPtBytes;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t ad = sm100::smem_desc_sw128(va + kk * 2048, 8192, 1024);
+                  const uint64_t bd = sm100::smem_desc_sw128(pt + h2 * (kNQ * 128) + kk * 32, 16, 1024);
+                  sm100::mma_bf16(tW + mc * kNQ, ad, bd, idW, (itW > 0 || h2 > 0 || kk > 0) ? 1u : 0u);
+                }
+                sm100::mma_commit(BV_EMPTY(s));
+                ++vit;
+                ++wst;
+                progressed = true;
+              }
+            }
+            if (wst == nws) {
+              sm100::tc_fence_after();
+              sm100::mma_commit(BW_DONE(itW & 1));
+              sm100::mma_commit(BP_EMPTY(itW & 1));
+              wst = 0;
+              ++itW;
+              pready = false;
+              progressed = true;
+            }
+          }
+        }
+        if (progressed) {
+          idle0 = sm100::global_ns();
+        } else if (sm100::global_ns() - idle0 > 2000000000ull) {
+          report_error(a.err, JOLT_ERR_TIMEOUT);
+          ok = false;
+        }
       }
-      if (ntl > 0 && ok) issue_w(ntl - 1);
       sm100::mma_commit(BDRAIN);
       sm100::mbar_wait(BDRAIN, 0, a.err);
     }
@@ -489,18 +524,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
     const __half2* szK = ck.sz ? ck.sz + int64_t(ll) * NKV * a.T : nullptr;
     const __half2* szV = cv.sz ? cv.sz + int64_t(ll) * NKV * a.T : nullptr;
 
+    // this thread's token's scale / zero pairs, loaded one tile ahead (the key ones reach the MMA
+    // lanes by shuffles)
+    uint32_t zk[NKV], zv[NKV], nzk[NKV], nzv[NKV];
+    auto load_sz = [&](int it2, uint32_t (&k_)[NKV], uint32_t (&v_)[NKV]) {
+      const int t2 = (tile0 + it2) * kBM + 32 * q + lane;
+      const bool ok2 = it2 < ntl && t2 < a.T;
+#pragma unroll
+      for (int h = 0; h < NKV; ++h) {
+        k_[h] = (bK && ok2) ? __ldg(reinterpret_cast<const uint32_t*>(szK + int64_t(h) * a.T + t2)) : 0u;
+        v_[h] = (bV && ok2) ? __ldg(reinterpret_cast<const uint32_t*>(szV + int64_t(h) * a.T + t2)) : 0u;
+      }
+    };
+    load_sz(0, nzk, nzv);
     for (int it = 0; it < ntl; ++it) {
       __syncwarp();  // every lane has read its row of the exchange buffer before it is rewritten
       const int t0 = (tile0 + it) * kBM;
       const int tl = 32 * q + lane, t = t0 + tl;
       const bool valid = t < a.T;
-      // this token's scale / zero pairs (the key ones reach the MMA lanes by shuffles)
-      uint32_t zk[NKV], zv[NKV];
 #pragma unroll
       for (int h = 0; h < NKV; ++h) {
-        zk[h] = (bK && valid) ? __ldg(reinterpret_cast<const uint32_t*>(szK + int64_t(h) * a.T + t)) : 0u;
-        zv[h] = (bV && valid) ? __ldg(reinterpret_cast<const uint32_t*>(szV + int64_t(h) * a.T + t)) : 0u;
+        zk[h] = nzk[h];
+        zv[h] = nzv[h];
       }
+      load_sz(it + 1, nzk, nzv);
       // ---- key residual: jobs of 8 / b heads per code stage ----
       if (bK) {
         const int hps = 8 / bK;
@@ -728,23 +775,68 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
   if (warp == 1) sm100::tmem_dealloc(tmem, kTmemCols);
 }
 
-// Key-cell token rank of every (sequence, layer) row of a launch set.
-struct RankTab {
-  int r_T[kMaxFusedRows];
+// One key cell's stored factors for a (sequence, layer) row of a launch set.
+struct PRow {
+  const __nv_bfloat16* G;   // G^K of the row's layer: [n_kv][r_T][r_d]
+  const __nv_bfloat16* Ud;  // U_d^K [128][r_d]
+  int r_T, r_d;
+};
+struct PTab {
+  PRow row[kMaxFusedRows];
 };
 
-// P (fp32, [B*Lc][32][q_cap]) -> bf16 hi rows then lo rows per (sequence, layer): [B*Lc][64][q_cap],
-// zero beyond the key cell's r_T (those columns meet the zero fill of U_T's tensor map)
-__global__ void k_split_p(const float* __restrict__ P, int q_cap, const RankTab rt, __nv_bfloat16* __restrict__ out) {
-  const int bl = blockIdx.y;
-  const int r_T = rt.r_T[bl];
+// P = G^K_h (U_d^K^T q) for the g_q query heads of one KV head, written as bf16 hi rows then lo rows
+// per (sequence, layer): out [B*Lc][64][q_cap], zero beyond r_T (those columns meet the zero fill
+// of U_T's tensor map). grid (n_kv, B*Lc), 256 threads: q-hat = U_d^T q for the KV head's query
+// heads in shared memory, then a warp per row r of G_h (lanes over r_d, 8-byte loads: each row
+// read once for all g_q heads) and a warp reduction per head.
+template <int GQ>
+__global__ void __launch_bounds__(256) k_prologue_p(const __nv_bfloat16* __restrict__ q, int q_cap, const PTab tab,
+                                                   __nv_bfloat16* __restrict__ out) {
+  const int h = blockIdx.x, bl = blockIdx.y;
+  const PRow pr = tab.row[bl];
+  __shared__ float qs[GQ][kD];
+  __shared__ float qh[GQ][kD];
+  for (int e = threadIdx.x; e < GQ * kD; e += blockDim.x)
+    qs[e / kD][e % kD] = __bfloat162float(q[(int64_t(bl) * kNQ + h * GQ) * kD + e]);
+  __syncthreads();
+  for (int e = threadIdx.x; e < GQ * kD; e += blockDim.x) {
+    const int j = e / kD, c = e % kD;
+    float a = 0.f;
+    if (c < pr.r_d)
+      for (int i = 0; i < kD; ++i) a = fmaf(__bfloat162float(pr.Ud[int64_t(i) * pr.r_d + c]), qs[j][i], a);
+    qh[j][c] = a;
+  }
+  __syncthreads();
   const int64_t n = int64_t(kNQ) * q_cap;
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
-    const int r = int(e % q_cap);
-    const float v = r < r_T ? P[int64_t(bl) * n + e] : 0.f;
-    const __nv_bfloat16 hh = __float2bfloat16_rn(v);
-    out[int64_t(bl) * 2 * n + e] = hh;
-    out[int64_t(bl) * 2 * n + n + e] = __float2bfloat16_rn(v - __bfloat162float(hh));
+  __nv_bfloat16* hi = out + int64_t(bl) * 2 * n;
+  __nv_bfloat16* lo = hi + n;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const __nv_bfloat16* Gh = pr.G + int64_t(h) * pr.r_T * pr.r_d;
+  for (int r = warp; r < q_cap; r += 8) {
+    float acc[GQ];
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) acc[j] = 0.f;
+    if (r < pr.r_T) {
+      for (int c0 = 4 * lane; c0 < pr.r_d; c0 += 128) {
+        const uint2 w = *reinterpret_cast<const uint2*>(Gh + int64_t(r) * pr.r_d + c0);
+        const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+        const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+#pragma unroll
+        for (int j = 0; j < GQ; ++j)
+          acc[j] = fmaf(g01.x, qh[j][c0], fmaf(g01.y, qh[j][c0 + 1], fmaf(g23.x, qh[j][c0 + 2], fmaf(g23.y, qh[j][c0 + 3], acc[j]))));
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) {
+      float v = acc[j];
+      for (int m = 16; m; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+      if (lane == j) {
+        const __nv_bfloat16 hh = __float2bfloat16_rn(v);
+        hi[int64_t(h * GQ + j) * q_cap + r] = hh;
+        lo[int64_t(h * GQ + j) * q_cap + r] = __float2bfloat16_rn(v - __bfloat162float(hh));
+      }
+    }
   }
 }
 
@@ -814,14 +906,24 @@ jolt_status launch_decode_fused(const DecodeParams& p, const TcCellView* views, 
   // ---- prologue: R q, sum(R q), P = G^K (U_d^K^T q); P as bf16 hi + lo rows ----
   {
     StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
-    if ((r = launch_decode_prologue_q(p, st))) return r;
-    RankTab rt{};
+    DecodeParams pq = p;
+    pq.skip_p = 1;
+    if ((r = launch_decode_prologue_q(pq, st))) return r;
+    static_assert(sizeof(PTab) <= 24 * 1024, "prologue parameter table");
+    PTab tab;
     for (int b = 0; b < p.B; ++b)
       for (int li = 0; li < p.Lc; ++li) {
-        const int g = (p.layer_begin + li) / p.Lg;
-        rt.r_T[b * p.Lc + li] = views[(b * p.Gc + (g - p.g_first)) * 2].r_T;
+        const int layer = p.layer_begin + li, g = layer / p.Lg, ll = layer % p.Lg;
+        const TcCellView& v = views[(b * p.Gc + (g - p.g_first)) * 2];
+        PRow& r = tab.row[b * p.Lc + li];
+        r.G = v.r_T ? v.G + int64_t(ll) * p.n_kv * v.r_T * v.r_d : nullptr;
+        r.Ud = v.Ud;
+        r.r_T = v.r_T;
+        r.r_d = v.r_d;
       }
-    k_split_p<<<dim3(std::max(1, std::min(64, (kNQ * qc + 255) / 256)), BL), 256, 0, st>>>(p.ws_P, qc, rt, hl);
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q);
+    if (p.gq == 4) k_prologue_p<4><<<dim3(p.n_kv, BL), 256, 0, st>>>(qb, qc, tab, hl);
+    else k_prologue_p<8><<<dim3(p.n_kv, BL), 256, 0, st>>>(qb, qc, tab, hl);
     JOLT_CUDA_TRY(cudaGetLastError());
   }
   // ---- tensor maps and per-cell arguments ----

@@ -55,7 +55,7 @@ __global__ void k_prologue_q(DecodeParams p) {
     sum = warp_sum(sum);
     if (threadIdx.x == 0) p.ws_qsum[qrow] = sum;
   }
-  if (p.pre_rope || ck.r_T == 0) return;
+  if (p.pre_rope || p.skip_p || ck.r_T == 0) return;
   const uint8_t* Ud = p.cache + ck.offset + so.ud;
   const uint8_t* G = p.cache + ck.offset + so.g + (int64_t(ll) * p.n_kv + h) * ck.r_T * ck.r_d *
                      (p.fac_f32 ? 4 : 2);
