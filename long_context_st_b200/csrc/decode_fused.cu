@@ -116,31 +116,35 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
 }
 
 // b-bit code fields of a word as exact f16 pairs. The mask-and-or puts each field into the
-// mantissa of 1024 (f16 0x6400), scaled by 2^shift; one fused multiply-add removes both.
-__device__ __forceinline__ uint32_t f16pair_field(uint32_t x, uint32_t mask, float inv, float off) {
-  const uint32_t v = (x & mask) | 0x64006400u;
-  __half2 h = *reinterpret_cast<const __half2*>(&v);
-  h = __hfma2(h, __float2half2_rn(inv), __float2half2_rn(off));
-  return *reinterpret_cast<const uint32_t*>(&h);
+// mantissa of 1024 (f16 0x6400), scaled by 2^shift; one f16x2 add or fused multiply-add with
+// constant pairs removes both (exact: every intermediate is a small integer or a power of two).
+__device__ __forceinline__ uint32_t h2_add(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+constexpr uint32_t kH2M1024 = 0xE400E400u;                            // (-1024, -1024)
+__device__ __forceinline__ uint32_t field_or(uint32_t x, uint32_t mask) { return (x & mask) | 0x64006400u; }
 // 4-bit fields at bits 0-3 / 16-19 (lo) or 4-7 / 20-23 (hi)
-__device__ __forceinline__ uint32_t nib_lo(uint32_t x) { return f16pair_field(x, 0x000F000Fu, 1.f, -1024.f); }
-__device__ __forceinline__ uint32_t nib_hi(uint32_t x) { return f16pair_field(x, 0x00F000F0u, 0.0625f, -64.f); }
-// 2-bit fields at bit 2s / 16 + 2s
+__device__ __forceinline__ uint32_t nib_lo(uint32_t x) { return h2_add(field_or(x, 0x000F000Fu), kH2M1024); }
+__device__ __forceinline__ uint32_t nib_hi(uint32_t x) { return h2_fma(field_or(x, 0x00F000F0u), 0x2C002C00u, 0xD400D400u); }
+// 2-bit fields at bit 2s / 16 + 2s: (1024 + 4^s c) * 4^-s - 1024 * 4^-s
 __device__ __forceinline__ uint32_t crumb(uint32_t x, int s) {
   switch (s) {
-    case 0: return f16pair_field(x, 0x00030003u, 1.f, -1024.f);
-    case 1: return f16pair_field(x, 0x000C000Cu, 0.25f, -256.f);
-    case 2: return f16pair_field(x, 0x00300030u, 0.0625f, -64.f);
-    default: return f16pair_field(x, 0x00C000C0u, 0.015625f, -16.f);
+    case 0: return h2_add(field_or(x, 0x00030003u), kH2M1024);
+    case 1: return h2_fma(field_or(x, 0x000C000Cu), 0x34003400u, 0xDC00DC00u);
+    case 2: return h2_fma(field_or(x, 0x00300030u), 0x2C002C00u, 0xD400D400u);
+    default: return h2_fma(field_or(x, 0x00C000C0u), 0x24002400u, 0xCC00CC00u);
   }
 }
-// bytes i and k of x -> f16 pair (x.byte_i, x.byte_k)
+// bytes of x chosen by sel next to 0x64 -> f16 pair (byte, byte)
 __device__ __forceinline__ uint32_t byte_pair(uint32_t x, uint32_t sel) {
-  const uint32_t v = __byte_perm(x, 0x64646464u, sel);
-  __half2 h = *reinterpret_cast<const __half2*>(&v);
-  h = __hsub2(h, __float2half2_rn(1024.f));
-  return *reinterpret_cast<const uint32_t*>(&h);
+  return h2_add(__byte_perm(x, 0x64646464u, sel), kH2M1024);
 }
 
 // Within a lane's 32-code segment of a key-residual row, pair p (16 pairs, in the order the
