@@ -54,7 +54,7 @@ constexpr int kVStageBytes = 2 * 64 * 64 * 2;                    // U_T^V: 128 r
 constexpr int kCStageBytes = 16384;                              // codes of 8/b heads x 128 tokens
 constexpr int kPtBytes = kNQ * kBM * 2;                          // P~ (bf16, K-major, 32 rows)
 constexpr int kWbBytes = kNQ * 256;                              // value weights (f16 fragments)
-constexpr int kScrStride = kNQ + 4;                              // floats per token row of the exchange
+constexpr int kScrStride = kNQ + 1;                              // floats per token row of the exchange (odd: no bank conflicts)
 constexpr int kScrBytes = 4 * 32 * kScrStride * 4;
 constexpr int kQfBytes = kNQ * 256;                              // query fragments (f16)
 
@@ -77,6 +77,7 @@ constexpr int kSmemUsed = kOffBars + kNumBars * 8 + 16;
 constexpr int kSmem = kSmemUsed + 1024;             // 1024-byte alignment of the swizzled tiles
 static_assert(kSmem <= 232448, "fused decode shared memory");
 static_assert(kOffV % 1024 == 0 && kOffPt % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(kOffCK % 16 == 0 && kOffCV % 16 == 0 && kOffBars % 8 == 0, "bulk-copy and mbarrier alignment");
 
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
@@ -289,7 +290,7 @@ template <int GQ>
 __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_constant__ FusedMaps maps, const FusedArgs a) {
   constexpr int NKV = kNQ / GQ;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = sm100::align_smem_1024(smem_raw);
   const uint32_t sb = sm100::smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
@@ -419,7 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       bool sfree = false, pready = false;
       const int nws = 2 * nmc;                // value stages per tile
       bool ok = true;
-      uint64_t idle0 = sm100::global_ns();
+      uint64_t idle0 = 0;  // start of the current idle stretch (read every 1024 idle polls)
+      int idle_polls = 0;
       while (ok && (itK < ntl || itW < ntl)) {
         bool progressed = false;
         if (itK < ntl) {
@@ -485,10 +487,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
           }
         }
         if (progressed) {
-          idle0 = sm100::global_ns();
-        } else if (sm100::global_ns() - idle0 > 2000000000ull) {
-          report_error(a.err, JOLT_ERR_TIMEOUT);
-          ok = false;
+          idle0 = 0;
+          idle_polls = 0;
+        } else if (++idle_polls == 1024) {
+          idle_polls = 0;
+          const uint64_t now = sm100::global_ns();
+          if (idle0 == 0) {
+            idle0 = now;
+          } else if (now - idle0 > 2000000000ull) {
+            report_error(a.err, JOLT_ERR_TIMEOUT);
+            ok = false;
+          }
         }
       }
       sm100::mma_commit(BDRAIN);
@@ -536,8 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       const bool ok2 = it2 < ntl && t2 < a.T;
 #pragma unroll
       for (int h = 0; h < NKV; ++h) {
-        k_[h] = (bK && ok2) ? __ldg(reinterpret_cast<const uint32_t*>(szK + int64_t(h) * a.T + t2)) : 0u;
-        v_[h] = (bV && ok2) ? __ldg(reinterpret_cast<const uint32_t*>(szV + int64_t(h) * a.T + t2)) : 0u;
+        k_[h] = (bK && ok2) ? sm100::ld_nc_early(szK + int64_t(h) * a.T + t2) : 0u;
+        v_[h] = (bV && ok2) ? sm100::ld_nc_early(szV + int64_t(h) * a.T + t2) : 0u;
       }
     };
     load_sz(0, nzk, nzv);

@@ -152,7 +152,7 @@ template <int BITS, int NT>
 __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ KeysMaps maps, const KeysArgs p) {
   using C = KeysCfg<NT>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = sm100::align_smem_1024(smem_raw);
   float* qs = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);  // [2 groups][kMaxG][kD]
   float4* rope = reinterpret_cast<float4*>(qs + 2 * kMaxG * kD);            // [32][kBM]
   float2* sgn = reinterpret_cast<float2*>(rope + kD / 4 * kBM);               // [64]

@@ -346,7 +346,7 @@ template <int BN, int AMAJ, int BMAJ, int MT, int EPI = 0>
 __global__ void __launch_bounds__(128, EPI ? 2 : 1) k_gemm(const __grid_constant__ TmaPack maps, GemmDev p) {
   using C = Cfg<BN, MT, EPI>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = sm100::align_smem_1024(smem_raw);
   float* epi = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes + C::kEpiBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 1);
@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(224, 1) k_gemm_p(const __grid_constant__ TmaPa
   constexpr int BN = C::BN;
   constexpr int ROWS = PAIR ? 2 * BM : BM;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = sm100::align_smem_1024(smem_raw);
   float* epi = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes + C::kEpiBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 4);

@@ -13,6 +13,23 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared memory rounded up to a 1024-byte boundary (swizzled TMA / UMMA tiles). The
+// offset is added to the __shared__ array itself, so every access through the result stays a
+// shared-memory access; rounding the address through an integer would make them generic loads and
+// stores, which wait on the long scoreboard.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
+// A 32-bit read-only global load issued where it stands in the program: the asm is volatile, so the
+// compiler cannot sink it next to its first use (a load meant to run a whole tile ahead would then
+// expose the full memory latency at that use).
+__device__ __forceinline__ uint32_t ld_nc_early(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
