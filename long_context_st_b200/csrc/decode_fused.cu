@@ -13,17 +13,22 @@
 //   partials (m, l, W, acc) per split go to the workspace; k_decode_merge combines the splits and
 //            applies U_d^V G^V^T and the inverse rotation.
 // Where each contraction runs:
-//   * U_T^K P (M = 128 tokens, N = 64: the 32 query heads' P as bf16 hi + lo columns, K = r_T) and
-//     W (M = 128 rank rows per chunk, N = 32 heads, K = tokens; U_T^V read MN-major, P~ K-major) on
-//     tcgen05 with TMEM accumulators, operands staged by TMA;
+//   * U_T^K P (M = 128 tokens, N = 32 query heads, K = r_T; P as bf16 hi and lo terms accumulated
+//     into the same columns) and W (M = 128 rank rows per chunk, N = 32 heads, K = tokens; U_T^V
+//     read MN-major, P~ K-major) on tcgen05 with TMEM accumulators, operands staged by TMA;
 //   * both residual contractions (codes . R q and P~-weighted codes) on mma.sync m16n8k16 with
 //     the f16 operands built in registers straight from the packed codes in shared memory (each
 //     b-bit field becomes an exact f16 integer with one mask-and-or and one add): the codes are
 //     never expanded to 16 bits in memory, which would cost four times their size in shared-memory
-//     traffic per contraction.
-// Warp roles (320 threads): 0 TMA producers (one lane per operand ring), 1 MMA issuer (owns TMEM), 2-5 score warps (thread =
-// token of the tile for the softmax; the same warps run the key-residual MMAs for their 32 tokens),
-// 6-9 value warps (value-residual MMAs, 32 features each).
+//     traffic per contraction. The key residual is stored into the tile's TMEM score buffer first
+//     and the factor products accumulate on top of it, so the scores arrive complete.
+// Warp roles (512 threads, four warpgroups whose register budgets are re-split with setmaxnreg):
+//   0: warp 0 TMA producers (one lane per operand ring), warp 1 MMA issuer (owns TMEM);
+//   1: key-residual warps (the MMAs for their 32 tokens, then the row into TMEM);
+//   2: softmax warps (thread = token of the tile: scores from TMEM, online softmax, P~);
+//   3: value warps (value-residual MMAs, 32 features each).
+// TMEM: two score buffers of 32 columns, W (32 columns per 128-rank chunk) from column 128, the
+// value-residual accumulators (8 columns per KV head) from column 384.
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
@@ -35,6 +40,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "gemm_tc.cuh"
+#include "mma_codes.cuh"
 #include "sm100.cuh"
 #include "stats.h"
 
@@ -71,7 +77,8 @@ constexpr int kOffAlpha = kOffRed + 2 * 4 * 32 * 4; // [2][64] floats: alpha[32]
 constexpr int kOffFin = kOffAlpha + 2 * 64 * 4;     // [4][32] float2
 constexpr int kOffZf = kOffFin + 4 * 32 * 8;        // [32]
 constexpr int kOffQs = kOffZf + 32 * 4;             // [32]
-constexpr int kOffBars = kOffQs + 32 * 4;
+constexpr int kOffZk = kOffQs + 32 * 4;             // [4 warps][8 heads][32 tokens] key scale/zero pairs
+constexpr int kOffBars = kOffZk + 4 * 8 * 32 * 4;
 constexpr int kNumBars = 32;
 constexpr int kSmemUsed = kOffBars + kNumBars * 8 + 16;
 constexpr int kSmem = kSmemUsed + 1024;             // 1024-byte alignment of the swizzled tiles
@@ -79,7 +86,9 @@ static_assert(kSmem <= 232448, "fused decode shared memory");
 static_assert(kOffV % 1024 == 0 && kOffPt % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(kOffCK % 16 == 0 && kOffCV % 16 == 0 && kOffBars % 8 == 0, "bulk-copy and mbarrier alignment");
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 512;  // four warpgroups: control, key residual, softmax, value residual
+// registers a thread after the warpgroups' re-split (launch: 128 each, 65536 in all)
+constexpr int kRegCtl = 40, kRegKres = 128, kRegSoft = 184, kRegVres = 160;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -108,46 +117,6 @@ struct FusedArgs {
 
 __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// b-bit code fields of a word as exact f16 pairs. The mask-and-or puts each field into the
-// mantissa of 1024 (f16 0x6400), scaled by 2^shift; one f16x2 add or fused multiply-add with
-// constant pairs removes both (exact: every intermediate is a small integer or a power of two).
-__device__ __forceinline__ uint32_t h2_add(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-constexpr uint32_t kH2M1024 = 0xE400E400u;                            // (-1024, -1024)
-__device__ __forceinline__ uint32_t field_or(uint32_t x, uint32_t mask) { return (x & mask) | 0x64006400u; }
-// 4-bit fields at bits 0-3 / 16-19 (lo) or 4-7 / 20-23 (hi)
-__device__ __forceinline__ uint32_t nib_lo(uint32_t x) { return h2_add(field_or(x, 0x000F000Fu), kH2M1024); }
-__device__ __forceinline__ uint32_t nib_hi(uint32_t x) { return h2_fma(field_or(x, 0x00F000F0u), 0x2C002C00u, 0xD400D400u); }
-// 2-bit fields at bit 2s / 16 + 2s: (1024 + 4^s c) * 4^-s - 1024 * 4^-s
-__device__ __forceinline__ uint32_t crumb(uint32_t x, int s) {
-  switch (s) {
-    case 0: return h2_add(field_or(x, 0x00030003u), kH2M1024);
-    case 1: return h2_fma(field_or(x, 0x000C000Cu), 0x34003400u, 0xDC00DC00u);
-    case 2: return h2_fma(field_or(x, 0x00300030u), 0x2C002C00u, 0xD400D400u);
-    default: return h2_fma(field_or(x, 0x00C000C0u), 0x24002400u, 0xCC00CC00u);
-  }
-}
-// bytes of x chosen by sel next to 0x64 -> f16 pair (byte, byte)
-__device__ __forceinline__ uint32_t byte_pair(uint32_t x, uint32_t sel) {
-  return h2_add(__byte_perm(x, 0x64646464u, sel), kH2M1024);
-}
-
 // Within a lane's 32-code segment of a key-residual row, pair p (16 pairs, in the order the
 // conversion produces them) holds the codes at offsets (lo, lo + gap).
 __device__ __forceinline__ int pair_lo(int bits, int p) {
@@ -173,11 +142,11 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
 }
 
 // Key residual of KV head h (codes in slot k of the stage at cs) for the 32 tokens of quarter q:
-// scr[token][h g_q + j] = scale (codes . R q_j) + zero sum(R q_j). zkh: lane i holds the
-// (scale, zero) pair of token 32 q + i.
+// scr[token][h g_q + j] = scale (codes . R q_j) + zero sum(R q_j). zrow[i]: the (scale, zero) pair
+// of token 32 q + i for this head.
 template <int BITS, int GQ>
 __device__ __forceinline__ void kres_head(const uint8_t* cs, int k, int h, int q, int lane, const uint2* qf,
-                                          const float* qs, float* scr, uint32_t zkh) {
+                                          const float* qs, float* scr, const uint32_t* zrow) {
   constexpr int RB = 16 * BITS;
   const int gr = lane >> 2, m4 = lane & 3;
 #pragma unroll
@@ -219,11 +188,11 @@ __device__ __forceinline__ void kres_head(const uint8_t* cs, int k, int h, int q
       }
       uint2 bq = make_uint2(0u, 0u);
       if (gr < GQ) bq = qf[((h * 8 + kc) * GQ + gr) * 4 + m4];
-      mma_f16(acc, af, bq.x, bq.y);
+      mma_f16_16816(acc, af, bq.x, bq.y);
     }
     // rows g (tile row rA) and g + 8, query heads 2 m4, 2 m4 + 1 of KV head h
-    const uint32_t zA = __shfl_sync(0xffffffffu, zkh, 16 * mb + gr);
-    const uint32_t zB = __shfl_sync(0xffffffffu, zkh, 16 * mb + gr + 8);
+    const uint32_t zA = zrow[16 * mb + gr];
+    const uint32_t zB = zrow[16 * mb + gr + 8];
     const float2 fA = __half22float2(*reinterpret_cast<const __half2*>(&zA));
     const float2 fB = __half22float2(*reinterpret_cast<const __half2*>(&zB));
 #pragma unroll
@@ -281,9 +250,68 @@ __device__ __forceinline__ void vres_head(float (&ac)[2][4], const uint8_t* cs, 
     }
     uint2 bw = make_uint2(0u, 0u);
     if (gr < GQ) bw = wbp[((h * 8 + kc) * 4 + m4) * GQ + gr];
-    mma_f16(ac[0], f0, bw.x, bw.y);
-    mma_f16(ac[1], f1, bw.x, bw.y);
+    mma_f16_16816(ac[0], f0, bw.x, bw.y);
+    mma_f16_16816(ac[1], f1, bw.x, bw.y);
   }
+}
+
+// The key residual of one tile for this warp's 32 tokens, head after head (a runtime loop: one
+// copy of the head's code per code width keeps the hot loop small), releasing each code stage.
+template <int BITS, int GQ>
+__device__ __noinline__ bool kres_tile(const uint8_t* cbase, uint32_t full0, uint32_t empty0, int& ckit, int q,
+                                       int lane, const uint2* qf, const float* qs, float* scr,
+                                       const uint32_t* zks, int32_t* err, bool ok) {
+  constexpr int NKV = kNQ / GQ, hps = 8 / BITS;
+  int s = 0;
+#pragma unroll 1
+  for (int h = 0; h < NKV; ++h) {
+    const int k = h % hps;
+    if (k == 0) {
+      s = ckit % kCStages;
+      if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(full0 + 8u * s, (ckit / kCStages) & 1, err));
+    }
+    kres_head<BITS, GQ>(cbase + s * kCStageBytes, k, h, q, lane, qf, qs, scr, zks + h * 32);
+    if (k == hps - 1 || h == NKV - 1) {
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(empty0 + 8u * s);
+      ++ckit;
+    }
+  }
+  return ok;
+}
+
+// The value residual of one tile for this warp's features, head after head; the accumulators of
+// head h live in TMEM columns tacc + 8 h of the warp's lane quarter (loaded, updated, stored back).
+template <int BITS, int GQ>
+__device__ __noinline__ bool vres_tile(const uint8_t* cbase, uint32_t full0, uint32_t empty0, int& cvit,
+                                       const uint2* wbp, uint32_t tacc, int vw, int lane, int32_t* err, bool ok) {
+  constexpr int NKV = kNQ / GQ, hps = 8 / BITS;
+  int s = 0;
+#pragma unroll 1
+  for (int h = 0; h < NKV; ++h) {
+    const int k = h % hps;
+    if (k == 0) {
+      s = cvit % kCStages;
+      if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(full0 + 8u * s, (cvit / kCStages) & 1, err));
+    }
+    uint32_t r[8];
+    sm100::tmem_ld8(tacc + 8 * h, r);
+    sm100::tmem_ld_wait();
+    float ac[2][4];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ac[e >> 2][e & 3] = __uint_as_float(r[e]);
+    vres_head<BITS, GQ>(ac, cbase + s * kCStageBytes, k, wbp, h, vw, lane);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) r[e] = __float_as_uint(ac[e >> 2][e & 3]);
+    sm100::tmem_st8(tacc + 8 * h, r);
+    if (k == hps - 1 || h == NKV - 1) {
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(empty0 + 8u * s);
+      ++cvit;
+    }
+  }
+  sm100::tmem_st_wait();
+  return ok;
 }
 
 template <int GQ>
@@ -303,14 +331,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
   auto BCK_EMPTY = [&](int s) { return bar0 + 8u * (12 + s); };
   auto BCV_FULL = [&](int s) { return bar0 + 8u * (14 + s); };
   auto BCV_EMPTY = [&](int s) { return bar0 + 8u * (16 + s); };
-  auto BS_FULL = [&](int s) { return bar0 + 8u * (18 + s); };
-  auto BS_EMPTY = [&](int s) { return bar0 + 8u * (20 + s); };
+  auto BS_FULL = [&](int s) { return bar0 + 8u * (18 + s); };   // score products done
+  auto BS_EMPTY = [&](int s) { return bar0 + 8u * (20 + s); };  // softmax warps have read S
   auto BP_FULL = [&](int s) { return bar0 + 8u * (22 + s); };
   auto BP_EMPTY = [&](int s) { return bar0 + 8u * (24 + s); };
   auto BW_DONE = [&](int s) { return bar0 + 8u * (26 + s); };
   const uint32_t BDRAIN = bar0 + 8u * 28;
+  auto BR_FULL = [&](int s) { return bar0 + 8u * (29 + s); };   // key residual stored into S
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wg = warp >> 2;
   // this CTA's (sequence, split, layer): layers fastest, so the CTAs of one layer group that share
   // U_T tiles run side by side
   const int li = blockIdx.x % a.Lc;
@@ -332,12 +362,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
   const size_t prow = size_t(2 + a.q_cap + kD);
 
   if (threadIdx.x == 0) {
-    // arrival counts: TMA / MMA-commit barriers 1; code-stage releases and score-warp hand-offs 4
-    // (one per consuming warp); a P~ buffer is free after the value products (1 commit) and the
-    // four value warps
-    for (int i = 0; i < 29; ++i) {
+    // arrival counts: TMA / MMA-commit barriers 1; code-stage releases, S releases, P~ hand-offs
+    // and residual hand-offs 4 (one per consuming warp); a P~ buffer is free after the value
+    // products (1 commit) and the four value warps
+    for (int i = 0; i < 31; ++i) {
       uint32_t cnt = 1;
-      if ((i >= 12 && i < 14) || (i >= 16 && i < 18) || (i >= 20 && i < 24)) cnt = 4;
+      if ((i >= 12 && i < 14) || (i >= 16 && i < 18) || (i >= 20 && i < 24) || i >= 29) cnt = 4;
       if (i >= 24 && i < 26) cnt = 5;
       sm100::mbar_init(bar0 + 8u * i, cnt);
     }
@@ -351,13 +381,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tW = tmem + 2 * 2 * kNQ;  // S: two buffers of 64 columns; W after them
+  // S: two buffers of 32 columns; W (up to 8 chunks of 32 columns) from column 128; the value
+  // residual accumulators (8 columns per KV head) from column 384
+  const uint32_t tS = tmem, tW = tmem + 128, tAcc = tmem + 384;
 
-  if (warp == 0) {
-    // ================= TMA producers: one lane per ring, each running ahead on its own =========
-    // lane 0: U_T^K + P chunks, lane 1: key code stages, lane 2: U_T^V chunks, lane 3: value code
-    // stages; a lane waits only for its own ring's free slots
-    if (lane < 4) {
+  if (wg == 0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegCtl));
+    if (warp == 0 && lane < 4) {
+      // ================= TMA producers: one lane per ring, each running ahead on its own =========
+      // lane 0: U_T^K + P chunks, lane 1: key code stages, lane 2: U_T^V chunks, lane 3: value code
+      // stages; a lane waits only for its own ring's free slots
       bool ok = true;
       int cnt = 0;
       const bool kside = lane < 2;
@@ -406,14 +439,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
         const uint32_t full = lane == 0 ? BK_FULL(s) : lane == 2 ? BV_FULL(s) : lane == 1 ? BCK_FULL(s) : BCV_FULL(s);
         sm100::mbar_wait(full, (i / depth) & 1, a.err);
       }
-    }
-  } else if (warp == 1) {
-    // ================= MMA issuer =================
-    // Two chains share the thread: the score products S(it) (key ring) and the value products
-    // W += U_T^V^T P~(it') for the tile whose probabilities are ready (value ring). Whichever ring
-    // has a stage ready is served, so the two rings' copies overlap instead of adding up.
-    if (lane == 0) {
-      constexpr uint32_t idK = sm100::idesc_bf16_f32(kBM, 2 * kNQ, 0, 0);
+    } else if (warp == 1 && lane == 0) {
+      // ================= MMA issuer =================
+      // Two chains share the thread: the score products S(it) += U_T^K (P_hi + P_lo) on the
+      // buffer the key-residual warps have filled (key ring), and the value products
+      // W += U_T^V^T P~(it') for the tile whose probabilities are ready (value ring). Whichever
+      // ring has a stage ready is served, so the two rings' copies overlap instead of adding up.
+      constexpr uint32_t idK = sm100::idesc_bf16_f32(kBM, kNQ, 0, 0);
       constexpr uint32_t idW = sm100::idesc_bf16_f32(128, kNQ, 1, 0);
       int kit = 0, vit = 0;
       int itK = 0, kb = 0, itW = 0, wst = 0;  // score tile / chunk, value tile / stage within it
@@ -429,17 +461,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
             ++itK;
             progressed = true;
           } else {
-            if (!sfree) sfree = sm100::mbar_test_wait(BS_EMPTY(itK & 1), ((itK >> 1) & 1) ^ 1);
+            if (!sfree) sfree = sm100::mbar_test_wait(BR_FULL(itK & 1), (itK >> 1) & 1);
             const int s = kit % kKStages;
             if (sfree && sm100::mbar_test_wait(BK_FULL(s), (kit / kKStages) & 1)) {
               sm100::tc_fence_after();
-              const uint32_t dt = tS + (itK & 1) * 2 * kNQ;
+              const uint32_t dt = tS + (itK & 1) * kNQ;
               const uint32_t ka = sb + kOffK + s * kKStageBytes;
 #pragma unroll
               for (int kk = 0; kk < kBK / 16; ++kk) {
                 const uint64_t ad = sm100::smem_desc_sw128(ka + kk * 32, 16, 1024);
-                const uint64_t bd = sm100::smem_desc_sw128(ka + kBM * kBK * 2 + kk * 32, 16, 1024);
-                sm100::mma_bf16(dt, ad, bd, idK, (kb > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int term = 0; term < 2; ++term) {  // P hi rows 0-31, P lo rows 32-63
+                  const uint64_t bd = sm100::smem_desc_sw128(ka + kBM * kBK * 2 + term * kNQ * 128 + kk * 32, 16, 1024);
+                  sm100::mma_bf16(dt, ad, bd, idK, (bK > 0 || kb > 0 || kk > 0 || term > 0) ? 1u : 0u);
+                }
               }
               sm100::mma_commit(BK_EMPTY(s));
               ++kit;
@@ -503,16 +538,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       sm100::mma_commit(BDRAIN);
       sm100::mbar_wait(BDRAIN, 0, a.err);
     }
-  } else if (warp < 6) {
-    // ================= score warps: key residual, scores, online softmax =================
+  } else if (wg == 1) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegKres));
+    // ================= key-residual warps: S(it) starts as scale (codes . R q) + zero sum(R q) ====
     const int q = warp & 3;            // TMEM lane quarter = tokens 32q .. 32q+31 of the tile
-    const int gr = lane >> 2, m4 = lane & 3;
-    const int tid = threadIdx.x - 64;  // 0..127
+    const int tid = threadIdx.x - 128; // 0..127
     float* scr = reinterpret_cast<float*>(smem + kOffScr) + q * 32 * kScrStride;
-    float* red = reinterpret_cast<float*>(smem + kOffRed);
-    float* alph = reinterpret_cast<float*>(smem + kOffAlpha);
-    float2* fin = reinterpret_cast<float2*>(smem + kOffFin);
-    float* zf = reinterpret_cast<float*>(smem + kOffZf);
     float* qs = reinterpret_cast<float*>(smem + kOffQs);
     uint2* qf = reinterpret_cast<uint2*>(smem + kOffQf);
     // query-side operands of the key residual: f16 fragments of R q in the pair order of this
@@ -530,85 +561,91 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       }
     }
     if (tid < kNQ) qs[tid] = a.qsum[int64_t(bl) * kNQ + tid];
-    named_bar(1, 128);
-    float mref = -INFINITY, ell = 0.f, zac = 0.f;  // of query head `lane`
+    named_bar(3, 128);
     int ckit = 0;
     bool ok = true;
     const __half2* szK = ck.sz ? ck.sz + int64_t(ll) * NKV * a.T : nullptr;
-    const __half2* szV = cv.sz ? cv.sz + int64_t(ll) * NKV * a.T : nullptr;
-
-    // this thread's token's scale / zero pairs, loaded one tile ahead (the key ones reach the MMA
-    // lanes by shuffles)
-    uint32_t zk[NKV], zv[NKV], nzk[NKV], nzv[NKV];
-    auto load_sz = [&](int it2, uint32_t (&k_)[NKV], uint32_t (&v_)[NKV]) {
+    // this thread's token's key scale / zero pairs, loaded one tile ahead (they reach the MMA lanes
+    // by shuffles)
+    uint32_t* zks = reinterpret_cast<uint32_t*>(smem + kOffZk) + q * 8 * 32;
+    uint32_t nzk[NKV];
+    auto load_sz = [&](int it2, uint32_t (&k_)[NKV]) {
       const int t2 = (tile0 + it2) * kBM + 32 * q + lane;
       const bool ok2 = it2 < ntl && t2 < a.T;
 #pragma unroll
-      for (int h = 0; h < NKV; ++h) {
-        k_[h] = (bK && ok2) ? sm100::ld_nc_early(szK + int64_t(h) * a.T + t2) : 0u;
-        v_[h] = (bV && ok2) ? sm100::ld_nc_early(szV + int64_t(h) * a.T + t2) : 0u;
-      }
+      for (int h = 0; h < NKV; ++h) k_[h] = (bK && ok2) ? sm100::ld_nc_early(szK + int64_t(h) * a.T + t2) : 0u;
     };
-    load_sz(0, nzk, nzv);
+    load_sz(0, nzk);
     for (int it = 0; it < ntl; ++it) {
-      __syncwarp();  // every lane has read its row of the exchange buffer before it is rewritten
+      __syncwarp();  // every lane has read its row of the exchange buffer and slab before they are rewritten
+#pragma unroll
+      for (int h = 0; h < NKV; ++h) zks[h * 32 + lane] = nzk[h];
+      __syncwarp();
+      load_sz(it + 1, nzk);
+      if (bK) {
+        const uint8_t* cbase = smem + kOffCK;
+        if (bK == 4) ok = kres_tile<4, GQ>(cbase, BCK_FULL(0), BCK_EMPTY(0), ckit, q, lane, qf, qs, scr, zks, a.err, ok);
+        else if (bK == 2) ok = kres_tile<2, GQ>(cbase, BCK_FULL(0), BCK_EMPTY(0), ckit, q, lane, qf, qs, scr, zks, a.err, ok);
+        else ok = kres_tile<8, GQ>(cbase, BCK_FULL(0), BCK_EMPTY(0), ckit, q, lane, qf, qs, scr, zks, a.err, ok);
+      }
+      // the S buffer is free once the softmax warps have read tile it - 2
+      if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BS_EMPTY(it & 1), ((it >> 1) & 1) ^ 1, a.err));
+      sm100::tc_fence_after();
+      if (bK || nkb == 0) {
+        uint32_t r[kNQ];
+#pragma unroll
+        for (int j = 0; j < kNQ; ++j) r[j] = bK ? __float_as_uint(scr[lane * kScrStride + j]) : 0u;
+        sm100::tmem_st32(tS + (it & 1) * kNQ + (uint32_t(32 * q) << 16), r);
+        sm100::tmem_st_wait();
+      }
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(BR_FULL(it & 1));
+    }
+  } else if (wg == 2) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoft));
+    // ================= softmax warps: complete scores from TMEM, online softmax, P~ =================
+    const int q = warp & 3;            // TMEM lane quarter = tokens 32q .. 32q+31 of the tile
+    float* red = reinterpret_cast<float*>(smem + kOffRed);
+    float* alph = reinterpret_cast<float*>(smem + kOffAlpha);
+    float2* fin = reinterpret_cast<float2*>(smem + kOffFin);
+    float* zf = reinterpret_cast<float*>(smem + kOffZf);
+    float mref = -INFINITY, ell = 0.f, zac = 0.f;  // of query head `lane`
+    bool ok = true;
+    const __half2* szV = cv.sz ? cv.sz + int64_t(ll) * NKV * a.T : nullptr;
+    uint32_t zv[NKV], nzv[NKV];
+    auto load_sz = [&](int it2, uint32_t (&v_)[NKV]) {
+      const int t2 = (tile0 + it2) * kBM + 32 * q + lane;
+      const bool ok2 = it2 < ntl && t2 < a.T;
+#pragma unroll
+      for (int h = 0; h < NKV; ++h) v_[h] = (bV && ok2) ? sm100::ld_nc_early(szV + int64_t(h) * a.T + t2) : 0u;
+    };
+    load_sz(0, nzv);
+    for (int it = 0; it < ntl; ++it) {
       const int t0 = (tile0 + it) * kBM;
       const int tl = 32 * q + lane, t = t0 + tl;
       const bool valid = t < a.T;
 #pragma unroll
-      for (int h = 0; h < NKV; ++h) {
-        zk[h] = nzk[h];
-        zv[h] = nzv[h];
-      }
-      load_sz(it + 1, nzk, nzv);
-      // ---- key residual: jobs of 8 / b heads per code stage ----
-      if (bK) {
-        const int hps = 8 / bK;
-        int s = 0;
-#pragma unroll
-        for (int h = 0; h < NKV; ++h) {
-          const int k = h % hps;
-          if (k == 0) {
-            s = ckit % kCStages;
-            if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BCK_FULL(s), (ckit / kCStages) & 1, a.err));
-          }
-          const uint8_t* cs = smem + kOffCK + s * kCStageBytes;
-          if (bK == 4) kres_head<4, GQ>(cs, k, h, q, lane, qf, qs, scr, zk[h]);
-          else if (bK == 2) kres_head<2, GQ>(cs, k, h, q, lane, qf, qs, scr, zk[h]);
-          else kres_head<8, GQ>(cs, k, h, q, lane, qf, qs, scr, zk[h]);
-          if (k == hps - 1 || h == NKV - 1) {
-            __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(BCK_EMPTY(s));
-            ++ckit;
-          }
-        }
-      }
-      // ---- scores of token t for the 32 query heads ----
+      for (int h = 0; h < NKV; ++h) zv[h] = nzv[h];
+      load_sz(it + 1, nzv);
+      // ---- scores of token t for the 32 query heads (factor part + key residual) ----
       float sv[kNQ];
-      if (nkb) {
-        if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BS_FULL(it & 1), (it >> 1) & 1, a.err));
+      {
+        const uint32_t ready = nkb ? BS_FULL(it & 1) : BR_FULL(it & 1);
+        if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(ready, (it >> 1) & 1, a.err));
         sm100::tc_fence_after();
-        uint32_t hi[32], lo[32];
-        const uint32_t ta = tS + (it & 1) * 2 * kNQ + (uint32_t(32 * q) << 16);
-        sm100::tmem_ld32(ta, hi);
-        sm100::tmem_ld32(ta + kNQ, lo);
+        uint32_t r[kNQ];
+        sm100::tmem_ld32(tS + (it & 1) * kNQ + (uint32_t(32 * q) << 16), r);
         sm100::tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < kNQ; ++j) sv[j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
+        for (int j = 0; j < kNQ; ++j) sv[j] = __uint_as_float(r[j]);
         sm100::tc_fence_before();
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive(BS_EMPTY(it & 1));
-      } else {
-#pragma unroll
-        for (int j = 0; j < kNQ; ++j) sv[j] = 0.f;
       }
-      __syncwarp();
       const float sc2 = a.attn_scale * kLog2e;
 #pragma unroll
-      for (int j = 0; j < kNQ; ++j) {
-        const float r = bK ? scr[lane * kScrStride + j] : 0.f;
-        sv[j] = valid ? (sv[j] + r) * sc2 : -INFINITY;
-      }
+      for (int j = 0; j < kNQ; ++j) sv[j] = valid ? sv[j] * sc2 : -INFINITY;
       // ---- tile maximum per query head; the reference maximum moves only by more than 2^8 ----
       float tmp[kNQ];
 #pragma unroll
@@ -708,18 +745,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
     }
     named_bar(2, 256);  // zf ready for the value warps
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegVres));
     // ================= value warps: acc[d][j] += sum_t weight[t][j] codes^V[t][d] =================
-    const int vw = warp - 6;  // features 16 g + 4 vw .. + 3
+    const int vw = warp & 3;  // features 16 g + 4 vw .. + 3
     const int gr = lane >> 2, m4 = lane & 3;
     const float* alph = reinterpret_cast<const float*>(smem + kOffAlpha);
     const float* zf = reinterpret_cast<const float*>(smem + kOffZf);
-    float acc[NKV][2][4];
+    // accumulators of head h: TMEM columns tAcc + 8 h of this warp's lane quarter
+    const uint32_t tacc = tAcc + (uint32_t(32 * vw) << 16);
+    {
+      const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int h = 0; h < NKV; ++h)
-#pragma unroll
-      for (int mb = 0; mb < 2; ++mb)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[h][mb][e] = 0.f;
+      for (int h = 0; h < NKV; ++h) sm100::tmem_st8(tacc + 8 * h, z);
+      sm100::tmem_st_wait();
+    }
     int cvit = 0;
     bool ok = true;
     for (int it = 0; it < ntl; ++it) {
@@ -727,37 +766,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       if (bV) {
         if (alph[(it & 1) * 64 + 32] != 0.f) {
           const float* al = alph + (it & 1) * 64;
-#pragma unroll
+#pragma unroll 1
           for (int h = 0; h < NKV; ++h) {
             const int j0 = h * GQ + 2 * m4;
             const float a0 = (2 * m4 < GQ) ? al[j0] : 0.f;
             const float a1 = (2 * m4 + 1 < GQ) ? al[j0 + 1] : 0.f;
+            uint32_t r[8];
+            sm100::tmem_ld8(tacc + 8 * h, r);
+            sm100::tmem_ld_wait();
 #pragma unroll
-            for (int mb = 0; mb < 2; ++mb) {
-              acc[h][mb][0] *= a0; acc[h][mb][1] *= a1; acc[h][mb][2] *= a0; acc[h][mb][3] *= a1;
-            }
+            for (int e = 0; e < 8; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * ((e & 1) ? a1 : a0));
+            sm100::tmem_st8(tacc + 8 * h, r);
           }
+          sm100::tmem_st_wait();
         }
         const uint2* wbp = reinterpret_cast<const uint2*>(smem + kOffWb + (it & 1) * kWbBytes);
-        const int hps = 8 / bV;
-        int s = 0;
-#pragma unroll
-        for (int h = 0; h < NKV; ++h) {
-          const int k = h % hps;
-          if (k == 0) {
-            s = cvit % kCStages;
-            if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BCV_FULL(s), (cvit / kCStages) & 1, a.err));
-          }
-          const uint8_t* cs = smem + kOffCV + s * kCStageBytes;
-          if (bV == 4) vres_head<4, GQ>(acc[h], cs, k, wbp, h, vw, lane);
-          else if (bV == 2) vres_head<2, GQ>(acc[h], cs, k, wbp, h, vw, lane);
-          else vres_head<8, GQ>(acc[h], cs, k, wbp, h, vw, lane);
-          if (k == hps - 1 || h == NKV - 1) {
-            __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(BCV_EMPTY(s));
-            ++cvit;
-          }
-        }
+        const uint8_t* cbase = smem + kOffCV;
+        if (bV == 4) ok = vres_tile<4, GQ>(cbase, BCV_FULL(0), BCV_EMPTY(0), cvit, wbp, tacc, vw, lane, a.err, ok);
+        else if (bV == 2) ok = vres_tile<2, GQ>(cbase, BCV_FULL(0), BCV_EMPTY(0), cvit, wbp, tacc, vw, lane, a.err, ok);
+        else ok = vres_tile<8, GQ>(cbase, BCV_FULL(0), BCV_EMPTY(0), cvit, wbp, tacc, vw, lane, a.err, ok);
       }
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(BP_EMPTY(it & 1));
@@ -765,8 +792,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
     named_bar(2, 256);
     // acc entries: features d = 16 g + 4 vw + 2 mb + (0 | 1), query heads h g_q + 2 m4 + (0 | 1);
     // the stored value is 256 acc (the weights carry 2^-8) + sum_t p~ zero
-#pragma unroll
+#pragma unroll 1
     for (int h = 0; h < NKV; ++h) {
+      uint32_t r[8];
+      sm100::tmem_ld8(tacc + 8 * h, r);
+      sm100::tmem_ld_wait();
+      float acc[2][4];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e >> 2][e & 3] = __uint_as_float(r[e]);
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int jj = 2 * m4 + e;
@@ -777,8 +810,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
 #pragma unroll
         for (int mb = 0; mb < 2; ++mb) {
           const int d = 16 * gr + 4 * vw + 2 * mb;
-          pr[d] = 256.f * acc[h][mb][e] + z;
-          pr[d + 1] = 256.f * acc[h][mb][2 + e] + z;
+          pr[d] = 256.f * acc[mb][e] + z;
+          pr[d + 1] = 256.f * acc[mb][2 + e] + z;
         }
       }
     }
@@ -980,6 +1013,14 @@ jolt_status launch_decode_fused(const DecodeParams& p, const TcCellView* views, 
   {
     StatScope sc(JOLT_K_DECODE_MAIN, st, flops, p.alg_bytes);
     const int grid = BL * wl.S;
+    // the warpgroups re-split the block's registers (setmaxnreg): decreases must not exceed and
+    // increases must not fall below the launch count, and the new shares must fit what the block
+    // was launched with, or an increasing warpgroup would wait for registers that never come
+    cudaFuncAttributes fat;
+    JOLT_CUDA_TRY(cudaFuncGetAttributes(&fat, p.gq == 4 ? k_decode_fused<4> : k_decode_fused<8>));
+    if (fat.numRegs < kRegCtl || fat.numRegs > kRegKres || fat.numRegs > kRegSoft || fat.numRegs > kRegVres ||
+        128 * (kRegCtl + kRegKres + kRegSoft + kRegVres) > kThreads * fat.numRegs)
+      return JOLT_ERR_CUDA;
     if (p.gq == 4) {
       JOLT_CUDA_TRY(cudaFuncSetAttribute(k_decode_fused<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
       k_decode_fused<4><<<grid, kThreads, kSmem, st>>>(maps, fa);

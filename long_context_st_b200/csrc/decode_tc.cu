@@ -25,6 +25,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "gemm_tc.cuh"
+#include "mma_codes.cuh"
 #include "pack.cuh"
 #include "sm100.cuh"
 #include "stats.h"
@@ -43,12 +44,14 @@ template <int NT>
 struct KeysCfg {
   static constexpr int kStages = NT == 1 ? 4 : 3;
   static constexpr int kStageBytes = kABytes + NT * kBBytes;
-  static constexpr int kQsBytes = 2 * kMaxG * kD * 4;      // queries of each epilogue group's pair, fp32
+  static constexpr int kQsBytes = 2 * kMaxG * kD * 4;      // queries of each score group's pair, fp32
   static constexpr int kRopeBytes = kD / 4 * kBM * 16;     // (cos, cos, sin, sin) of frequency pairs
   static constexpr int kSmem = 1024 + kStages * kStageBytes + kQsBytes + kRopeBytes + kD * 4 + 256;
-  static constexpr int kThreads = 320;                     // producer, MMA, two groups of four epilogue warps
+  static constexpr int kThreads = 512;                     // four warpgroups: control, residual, 2 x score
+  static constexpr int kNB = 4;                            // TMEM key buffers of 128 columns
+  // registers a thread after the warpgroups' re-split (launch: 128 each, 65536 in all)
+  static constexpr int kRegCtl = 40, kRegRes = 200, kRegScore = 120;
 };
-
 struct KeysMaps {
   CUtensorMap a;       // U_T^K [T][r_T], K-major, box 64 x 128
   CUtensorMap b[2];    // B_h hi / lo [pairs][r_T][128], MN-major, box 64 x 64
@@ -143,13 +146,17 @@ __device__ __forceinline__ void fwht128x2(float2 (&v)[kD / 2]) {
   }
 }
 
-// grid.x = token tiles; 320 threads (three warps share some SM sub-partitions, whose register files
-// hold 16384 registers each, so at most 168 registers a thread): warp 0 TMA producer, warp 1 MMA
-// issuer (+ TMEM owner),
-// warps 2..5 and 6..9 two epilogue groups taking alternate (layer, head) pairs and TMEM buffers
-// (warp w reads TMEM lanes 32 * (w % 4) .. +31, i.e. token rows of the tile).
+// grid.x = token tiles; 512 threads in four warpgroups with re-split register budgets:
+//   warpgroup 0: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warps 2-3 idle after setup;
+//   warpgroup 1: residual warps — thread = token row of the tile (warp w: TMEM lanes 32 (w % 4) ..
+//                +31); per (layer, KV head) pair they dequantise the residual row, undo the
+//                rotation (FWHT and signs) and store it into the pair's TMEM key buffer, on which
+//                the MMAs then accumulate U_T B_h (so the key arrives complete in TMEM);
+//   warpgroups 2, 3: two score groups taking alternate pairs: RoPE at the token's position and
+//                q . k for the pair's g_q query heads, straight from TMEM in 16-column pieces.
+// Four TMEM buffers of 128 columns rotate over the pairs: residual -> MMA -> score.
 template <int BITS, int NT>
-__global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ KeysMaps maps, const KeysArgs p) {
+__global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ KeysMaps maps, const KeysArgs p) {
   using C = KeysCfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = sm100::align_smem_1024(smem_raw);
@@ -157,7 +164,7 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
   float4* rope = reinterpret_cast<float4*>(qs + 2 * kMaxG * kD);            // [32][kBM]
   float2* sgn = reinterpret_cast<float2*>(rope + kD / 4 * kBM);               // [64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sgn + kD / 2);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 5);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 3 * C::kNB + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kBM;
@@ -167,18 +174,20 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
   const uint32_t bar0 = sm100::smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
-  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 + b); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 4);
+  auto rfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };             // residual stored
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + C::kNB + b); };    // MMAs done
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 * C::kNB + b); };  // scores read it
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 3 * C::kNB);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       sm100::mbar_init(full_bar(s), 1);
       sm100::mbar_init(empty_bar(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kNB; ++b) {
+      sm100::mbar_init(rfull_bar(b), 4);  // one arrival per residual warp
       sm100::mbar_init(tfull_bar(b), 1);
-      sm100::mbar_init(tempty_bar(b), 128);
+      sm100::mbar_init(tempty_bar(b), 4);  // one arrival per warp of the score group
     }
     sm100::mbar_init(drain_bar, 1);
     sm100::fence_mbar_init();
@@ -204,15 +213,17 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
     }
     rope[e] = make_float4(cs[0] * p.rope_scaling, cs[1] * p.rope_scaling, sn[0] * p.rope_scaling, sn[1] * p.rope_scaling);
   }
-  if (warp == 1) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), 256);
+  if (warp == 1) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), 128 * C::kNB);
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = sm100::smem_u32(smem);
+  const int wg = warp >> 2;
 
-  if (warp == 0) {
-    if (lane == 0 && fac) {
+  if (wg == 0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegCtl));
+    if (warp == 0 && lane == 0 && fac) {
       // ---- TMA producer: per (layer, head) pair, the U_T tile chunk and the B_h chunk(s) ----
       int it = 0;
       bool ok = true;
@@ -242,16 +253,14 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
       // wait (bounded) for the copies still in flight before the block may exit
       for (int i = max(0, it - C::kStages); i < it; ++i)
         sm100::mbar_wait(full_bar(i % C::kStages), (i / C::kStages) & 1, p.err);
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && fac) {
-      // ---- MMA issuer: D[pr % 2] = sum_k U_T[t][k] (B_hi + B_lo)[k][:] ----
+    } else if (warp == 1 && lane == 0 && fac) {
+      // ---- MMA issuer: D[pr % kNB] (= residual, or nothing for b = 0) += sum_k U_T (B_hi + B_lo) ----
       constexpr uint32_t idesc = sm100::idesc_bf16_f32(kBM, kD, 0, 1);
       int it = 0;
       bool ok = true;
       for (int pr = 0; pr < npairs && ok; ++pr) {
-        const int bi = pr & 1;
-        if (!sm100::mbar_wait(tempty_bar(bi), ((pr >> 1) & 1) ^ 1, p.err)) break;
+        const int bi = pr % C::kNB;
+        if (!sm100::mbar_wait(rfull_bar(bi), (pr / C::kNB) & 1, p.err)) break;
         sm100::tc_fence_after();
         const uint32_t dt = tmem + bi * kD;
         for (int kb = 0; kb < p.nkb; ++kb, ++it) {
@@ -268,7 +277,7 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
               const uint64_t bd = sm100::smem_desc_sw128(sa + kABytes + t * kBBytes + kk * 2048, 8192, 1024);
-              sm100::mma_bf16(dt, ad, bd, idesc, (kb > 0 || kk > 0 || t > 0) ? 1u : 0u);
+              sm100::mma_bf16(dt, ad, bd, idesc, (BITS > 0 || kb > 0 || kk > 0 || t > 0) ? 1u : 0u);
             }
           }
           sm100::mma_commit(empty_bar(s));
@@ -279,14 +288,71 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
       sm100::mma_commit(drain_bar);
       sm100::mbar_wait(drain_bar, 0, p.err);
     }
-  } else {
-    // ---- epilogue: group g takes pairs g, g + 2, ... (TMEM buffer g); thread = token row ----
-    const int g = (warp - 2) >> 2;
+  } else if (wg == 1) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kRegRes));
+    // ---- residual warps: the inverse-rotated residual row of each pair into its TMEM buffer ----
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int et = threadIdx.x - 64 - 128 * g;
     const int t = t0 + row;
     const bool valid = t < p.T;
+    bool live = true;
+    uint32_t cw[4 * BITS + 1];
+    float scv = 0.f, zrv = 0.f;
+    auto load_res = [&](int prr) {
+      const int li = prr / p.n_kv, h = prr % p.n_kv;
+      const int64_t rr = (int64_t(li) * p.n_kv + h) * p.T + t;
+      const __half2 szv = p.sz[rr];
+      load_codes_raw<BITS>(p.codes + rr * (kD * BITS / 8), cw);
+      scv = __low2float(szv);
+      zrv = __high2float(szv);
+    };
+    if (BITS > 0 && valid) load_res(0);
+    for (int pr = 0; pr < npairs; ++pr) {
+      const int bi = pr % C::kNB;
+      float2 v[kD / 2];
+      if (BITS > 0) {
+        if (valid) {
+          dequant2<BITS>(cw, scv, zrv, v);
+          if (pr + 1 < npairs) load_res(pr + 1);  // the next pair's row is in flight meanwhile
+          fwht128x2(v);
+#pragma unroll
+          for (int m = 0; m < kD / 2; ++m) v[m] = __fmul2_rn(v[m], sgn[m]);
+        } else {
+#pragma unroll
+          for (int m = 0; m < kD / 2; ++m) v[m] = make_float2(0.f, 0.f);
+        }
+      }
+      // the buffer is free once the score group has read the pair kNB earlier
+      if (live) live = __all_sync(0xffffffffu, sm100::mbar_wait(tempty_bar(bi), ((pr / C::kNB) & 1) ^ 1, p.err));
+      sm100::tc_fence_after();
+      if (BITS > 0) {
+        const uint32_t ta = tmem + bi * kD + (uint32_t(quarter * 32) << 16);
+#pragma unroll
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            r[2 * k] = __float_as_uint(v[16 * c + k].x);
+            r[2 * k + 1] = __float_as_uint(v[16 * c + k].y);
+          }
+          sm100::tmem_st32(ta + 32 * c, r);
+        }
+        sm100::tmem_st_wait();
+      }
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(rfull_bar(bi));
+    }
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::kRegScore));
+    // ---- score groups: group g takes pairs g, g + 2, ...; thread = token row ----
+    const int g = wg - 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int et = threadIdx.x - 256 - 128 * g;
+    const int t = t0 + row;
+    const bool valid = t < p.T;
+    // queries as [g_q][32 frequency pairs m][q_2m, q_2m+1, q_2m+64, q_2m+65] (fp32)
     float* qb = qs + g * kMaxG * kD;
     bool live = true;
     // a pair's g_q query rows (g_q * 128 bf16): thread et holds 8 consecutive values of each 1024,
@@ -303,90 +369,71 @@ __global__ void __launch_bounds__(320, 1) k_keys_tc(const __grid_constant__ Keys
     if (g < npairs) q_issue(g);
     for (int pr = g; pr < npairs; pr += 2) {
       const int li = pr / p.n_kv, h = pr % p.n_kv;
-      // this pair's residual row first: its loads overlap the query staging below
-      uint32_t cw[4 * BITS + 1];
-      float scv = 0.f, zrv = 0.f;
-      if (BITS > 0 && valid) {
-        const int64_t rr = (int64_t(li) * p.n_kv + h) * p.T + t;
-        const __half2 szv = p.sz[rr];
-        load_codes_raw<BITS>(p.codes + rr * (kD * BITS / 8), cw);
-        scv = __low2float(szv);
-        zrv = __high2float(szv);
-      }
+      const int bi = pr % C::kNB;
 #pragma unroll
       for (int j = 0; j < kMaxG * kD / 1024; ++j) {
-        const int e0 = (et + 128 * j) * 8;
+        const int e0 = (et + 128 * j) * 8;  // query row e0 / 128, features d0 .. d0 + 7
         if (e0 < p.gq * kD) {
           const uint32_t wq[4] = {qn[j].x, qn[j].y, qn[j].z, qn[j].w};
-          float f[8];
+          const int gg = e0 / kD, d0 = e0 % kD;
+          const int hi = d0 >= kD / 2 ? 2 : 0, m0 = (d0 % (kD / 2)) / 2;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const float2 ff = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wq[u]));
-            f[2 * u] = ff.x;
-            f[2 * u + 1] = ff.y;
+            *reinterpret_cast<float2*>(qb + gg * kD + 4 * (m0 + u) + hi) = ff;
           }
-          *reinterpret_cast<float4*>(qb + e0) = make_float4(f[0], f[1], f[2], f[3]);
-          *reinterpret_cast<float4*>(qb + e0 + 4) = make_float4(f[4], f[5], f[6], f[7]);
         }
       }
       if (pr + 2 < npairs) q_issue(pr + 2);
       group_bar(g);
-      float2 v[kD / 2];
-      if (BITS > 0 && valid) {
-        dequant2<BITS>(cw, scv, zrv, v);
-        fwht128x2(v);
+      const uint32_t ready = fac ? tfull_bar(bi) : rfull_bar(bi);
+      if (live) live = __all_sync(0xffffffffu, sm100::mbar_wait(ready, (pr / C::kNB) & 1, p.err));
+      sm100::tc_fence_after();
+      float2 acc[kMaxG];
 #pragma unroll
-        for (int m = 0; m < kD / 2; ++m) v[m] = __fmul2_rn(v[m], sgn[m]);
-      } else {
+      for (int gg = 0; gg < kMaxG; ++gg) acc[gg] = make_float2(0.f, 0.f);
+      const uint32_t ta = tmem + bi * kD + (uint32_t(quarter * 32) << 16);
 #pragma unroll
-        for (int m = 0; m < kD / 2; ++m) v[m] = make_float2(0.f, 0.f);
-      }
-      if (fac) {
-        // warp-uniform: the TMEM loads below are warp-collective
-        if (live) live = __all_sync(0xffffffffu, sm100::mbar_wait(tfull_bar(g), (pr >> 1) & 1, p.err));
-        sm100::tc_fence_after();
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t r1[16], r2[16];
+        sm100::tmem_ld16(ta + 16 * c, r1);           // features 16c .. 16c + 15
+        sm100::tmem_ld16(ta + kD / 2 + 16 * c, r2);  // their RoPE partners, + 64
+        sm100::tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < kD / 16; ++c) {
-          uint32_t r[16];
-          sm100::tmem_ld16(tmem + g * kD + c * 16 + (uint32_t(quarter * 32) << 16), r);
-          sm100::tmem_ld_wait();
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            v[c * 8 + k] = __fadd2_rn(v[c * 8 + k], make_float2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])));
-        }
-        sm100::tc_fence_before();
-        sm100::mbar_arrive(tempty_bar(g));
-      }
-      if (valid && live) {
-#pragma unroll
-        for (int m = 0; m < kD / 4; ++m) {  // features (2m, 2m+1) with (2m+64, 2m+65)
+        for (int k = 0; k < 8; ++k) {
+          const int m = 8 * c + k;  // features (2m, 2m+1) with (2m+64, 2m+65)
           const float4 r4 = rope[m * kBM + row];
           const float2 cs = make_float2(r4.x, r4.y), sn = make_float2(r4.z, r4.w);
-          const float2 x1 = v[m], x2 = v[m + kD / 4];
-          const float2 a = __fmul2_rn(x2, sn), b = __fmul2_rn(x1, sn);
-          v[m] = __ffma2_rn(x1, cs, make_float2(-a.x, -a.y));
-          v[m + kD / 4] = __ffma2_rn(x2, cs, b);
-        }
-        float* out = p.scores + (int64_t(li) * p.n_q + int64_t(h) * p.gq) * p.T + t;
-#pragma unroll 1
-        for (int gg = 0; gg < p.gq; ++gg) {
-          const float4* qg = reinterpret_cast<const float4*>(qb + gg * kD);
-          float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+          const float2 x1 = make_float2(__uint_as_float(r1[2 * k]), __uint_as_float(r1[2 * k + 1]));
+          const float2 x2 = make_float2(__uint_as_float(r2[2 * k]), __uint_as_float(r2[2 * k + 1]));
+          const float2 a = __fmul2_rn(x2, sn), bb = __fmul2_rn(x1, sn);
+          const float2 y1 = __ffma2_rn(x1, cs, make_float2(-a.x, -a.y));
+          const float2 y2 = __ffma2_rn(x2, cs, bb);
 #pragma unroll
-          for (int k = 0; k < kD / 4; ++k) {
-            const float4 qq = qg[k];
-            a0 = __ffma2_rn(v[2 * k], make_float2(qq.x, qq.y), a0);
-            a1 = __ffma2_rn(v[2 * k + 1], make_float2(qq.z, qq.w), a1);
+          for (int gg = 0; gg < kMaxG; ++gg) {
+            if (gg < p.gq) {
+              const float4 qq = *reinterpret_cast<const float4*>(qb + gg * kD + 4 * m);
+              acc[gg] = __ffma2_rn(y1, make_float2(qq.x, qq.y), acc[gg]);
+              acc[gg] = __ffma2_rn(y2, make_float2(qq.z, qq.w), acc[gg]);
+            }
           }
-          out[int64_t(gg) * p.T] = ((a0.x + a0.y) + (a1.x + a1.y)) * p.attn_scale;
         }
+      }
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(tempty_bar(bi));
+      if (valid && live) {
+        float* out = p.scores + (int64_t(li) * p.n_q + int64_t(h) * p.gq) * p.T + t;
+#pragma unroll
+        for (int gg = 0; gg < kMaxG; ++gg)
+          if (gg < p.gq) out[int64_t(gg) * p.T] = (acc[gg].x + acc[gg].y) * p.attn_scale;
       }
       group_bar(g);  // every thread is done with this pair's queries
     }
   }
   sm100::tc_fence_before();
   __syncthreads();
-  if (warp == 1) sm100::tmem_dealloc(tmem, 256);
+  if (warp == 1) sm100::tmem_dealloc(tmem, 128 * C::kNB);
 }
 
 // ---- CUDA-core stages -------------------------------------------------------------------------
@@ -525,102 +572,156 @@ struct ValArgs {
   float* acc;                 // [nl][n_q][128], rotated domain
 };
 
-// acc[h'][j] += sum_t P~[h'][t] deq(code_t[j]) (rotated domain). grid (token chunks, n_kv, nl),
-// 128 threads: lane l owns features 4l .. 4l+3 (one 4-code word per token), warp w the tokens
-// w, w+4, ... of every 128-token sub-tile, whose code rows (16-byte loads), scale/zero pairs and
-// probabilities are staged in shared memory first; the four warps' partial sums are added in
-// shared memory before one atomic add per (query head, feature).
+// acc[j][d] += sum_t P~[j][t] (scale_t code_t[d] + zero_t) for the query heads j of one KV head, in
+// the rotated domain, on mma.sync: per 16-token step D[d][j] += sum_t code[t][d] (P~[j][t] scale_t)
+// (M = 16 features per m-tile, eight m-tiles; N = 8 query heads per n-tile; K = 16 tokens), the codes
+// widened to exact f16 in registers and the weights P~ scale rounded to f16; sum_t P~ zero_t is
+// accumulated per query head on the side. grid (token chunks, n_kv, nl), 256 threads: warp w takes
+// the steps w, w + 8, ... of the chunk; lane (g, m) loads features 16 g .. 16 g + 15 of its four
+// tokens 2m, 2m+1, 2m+8, 2m+9 (one 4 / 8 / 16-byte load per code row for b = 2 / 4 / 8) and the
+// weights of query head 8 n + g; the warps' partials meet in shared memory, one atomic add per
+// (query head, feature) and CTA goes to the workspace accumulator.
 template <int BITS>
-__global__ void __launch_bounds__(128) k_values_res(const ValArgs a) {
-  constexpr int RB = kD * BITS / 8;        // bytes of one code row
-  constexpr uint32_t mask = (1u << BITS) - 1u;
-  __shared__ __align__(16) uint8_t cs[128][RB];
-  __shared__ __align__(16) __nv_bfloat16 pr[128][kMaxG];  // P~ as stored (bf16): 8 heads per 16-byte load
-  __shared__ float2 szs[128];
-  __shared__ __align__(16) float red[2][kMaxG][kD];
-  const int h = blockIdx.y, li = blockIdx.z, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+__device__ __forceinline__ int vres_feature(int mt, int hi, int g) {
+  return BITS == 2 ? 16 * g + 4 * (mt >> 1) + 2 * (mt & 1) + hi : BITS == 4 ? 16 * g + 2 * mt + hi : 16 * g + mt + 8 * hi;
+}
+
+template <int BITS, int NT>
+__global__ void __launch_bounds__(256) k_values_res_mma(const ValArgs a) {
+  constexpr int RB = kD * BITS / 8;  // bytes of one code row
+  constexpr int LW = BITS / 2;       // 32-bit words of a lane's 16 features
+  __shared__ float red[8 * NT][kD];
+  __shared__ float zsh[8 * NT];
+  const int h = blockIdx.y, li = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gr = lane >> 2, m4 = lane & 3;
   const int64_t qrow0 = int64_t(li) * a.n_q + int64_t(h) * a.gq;
   const int64_t rbase = (int64_t(li) * a.n_kv + h) * a.T;
-  float acc[kMaxG][4];
+  for (int e = threadIdx.x; e < 8 * NT * kD; e += blockDim.x) (&red[0][0])[e] = 0.f;
+  if (threadIdx.x < 8 * NT) zsh[threadIdx.x] = 0.f;
+  __syncthreads();
+  float acc[8][NT][4];
 #pragma unroll
-  for (int g = 0; g < kMaxG; ++g)
+  for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-    for (int f = 0; f < 4; ++f) acc[g][f] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+  float zacc[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) zacc[nt] = 0.f;
   const int t_beg = blockIdx.x * a.chunk, t_end = min(a.T, t_beg + a.chunk);
-  for (int tb = t_beg; tb < t_end; tb += 128) {
-    const int nt = min(128, t_end - tb);
-    __syncthreads();
-    if (threadIdx.x < nt) {
-      const int64_t rr = rbase + tb + threadIdx.x;
-      const uint4* src = reinterpret_cast<const uint4*>(a.codes + rr * RB);
+  // raw operands of one 16-token step (code words, scale/zero pairs, P~ pairs), loaded one step
+  // ahead of their use
+  struct Raw {
+    uint32_t w[4][LW];
+    uint32_t sz[4];
+    uint32_t pp[NT][2];
+  };
+  auto load = [&](int tb, Raw& r) {
+    const int tA = tb + 2 * m4;
 #pragma unroll
-      for (int q = 0; q < RB / 16; ++q) reinterpret_cast<uint4*>(cs[threadIdx.x])[q] = __ldg(src + q);
-      const __half2 szv = a.sz[rr];
-      szs[threadIdx.x] = make_float2(__low2float(szv), __high2float(szv));
-#pragma unroll
-      for (int g = 0; g < kMaxG; ++g)
-        pr[threadIdx.x][g] = g < a.gq ? a.ptil[(qrow0 + g) * a.ldp + tb + threadIdx.x] : __float2bfloat16_rn(0.f);
-    }
-    __syncthreads();
-    for (int tt = w; tt < nt; tt += 4) {
-      uint32_t word;
-      if (BITS == 2) word = cs[tt][lane];
-      else if (BITS == 4) word = reinterpret_cast<const uint16_t*>(cs[tt])[lane];
-      else word = reinterpret_cast<const uint32_t*>(cs[tt])[lane];
-      const float2 z = szs[tt];
-      float dv[4];
-#pragma unroll
-      for (int f = 0; f < 4; ++f) dv[f] = dequant((word >> (f * BITS)) & mask, z.x, z.y);
-      const uint4* p8 = reinterpret_cast<const uint4*>(pr[tt]);
-#pragma unroll
-      for (int g8 = 0; g8 < kMaxG / 8; ++g8) {
-        if (8 * g8 < a.gq) {
-          const uint4 pw = p8[g8];
-          const uint32_t pb[4] = {pw.x, pw.y, pw.z, pw.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 pv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pb[e]));
-#pragma unroll
-            for (int f = 0; f < 4; ++f) {
-              acc[8 * g8 + 2 * e][f] = fmaf(pv.x, dv[f], acc[8 * g8 + 2 * e][f]);
-              acc[8 * g8 + 2 * e + 1][f] = fmaf(pv.y, dv[f], acc[8 * g8 + 2 * e + 1][f]);
-            }
-          }
-        }
+    for (int k = 0; k < 4; ++k) {
+      const int t = tA + (k & 1) + 8 * (k >> 1);
+      const bool ok = t < t_end;
+      const uint8_t* row = a.codes + (rbase + t) * RB + 4 * LW * gr;
+      if (LW == 1) {
+        r.w[k][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(row)) : 0u;
+      } else if (LW == 2) {
+        const uint2 u = ok ? __ldg(reinterpret_cast<const uint2*>(row)) : make_uint2(0u, 0u);
+        r.w[k][0] = u.x; r.w[k][LW > 1 ? 1 : 0] = u.y;
+      } else {
+        const uint4 u = ok ? __ldg(reinterpret_cast<const uint4*>(row)) : make_uint4(0u, 0u, 0u, 0u);
+        r.w[k][0] = u.x; r.w[k][LW > 1 ? 1 : 0] = u.y; r.w[k][LW > 2 ? 2 : 0] = u.z; r.w[k][LW > 3 ? 3 : 0] = u.w;
       }
+      r.sz[k] = ok ? __ldg(reinterpret_cast<const uint32_t*>(a.sz + rbase + t)) : 0u;
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int j = 8 * nt + gr;
+      const __nv_bfloat16* pr = a.ptil + (qrow0 + j) * a.ldp;
+#pragma unroll
+      for (int k2 = 0; k2 < 2; ++k2) {
+        const int t = tA + 8 * k2;  // even: the pair (t, t + 1) is one aligned 4-byte word
+        uint32_t v = 0u;
+        if (j < a.gq) {
+          if (t + 1 < t_end) v = __ldg(reinterpret_cast<const uint32_t*>(pr + t));
+          else if (t < t_end) v = uint32_t(__ldg(reinterpret_cast<const unsigned short*>(pr + t)));
+        }
+        r.pp[nt][k2] = v;
+      }
+    }
+  };
+  Raw nxt;
+  int tb = t_beg + 16 * warp;
+  if (tb < t_end) load(tb, nxt);
+  for (; tb < t_end; tb += 16 * 8) {
+    const Raw cur = nxt;
+    if (tb + 16 * 8 < t_end) load(tb + 16 * 8, nxt);
+    float sc[4], zr[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&cur.sz[k]));
+      sc[k] = f.x;
+      zr[k] = f.y;
+    }
+    // weights of query heads 8 nt + g: B fragments (tokens 2m, 2m+1 | 2m+8, 2m+9)
+    uint32_t bw[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const float2 p01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cur.pp[nt][0]));
+      const float2 p23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cur.pp[nt][1]));
+      zacc[nt] += (p01.x * zr[0] + p01.y * zr[1]) + (p23.x * zr[2] + p23.y * zr[3]);
+      const __half2 b0 = __floats2half2_rn(p01.x * sc[0], p01.y * sc[1]);
+      const __half2 b1 = __floats2half2_rn(p23.x * sc[2], p23.y * sc[3]);
+      bw[nt][0] = *reinterpret_cast<const uint32_t*>(&b0);
+      bw[nt][1] = *reinterpret_cast<const uint32_t*>(&b1);
+    }
+    const uint32_t(&w)[4][LW] = cur.w;
+    // A fragments straight from the code words, eight m-tiles
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      uint32_t af[4];
+      if (BITS == 2) {
+        const int bb = mt >> 1, s0 = 2 * (mt & 1);
+        const uint32_t xab = bytes_xy(w[0][0], w[1][0], bb), xcd = bytes_xy(w[2][0], w[3][0], bb);
+        af[0] = crumb(xab, s0); af[1] = crumb(xab, s0 + 1);
+        af[2] = crumb(xcd, s0); af[3] = crumb(xcd, s0 + 1);
+      } else if (BITS == 4) {
+        const int wi = (mt >> 2) & (LW - 1), bb = mt & 3;
+        const uint32_t xab = bytes_xy(w[0][wi], w[1][wi], bb), xcd = bytes_xy(w[2][wi], w[3][wi], bb);
+        af[0] = nib_lo(xab); af[1] = nib_hi(xab);
+        af[2] = nib_lo(xcd); af[3] = nib_hi(xcd);
+      } else {
+        const int wl = (mt >> 2) & (LW - 1), wh = (2 + (mt >> 2)) & (LW - 1), bb = mt & 3;
+        af[0] = byte_lo(bytes_xy(w[0][wl], w[1][wl], bb)); af[1] = byte_lo(bytes_xy(w[0][wh], w[1][wh], bb));
+        af[2] = byte_lo(bytes_xy(w[2][wl], w[3][wl], bb)); af[3] = byte_lo(bytes_xy(w[2][wh], w[3][wh], bb));
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_f16_16816(acc[mt][nt], af, bw[nt][0], bw[nt][1]);
     }
   }
-  // warps 2, 3 -> shared; warps 0, 1 add; warp 1 -> shared; warp 0 adds and commits
-  __syncthreads();
-  if (w >= 2)
+  // the warps' partials in shared memory, then one global add per (query head, feature)
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g)
-      if (g < a.gq) *reinterpret_cast<float4*>(&red[w - 2][g][4 * lane]) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
-  __syncthreads();
-  if (w < 2)
+  for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g)
-      if (g < a.gq) {
-        const float4 o = *reinterpret_cast<const float4*>(&red[w][g][4 * lane]);
-        acc[g][0] += o.x; acc[g][1] += o.y; acc[g][2] += o.z; acc[g][3] += o.w;
-      }
+    for (int mt = 0; mt < 8; ++mt) {
+      const int f0 = vres_feature<BITS>(mt, 0, gr), f1 = vres_feature<BITS>(mt, 1, gr);
+      const int j = 8 * nt + 2 * m4;
+      atomicAdd(&red[j][f0], acc[mt][nt][0]);
+      atomicAdd(&red[j + 1][f0], acc[mt][nt][1]);
+      atomicAdd(&red[j][f1], acc[mt][nt][2]);
+      atomicAdd(&red[j + 1][f1], acc[mt][nt][3]);
+    }
+    float z = zacc[nt];
+    z += __shfl_xor_sync(0xffffffffu, z, 1);
+    z += __shfl_xor_sync(0xffffffffu, z, 2);
+    if (m4 == 0) atomicAdd(&zsh[8 * nt + gr], z);
+  }
   __syncthreads();
-  if (w == 1)
-#pragma unroll
-    for (int g = 0; g < kMaxG; ++g)
-      if (g < a.gq) *reinterpret_cast<float4*>(&red[0][g][4 * lane]) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
-  __syncthreads();
-  if (w == 0)
-#pragma unroll
-    for (int g = 0; g < kMaxG; ++g)
-      if (g < a.gq) {
-        const float4 o = *reinterpret_cast<const float4*>(&red[0][g][4 * lane]);
-        float* dst = &a.acc[(qrow0 + g) * kD + 4 * lane];
-        atomicAdd(dst + 0, acc[g][0] + o.x);
-        atomicAdd(dst + 1, acc[g][1] + o.y);
-        atomicAdd(dst + 2, acc[g][2] + o.z);
-        atomicAdd(dst + 3, acc[g][3] + o.w);
-      }
+  for (int e = threadIdx.x; e < a.gq * kD; e += blockDim.x) {
+    const int j = e / kD, d = e % kD;
+    atomicAdd(&a.acc[(qrow0 + j) * kD + d], red[j][d] + zsh[j]);
+  }
 }
 
 struct FinArgs {
@@ -636,49 +737,84 @@ struct FinArgs {
   float* lse;                // [nl][n_q] or null
 };
 
-// out = (U_d^V (G_h^V^T w) + R^T acc) / l, lse = m + log l for one query head.
-// grid (n_kv, nl, g_q), 128 threads; dynamic smem: w [r_T] floats.
-__global__ void __launch_bounds__(128) k_finalize(const FinArgs a) {
-  extern __shared__ float w[];
-  __shared__ float v[kD];
-  __shared__ float x[kD];
-  const int h = blockIdx.x, li = blockIdx.y, g = blockIdx.z, tid = threadIdx.x;
-  const int64_t qr = int64_t(li) * a.n_q + int64_t(h) * a.gq + g;
-  for (int r = tid; r < a.r_T; r += blockDim.x) w[r] = a.W[qr * a.q_cap + r];
-  x[tid] = a.bits ? a.acc[qr * kD + tid] : 0.f;
+// out = (U_d^V (G_h^V^T w) + R^T acc) / l, lse = m + log l for the g_q query heads of one KV head.
+// grid (n_kv, nl), 512 threads; dynamic shared memory: w [g_q][r_T], v partials [4][g_q][128],
+// v [g_q][128], x [g_q][128]. G_h^V is read once for all g_q heads: thread (j, quarter) takes rows
+// r = quarter, quarter + 4, ... of column j; the U_d^V rows are read by one warp each (lanes over
+// the r_d columns) and reduced per query head.
+__global__ void __launch_bounds__(512) k_finalize(const FinArgs a) {
+  extern __shared__ float fsm[];
+  const int gq = a.gq, rT = a.r_T, rd = a.r_d;
+  float* w = fsm;                          // [gq][rT]
+  float* vp = w + gq * max(rT, 1);         // [4][gq][128]
+  float* v = vp + 4 * gq * kD;             // [gq][128]
+  float* x = v + gq * kD;                  // [gq][128]
+  const int h = blockIdx.x, li = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t qr0 = int64_t(li) * a.n_q + int64_t(h) * gq;
+  for (int e = tid; e < gq * rT; e += blockDim.x) w[e] = a.W[(qr0 + e / rT) * a.q_cap + e % rT];
+  for (int e = tid; e < gq * kD; e += blockDim.x) x[e] = a.bits ? a.acc[qr0 * kD + e] : 0.f;
   __syncthreads();
-  // v[j] = sum_r G[r][j] w[r]
-  if (tid < a.r_d) {
-    const __nv_bfloat16* G = a.G + (int64_t(li) * a.n_kv + h) * a.r_T * a.r_d + tid;
-    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-    int r = 0;
-    for (; r + 4 <= a.r_T; r += 4) {
-      s0 = fmaf(__bfloat162float(G[int64_t(r) * a.r_d]), w[r], s0);
-      s1 = fmaf(__bfloat162float(G[int64_t(r + 1) * a.r_d]), w[r + 1], s1);
-      s2 = fmaf(__bfloat162float(G[int64_t(r + 2) * a.r_d]), w[r + 2], s2);
-      s3 = fmaf(__bfloat162float(G[int64_t(r + 3) * a.r_d]), w[r + 3], s3);
+  {
+    const int j = tid & (kD - 1), qt = tid >> 7;
+    float s[kMaxG];
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g) s[g] = 0.f;
+    if (j < rd && rT > 0) {
+      const __nv_bfloat16* G = a.G + (int64_t(li) * a.n_kv + h) * rT * rd + j;
+#pragma unroll 8
+      for (int r = qt; r < rT; r += 4) {
+        const float gv = __bfloat162float(G[int64_t(r) * rd]);
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < gq) s[g] = fmaf(gv, w[g * rT + r], s[g]);
+      }
     }
-    for (; r < a.r_T; ++r) s0 = fmaf(__bfloat162float(G[int64_t(r) * a.r_d]), w[r], s0);
-    v[tid] = (s0 + s1) + (s2 + s3);
+#pragma unroll
+    for (int g = 0; g < kMaxG; ++g)
+      if (g < gq) vp[(qt * gq + g) * kD + j] = s[g];
   }
-  // inverse rotation of the residual accumulator (one warp)
-  if (a.bits && tid < 32) {
+  __syncthreads();
+  for (int e = tid; e < gq * kD; e += blockDim.x) {
+    const int j = e % kD;
+    v[e] = j < rd ? (vp[e] + vp[gq * kD + e]) + (vp[2 * gq * kD + e] + vp[3 * gq * kD + e]) : 0.f;
+  }
+  // inverse rotation of each head's residual accumulator (one warp per head)
+  if (a.bits && warp < gq) {
     float xv[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) xv[i] = x[tid * 4 + i];
+    for (int i = 0; i < 4; ++i) xv[i] = x[warp * kD + lane * 4 + i];
     warp_unrotate<4>(xv, a.rot_seed, rsqrtf(float(kD)));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) x[tid * 4 + i] = xv[i];
+    for (int i = 0; i < 4; ++i) x[warp * kD + lane * 4 + i] = xv[i];
   }
   __syncthreads();
-  float o = x[tid];
-  if (a.r_T > 0) {
-    const __nv_bfloat16* ud = a.Ud + int64_t(tid) * a.r_d;
-    for (int jj = 0; jj < a.r_d; ++jj) o = fmaf(__bfloat162float(ud[jj]), v[jj], o);
+  // each warp's eight U_d rows are loaded before any is used
+  float udr[kD / 16][4];
+#pragma unroll
+  for (int u = 0; u < kD / 16; ++u)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = warp + 16 * u, j = lane * 4 + k;
+      udr[u][k] = (rT > 0 && j < rd) ? __bfloat162float(a.Ud[int64_t(i) * rd + j]) : 0.f;
+    }
+#pragma unroll
+  for (int u = 0; u < kD / 16; ++u) {
+    const int i = warp + 16 * u;
+    const float(&ud)[4] = udr[u];
+    for (int g = 0; g < gq; ++g) {
+      const float* vg = v + g * kD + lane * 4;
+      float o = (ud[0] * vg[0] + ud[1] * vg[1]) + (ud[2] * vg[2] + ud[3] * vg[3]);
+      o = warp_sum(o);
+      if (lane == 0) {
+        const int64_t qr = qr0 + g;
+        a.out[qr * kD + i] = __float2bfloat16_rn((x[g * kD + i] + o) / a.lrow[qr]);
+      }
+    }
   }
-  a.out[qr * kD + tid] = __float2bfloat16_rn(o / a.lrow[qr]);
-  if (tid == 0 && a.lse) a.lse[qr] = a.mrow[qr] + logf(a.lrow[qr]);
+  if (tid < gq && a.lse) a.lse[qr0 + tid] = a.mrow[qr0 + tid] + logf(a.lrow[qr0 + tid]);
 }
+
+size_t finalize_smem(int gq, int r_T) { return (size_t(gq) * std::max(r_T, 1) + size_t(6) * gq * kD) * sizeof(float); }
 
 int grid1(int64_t n) { return int(std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 148 * 16))); }
 
@@ -731,6 +867,15 @@ jolt_status launch_keys(const KeysMaps& maps, const KeysArgs& a, cudaStream_t st
     if (kDebug)
       std::fprintf(stderr, "jolt: k_keys_tc needs %d threads, registers allow %d (%d per thread)\n",
                    KeysCfg<NT>::kThreads, fa.maxThreadsPerBlock, fa.numRegs);
+    return JOLT_ERR_CUDA;
+  }
+  // the warpgroups re-split the block's registers (setmaxnreg): the decreases must not exceed and
+  // the increase must not fall below the launch count, and the new shares must fit what the block
+  // was launched with, or the increasing warpgroup would wait for registers that never come
+  using C = KeysCfg<NT>;
+  if (fa.numRegs < C::kRegCtl || fa.numRegs < C::kRegScore || fa.numRegs > C::kRegRes ||
+      128 * (C::kRegCtl + C::kRegRes + 2 * C::kRegScore) > C::kThreads * fa.numRegs) {
+    if (kDebug) std::fprintf(stderr, "jolt: k_keys_tc launched with %d registers a thread\n", fa.numRegs);
     return JOLT_ERR_CUDA;
   }
   JOLT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, KeysCfg<NT>::kSmem));
@@ -911,14 +1056,33 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
       if (cv.bits) {
         ValArgs va{};
         va.T = T; va.n_kv = n_kv; va.gq = gq; va.n_q = nq; va.bits = cv.bits; va.ldp = Tp;
-        va.chunk = 512;
+        // one wave: as many CTAs as fit on the device at once, spread over the group's (layer, KV
+        // head) pairs (a second, partial wave would double the time of the last CTAs)
+        const void* kv = gq <= 8 ? (cv.bits == 2 ? (const void*)k_values_res_mma<2, 1>
+                                               : cv.bits == 4 ? (const void*)k_values_res_mma<4, 1>
+                                                              : (const void*)k_values_res_mma<8, 1>)
+                                 : (cv.bits == 2 ? (const void*)k_values_res_mma<2, 2>
+                                               : cv.bits == 4 ? (const void*)k_values_res_mma<4, 2>
+                                                              : (const void*)k_values_res_mma<8, 2>);
+        int per_sm = 0, dev = 0, nsm = 0;
+        JOLT_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kv, 256, 0));
+        JOLT_CUDA_TRY(cudaGetDevice(&dev));
+        JOLT_CUDA_TRY(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+        const int nch = std::max(1, std::min(std::max(1, per_sm) * nsm / (n_kv * nl), (T + 1023) / 1024));
+        va.chunk = ((T + nch - 1) / nch + 15) / 16 * 16;
         va.codes = cv.codes + res_off * (kD * cv.bits / 8);
         va.sz = cv.sz + res_off;
         va.ptil = ptil; va.acc = acc;
         const dim3 vg((T + va.chunk - 1) / va.chunk, n_kv, nl);
-        if (cv.bits == 2) k_values_res<2><<<vg, 128, 0, st>>>(va);
-        else if (cv.bits == 4) k_values_res<4><<<vg, 128, 0, st>>>(va);
-        else k_values_res<8><<<vg, 128, 0, st>>>(va);
+        if (gq <= 8) {
+          if (cv.bits == 2) k_values_res_mma<2, 1><<<vg, 256, 0, st>>>(va);
+          else if (cv.bits == 4) k_values_res_mma<4, 1><<<vg, 256, 0, st>>>(va);
+          else k_values_res_mma<8, 1><<<vg, 256, 0, st>>>(va);
+        } else {
+          if (cv.bits == 2) k_values_res_mma<2, 2><<<vg, 256, 0, st>>>(va);
+          else if (cv.bits == 4) k_values_res_mma<4, 2><<<vg, 256, 0, st>>>(va);
+          else k_values_res_mma<8, 2><<<vg, 256, 0, st>>>(va);
+        }
         JOLT_CUDA_TRY(cudaGetLastError());
       }
       // ---- finalize ----
@@ -930,7 +1094,9 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
       fa.W = W; fa.acc = acc; fa.mrow = mrow; fa.lrow = lrow;
       fa.out = oall + row0 * kD;
       fa.lse = p.lse ? p.lse + row0 : nullptr;
-      k_finalize<<<dim3(n_kv, nl, gq), 128, size_t(std::max(cv.r_T, 1)) * 4, st>>>(fa);
+      const size_t fsm = finalize_smem(gq, cv.r_T);
+      if (fsm > 48 * 1024) JOLT_CUDA_TRY(cudaFuncSetAttribute(k_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, int(fsm)));
+      k_finalize<<<dim3(n_kv, nl), 512, fsm, st>>>(fa);
       JOLT_CUDA_TRY(cudaGetLastError());
     }
   }

@@ -120,3 +120,12 @@ def test_70b_shape_gqa8_two_row_tiles(cuda_ok):
         rng = np.random.default_rng(7)
         ch = [(int(rng.integers(1, 9)) * 32, 128, int(rng.choice([2, 4]))) for _ in range(2)]
         run_case(w, ch, 1e-2, layer_calls=[(0, 4)], pos_offset=11)
+
+
+def test_gqa16_value_residual_two_head_tiles(cuda_ok):
+    # 16 query heads per KV head: the value-residual MMA runs two 8-head column tiles; ragged T,
+    # value codes of every width, keys with and without RoPE
+    for pre in (False, True):
+        w = get_workload("llama8b_layer", n_kv=2, T=531, keys_pre_rope=pre)
+        ch = [(64, 96, 4), (48, 128, 8)] if pre else [(32, 128, 2), (80, 64, 2)]
+        run_case(w, ch, 1e-2, pos_offset=9)
