@@ -44,11 +44,12 @@ template <int NT>
 struct KeysCfg {
   static constexpr int kStages = NT == 1 ? 4 : 3;
   static constexpr int kStageBytes = kABytes + NT * kBBytes;
-  static constexpr int kQsBytes = 2 * kMaxG * kD * 4;      // queries of each score group's pair, fp32
+  static constexpr int kQbBytes = 16 * kD * 2;             // a score group's queries: B of q . k (16 x 128 bf16)
   static constexpr int kRopeBytes = kD / 4 * kBM * 16;     // (cos, cos, sin, sin) of frequency pairs
-  static constexpr int kSmem = 1024 + kStages * kStageBytes + kQsBytes + kRopeBytes + kD * 4 + 256;
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + 2 * kQbBytes + kRopeBytes + kD * 4 + 256;
   static constexpr int kThreads = 512;                     // four warpgroups: control, residual, 2 x score
-  static constexpr int kNB = 4;                            // TMEM key buffers of 128 columns
+  static constexpr int kNB = 3;                            // TMEM key buffers of 128 columns
+  static constexpr int kScoreCol = kNB * 128;              // q . k accumulators: 16 columns per score group
   // registers a thread after the warpgroups' re-split (launch: 128 each, 65536 in all)
   static constexpr int kRegCtl = 40, kRegRes = 200, kRegScore = 120;
 };
@@ -72,8 +73,6 @@ struct KeysArgs {
   int32_t* err;
 };
 
-// Named barrier of one epilogue group (ids 1 and 2; 0 is __syncthreads).
-__device__ __forceinline__ void group_bar(int g) { asm volatile("bar.sync %0, 128;" ::"r"(1 + g) : "memory"); }
 
 // Residual row of one token: 128 codes of BITS bits (little-endian bit stream) as floats.
 template <int BITS>
@@ -147,24 +146,32 @@ __device__ __forceinline__ void fwht128x2(float2 (&v)[kD / 2]) {
 }
 
 // grid.x = token tiles; 512 threads in four warpgroups with re-split register budgets:
-//   warpgroup 0: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warps 2-3 idle after setup;
+//   warpgroup 0: warp 0 TMA producer, warp 1 key-MMA issuer (+ TMEM owner), warp 2 score-MMA
+//                issuer, warp 3 idle after setup;
 //   warpgroup 1: residual warps — thread = token row of the tile (warp w: TMEM lanes 32 (w % 4) ..
 //                +31); per (layer, KV head) pair they dequantise the residual row, undo the
 //                rotation (FWHT and signs) and store it into the pair's TMEM key buffer, on which
-//                the MMAs then accumulate U_T B_h (so the key arrives complete in TMEM);
-//   warpgroups 2, 3: two score groups taking alternate pairs: RoPE at the token's position and
-//                q . k for the pair's g_q query heads, straight from TMEM in 16-column pieces.
-// Four TMEM buffers of 128 columns rotate over the pairs: residual -> MMA -> score.
+//                the key MMAs then accumulate U_T B_h (so the key arrives complete in TMEM);
+//   warpgroups 2, 3: two score groups taking alternate pairs: they read the key in 16-column
+//                pieces, apply RoPE at the token's position and write the rotated key back in place
+//                as bf16 hi and lo halves (columns 0-63 and 64-127 of the buffer); a tensor-core
+//                product with the pair's queries (A = the rotated key in TMEM, B = the g_q query
+//                rows in shared memory, N = 16) then forms q . k, which the group reads back.
+// Three TMEM key buffers of 128 columns rotate over the pairs: residual -> key MMA -> RoPE ->
+// score MMA -> free; each score group has its own 16 accumulator columns.
+// The queries' features are ordered to match the rotated key's column layout: K index 32 c + r is
+// feature 16 c + r for r < 16 and feature 64 + 16 c + (r - 16) otherwise (c = 0 .. 3).
 template <int BITS, int NT>
 __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ KeysMaps maps, const KeysArgs p) {
   using C = KeysCfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = sm100::align_smem_1024(smem_raw);
-  float* qs = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);  // [2 groups][kMaxG][kD]
-  float4* rope = reinterpret_cast<float4*>(qs + 2 * kMaxG * kD);            // [32][kBM]
+  uint8_t* qb_all = smem + C::kStages * C::kStageBytes;                      // [2 groups][16][128] bf16, SW128
+  float4* rope = reinterpret_cast<float4*>(qb_all + 2 * C::kQbBytes);        // [32][kBM]
   float2* sgn = reinterpret_cast<float2*>(rope + kD / 4 * kBM);               // [64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sgn + kD / 2);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 3 * C::kNB + 1);
+  constexpr int kNumBars = 2 * C::kStages + 4 * C::kNB + 2 + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kBM;
@@ -174,10 +181,12 @@ __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ Keys
   const uint32_t bar0 = sm100::smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
-  auto rfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };             // residual stored
-  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + C::kNB + b); };    // MMAs done
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 * C::kNB + b); };  // scores read it
-  const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 3 * C::kNB);
+  auto rfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };               // residual stored
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + C::kNB + b); };      // key MMAs done
+  auto afull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 * C::kNB + b); };  // rotated key stored
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 3 * C::kNB + b); }; // score MMAs done
+  auto sfull_bar = [&](int g) { return bar0 + 8u * (2 * C::kStages + 4 * C::kNB + g); };  // q . k ready
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 4 * C::kNB + 2);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -187,9 +196,11 @@ __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ Keys
     for (int b = 0; b < C::kNB; ++b) {
       sm100::mbar_init(rfull_bar(b), 4);  // one arrival per residual warp
       sm100::mbar_init(tfull_bar(b), 1);
-      sm100::mbar_init(tempty_bar(b), 4);  // one arrival per warp of the score group
+      sm100::mbar_init(afull_bar(b), 4);  // one arrival per warp of the score group
+      sm100::mbar_init(tempty_bar(b), 1);
     }
-    sm100::mbar_init(drain_bar, 1);
+    for (int g = 0; g < 2; ++g) sm100::mbar_init(sfull_bar(g), 1);
+    sm100::mbar_init(drain_bar, 2);  // one commit per MMA-issuing thread
     sm100::fence_mbar_init();
     if (fac) {
       sm100::prefetch_tmap(&maps.a);
@@ -213,7 +224,10 @@ __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ Keys
     }
     rope[e] = make_float4(cs[0] * p.rope_scaling, cs[1] * p.rope_scaling, sn[0] * p.rope_scaling, sn[1] * p.rope_scaling);
   }
-  if (warp == 1) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), 128 * C::kNB);
+  // the query tiles start as zeros: rows g_q .. 15 stay zero
+  for (int e = threadIdx.x; e < 2 * C::kQbBytes / 16; e += blockDim.x)
+    reinterpret_cast<uint4*>(qb_all)[e] = make_uint4(0u, 0u, 0u, 0u);
+  if (warp == 1) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), 512);
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
@@ -253,12 +267,12 @@ __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ Keys
       // wait (bounded) for the copies still in flight before the block may exit
       for (int i = max(0, it - C::kStages); i < it; ++i)
         sm100::mbar_wait(full_bar(i % C::kStages), (i / C::kStages) & 1, p.err);
-    } else if (warp == 1 && lane == 0 && fac) {
-      // ---- MMA issuer: D[pr % kNB] (= residual, or nothing for b = 0) += sum_k U_T (B_hi + B_lo) ----
+    } else if (warp == 1 && lane == 0) {
+      // ---- key MMAs: D[pr % kNB] (= residual, or nothing for b = 0) += sum_k U_T (B_hi + B_lo) ----
       constexpr uint32_t idesc = sm100::idesc_bf16_f32(kBM, kD, 0, 1);
       int it = 0;
       bool ok = true;
-      for (int pr = 0; pr < npairs && ok; ++pr) {
+      for (int pr = 0; pr < npairs && ok && fac; ++pr) {
         const int bi = pr % C::kNB;
         if (!sm100::mbar_wait(rfull_bar(bi), (pr / C::kNB) & 1, p.err)) break;
         sm100::tc_fence_after();
@@ -287,6 +301,27 @@ __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ Keys
       // every MMA this thread issued has completed before TMEM is released
       sm100::mma_commit(drain_bar);
       sm100::mbar_wait(drain_bar, 0, p.err);
+    } else if (warp == 2 && lane == 0) {
+      // ---- score MMAs: q . k[g] = (rotated key hi + lo, in TMEM) x (queries of the pair) ----
+      constexpr uint32_t idesc = sm100::idesc_bf16_f32(kBM, 16, 0, 0);
+      for (int pr = 0; pr < npairs; ++pr) {
+        const int bi = pr % C::kNB, g = pr & 1;
+        if (!sm100::mbar_wait(afull_bar(bi), (pr / C::kNB) & 1, p.err)) break;
+        sm100::tc_fence_after();
+        const uint32_t qb = sbase + uint32_t(qb_all - smem) + g * C::kQbBytes;
+        const uint32_t dt = tmem + C::kScoreCol + 16 * g;
+#pragma unroll
+        for (int term = 0; term < 2; ++term)
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint64_t bd = sm100::smem_desc_sw128(qb + (kk >> 2) * (16 * 128) + (kk & 3) * 32, 16, 1024);
+            sm100::mma_bf16_tmem_a(dt, tmem + bi * kD + term * (kD / 2) + kk * 8, bd, idesc, (term > 0 || kk > 0) ? 1u : 0u);
+          }
+        sm100::mma_commit(sfull_bar(g));
+        sm100::mma_commit(tempty_bar(bi));
+      }
+      sm100::mma_commit(drain_bar);
+      sm100::mbar_wait(drain_bar, 0, p.err);
     }
   } else if (wg == 1) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::kRegRes));
@@ -307,11 +342,13 @@ __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ Keys
       zrv = __high2float(szv);
     };
     if (BITS > 0 && valid) load_res(0);
+    // without a factor part (r_T = 0) the buffer starts as the residual alone, or as zeros
+    const bool store = BITS > 0 || !fac;
     for (int pr = 0; pr < npairs; ++pr) {
       const int bi = pr % C::kNB;
       float2 v[kD / 2];
-      if (BITS > 0) {
-        if (valid) {
+      if (store) {
+        if (BITS > 0 && valid) {
           dequant2<BITS>(cw, scv, zrv, v);
           if (pr + 1 < npairs) load_res(pr + 1);  // the next pair's row is in flight meanwhile
           fwht128x2(v);
@@ -322,10 +359,10 @@ __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ Keys
           for (int m = 0; m < kD / 2; ++m) v[m] = make_float2(0.f, 0.f);
         }
       }
-      // the buffer is free once the score group has read the pair kNB earlier
+      // the buffer is free once the score MMAs of the pair kNB earlier have completed
       if (live) live = __all_sync(0xffffffffu, sm100::mbar_wait(tempty_bar(bi), ((pr / C::kNB) & 1) ^ 1, p.err));
       sm100::tc_fence_after();
-      if (BITS > 0) {
+      if (store) {
         const uint32_t ta = tmem + bi * kD + (uint32_t(quarter * 32) << 16);
 #pragma unroll
         for (int c = 0; c < kD / 32; ++c) {
@@ -352,8 +389,7 @@ __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ Keys
     const int et = threadIdx.x - 256 - 128 * g;
     const int t = t0 + row;
     const bool valid = t < p.T;
-    // queries as [g_q][32 frequency pairs m][q_2m, q_2m+1, q_2m+64, q_2m+65] (fp32)
-    float* qb = qs + g * kMaxG * kD;
+    uint8_t* qb = qb_all + g * C::kQbBytes;
     bool live = true;
     // a pair's g_q query rows (g_q * 128 bf16): thread et holds 8 consecutive values of each 1024,
     // loaded one pair ahead of their use
@@ -367,31 +403,27 @@ __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ Keys
         qn[j] = et + 128 * j < nq8 ? __ldg(src + et + 128 * j) : make_uint4(0u, 0u, 0u, 0u);
     };
     if (g < npairs) q_issue(g);
-    for (int pr = g; pr < npairs; pr += 2) {
+    int use = 0;  // pairs this group has taken
+    for (int pr = g; pr < npairs; pr += 2, ++use) {
       const int li = pr / p.n_kv, h = pr % p.n_kv;
       const int bi = pr % C::kNB;
+      // the pair's queries as B (16 x 128 bf16, K-major, 128-byte swizzle) in the key's column order;
+      // the previous pair's score MMAs, which read this tile, completed before its scores were read
 #pragma unroll
       for (int j = 0; j < kMaxG * kD / 1024; ++j) {
         const int e0 = (et + 128 * j) * 8;  // query row e0 / 128, features d0 .. d0 + 7
         if (e0 < p.gq * kD) {
-          const uint32_t wq[4] = {qn[j].x, qn[j].y, qn[j].z, qn[j].w};
-          const int gg = e0 / kD, d0 = e0 % kD;
-          const int hi = d0 >= kD / 2 ? 2 : 0, m0 = (d0 % (kD / 2)) / 2;
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float2 ff = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wq[u]));
-            *reinterpret_cast<float2*>(qb + gg * kD + 4 * (m0 + u) + hi) = ff;
-          }
+          const int n = e0 / kD, d0 = e0 % kD;
+          const int k0 = d0 < kD / 2 ? 32 * (d0 / 16) + d0 % 16 : 32 * ((d0 - kD / 2) / 16) + 16 + (d0 - kD / 2) % 16;
+          const int chunk = k0 / 64, within = k0 % 64;  // 8 bf16 = one 16-byte unit of the row
+          *reinterpret_cast<uint4*>(qb + chunk * (16 * 128) + n * 128 + (((within / 8) ^ (n & 7)) << 4)) = qn[j];
         }
       }
+      sm100::fence_proxy_async_smem();
       if (pr + 2 < npairs) q_issue(pr + 2);
-      group_bar(g);
       const uint32_t ready = fac ? tfull_bar(bi) : rfull_bar(bi);
       if (live) live = __all_sync(0xffffffffu, sm100::mbar_wait(ready, (pr / C::kNB) & 1, p.err));
       sm100::tc_fence_after();
-      float2 acc[kMaxG];
-#pragma unroll
-      for (int gg = 0; gg < kMaxG; ++gg) acc[gg] = make_float2(0.f, 0.f);
       const uint32_t ta = tmem + bi * kD + (uint32_t(quarter * 32) << 16);
 #pragma unroll
       for (int c = 0; c < kD / 32; ++c) {
@@ -399,6 +431,7 @@ __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ Keys
         sm100::tmem_ld16(ta + 16 * c, r1);           // features 16c .. 16c + 15
         sm100::tmem_ld16(ta + kD / 2 + 16 * c, r2);  // their RoPE partners, + 64
         sm100::tmem_ld_wait();
+        uint32_t hi[16], lo[16];  // hi: columns 16c .. 16c + 15, lo: the same + 64
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int m = 8 * c + k;  // features (2m, 2m+1) with (2m+64, 2m+65)
@@ -409,31 +442,39 @@ __global__ void __launch_bounds__(512, 1) k_keys_tc(const __grid_constant__ Keys
           const float2 a = __fmul2_rn(x2, sn), bb = __fmul2_rn(x1, sn);
           const float2 y1 = __ffma2_rn(x1, cs, make_float2(-a.x, -a.y));
           const float2 y2 = __ffma2_rn(x2, cs, bb);
-#pragma unroll
-          for (int gg = 0; gg < kMaxG; ++gg) {
-            if (gg < p.gq) {
-              const float4 qq = *reinterpret_cast<const float4*>(qb + gg * kD + 4 * m);
-              acc[gg] = __ffma2_rn(y1, make_float2(qq.x, qq.y), acc[gg]);
-              acc[gg] = __ffma2_rn(y2, make_float2(qq.z, qq.w), acc[gg]);
-            }
-          }
+          const __nv_bfloat162 h1 = __floats2bfloat162_rn(y1.x, y1.y), h2 = __floats2bfloat162_rn(y2.x, y2.y);
+          const float2 f1 = __bfloat1622float2(h1), f2 = __bfloat1622float2(h2);
+          const __nv_bfloat162 l1 = __floats2bfloat162_rn(y1.x - f1.x, y1.y - f1.y);
+          const __nv_bfloat162 l2 = __floats2bfloat162_rn(y2.x - f2.x, y2.y - f2.y);
+          hi[k] = *reinterpret_cast<const uint32_t*>(&h1);
+          hi[8 + k] = *reinterpret_cast<const uint32_t*>(&h2);
+          lo[k] = *reinterpret_cast<const uint32_t*>(&l1);
+          lo[8 + k] = *reinterpret_cast<const uint32_t*>(&l2);
         }
+        sm100::tmem_st16(ta + 16 * c, hi);
+        sm100::tmem_st16(ta + kD / 2 + 16 * c, lo);
       }
+      sm100::tmem_st_wait();
       sm100::tc_fence_before();
       __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(tempty_bar(bi));
+      if (lane == 0) sm100::mbar_arrive(afull_bar(bi));
+      if (live) live = __all_sync(0xffffffffu, sm100::mbar_wait(sfull_bar(g), use & 1, p.err));
+      sm100::tc_fence_after();
+      uint32_t sc[16];
+      sm100::tmem_ld16(tmem + C::kScoreCol + 16 * g + (uint32_t(quarter * 32) << 16), sc);
+      sm100::tmem_ld_wait();
+      sm100::tc_fence_before();
       if (valid && live) {
         float* out = p.scores + (int64_t(li) * p.n_q + int64_t(h) * p.gq) * p.T + t;
 #pragma unroll
         for (int gg = 0; gg < kMaxG; ++gg)
-          if (gg < p.gq) out[int64_t(gg) * p.T] = (acc[gg].x + acc[gg].y) * p.attn_scale;
+          if (gg < p.gq) out[int64_t(gg) * p.T] = __uint_as_float(sc[gg]) * p.attn_scale;
       }
-      group_bar(g);  // every thread is done with this pair's queries
     }
   }
   sm100::tc_fence_before();
   __syncthreads();
-  if (warp == 1) sm100::tmem_dealloc(tmem, 128 * C::kNB);
+  if (warp == 1) sm100::tmem_dealloc(tmem, 512);
 }
 
 // ---- CUDA-core stages -------------------------------------------------------------------------
@@ -610,7 +651,7 @@ __global__ void __launch_bounds__(256) k_values_res_mma(const ValArgs a) {
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) zacc[nt] = 0.f;
   const int t_beg = blockIdx.x * a.chunk, t_end = min(a.T, t_beg + a.chunk);
-  // raw operands of one 16-token step (code words, scale/zero pairs, P~ pairs), loaded one step
+  // raw operands of one 16-token step (code words, scale/zero pairs, P~ pairs), loaded two steps
   // ahead of their use
   struct Raw {
     uint32_t w[4][LW];
@@ -651,12 +692,15 @@ __global__ void __launch_bounds__(256) k_values_res_mma(const ValArgs a) {
       }
     }
   };
-  Raw nxt;
+  // two steps in flight ahead of the one being computed
+  Raw n1, n2;
   int tb = t_beg + 16 * warp;
-  if (tb < t_end) load(tb, nxt);
+  if (tb < t_end) load(tb, n1);
+  if (tb + 16 * 8 < t_end) load(tb + 16 * 8, n2);
   for (; tb < t_end; tb += 16 * 8) {
-    const Raw cur = nxt;
-    if (tb + 16 * 8 < t_end) load(tb + 16 * 8, nxt);
+    const Raw cur = n1;
+    n1 = n2;
+    if (tb + 2 * 16 * 8 < t_end) load(tb + 2 * 16 * 8, n2);
     float sc[4], zr[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -725,34 +769,45 @@ __global__ void __launch_bounds__(256) k_values_res_mma(const ValArgs a) {
 }
 
 struct FinArgs {
-  int n_kv, gq, n_q, r_T, r_d, bits, q_cap;
+  int n_kv, gq, n_q, q_cap, row_base;
   uint64_t rot_seed;
-  const __nv_bfloat16* G;    // value core of layer ll0: [nl][n_kv][r_T][r_d]
-  const __nv_bfloat16* Ud;   // [128][r_d]
-  const float* W;            // [nl][n_q][q_cap]
-  const float* acc;          // [nl][n_q][128]
-  const float* mrow;         // [nl][n_q]
+  const float* W;            // [rows][n_q][q_cap], rows = (b, layer) of the call
+  const float* acc;          // [rows][n_q][128]
+  const float* mrow;         // [rows][n_q]
   const float* lrow;
-  __nv_bfloat16* out;        // [nl][n_q][128] rows of (b, li0)
-  float* lse;                // [nl][n_q] or null
+  __nv_bfloat16* out;        // [rows][n_q][128]
+  float* lse;                // [rows][n_q] or null
+};
+
+// The value cell of one (sequence, layer) row: the layer's core, the group's U_d and the sizes.
+struct FinRow {
+  const __nv_bfloat16* G;    // [n_kv][r_T][r_d] of the row's layer
+  const __nv_bfloat16* Ud;   // [128][r_d]
+  int r_T, r_d, bits;
+};
+constexpr int kMaxFinRows = 512;
+struct FinTab {
+  FinRow row[kMaxFinRows];
 };
 
 // out = (U_d^V (G_h^V^T w) + R^T acc) / l, lse = m + log l for the g_q query heads of one KV head.
-// grid (n_kv, nl), 512 threads; dynamic shared memory: w [g_q][r_T], v partials [4][g_q][128],
+// One launch for the whole call after every group's values: grid (n_kv, rows of this launch),
+// 512 threads; dynamic shared memory: w [g_q][r_T], v partials [4][g_q][128],
 // v [g_q][128], x [g_q][128]. G_h^V is read once for all g_q heads: thread (j, quarter) takes rows
 // r = quarter, quarter + 4, ... of column j; the U_d^V rows are read by one warp each (lanes over
 // the r_d columns) and reduced per query head.
-__global__ void __launch_bounds__(512) k_finalize(const FinArgs a) {
+__global__ void __launch_bounds__(512) k_finalize(const FinArgs a, const __grid_constant__ FinTab tab) {
   extern __shared__ float fsm[];
-  const int gq = a.gq, rT = a.r_T, rd = a.r_d;
+  const FinRow fr = tab.row[blockIdx.y];
+  const int gq = a.gq, rT = fr.r_T, rd = fr.r_d;
   float* w = fsm;                          // [gq][rT]
   float* vp = w + gq * max(rT, 1);         // [4][gq][128]
   float* v = vp + 4 * gq * kD;             // [gq][128]
   float* x = v + gq * kD;                  // [gq][128]
-  const int h = blockIdx.x, li = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t qr0 = int64_t(li) * a.n_q + int64_t(h) * gq;
+  const int h = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t qr0 = int64_t(a.row_base + blockIdx.y) * a.n_q + int64_t(h) * gq;
   for (int e = tid; e < gq * rT; e += blockDim.x) w[e] = a.W[(qr0 + e / rT) * a.q_cap + e % rT];
-  for (int e = tid; e < gq * kD; e += blockDim.x) x[e] = a.bits ? a.acc[qr0 * kD + e] : 0.f;
+  for (int e = tid; e < gq * kD; e += blockDim.x) x[e] = fr.bits ? a.acc[qr0 * kD + e] : 0.f;
   __syncthreads();
   {
     const int j = tid & (kD - 1), qt = tid >> 7;
@@ -760,7 +815,7 @@ __global__ void __launch_bounds__(512) k_finalize(const FinArgs a) {
 #pragma unroll
     for (int g = 0; g < kMaxG; ++g) s[g] = 0.f;
     if (j < rd && rT > 0) {
-      const __nv_bfloat16* G = a.G + (int64_t(li) * a.n_kv + h) * rT * rd + j;
+      const __nv_bfloat16* G = fr.G + int64_t(h) * rT * rd + j;
 #pragma unroll 8
       for (int r = qt; r < rT; r += 4) {
         const float gv = __bfloat162float(G[int64_t(r) * rd]);
@@ -779,7 +834,7 @@ __global__ void __launch_bounds__(512) k_finalize(const FinArgs a) {
     v[e] = j < rd ? (vp[e] + vp[gq * kD + e]) + (vp[2 * gq * kD + e] + vp[3 * gq * kD + e]) : 0.f;
   }
   // inverse rotation of each head's residual accumulator (one warp per head)
-  if (a.bits && warp < gq) {
+  if (fr.bits && warp < gq) {
     float xv[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) xv[i] = x[warp * kD + lane * 4 + i];
@@ -795,7 +850,7 @@ __global__ void __launch_bounds__(512) k_finalize(const FinArgs a) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int i = warp + 16 * u, j = lane * 4 + k;
-      udr[u][k] = (rT > 0 && j < rd) ? __bfloat162float(a.Ud[int64_t(i) * rd + j]) : 0.f;
+      udr[u][k] = (rT > 0 && j < rd) ? __bfloat162float(fr.Ud[int64_t(i) * rd + j]) : 0.f;
     }
 #pragma unroll
   for (int u = 0; u < kD / 16; ++u) {
@@ -851,9 +906,9 @@ TcWs tc_layout(const jolt_shape& s, int Lc) {
   w.bh = take(s.keys_pre_rope ? nl * s.n_kv * qc * kD * 4 : 0);
   w.scores = take(nl * nq * T * 4);
   w.ptil = take(nl * nq * Tp * 2);
-  w.ml = take(2 * nl * nq * 4);
-  w.W = take(nl * nq * qc * 4);
-  w.acc = take(nl * nq * kD * 4);
+  w.ml = take(2 * B * Lc * nq * 4);
+  w.W = take(B * Lc * nq * qc * 4);
+  w.acc = take(B * Lc * nq * kD * 4);
   w.total = off;
   return w;
 }
@@ -932,8 +987,28 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
   float* mrow = reinterpret_cast<float*>(tcws + wl.ml);
   float* W = reinterpret_cast<float*>(tcws + wl.W);
   float* acc = reinterpret_cast<float*>(tcws + wl.acc);
-  const int nlmax = std::min(p.Lc, p.Lg);
-  float* lrow = mrow + size_t(nlmax) * nq;
+  const int nrows = p.B * p.Lc;  // (sequence, layer) rows of the call
+  float* lrow = mrow + size_t(nrows) * nq;
+  // the finalize table (passed by value at launch) holds rows fin_base .. fin_base + kMaxFinRows - 1
+  FinTab ftab;
+  int fin_base = 0, fin_rmax = 1;
+  auto fin_flush = [&](int upto) -> jolt_status {
+    if (upto <= fin_base) return JOLT_OK;
+    FinArgs fa{};
+    fa.n_kv = n_kv; fa.gq = gq; fa.n_q = nq; fa.q_cap = qc; fa.row_base = fin_base;
+    fa.rot_seed = p.rot_seed;
+    fa.W = reinterpret_cast<float*>(tcws + wl.W); fa.acc = reinterpret_cast<float*>(tcws + wl.acc);
+    fa.mrow = mrow; fa.lrow = lrow;
+    fa.out = static_cast<__nv_bfloat16*>(p.out);
+    fa.lse = p.lse;
+    const size_t fsm = finalize_smem(gq, fin_rmax);
+    if (fsm > 48 * 1024) JOLT_CUDA_TRY(cudaFuncSetAttribute(k_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, int(fsm)));
+    k_finalize<<<dim3(n_kv, upto - fin_base), 512, fsm, st>>>(fa, ftab);
+    JOLT_CUDA_TRY(cudaGetLastError());
+    fin_base = upto;
+    fin_rmax = 1;
+    return JOLT_OK;
+  };
   jolt_status r;
 
   // ---- per-call prologue: R q, sum(R q), P (non-RoPE, as hi + lo) ----
@@ -947,7 +1022,6 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
     }
   }
   const __nv_bfloat16* qall = static_cast<const __nv_bfloat16*>(p.q);
-  __nv_bfloat16* oall = static_cast<__nv_bfloat16*>(p.out);
 
   for (int b = 0; b < p.B; ++b) {
     for (int gi = 0; gi < p.Gc; ++gi) {
@@ -1035,18 +1109,20 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
       // ---- softmax rows ----
       {
         StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
-        k_softmax_rows<<<rows, 512, 0, st>>>(scores, T, Tp, mrow, lrow, ptil);
+        k_softmax_rows<<<rows, 512, 0, st>>>(scores, T, Tp, mrow + row0, lrow + row0, ptil);
         JOLT_CUDA_TRY(cudaGetLastError());
       }
       // ---- values ----
-      JOLT_CUDA_TRY(cudaMemsetAsync(W, 0, size_t(rows) * qc * 4, st));
-      if (cv.bits) JOLT_CUDA_TRY(cudaMemsetAsync(acc, 0, size_t(rows) * kD * 4, st));
+      float* Wg = W + row0 * qc;
+      float* accg = acc + row0 * kD;
+      JOLT_CUDA_TRY(cudaMemsetAsync(Wg, 0, size_t(rows) * qc * 4, st));
+      if (cv.bits) JOLT_CUDA_TRY(cudaMemsetAsync(accg, 0, size_t(rows) * kD * 4, st));
       if (cv.r_T > 0) {
         GemmCall gc;
         gc.M = rows; gc.N = cv.r_T; gc.K = T;
         gc.A[0] = op(ptil, kMajorK, T, rows, Tp);
         gc.B[0] = op(cv.Ut, kMajorMN, cv.r_T, T, cv.r_T);
-        gc.C = W; gc.ldc = qc; gc.err = p.err;
+        gc.C = Wg; gc.ldc = qc; gc.err = p.err;
         gc.k_split = 0;  // split K to fill whole waves
         gc.accumulate = true;
         gc.plan = s.gemm_plan;
@@ -1072,7 +1148,7 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
         va.chunk = ((T + nch - 1) / nch + 15) / 16 * 16;
         va.codes = cv.codes + res_off * (kD * cv.bits / 8);
         va.sz = cv.sz + res_off;
-        va.ptil = ptil; va.acc = acc;
+        va.ptil = ptil; va.acc = accg;
         const dim3 vg((T + va.chunk - 1) / va.chunk, n_kv, nl);
         if (gq <= 8) {
           if (cv.bits == 2) k_values_res_mma<2, 1><<<vg, 256, 0, st>>>(va);
@@ -1085,20 +1161,23 @@ jolt_status launch_decode_tc(const DecodeParams& p, const TcCellView* views, uin
         }
         JOLT_CUDA_TRY(cudaGetLastError());
       }
-      // ---- finalize ----
-      FinArgs fa{};
-      fa.n_kv = n_kv; fa.gq = gq; fa.n_q = nq; fa.r_T = cv.r_T; fa.r_d = cv.r_d; fa.bits = cv.bits; fa.q_cap = qc;
-      fa.rot_seed = p.rot_seed;
-      fa.G = cv.r_T ? cv.G + int64_t(ll0) * n_kv * cv.r_T * cv.r_d : nullptr;
-      fa.Ud = cv.Ud;
-      fa.W = W; fa.acc = acc; fa.mrow = mrow; fa.lrow = lrow;
-      fa.out = oall + row0 * kD;
-      fa.lse = p.lse ? p.lse + row0 : nullptr;
-      const size_t fsm = finalize_smem(gq, cv.r_T);
-      if (fsm > 48 * 1024) JOLT_CUDA_TRY(cudaFuncSetAttribute(k_finalize, cudaFuncAttributeMaxDynamicSharedMemorySize, int(fsm)));
-      k_finalize<<<dim3(n_kv, nl), 512, fsm, st>>>(fa);
-      JOLT_CUDA_TRY(cudaGetLastError());
+      // ---- the group's rows for the finalize launch (rows arrive in increasing order) ----
+      for (int l = 0; l < nl; ++l) {
+        const int row = b * p.Lc + li0 + l;
+        if (row - fin_base >= kMaxFinRows && (r = fin_flush(row))) return r;
+        FinRow& fr = ftab.row[row - fin_base];
+        fr.G = cv.r_T ? cv.G + int64_t(ll0 + l) * n_kv * cv.r_T * cv.r_d : nullptr;
+        fr.Ud = cv.Ud;
+        fr.r_T = cv.r_T;
+        fr.r_d = cv.r_d;
+        fr.bits = cv.bits;
+        fin_rmax = std::max(fin_rmax, cv.r_T);
+      }
     }
+  }
+  {
+    StatScope sc(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
+    if ((r = fin_flush(nrows))) return r;
   }
   return JOLT_OK;
 }

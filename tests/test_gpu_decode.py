@@ -129,3 +129,10 @@ def test_gqa16_value_residual_two_head_tiles(cuda_ok):
         w = get_workload("llama8b_layer", n_kv=2, T=531, keys_pre_rope=pre)
         ch = [(64, 96, 4), (48, 128, 8)] if pre else [(32, 128, 2), (80, 64, 2)]
         run_case(w, ch, 1e-2, pos_offset=9)
+
+
+def test_pre_rope_more_rows_than_one_finalize_launch(cuda_ok):
+    # 17 sequences x 32 layers = 544 (sequence, layer) rows: the output projection runs as two
+    # launches (512 rows, then the rest) after every group's values
+    w = get_workload("llama8b_64k_b4", batch=17, T=130)
+    run_case(w, uniform(w, (32, 32, 4)), 1e-2, pos_offset=2)
