@@ -13,8 +13,8 @@
 //   partials (m, l, W, acc) per split go to the workspace; k_decode_merge combines the splits and
 //            applies U_d^V G^V^T and the inverse rotation.
 // Where each contraction runs:
-//   * U_T^K P (M = 128 tokens, N = 32 query heads, K = r_T; P as bf16 hi and lo terms accumulated
-//     into the same columns) and W (M = 128 rank rows per chunk, N = 32 heads, K = tokens; U_T^V
+//   * U_T^K P (M = 128 tokens, N = 64: the 32 query heads' P as bf16 hi and lo columns, K = r_T)
+//     and W (M = 128 rank rows per chunk, N = 32 heads, K = tokens; U_T^V
 //     read MN-major, P~ K-major) on tcgen05 with TMEM accumulators, operands staged by TMA;
 //   * both residual contractions (codes . R q and P~-weighted codes) on mma.sync m16n8k16 with
 //     the f16 operands built in registers straight from the packed codes in shared memory (each
@@ -23,11 +23,12 @@
 //     traffic per contraction. The key residual is stored into the tile's TMEM score buffer first
 //     and the factor products accumulate on top of it, so the scores arrive complete.
 // Warp roles (512 threads, four warpgroups whose register budgets are re-split with setmaxnreg):
-//   0: warp 0 TMA producers (one lane per operand ring), warp 1 MMA issuer (owns TMEM);
+//   0: warp 0 TMA producers (one lane per operand ring), warp 1 score-product issuer (owns TMEM),
+//      warp 2 value-product issuer;
 //   1: key-residual warps (the MMAs for their 32 tokens, then the row into TMEM);
 //   2: softmax warps (thread = token of the tile: scores from TMEM, online softmax, P~);
 //   3: value warps (value-residual MMAs, 32 features each).
-// TMEM: two score buffers of 32 columns, W (32 columns per 128-rank chunk) from column 128, the
+// TMEM: two score buffers of 64 columns, W (32 columns per 128-rank chunk) from column 128, the
 // value-residual accumulators (8 columns per KV head) from column 384.
 #include <algorithm>
 #include <cmath>
@@ -149,6 +150,9 @@ __device__ __forceinline__ void kres_head(const uint8_t* cs, int k, int h, int q
                                           const float* qs, float* scr, const uint32_t* zrow) {
   constexpr int RB = 16 * BITS;
   const int gr = lane >> 2, m4 = lane & 3;
+  uint2 bqs[8];  // the head's query fragments, shared by both 16-token row blocks
+#pragma unroll
+  for (int kc = 0; kc < 8; ++kc) bqs[kc] = gr < GQ ? qf[((h * 8 + kc) * GQ + gr) * 4 + m4] : make_uint2(0u, 0u);
 #pragma unroll
   for (int mb = 0; mb < 2; ++mb) {
     const int rA = 32 * q + 16 * mb + gr;  // tile rows of fragment rows g and g + 8
@@ -186,9 +190,7 @@ __device__ __forceinline__ void kres_head(const uint8_t* cs, int k, int h, int q
         af[0] = byte_pair(xa[kc], 0x4240); af[2] = byte_pair(xa[kc], 0x4341);
         af[1] = byte_pair(xb[kc], 0x4240); af[3] = byte_pair(xb[kc], 0x4341);
       }
-      uint2 bq = make_uint2(0u, 0u);
-      if (gr < GQ) bq = qf[((h * 8 + kc) * GQ + gr) * 4 + m4];
-      mma_f16_16816(acc, af, bq.x, bq.y);
+      mma_f16_16816(acc, af, bqs[kc].x, bqs[kc].y);
     }
     // rows g (tile row rA) and g + 8, query heads 2 m4, 2 m4 + 1 of KV head h
     const uint32_t zA = zrow[16 * mb + gr];
@@ -258,7 +260,7 @@ __device__ __forceinline__ void vres_head(float (&ac)[2][4], const uint8_t* cs, 
 // The key residual of one tile for this warp's 32 tokens, head after head (a runtime loop: one
 // copy of the head's code per code width keeps the hot loop small), releasing each code stage.
 template <int BITS, int GQ>
-__device__ __noinline__ bool kres_tile(const uint8_t* cbase, uint32_t full0, uint32_t empty0, int& ckit, int q,
+__device__ __forceinline__ bool kres_tile(const uint8_t* cbase, uint32_t full0, uint32_t empty0, int& ckit, int q,
                                        int lane, const uint2* qf, const float* qs, float* scr,
                                        const uint32_t* zks, int32_t* err, bool ok) {
   constexpr int NKV = kNQ / GQ, hps = 8 / BITS;
@@ -283,7 +285,7 @@ __device__ __noinline__ bool kres_tile(const uint8_t* cbase, uint32_t full0, uin
 // The value residual of one tile for this warp's features, head after head; the accumulators of
 // head h live in TMEM columns tacc + 8 h of the warp's lane quarter (loaded, updated, stored back).
 template <int BITS, int GQ>
-__device__ __noinline__ bool vres_tile(const uint8_t* cbase, uint32_t full0, uint32_t empty0, int& cvit,
+__device__ __forceinline__ bool vres_tile(const uint8_t* cbase, uint32_t full0, uint32_t empty0, int& cvit,
                                        const uint2* wbp, uint32_t tacc, int vw, int lane, int32_t* err, bool ok) {
   constexpr int NKV = kNQ / GQ, hps = 8 / BITS;
   int s = 0;
@@ -369,6 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       uint32_t cnt = 1;
       if ((i >= 12 && i < 14) || (i >= 16 && i < 18) || (i >= 20 && i < 24) || i >= 29) cnt = 4;
       if (i >= 24 && i < 26) cnt = 5;
+      if (i == 28) cnt = 2;  // the drain: one commit per MMA-issuing thread
       sm100::mbar_init(bar0 + 8u * i, cnt);
     }
     sm100::fence_mbar_init();
@@ -381,8 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // S: two buffers of 32 columns; W (up to 8 chunks of 32 columns) from column 128; the value
-  // residual accumulators (8 columns per KV head) from column 384
+  // S: two buffers of 64 columns (hi and lo halves); W (up to 8 chunks of 32 columns) from column
+  // 128; the value residual accumulators (8 columns per KV head) from column 384
   const uint32_t tS = tmem, tW = tmem + 128, tAcc = tmem + 384;
 
   if (wg == 0) {
@@ -440,100 +443,58 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
         sm100::mbar_wait(full, (i / depth) & 1, a.err);
       }
     } else if (warp == 1 && lane == 0) {
-      // ================= MMA issuer =================
-      // Two chains share the thread: the score products S(it) += U_T^K (P_hi + P_lo) on the
-      // buffer the key-residual warps have filled (key ring), and the value products
-      // W += U_T^V^T P~(it') for the tile whose probabilities are ready (value ring). Whichever
-      // ring has a stage ready is served, so the two rings' copies overlap instead of adding up.
-      constexpr uint32_t idK = sm100::idesc_bf16_f32(kBM, kNQ, 0, 0);
-      constexpr uint32_t idW = sm100::idesc_bf16_f32(128, kNQ, 1, 0);
-      int kit = 0, vit = 0;
-      int itK = 0, kb = 0, itW = 0, wst = 0;  // score tile / chunk, value tile / stage within it
-      bool sfree = false, pready = false;
-      const int nws = 2 * nmc;                // value stages per tile
+      // ================= score-product issuer: S(it) += U_T^K (P_hi + P_lo) =================
+      // on the buffer the key-residual warps have filled (or overwriting it when there is no key
+      // residual); blocking waits, so the thread spends no issue slots while it waits
+      constexpr uint32_t idK = sm100::idesc_bf16_f32(kBM, 2 * kNQ, 0, 0);
       bool ok = true;
-      uint64_t idle0 = 0;  // start of the current idle stretch (read every 1024 idle polls)
-      int idle_polls = 0;
-      while (ok && (itK < ntl || itW < ntl)) {
-        bool progressed = false;
-        if (itK < ntl) {
-          if (nkb == 0) {
-            ++itK;
-            progressed = true;
-          } else {
-            if (!sfree) sfree = sm100::mbar_test_wait(BR_FULL(itK & 1), (itK >> 1) & 1);
-            const int s = kit % kKStages;
-            if (sfree && sm100::mbar_test_wait(BK_FULL(s), (kit / kKStages) & 1)) {
-              sm100::tc_fence_after();
-              const uint32_t dt = tS + (itK & 1) * kNQ;
-              const uint32_t ka = sb + kOffK + s * kKStageBytes;
+      int kit = 0;
+      for (int it = 0; it < ntl && ok && nkb > 0; ++it) {
+        if (!(ok = sm100::mbar_wait(BR_FULL(it & 1), (it >> 1) & 1, a.err))) break;
+        sm100::tc_fence_after();
+        const uint32_t dt = tS + (it & 1) * 2 * kNQ;
+        for (int kb = 0; kb < nkb; ++kb, ++kit) {
+          const int s = kit % kKStages;
+          if (!(ok = sm100::mbar_wait(BK_FULL(s), (kit / kKStages) & 1, a.err))) break;
+          sm100::tc_fence_after();
+          const uint32_t ka = sb + kOffK + s * kKStageBytes;
 #pragma unroll
-              for (int kk = 0; kk < kBK / 16; ++kk) {
-                const uint64_t ad = sm100::smem_desc_sw128(ka + kk * 32, 16, 1024);
+          for (int kk = 0; kk < kBK / 16; ++kk) {  // N = 64: P hi rows 0-31 and lo rows 32-63
+            const uint64_t ad = sm100::smem_desc_sw128(ka + kk * 32, 16, 1024);
+            const uint64_t bd = sm100::smem_desc_sw128(ka + kBM * kBK * 2 + kk * 32, 16, 1024);
+            sm100::mma_bf16(dt, ad, bd, idK, (bK > 0 || kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          sm100::mma_commit(BK_EMPTY(s));
+        }
+        if (ok) sm100::mma_commit(BS_FULL(it & 1));
+      }
+      sm100::mma_commit(BDRAIN);
+      sm100::mbar_wait(BDRAIN, 0, a.err);
+    } else if (warp == 2 && lane == 0) {
+      // ================= value-product issuer: W += U_T^V^T P~(it) =================
+      constexpr uint32_t idW = sm100::idesc_bf16_f32(128, kNQ, 1, 0);
+      bool ok = true;
+      int vit = 0;
+      for (int it = 0; it < ntl && ok; ++it) {
+        if (!(ok = sm100::mbar_wait(BP_FULL(it & 1), (it >> 1) & 1, a.err))) break;
+        for (int wst = 0; wst < 2 * nmc; ++wst, ++vit) {
+          const int s = vit % kVStages;
+          if (!(ok = sm100::mbar_wait(BV_FULL(s), (vit / kVStages) & 1, a.err))) break;
+          sm100::tc_fence_after();
+          const int mc = wst >> 1, h2 = wst & 1;
+          const uint32_t va = sb + kOffV + s * kVStageBytes;
+          const uint32_t pt = sb + kOffPt + (it & 1) * kPtBytes;
 #pragma unroll
-                for (int term = 0; term < 2; ++term) {  // P hi rows 0-31, P lo rows 32-63
-                  const uint64_t bd = sm100::smem_desc_sw128(ka + kBM * kBK * 2 + term * kNQ * 128 + kk * 32, 16, 1024);
-                  sm100::mma_bf16(dt, ad, bd, idK, (bK > 0 || kb > 0 || kk > 0 || term > 0) ? 1u : 0u);
-                }
-              }
-              sm100::mma_commit(BK_EMPTY(s));
-              ++kit;
-              if (++kb == nkb) {
-                sm100::mma_commit(BS_FULL(itK & 1));
-                kb = 0;
-                ++itK;
-                sfree = false;
-              }
-              progressed = true;
-            }
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = sm100::smem_desc_sw128(va + kk * 2048, 8192, 1024);
+            const uint64_t bd = sm100::smem_desc_sw128(pt + h2 * (kNQ * 128) + kk * 32, 16, 1024);
+            sm100::mma_bf16(tW + mc * kNQ, ad, bd, idW, (it > 0 || h2 > 0 || kk > 0) ? 1u : 0u);
           }
+          sm100::mma_commit(BV_EMPTY(s));
         }
-        if (itW < ntl) {
-          if (!pready) pready = sm100::mbar_test_wait(BP_FULL(itW & 1), (itW >> 1) & 1);
-          if (pready) {
-            if (wst < nws) {
-              const int s = vit % kVStages;
-              if (sm100::mbar_test_wait(BV_FULL(s), (vit / kVStages) & 1)) {
-                sm100::tc_fence_after();
-                const int mc = wst >> 1, h2 = wst & 1;
-                const uint32_t va = sb + kOffV + s * kVStageBytes;
-                const uint32_t pt = sb + kOffPt + (itW & 1) * kPtBytes;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const uint64_t ad = sm100::smem_desc_sw128(va + kk * 2048, 8192, 1024);
-                  const uint64_t bd = sm100::smem_desc_sw128(pt + h2 * (kNQ * 128) + kk * 32, 16, 1024);
-                  sm100::mma_bf16(tW + mc * kNQ, ad, bd, idW, (itW > 0 || h2 > 0 || kk > 0) ? 1u : 0u);
-                }
-                sm100::mma_commit(BV_EMPTY(s));
-                ++vit;
-                ++wst;
-                progressed = true;
-              }
-            }
-            if (wst == nws) {
-              sm100::tc_fence_after();
-              sm100::mma_commit(BW_DONE(itW & 1));
-              sm100::mma_commit(BP_EMPTY(itW & 1));
-              wst = 0;
-              ++itW;
-              pready = false;
-              progressed = true;
-            }
-          }
-        }
-        if (progressed) {
-          idle0 = 0;
-          idle_polls = 0;
-        } else if (++idle_polls == 1024) {
-          idle_polls = 0;
-          const uint64_t now = sm100::global_ns();
-          if (idle0 == 0) {
-            idle0 = now;
-          } else if (now - idle0 > 2000000000ull) {
-            report_error(a.err, JOLT_ERR_TIMEOUT);
-            ok = false;
-          }
-        }
+        if (!ok) break;
+        sm100::mma_commit(BW_DONE(it & 1));
+        sm100::mma_commit(BP_EMPTY(it & 1));
       }
       sm100::mma_commit(BDRAIN);
       sm100::mbar_wait(BDRAIN, 0, a.err);
@@ -592,10 +553,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BS_EMPTY(it & 1), ((it >> 1) & 1) ^ 1, a.err));
       sm100::tc_fence_after();
       if (bK || nkb == 0) {
+        // the residual into the hi columns, zeros into the lo columns (the products accumulate)
         uint32_t r[kNQ];
+        const uint32_t ta = tS + (it & 1) * 2 * kNQ + (uint32_t(32 * q) << 16);
 #pragma unroll
         for (int j = 0; j < kNQ; ++j) r[j] = bK ? __float_as_uint(scr[lane * kScrStride + j]) : 0u;
-        sm100::tmem_st32(tS + (it & 1) * kNQ + (uint32_t(32 * q) << 16), r);
+        sm100::tmem_st32(ta, r);
+#pragma unroll
+        for (int j = 0; j < kNQ; ++j) r[j] = 0u;
+        sm100::tmem_st32(ta + kNQ, r);
         sm100::tmem_st_wait();
       }
       sm100::tc_fence_before();
@@ -610,7 +576,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
     float* alph = reinterpret_cast<float*>(smem + kOffAlpha);
     float2* fin = reinterpret_cast<float2*>(smem + kOffFin);
     float* zf = reinterpret_cast<float*>(smem + kOffZf);
-    float mref = -INFINITY, ell = 0.f, zac = 0.f;  // of query head `lane`
+    // the reference maximum of query head `lane` (mref) and of every head (mr, the same in all
+    // threads); this thread's partial sums of p~ (ell) and of p~ zero (zac) per head over its tokens
+    float mref = -INFINITY;
+    float mr[kNQ], ell[kNQ], zac[kNQ];
+#pragma unroll
+    for (int j = 0; j < kNQ; ++j) {
+      mr[j] = -INFINITY;
+      ell[j] = 0.f;
+      zac[j] = 0.f;
+    }
     bool ok = true;
     const __half2* szV = cv.sz ? cv.sz + int64_t(ll) * NKV * a.T : nullptr;
     uint32_t zv[NKV], nzv[NKV];
@@ -634,11 +609,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
         const uint32_t ready = nkb ? BS_FULL(it & 1) : BR_FULL(it & 1);
         if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(ready, (it >> 1) & 1, a.err));
         sm100::tc_fence_after();
-        uint32_t r[kNQ];
-        sm100::tmem_ld32(tS + (it & 1) * kNQ + (uint32_t(32 * q) << 16), r);
+        uint32_t r[kNQ], r2[kNQ];
+        const uint32_t ta = tS + (it & 1) * 2 * kNQ + (uint32_t(32 * q) << 16);
+        sm100::tmem_ld32(ta, r);
+        sm100::tmem_ld32(ta + kNQ, r2);
         sm100::tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < kNQ; ++j) sv[j] = __uint_as_float(r[j]);
+        for (int j = 0; j < kNQ; ++j) sv[j] = __uint_as_float(r[j]) + __uint_as_float(r2[j]);
         sm100::tc_fence_before();
         __syncwarp();
         if (lane == 0) sm100::mbar_arrive(BS_EMPTY(it & 1));
@@ -646,21 +623,39 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       const float sc2 = a.attn_scale * kLog2e;
 #pragma unroll
       for (int j = 0; j < kNQ; ++j) sv[j] = valid ? sv[j] * sc2 : -INFINITY;
-      // ---- tile maximum per query head; the reference maximum moves only by more than 2^8 ----
-      float tmp[kNQ];
+      // ---- the reference maximum moves only when a tile exceeds it by more than 2^8: each thread
+      // checks its token against every head's reference; only then is the tile maximum formed ----
+      bool ex = false;
 #pragma unroll
-      for (int j = 0; j < kNQ; ++j) tmp[j] = sv[j];
-      const float wmax = reduce_scatter32<true>(tmp, lane);
-      float* rd = red + (it & 1) * 128;
-      rd[q * 32 + lane] = wmax;
+      for (int j = 0; j < kNQ; ++j) ex |= sv[j] > mr[j] + kRescaleThreshold;
+      float* exf = alph + (it & 1) * 64 + 40;  // one flag per warp (alpha and rescale flag sit below)
+      const bool wex = __any_sync(0xffffffffu, ex);  // every lane votes; lane 0 publishes
+      if (lane == 0) exf[q] = wex ? 1.f : 0.f;
       named_bar(1, 128);
-      const float tmax = fmaxf(fmaxf(rd[lane], rd[32 + lane]), fmaxf(rd[64 + lane], rd[96 + lane]));
-      const float mnew = (tmax > mref + kRescaleThreshold || mref == -INFINITY) ? fmaxf(tmax, mref) : mref;
-      const float al = (mnew == mref) ? 1.f : exp2f(mref - mnew);
-      const bool resc = __any_sync(0xffffffffu, mnew != mref);
-      mref = mnew;
-      ell *= al;
-      zac *= al;
+      const bool any_ex = (exf[0] + exf[1]) + (exf[2] + exf[3]) != 0.f;
+      float al = 1.f;
+      bool resc = false;
+      if (any_ex) {
+        float tmp[kNQ];
+#pragma unroll
+        for (int j = 0; j < kNQ; ++j) tmp[j] = sv[j];
+        const float wmax = reduce_scatter32<true>(tmp, lane);
+        float* rd = red + (it & 1) * 128;
+        rd[q * 32 + lane] = wmax;
+        named_bar(1, 128);
+        const float tmax = fmaxf(fmaxf(rd[lane], rd[32 + lane]), fmaxf(rd[64 + lane], rd[96 + lane]));
+        const float mnew = (tmax > mref + kRescaleThreshold || mref == -INFINITY) ? fmaxf(tmax, mref) : mref;
+        al = (mnew == mref) ? 1.f : exp2f(mref - mnew);
+        resc = __any_sync(0xffffffffu, mnew != mref);
+        mref = mnew;
+#pragma unroll
+        for (int j = 0; j < kNQ; ++j) {
+          const float alj = __shfl_sync(0xffffffffu, al, j);
+          mr[j] = __shfl_sync(0xffffffffu, mnew, j);
+          ell[j] *= alj;
+          zac[j] *= alj;
+        }
+      }
       // the P~ / weight buffer of this tile is free once tile it - 2's value products are done
       if (it >= 2 && ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BP_EMPTY(it & 1), ((it >> 1) & 1) ^ 1, a.err));
       if (resc && it > 0 && nmc > 0) {
@@ -683,26 +678,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       // ---- probabilities: P~ (bf16) for the U_T^V product, f16 weights for the value residual ----
       uint8_t* pt = smem + kOffPt + (it & 1) * kPtBytes;
       uint8_t* wbp = smem + kOffWb + (it & 1) * kWbBytes;
-      float zsum[kNQ];
       const int kcT = tl >> 4, rT = tl & 15, eT = rT >> 2, mT = rT & 3;
       const int pc = tl >> 6, pu = (tl & 63) >> 3;
 #pragma unroll
       for (int j = 0; j < kNQ; ++j) {
-        const float mj = __shfl_sync(0xffffffffu, mref, j);
-        const __nv_bfloat16 pb = __float2bfloat16_rn(valid ? exp2f(sv[j] - mj) : 0.f);
+        const __nv_bfloat16 pb = __float2bfloat16_rn(valid ? exp2f(sv[j] - mr[j]) : 0.f);
         const float pf = __bfloat162float(pb);
-        tmp[j] = pf;
+        ell[j] += pf;
         // K-major, 128-byte swizzle: row j, tokens in two 64-token chunks
         *reinterpret_cast<__nv_bfloat16*>(pt + pc * (kNQ * 128) + j * 128 + ((pu ^ (j & 7)) << 4) + (tl & 7) * 2) = pb;
         const int h = j / GQ, gg = j % GQ;
-        float zz = 0.f;
         if (bV) {
           const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&zv[h]));
-          zz = f.y * pf;
+          zac[j] += f.y * pf;
           const __half w = __float2half_rn(pf * f.x * 0.00390625f);
           *reinterpret_cast<__half*>(wbp + ((((h * 8 + kcT) * 4 + mT) * GQ + gg) * 2 + (eT >> 1)) * 4 + (eT & 1) * 2) = w;
         }
-        zsum[j] = zz;
       }
       if (q == 0) {
         alph[(it & 1) * 64 + lane] = al;
@@ -711,11 +702,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       sm100::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(BP_FULL(it & 1));
-      ell += reduce_scatter32<false>(tmp, lane);
-      zac += reduce_scatter32<false>(zsum, lane);
     }
     // ---- partials of this split: m (natural log), l; W from TMEM ----
-    fin[q * 32 + lane] = make_float2(ell, zac);
+    {
+      const float L = reduce_scatter32<false>(ell, lane), Z = reduce_scatter32<false>(zac, lane);
+      fin[q * 32 + lane] = make_float2(L, Z);
+    }
     named_bar(1, 128);
     if (q == 0) {
       float L = 0.f, Z = 0.f;
@@ -832,58 +824,210 @@ struct PTab {
 };
 
 // P = G^K_h (U_d^K^T q) for the g_q query heads of one KV head, written as bf16 hi rows then lo rows
-// per (sequence, layer): out [B*Lc][64][q_cap], zero beyond r_T (those columns meet the zero fill
-// of U_T's tensor map). grid (n_kv, B*Lc), 256 threads: q-hat = U_d^T q for the KV head's query
-// heads in shared memory, then a warp per row r of G_h (lanes over r_d, 8-byte loads: each row
-// read once for all g_q heads) and a warp reduction per head.
+// per (sequence, layer): out [B*Lc][64][q_cap], zero from r_T up to the 64-rank chunk boundary
+// (those columns meet the zero fill of U_T's tensor map). grid (n_kv, B*Lc), 256 threads: q-hat =
+// U_d^T q for the KV head's query heads in shared memory (thread c over the U_d rows, one load per
+// row for all g_q heads), then a thread per row r of G_h (sixteen 16-byte loads in flight, q-hat
+// read as broadcasts), no cross-lane reductions.
 template <int GQ>
 __global__ void __launch_bounds__(256) k_prologue_p(const __nv_bfloat16* __restrict__ q, int q_cap, const PTab tab,
                                                    __nv_bfloat16* __restrict__ out) {
   const int h = blockIdx.x, bl = blockIdx.y;
   const PRow pr = tab.row[bl];
   __shared__ float qs[GQ][kD];
-  __shared__ float qh[GQ][kD];
+  __shared__ __align__(16) float qh[kD][GQ];  // [feature][head]
   for (int e = threadIdx.x; e < GQ * kD; e += blockDim.x)
     qs[e / kD][e % kD] = __bfloat162float(q[(int64_t(bl) * kNQ + h * GQ) * kD + e]);
   __syncthreads();
-  for (int e = threadIdx.x; e < GQ * kD; e += blockDim.x) {
-    const int j = e / kD, c = e % kD;
-    float a = 0.f;
-    if (c < pr.r_d)
-      for (int i = 0; i < kD; ++i) a = fmaf(__bfloat162float(pr.Ud[int64_t(i) * pr.r_d + c]), qs[j][i], a);
-    qh[j][c] = a;
+  {
+    // thread (c, half): rows i of U_d in one half of the features; halves added through shared memory
+    const int c = threadIdx.x & (kD - 1), half = threadIdx.x >> 7;
+    float acc[GQ];
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) acc[j] = 0.f;
+    if (c < pr.r_d && pr.r_T > 0) {
+#pragma unroll 8
+      for (int i = half * (kD / 2); i < (half + 1) * (kD / 2); ++i) {
+        const float u = __bfloat162float(pr.Ud[int64_t(i) * pr.r_d + c]);
+#pragma unroll
+        for (int j = 0; j < GQ; ++j) acc[j] = fmaf(u, qs[j][i], acc[j]);
+      }
+    }
+    if (half == 1)
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) qh[c][j] = acc[j];
+    __syncthreads();
+    if (half == 0)
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) qh[c][j] = c < pr.r_d ? acc[j] + qh[c][j] : 0.f;
   }
   __syncthreads();
   const int64_t n = int64_t(kNQ) * q_cap;
   __nv_bfloat16* hi = out + int64_t(bl) * 2 * n;
   __nv_bfloat16* lo = hi + n;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rend = min(q_cap, (pr.r_T + 63) / 64 * 64);
   const __nv_bfloat16* Gh = pr.G + int64_t(h) * pr.r_T * pr.r_d;
-  for (int r = warp; r < q_cap; r += 8) {
+  for (int r = threadIdx.x; r < rend; r += blockDim.x) {
     float acc[GQ];
 #pragma unroll
     for (int j = 0; j < GQ; ++j) acc[j] = 0.f;
     if (r < pr.r_T) {
-      for (int c0 = 4 * lane; c0 < pr.r_d; c0 += 128) {
-        const uint2 w = *reinterpret_cast<const uint2*>(Gh + int64_t(r) * pr.r_d + c0);
-        const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
-        const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+      const __nv_bfloat16* row = Gh + int64_t(r) * pr.r_d;
+      if (pr.r_d == kD && (reinterpret_cast<uintptr_t>(row) & 15) == 0) {
+        uint4 w[kD / 8];
 #pragma unroll
-        for (int j = 0; j < GQ; ++j)
-          acc[j] = fmaf(g01.x, qh[j][c0], fmaf(g01.y, qh[j][c0 + 1], fmaf(g23.x, qh[j][c0 + 2], fmaf(g23.y, qh[j][c0 + 3], acc[j]))));
+        for (int k = 0; k < kD / 8; ++k) w[k] = __ldg(reinterpret_cast<const uint4*>(row) + k);
+#pragma unroll
+        for (int k = 0; k < kD / 8; ++k) {
+          const uint32_t ww[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 g2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ww[u]));
+            const int c = 8 * k + 2 * u;
+#pragma unroll
+            for (int j = 0; j < GQ; ++j) acc[j] = fmaf(g2.x, qh[c][j], fmaf(g2.y, qh[c + 1][j], acc[j]));
+          }
+        }
+      } else {
+        for (int c = 0; c < pr.r_d; ++c) {
+          const float g1 = __bfloat162float(row[c]);
+#pragma unroll
+          for (int j = 0; j < GQ; ++j) acc[j] = fmaf(g1, qh[c][j], acc[j]);
+        }
       }
     }
 #pragma unroll
     for (int j = 0; j < GQ; ++j) {
-      float v = acc[j];
-      for (int m = 16; m; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-      if (lane == j) {
-        const __nv_bfloat16 hh = __float2bfloat16_rn(v);
-        hi[int64_t(h * GQ + j) * q_cap + r] = hh;
-        lo[int64_t(h * GQ + j) * q_cap + r] = __float2bfloat16_rn(v - __bfloat162float(hh));
-      }
+      const __nv_bfloat16 hh = __float2bfloat16_rn(acc[j]);
+      hi[int64_t(h * GQ + j) * q_cap + r] = hh;
+      lo[int64_t(h * GQ + j) * q_cap + r] = __float2bfloat16_rn(acc[j] - __bfloat162float(hh));
     }
   }
+}
+
+// One value cell's stored factors and the output rows of a (sequence, layer) row of a launch set.
+struct MRow {
+  const __nv_bfloat16* G;   // G^V of the row's layer: [n_kv][r_T][r_d]
+  const __nv_bfloat16* Ud;  // U_d^V [128][r_d]
+  int r_T, r_d, bits;
+};
+struct MTab {
+  MRow row[kMaxFusedRows];
+};
+
+// Merge of the split partials and the output projection for the g_q query heads of one KV head:
+//   M = max_s m_s, c_s = exp(m_s - M), L = sum_s c_s l_s, w = sum_s c_s W_s, a = sum_s c_s acc_s,
+//   out = (R^T a + U_d^V (G^V_h^T w)) / L, lse = M + log L.
+// grid (n_kv, B*Lc), 512 threads; dynamic shared memory: c [g_q][S], w [g_q][r_T],
+// v partials [4][g_q][128], v [g_q][128], a [g_q][128]. G^V_h is read once for all g_q heads.
+template <int GQ>
+__global__ void __launch_bounds__(512) k_merge_fused(const float* __restrict__ part, int S, int q_cap,
+                                                    const __grid_constant__ MTab tab,
+                                                    uint64_t rot_seed, __nv_bfloat16* __restrict__ out,
+                                                    float* __restrict__ lse) {
+  extern __shared__ float msm[];
+  const int h = blockIdx.x, bl = blockIdx.y;
+  const MRow mr = tab.row[bl];
+  const int rT = mr.r_T, rd = mr.r_d;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const size_t prow = size_t(2 + q_cap + kD);
+  float* cf = msm;                          // [GQ][S]
+  float* w = cf + GQ * S;                   // [GQ][rT]
+  float* vp = w + GQ * max(rT, 1);          // [4][GQ][128]
+  float* v = vp + 4 * GQ * kD;              // [GQ][128]
+  float* x = v + GQ * kD;                   // [GQ][128]
+  __shared__ float sM[GQ], sL[GQ];
+  auto prow_of = [&](int g, int sp) { return part + ((size_t(bl) * kNQ + h * GQ + g) * S + sp) * prow; };
+  if (warp < GQ) {
+    const int g = warp;
+    float M = -INFINITY;
+    for (int sp = lane; sp < S; sp += 32) M = fmaxf(M, prow_of(g, sp)[0]);
+    M = warp_max(M);
+    float L = 0.f;
+    for (int sp = lane; sp < S; sp += 32) {
+      const float* pr = prow_of(g, sp);
+      const float c = pr[0] == -INFINITY ? 0.f : __expf(pr[0] - M);
+      cf[g * S + sp] = c;
+      L += c * pr[1];
+    }
+    L = warp_sum(L);
+    if (lane == 0) {
+      sM[g] = M;
+      sL[g] = L;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < GQ * rT; e += blockDim.x) {
+    const int g = e / rT, r = e % rT;
+    float a = 0.f;
+    for (int sp = 0; sp < S; ++sp) a = fmaf(cf[g * S + sp], prow_of(g, sp)[2 + r], a);
+    w[e] = a;
+  }
+  for (int e = tid; e < GQ * kD; e += blockDim.x) {
+    const int g = e / kD, d = e % kD;
+    float a = 0.f;
+    if (mr.bits)
+      for (int sp = 0; sp < S; ++sp) a = fmaf(cf[g * S + sp], prow_of(g, sp)[2 + q_cap + d], a);
+    x[e] = a;
+  }
+  __syncthreads();
+  {
+    const int j = tid & (kD - 1), qt = tid >> 7;
+    float sacc[GQ];
+#pragma unroll
+    for (int g = 0; g < GQ; ++g) sacc[g] = 0.f;
+    if (j < rd && rT > 0) {
+      const __nv_bfloat16* G = mr.G + int64_t(h) * rT * rd + j;
+#pragma unroll 8
+      for (int r = qt; r < rT; r += 4) {
+        const float gv = __bfloat162float(G[int64_t(r) * rd]);
+#pragma unroll
+        for (int g = 0; g < GQ; ++g) sacc[g] = fmaf(gv, w[g * rT + r], sacc[g]);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < GQ; ++g) vp[(qt * GQ + g) * kD + j] = sacc[g];
+  }
+  __syncthreads();
+  for (int e = tid; e < GQ * kD; e += blockDim.x) {
+    const int j = e % kD;
+    v[e] = j < rd ? (vp[e] + vp[GQ * kD + e]) + (vp[2 * GQ * kD + e] + vp[3 * GQ * kD + e]) : 0.f;
+  }
+  if (mr.bits && warp < GQ) {
+    float xv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xv[i] = x[warp * kD + lane * 4 + i];
+    warp_unrotate<4>(xv, rot_seed, rsqrtf(float(kD)));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[warp * kD + lane * 4 + i] = xv[i];
+  }
+  __syncthreads();
+  // each warp's eight U_d rows are loaded before any is used
+  float udr[kD / 16][4];
+#pragma unroll
+  for (int u = 0; u < kD / 16; ++u)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = warp + 16 * u, j = lane * 4 + k;
+      udr[u][k] = (rT > 0 && j < rd) ? __bfloat162float(mr.Ud[int64_t(i) * rd + j]) : 0.f;
+    }
+  const int64_t qr0 = int64_t(bl) * kNQ + h * GQ;
+#pragma unroll
+  for (int u = 0; u < kD / 16; ++u) {
+    const int i = warp + 16 * u;
+#pragma unroll
+    for (int g = 0; g < GQ; ++g) {
+      const float* vg = v + g * kD + lane * 4;
+      float o = (udr[u][0] * vg[0] + udr[u][1] * vg[1]) + (udr[u][2] * vg[2] + udr[u][3] * vg[3]);
+      o = warp_sum(o);
+      if (lane == 0) out[(qr0 + g) * kD + i] = __float2bfloat16_rn((x[g * kD + i] + o) / sL[g]);
+    }
+  }
+  if (tid < GQ && lse) lse[qr0 + tid] = sM[tid] + logf(sL[tid]);
+}
+
+size_t merge_fused_smem(int gq, int S, int r_T) {
+  return (size_t(gq) * S + size_t(gq) * std::max(r_T, 1) + size_t(6) * gq * kD) * sizeof(float);
 }
 
 constexpr int kSMs = 148;
@@ -1030,12 +1174,36 @@ jolt_status launch_decode_fused(const DecodeParams& p, const TcCellView* views, 
     }
     JOLT_CUDA_TRY(cudaGetLastError());
   }
-  // ---- merge of the splits and finalize ----
-  DecodeParams pm = p;
-  pm.S = wl.S;
-  pm.ws_part = part;
+  // ---- merge of the splits and the output projection ----
   StatScope sc2(JOLT_K_DECODE_AUX, st, 0.0, 0.0);
-  return launch_decode_merge(pm, st);
+  static_assert(sizeof(MTab) <= 24 * 1024, "merge parameter table");
+  MTab mt;
+  int rmax = 1;
+  for (int b = 0; b < p.B; ++b)
+    for (int li = 0; li < p.Lc; ++li) {
+      const int layer = p.layer_begin + li, g = layer / p.Lg, ll = layer % p.Lg;
+      const TcCellView& v = views[(b * p.Gc + (g - p.g_first)) * 2 + 1];
+      MRow& r = mt.row[b * p.Lc + li];
+      r.G = v.r_T ? v.G + int64_t(ll) * p.n_kv * v.r_T * v.r_d : nullptr;
+      r.Ud = v.Ud;
+      r.r_T = v.r_T;
+      r.r_d = v.r_d;
+      r.bits = v.bits;
+      rmax = std::max(rmax, v.r_T);
+    }
+  const size_t msm = merge_fused_smem(p.gq, wl.S, rmax);
+  __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(p.out);
+  if (p.gq == 4) {
+    if (msm > 48 * 1024)
+      JOLT_CUDA_TRY(cudaFuncSetAttribute(k_merge_fused<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(msm)));
+    k_merge_fused<4><<<dim3(p.n_kv, BL), 512, msm, st>>>(part, wl.S, qc, mt, p.rot_seed, ob, p.lse);
+  } else {
+    if (msm > 48 * 1024)
+      JOLT_CUDA_TRY(cudaFuncSetAttribute(k_merge_fused<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(msm)));
+    k_merge_fused<8><<<dim3(p.n_kv, BL), 512, msm, st>>>(part, wl.S, qc, mt, p.rot_seed, ob, p.lse);
+  }
+  JOLT_CUDA_TRY(cudaGetLastError());
+  return JOLT_OK;
 }
 
 }  // namespace jolt
