@@ -108,17 +108,20 @@ __device__ __forceinline__ void load_codes_raw(const uint8_t* row, uint32_t (&w)
 }
 
 // The row dequantised (code * scale + zero, one fp32 fused multiply-add per code), as 64 packed
-// pairs of consecutive features.
+// pairs of consecutive features. Each code becomes an exact float by placing it in the mantissa of
+// 2^23 and subtracting 2^23 (no integer-to-float conversion).
 template <int BITS>
 __device__ __forceinline__ void dequant2(const uint32_t (&w)[4 * BITS + 1], float sc, float zr, float2 (&v)[kD / 2]) {
   constexpr uint32_t mask = (1u << BITS) - 1u;
   const float2 sc2 = make_float2(sc, sc), zr2 = make_float2(zr, zr);
+  const float2 m23 = make_float2(-8388608.f, -8388608.f);
 #pragma unroll
   for (int m = 0; m < kD / 2; ++m) {
     const int j0 = 2 * m, j1 = 2 * m + 1;
-    const float c0 = float((w[(j0 * BITS) >> 5] >> ((j0 * BITS) & 31)) & mask);
-    const float c1 = float((w[(j1 * BITS) >> 5] >> ((j1 * BITS) & 31)) & mask);
-    v[m] = __ffma2_rn(make_float2(c0, c1), sc2, zr2);
+    const uint32_t f0 = ((w[(j0 * BITS) >> 5] >> ((j0 * BITS) & 31)) & mask) | 0x4B000000u;
+    const uint32_t f1 = ((w[(j1 * BITS) >> 5] >> ((j1 * BITS) & 31)) & mask) | 0x4B000000u;
+    const float2 c = __fadd2_rn(make_float2(__uint_as_float(f0), __uint_as_float(f1)), m23);
+    v[m] = __ffma2_rn(c, sc2, zr2);
   }
 }
 
