@@ -654,8 +654,8 @@ __global__ void __launch_bounds__(256) k_values_res_mma(const ValArgs a) {
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) zacc[nt] = 0.f;
   const int t_beg = blockIdx.x * a.chunk, t_end = min(a.T, t_beg + a.chunk);
-  // raw operands of one 16-token step (code words, scale/zero pairs, P~ pairs), loaded two steps
-  // ahead of their use
+  // raw operands of one 16-token step (code words, scale/zero pairs, P~ pairs), loaded ahead of
+  // their use
   struct Raw {
     uint32_t w[4][LW];
     uint32_t sz[4];
@@ -695,15 +695,21 @@ __global__ void __launch_bounds__(256) k_values_res_mma(const ValArgs a) {
       }
     }
   };
-  // two steps in flight ahead of the one being computed
+  // steps in flight ahead of the one being computed: two for 2-bit codes (small rows), one for
+  // wider codes (the extra register set would cost CTAs per SM)
+  constexpr int kAhead = BITS == 2 ? 2 : 1;
   Raw n1, n2;
   int tb = t_beg + 16 * warp;
   if (tb < t_end) load(tb, n1);
-  if (tb + 16 * 8 < t_end) load(tb + 16 * 8, n2);
+  if (kAhead == 2 && tb + 16 * 8 < t_end) load(tb + 16 * 8, n2);
   for (; tb < t_end; tb += 16 * 8) {
     const Raw cur = n1;
-    n1 = n2;
-    if (tb + 2 * 16 * 8 < t_end) load(tb + 2 * 16 * 8, n2);
+    if (kAhead == 2) {
+      n1 = n2;
+      if (tb + 2 * 16 * 8 < t_end) load(tb + 2 * 16 * 8, n2);
+    } else if (tb + 16 * 8 < t_end) {
+      load(tb + 16 * 8, n1);
+    }
     float sc[4], zr[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
