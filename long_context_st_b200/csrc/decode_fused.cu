@@ -22,12 +22,13 @@
 //     never expanded to 16 bits in memory, which would cost four times their size in shared-memory
 //     traffic per contraction. The key residual is stored into the tile's TMEM score buffer first
 //     and the factor products accumulate on top of it, so the scores arrive complete.
-// Warp roles (512 threads, four warpgroups whose register budgets are re-split with setmaxnreg):
+// Warp roles (640 threads, five warpgroups whose register budgets are re-split with setmaxnreg):
 //   0: warp 0 TMA producers (one lane per operand ring), warp 1 score-product issuer (owns TMEM),
 //      warp 2 value-product issuer;
-//   1: key-residual warps (the MMAs for their 32 tokens, then the row into TMEM);
-//   2: softmax warps (thread = token of the tile: scores from TMEM, online softmax, P~);
-//   3: value warps (value-residual MMAs, 32 features each).
+//   1, 2: key-residual warps, two per TMEM lane quarter (16 tokens each; the first stores the
+//      quarter's 32 rows into TMEM);
+//   3: softmax warps (thread = token of the tile: scores from TMEM, online softmax, P~);
+//   4: value warps (value-residual MMAs, 32 features each).
 // TMEM: two score buffers of 64 columns, W (32 columns per 128-rank chunk) from column 128, the
 // value-residual accumulators (8 columns per KV head) from column 384.
 #include <algorithm>
@@ -87,9 +88,9 @@ static_assert(kSmem <= 232448, "fused decode shared memory");
 static_assert(kOffV % 1024 == 0 && kOffPt % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(kOffCK % 16 == 0 && kOffCV % 16 == 0 && kOffBars % 8 == 0, "bulk-copy and mbarrier alignment");
 
-constexpr int kThreads = 512;  // four warpgroups: control, key residual, softmax, value residual
+constexpr int kThreads = 640;  // five warpgroups: control, key residual (two), softmax, value residual
 // registers a thread after the warpgroups' re-split (launch: 128 each, 65536 in all)
-constexpr int kRegCtl = 40, kRegKres = 128, kRegSoft = 184, kRegVres = 160;
+constexpr int kRegCtl = 40, kRegKres = 96, kRegSoft = 168, kRegVres = 80;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -142,19 +143,18 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
   return v[0];
 }
 
-// Key residual of KV head h (codes in slot k of the stage at cs) for the 32 tokens of quarter q:
-// scr[token][h g_q + j] = scale (codes . R q_j) + zero sum(R q_j). zrow[i]: the (scale, zero) pair
-// of token 32 q + i for this head.
+// Key residual of KV head h (codes in slot k of the stage at cs) for the 16 tokens 32 q + 16 mb ..
+// of quarter q: scr[token][h g_q + j] = scale (codes . R q_j) + zero sum(R q_j). zrow[i]: the
+// (scale, zero) pair of token 32 q + 16 mb + i for this head.
 template <int BITS, int GQ>
-__device__ __forceinline__ void kres_head(const uint8_t* cs, int k, int h, int q, int lane, const uint2* qf,
+__device__ __forceinline__ void kres_head(const uint8_t* cs, int k, int h, int q, int mb, int lane, const uint2* qf,
                                           const float* qs, float* scr, const uint32_t* zrow) {
   constexpr int RB = 16 * BITS;
   const int gr = lane >> 2, m4 = lane & 3;
-  uint2 bqs[8];  // the head's query fragments, shared by both 16-token row blocks
+  uint2 bqs[8];  // the head's query fragments
 #pragma unroll
   for (int kc = 0; kc < 8; ++kc) bqs[kc] = gr < GQ ? qf[((h * 8 + kc) * GQ + gr) * 4 + m4] : make_uint2(0u, 0u);
-#pragma unroll
-  for (int mb = 0; mb < 2; ++mb) {
+  {
     const int rA = 32 * q + 16 * mb + gr;  // tile rows of fragment rows g and g + 8
     const uint8_t* rowA = cs + (k * kBM + rA) * RB;
     const uint8_t* rowB = rowA + 8 * RB;
@@ -193,8 +193,8 @@ __device__ __forceinline__ void kres_head(const uint8_t* cs, int k, int h, int q
       mma_f16_16816(acc, af, bqs[kc].x, bqs[kc].y);
     }
     // rows g (tile row rA) and g + 8, query heads 2 m4, 2 m4 + 1 of KV head h
-    const uint32_t zA = zrow[16 * mb + gr];
-    const uint32_t zB = zrow[16 * mb + gr + 8];
+    const uint32_t zA = zrow[gr];
+    const uint32_t zB = zrow[gr + 8];
     const float2 fA = __half22float2(*reinterpret_cast<const __half2*>(&zA));
     const float2 fB = __half22float2(*reinterpret_cast<const __half2*>(&zB));
 #pragma unroll
@@ -261,7 +261,7 @@ __device__ __forceinline__ void vres_head(float (&ac)[2][4], const uint8_t* cs, 
 // copy of the head's code per code width keeps the hot loop small), releasing each code stage.
 template <int BITS, int GQ>
 __device__ __forceinline__ bool kres_tile(const uint8_t* cbase, uint32_t full0, uint32_t empty0, int& ckit, int q,
-                                       int lane, const uint2* qf, const float* qs, float* scr,
+                                       int mb, int lane, const uint2* qf, const float* qs, float* scr,
                                        const uint32_t* zks, int32_t* err, bool ok) {
   constexpr int NKV = kNQ / GQ, hps = 8 / BITS;
   int s = 0;
@@ -272,7 +272,7 @@ __device__ __forceinline__ bool kres_tile(const uint8_t* cbase, uint32_t full0, 
       s = ckit % kCStages;
       if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(full0 + 8u * s, (ckit / kCStages) & 1, err));
     }
-    kres_head<BITS, GQ>(cbase + s * kCStageBytes, k, h, q, lane, qf, qs, scr, zks + h * 32);
+    kres_head<BITS, GQ>(cbase + s * kCStageBytes, k, h, q, mb, lane, qf, qs, scr, zks + h * 16);
     if (k == hps - 1 || h == NKV - 1) {
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(empty0 + 8u * s);
@@ -369,7 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
     // products (1 commit) and the four value warps
     for (int i = 0; i < 31; ++i) {
       uint32_t cnt = 1;
-      if ((i >= 12 && i < 14) || (i >= 16 && i < 18) || (i >= 20 && i < 24) || i >= 29) cnt = 4;
+      if ((i >= 16 && i < 18) || (i >= 20 && i < 24) || i >= 29) cnt = 4;
+      if (i >= 12 && i < 14) cnt = 8;  // key code stages: released by all eight key-residual warps
       if (i >= 24 && i < 26) cnt = 5;
       if (i == 28) cnt = 2;  // the drain: one commit per MMA-issuing thread
       sm100::mbar_init(bar0 + 8u * i, cnt);
@@ -499,11 +500,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       sm100::mma_commit(BDRAIN);
       sm100::mbar_wait(BDRAIN, 0, a.err);
     }
-  } else if (wg == 1) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegKres));
+  } else if (wg <= 2) {
     // ================= key-residual warps: S(it) starts as scale (codes . R q) + zero sum(R q) ====
+    // two warps per TMEM lane quarter: warpgroup 1 takes tokens 32q .. 32q+15 of the tile (mb = 0),
+    // warpgroup 2 tokens 32q+16 .. 32q+31 (mb = 1); the mb = 0 warp stores the quarter's rows
     const int q = warp & 3;            // TMEM lane quarter = tokens 32q .. 32q+31 of the tile
-    const int tid = threadIdx.x - 128; // 0..127
+    const int mb = wg - 1;
+    const int tid = threadIdx.x - 128; // 0..255
     float* scr = reinterpret_cast<float*>(smem + kOffScr) + q * 32 * kScrStride;
     float* qs = reinterpret_cast<float*>(smem + kOffQs);
     uint2* qf = reinterpret_cast<uint2*>(smem + kOffQf);
@@ -512,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
     const float* qr = a.qrot + int64_t(bl) * kNQ * kD;
     if (bK) {
       const int gap = pair_gap(bK);
-      for (int e = tid; e < NKV * 8 * GQ * 4; e += 128) {
+      for (int e = tid; e < NKV * 8 * GQ * 4; e += 256) {
         const int mm = e & 3, gg = (e >> 2) % GQ, kc = (e / (4 * GQ)) & 7, h = e / (32 * GQ);
         const float* qj = qr + (h * GQ + gg) * kD + 32 * mm;
         const int p0 = pair_lo(bK, 2 * kc), p1 = pair_lo(bK, 2 * kc + 1);
@@ -522,53 +525,58 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
       }
     }
     if (tid < kNQ) qs[tid] = a.qsum[int64_t(bl) * kNQ + tid];
-    named_bar(3, 128);
+    named_bar(3, 256);
     int ckit = 0;
     bool ok = true;
     const __half2* szK = ck.sz ? ck.sz + int64_t(ll) * NKV * a.T : nullptr;
-    // this thread's token's key scale / zero pairs, loaded one tile ahead (they reach the MMA lanes
-    // by shuffles)
-    uint32_t* zks = reinterpret_cast<uint32_t*>(smem + kOffZk) + q * 8 * 32;
+    // the key scale / zero pairs of this warp's 16 tokens (lane & 15), loaded one tile ahead into
+    // registers, then into the warp's slab [head][16 tokens]
+    uint32_t* zks = reinterpret_cast<uint32_t*>(smem + kOffZk) + (mb * 4 + q) * 8 * 16;
     uint32_t nzk[NKV];
     auto load_sz = [&](int it2, uint32_t (&k_)[NKV]) {
-      const int t2 = (tile0 + it2) * kBM + 32 * q + lane;
+      const int t2 = (tile0 + it2) * kBM + 32 * q + 16 * mb + (lane & 15);
       const bool ok2 = it2 < ntl && t2 < a.T;
 #pragma unroll
       for (int h = 0; h < NKV; ++h) k_[h] = (bK && ok2) ? sm100::ld_nc_early(szK + int64_t(h) * a.T + t2) : 0u;
     };
     load_sz(0, nzk);
     for (int it = 0; it < ntl; ++it) {
-      __syncwarp();  // every lane has read its row of the exchange buffer and slab before they are rewritten
+      __syncwarp();  // every lane has read the slab before it is rewritten
+      if (lane < 16)
 #pragma unroll
-      for (int h = 0; h < NKV; ++h) zks[h * 32 + lane] = nzk[h];
+        for (int h = 0; h < NKV; ++h) zks[h * 16 + lane] = nzk[h];
       __syncwarp();
       load_sz(it + 1, nzk);
       if (bK) {
         const uint8_t* cbase = smem + kOffCK;
-        if (bK == 4) ok = kres_tile<4, GQ>(cbase, BCK_FULL(0), BCK_EMPTY(0), ckit, q, lane, qf, qs, scr, zks, a.err, ok);
-        else if (bK == 2) ok = kres_tile<2, GQ>(cbase, BCK_FULL(0), BCK_EMPTY(0), ckit, q, lane, qf, qs, scr, zks, a.err, ok);
-        else ok = kres_tile<8, GQ>(cbase, BCK_FULL(0), BCK_EMPTY(0), ckit, q, lane, qf, qs, scr, zks, a.err, ok);
+        if (bK == 4) ok = kres_tile<4, GQ>(cbase, BCK_FULL(0), BCK_EMPTY(0), ckit, q, mb, lane, qf, qs, scr, zks, a.err, ok);
+        else if (bK == 2) ok = kres_tile<2, GQ>(cbase, BCK_FULL(0), BCK_EMPTY(0), ckit, q, mb, lane, qf, qs, scr, zks, a.err, ok);
+        else ok = kres_tile<8, GQ>(cbase, BCK_FULL(0), BCK_EMPTY(0), ckit, q, mb, lane, qf, qs, scr, zks, a.err, ok);
       }
-      // the S buffer is free once the softmax warps have read tile it - 2
-      if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BS_EMPTY(it & 1), ((it >> 1) & 1) ^ 1, a.err));
-      sm100::tc_fence_after();
-      if (bK || nkb == 0) {
-        // the residual into the hi columns, zeros into the lo columns (the products accumulate)
-        uint32_t r[kNQ];
-        const uint32_t ta = tS + (it & 1) * 2 * kNQ + (uint32_t(32 * q) << 16);
+      named_bar(4 + q, 64);  // both halves of the quarter's rows are in the exchange buffer
+      if (mb == 0) {
+        // the S buffer is free once the softmax warps have read tile it - 2
+        if (ok) ok = __all_sync(0xffffffffu, sm100::mbar_wait(BS_EMPTY(it & 1), ((it >> 1) & 1) ^ 1, a.err));
+        sm100::tc_fence_after();
+        if (bK || nkb == 0) {
+          // the residual into the hi columns, zeros into the lo columns (the products accumulate)
+          uint32_t r[kNQ];
+          const uint32_t ta = tS + (it & 1) * 2 * kNQ + (uint32_t(32 * q) << 16);
 #pragma unroll
-        for (int j = 0; j < kNQ; ++j) r[j] = bK ? __float_as_uint(scr[lane * kScrStride + j]) : 0u;
-        sm100::tmem_st32(ta, r);
+          for (int j = 0; j < kNQ; ++j) r[j] = bK ? __float_as_uint(scr[lane * kScrStride + j]) : 0u;
+          sm100::tmem_st32(ta, r);
 #pragma unroll
-        for (int j = 0; j < kNQ; ++j) r[j] = 0u;
-        sm100::tmem_st32(ta + kNQ, r);
-        sm100::tmem_st_wait();
+          for (int j = 0; j < kNQ; ++j) r[j] = 0u;
+          sm100::tmem_st32(ta + kNQ, r);
+          sm100::tmem_st_wait();
+        }
+        sm100::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(BR_FULL(it & 1));
       }
-      sm100::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(BR_FULL(it & 1));
+      named_bar(4 + q, 64);  // the rows have been read before the next tile rewrites them
     }
-  } else if (wg == 2) {
+  } else if (wg == 3) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoft));
     // ================= softmax warps: complete scores from TMEM, online softmax, P~ =================
     const int q = warp & 3;            // TMEM lane quarter = tokens 32q .. 32q+31 of the tile
@@ -737,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const __grid_const
     }
     named_bar(2, 256);  // zf ready for the value warps
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegVres));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegVres));
     // ================= value warps: acc[d][j] += sum_t weight[t][j] codes^V[t][d] =================
     const int vw = warp & 3;  // features 16 g + 4 vw .. + 3
     const int gr = lane >> 2, m4 = lane & 3;
@@ -1162,8 +1170,9 @@ jolt_status launch_decode_fused(const DecodeParams& p, const TcCellView* views, 
     // was launched with, or an increasing warpgroup would wait for registers that never come
     cudaFuncAttributes fat;
     JOLT_CUDA_TRY(cudaFuncGetAttributes(&fat, p.gq == 4 ? k_decode_fused<4> : k_decode_fused<8>));
-    if (fat.numRegs < kRegCtl || fat.numRegs > kRegKres || fat.numRegs > kRegSoft || fat.numRegs > kRegVres ||
-        128 * (kRegCtl + kRegKres + kRegSoft + kRegVres) > kThreads * fat.numRegs)
+    // (the key-residual warpgroups keep the launch count: they do not re-split)
+    if (fat.numRegs != kRegKres || fat.numRegs < kRegCtl || fat.numRegs > kRegSoft || fat.numRegs < kRegVres ||
+        128 * (kRegCtl + 2 * kRegKres + kRegSoft + kRegVres) > kThreads * fat.numRegs)
       return JOLT_ERR_CUDA;
     if (p.gq == 4) {
       JOLT_CUDA_TRY(cudaFuncSetAttribute(k_decode_fused<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
