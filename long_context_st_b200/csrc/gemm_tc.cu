@@ -238,10 +238,16 @@ __device__ __forceinline__ void op_issue(const CUtensorMap* map, OpCoord& o, uin
 // fast Walsh-Hadamard butterflies with strides 1, 2, ..., 64 ((lo, hi) -> (lo + hi, lo - hi)),
 // x rsqrt(128); min / max; step = (max - min) / (2^b - 1) and zero = min rounded to fp16;
 // code = clip(rint((x - zero) / scale)), packed little-endian.
+// The code is clip(rint(fl((x - zero) / scale))). The quotient is first taken as fl(a * fl(1/scale)):
+// two correctly rounded operations put it within 1.5 * 2^-23 |a / scale| of the exact quotient,
+// and the correctly rounded fl(a / scale) within 2^-24 |a / scale| of it, so for |q| <= 512 they
+// are within 2^-13 of each other and round to the same integer unless q lies within 2^-12 of a
+// half-integer; only then is the division itself done (beyond 512 both clip alike).
 template <int B>
 __device__ __forceinline__ void res_pack_store(const float (&v)[128], float s, float zf, uint8_t* dst) {
   constexpr int kPer = 32 / B;
   const float levels = float((1 << B) - 1);
+  const float rs = s != 0.f ? __frcp_rn(s) : 0.f;
 #pragma unroll
   for (int q = 0; q < B; ++q) {
     uint32_t w[4];
@@ -253,7 +259,10 @@ __device__ __forceinline__ void res_pack_store(const float (&v)[128], float s, f
         const int i = (q * 4 + e) * kPer + k;
         float c = 0.f;
         if (s != 0.f) {
-          c = rintf(__fdiv_rn(__fsub_rn(v[i], zf), s));
+          const float a = __fsub_rn(v[i], zf);
+          const float qt = __fmul_rn(a, rs);
+          c = rintf(qt);
+          if (fabsf(qt) <= 512.f && fabsf(qt - c) >= 0.5f - 0.000244140625f) c = rintf(__fdiv_rn(a, s));
           c = fminf(fmaxf(c, 0.f), levels);
         }
         acc |= uint32_t(c) << (k * B);
